@@ -1,0 +1,225 @@
+/*
+ * pkv.h -- C ABI of a paged, block-quantized KV cache for decode-phase attention (sm_100a).
+ *
+ * Sources the operations follow (web pages; cited by page and section):
+ *   [tbr8]      tbr8.org, "如何通过 PagedAttention 与分块量化结合：解决移动端内存碎片化导致的长文本 OOM"
+ *               (PagedAttention + group-wise block quantization against long-context OOM on phones).
+ *   [deepinsea] deepinsea.top, "PagedAttention 内存管理深度解析" (PagedAttention memory management).
+ *   [yunthe]    yunthe.com, "LLM推理显存优化KV Cache量化与PagedAttention实现详解"
+ *               (KV-cache quantization and PagedAttention).
+ *
+ * What lives where
+ *   - The KV cache is a pool of fixed-size physical blocks ([tbr8] §2 "PagedAttention 虚拟化管理";
+ *     [yunthe] section "PagedAttention分页注意力机制与vLLM实现", block_table data structure).
+ *     A block holds block_size tokens (16 or 32, [deepinsea] section "块大小选择") of every KV head.
+ *   - Each (block, KV head) tile is quantized on its own ([tbr8] §3 "分块量化", §4 store_kv):
+ *     K is INT8 symmetric with scale = absmax/127; V is INT8 symmetric or INT4 asymmetric with
+ *     Q(x) = clamp(round(x/scale + zp), 0, 2^bits - 1) and x_hat = (Q - zp) * scale
+ *     ([yunthe] section "KV Cache量化技术原理", quantize and dequantize formulas; K INT8 / V INT4
+ *     split from [tbr8] §5 item 1). An unquantized FP16 cache is supported for comparison
+ *     ([yunthe] section "vLLM推理引擎部署", --kv-cache-dtype fp16 vs int8).
+ *   - Dequantization happens inside the attention kernel; no fp16 copy of the cache is ever
+ *     written ([tbr8] §5 item 2, fused QuantizedPagedAttention operator).
+ *
+ * Device memory layout (all row-major, all owned by the caller):
+ *   k_codes  [num_blocks][num_kv_heads][block_size][head_dim]   int8   (PKV_INT8_SYM)
+ *                                                              fp16   (PKV_FP16)
+ *   v_codes  [num_blocks][num_kv_heads][block_size][head_dim]   int8 / fp16
+ *            [num_blocks][num_kv_heads][block_size][head_dim/2] uint8  (PKV_INT4_ASYM):
+ *            byte j of a token row = code[2j] | code[2j+1] << 4 (low nibble = even dim)
+ *   k_scale, v_scale [num_blocks][num_kv_heads] fp32   (NULL for an FP16 cache side)
+ *   v_zp     [num_blocks][num_kv_heads] uint8           (PKV_INT4_ASYM only, else NULL)
+ *   q, out   [num_seqs][num_q_heads][head_dim] fp16
+ *   block_tables [num_seqs][max_blocks_per_seq] int32: logical block i of sequence s lives in
+ *            physical block block_tables[s][i]
+ *   context_lens [num_seqs] int32 (tokens to attend over, including the token just stored)
+ *   slot_mapping [T] int64: slot = physical_block * block_size + offset; a negative slot skips
+ *            that token
+ *   new k, v [T][num_kv_heads][head_dim] fp16
+ *
+ * Conventions
+ *   - Every GPU entry point only enqueues work on `stream` and returns. PKV_OK means the launch
+ *     was accepted; argument errors are detected on the host before anything is launched and
+ *     leave all buffers untouched.
+ *   - The library allocates no device memory and keeps no global state; scratch space for the
+ *     decode is a caller-provided workspace (size from pkv_decode_workspace_size).
+ *   - Data errors that can only be seen on the device (a bad block id in a table, a bad slot)
+ *     never trap: the offending work is skipped and, if `dev_error` is non-NULL, the first error
+ *     code (PKV_DEVERR_*) is stored there with an atomic compare-and-swap (caller zeroes it).
+ *   - A cudaStream_t may be passed wherever pkv_stream_t is expected (same type).
+ */
+#ifndef PKV_H
+#define PKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st* pkv_stream_t; /* identical to cudaStream_t; NULL = legacy stream */
+
+typedef enum pkv_status {
+  PKV_OK = 0,
+  PKV_ERR_INVALID_ARG = 1,    /* null/misaligned pointer, bad size, inconsistent shapes */
+  PKV_ERR_UNSUPPORTED = 2,    /* well-formed but not built: dtype combination, head_dim, ... */
+  PKV_ERR_OUT_OF_BLOCKS = 3,  /* host allocator: not enough free blocks */
+  PKV_ERR_CUDA = 4,           /* a CUDA launch or query failed */
+  PKV_ERR_DEVICE_TIMEOUT = 5  /* reserved: a bounded device-side wait gave up */
+} pkv_status;
+
+typedef enum pkv_dtype {
+  PKV_FP16 = 0,      /* unquantized half precision */
+  PKV_INT8_SYM = 1,  /* int8 codes in [-127, 127], x_hat = code * scale */
+  PKV_INT4_ASYM = 2  /* uint4 codes in [0, 15], x_hat = (code - zp) * scale (V only) */
+} pkv_dtype;
+
+/* Device-side error codes written to *dev_error (first one wins). */
+enum {
+  PKV_DEVERR_NONE = 0,
+  PKV_DEVERR_BLOCK_ID = 1,     /* block id in a table / mapping outside [0, num_blocks) */
+  PKV_DEVERR_SLOT = 2,         /* slot_mapping entry beyond num_blocks * block_size */
+  PKV_DEVERR_SLOT_GROUP = 3,   /* tokens bound for one block are not consecutive offsets */
+  PKV_DEVERR_CONTEXT_LEN = 4,  /* context_len < 0, > max_context_len or > max_blocks*block_size */
+  PKV_DEVERR_TIMEOUT = 5       /* a bounded wait on an asynchronous copy gave up */
+};
+
+/* Describes one layer's cache pool. Pointers are device pointers, 16-byte aligned. */
+typedef struct pkv_cache_desc {
+  int32_t num_blocks;    /* nb: physical blocks in the pool */
+  int32_t block_size;    /* bs: tokens per block, 16 or 32 */
+  int32_t num_kv_heads;  /* Hkv */
+  int32_t head_dim;      /* D: 64, 128 or 256 */
+  int32_t k_dtype;       /* pkv_dtype: PKV_INT8_SYM or PKV_FP16 */
+  int32_t v_dtype;       /* pkv_dtype: PKV_INT8_SYM, PKV_INT4_ASYM or PKV_FP16 */
+  void* k_codes;
+  void* v_codes;
+  float* k_scale;        /* required when k_dtype != PKV_FP16 */
+  float* v_scale;        /* required when v_dtype != PKV_FP16 */
+  uint8_t* v_zp;         /* required when v_dtype == PKV_INT4_ASYM */
+} pkv_cache_desc;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* pkv_status_string(pkv_status status);
+
+/* Bytes of one (block, head) tile of K or V codes for this descriptor (0 on bad input). */
+size_t pkv_tile_bytes(const pkv_cache_desc* desc, int32_t which_v);
+
+/*
+ * pkv_store_quantized -- quantize T new tokens and scatter them into the pool.
+ *
+ * Follows [tbr8] §4 (store_kv: scale = absmax/127, codes = x/scale, scale stored per block) and
+ * [yunthe] "KV Cache量化技术原理" (Q(x) for the asymmetric INT4 form), with the readings:
+ * one scale (and zero point) per (block, KV head); round half to even; codes clamped to
+ * [-127, 127] (INT8) or [0, 15] (INT4); INT4 range [min(0, min x), max(0, max x)],
+ * scale = (hi - lo)/15, zp = clamp(rint(-lo/scale), 0, 15); scale 0 encodes an all-zero tile.
+ * All code arithmetic is IEEE binary32, round to nearest even, one rounding per operation.
+ *
+ * Tokens of one call that land in the same block must be adjacent in slot_mapping with
+ * consecutive increasing offsets (a "group"); a block may appear in at most one group per call.
+ * For a group at offsets o0..o1 of block b and each KV head:
+ *   o0 == 0:  the tile's scale (and zp) is derived from the group alone; codes [o0, o1] written.
+ *   o0 > 0:   if every new value is representable under the stored scale/zp ("fits"), new codes
+ *             use it and offsets < o0 are untouched; otherwise the tile is rebuilt: old codes at
+ *             offsets < o0 are dequantized in binary32, a new scale/zp is derived from them plus
+ *             the new values, and offsets 0..o1 are requantized.
+ * FP16 sides are copied as is.
+ *
+ *   k_new, v_new  device fp16 [T][num_kv_heads][head_dim]
+ *   slot_mapping  device int64 [T]; negative = skip; >= num_blocks*block_size -> PKV_DEVERR_SLOT
+ *   dev_error     device int32 or NULL
+ * Returns PKV_OK, PKV_ERR_INVALID_ARG, PKV_ERR_UNSUPPORTED or PKV_ERR_CUDA. T == 0 is a no-op.
+ */
+pkv_status pkv_store_quantized(const pkv_cache_desc* desc, const void* k_new, const void* v_new,
+                               const int64_t* slot_mapping, int32_t T, int32_t* dev_error,
+                               pkv_stream_t stream);
+
+/*
+ * pkv_decode_workspace_size -- bytes of scratch pkv_paged_attention_decode needs for these
+ * sizes: split-K partials (max, sum and fp32 accumulator per (seq, q head, partition)) only;
+ * never a dequantized copy of the cache. partition_tokens 0 selects the same automatic choice
+ * as the decode call. Returns PKV_ERR_INVALID_ARG on bad sizes.
+ */
+pkv_status pkv_decode_workspace_size(const pkv_cache_desc* desc, int32_t num_seqs,
+                                     int32_t num_q_heads, int32_t max_context_len,
+                                     int32_t partition_tokens, size_t* bytes);
+
+/*
+ * pkv_paged_attention_decode -- one decode step of attention over the paged, quantized cache.
+ *
+ * For every sequence s and query head h (KV head g = h / (num_q_heads / num_kv_heads)):
+ *   token t < L_s lives at physical block b = block_tables[s][t / bs], offset t % bs
+ *   ([yunthe] "PagedAttention分页注意力机制" block_table; [tbr8] §2);
+ *   k_hat = code * k_scale[b][g]; v_hat = (code - zp) * v_scale[b][g] ([yunthe] x_hat formula);
+ *   z_t = softmax_scale * dot(q[s][h], k_hat_t); out[s][h] = sum_t softmax(z)_t * v_hat_t,
+ *   written as fp16 (round to nearest). L_s == 0 gives out = 0.
+ * Long contexts are split into partitions of partition_tokens tokens (a multiple of block_size;
+ * 0 = automatic) whose partial results are merged by a second kernel.
+ *
+ *   q            device fp16 [num_seqs][num_q_heads][head_dim]
+ *   out          device fp16 [num_seqs][num_q_heads][head_dim]
+ *   block_tables device int32 [num_seqs][max_blocks_per_seq]
+ *   context_lens device int32 [num_seqs]; each <= max_context_len (host bound used to size the
+ *                grid) and <= max_blocks_per_seq * block_size, else PKV_DEVERR_CONTEXT_LEN and the
+ *                sequence is clamped
+ *   workspace    device, >= pkv_decode_workspace_size(...) bytes, 16-byte aligned; may be NULL
+ *                when that size is 0
+ *   dev_error    device int32 or NULL
+ * num_q_heads must be a multiple of num_kv_heads.
+ */
+pkv_status pkv_paged_attention_decode(const pkv_cache_desc* desc, void* out, const void* q,
+                                      int32_t num_seqs, int32_t num_q_heads,
+                                      const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                      const int32_t* context_lens, int32_t max_context_len,
+                                      float softmax_scale, int32_t partition_tokens,
+                                      void* workspace, size_t workspace_bytes, int32_t* dev_error,
+                                      pkv_stream_t stream);
+
+/*
+ * pkv_copy_blocks -- copy-on-write block copies ([deepinsea] section "Copy-on-Write 机制";
+ * [yunthe] "PagedAttention分页注意力机制", fork writes new tokens into new blocks).
+ * For each pair (src, dst) in block_mapping, copies every head's K codes, V codes, scales and
+ * zero points of block src into block dst. Pairs must not chain (no dst is another pair's src)
+ * and no dst may repeat. An id outside [0, num_blocks) skips the pair and sets
+ * PKV_DEVERR_BLOCK_ID.
+ *   block_mapping device int32 [n_pairs][2] = {src, dst}
+ */
+pkv_status pkv_copy_blocks(const pkv_cache_desc* desc, const int32_t* block_mapping,
+                           int32_t n_pairs, int32_t* dev_error, pkv_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Host block allocator: free list plus per-block reference counts, host memory only.
+ * Ceil-division sizing and the out-of-blocks failure follow [deepinsea] "分页机制设计"
+ * (BlockManager.allocate returns False when short); release-on-refcount follows [tbr8] §5
+ * item 3; fork/copy-on-write follows [deepinsea] "Copy-on-Write 机制". The free list is LIFO.
+ * A handle is not thread-safe.
+ * ------------------------------------------------------------------------------------------ */
+typedef struct pkv_allocator pkv_allocator;
+
+/* Number of blocks needed for num_tokens tokens: ceil(num_tokens / block_size); -1 if invalid. */
+int32_t pkv_blocks_for_tokens(int64_t num_tokens, int32_t block_size);
+
+pkv_status pkv_alloc_create(int32_t num_blocks, pkv_allocator** out_handle);
+void pkv_alloc_destroy(pkv_allocator* h);
+int32_t pkv_alloc_num_free(const pkv_allocator* h);
+/* Reference count of a block (0 = free); -1 for an id out of range. */
+int32_t pkv_alloc_refcount(const pkv_allocator* h, int32_t block_id);
+/* Take n blocks (refcount 1 each) into ids[0..n). All-or-nothing: PKV_ERR_OUT_OF_BLOCKS if
+ * fewer than n are free, in which case nothing is taken. */
+pkv_status pkv_alloc_blocks(pkv_allocator* h, int32_t n, int32_t* ids);
+/* Share n blocks with another sequence: refcount += 1 each. Ids must be allocated. */
+pkv_status pkv_alloc_fork(pkv_allocator* h, const int32_t* ids, int32_t n);
+/* Drop one reference from each of n blocks; a block returns to the free list at 0. */
+pkv_status pkv_alloc_release(pkv_allocator* h, const int32_t* ids, int32_t n);
+/* Make block_id private before a write. If its refcount is 1, *new_id = block_id and nothing
+ * changes. Otherwise a fresh block is taken (*new_id), the old block's refcount drops by one,
+ * and the caller must copy old -> new (pkv_copy_blocks) before writing. */
+pkv_status pkv_alloc_cow(pkv_allocator* h, int32_t block_id, int32_t* new_id);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKV_H */
