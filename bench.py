@@ -1,0 +1,410 @@
+#!/usr/bin/env python
+"""Benchmark: one decode step over a paged, block-quantized KV cache on B200, through the C ABI.
+
+A step is the whole hot path once: copy-on-write block copies (when the workload forks), store of
+one new token per sequence (quantize + scatter, pkv_store_quantized), then decode attention over
+every sequence (pkv_paged_attention_decode). The default workload is the Llama-2-7B-shaped
+decode layer (32 sequences, context lengths U{500..2000}, 32 heads MHA, head_dim 128, block size
+16, 8192-block pool, INT8 K and V with 1% outlier channels).
+
+Prints ONE JSON line (rank 0). `value` is whole-job decode KV tokens/s: tokens attended by all
+ranks / the slowest rank's device time (CUDA events, per step, L2 flushed between steps, inputs
+resident in HBM). `e2e` is the same metric with each step's inputs copied from pinned host memory
+and the output copied back inside the timed region. `roofline` rates the decode kernel's own
+event-timed duration against the measured HBM copy bandwidth. `cpu_baseline` times the CPU
+oracle (binary64) on a bounded sample of the workload (rank 0, one GPU only).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl pkv|reference]
+Multi-GPU: launched under torch.distributed.run, one process per GPU; each rank runs its own
+independently seeded copy of the workload (data-parallel over sequences, no exchange): weak scaling.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "decode KV tokens/s and effective HBM GB/s (fraction of ~8 TB/s) on 1 B200"
+UNIT = "KV tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+KV_NAMES = {0: "fp16", 1: "int8", 2: "int4"}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("pkv", "reference"), default="pkv")
+    ap.add_argument("--config", default="llama7b")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--partition-tokens", type=int, default=None)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- distributed
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and args.impl == "pkv":  # the reference arm runs on rank 0 alone, no group
+        import torch.distributed as dist
+        import torch
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def dist_max(value: float, world: int, device=None) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None:
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: str, enabled: bool = True):
+        self.gpu_index = gpu_index
+        self.enabled = enabled
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        if self.enabled:
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                     "-i", str(self.gpu_index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self.reader = threading.Thread(target=self._read, daemon=True)
+                self.reader.start()
+                time.sleep(0.3)
+            except OSError:
+                self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.reader.join(timeout=2)
+
+    def summary(self):
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, mx, reasons = [], 0.0, set()
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = max(mx, float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- helpers
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs: STREAM-style copy)"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback 6.65 TB/s (earlier copy measurement on this pool)"
+
+
+def decode_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("decode.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "paged_block_quantized_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(config: str):
+    """DRAM bytes per decode launch from the committed ncu summary of this workload, if the
+    summary was taken on the current decode kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", f"paged_decode_{config}.md")
+    try:
+        text = open(path, encoding="utf-8").read()
+    except OSError:
+        return None, None
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    hsh = re.search(r"decode_source_sha256_16:\s*([0-9a-f]+)", text)
+    if not m or not hsh or hsh.group(1) != decode_source_hash():
+        return None, path
+    return float(m.group(1)), path
+
+
+def config_block(w, g, step_desc):
+    return {
+        "workload": f"{w.name}: {w.description}",
+        "num_seqs": w.num_seqs, "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads,
+        "head_dim": w.head_dim, "block_size": w.block_size, "num_blocks": w.num_blocks,
+        "kv_dtype": f"{KV_NAMES[w.k_dtype]}/{KV_NAMES[w.v_dtype]}",
+        "tokens_per_step": w.total_tokens, "max_context_len": w.max_context_len,
+        "partition_tokens": g.partition_tokens if g is not None else w.partition_tokens,
+        "step": step_desc, "seed": w.seed,
+    }
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_pool_for(w, seqs):
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from _oracle_run import oracle_step  # noqa: E402
+    return oracle_step(w, seqs)
+
+
+def time_oracle_decode(w, budget_s: float, threads: int):
+    """Time the binary64 oracle decode on a bounded sample of the workload's sequences."""
+    import numpy as np
+    import oracle
+    order = list(range(w.num_seqs))
+    # calibrate on one sequence, then take as many sequences as fit about half the budget per run
+    o1 = oracle_pool_for(w, order[:1])
+    t0 = time.perf_counter()
+    oracle.decode(o1["cache"], o1["q"], o1["tables"], w.context_lens[o1["seqs"]], w.softmax_scale,
+                  max_context_len=w.max_context_len, num_threads=threads)
+    per_tok = max((time.perf_counter() - t0) / max(int(w.context_lens[0]), 1), 1e-9)
+    n = 1
+    while n < w.num_seqs and per_tok * w.context_lens[:n + 1].sum() < budget_s / 2:
+        n += 1
+    o = oracle_pool_for(w, order[:n])
+    lens = w.context_lens[o["seqs"]]
+    reps, elapsed = 0, 0.0
+    while elapsed < budget_s / 2 or reps == 0:
+        t0 = time.perf_counter()
+        oracle.decode(o["cache"], o["q"], o["tables"], lens, w.softmax_scale, max_context_len=w.max_context_len,
+                      num_threads=threads)
+        elapsed += time.perf_counter() - t0
+        reps += 1
+    tokens = int(lens.sum()) * reps
+    return {"value": tokens / elapsed, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{n} of {w.num_seqs} sequences ({int(lens.sum())} KV tokens) x {reps} runs of the binary64 "
+                      f"oracle decode ({elapsed:.1f} s, OpenMP over (sequence, head), {threads} threads)"}
+
+
+# ----------------------------------------------------------------------------- pkv arm
+def run_pkv(args, rank, world, local):
+    import numpy as np
+    import torch
+    from paged_block_quantized_b200 import workloads as W
+    from paged_block_quantized_b200.step import DeviceStep
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = W.make(args.config, seed=args.seed + rank)
+    g = DeviceStep(w, device=dev, poison=None, partition_tokens=args.partition_tokens)
+    g.prefill()
+    has_cow = w.cow_pairs.shape[0] > 0
+    launches_per_step = (1 if has_cow else 0) + 2
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        g.step()
+    torch.cuda.synchronize(dev)
+    assert g.error() == 0, f"device error {g.error()} in warm-up"
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    props = torch.cuda.get_device_properties(dev)
+    smi_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) is not None else str(dev.index)
+    with ClockSampler(smi_id, enabled=not args.no_clocks) as clk:
+        dist_barrier(world, dev)
+        torch.cuda.synchronize(dev)
+        wall0 = time.perf_counter()
+        for i in range(K):
+            flush.zero_()                 # outside the events: every step starts with a cold L2
+            ev[i][0].record(stream)
+            g.copy()
+            g.store()
+            ev[i][1].record(stream)
+            g.decode()
+            ev[i][2].record(stream)
+        torch.cuda.synchronize(dev)
+        dist_barrier(world, dev)
+        wall_ms = (time.perf_counter() - wall0) * 1e3
+    step_ms = [ev[i][0].elapsed_time(ev[i][2]) for i in range(K)]
+    dec_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+    total_s = dist_max(sum(step_ms) / 1e3, world, dev)
+    tokens_all = w.total_tokens * K * world
+    value = tokens_all / total_s
+
+    # ---- e2e: same step through the public runner with host buffers copied in and out ----
+    e2e = None
+    if not args.no_e2e:
+        pin = lambda t: t.cpu().pin_memory()
+        host_in = {"q": pin(g.q), "k_new": pin(g.k_new), "v_new": pin(g.v_new), "step_slots": pin(g.step_slots),
+                   "block_tables": pin(g.block_tables), "context_lens": pin(g.context_lens), "cow": pin(g.cow)}
+        host_out = torch.empty_like(g.out, device="cpu").pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+        d2h = host_out.numel() * host_out.element_size()
+
+        def e2e_step():
+            for name, t in host_in.items():
+                getattr(g, name).copy_(t, non_blocking=True)
+            g.step()
+            host_out.copy_(g.out, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+        dist_barrier(world, dev)
+        for i in range(K):
+            flush.zero_()
+            e_ev[i][0].record(stream)
+            e2e_step()
+            e_ev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        e_total = dist_max(sum(e_ev[i][0].elapsed_time(e_ev[i][1]) for i in range(K)) / 1e3, world, dev)
+        e2e = {"value": tokens_all / e_total, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "ms_per_step": e_total * 1e3 / K}
+        assert np.array_equal(host_out.numpy(), g.out.cpu().numpy())
+
+    assert g.error() == 0, f"device error {g.error()}"
+    dec_s = dist_max(statistics.mean(dec_ms) / 1e3, world, dev)
+    alg_bytes = w.decode_bytes(unique=True)
+    achieved = alg_bytes / dec_s / 1e9
+    peak, peak_src = measured_hbm_peak()
+    traffic, _ = ncu_traffic(args.config)
+    step_desc = ("copy-on-write copies + " if has_cow else "") + "store 1 token/seq (quantize+scatter) + decode"
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": total_s * 1e3 / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic (seeded N(0,1) fp16 K/V/q, permuted block pool)",
+        "config": {**config_block(w, g, step_desc), "parallelism": f"dp{world} (independent sequences per rank)",
+                   "l2": "flushed before every timed step (write of 2x L2)", "timing": "CUDA events per step"},
+        "effective_hbm_gbs": achieved, "frac_of_8tbs": achieved / 8000.0,
+        "decode_us": dec_s * 1e6,
+        "roofline": {"bound": "hbm", "kernel": "paged_decode_kernel", "achieved": achieved, "peak": peak,
+                     "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
+                     "algorithmic_bytes_per_launch": alg_bytes, "peak_source": peak_src},
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * K,
+        "wall_ms_timed_region": wall_ms,
+    }
+    clocks = clk.summary()
+    if clocks is not None:
+        line["clocks"] = clocks
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        threads = os.cpu_count() or 1
+        line["cpu_baseline"] = time_oracle_decode(w, args.cpu_seconds, threads)
+    return line
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args, rank, world):
+    """The CPU oracle as the reference arm: each step decodes a bounded sample of the workload."""
+    if rank != 0:
+        return None
+    import numpy as np
+    import oracle
+    from paged_block_quantized_b200 import workloads as W
+
+    w = W.make(args.config, seed=args.seed)
+    threads = os.cpu_count() or 1
+    per_step_budget = max(0.5, 150.0 / max(args.steps + args.warmup, 1))
+    o1 = oracle_pool_for(w, [0])
+    t0 = time.perf_counter()
+    oracle.decode(o1["cache"], o1["q"], o1["tables"], w.context_lens[:1], w.softmax_scale,
+                  max_context_len=w.max_context_len, num_threads=threads)
+    per_tok = max((time.perf_counter() - t0) / int(w.context_lens[0]), 1e-9)
+    n = 1
+    while n < w.num_seqs and per_tok * w.context_lens[:n + 1].sum() < per_step_budget:
+        n += 1
+    o = oracle_pool_for(w, list(range(n)))
+    lens = w.context_lens[o["seqs"]]
+    run = lambda: oracle.decode(o["cache"], o["q"], o["tables"], lens, w.softmax_scale,
+                                max_context_len=w.max_context_len, num_threads=threads)
+    for _ in range(args.warmup):
+        run()
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        run()
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = int(lens.sum()) * args.steps / total
+    sample = (f"{n} of {w.num_seqs} sequences ({int(lens.sum())} KV tokens) per step, binary64 oracle decode, "
+              f"OpenMP over (sequence, head), {threads} threads")
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total * 1e3 / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {**config_block(w, None, "decode (oracle, sampled sequences)"), "parallelism": "rank 0 only"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse_args()
+    rank, world, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, rank, world)
+        else:
+            line = run_pkv(args, rank, world, local)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1 and args.impl == "pkv":
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -58,6 +58,12 @@
 extern "C" {
 #endif
 
+#if defined(__GNUC__)
+#define PKV_API __attribute__((visibility("default")))
+#else
+#define PKV_API
+#endif
+
 struct CUstream_st;
 typedef struct CUstream_st* pkv_stream_t; /* identical to cudaStream_t; NULL = legacy stream */
 
@@ -102,10 +108,10 @@ typedef struct pkv_cache_desc {
 } pkv_cache_desc;
 
 /* Human-readable name of a status code (static string, never NULL). */
-const char* pkv_status_string(pkv_status status);
+PKV_API const char* pkv_status_string(pkv_status status);
 
 /* Bytes of one (block, head) tile of K or V codes for this descriptor (0 on bad input). */
-size_t pkv_tile_bytes(const pkv_cache_desc* desc, int32_t which_v);
+PKV_API size_t pkv_tile_bytes(const pkv_cache_desc* desc, int32_t which_v);
 
 /*
  * pkv_store_quantized -- quantize T new tokens and scatter them into the pool.
@@ -132,17 +138,18 @@ size_t pkv_tile_bytes(const pkv_cache_desc* desc, int32_t which_v);
  *   dev_error     device int32 or NULL
  * Returns PKV_OK, PKV_ERR_INVALID_ARG, PKV_ERR_UNSUPPORTED or PKV_ERR_CUDA. T == 0 is a no-op.
  */
-pkv_status pkv_store_quantized(const pkv_cache_desc* desc, const void* k_new, const void* v_new,
+PKV_API pkv_status pkv_store_quantized(const pkv_cache_desc* desc, const void* k_new, const void* v_new,
                                const int64_t* slot_mapping, int32_t T, int32_t* dev_error,
                                pkv_stream_t stream);
 
 /*
  * pkv_decode_workspace_size -- bytes of scratch pkv_paged_attention_decode needs for these
- * sizes: split-K partials (max, sum and fp32 accumulator per (seq, q head, partition)) only;
- * never a dequantized copy of the cache. partition_tokens 0 selects the same automatic choice
- * as the decode call. Returns PKV_ERR_INVALID_ARG on bad sizes.
+ * sizes: one arrival counter per (seq, CTA head group) plus the split-K partials (max, sum and
+ * fp32 accumulator per (seq, q head, partition)); never a dequantized copy of the cache.
+ * 0 when every sequence fits one partition. partition_tokens 0 selects the same automatic
+ * choice as the decode call. Returns PKV_ERR_INVALID_ARG on bad sizes.
  */
-pkv_status pkv_decode_workspace_size(const pkv_cache_desc* desc, int32_t num_seqs,
+PKV_API pkv_status pkv_decode_workspace_size(const pkv_cache_desc* desc, int32_t num_seqs,
                                      int32_t num_q_heads, int32_t max_context_len,
                                      int32_t partition_tokens, size_t* bytes);
 
@@ -155,8 +162,9 @@ pkv_status pkv_decode_workspace_size(const pkv_cache_desc* desc, int32_t num_seq
  *   k_hat = code * k_scale[b][g]; v_hat = (code - zp) * v_scale[b][g] ([yunthe] x_hat formula);
  *   z_t = softmax_scale * dot(q[s][h], k_hat_t); out[s][h] = sum_t softmax(z)_t * v_hat_t,
  *   written as fp16 (round to nearest). L_s == 0 gives out = 0.
- * Long contexts are split into partitions of partition_tokens tokens (a multiple of block_size;
- * 0 = automatic) whose partial results are merged by a second kernel.
+ * Long contexts are split into partitions of partition_tokens tokens (a multiple of block_size,
+ * at most 128 * block_size; 0 = automatic). Partition CTAs publish partial results to the
+ * workspace and the last one of a sequence to finish merges them, all in one kernel launch.
  *
  *   q            device fp16 [num_seqs][num_q_heads][head_dim]
  *   out          device fp16 [num_seqs][num_q_heads][head_dim]
@@ -165,11 +173,14 @@ pkv_status pkv_decode_workspace_size(const pkv_cache_desc* desc, int32_t num_seq
  *                grid) and <= max_blocks_per_seq * block_size, else PKV_DEVERR_CONTEXT_LEN and the
  *                sequence is clamped
  *   workspace    device, >= pkv_decode_workspace_size(...) bytes, 16-byte aligned; may be NULL
- *                when that size is 0
+ *                when that size is 0. It must be zero-filled before its first use: every call
+ *                that completes leaves its arrival counters at zero again, so one zeroing serves
+ *                any number of later calls (zero it again after a PKV_DEVERR_TIMEOUT). Calls that
+ *                share a workspace must not overlap on the GPU.
  *   dev_error    device int32 or NULL
  * num_q_heads must be a multiple of num_kv_heads.
  */
-pkv_status pkv_paged_attention_decode(const pkv_cache_desc* desc, void* out, const void* q,
+PKV_API pkv_status pkv_paged_attention_decode(const pkv_cache_desc* desc, void* out, const void* q,
                                       int32_t num_seqs, int32_t num_q_heads,
                                       const int32_t* block_tables, int32_t max_blocks_per_seq,
                                       const int32_t* context_lens, int32_t max_context_len,
@@ -186,7 +197,7 @@ pkv_status pkv_paged_attention_decode(const pkv_cache_desc* desc, void* out, con
  * PKV_DEVERR_BLOCK_ID.
  *   block_mapping device int32 [n_pairs][2] = {src, dst}
  */
-pkv_status pkv_copy_blocks(const pkv_cache_desc* desc, const int32_t* block_mapping,
+PKV_API pkv_status pkv_copy_blocks(const pkv_cache_desc* desc, const int32_t* block_mapping,
                            int32_t n_pairs, int32_t* dev_error, pkv_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------
@@ -199,24 +210,24 @@ pkv_status pkv_copy_blocks(const pkv_cache_desc* desc, const int32_t* block_mapp
 typedef struct pkv_allocator pkv_allocator;
 
 /* Number of blocks needed for num_tokens tokens: ceil(num_tokens / block_size); -1 if invalid. */
-int32_t pkv_blocks_for_tokens(int64_t num_tokens, int32_t block_size);
+PKV_API int32_t pkv_blocks_for_tokens(int64_t num_tokens, int32_t block_size);
 
-pkv_status pkv_alloc_create(int32_t num_blocks, pkv_allocator** out_handle);
-void pkv_alloc_destroy(pkv_allocator* h);
-int32_t pkv_alloc_num_free(const pkv_allocator* h);
+PKV_API pkv_status pkv_alloc_create(int32_t num_blocks, pkv_allocator** out_handle);
+PKV_API void pkv_alloc_destroy(pkv_allocator* h);
+PKV_API int32_t pkv_alloc_num_free(const pkv_allocator* h);
 /* Reference count of a block (0 = free); -1 for an id out of range. */
-int32_t pkv_alloc_refcount(const pkv_allocator* h, int32_t block_id);
+PKV_API int32_t pkv_alloc_refcount(const pkv_allocator* h, int32_t block_id);
 /* Take n blocks (refcount 1 each) into ids[0..n). All-or-nothing: PKV_ERR_OUT_OF_BLOCKS if
  * fewer than n are free, in which case nothing is taken. */
-pkv_status pkv_alloc_blocks(pkv_allocator* h, int32_t n, int32_t* ids);
+PKV_API pkv_status pkv_alloc_blocks(pkv_allocator* h, int32_t n, int32_t* ids);
 /* Share n blocks with another sequence: refcount += 1 each. Ids must be allocated. */
-pkv_status pkv_alloc_fork(pkv_allocator* h, const int32_t* ids, int32_t n);
+PKV_API pkv_status pkv_alloc_fork(pkv_allocator* h, const int32_t* ids, int32_t n);
 /* Drop one reference from each of n blocks; a block returns to the free list at 0. */
-pkv_status pkv_alloc_release(pkv_allocator* h, const int32_t* ids, int32_t n);
+PKV_API pkv_status pkv_alloc_release(pkv_allocator* h, const int32_t* ids, int32_t n);
 /* Make block_id private before a write. If its refcount is 1, *new_id = block_id and nothing
  * changes. Otherwise a fresh block is taken (*new_id), the old block's refcount drops by one,
  * and the caller must copy old -> new (pkv_copy_blocks) before writing. */
-pkv_status pkv_alloc_cow(pkv_allocator* h, int32_t block_id, int32_t* new_id);
+PKV_API pkv_status pkv_alloc_cow(pkv_allocator* h, int32_t block_id, int32_t* new_id);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,257 @@
+// api.cu -- the C ABI of include/pkv.h: host-side validation, launch geometry, dispatch.
+//
+// Every entry point checks its arguments on the host before anything is enqueued and returns
+// PKV_ERR_INVALID_ARG / PKV_ERR_UNSUPPORTED without touching device memory; a launch failure is
+// reported as PKV_ERR_CUDA. Nothing here allocates device memory or keeps per-call state.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "../../include/pkv.h"
+#include "internal.h"
+
+namespace {
+
+using namespace pkv;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool dtype_known_k(int32_t d) { return d == PKV_FP16 || d == PKV_INT8_SYM; }
+bool dtype_known_v(int32_t d) { return d == PKV_FP16 || d == PKV_INT8_SYM || d == PKV_INT4_ASYM; }
+
+int64_t row_bytes(int32_t dtype, int32_t head_dim) {
+  if (dtype == PKV_FP16) return 2 * (int64_t)head_dim;
+  if (dtype == PKV_INT8_SYM) return head_dim;
+  return head_dim / 2;
+}
+
+// Checks shared by every call that reads or writes the pool.
+pkv_status check_desc(const pkv_cache_desc* d) {
+  if (d == nullptr) return PKV_ERR_INVALID_ARG;
+  if (d->num_blocks <= 0 || d->num_kv_heads <= 0 || d->head_dim <= 0 || d->block_size <= 0)
+    return PKV_ERR_INVALID_ARG;
+  if (d->head_dim % 16 != 0) return PKV_ERR_INVALID_ARG;
+  if (!dtype_known_k(d->k_dtype) || !dtype_known_v(d->v_dtype)) return PKV_ERR_INVALID_ARG;
+  if (d->block_size != 16 && d->block_size != 32) return PKV_ERR_UNSUPPORTED;
+  if (d->head_dim != 64 && d->head_dim != 128 && d->head_dim != 256) return PKV_ERR_UNSUPPORTED;
+  if (d->k_codes == nullptr || d->v_codes == nullptr) return PKV_ERR_INVALID_ARG;
+  if (!aligned(d->k_codes, 16) || !aligned(d->v_codes, 16)) return PKV_ERR_INVALID_ARG;
+  if (d->k_dtype != PKV_FP16 && (d->k_scale == nullptr || !aligned(d->k_scale, 4))) return PKV_ERR_INVALID_ARG;
+  if (d->v_dtype != PKV_FP16 && (d->v_scale == nullptr || !aligned(d->v_scale, 4))) return PKV_ERR_INVALID_ARG;
+  if (d->v_dtype == PKV_INT4_ASYM && d->v_zp == nullptr) return PKV_ERR_INVALID_ARG;
+  return PKV_OK;
+}
+
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  int& c = cached[dev & 63];
+  if (c == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    c = n;
+  }
+  return c;
+}
+
+// Automatic partition size: the longest partition (fewest partials to merge) that still gives
+// every SM several CTAs of work; never shorter than one block per warp.
+int32_t auto_partition(const pkv_cache_desc* d, int32_t num_seqs, int32_t num_q_heads, int32_t max_context_len) {
+  const int32_t bs = d->block_size;
+  const int32_t group = num_q_heads / d->num_kv_heads;
+  const int64_t units = (int64_t)num_seqs * (num_q_heads / decode_heads_per_cta(group));
+  const int64_t target = (int64_t)sm_count() * 12;
+  const int32_t cap = decode_max_partition_tokens(bs);
+  int32_t pt = cap < 1024 ? cap : 1024;
+  const int32_t floor_pt = 4 * bs;
+  while (pt > floor_pt) {
+    const int64_t parts = (max_context_len + pt - 1) / pt;
+    if (units * (parts > 0 ? parts : 1) >= target) break;
+    pt /= 2;
+  }
+  if (pt < floor_pt) pt = floor_pt;
+  return pt - pt % bs;
+}
+
+struct DecodeGeometry {
+  int32_t partition_tokens;
+  int32_t max_partitions;
+  size_t counter_bytes;    // arrival counters at the start of the workspace (256-byte padded)
+  size_t workspace_bytes;  // counters + partial (max, sum) + partial accumulators
+};
+
+pkv_status decode_geometry(const pkv_cache_desc* d, int32_t num_seqs, int32_t num_q_heads,
+                           int32_t max_context_len, int32_t partition_tokens, DecodeGeometry* g) {
+  if (num_seqs < 0 || num_q_heads <= 0 || max_context_len < 0 || partition_tokens < 0) return PKV_ERR_INVALID_ARG;
+  if (num_q_heads % d->num_kv_heads != 0) return PKV_ERR_INVALID_ARG;
+  int32_t pt = partition_tokens;
+  if (pt == 0) {
+    pt = auto_partition(d, num_seqs, num_q_heads, max_context_len);
+  } else {
+    if (pt % d->block_size != 0) return PKV_ERR_INVALID_ARG;
+    if (pt > decode_max_partition_tokens(d->block_size)) return PKV_ERR_UNSUPPORTED;
+  }
+  int64_t parts = ((int64_t)max_context_len + pt - 1) / pt;
+  if (parts < 1) parts = 1;
+  if (parts > 65535 || num_seqs > 65535) return PKV_ERR_UNSUPPORTED;  // grid limits
+  g->partition_tokens = pt;
+  g->max_partitions = (int32_t)parts;
+  if (parts > 1) {
+    const size_t counters = (size_t)num_seqs * (num_q_heads / decode_heads_per_cta(num_q_heads / d->num_kv_heads));
+    g->counter_bytes = (counters * sizeof(uint32_t) + 255) / 256 * 256;
+    g->workspace_bytes = g->counter_bytes + (size_t)num_seqs * num_q_heads * parts * (d->head_dim + 2) * sizeof(float);
+  } else {
+    g->counter_bytes = 0;
+    g->workspace_bytes = 0;
+  }
+  return PKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pkv_status_string(pkv_status status) {
+  switch (status) {
+    case PKV_OK: return "PKV_OK";
+    case PKV_ERR_INVALID_ARG: return "PKV_ERR_INVALID_ARG";
+    case PKV_ERR_UNSUPPORTED: return "PKV_ERR_UNSUPPORTED";
+    case PKV_ERR_OUT_OF_BLOCKS: return "PKV_ERR_OUT_OF_BLOCKS";
+    case PKV_ERR_CUDA: return "PKV_ERR_CUDA";
+    case PKV_ERR_DEVICE_TIMEOUT: return "PKV_ERR_DEVICE_TIMEOUT";
+  }
+  return "PKV_ERR_UNKNOWN";
+}
+
+size_t pkv_tile_bytes(const pkv_cache_desc* desc, int32_t which_v) {
+  if (desc == nullptr || desc->head_dim <= 0 || desc->block_size <= 0) return 0;
+  const int32_t dt = which_v ? desc->v_dtype : desc->k_dtype;
+  if (which_v ? !dtype_known_v(dt) : !dtype_known_k(dt)) return 0;
+  return (size_t)desc->block_size * (size_t)row_bytes(dt, desc->head_dim);
+}
+
+pkv_status pkv_store_quantized(const pkv_cache_desc* desc, const void* k_new, const void* v_new,
+                               const int64_t* slot_mapping, int32_t T, int32_t* dev_error, pkv_stream_t stream) {
+  pkv_status st = check_desc(desc);
+  if (st != PKV_OK) return st;
+  if (T < 0) return PKV_ERR_INVALID_ARG;
+  if (T == 0) return PKV_OK;
+  if (k_new == nullptr || v_new == nullptr || slot_mapping == nullptr) return PKV_ERR_INVALID_ARG;
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(slot_mapping, 8)) return PKV_ERR_INVALID_ARG;
+  if (dev_error != nullptr && !aligned(dev_error, 4)) return PKV_ERR_INVALID_ARG;
+  StoreParams p;
+  p.k_codes = desc->k_codes;
+  p.v_codes = desc->v_codes;
+  p.k_scale = desc->k_scale;
+  p.v_scale = desc->v_scale;
+  p.v_zp = desc->v_zp;
+  p.k_new = static_cast<const __half*>(k_new);
+  p.v_new = static_cast<const __half*>(v_new);
+  p.slot_mapping = slot_mapping;
+  p.dev_error = dev_error;
+  p.T = T;
+  p.num_blocks = desc->num_blocks;
+  p.num_kv_heads = desc->num_kv_heads;
+  p.block_size = desc->block_size;
+  p.head_dim = desc->head_dim;
+  p.k_dtype = desc->k_dtype;
+  p.v_dtype = desc->v_dtype;
+  return launch_store(p, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+pkv_status pkv_decode_workspace_size(const pkv_cache_desc* desc, int32_t num_seqs, int32_t num_q_heads,
+                                     int32_t max_context_len, int32_t partition_tokens, size_t* bytes) {
+  if (bytes == nullptr) return PKV_ERR_INVALID_ARG;
+  pkv_status st = check_desc(desc);
+  if (st != PKV_OK) return st;
+  DecodeGeometry g;
+  st = decode_geometry(desc, num_seqs, num_q_heads, max_context_len, partition_tokens, &g);
+  if (st != PKV_OK) return st;
+  *bytes = g.workspace_bytes;
+  return PKV_OK;
+}
+
+pkv_status pkv_paged_attention_decode(const pkv_cache_desc* desc, void* out, const void* q, int32_t num_seqs,
+                                      int32_t num_q_heads, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                      const int32_t* context_lens, int32_t max_context_len, float softmax_scale,
+                                      int32_t partition_tokens, void* workspace, size_t workspace_bytes,
+                                      int32_t* dev_error, pkv_stream_t stream) {
+  pkv_status st = check_desc(desc);
+  if (st != PKV_OK) return st;
+  if (!decode_supported(desc->k_dtype, desc->v_dtype, desc->block_size, desc->head_dim)) return PKV_ERR_UNSUPPORTED;
+  DecodeGeometry g;
+  st = decode_geometry(desc, num_seqs, num_q_heads, max_context_len, partition_tokens, &g);
+  if (st != PKV_OK) return st;
+  if (num_seqs == 0) return PKV_OK;
+  if (out == nullptr || q == nullptr || block_tables == nullptr || context_lens == nullptr) return PKV_ERR_INVALID_ARG;
+  if (!aligned(out, 16) || !aligned(q, 16) || !aligned(block_tables, 4) || !aligned(context_lens, 4))
+    return PKV_ERR_INVALID_ARG;
+  if (max_blocks_per_seq <= 0) return PKV_ERR_INVALID_ARG;
+  if (dev_error != nullptr && !aligned(dev_error, 4)) return PKV_ERR_INVALID_ARG;
+  if (g.workspace_bytes > 0 && (workspace == nullptr || workspace_bytes < g.workspace_bytes || !aligned(workspace, 16)))
+    return PKV_ERR_INVALID_ARG;
+  if (!(softmax_scale == softmax_scale)) return PKV_ERR_INVALID_ARG;  // NaN
+
+  DecodeParams p;
+  p.k_codes = desc->k_codes;
+  p.v_codes = desc->v_codes;
+  p.k_scale = desc->k_scale;
+  p.v_scale = desc->v_scale;
+  p.v_zp = desc->v_zp;
+  p.q = static_cast<const __half*>(q);
+  p.out = static_cast<__half*>(out);
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  const size_t ml_floats = (size_t)num_seqs * num_q_heads * g.max_partitions * 2;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  p.ws_count = g.workspace_bytes ? reinterpret_cast<uint32_t*>(ws) : nullptr;
+  p.ws_ml = g.workspace_bytes ? reinterpret_cast<float*>(ws + g.counter_bytes) : nullptr;
+  p.ws_acc = g.workspace_bytes ? reinterpret_cast<float*>(ws + g.counter_bytes) + ml_floats : nullptr;
+  p.dev_error = dev_error;
+  p.num_blocks = desc->num_blocks;
+  p.num_kv_heads = desc->num_kv_heads;
+  p.num_q_heads = num_q_heads;
+  p.group = num_q_heads / desc->num_kv_heads;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.max_context_len = max_context_len;
+  p.partition_tokens = g.partition_tokens;
+  p.max_partitions = g.max_partitions;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;  // log2(e)
+
+  DecodeShape sh;
+  sh.k_dtype = desc->k_dtype;
+  sh.v_dtype = desc->v_dtype;
+  sh.block_size = desc->block_size;
+  sh.head_dim = desc->head_dim;
+  sh.heads_per_cta = decode_heads_per_cta(p.group);
+  sh.num_seqs = num_seqs;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return launch_decode(p, sh, s) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+pkv_status pkv_copy_blocks(const pkv_cache_desc* desc, const int32_t* block_mapping, int32_t n_pairs,
+                           int32_t* dev_error, pkv_stream_t stream) {
+  pkv_status st = check_desc(desc);
+  if (st != PKV_OK) return st;
+  if (n_pairs < 0) return PKV_ERR_INVALID_ARG;
+  if (n_pairs == 0) return PKV_OK;
+  if (block_mapping == nullptr || !aligned(block_mapping, 4)) return PKV_ERR_INVALID_ARG;
+  if (dev_error != nullptr && !aligned(dev_error, 4)) return PKV_ERR_INVALID_ARG;
+  CopyParams p;
+  p.k_codes = static_cast<uint8_t*>(desc->k_codes);
+  p.v_codes = static_cast<uint8_t*>(desc->v_codes);
+  p.k_scale = desc->k_dtype != PKV_FP16 ? desc->k_scale : nullptr;
+  p.v_scale = desc->v_dtype != PKV_FP16 ? desc->v_scale : nullptr;
+  p.v_zp = desc->v_dtype == PKV_INT4_ASYM ? desc->v_zp : nullptr;
+  p.block_mapping = block_mapping;
+  p.dev_error = dev_error;
+  p.n_pairs = n_pairs;
+  p.num_blocks = desc->num_blocks;
+  p.num_kv_heads = desc->num_kv_heads;
+  p.k_block_bytes = (int64_t)desc->num_kv_heads * desc->block_size * row_bytes(desc->k_dtype, desc->head_dim);
+  p.v_block_bytes = (int64_t)desc->num_kv_heads * desc->block_size * row_bytes(desc->v_dtype, desc->head_dim);
+  return launch_copy(p, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+}  // extern "C"

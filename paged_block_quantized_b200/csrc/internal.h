@@ -1,0 +1,91 @@
+// internal.h -- kernel launch interfaces behind the C ABI (not part of the public header).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/pkv.h"
+
+namespace pkv {
+
+// ---------------------------------------------------------------- decode
+struct DecodeParams {
+  const void* k_codes;
+  const void* v_codes;
+  const float* k_scale;
+  const float* v_scale;
+  const uint8_t* v_zp;
+  const __half* q;
+  __half* out;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  uint32_t* ws_count;  // [S][Hq / heads_per_cta] arrival counters (zero between calls)
+  float* ws_ml;        // [S][Hq][max_partitions][2] running max (log2 domain) and sum
+  float* ws_acc;       // [S][Hq][max_partitions][D] un-normalised accumulators
+  int32_t* dev_error;
+  int32_t num_blocks;
+  int32_t num_kv_heads;
+  int32_t num_q_heads;
+  int32_t group;  // num_q_heads / num_kv_heads
+  int32_t max_blocks_per_seq;
+  int32_t max_context_len;
+  int32_t partition_tokens;
+  int32_t max_partitions;
+  float scale_log2;  // softmax_scale * log2(e)
+};
+
+struct DecodeShape {
+  int32_t k_dtype, v_dtype, block_size, head_dim;
+  int32_t heads_per_cta;  // query heads handled by one CTA (divides group)
+  int32_t num_seqs;
+};
+
+// Query heads per CTA for a group size (largest of 4, 2, 1 that divides it).
+int32_t decode_heads_per_cta(int32_t group);
+// Largest partition the decode kernel accepts for this block size (a warp keeps the ids of its
+// blocks in registers, one per lane).
+int32_t decode_max_partition_tokens(int32_t block_size);
+bool decode_supported(int32_t k_dtype, int32_t v_dtype, int32_t block_size, int32_t head_dim);
+
+cudaError_t launch_decode(const DecodeParams& p, const DecodeShape& sh, cudaStream_t stream);
+
+// ---------------------------------------------------------------- store
+struct StoreParams {
+  void* k_codes;
+  void* v_codes;
+  float* k_scale;
+  float* v_scale;
+  uint8_t* v_zp;
+  const __half* k_new;
+  const __half* v_new;
+  const int64_t* slot_mapping;
+  int32_t* dev_error;
+  int32_t T;
+  int32_t num_blocks;
+  int32_t num_kv_heads;
+  int32_t block_size;
+  int32_t head_dim;
+  int32_t k_dtype;
+  int32_t v_dtype;
+};
+cudaError_t launch_store(const StoreParams& p, cudaStream_t stream);
+
+// ---------------------------------------------------------------- copy
+struct CopyParams {
+  uint8_t* k_codes;
+  uint8_t* v_codes;
+  float* k_scale;
+  float* v_scale;
+  uint8_t* v_zp;
+  const int32_t* block_mapping;
+  int32_t* dev_error;
+  int32_t n_pairs;
+  int32_t num_blocks;
+  int32_t num_kv_heads;
+  int64_t k_block_bytes;  // bytes of one block of K codes (all heads)
+  int64_t v_block_bytes;
+};
+cudaError_t launch_copy(const CopyParams& p, cudaStream_t stream);
+
+}  // namespace pkv

@@ -1,0 +1,327 @@
+// store.cu -- quantize new K/V tokens and scatter them into pool blocks (sm_100a).
+//
+// Follows tbr8.org "如何通过 PagedAttention 与分块量化结合：解决移动端内存碎片化导致的长文本 OOM" §4
+// (store_kv: scale = absmax / 127 per block, codes = x / scale, one scale stored per block and
+// head) and yunthe.com "LLM推理显存优化KV Cache量化与PagedAttention实现详解", section
+// "KV Cache量化技术原理" (asymmetric Q(x) = clamp(round(x/scale + zero_point), 0, 2^bits - 1)),
+// with K INT8 / V INT4 as the tbr8.org page advises in §5 item 1. Readings where the pages are
+// silent: ties round to even; INT8 codes in [-127, 127]; INT4 range [min(0, min x), max(0, max x)],
+// scale = (hi - lo) / 15, zp = clamp(rint(-lo / scale), 0, 15); scale 0 encodes an all-zero tile;
+// nibbles packed along head_dim, low nibble = even dim; appending into a partly filled tile keeps
+// the stored scale when every new value fits and otherwise rebuilds the tile from the
+// dequantized old codes plus the new values.
+//
+// Bit-exactness: every arithmetic step is an explicit IEEE binary32 round-to-nearest intrinsic
+// (__fdiv_rn, __fmul_rn, __fadd_rn, __fsub_rn) so nvcc cannot contract or reorder it, and
+// __float2int_rn rounds half to even. Maxima and minima are order independent.
+//
+// Work split: one warp per (token, KV head). The warp of the first token of a group (the run of
+// tokens bound for one block) does the whole group; the others return at once.
+#include "common.cuh"
+#include "internal.h"
+
+namespace pkv {
+
+namespace {
+
+constexpr uint32_t kFull = 0xffffffffu;
+constexpr int kWarpsPerCta = 4;
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, off));
+  return v;
+}
+__device__ __forceinline__ float warp_min(float v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v = fminf(v, __shfl_xor_sync(kFull, v, off));
+  return v;
+}
+
+// 4 fp16 values at p (8-byte aligned) -> floats (exact widening)
+__device__ __forceinline__ void load4(const __half* p, float f[4]) {
+  const uint2 w = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&w.x));
+  const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&w.y));
+  f[0] = a.x;
+  f[1] = a.y;
+  f[2] = b.x;
+  f[3] = b.y;
+}
+
+// symmetric: 0 if s == 0, else clamp(rint(x / s), -127, 127)
+__device__ __forceinline__ int quant_sym(float x, float s) {
+  if (s == 0.0f) return 0;
+  const int r = __float2int_rn(__fdiv_rn(x, s));
+  return min(127, max(-127, r));
+}
+
+// asymmetric 4-bit: zp if s == 0, else clamp(rint(x / s + zp), 0, 15)
+__device__ __forceinline__ int quant_asym(float x, float s, int zp) {
+  if (s == 0.0f) return zp;
+  const int r = __float2int_rn(__fadd_rn(__fdiv_rn(x, s), (float)zp));
+  return min(15, max(0, r));
+}
+
+__device__ __forceinline__ void derive_asym(float lo, float hi, float& s, int& zp) {
+  s = __fdiv_rn(__fsub_rn(hi, lo), 15.0f);
+  zp = 0;
+  if (s != 0.0f) zp = min(15, max(0, __float2int_rn(__fdiv_rn(-lo, s))));
+}
+
+// Values of the group for one head: element e of token i at src + i * row_stride + e.
+struct GroupSrc {
+  const __half* base;  // token 0 of the group, this head
+  int64_t row_stride;  // elements between tokens (num_kv_heads * head_dim)
+  int n;               // tokens in the group
+  int d;               // head_dim
+};
+
+// ---- INT8 symmetric side of one (block, head) tile ----
+__device__ void store_sym(const GroupSrc& src, int8_t* tile, float* scale_ptr, int o0, int lane) {
+  const int d = src.d, n = src.n;
+  const int quads = n * d / 4;
+  float m_new = 0.0f;
+  for (int e = lane; e < quads; e += 32) {
+    const int i = (4 * e) / d, j = (4 * e) % d;
+    float f[4];
+    load4(src.base + i * src.row_stride + j, f);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) m_new = fmaxf(m_new, fabsf(f[u]));
+  }
+  m_new = warp_max(m_new);
+
+  float s;
+  if (o0 == 0) {
+    s = __fdiv_rn(m_new, 127.0f);
+  } else {
+    const float s_old = *scale_ptr;
+    bool fits = true;
+    for (int e = lane; e < quads; e += 32) {
+      const int i = (4 * e) / d, j = (4 * e) % d;
+      float f[4];
+      load4(src.base + i * src.row_stride + j, f);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (s_old == 0.0f) {
+          fits = fits && (f[u] == 0.0f);
+        } else {
+          const int r = __float2int_rn(__fdiv_rn(f[u], s_old));
+          fits = fits && (r <= 127 && r >= -127);
+        }
+      }
+    }
+    fits = __all_sync(kFull, fits);
+    if (fits) {
+      s = s_old;
+    } else {
+      // rebuild: old codes -> binary32 x_hat = code * s_old; scale from old and new together
+      const int old_quads = o0 * d / 4;
+      float m_old = 0.0f;
+      for (int e = lane; e < old_quads; e += 32) {
+        const uint32_t w = reinterpret_cast<const uint32_t*>(tile)[e];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int q = (int)(int8_t)((w >> (8 * u)) & 0xff);
+          m_old = fmaxf(m_old, fabsf(__fmul_rn((float)q, s_old)));
+        }
+      }
+      m_old = warp_max(m_old);
+      s = __fdiv_rn(fmaxf(m_old, m_new), 127.0f);
+      for (int e = lane; e < old_quads; e += 32) {
+        uint32_t w = reinterpret_cast<const uint32_t*>(tile)[e];
+        uint32_t out = 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int q = (int)(int8_t)((w >> (8 * u)) & 0xff);
+          const int r = quant_sym(__fmul_rn((float)q, s_old), s);
+          out |= ((uint32_t)(r & 0xff)) << (8 * u);
+        }
+        reinterpret_cast<uint32_t*>(tile)[e] = out;
+      }
+    }
+  }
+  // new codes
+  int8_t* dst = tile + (size_t)o0 * d;
+  for (int e = lane; e < quads; e += 32) {
+    const int i = (4 * e) / d, j = (4 * e) % d;
+    float f[4];
+    load4(src.base + i * src.row_stride + j, f);
+    uint32_t out = 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) out |= ((uint32_t)(quant_sym(f[u], s) & 0xff)) << (8 * u);
+    reinterpret_cast<uint32_t*>(dst)[e] = out;
+  }
+  if (lane == 0) *scale_ptr = s;
+}
+
+// ---- INT4 asymmetric side: tile is [bs][d/2] bytes, byte j = code[2j] | code[2j+1] << 4 ----
+__device__ void store_asym4(const GroupSrc& src, uint8_t* tile, float* scale_ptr, uint8_t* zp_ptr, int o0,
+                            int lane) {
+  const int d = src.d, n = src.n;
+  const int quads = n * d / 4;  // 4 values -> 2 bytes
+  float lo = 0.0f, hi = 0.0f;
+  for (int e = lane; e < quads; e += 32) {
+    const int i = (4 * e) / d, j = (4 * e) % d;
+    float f[4];
+    load4(src.base + i * src.row_stride + j, f);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      lo = fminf(lo, f[u]);
+      hi = fmaxf(hi, f[u]);
+    }
+  }
+  lo = warp_min(lo);
+  hi = warp_max(hi);
+
+  float s;
+  int zp;
+  if (o0 == 0) {
+    derive_asym(lo, hi, s, zp);
+  } else {
+    const float s_old = *scale_ptr;
+    const int zp_old = *zp_ptr;
+    bool fits = true;
+    for (int e = lane; e < quads; e += 32) {
+      const int i = (4 * e) / d, j = (4 * e) % d;
+      float f[4];
+      load4(src.base + i * src.row_stride + j, f);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (s_old == 0.0f) {
+          fits = fits && (f[u] == 0.0f);
+        } else {
+          const int r = __float2int_rn(__fadd_rn(__fdiv_rn(f[u], s_old), (float)zp_old));
+          fits = fits && (r >= 0 && r <= 15);
+        }
+      }
+    }
+    fits = __all_sync(kFull, fits);
+    if (fits) {
+      s = s_old;
+      zp = zp_old;
+    } else {
+      // rebuild: x_hat = (code - zp_old) * s_old in binary32; range over old and new values
+      const int old_bytes = o0 * d / 2;
+      for (int e = lane; e < old_bytes; e += 32) {
+        const uint8_t byte = tile[e];
+        const float a = __fmul_rn((float)((int)(byte & 0xF) - zp_old), s_old);
+        const float b = __fmul_rn((float)((int)(byte >> 4) - zp_old), s_old);
+        lo = fminf(lo, fminf(a, b));
+        hi = fmaxf(hi, fmaxf(a, b));
+      }
+      lo = warp_min(lo);
+      hi = warp_max(hi);
+      derive_asym(lo, hi, s, zp);
+      for (int e = lane; e < old_bytes; e += 32) {
+        const uint8_t byte = tile[e];
+        const float a = __fmul_rn((float)((int)(byte & 0xF) - zp_old), s_old);
+        const float b = __fmul_rn((float)((int)(byte >> 4) - zp_old), s_old);
+        tile[e] = (uint8_t)(quant_asym(a, s, zp) | (quant_asym(b, s, zp) << 4));
+      }
+    }
+  }
+  uint8_t* dst = tile + (size_t)o0 * (d / 2);
+  for (int e = lane; e < quads; e += 32) {
+    const int i = (4 * e) / d, j = (4 * e) % d;
+    float f[4];
+    load4(src.base + i * src.row_stride + j, f);
+    const uint32_t b0 = (uint32_t)(quant_asym(f[0], s, zp) | (quant_asym(f[1], s, zp) << 4));
+    const uint32_t b1 = (uint32_t)(quant_asym(f[2], s, zp) | (quant_asym(f[3], s, zp) << 4));
+    reinterpret_cast<uint16_t*>(dst)[e] = (uint16_t)(b0 | (b1 << 8));
+  }
+  if (lane == 0) {
+    *scale_ptr = s;
+    *zp_ptr = (uint8_t)zp;
+  }
+}
+
+// ---- FP16 side: values stored as given ----
+__device__ void store_fp16(const GroupSrc& src, __half* tile, int o0, int lane) {
+  const int d = src.d, n = src.n;
+  const int vecs = n * d / 8;  // 16-byte vectors
+  __half* dst = tile + (size_t)o0 * d;
+  for (int e = lane; e < vecs; e += 32) {
+    const int i = (8 * e) / d, j = (8 * e) % d;
+    reinterpret_cast<uint4*>(dst + (size_t)i * d)[j / 8] =
+        *reinterpret_cast<const uint4*>(src.base + i * src.row_stride + j);
+  }
+}
+
+__global__ void __launch_bounds__(32 * kWarpsPerCta) store_quantized_kernel(const StoreParams p) {
+  const int t = blockIdx.x;
+  const int h = blockIdx.y * kWarpsPerCta + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (h >= p.num_kv_heads) return;
+  const int bs = p.block_size;
+  const int64_t num_slots = (int64_t)p.num_blocks * bs;
+  const int64_t slot = p.slot_mapping[t];
+  if (slot < 0) return;  // padding token
+  if (slot >= num_slots) {
+    if (h == 0 && lane == 0) record_error(p.dev_error, PKV_DEVERR_SLOT);
+    return;
+  }
+  const int64_t block = slot / bs;
+  if (t > 0) {
+    const int64_t prev = p.slot_mapping[t - 1];
+    if (prev >= 0 && prev < num_slots && prev / bs == block) return;  // not the group's first token
+  }
+  // the group: following tokens with a valid slot in the same block; offsets must be consecutive
+  int n = 1;
+  bool consecutive = true;
+  while (true) {
+    const int idx = t + n + lane;
+    bool same = false, step_ok = true;
+    if (idx < p.T) {
+      const int64_t sl = p.slot_mapping[idx];
+      same = sl >= 0 && sl < num_slots && sl / bs == block;
+      step_ok = sl == slot + n + lane;
+    }
+    const uint32_t run_mask = __ballot_sync(kFull, same);
+    const int run = (run_mask == kFull) ? 32 : (__ffs(~run_mask) - 1);
+    const uint32_t bad = __ballot_sync(kFull, same && !step_ok && lane < run);
+    if (bad) consecutive = false;
+    n += run;
+    if (run < 32 || n > bs) break;
+  }
+  if (!consecutive || n > bs) {
+    if (h == 0 && lane == 0) record_error(p.dev_error, PKV_DEVERR_SLOT_GROUP);
+    return;
+  }
+  const int o0 = (int)(slot % bs);
+  const int d = p.head_dim;
+  const size_t tile_idx = (size_t)block * p.num_kv_heads + h;
+  GroupSrc src;
+  src.row_stride = (int64_t)p.num_kv_heads * d;
+  src.n = n;
+  src.d = d;
+
+  // K side
+  src.base = p.k_new + (size_t)t * src.row_stride + (size_t)h * d;
+  if (p.k_dtype == PKV_INT8_SYM) {
+    store_sym(src, static_cast<int8_t*>(p.k_codes) + tile_idx * bs * d, p.k_scale + tile_idx, o0, lane);
+  } else {
+    store_fp16(src, static_cast<__half*>(p.k_codes) + tile_idx * bs * d, o0, lane);
+  }
+  // V side
+  src.base = p.v_new + (size_t)t * src.row_stride + (size_t)h * d;
+  if (p.v_dtype == PKV_INT8_SYM) {
+    store_sym(src, static_cast<int8_t*>(p.v_codes) + tile_idx * bs * d, p.v_scale + tile_idx, o0, lane);
+  } else if (p.v_dtype == PKV_INT4_ASYM) {
+    store_asym4(src, static_cast<uint8_t*>(p.v_codes) + tile_idx * bs * (d / 2), p.v_scale + tile_idx,
+                p.v_zp + tile_idx, o0, lane);
+  } else {
+    store_fp16(src, static_cast<__half*>(p.v_codes) + tile_idx * bs * d, o0, lane);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_store(const StoreParams& p, cudaStream_t stream) {
+  if (p.T == 0) return cudaSuccess;
+  dim3 grid(p.T, (p.num_kv_heads + kWarpsPerCta - 1) / kWarpsPerCta);
+  store_quantized_kernel<<<grid, 32 * kWarpsPerCta, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace pkv

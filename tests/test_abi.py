@@ -1,0 +1,110 @@
+"""The C-ABI library loads without a GPU, exports every function include/pkv.h declares, and
+rejects bad arguments on the host before any launch (no CUDA device needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def pkv():
+    from paged_block_quantized_b200 import build
+    build.build()
+    from paged_block_quantized_b200 import pkv as mod
+    return mod
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "pkv.h")).read()
+    return sorted(set(re.findall(r"PKV_API\s+[\w\s\*]+?\b(pkv_\w+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(pkv):
+    names = declared_functions()
+    assert len(names) >= 15
+    lib = ctypes.CDLL(pkv.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(pkv.EXPORTED) == names
+
+
+def desc(pkv, **kw):
+    d = dict(num_blocks=8, block_size=16, num_kv_heads=2, head_dim=64, k_dtype=pkv.PKV_INT8_SYM,
+             v_dtype=pkv.PKV_INT4_ASYM, k_codes=0x1000, v_codes=0x2000, k_scale=0x3000, v_scale=0x4000,
+             v_zp=0x5000)
+    d.update(kw)
+    return pkv.pkv_cache_desc(**d)
+
+
+def test_status_strings(pkv):
+    assert pkv.pkv_status_string(pkv.PKV_OK) == "PKV_OK"
+    assert pkv.pkv_status_string(pkv.PKV_ERR_UNSUPPORTED) == "PKV_ERR_UNSUPPORTED"
+    assert pkv.pkv_status_string(99) == "PKV_ERR_UNKNOWN"
+
+
+def test_tile_bytes(pkv):
+    d = desc(pkv)
+    assert pkv.pkv_tile_bytes(d, 0) == 16 * 64
+    assert pkv.pkv_tile_bytes(d, 1) == 16 * 32
+    assert pkv.pkv_tile_bytes(desc(pkv, k_dtype=pkv.PKV_FP16), 0) == 16 * 128
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(block_size=8), "PKV_ERR_UNSUPPORTED"),
+    (dict(head_dim=96), "PKV_ERR_UNSUPPORTED"),
+    (dict(head_dim=72), "PKV_ERR_INVALID_ARG"),
+    (dict(num_blocks=0), "PKV_ERR_INVALID_ARG"),
+    (dict(k_dtype=2), "PKV_ERR_INVALID_ARG"),      # INT4 is V-only
+    (dict(v_dtype=7), "PKV_ERR_INVALID_ARG"),
+    (dict(k_codes=0x1001), "PKV_ERR_INVALID_ARG"),  # misaligned
+    (dict(v_zp=0), "PKV_ERR_INVALID_ARG"),          # INT4 needs zero points
+    (dict(k_scale=0), "PKV_ERR_INVALID_ARG"),
+])
+def test_descriptor_validation(pkv, bad, code):
+    d = desc(pkv, **bad)
+    st = pkv.pkv_store_quantized(d, 0x6000, 0x7000, 0x8000, 4, stream=0, raise_on_error=False)
+    assert pkv.pkv_status_string(st) == code
+    st = pkv.pkv_copy_blocks(d, 0x6000, 1, stream=0, raise_on_error=False)
+    assert pkv.pkv_status_string(st) == code
+
+
+def test_call_validation(pkv):
+    d = desc(pkv)
+    E = pkv.PKV_ERR_INVALID_ARG
+    assert pkv.pkv_store_quantized(d, 0x6000, 0x7000, 0x8000, -1, stream=0, raise_on_error=False) == E
+    assert pkv.pkv_store_quantized(d, 0x6008, 0x7000, 0x8000, 1, stream=0, raise_on_error=False) == E
+    assert pkv.pkv_store_quantized(d, None, 0x7000, 0x8000, 1, stream=0, raise_on_error=False) == E
+    assert pkv.pkv_store_quantized(d, 0x6000, 0x7000, 0x8000, 0, stream=0, raise_on_error=False) == pkv.PKV_OK
+    assert pkv.pkv_copy_blocks(d, 0x6000, -2, stream=0, raise_on_error=False) == E
+    assert pkv.pkv_copy_blocks(d, 0x6000, 0, stream=0, raise_on_error=False) == pkv.PKV_OK
+    dec = lambda **kw: pkv.pkv_paged_attention_decode(
+        d, kw.get("out", 0x9000), kw.get("q", 0xA000), kw.get("S", 2), kw.get("Hq", 4), 0xB000,
+        kw.get("mbps", 4), 0xC000, kw.get("max_len", 64), kw.get("scale", 0.125), kw.get("pt", 0),
+        kw.get("ws", None), kw.get("ws_bytes", 0), stream=0, raise_on_error=False)
+    assert dec(Hq=3) == E                        # not a multiple of the KV heads
+    assert dec(q=0xA004) == E                    # misaligned
+    assert dec(mbps=0) == E
+    assert dec(pt=24) == E                       # not a multiple of the block size
+    assert dec(pt=16 * 128 + 16) == pkv.PKV_ERR_UNSUPPORTED
+    assert dec(scale=float("nan")) == E
+    assert dec(max_len=-1) == E
+    assert dec(S=0) == pkv.PKV_OK                # nothing to do
+    assert dec(max_len=4096, pt=64) == E         # needs a workspace
+    assert pkv.pkv_paged_attention_decode(desc(pkv, k_dtype=pkv.PKV_FP16), 0x9000, 0xA000, 2, 4, 0xB000, 4,
+                                          0xC000, 64, 0.1, stream=0, raise_on_error=False) == pkv.PKV_ERR_UNSUPPORTED
+
+
+def test_workspace_size(pkv):
+    d = desc(pkv)
+    # 256 bytes of arrival counters (one per sequence and CTA head group), then the partials
+    assert pkv.pkv_decode_workspace_size(d, 2, 4, 64, 64) == 0          # one partition: nothing
+    assert pkv.pkv_decode_workspace_size(d, 2, 4, 65, 64) == 256 + 2 * 4 * 2 * (64 + 2) * 4
+    assert pkv.pkv_decode_workspace_size(d, 3, 4, 1000, 128) == 256 + 3 * 4 * 8 * (64 + 2) * 4
+    # partials only: never proportional to the cache (no dequantized copy of K/V)
+    big = pkv.pkv_decode_workspace_size(d, 8, 32, 32768, 512)
+    assert big == 256 + 8 * 32 * 64 * 66 * 4
+    auto = pkv.pkv_decode_workspace_size(d, 8, 32, 32768, 0)
+    assert (auto - 256) % ((64 + 2) * 4 * 8 * 32) == 0

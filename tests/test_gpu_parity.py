@@ -1,0 +1,245 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle on the same seeded inputs.
+
+Bar: quantized codes, scales, zero points, slot scatter and copy-on-write bytes bit-exact (whole
+blocks, including never-written rows, starting from identically poisoned pools); attention output
+(fp16) within max-abs 2e-3 of the oracle's binary64 result computed on the oracle's own codes.
+Reduced sizes run the oracle over everything; full sizes (the benchmark's launch configuration)
+compare sampled sequences.
+"""
+import numpy as np
+import pytest
+import torch
+
+from paged_block_quantized_b200 import workloads as W
+from _oracle_run import oracle_step
+
+pytestmark = pytest.mark.gpu
+TOL = 2e-3
+
+
+def run_gpu(w, partition_tokens=None):
+    from paged_block_quantized_b200.step import DeviceStep
+    g = DeviceStep(w, partition_tokens=partition_tokens)
+    g.prefill()
+    pre = g.pool_numpy()
+    g.step()
+    torch.cuda.synchronize()
+    return g, pre
+
+
+def assert_pool_equal(gpu_arrays, cache, phys, what):
+    k, v, ks, vs, zp = gpu_arrays
+    phys = np.asarray(phys)
+    np.testing.assert_array_equal(k[phys], cache.k_codes, err_msg=f"{what}: K codes")
+    np.testing.assert_array_equal(v[phys], cache.v_codes, err_msg=f"{what}: V codes")
+    np.testing.assert_array_equal(ks[phys].view(np.uint32), cache.k_scale.view(np.uint32), err_msg=f"{what}: K scales")
+    np.testing.assert_array_equal(vs[phys].view(np.uint32), cache.v_scale.view(np.uint32), err_msg=f"{what}: V scales")
+    np.testing.assert_array_equal(zp[phys], cache.v_zp, err_msg=f"{what}: zero points")
+
+
+def check(w, seqs=None, partition_tokens=None):
+    g, pre = run_gpu(w, partition_tokens)
+    o = oracle_step(w, seqs)
+    assert all(e == 0 for e in o["errors"]), o["errors"]
+    assert g.error() == 0
+    assert_pool_equal(pre, o["prefill_cache"], o["phys"], "prefill store")
+    assert_pool_equal(g.pool_numpy(), o["cache"], o["phys"], "after copy + append")
+    out = g.out.float().cpu().numpy()[o["seqs"]]
+    err = np.abs(out - o["out"]).max()
+    assert err <= TOL, f"max abs error {err}"
+    return g, o
+
+
+REDUCED = {
+    "tiny": {},
+    "llama7b": dict(num_seqs=4),
+    "llama7b_fp16": dict(num_seqs=4),
+    "long": dict(num_seqs=2, context_lens=[8192 + 37, 9001]),
+    "gqa_prefix": dict(num_seqs=4, prefix_blocks=8, private_blocks=9),
+    "mixed": dict(num_seqs=24, children=4),
+}
+
+
+@pytest.mark.parametrize("name", list(REDUCED))
+def test_config_reduced_sizes(name):
+    check(W.make(name, seed=0, **REDUCED[name]))
+
+
+FULL_SAMPLES = {
+    "llama7b": [0, 7, 31],
+    "llama7b_fp16": [3, 30],
+    "long": [int(np.argmin(W.make("long").context_lens))],
+    "gqa_prefix": [0, 33, 63],
+    "mixed": None,  # a parent, its child and two others, chosen below
+}
+
+
+@pytest.mark.parametrize("name", list(FULL_SAMPLES))
+def test_config_full_size_sampled(name):
+    w = W.make(name, seed=0)
+    seqs = FULL_SAMPLES[name]
+    if seqs is None:
+        src, dst = (int(x) for x in w.cow_pairs[0])
+        child = int(np.nonzero((w.block_tables == dst).any(axis=1))[0][0])
+        parent = int(np.nonzero((w.block_tables == src).any(axis=1))[0][0])
+        seqs = [parent, child, 1, int(np.argmax(w.context_lens))]
+    check(w, seqs)
+
+
+def test_split_matches_unsplit():
+    w = W.make("llama7b", seed=1, num_seqs=3)
+    g_small, o = check(w, partition_tokens=64)
+    g_big, _ = check(w, partition_tokens=2048)
+    a = g_small.out.float().cpu().numpy()
+    b = g_big.out.float().cpu().numpy()
+    assert np.abs(a - b).max() <= 1e-3
+
+
+@pytest.mark.parametrize("case", [
+    dict(head_dim=64, block_size=32, num_q_heads=4, num_kv_heads=4),
+    dict(head_dim=256, block_size=16, num_q_heads=2, num_kv_heads=2),
+    dict(head_dim=128, block_size=32, num_q_heads=8, num_kv_heads=4),
+    dict(head_dim=128, block_size=16, num_q_heads=16, num_kv_heads=2),
+    dict(head_dim=64, block_size=16, num_q_heads=12, num_kv_heads=4, v_dtype=W.INT4_ASYM),
+    dict(head_dim=256, block_size=32, num_q_heads=4, num_kv_heads=1, v_dtype=W.INT4_ASYM),
+    dict(head_dim=64, block_size=16, num_q_heads=4, num_kv_heads=2, k_dtype=W.FP16, v_dtype=W.FP16),
+])
+def test_shapes_and_groups(case):
+    lens = [1, 2, 16, 17, 31, 32, 33, 100, 700]
+    w = W.make("tiny", seed=2, num_seqs=len(lens), context_lens=lens, num_blocks=128, **case)
+    check(w)
+
+
+@pytest.mark.parametrize("pt", [64, 128, 512])
+def test_partition_boundaries(pt):
+    lens = [pt - 1, pt, pt + 1, 2 * pt, 2 * pt + 1, 5 * pt - 3]
+    w = W.make("llama7b", seed=3, num_seqs=len(lens), context_lens=lens)
+    check(w, partition_tokens=pt)
+
+
+def test_max_partition_and_long_sequence():
+    from paged_block_quantized_b200 import pkv
+    w = W.make("long", seed=4, num_seqs=1, context_lens=[32768])
+    g, _ = check(w, partition_tokens=32 * 4 * 32)  # the largest partition for block size 32
+    assert g.partition_tokens == 4096
+    with pytest.raises(pkv.PkvError):
+        pkv.pkv_decode_workspace_size(g.pool.desc, 1, 32, 32768, 4096 + 32)
+
+
+def test_zero_length_and_empty_batch():
+    from paged_block_quantized_b200 import pkv
+    import oracle
+    w = W.make("tiny", seed=5)
+    g, o = check(w)
+    lens = w.context_lens.copy()
+    lens[1] = 0
+    lens[3] = 1
+    g.context_lens.copy_(torch.from_numpy(lens))
+    g.decode()
+    torch.cuda.synchronize()
+    ref, err = oracle.decode(o["cache"], o["q"], o["tables"], lens, w.softmax_scale, max_context_len=w.max_context_len)
+    assert err == 0 and g.error() == 0
+    out = g.out.float().cpu().numpy()
+    assert not out[1].any()
+    assert np.abs(out - ref).max() <= TOL
+    # no sequences / no tokens: accepted, nothing launched
+    assert pkv.pkv_paged_attention_decode(g.pool.desc, g.out, g.q, 0, w.num_q_heads, g.block_tables,
+                                          w.max_blocks_per_seq, g.context_lens, 0, 0.1) == pkv.PKV_OK
+    assert pkv.pkv_store_quantized(g.pool.desc, g.k_new, g.v_new, g.step_slots, 0) == pkv.PKV_OK
+
+
+def test_bad_block_id_is_skipped_and_flagged():
+    import oracle
+    w = W.make("tiny", seed=6)
+    g, o = check(w)
+    tables = o["tables"].copy()
+    bad_gpu = g.block_tables.clone()
+    bad_gpu[2, 1] = w.num_blocks + 5
+    tables[2, 1] = len(o["phys"]) + 5
+    from paged_block_quantized_b200 import pkv
+    pkv.pkv_paged_attention_decode(g.pool.desc, g.out, g.q, w.num_seqs, w.num_q_heads, bad_gpu,
+                                   w.max_blocks_per_seq, g.context_lens, w.max_context_len, w.softmax_scale,
+                                   g.partition_tokens, g.workspace, g.ws_bytes, g.dev_error)
+    torch.cuda.synchronize()
+    assert g.error() == pkv.PKV_DEVERR_BLOCK_ID
+    ref, err = oracle.decode(o["cache"], o["q"], tables, w.context_lens, w.softmax_scale)
+    assert err == oracle.DEVERR_BLOCK_ID
+    assert np.abs(g.out.float().cpu().numpy() - ref).max() <= TOL
+
+
+def test_context_longer_than_table_is_flagged():
+    from paged_block_quantized_b200 import pkv
+    w = W.make("tiny", seed=7)
+    g, _ = check(w)
+    lens = g.context_lens.clone()
+    lens[0] = w.max_blocks_per_seq * w.block_size + 1
+    g.dev_error.zero_()
+    pkv.pkv_paged_attention_decode(g.pool.desc, g.out, g.q, w.num_seqs, w.num_q_heads, g.block_tables,
+                                   w.max_blocks_per_seq, lens, int(lens.max()), w.softmax_scale,
+                                   g.partition_tokens, g.workspace, g.ws_bytes, g.dev_error)
+    torch.cuda.synchronize()
+    assert g.error() == pkv.PKV_DEVERR_CONTEXT_LEN
+
+
+def test_store_slot_errors_are_flagged():
+    from paged_block_quantized_b200 import pkv
+    w = W.make("tiny", seed=8)
+    g, _ = check(w)
+    for slots, code in (([w.num_blocks * w.block_size, -1, -1, -1], pkv.PKV_DEVERR_SLOT),
+                        ([5, 7, -1, -1], pkv.PKV_DEVERR_SLOT_GROUP)):
+        g.dev_error.zero_()
+        st = torch.tensor(slots, dtype=torch.int64, device="cuda")
+        pkv.pkv_store_quantized(g.pool.desc, g.k_new, g.v_new, st, 4, g.dev_error)
+        torch.cuda.synchronize()
+        assert g.error() == code
+
+
+def test_append_rebuild_bit_exact():
+    """Tokens far outside a tile's stored range force the rebuild path; bytes match the oracle."""
+    import oracle
+    from paged_block_quantized_b200 import pkv
+    rng = np.random.default_rng(9)
+    nb, bs, H, D = 8, 16, 4, 128
+    for v_dtype in (W.INT8_SYM, W.INT4_ASYM):
+        pool = pkv.DevicePool.allocate(nb, bs, H, D, W.INT8_SYM, v_dtype, fill=0xA5)
+        c = oracle.OracleCache.empty(nb, bs, H, D, oracle.INT8_SYM, {1: oracle.INT8_SYM, 2: oracle.INT4_ASYM}[v_dtype])
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        # 5 tokens; appends of 1 that does not fit, 3 that fit, 2 that do not, 4 that do not
+        plan = [(0, 5, 1.0), (5, 1, 50.0), (6, 3, 0.01), (9, 2, 30.0), (11, 4, 400.0)]
+        for start, n, scale in plan:
+            k = (rng.standard_normal((n, H, D)) * scale).astype(np.float16)
+            v = (rng.standard_normal((n, H, D)) * scale - scale / 3).astype(np.float16)
+            slots = 3 * bs + start + np.arange(n, dtype=np.int64)
+            oracle.store(c, k, v, slots)
+            pkv.pkv_store_quantized(pool.desc, torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda(),
+                                    torch.from_numpy(slots).cuda(), n, err)
+        torch.cuda.synchronize()
+        assert err.item() == 0
+        np.testing.assert_array_equal(pool.k_codes.cpu().numpy().view(np.int8), c.k_codes)
+        np.testing.assert_array_equal(pool.v_codes.cpu().numpy().view(c.v_codes.dtype), c.v_codes)
+        np.testing.assert_array_equal(pool.k_scale.cpu().numpy().view(np.uint32), c.k_scale.view(np.uint32))
+        np.testing.assert_array_equal(pool.v_scale.cpu().numpy().view(np.uint32), c.v_scale.view(np.uint32))
+        np.testing.assert_array_equal(pool.v_zp.cpu().numpy(), c.v_zp)
+
+
+def test_copy_blocks_bit_exact_and_bad_ids():
+    import oracle
+    from paged_block_quantized_b200 import pkv
+    w = W.make("mixed", seed=10, num_seqs=12, children=2)
+    g, o = check(w)
+    before = g.pool_numpy()
+    pairs = np.array([[1, 40], [7, 41], [w.num_blocks - 1, 0]], np.int32)
+    gp = torch.from_numpy(pairs).cuda()
+    pkv.pkv_copy_blocks(g.pool.desc, gp, 3, g.dev_error)
+    torch.cuda.synchronize()
+    after = g.pool_numpy()
+    for a, b in zip(before, after):
+        exp = a.copy()
+        exp[pairs[:, 1]] = a[pairs[:, 0]]
+        np.testing.assert_array_equal(b.view(np.uint8), exp.view(np.uint8))
+    g.dev_error.zero_()
+    pkv.pkv_copy_blocks(g.pool.desc, torch.tensor([[0, w.num_blocks]], dtype=torch.int32, device="cuda"), 1,
+                        g.dev_error)
+    torch.cuda.synchronize()
+    assert g.error() == pkv.PKV_DEVERR_BLOCK_ID
+    np.testing.assert_array_equal(g.pool_numpy()[0], after[0])

@@ -1,0 +1,78 @@
+"""Structure of the seeded synthetic workloads (shapes, block assignment, sharing, slots)."""
+import numpy as np
+import pytest
+
+from paged_block_quantized_b200 import workloads as W
+
+
+@pytest.mark.parametrize("name", W.CONFIGS + ("llama7b_fp16",))
+def test_layout_is_consistent(name):
+    w = W.make(name)
+    bs = w.block_size
+    assert w.context_lens.min() >= 1
+    used = []
+    for s in range(w.num_seqs):
+        nblk = (int(w.context_lens[s]) + bs - 1) // bs
+        row = w.block_tables[s, :nblk]
+        assert (row >= 0).all() and (row < w.num_blocks).all()
+        assert (w.block_tables[s, nblk:] == -1).all()
+        used.extend(row.tolist())
+    # a physical block is shared only where the workload says so (prefix or fork)
+    counts = np.bincount(used, minlength=w.num_blocks)
+    if name == "gqa_prefix":
+        assert (counts == w.num_seqs).sum() == 64 and counts.max() == 64
+    elif name == "mixed":
+        assert w.cow_pairs.shape == (16, 2)
+        assert len(set(w.cow_pairs[:, 1])) == 16
+        assert counts.max() == 2
+    else:
+        assert counts.max() == 1
+    # the step's slots land in each sequence's last block at offset (L-1) % bs
+    slots = w.step_slots()
+    for s in range(w.num_seqs):
+        p = int(w.context_lens[s]) - 1
+        assert slots[s] == w.block_tables[s, p // bs] * bs + p % bs
+
+
+def test_named_sizes():
+    assert list(W.make("tiny").context_lens) == [17, 33, 50, 64]
+    w = W.make("llama7b")
+    assert w.num_seqs == 32 and w.num_blocks == 8192 and 500 <= w.context_lens.min() and w.context_lens.max() <= 2000
+    w = W.make("long")
+    assert w.num_seqs == 8 and 8192 <= w.context_lens.min() and w.context_lens.max() <= 32768 and w.block_size == 32
+    w = W.make("gqa_prefix")
+    assert (w.num_q_heads, w.num_kv_heads, int(w.context_lens[0])) == (64, 8, 2048)
+    w = W.make("mixed")
+    assert w.num_seqs == 128 and 16 <= w.context_lens.min() and w.context_lens.max() <= 16384
+    for src, dst in w.cow_pairs:
+        parent = np.nonzero((w.block_tables == src).any(axis=1))[0]
+        assert len(parent) == 1
+        assert (w.context_lens[parent[0]] - 1) % 16 != 0  # the shared last block is partial
+
+
+def test_values_are_deterministic_and_fp16():
+    w = W.make("llama7b", seed=3, num_seqs=2)
+    a = w.block_values(1, 5)
+    b = W.make("llama7b", seed=3, num_seqs=2).block_values(1, 5)
+    assert a[0].dtype == np.float16
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
+    # outlier channels: about 1% of channels scaled by 8
+    k = np.concatenate([w.block_values(0, j)[0] for j in range(40)]).astype(np.float32)
+    ch_std = k.reshape(-1, w.num_kv_heads * w.head_dim).std(axis=0)
+    assert (ch_std > 4).sum() == round(0.01 * w.num_kv_heads * w.head_dim)
+
+
+def test_prefill_covers_positions_once():
+    w = W.make("mixed", num_seqs=20, children=3)
+    seen = set()
+    for k, v, slots in w.prefill_batches(max_tokens=100):
+        assert k.shape == v.shape and k.shape[0] == slots.shape[0]
+        for sl in slots.tolist():
+            assert sl not in seen
+            seen.add(sl)
+    expected = set()
+    for s in range(w.num_seqs):
+        for p in range(int(w.context_lens[s]) - 1):
+            expected.add(int(w.prefill_tables[s, p // w.block_size]) * w.block_size + p % w.block_size)
+    assert seen == expected
