@@ -154,6 +154,16 @@ PKV_API pkv_status pkv_decode_workspace_size(const pkv_cache_desc* desc, int32_t
                                      int32_t partition_tokens, size_t* bytes);
 
 /*
+ * pkv_decode_partitioning -- the split the decode call will use for these sizes: tokens per
+ * partition (the given value, or the automatic choice when partition_tokens is 0) and the
+ * number of partitions of the longest sequence. Either output pointer may be NULL.
+ */
+PKV_API pkv_status pkv_decode_partitioning(const pkv_cache_desc* desc, int32_t num_seqs,
+                                           int32_t num_q_heads, int32_t max_context_len,
+                                           int32_t partition_tokens, int32_t* partition_tokens_out,
+                                           int32_t* num_partitions_out);
+
+/*
  * pkv_paged_attention_decode -- one decode step of attention over the paged, quantized cache.
  *
  * For every sequence s and query head h (KV head g = h / (num_q_heads / num_kv_heads)):

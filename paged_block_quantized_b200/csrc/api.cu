@@ -172,6 +172,19 @@ pkv_status pkv_decode_workspace_size(const pkv_cache_desc* desc, int32_t num_seq
   return PKV_OK;
 }
 
+pkv_status pkv_decode_partitioning(const pkv_cache_desc* desc, int32_t num_seqs, int32_t num_q_heads,
+                                   int32_t max_context_len, int32_t partition_tokens, int32_t* partition_tokens_out,
+                                   int32_t* num_partitions_out) {
+  pkv_status st = check_desc(desc);
+  if (st != PKV_OK) return st;
+  DecodeGeometry g;
+  st = decode_geometry(desc, num_seqs, num_q_heads, max_context_len, partition_tokens, &g);
+  if (st != PKV_OK) return st;
+  if (partition_tokens_out) *partition_tokens_out = g.partition_tokens;
+  if (num_partitions_out) *num_partitions_out = g.max_partitions;
+  return PKV_OK;
+}
+
 pkv_status pkv_paged_attention_decode(const pkv_cache_desc* desc, void* out, const void* q, int32_t num_seqs,
                                       int32_t num_q_heads, const int32_t* block_tables, int32_t max_blocks_per_seq,
                                       const int32_t* context_lens, int32_t max_context_len, float softmax_scale,

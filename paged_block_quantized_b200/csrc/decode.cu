@@ -117,42 +117,27 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS)
   const int tg = lane / C::CH;  // token-row group of this lane
   const int PT = p.partition_tokens;
 
-  // ---- context length (validated; clamped on error) ----
+  // ---- pipeline set-up: this warp's NS stages and barriers (no memory dependence) ----
+  uint8_t* my_stages = stages + (size_t)warp * C::NS * C::STAGE;
+  uint64_t* my_bars = bars + warp * C::NS;
+  if (lane == 0) {
+#pragma unroll
+    for (int st = 0; st < C::NS; ++st) mbar_init(&my_bars[st], 1);
+    fence_mbar_init();
+  }
+
+  // ---- first round of global loads, all independent of one another ----
+  // The partition's first block index does not depend on the context length, so this warp's
+  // block-table entries are read speculatively (in bounds of the table row) together with the
+  // length; entries past the sequence's end are never used.
+  const int blk_begin = (part * PT) / BS;
+  const int j_lane = blk_begin + warp + C::NW * lane;
+  int b_raw = -1;
+  if (lane * C::NW * BS < PT && j_lane < p.max_blocks_per_seq)
+    b_raw = p.block_tables[(size_t)s * p.max_blocks_per_seq + j_lane];
   int L = p.context_lens[s];
-  {
-    const int cap = min(p.max_context_len, p.max_blocks_per_seq * BS);
-    if (L < 0 || L > cap) {
-      if (part == 0 && blockIdx.x == 0 && threadIdx.x == 0) record_error(p.dev_error, PKV_DEVERR_CONTEXT_LEN);
-      L = max(0, min(L, cap));
-    }
-  }
-  const int num_parts = (L + PT - 1) / PT;
-  if (part >= (num_parts > 0 ? num_parts : 1)) return;  // beyond this sequence's partitions
 
-  const int t_begin = part * PT;
-  const int t_end = min(L, t_begin + PT);
-  const int blk_begin = t_begin / BS;
-  const int n_blk = t_end > t_begin ? (t_end - t_begin + BS - 1) / BS : 0;
-  // this warp's blocks: blk_begin + warp + NW * k, k < my_blocks (<= 32 by the partition cap)
-  const int my_blocks = n_blk > warp ? (n_blk - warp + C::NW - 1) / C::NW : 0;
-
-  // ---- per-lane prefetch of block ids and per-block metadata for this warp's blocks ----
-  int my_b = 0;          // physical block to copy (0 stands in for an invalid id)
-  bool my_valid = false;
-  float my_ks = 0.f, my_vs = 0.f, my_zp = 0.f;
-  if (lane < my_blocks) {
-    const int j = blk_begin + warp + C::NW * lane;
-    const int b = p.block_tables[(size_t)s * p.max_blocks_per_seq + j];
-    my_valid = (b >= 0 && b < p.num_blocks);
-    if (!my_valid) record_error(p.dev_error, PKV_DEVERR_BLOCK_ID);
-    my_b = my_valid ? b : 0;
-    const size_t meta = (size_t)my_b * p.num_kv_heads + g;
-    if constexpr (KT != PKV_FP16) my_ks = p.k_scale[meta];
-    if constexpr (VT != PKV_FP16) my_vs = p.v_scale[meta];
-    if constexpr (VT == PKV_INT4_ASYM) my_zp = (float)p.v_zp[meta];
-  }
-
-  // ---- query heads of the CTA, this lane's 16 dims, fp32 ----
+  // query heads of the CTA, this lane's 16 dims, fp32
   float qf[GT][16];
 #pragma unroll
   for (int hh = 0; hh < GT; ++hh) {
@@ -168,18 +153,30 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS)
     }
   }
 
-  // ---- pipeline set-up: this warp's NS stages and barriers ----
-  uint8_t* my_stages = stages + (size_t)warp * C::NS * C::STAGE;
-  uint64_t* my_bars = bars + warp * C::NS;
-  if (lane == 0) {
-#pragma unroll
-    for (int st = 0; st < C::NS; ++st) mbar_init(&my_bars[st], 1);
-    fence_mbar_init();
+  // ---- context length (validated; clamped on error) and this warp's share of the partition ----
+  {
+    const int cap = min(p.max_context_len, p.max_blocks_per_seq * BS);
+    if (L < 0 || L > cap) {
+      if (part == 0 && blockIdx.x == 0 && threadIdx.x == 0) record_error(p.dev_error, PKV_DEVERR_CONTEXT_LEN);
+      L = max(0, min(L, cap));
+    }
   }
-  __syncwarp();
+  const int num_parts = (L + PT - 1) / PT;
+  if (part >= (num_parts > 0 ? num_parts : 1)) return;  // beyond this sequence's partitions (CTA-uniform)
+
+  const int t_begin = part * PT;
+  const int t_end = min(L, t_begin + PT);
+  const int n_blk = t_end > t_begin ? (t_end - t_begin + BS - 1) / BS : 0;
+  // this warp's blocks: blk_begin + warp + NW * k, k < my_blocks (<= 32 by the partition cap)
+  const int my_blocks = n_blk > warp ? (n_blk - warp + C::NW - 1) / C::NW : 0;
+
+  const bool my_valid = lane < my_blocks && b_raw >= 0 && b_raw < p.num_blocks;
+  if (lane < my_blocks && !my_valid) record_error(p.dev_error, PKV_DEVERR_BLOCK_ID);
+  const int my_b = my_valid ? b_raw : 0;  // block 0 stands in for an invalid id (its tokens are masked)
+  __syncwarp();  // barrier initialisation by lane 0 is visible to the warp
 
   const size_t head_tile = (size_t)p.num_kv_heads;
-  auto issue = [&](int k, int st, int b) {
+  auto issue = [&](int st, int b) {
     const size_t tile = (size_t)b * head_tile + g;
     uint8_t* dst = my_stages + (size_t)st * C::STAGE;
     mbar_arrive_expect_tx(&my_bars[st], (uint32_t)C::STAGE);
@@ -188,13 +185,20 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS)
              &my_bars[st]);
   };
 
-  // prologue
-  {
+  // ---- fill the ring: the first NS tiles of this warp are in flight from here on ----
 #pragma unroll
-    for (int k = 0; k < C::NS; ++k) {
-      const int b = __shfl_sync(kFull, my_b, k);
-      if (lane == 0 && k < my_blocks) issue(k, k, b);
-    }
+  for (int k = 0; k < C::NS; ++k) {
+    const int b = __shfl_sync(kFull, my_b, k);
+    if (lane == 0 && k < my_blocks) issue(k, b);
+  }
+
+  // ---- per-block scales / zero points: their latency overlaps the copies in flight ----
+  float my_ks = 0.f, my_vs = 0.f, my_zp = 0.f;
+  if (lane < my_blocks) {
+    const size_t meta = (size_t)my_b * p.num_kv_heads + g;
+    if constexpr (KT != PKV_FP16) my_ks = p.k_scale[meta];
+    if constexpr (VT != PKV_FP16) my_vs = p.v_scale[meta];
+    if constexpr (VT == PKV_INT4_ASYM) my_zp = (float)p.v_zp[meta];
   }
 
   float m_run[GT], l_run[GT], acc[GT][16];
@@ -299,7 +303,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS)
     const int bn = __shfl_sync(kFull, my_b, kn & 31);
     if (lane == 0 && kn < my_blocks) {
       fence_proxy_async_smem();
-      issue(kn, st, bn);
+      issue(st, bn);
     }
   }
 

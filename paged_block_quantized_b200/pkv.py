@@ -28,6 +28,7 @@ PKV_FP16, PKV_INT8_SYM, PKV_INT4_ASYM = 0, 1, 2
 
 EXPORTED = (
     "pkv_status_string", "pkv_tile_bytes", "pkv_store_quantized", "pkv_decode_workspace_size",
+    "pkv_decode_partitioning",
     "pkv_paged_attention_decode", "pkv_copy_blocks", "pkv_blocks_for_tokens", "pkv_alloc_create",
     "pkv_alloc_destroy", "pkv_alloc_num_free", "pkv_alloc_refcount", "pkv_alloc_blocks", "pkv_alloc_fork",
     "pkv_alloc_release", "pkv_alloc_cow",
@@ -67,6 +68,8 @@ _tile_bytes = _sig("pkv_tile_bytes", ctypes.c_size_t, _DESC, _I32)
 _store = _sig("pkv_store_quantized", ctypes.c_int, _DESC, _P, _P, _P, _I32, _P, _P)
 _ws_size = _sig("pkv_decode_workspace_size", ctypes.c_int, _DESC, _I32, _I32, _I32, _I32,
                 ctypes.POINTER(ctypes.c_size_t))
+_partitioning = _sig("pkv_decode_partitioning", ctypes.c_int, _DESC, _I32, _I32, _I32, _I32,
+                     ctypes.POINTER(_I32), ctypes.POINTER(_I32))
 _decode = _sig("pkv_paged_attention_decode", ctypes.c_int, _DESC, _P, _P, _I32, _I32, _P, _I32, _P, _I32,
                ctypes.c_float, _I32, _P, ctypes.c_size_t, _P, _P)
 _copy = _sig("pkv_copy_blocks", ctypes.c_int, _DESC, _P, _I32, _P, _P)
@@ -135,6 +138,15 @@ def pkv_decode_workspace_size(desc, num_seqs, num_q_heads, max_context_len, part
                   int(partition_tokens), ctypes.byref(out))
     _check(st, "pkv_decode_workspace_size", True)
     return int(out.value)
+
+
+def pkv_decode_partitioning(desc, num_seqs, num_q_heads, max_context_len, partition_tokens=0):
+    """(tokens per partition, partitions of the longest sequence) the decode will use."""
+    pt, n = _I32(0), _I32(0)
+    st = _partitioning(ctypes.byref(desc), int(num_seqs), int(num_q_heads), int(max_context_len),
+                       int(partition_tokens), ctypes.byref(pt), ctypes.byref(n))
+    _check(st, "pkv_decode_partitioning", True)
+    return int(pt.value), int(n.value)
 
 
 def pkv_paged_attention_decode(desc, out, q, num_seqs, num_q_heads, block_tables, max_blocks_per_seq,

@@ -24,7 +24,7 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported(pkv):
     names = declared_functions()
-    assert len(names) >= 15
+    assert len(names) >= 16
     lib = ctypes.CDLL(pkv.LIB_PATH)
     for n in names:
         assert hasattr(lib, n), n
@@ -95,6 +95,14 @@ def test_call_validation(pkv):
     assert dec(max_len=4096, pt=64) == E         # needs a workspace
     assert pkv.pkv_paged_attention_decode(desc(pkv, k_dtype=pkv.PKV_FP16), 0x9000, 0xA000, 2, 4, 0xB000, 4,
                                           0xC000, 64, 0.1, stream=0, raise_on_error=False) == pkv.PKV_ERR_UNSUPPORTED
+
+
+def test_partitioning(pkv):
+    d = desc(pkv)
+    assert pkv.pkv_decode_partitioning(d, 2, 4, 1000, 128) == (128, 8)
+    assert pkv.pkv_decode_partitioning(d, 2, 4, 0, 64) == (64, 1)
+    pt, n = pkv.pkv_decode_partitioning(d, 2, 4, 5000, 0)
+    assert pt % 16 == 0 and 64 <= pt <= 2048 and n == -(-5000 // pt)
 
 
 def test_workspace_size(pkv):

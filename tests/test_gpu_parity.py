@@ -174,11 +174,21 @@ def test_context_longer_than_table_is_flagged():
     lens = g.context_lens.clone()
     lens[0] = w.max_blocks_per_seq * w.block_size + 1
     g.dev_error.zero_()
+    # longer than both the table and max_context_len (which sizes the grid and workspace)
     pkv.pkv_paged_attention_decode(g.pool.desc, g.out, g.q, w.num_seqs, w.num_q_heads, g.block_tables,
-                                   w.max_blocks_per_seq, lens, int(lens.max()), w.softmax_scale,
+                                   w.max_blocks_per_seq, lens, w.max_context_len, w.softmax_scale,
                                    g.partition_tokens, g.workspace, g.ws_bytes, g.dev_error)
     torch.cuda.synchronize()
     assert g.error() == pkv.PKV_DEVERR_CONTEXT_LEN
+    # negative lengths are flagged too and treated as empty
+    lens[0] = -3
+    g.dev_error.zero_()
+    pkv.pkv_paged_attention_decode(g.pool.desc, g.out, g.q, w.num_seqs, w.num_q_heads, g.block_tables,
+                                   w.max_blocks_per_seq, lens, w.max_context_len, w.softmax_scale,
+                                   g.partition_tokens, g.workspace, g.ws_bytes, g.dev_error)
+    torch.cuda.synchronize()
+    assert g.error() == pkv.PKV_DEVERR_CONTEXT_LEN
+    assert not g.out[0].float().abs().sum().item()
 
 
 def test_store_slot_errors_are_flagged():
