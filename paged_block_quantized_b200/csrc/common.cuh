@@ -40,6 +40,24 @@ __device__ __forceinline__ void s8x4_to_f32(uint32_t w, float& f0, float& f1, fl
   f3 = byte_to_magic(u, 3) - bias;
 }
 
+// Packed forms for the sm_100 paired fp32 pipe (__fadd2_rn / __ffma2_rn): one FADD2 removes the
+// bias from two codes. `neg_bias` = -(2^23 + bias) in both lanes.
+__device__ __forceinline__ void s8x4_to_f32x2(uint32_t w, float2& lo, float2& hi) {
+  const uint32_t u = w ^ 0x80808080u;  // c + 128 in 0..255
+  const float2 neg_bias = make_float2(-(kMagic + 128.0f), -(kMagic + 128.0f));
+  lo = __fadd2_rn(make_float2(byte_to_magic(u, 0), byte_to_magic(u, 1)), neg_bias);
+  hi = __fadd2_rn(make_float2(byte_to_magic(u, 2), byte_to_magic(u, 3)), neg_bias);
+}
+
+// 8 unsigned 4-bit codes (nibble k = dim k) -> 4 float2 of (code - zp), dims in order.
+__device__ __forceinline__ void u4x8_to_f32x2(uint32_t w, float2 neg_bias, float2 f[4]) {
+  const uint32_t even = w & 0x0F0F0F0Fu;        // nibbles 0,2,4,6 in bytes 0..3
+  const uint32_t odd = (w >> 4) & 0x0F0F0F0Fu;  // nibbles 1,3,5,7
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    f[i] = __fadd2_rn(make_float2(byte_to_magic(even, i), byte_to_magic(odd, i)), neg_bias);
+}
+
 // 8 unsigned 4-bit codes packed in w (nibble k = dim k, low nibble first) -> (code - zp) exact.
 // bias = 2^23 + zp.
 __device__ __forceinline__ void u4x8_to_f32(uint32_t w, float bias, float f[8]) {
@@ -72,10 +90,6 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
 
 __device__ __forceinline__ void fence_mbar_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {

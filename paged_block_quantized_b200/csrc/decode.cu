@@ -61,37 +61,34 @@ struct Cfg {
   static_assert(K_TILE % 16 == 0 && V_TILE % 16 == 0 && STAGE % 16 == 0, "bulk copy granularity");
 };
 
-// 16 consecutive K values of one token row (lane chunk) -> fp32
+// 16 consecutive K values of one token row (lane chunk) -> 8 float2 (dims in order)
 template <int KT>
-__device__ __forceinline__ void load_k16(const uint8_t* p, float f[16]) {
+__device__ __forceinline__ void load_k16(const uint8_t* p, float2 f[8]) {
   if constexpr (KT == PKV_INT8_SYM) {
     const uint4 w = *reinterpret_cast<const uint4*>(p);
-    s8x4_to_f32(w.x, f[0], f[1], f[2], f[3]);
-    s8x4_to_f32(w.y, f[4], f[5], f[6], f[7]);
-    s8x4_to_f32(w.z, f[8], f[9], f[10], f[11]);
-    s8x4_to_f32(w.w, f[12], f[13], f[14], f[15]);
+    s8x4_to_f32x2(w.x, f[0], f[1]);
+    s8x4_to_f32x2(w.y, f[2], f[3]);
+    s8x4_to_f32x2(w.z, f[4], f[5]);
+    s8x4_to_f32x2(w.w, f[6], f[7]);
   } else {
     const uint4 w0 = *reinterpret_cast<const uint4*>(p);
     const uint4 w1 = *reinterpret_cast<const uint4*>(p + 16);
     const uint32_t u[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&u[i]));
-      f[2 * i] = v.x;
-      f[2 * i + 1] = v.y;
-    }
+    for (int i = 0; i < 8; ++i) f[i] = __half22float2(*reinterpret_cast<const __half2*>(&u[i]));
   }
 }
 
-// 16 consecutive V values of one token row (lane chunk) -> fp32 (code - zp); bias = 2^23 + zp
+// 16 consecutive V values of one token row (lane chunk) -> 8 float2 of (code - zp);
+// neg_bias = -(2^23 + zp) in both lanes (INT4 only)
 template <int VT>
-__device__ __forceinline__ void load_v16(const uint8_t* p, float bias, float f[16]) {
+__device__ __forceinline__ void load_v16(const uint8_t* p, float2 neg_bias, float2 f[8]) {
   if constexpr (VT == PKV_INT8_SYM) {
     load_k16<PKV_INT8_SYM>(p, f);
   } else if constexpr (VT == PKV_INT4_ASYM) {
     const uint2 w = *reinterpret_cast<const uint2*>(p);
-    u4x8_to_f32(w.x, bias, f);
-    u4x8_to_f32(w.y, bias, f + 8);
+    u4x8_to_f32x2(w.x, neg_bias, f);
+    u4x8_to_f32x2(w.y, neg_bias, f + 4);
   } else {
     load_k16<PKV_FP16>(p, f);
   }
@@ -138,7 +135,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS)
   int L = p.context_lens[s];
 
   // query heads of the CTA, this lane's 16 dims, fp32
-  float qf[GT][16];
+  float2 qf[GT][8];
 #pragma unroll
   for (int hh = 0; hh < GT; ++hh) {
     const __half* qp = p.q + ((size_t)s * p.num_q_heads + h0 + hh) * D + c * 16;
@@ -146,11 +143,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS)
     const uint4 w1 = *reinterpret_cast<const uint4*>(qp + 8);
     const uint32_t u[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&u[i]));
-      qf[hh][2 * i] = v.x;
-      qf[hh][2 * i + 1] = v.y;
-    }
+    for (int i = 0; i < 8; ++i) qf[hh][i] = __half22float2(*reinterpret_cast<const __half2*>(&u[i]));
   }
 
   // ---- context length (validated; clamped on error) and this warp's share of the partition ----
@@ -201,13 +194,14 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS)
     if constexpr (VT == PKV_INT4_ASYM) my_zp = (float)p.v_zp[meta];
   }
 
-  float m_run[GT], l_run[GT], acc[GT][16];
+  float m_run[GT], l_run[GT];
+  float2 acc[GT][8];  // this lane's 16 dims, as pairs
 #pragma unroll
   for (int hh = 0; hh < GT; ++hh) {
     m_run[hh] = kNegBig;
     l_run[hh] = 0.f;
 #pragma unroll
-    for (int j = 0; j < 16; ++j) acc[hh][j] = 0.f;
+    for (int j = 0; j < 8; ++j) acc[hh][j] = make_float2(0.f, 0.f);
   }
 
   bool aborted = false;
@@ -224,7 +218,8 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS)
     }
     const float ks = __shfl_sync(kFull, my_ks, k) * p.scale_log2;
     const float vs = __shfl_sync(kFull, my_vs, k);
-    const float zp_bias = kMagic + __shfl_sync(kFull, my_zp, k);
+    const float nzb = -(kMagic + __shfl_sync(kFull, my_zp, k));
+    const float2 neg_zp_bias = make_float2(nzb, nzb);
     const bool valid = __shfl_sync(kFull, my_valid ? 1 : 0, k) != 0;
     const int tok0 = (blk_begin + warp + C::NW * k) * BS;
     const uint8_t* kt = my_stages + (size_t)st * C::STAGE;
@@ -235,17 +230,17 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS)
 #pragma unroll
     for (int i = 0; i < C::TPL; ++i) {
       const int row = tg + C::TG * i;
-      float kf[16];
+      float2 kf[8];
       load_k16<KT>(kt + row * C::K_ROW + c * (C::K_ROW / C::CH), kf);
 #pragma unroll
       for (int hh = 0; hh < GT; ++hh) {
-        float a0 = 0.f, a1 = 0.f;
+        float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int j = 0; j < 16; j += 2) {
-          a0 = fmaf(qf[hh][j], kf[j], a0);
-          a1 = fmaf(qf[hh][j + 1], kf[j + 1], a1);
+        for (int j = 0; j < 8; j += 2) {
+          a0 = __ffma2_rn(qf[hh][j], kf[j], a0);
+          a1 = __ffma2_rn(qf[hh][j + 1], kf[j + 1], a1);
         }
-        z[i][hh] = a0 + a1;
+        z[i][hh] = (a0.x + a0.y) + (a1.x + a1.y);
       }
     }
 #pragma unroll
@@ -281,30 +276,31 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS)
         pv[i][hh] = (VT == PKV_FP16) ? pr : pr * vs;
       }
       l_run[hh] = fmaf(l_run[hh], alpha, lsum);
+      const float2 alpha2 = make_float2(alpha, alpha);
 #pragma unroll
-      for (int j = 0; j < 16; ++j) acc[hh][j] *= alpha;
+      for (int j = 0; j < 8; ++j) acc[hh][j] = __fmul2_rn(acc[hh][j], alpha2);
     }
 
     // p . v_hat for this lane's rows and dims
 #pragma unroll
     for (int i = 0; i < C::TPL; ++i) {
       const int row = tg + C::TG * i;
-      float vf[16];
-      load_v16<VT>(vt + row * C::V_ROW + c * (C::V_ROW / C::CH), zp_bias, vf);
+      float2 vf[8];
+      load_v16<VT>(vt + row * C::V_ROW + c * (C::V_ROW / C::CH), neg_zp_bias, vf);
 #pragma unroll
-      for (int hh = 0; hh < GT; ++hh)
+      for (int hh = 0; hh < GT; ++hh) {
+        const float2 pv2 = make_float2(pv[i][hh], pv[i][hh]);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) acc[hh][j] = fmaf(pv[i][hh], vf[j], acc[hh][j]);
+        for (int j = 0; j < 8; ++j) acc[hh][j] = __ffma2_rn(pv2, vf[j], acc[hh][j]);
+      }
     }
 
     // stage st is free again: refill it with block k + NS
     __syncwarp();
     const int kn = k + C::NS;
     const int bn = __shfl_sync(kFull, my_b, kn & 31);
-    if (lane == 0 && kn < my_blocks) {
-      fence_proxy_async_smem();
-      issue(st, bn);
-    }
+    // (the warp's reads of this stage have completed: their values were consumed above)
+    if (lane == 0 && kn < my_blocks) issue(st, bn);
   }
 
   if (aborted) {
@@ -320,7 +316,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS)
       m_run[hh] = kNegBig;
       l_run[hh] = 0.f;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) acc[hh][j] = 0.f;
+      for (int j = 0; j < 8; ++j) acc[hh][j] = make_float2(0.f, 0.f);
     }
   }
 
@@ -330,16 +326,20 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS)
 #pragma unroll
     for (int off = C::CH; off < 32; off <<= 1) l_run[hh] += __shfl_xor_sync(kFull, l_run[hh], off);
 #pragma unroll
-    for (int j = 0; j < 16; ++j)
+    for (int j = 0; j < 8; ++j)
 #pragma unroll
-      for (int off = C::CH; off < 32; off <<= 1) acc[hh][j] += __shfl_xor_sync(kFull, acc[hh][j], off);
+      for (int off = C::CH; off < 32; off <<= 1) {
+        acc[hh][j].x += __shfl_xor_sync(kFull, acc[hh][j].x, off);
+        acc[hh][j].y += __shfl_xor_sync(kFull, acc[hh][j].y, off);
+      }
   }
   if (tg == 0) {
 #pragma unroll
     for (int hh = 0; hh < GT; ++hh) {
       float4* dst = reinterpret_cast<float4*>(merge_acc + ((size_t)warp * GT + hh) * D + c * 16);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) dst[j] = make_float4(acc[hh][4 * j], acc[hh][4 * j + 1], acc[hh][4 * j + 2], acc[hh][4 * j + 3]);
+      for (int j = 0; j < 4; ++j)
+        dst[j] = make_float4(acc[hh][2 * j].x, acc[hh][2 * j].y, acc[hh][2 * j + 1].x, acc[hh][2 * j + 1].y);
     }
   }
   if (lane == 0) {
