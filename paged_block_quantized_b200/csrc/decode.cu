@@ -134,7 +134,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS)
     b_raw = p.block_tables[(size_t)s * p.max_blocks_per_seq + j_lane];
   int L = p.context_lens[s];
 
-  // query heads of the CTA, this lane's 16 dims, fp32
+  // query heads of the CTA, this lane's 16 dims
   float2 qf[GT][8];
 #pragma unroll
   for (int hh = 0; hh < GT; ++hh) {
@@ -144,6 +144,46 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS)
     const uint32_t u[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
     for (int i = 0; i < 8; ++i) qf[hh][i] = __half22float2(*reinterpret_cast<const __half2*>(&u[i]));
+  }
+  // INT8 K: q . k is computed exactly in integers. Each head's q is put on a fixed-point grid of
+  // 2^-shift (22 bits below its largest magnitude; fp16 q loses nothing above 2^-22 of its max)
+  // and split into three signed byte planes, q_fixed = 2^16 b2 + 2^8 b1 + b0, so a 4-code word
+  // costs three dp4a with int32 accumulation and no code ever has to be converted to float.
+  uint32_t qplane[GT][3][4];
+  float qinv[GT];  // 2^-shift
+  if constexpr (KT == PKV_INT8_SYM) {
+#pragma unroll
+    for (int hh = 0; hh < GT; ++hh) {
+      float amax = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fmaxf(fabsf(qf[hh][i].x), fabsf(qf[hh][i].y)));
+#pragma unroll
+      for (int off = 1; off < C::CH; off <<= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, off));
+      int e = 0;
+      (void)frexpf(amax, &e);                    // amax < 2^e
+      const int shift = amax > 0.f ? 22 - e : 0;  // |q| * 2^shift < 2^22
+      const float up = __int_as_float((127 + shift) << 23);
+      qinv[hh] = __int_as_float((127 - shift) << 23);
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        uint32_t p0 = 0, p1 = 0, p2 = 0;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 pr = qf[hh][(4 * w + k) / 2];
+          const int qi = __float2int_rn((((4 * w + k) & 1) ? pr.y : pr.x) * up);
+          const int b0 = ((qi + 128) & 0xFF) - 128;
+          const int r1 = (qi - b0) >> 8;
+          const int b1 = ((r1 + 128) & 0xFF) - 128;
+          const int b2 = (r1 - b1) >> 8;
+          p0 |= (uint32_t)(b0 & 0xFF) << (8 * k);
+          p1 |= (uint32_t)(b1 & 0xFF) << (8 * k);
+          p2 |= (uint32_t)(b2 & 0xFF) << (8 * k);
+        }
+        qplane[hh][0][w] = p0;
+        qplane[hh][1][w] = p1;
+        qplane[hh][2][w] = p2;
+      }
+    }
   }
 
   // ---- context length (validated; clamped on error) and this warp's share of the partition ----
@@ -216,7 +256,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS)
       k_stop = k;
       break;
     }
-    const float ks = __shfl_sync(kFull, my_ks, k) * p.scale_log2;
+    const float ks = __shfl_sync(kFull, my_ks, k) * p.scale_log2;  // per-block K scale, log2 domain
     const float vs = __shfl_sync(kFull, my_vs, k);
     const float nzb = -(kMagic + __shfl_sync(kFull, my_zp, k));
     const float2 neg_zp_bias = make_float2(nzb, nzb);
@@ -230,17 +270,36 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS)
 #pragma unroll
     for (int i = 0; i < C::TPL; ++i) {
       const int row = tg + C::TG * i;
-      float2 kf[8];
-      load_k16<KT>(kt + row * C::K_ROW + c * (C::K_ROW / C::CH), kf);
+      const uint8_t* krow = kt + row * C::K_ROW + c * (C::K_ROW / C::CH);
+      if constexpr (KT == PKV_INT8_SYM) {
+        const uint4 w = *reinterpret_cast<const uint4*>(krow);
+        const int kw[4] = {(int)w.x, (int)w.y, (int)w.z, (int)w.w};
 #pragma unroll
-      for (int hh = 0; hh < GT; ++hh) {
-        float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+        for (int hh = 0; hh < GT; ++hh) {
+          int acc_p[3];
 #pragma unroll
-        for (int j = 0; j < 8; j += 2) {
-          a0 = __ffma2_rn(qf[hh][j], kf[j], a0);
-          a1 = __ffma2_rn(qf[hh][j + 1], kf[j + 1], a1);
+          for (int pl = 0; pl < 3; ++pl) {
+            int a = __dp4a((int)qplane[hh][pl][0], kw[0], 0);
+            a = __dp4a((int)qplane[hh][pl][1], kw[1], a);
+            a = __dp4a((int)qplane[hh][pl][2], kw[2], a);
+            acc_p[pl] = __dp4a((int)qplane[hh][pl][3], kw[3], a);
+          }
+          // |acc_p| < 2^18: the low two planes combine exactly in int32, the top one in fp32
+          z[i][hh] = __fmaf_rn((float)acc_p[2], 65536.f, (float)(acc_p[1] * 256 + acc_p[0]));
         }
-        z[i][hh] = (a0.x + a0.y) + (a1.x + a1.y);
+      } else {
+        float2 kf[8];
+        load_k16<KT>(krow, kf);
+#pragma unroll
+        for (int hh = 0; hh < GT; ++hh) {
+          float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int j = 0; j < 8; j += 2) {
+            a0 = __ffma2_rn(qf[hh][j], kf[j], a0);
+            a1 = __ffma2_rn(qf[hh][j + 1], kf[j + 1], a1);
+          }
+          z[i][hh] = (a0.x + a0.y) + (a1.x + a1.y);
+        }
       }
     }
 #pragma unroll
@@ -256,18 +315,26 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS)
     for (int hh = 0; hh < GT; ++hh) {
       float mloc = -INFINITY;
 #pragma unroll
+      const float zscale = (KT == PKV_FP16) ? p.scale_log2 : ks * qinv[hh];
       for (int i = 0; i < C::TPL; ++i) {
         const int t = tok0 + tg + C::TG * i;
-        float zz = z[i][hh] * (KT == PKV_FP16 ? p.scale_log2 : ks);
+        float zz = z[i][hh] * zscale;
         zz = (valid && t < t_end) ? zz : -INFINITY;
         z[i][hh] = zz;
         mloc = fmaxf(mloc, zz);
       }
 #pragma unroll
       for (int off = C::CH; off < 32; off <<= 1) mloc = fmaxf(mloc, __shfl_xor_sync(kFull, mloc, off));
-      const float m_new = fmaxf(m_run[hh], mloc);
-      const float alpha = ex2(m_run[hh] - m_new);
-      m_run[hh] = m_new;
+      // the running max is warp-uniform; rescale only when it grows (rare after the first blocks)
+      if (mloc > m_run[hh]) {
+        const float alpha = ex2(m_run[hh] - mloc);
+        m_run[hh] = mloc;
+        l_run[hh] *= alpha;
+        const float2 alpha2 = make_float2(alpha, alpha);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[hh][j] = __fmul2_rn(acc[hh][j], alpha2);
+      }
+      const float m_new = m_run[hh];
       float lsum = 0.f;
 #pragma unroll
       for (int i = 0; i < C::TPL; ++i) {
@@ -275,10 +342,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS)
         lsum += pr;
         pv[i][hh] = (VT == PKV_FP16) ? pr : pr * vs;
       }
-      l_run[hh] = fmaf(l_run[hh], alpha, lsum);
-      const float2 alpha2 = make_float2(alpha, alpha);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) acc[hh][j] = __fmul2_rn(acc[hh][j], alpha2);
+      l_run[hh] += lsum;
     }
 
     // p . v_hat for this lane's rows and dims
@@ -385,14 +449,14 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS)
   // next call without a reset. The CTA that sees num_parts - 1 merges
   //   out = sum_p 2^(m_p - M) acc_p / sum_p 2^(m_p - M) l_p.
   __shared__ uint32_t s_ticket;
-  __threadfence();  // this CTA's partial is visible device-wide before the counter moves
-  __syncthreads();
+  __syncthreads();  // every partial write of this CTA precedes thread 0's fence (CTA scope)
   if (threadIdx.x == 0) {
+    __threadfence();  // release: the CTA's partial is visible device-wide before the counter moves
     s_ticket = atomicInc(&p.ws_count[(size_t)s * gridDim.x + blockIdx.x], (uint32_t)(num_parts - 1));
+    __threadfence();  // acquire side for the merging CTA
   }
   __syncthreads();
   if (s_ticket != (uint32_t)(num_parts - 1)) return;
-  __threadfence();  // order the reads of the other CTAs' partials after the ticket
   for (int o = threadIdx.x; o < GT * D; o += C::THREADS) {
     const int hh = o / D, d = o % D;
     const size_t base = ((size_t)s * p.num_q_heads + h0 + hh) * p.max_partitions;
