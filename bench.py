@@ -192,7 +192,8 @@ def config_block(w, g, step_desc):
         "head_dim": w.head_dim, "block_size": w.block_size, "num_blocks": w.num_blocks,
         "kv_dtype": f"{KV_NAMES[w.k_dtype]}/{KV_NAMES[w.v_dtype]}",
         "tokens_per_step": w.total_tokens, "max_context_len": w.max_context_len,
-        "partition_tokens": g.effective_partition_tokens if g is not None else w.partition_tokens,
+        "partition_tokens": g.partition_tokens if g is not None else w.partition_tokens,
+        "decode_worker_warps": g.num_workers if g is not None else None,
         "step": step_desc, "seed": w.seed,
     }
 

@@ -144,24 +144,24 @@ PKV_API pkv_status pkv_store_quantized(const pkv_cache_desc* desc, const void* k
 
 /*
  * pkv_decode_workspace_size -- bytes of scratch pkv_paged_attention_decode needs for these
- * sizes: one arrival counter per (seq, CTA head group) plus the split-K partials (max, sum and
- * fp32 accumulator per (seq, q head, partition)); never a dequantized copy of the cache.
- * 0 when every sequence fits one partition. partition_tokens 0 selects the same automatic
- * choice as the decode call. Returns PKV_ERR_INVALID_ARG on bad sizes.
+ * sizes: one ticket per (sequence, head group) plus one partial (max, sum, fp32 accumulator)
+ * slot per (sequence, head group) and per worker warp; never a dequantized copy of the cache.
+ * The value depends on the current device (its SM count sets the number of worker warps).
+ * Returns PKV_ERR_INVALID_ARG on bad sizes.
  */
 PKV_API pkv_status pkv_decode_workspace_size(const pkv_cache_desc* desc, int32_t num_seqs,
-                                     int32_t num_q_heads, int32_t max_context_len,
-                                     int32_t partition_tokens, size_t* bytes);
+                                             int32_t num_q_heads, int32_t max_context_len,
+                                             int32_t partition_tokens, size_t* bytes);
 
 /*
- * pkv_decode_partitioning -- the split the decode call will use for these sizes: tokens per
- * partition (the given value, or the automatic choice when partition_tokens is 0) and the
- * number of partitions of the longest sequence. Either output pointer may be NULL.
+ * pkv_decode_partitioning -- how the decode call splits the work for these sizes: the number of
+ * worker warps (each takes an equal share of all KV blocks) and of persistent CTAs on the
+ * current device. Either output pointer may be NULL.
  */
 PKV_API pkv_status pkv_decode_partitioning(const pkv_cache_desc* desc, int32_t num_seqs,
                                            int32_t num_q_heads, int32_t max_context_len,
-                                           int32_t partition_tokens, int32_t* partition_tokens_out,
-                                           int32_t* num_partitions_out);
+                                           int32_t partition_tokens, int32_t* num_workers_out,
+                                           int32_t* num_ctas_out);
 
 /*
  * pkv_paged_attention_decode -- one decode step of attention over the paged, quantized cache.
@@ -172,9 +172,13 @@ PKV_API pkv_status pkv_decode_partitioning(const pkv_cache_desc* desc, int32_t n
  *   k_hat = code * k_scale[b][g]; v_hat = (code - zp) * v_scale[b][g] ([yunthe] x_hat formula);
  *   z_t = softmax_scale * dot(q[s][h], k_hat_t); out[s][h] = sum_t softmax(z)_t * v_hat_t,
  *   written as fp16 (round to nearest). L_s == 0 gives out = 0.
- * Long contexts are split into partitions of partition_tokens tokens (a multiple of block_size,
- * at most 128 * block_size; 0 = automatic). Partition CTAs publish partial results to the
- * workspace and the last one of a sequence to finish merges them, all in one kernel launch.
+ * Work split: all KV blocks of the batch form one stream, ordered (sequence, head group, block),
+ * cut into equal contiguous shares for a persistent set of worker warps, so any length mix is
+ * balanced. A (sequence, head group) cut between warps gets one partial per warp in the
+ * workspace and the last of them to finish merges them, all in one kernel launch.
+ * partition_tokens 0 uses every resident warp of the device; a positive multiple of block_size
+ * asks for about one worker per partition_tokens tokens of the largest possible work
+ * (num_seqs * heads * max_context_len), i.e. fewer workers and fewer cuts.
  *
  *   q            device fp16 [num_seqs][num_q_heads][head_dim]
  *   out          device fp16 [num_seqs][num_q_heads][head_dim]
@@ -182,11 +186,11 @@ PKV_API pkv_status pkv_decode_partitioning(const pkv_cache_desc* desc, int32_t n
  *   context_lens device int32 [num_seqs]; each <= max_context_len (host bound used to size the
  *                grid) and <= max_blocks_per_seq * block_size, else PKV_DEVERR_CONTEXT_LEN and the
  *                sequence is clamped
- *   workspace    device, >= pkv_decode_workspace_size(...) bytes, 16-byte aligned; may be NULL
- *                when that size is 0. It must be zero-filled before its first use: every call
- *                that completes leaves its arrival counters at zero again, so one zeroing serves
- *                any number of later calls (zero it again after a PKV_DEVERR_TIMEOUT). Calls that
- *                share a workspace must not overlap on the GPU.
+ *   workspace    device, >= pkv_decode_workspace_size(...) bytes, 16-byte aligned. It must be
+ *                zero-filled before its first use: every call that completes leaves its tickets
+ *                at zero again, so one zeroing serves any number of later calls (zero it again
+ *                after a PKV_DEVERR_TIMEOUT). Calls that share a workspace must not overlap on
+ *                the GPU.
  *   dev_error    device int32 or NULL
  * num_q_heads must be a multiple of num_kv_heads.
  */

@@ -55,56 +55,49 @@ int sm_count() {
   return c;
 }
 
-// Automatic partition size: the longest partition (fewest partials to merge) that still gives
-// every SM several CTAs of work; never shorter than one block per warp.
-int32_t auto_partition(const pkv_cache_desc* d, int32_t num_seqs, int32_t num_q_heads, int32_t max_context_len) {
-  const int32_t bs = d->block_size;
-  const int32_t group = num_q_heads / d->num_kv_heads;
-  const int64_t units = (int64_t)num_seqs * (num_q_heads / decode_heads_per_cta(group));
-  const int64_t target = (int64_t)sm_count() * 12;
-  const int32_t cap = decode_max_partition_tokens(bs);
-  int32_t pt = cap < 1024 ? cap : 1024;
-  const int32_t floor_pt = 4 * bs;
-  while (pt > floor_pt) {
-    const int64_t parts = (max_context_len + pt - 1) / pt;
-    if (units * (parts > 0 ? parts : 1) >= target) break;
-    pt /= 2;
-  }
-  if (pt < floor_pt) pt = floor_pt;
-  return pt - pt % bs;
-}
-
 struct DecodeGeometry {
-  int32_t partition_tokens;
-  int32_t max_partitions;
-  size_t counter_bytes;    // arrival counters at the start of the workspace (256-byte padded)
-  size_t workspace_bytes;  // counters + partial (max, sum) + partial accumulators
+  DecodeShape shape;
+  int32_t workers;          // worker warps of the persistent grid
+  size_t counter_bytes;     // split-unit tickets at the start of the workspace (256-byte padded)
+  size_t ml_bytes;          // partial (max, sum) pairs (256-byte padded)
+  size_t workspace_bytes;   // counters + (max, sum) + partial accumulators
 };
 
+// Worker warps: every resident warp of the GPU by default; with partition_tokens > 0, about one
+// warp per partition_tokens tokens of the largest possible work (fewer warps, fewer splits).
 pkv_status decode_geometry(const pkv_cache_desc* d, int32_t num_seqs, int32_t num_q_heads,
                            int32_t max_context_len, int32_t partition_tokens, DecodeGeometry* g) {
   if (num_seqs < 0 || num_q_heads <= 0 || max_context_len < 0 || partition_tokens < 0) return PKV_ERR_INVALID_ARG;
   if (num_q_heads % d->num_kv_heads != 0) return PKV_ERR_INVALID_ARG;
-  int32_t pt = partition_tokens;
-  if (pt == 0) {
-    pt = auto_partition(d, num_seqs, num_q_heads, max_context_len);
-  } else {
-    if (pt % d->block_size != 0) return PKV_ERR_INVALID_ARG;
-    if (pt > decode_max_partition_tokens(d->block_size)) return PKV_ERR_UNSUPPORTED;
+  if (partition_tokens % d->block_size != 0) return PKV_ERR_INVALID_ARG;
+  const int32_t group = num_q_heads / d->num_kv_heads;
+  DecodeShape& sh = g->shape;
+  sh.k_dtype = d->k_dtype;
+  sh.v_dtype = d->v_dtype;
+  sh.block_size = d->block_size;
+  sh.head_dim = d->head_dim;
+  sh.heads_per_warp = decode_heads_per_warp(group);
+  DecodeKernelInfo info;
+  if (!decode_kernel_info(sh, &info)) return PKV_ERR_UNSUPPORTED;
+  const int64_t max_workers = (int64_t)sm_count() * info.ctas_per_sm * info.warps_per_cta;
+  int64_t workers = max_workers;
+  if (partition_tokens > 0) {
+    const int64_t hg = num_q_heads / sh.heads_per_warp;
+    const int64_t blocks = (int64_t)num_seqs * hg * ((max_context_len + d->block_size - 1) / d->block_size);
+    const int64_t per = partition_tokens / d->block_size;
+    workers = (blocks + per - 1) / per;
+    workers = (workers + info.warps_per_cta - 1) / info.warps_per_cta * info.warps_per_cta;
+    if (workers < info.warps_per_cta) workers = info.warps_per_cta;
+    if (workers > max_workers) workers = max_workers;
   }
-  int64_t parts = ((int64_t)max_context_len + pt - 1) / pt;
-  if (parts < 1) parts = 1;
-  if (parts > 65535 || num_seqs > 65535) return PKV_ERR_UNSUPPORTED;  // grid limits
-  g->partition_tokens = pt;
-  g->max_partitions = (int32_t)parts;
-  if (parts > 1) {
-    const size_t counters = (size_t)num_seqs * (num_q_heads / decode_heads_per_cta(num_q_heads / d->num_kv_heads));
-    g->counter_bytes = (counters * sizeof(uint32_t) + 255) / 256 * 256;
-    g->workspace_bytes = g->counter_bytes + (size_t)num_seqs * num_q_heads * parts * (d->head_dim + 2) * sizeof(float);
-  } else {
-    g->counter_bytes = 0;
-    g->workspace_bytes = 0;
-  }
+  sh.grid_ctas = (int32_t)(workers / info.warps_per_cta);
+  g->workers = (int32_t)workers;
+  const size_t units = (size_t)num_seqs * (num_q_heads / sh.heads_per_warp);
+  const size_t slots = units + (size_t)workers;
+  g->counter_bytes = (units * sizeof(uint32_t) + 255) / 256 * 256;
+  g->ml_bytes = (slots * sh.heads_per_warp * 2 * sizeof(float) + 255) / 256 * 256;
+  g->workspace_bytes =
+      num_seqs > 0 ? g->counter_bytes + g->ml_bytes + slots * sh.heads_per_warp * d->head_dim * sizeof(float) : 0;
   return PKV_OK;
 }
 
@@ -173,15 +166,15 @@ pkv_status pkv_decode_workspace_size(const pkv_cache_desc* desc, int32_t num_seq
 }
 
 pkv_status pkv_decode_partitioning(const pkv_cache_desc* desc, int32_t num_seqs, int32_t num_q_heads,
-                                   int32_t max_context_len, int32_t partition_tokens, int32_t* partition_tokens_out,
-                                   int32_t* num_partitions_out) {
+                                   int32_t max_context_len, int32_t partition_tokens, int32_t* num_workers_out,
+                                   int32_t* num_ctas_out) {
   pkv_status st = check_desc(desc);
   if (st != PKV_OK) return st;
   DecodeGeometry g;
   st = decode_geometry(desc, num_seqs, num_q_heads, max_context_len, partition_tokens, &g);
   if (st != PKV_OK) return st;
-  if (partition_tokens_out) *partition_tokens_out = g.partition_tokens;
-  if (num_partitions_out) *num_partitions_out = g.max_partitions;
+  if (num_workers_out) *num_workers_out = g.workers;
+  if (num_ctas_out) *num_ctas_out = g.shape.grid_ctas;
   return PKV_OK;
 }
 
@@ -202,8 +195,7 @@ pkv_status pkv_paged_attention_decode(const pkv_cache_desc* desc, void* out, con
     return PKV_ERR_INVALID_ARG;
   if (max_blocks_per_seq <= 0) return PKV_ERR_INVALID_ARG;
   if (dev_error != nullptr && !aligned(dev_error, 4)) return PKV_ERR_INVALID_ARG;
-  if (g.workspace_bytes > 0 && (workspace == nullptr || workspace_bytes < g.workspace_bytes || !aligned(workspace, 16)))
-    return PKV_ERR_INVALID_ARG;
+  if (workspace == nullptr || workspace_bytes < g.workspace_bytes || !aligned(workspace, 16)) return PKV_ERR_INVALID_ARG;
   if (!(softmax_scale == softmax_scale)) return PKV_ERR_INVALID_ARG;  // NaN
 
   DecodeParams p;
@@ -216,31 +208,20 @@ pkv_status pkv_paged_attention_decode(const pkv_cache_desc* desc, void* out, con
   p.out = static_cast<__half*>(out);
   p.block_tables = block_tables;
   p.context_lens = context_lens;
-  const size_t ml_floats = (size_t)num_seqs * num_q_heads * g.max_partitions * 2;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  p.ws_count = g.workspace_bytes ? reinterpret_cast<uint32_t*>(ws) : nullptr;
-  p.ws_ml = g.workspace_bytes ? reinterpret_cast<float*>(ws + g.counter_bytes) : nullptr;
-  p.ws_acc = g.workspace_bytes ? reinterpret_cast<float*>(ws + g.counter_bytes) + ml_floats : nullptr;
+  p.ws_count = reinterpret_cast<uint32_t*>(ws);
+  p.ws_ml = reinterpret_cast<float*>(ws + g.counter_bytes);
+  p.ws_acc = reinterpret_cast<float*>(ws + g.counter_bytes + g.ml_bytes);
   p.dev_error = dev_error;
+  p.num_seqs = num_seqs;
   p.num_blocks = desc->num_blocks;
   p.num_kv_heads = desc->num_kv_heads;
   p.num_q_heads = num_q_heads;
   p.group = num_q_heads / desc->num_kv_heads;
   p.max_blocks_per_seq = max_blocks_per_seq;
   p.max_context_len = max_context_len;
-  p.partition_tokens = g.partition_tokens;
-  p.max_partitions = g.max_partitions;
   p.scale_log2 = softmax_scale * 1.4426950408889634f;  // log2(e)
-
-  DecodeShape sh;
-  sh.k_dtype = desc->k_dtype;
-  sh.v_dtype = desc->v_dtype;
-  sh.block_size = desc->block_size;
-  sh.head_dim = desc->head_dim;
-  sh.heads_per_cta = decode_heads_per_cta(p.group);
-  sh.num_seqs = num_seqs;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  return launch_decode(p, sh, s) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+  return launch_decode(p, g.shape, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
 pkv_status pkv_copy_blocks(const pkv_cache_desc* desc, const int32_t* block_mapping, int32_t n_pairs,

@@ -12,20 +12,25 @@
 // dequantized copy of the cache exists anywhere (tbr8.org page, §5 item 2: dequantize inside the
 // attention operator so no intermediate product occupies memory).
 //
-// How (B200 design, not taken from the pages):
-//   * grid = (query-head groups, partitions, sequences). A CTA owns one KV head, `GT` query heads
-//     of its group and one partition of `partition_tokens` tokens of one sequence.
-//   * Each of the NW warps streams every NW-th block of the partition through its own ring of NS
-//     shared-memory stages. One lane issues two 1-D bulk asynchronous copies per block (the
-//     contiguous bs x D K tile and V tile of this head, 1-4 KiB each) that complete on the
-//     stage's mbarrier; the warp then reads the tile with 16-byte shared loads.
-//   * Lane mapping: a lane owns 16 consecutive dims (D/16 lanes per token row) and bs/(32*16/D)
-//     token rows of each block. Codes become exact floats through the float bit layout (no I2F),
-//     dot products accumulate in fp32, the per-block scale multiplies the 16-term dot once.
-//   * Online softmax per warp in the log2 domain (ex2.approx); warps are merged through shared
-//     memory at the end; a sequence with one partition is written out directly, otherwise the
-//     partition's (max, sum, accumulator) goes to the workspace and the last of the sequence's
-//     partition CTAs to finish merges them (split-K in one launch, no second kernel).
+// How (B200 design, not taken from the pages): a persistent, stream-K kernel.
+//   * A "unit" is (sequence s, head group hg): GT query heads sharing one KV head. Every unit
+//     contributes ceil(L_s / bs) blocks to one global stream, ordered (s, hg, block). The grid
+//     is a fixed set of worker warps (a few CTAs per SM, each warp independent); warp w owns
+//     the contiguous stream range [w*T/W, (w+1)*T/W), so every warp gets the same number of
+//     blocks whatever the length mix.
+//   * Each warp streams its range through its own ring of NS shared-memory stages: lane 0
+//     issues two 1-D bulk asynchronous copies per block (the contiguous bs x D K tile and V tile
+//     of this head, 1-4 KiB each) that complete on the stage's mbarrier, up to NS blocks ahead
+//     and straight across unit boundaries; the warp reads tiles with 16-byte shared loads.
+//   * Block ids are read 32 at a time ("windows", one id per lane) one window ahead; per-block
+//     scales are fetched when the window's first copy is issued, NS blocks before use.
+//   * q . k for INT8 K is exact integer arithmetic: q on a 22-bit fixed-point grid split into
+//     three signed byte planes, three dp4a per 4 codes. V codes become exact floats through the
+//     float bit layout (PRMT + paired FADD, no I2F); p . v accumulates with paired FFMA.
+//   * Online softmax in the log2 domain (ex2.approx), rescaling only when the running max grows.
+//   * A unit processed entirely by one warp is written out directly. A unit split across warps
+//     gets one partial (max, sum, acc) per warp in the workspace; the last warp to finish (a
+//     self-resetting atomicInc ticket) merges them. No CTA barrier, no second kernel.
 #include "common.cuh"
 #include "internal.h"
 
@@ -38,45 +43,39 @@ constexpr float kNegBig = -1.0e30f;  // finite "minus infinity" for running maxi
 
 template <int KT, int VT, int BS, int D, int GT>
 struct Cfg {
-  static constexpr int NW = 4;  // warps per CTA
   static constexpr int K_ROW = (KT == PKV_FP16) ? 2 * D : D;
   static constexpr int V_ROW = (VT == PKV_FP16) ? 2 * D : (VT == PKV_INT8_SYM ? D : D / 2);
   static constexpr int K_TILE = BS * K_ROW;
   static constexpr int V_TILE = BS * V_ROW;
   static constexpr int STAGE = K_TILE + V_TILE;
-  // ~64 KiB of stages per CTA, 2..4 stages per warp
-  static constexpr int NS_RAW = 65536 / (NW * STAGE);
-  static constexpr int NS = NS_RAW < 2 ? 2 : (NS_RAW > 4 ? 4 : NS_RAW);
-  static constexpr int CH = D / 16;    // lanes per token row
+  static constexpr int NW = (4 * 2 * STAGE <= 200 * 1024) ? 4 : 2;  // warps per CTA
+  // about 48 KiB of stages per CTA, 2..6 stages per warp
+  static constexpr int NS_RAW = 49152 / (NW * STAGE);
+  static constexpr int NS = NS_RAW < 2 ? 2 : (NS_RAW > 6 ? 6 : NS_RAW);
+  static constexpr int CH = D / 16;    // lanes per token row (16 dims each)
   static constexpr int TG = 32 / CH;   // token rows a warp covers per pass
   static constexpr int TPL = BS / TG;  // token rows per lane per block
   static constexpr int THREADS = 32 * NW;
   static constexpr int SMEM_STAGES = NW * NS * STAGE;
-  static constexpr int SMEM_MERGE_ACC = NW * GT * D * 4;
-  static constexpr int SMEM_MERGE_ML = NW * GT * 2 * 4;
-  static constexpr int SMEM_BARS = NW * NS * 8;
-  static constexpr int SMEM = SMEM_STAGES + SMEM_MERGE_ACC + SMEM_MERGE_ML + SMEM_BARS;
+  static constexpr int SMEM = SMEM_STAGES + NW * NS * 8;
+  // resident CTAs per SM: bounded by shared memory (227 KiB per SM) and by the registers a
+  // thread needs for GT heads of state
+  static constexpr int CPS_SMEM = (220 * 1024) / (SMEM + 1024);
+  static constexpr int CPS_CAP = (GT == 1) ? 4 : (GT == 2 ? 3 : 2);  // 128 / 170 / 255 registers
+  static constexpr int CTAS_PER_SM = CPS_SMEM < 1 ? 1 : (CPS_SMEM > CPS_CAP ? CPS_CAP : CPS_SMEM);
   static_assert(D % 16 == 0 && CH <= 32 && 32 % CH == 0, "head_dim");
   static_assert(BS % TG == 0, "block_size must cover the token rows of a warp pass");
   static_assert(K_TILE % 16 == 0 && V_TILE % 16 == 0 && STAGE % 16 == 0, "bulk copy granularity");
+  static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 };
 
-// 16 consecutive K values of one token row (lane chunk) -> 8 float2 (dims in order)
-template <int KT>
-__device__ __forceinline__ void load_k16(const uint8_t* p, float2 f[8]) {
-  if constexpr (KT == PKV_INT8_SYM) {
-    const uint4 w = *reinterpret_cast<const uint4*>(p);
-    s8x4_to_f32x2(w.x, f[0], f[1]);
-    s8x4_to_f32x2(w.y, f[2], f[3]);
-    s8x4_to_f32x2(w.z, f[4], f[5]);
-    s8x4_to_f32x2(w.w, f[6], f[7]);
-  } else {
-    const uint4 w0 = *reinterpret_cast<const uint4*>(p);
-    const uint4 w1 = *reinterpret_cast<const uint4*>(p + 16);
-    const uint32_t u[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+// 16 consecutive fp16 values of one token row (lane chunk) -> 8 float2 (dims in order)
+__device__ __forceinline__ void load_h16(const uint8_t* p, float2 f[8]) {
+  const uint4 w0 = *reinterpret_cast<const uint4*>(p);
+  const uint4 w1 = *reinterpret_cast<const uint4*>(p + 16);
+  const uint32_t u[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-    for (int i = 0; i < 8; ++i) f[i] = __half22float2(*reinterpret_cast<const __half2*>(&u[i]));
-  }
+  for (int i = 0; i < 8; ++i) f[i] = __half22float2(*reinterpret_cast<const __half2*>(&u[i]));
 }
 
 // 16 consecutive V values of one token row (lane chunk) -> 8 float2 of (code - zp);
@@ -84,196 +83,344 @@ __device__ __forceinline__ void load_k16(const uint8_t* p, float2 f[8]) {
 template <int VT>
 __device__ __forceinline__ void load_v16(const uint8_t* p, float2 neg_bias, float2 f[8]) {
   if constexpr (VT == PKV_INT8_SYM) {
-    load_k16<PKV_INT8_SYM>(p, f);
+    const uint4 w = *reinterpret_cast<const uint4*>(p);
+    s8x4_to_f32x2(w.x, f[0], f[1]);
+    s8x4_to_f32x2(w.y, f[2], f[3]);
+    s8x4_to_f32x2(w.z, f[4], f[5]);
+    s8x4_to_f32x2(w.w, f[6], f[7]);
   } else if constexpr (VT == PKV_INT4_ASYM) {
     const uint2 w = *reinterpret_cast<const uint2*>(p);
     u4x8_to_f32x2(w.x, neg_bias, f);
     u4x8_to_f32x2(w.y, neg_bias, f + 4);
   } else {
-    load_k16<PKV_FP16>(p, f);
+    load_h16(p, f);
   }
 }
 
+__device__ __forceinline__ int clamp_len(const DecodeParams& p, int L, int bs) {
+  const int cap = min(p.max_context_len, p.max_blocks_per_seq * bs);
+  return max(0, min(L, cap));
+}
+
+// The worker warp whose stream range contains position g (start_w = floor(w*T/W) <= g).
+__device__ __forceinline__ int owner_of(long long g, long long T, int W) {
+  return (int)(((g + 1) * (long long)W - 1) / T);
+}
+
+// A window: up to 32 consecutive blocks of one unit (warp-uniform description; lane k holds
+// block j0 + k in the per-lane registers of the window).
+struct Win {
+  int s, hg, j0, n;     // sequence, head group, first block, blocks in the window (0 = none)
+  int L, nblk;          // clamped length of the sequence and its block count
+  long long p0;         // stream position of block j0
+  long long seq_p0;     // stream position of the sequence's first block (head group 0)
+};
+
+struct WinLanes {
+  int b;        // physical block (0 stands in for an invalid id)
+  int raw;      // block id as read from the table
+  bool valid;
+  bool meta;    // scales fetched (warp-uniform)
+  float ks, vs, zp;
+};
+
 template <int KT, int VT, int BS, int D, int GT>
-__global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS)
+__global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, BS, D, GT>::CTAS_PER_SM)
     paged_decode_kernel(const DecodeParams p) {
   using C = Cfg<KT, VT, BS, D, GT>;
   extern __shared__ __align__(128) uint8_t smem[];
-  uint8_t* stages = smem;
-  float* merge_acc = reinterpret_cast<float*>(smem + C::SMEM_STAGES);                 // [NW][GT][D]
-  float* merge_ml = reinterpret_cast<float*>(smem + C::SMEM_STAGES + C::SMEM_MERGE_ACC);  // [NW][GT][2]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SMEM_STAGES + C::SMEM_MERGE_ACC + C::SMEM_MERGE_ML);
-
-  const int h0 = blockIdx.x * GT;  // first query head of this CTA
-  const int part = blockIdx.y;
-  const int s = blockIdx.z;
-  const int g = h0 / p.group;  // KV head shared by the CTA's query heads
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int c = lane % C::CH;   // 16-dim chunk of this lane
   const int tg = lane / C::CH;  // token-row group of this lane
-  const int PT = p.partition_tokens;
+  const int W = gridDim.x * C::NW;
+  const int w = blockIdx.x * C::NW + warp;
+  const int HG = p.num_q_heads / GT;
+  const int S = p.num_seqs;
 
-  // ---- pipeline set-up: this warp's NS stages and barriers (no memory dependence) ----
-  uint8_t* my_stages = stages + (size_t)warp * C::NS * C::STAGE;
-  uint64_t* my_bars = bars + warp * C::NS;
+  uint8_t* my_stages = smem + (size_t)warp * C::NS * C::STAGE;
+  uint64_t* my_bars = reinterpret_cast<uint64_t*>(smem + C::SMEM_STAGES) + warp * C::NS;
   if (lane == 0) {
 #pragma unroll
     for (int st = 0; st < C::NS; ++st) mbar_init(&my_bars[st], 1);
     fence_mbar_init();
   }
 
-  // ---- first round of global loads, all independent of one another ----
-  // The partition's first block index does not depend on the context length, so this warp's
-  // block-table entries are read speculatively (in bounds of the table row) together with the
-  // length; entries past the sequence's end are never used.
-  const int blk_begin = (part * PT) / BS;
-  const int j_lane = blk_begin + warp + C::NW * lane;
-  int b_raw = -1;
-  if (lane * C::NW * BS < PT && j_lane < p.max_blocks_per_seq)
-    b_raw = p.block_tables[(size_t)s * p.max_blocks_per_seq + j_lane];
-  int L = p.context_lens[s];
-
-  // query heads of the CTA, this lane's 16 dims
-  float2 qf[GT][8];
+  // ---- pass 1: total stream length T; zero the outputs of empty sequences ----
+  long long T = 0;
+  for (int base = 0; base < S; base += 32) {
+    const int s = base + lane;
+    int L = 0;
+    if (s < S) {
+      const int raw = p.context_lens[s];
+      L = clamp_len(p, raw, BS);
+      if (raw != L && w == 0) record_error(p.dev_error, PKV_DEVERR_CONTEXT_LEN);
+    }
+    int sum = (L + BS - 1) / BS;
 #pragma unroll
-  for (int hh = 0; hh < GT; ++hh) {
-    const __half* qp = p.q + ((size_t)s * p.num_q_heads + h0 + hh) * D + c * 16;
-    const uint4 w0 = *reinterpret_cast<const uint4*>(qp);
-    const uint4 w1 = *reinterpret_cast<const uint4*>(qp + 8);
-    const uint32_t u[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) qf[hh][i] = __half22float2(*reinterpret_cast<const __half2*>(&u[i]));
-  }
-  // INT8 K: q . k is computed exactly in integers. Each head's q is put on a fixed-point grid of
-  // 2^-shift (22 bits below its largest magnitude; fp16 q loses nothing above 2^-22 of its max)
-  // and split into three signed byte planes, q_fixed = 2^16 b2 + 2^8 b1 + b0, so a 4-code word
-  // costs three dp4a with int32 accumulation and no code ever has to be converted to float.
-  uint32_t qplane[GT][3][4];
-  float qinv[GT];  // 2^-shift
-  if constexpr (KT == PKV_INT8_SYM) {
-#pragma unroll
-    for (int hh = 0; hh < GT; ++hh) {
-      float amax = 0.f;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fmaxf(fabsf(qf[hh][i].x), fabsf(qf[hh][i].y)));
-#pragma unroll
-      for (int off = 1; off < C::CH; off <<= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, off));
-      int e = 0;
-      (void)frexpf(amax, &e);                    // amax < 2^e
-      const int shift = amax > 0.f ? 22 - e : 0;  // |q| * 2^shift < 2^22
-      const float up = __int_as_float((127 + shift) << 23);
-      qinv[hh] = __int_as_float((127 - shift) << 23);
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        uint32_t p0 = 0, p1 = 0, p2 = 0;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float2 pr = qf[hh][(4 * w + k) / 2];
-          const int qi = __float2int_rn((((4 * w + k) & 1) ? pr.y : pr.x) * up);
-          const int b0 = ((qi + 128) & 0xFF) - 128;
-          const int r1 = (qi - b0) >> 8;
-          const int b1 = ((r1 + 128) & 0xFF) - 128;
-          const int b2 = (r1 - b1) >> 8;
-          p0 |= (uint32_t)(b0 & 0xFF) << (8 * k);
-          p1 |= (uint32_t)(b1 & 0xFF) << (8 * k);
-          p2 |= (uint32_t)(b2 & 0xFF) << (8 * k);
-        }
-        qplane[hh][0][w] = p0;
-        qplane[hh][1][w] = p1;
-        qplane[hh][2][w] = p2;
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(kFull, sum, off);
+    T += sum;
+    uint32_t empty = __ballot_sync(kFull, s < S && L == 0);
+    while (empty) {  // outputs of sequences with nothing to attend over are 0
+      const int e = __ffs(empty) - 1;
+      empty &= empty - 1;
+      const int se = base + e;
+      for (int hg = 0; hg < HG; ++hg) {
+        if ((int)(((long long)se * HG + hg) % W) != w) continue;
+        __half2* o = reinterpret_cast<__half2*>(p.out + ((size_t)se * p.num_q_heads + (size_t)hg * GT) * D);
+        for (int i = lane; i < GT * D / 2; i += 32) o[i] = __floats2half2_rn(0.f, 0.f);
       }
     }
   }
+  T *= HG;
+  __syncwarp();
+  // With fewer blocks than warps only the first T warps work, so that every working warp owns
+  // at least one block and the warps sharing a unit are consecutive (the merge relies on it).
+  const int We = (int)min((long long)W, T);
+  if (w >= We) return;
+  const long long start = (long long)w * T / We;
+  const long long end = (long long)(w + 1) * T / We;
 
-  // ---- context length (validated; clamped on error) and this warp's share of the partition ----
+  // ---- pass 2: the unit and block of `start` ----
+  Win cur;
+  int Lchunk = 0, chunk_base = 0;  // lane holds the clamped length of sequence chunk_base + lane
   {
-    const int cap = min(p.max_context_len, p.max_blocks_per_seq * BS);
-    if (L < 0 || L > cap) {
-      if (part == 0 && blockIdx.x == 0 && threadIdx.x == 0) record_error(p.dev_error, PKV_DEVERR_CONTEXT_LEN);
-      L = max(0, min(L, cap));
+    long long acc0 = 0;
+    for (int base = 0;; base += 32) {
+      const int s = base + lane;
+      const int L = s < S ? clamp_len(p, p.context_lens[s], BS) : 0;
+      const long long cnt = (long long)((L + BS - 1) / BS) * HG;
+      long long incl = cnt;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const long long o = __shfl_up_sync(kFull, incl, off);
+        if (lane >= off) incl += o;
+      }
+      const long long total = __shfl_sync(kFull, incl, 31);
+      if (acc0 + total > start) {
+        const uint32_t m = __ballot_sync(kFull, acc0 + incl > start);
+        const int f = __ffs(m) - 1;
+        cur.s = base + f;
+        cur.L = __shfl_sync(kFull, L, f);
+        cur.nblk = (cur.L + BS - 1) / BS;
+        cur.seq_p0 = acc0 + __shfl_sync(kFull, incl - cnt, f);
+        Lchunk = L;
+        chunk_base = base;
+        break;
+      }
+      acc0 += total;
     }
+    const long long o = start - cur.seq_p0;
+    cur.hg = (int)(o / cur.nblk);
+    cur.j0 = (int)(o % cur.nblk);
+    cur.p0 = start;
+    cur.n = (int)min((long long)min(32, cur.nblk - cur.j0), end - start);
   }
-  const int num_parts = (L + PT - 1) / PT;
-  if (part >= (num_parts > 0 ? num_parts : 1)) return;  // beyond this sequence's partitions (CTA-uniform)
 
-  const int t_begin = part * PT;
-  const int t_end = min(L, t_begin + PT);
-  const int n_blk = t_end > t_begin ? (t_end - t_begin + BS - 1) / BS : 0;
-  // this warp's blocks: blk_begin + warp + NW * k, k < my_blocks (<= 32 by the partition cap)
-  const int my_blocks = n_blk > warp ? (n_blk - warp + C::NW - 1) / C::NW : 0;
+  // clamped length of sequence s, from the lane-held chunk when possible
+  auto seq_len = [&](int s) -> int {
+    if (s < chunk_base || s >= chunk_base + 32) {
+      chunk_base = s;
+      Lchunk = (s + lane < S) ? clamp_len(p, p.context_lens[s + lane], BS) : 0;
+    }
+    return __shfl_sync(kFull, Lchunk, s - chunk_base);
+  };
 
-  const bool my_valid = lane < my_blocks && b_raw >= 0 && b_raw < p.num_blocks;
-  if (lane < my_blocks && !my_valid) record_error(p.dev_error, PKV_DEVERR_BLOCK_ID);
-  const int my_b = my_valid ? b_raw : 0;  // block 0 stands in for an invalid id (its tokens are masked)
+  // the window after `a`, within [.., end); n = 0 if none
+  auto next_win = [&](const Win& a) -> Win {
+    Win b = a;
+    b.p0 = a.p0 + a.n;
+    b.n = 0;
+    if (a.n == 0 || b.p0 >= end) return b;
+    b.j0 = a.j0 + a.n;
+    if (b.j0 >= a.nblk) {
+      b.j0 = 0;
+      b.hg = a.hg + 1;
+      if (b.hg >= HG) {
+        b.hg = 0;
+        b.seq_p0 = a.seq_p0 + (long long)HG * a.nblk;
+        int s = a.s, L = 0;
+        do {  // sequences without blocks contribute no stream positions
+          ++s;
+          L = s < S ? seq_len(s) : 0;
+        } while (L == 0 && s < S);
+        b.s = s;
+        b.L = L;
+        b.nblk = (L + BS - 1) / BS;
+      }
+    }
+    b.n = (int)min((long long)min(32, b.nblk - b.j0), end - b.p0);
+    return b;
+  };
+
+  // phase A of a window: block ids (one per lane); phase B (at its first copy): scales
+  auto load_ids = [&](const Win& a, WinLanes& r) {
+    r.meta = false;
+    r.raw = -1;
+    if (lane < a.n) r.raw = p.block_tables[(size_t)a.s * p.max_blocks_per_seq + a.j0 + lane];
+  };
+  auto load_meta = [&](const Win& a, WinLanes& r) {
+    r.valid = lane < a.n && r.raw >= 0 && r.raw < p.num_blocks;
+    if (lane < a.n && !r.valid) record_error(p.dev_error, PKV_DEVERR_BLOCK_ID);
+    r.b = r.valid ? r.raw : 0;
+    r.ks = r.vs = r.zp = 0.f;
+    if (lane < a.n) {
+      const int g = (a.hg * GT) / p.group;
+      const size_t meta = (size_t)r.b * p.num_kv_heads + g;
+      if constexpr (KT != PKV_FP16) r.ks = p.k_scale[meta];
+      if constexpr (VT != PKV_FP16) r.vs = p.v_scale[meta];
+      if constexpr (VT == PKV_INT4_ASYM) r.zp = (float)p.v_zp[meta];
+    }
+    r.meta = true;
+  };
+
+  WinLanes rc, rn;
+  load_ids(cur, rc);
+  Win nxt = next_win(cur);
+  load_ids(nxt, rn);
+  load_meta(cur, rc);
   __syncwarp();  // barrier initialisation by lane 0 is visible to the warp
 
-  const size_t head_tile = (size_t)p.num_kv_heads;
-  auto issue = [&](int st, int b) {
-    const size_t tile = (size_t)b * head_tile + g;
+  // ---- per-unit state ----
+  float2 qf[GT][8];
+  uint32_t qplane[GT][3][4];
+  float qinv[GT];
+  float m_run[GT], l_run[GT];
+  float2 acc[GT][8];
+  int seg_j0 = cur.j0;  // first block of the current segment within its unit
+
+  auto begin_unit = [&](const Win& a) {
+#pragma unroll
+    for (int hh = 0; hh < GT; ++hh) {
+      const __half* qp = p.q + ((size_t)a.s * p.num_q_heads + (size_t)a.hg * GT + hh) * D + c * 16;
+      const uint4 w0 = *reinterpret_cast<const uint4*>(qp);
+      const uint4 w1 = *reinterpret_cast<const uint4*>(qp + 8);
+      const uint32_t u[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) qf[hh][i] = __half22float2(*reinterpret_cast<const __half2*>(&u[i]));
+      m_run[hh] = kNegBig;
+      l_run[hh] = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[hh][j] = make_float2(0.f, 0.f);
+    }
+    // INT8 K: q . k is computed exactly in integers. Each head's q is put on a fixed-point grid
+    // of 2^-shift (22 bits below its largest magnitude; fp16 q loses nothing above 2^-22 of its
+    // max) and split into three signed byte planes, q_fixed = 2^16 b2 + 2^8 b1 + b0, so a
+    // 4-code word costs three dp4a with int32 accumulation and no code is converted to float.
+    if constexpr (KT == PKV_INT8_SYM) {
+#pragma unroll
+      for (int hh = 0; hh < GT; ++hh) {
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fmaxf(fabsf(qf[hh][i].x), fabsf(qf[hh][i].y)));
+#pragma unroll
+        for (int off = 1; off < C::CH; off <<= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, off));
+        int e = 0;
+        (void)frexpf(amax, &e);                    // amax < 2^e
+        const int shift = amax > 0.f ? 22 - e : 0;  // |q| * 2^shift < 2^22
+        const float up = __int_as_float((127 + shift) << 23);
+        qinv[hh] = __int_as_float((127 - shift) << 23);
+#pragma unroll
+        for (int wd = 0; wd < 4; ++wd) {
+          uint32_t p0 = 0, p1 = 0, p2 = 0;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 pr = qf[hh][(4 * wd + k) / 2];
+            const int qi = __float2int_rn((((4 * wd + k) & 1) ? pr.y : pr.x) * up);
+            const int b0 = ((qi + 128) & 0xFF) - 128;
+            const int r1 = (qi - b0) >> 8;
+            const int b1 = ((r1 + 128) & 0xFF) - 128;
+            const int b2 = (r1 - b1) >> 8;
+            p0 |= (uint32_t)(b0 & 0xFF) << (8 * k);
+            p1 |= (uint32_t)(b1 & 0xFF) << (8 * k);
+            p2 |= (uint32_t)(b2 & 0xFF) << (8 * k);
+          }
+          qplane[hh][0][wd] = p0;
+          qplane[hh][1][wd] = p1;
+          qplane[hh][2][wd] = p2;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int hh = 0; hh < GT; ++hh) qinv[hh] = 1.f;
+    }
+  };
+  begin_unit(cur);
+
+  // ---- the copy ring ----
+  auto issue = [&](int st, int b, int g) {
+    const size_t tile = (size_t)b * p.num_kv_heads + g;
     uint8_t* dst = my_stages + (size_t)st * C::STAGE;
     mbar_arrive_expect_tx(&my_bars[st], (uint32_t)C::STAGE);
     bulk_g2s(dst, static_cast<const uint8_t*>(p.k_codes) + tile * C::K_TILE, (uint32_t)C::K_TILE, &my_bars[st]);
     bulk_g2s(dst + C::K_TILE, static_cast<const uint8_t*>(p.v_codes) + tile * C::V_TILE, (uint32_t)C::V_TILE,
              &my_bars[st]);
   };
-
-  // ---- fill the ring: the first NS tiles of this warp are in flight from here on ----
-#pragma unroll
-  for (int k = 0; k < C::NS; ++k) {
-    const int b = __shfl_sync(kFull, my_b, k);
-    if (lane == 0 && k < my_blocks) issue(k, b);
-  }
-
-  // ---- per-block scales / zero points: their latency overlaps the copies in flight ----
-  float my_ks = 0.f, my_vs = 0.f, my_zp = 0.f;
-  if (lane < my_blocks) {
-    const size_t meta = (size_t)my_b * p.num_kv_heads + g;
-    if constexpr (KT != PKV_FP16) my_ks = p.k_scale[meta];
-    if constexpr (VT != PKV_FP16) my_vs = p.v_scale[meta];
-    if constexpr (VT == PKV_INT4_ASYM) my_zp = (float)p.v_zp[meta];
-  }
-
-  float m_run[GT], l_run[GT];
-  float2 acc[GT][8];  // this lane's 16 dims, as pairs
-#pragma unroll
-  for (int hh = 0; hh < GT; ++hh) {
-    m_run[hh] = kNegBig;
-    l_run[hh] = 0.f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[hh][j] = make_float2(0.f, 0.f);
-  }
+  long long pos = start, iss = start;
+  // issue every position below min(pos + NS, end) whose window is known (cur or nxt); a stage
+  // is reused only after the position NS before it has been consumed
+  auto issue_ahead = [&]() {
+    const long long lim = min(pos + C::NS, end);
+    while (iss < lim) {
+      int b, g;
+      if (iss < cur.p0 + cur.n) {
+        b = __shfl_sync(kFull, rc.b, (int)(iss - cur.p0));
+        g = (cur.hg * GT) / p.group;
+      } else if (nxt.n > 0 && iss < nxt.p0 + nxt.n) {
+        if (!rn.meta) load_meta(nxt, rn);
+        b = __shfl_sync(kFull, rn.b, (int)(iss - nxt.p0));
+        g = (nxt.hg * GT) / p.group;
+      } else {
+        break;
+      }
+      if (lane == 0) issue((int)((iss - start) % C::NS), b, g);
+      ++iss;
+    }
+  };
 
   bool aborted = false;
-  int k_stop = my_blocks;  // first block not consumed (differs from my_blocks after a timeout)
-  for (int k = 0; k < my_blocks; ++k) {
-    const int st = k % C::NS;
-    const uint32_t parity = (uint32_t)((k / C::NS) & 1);
-    const bool ok = __all_sync(kFull, mbar_wait_bounded(&my_bars[st], parity));
-    if (!ok) {
+  while (pos < end) {
+    if (pos == cur.p0 + cur.n) {  // step into the next window
+      const bool new_unit = (nxt.s != cur.s) || (nxt.hg != cur.hg);
+      cur = nxt;
+      rc = rn;
+      if (!rc.meta) load_meta(cur, rc);
+      nxt = next_win(cur);
+      load_ids(nxt, rn);
+      if (new_unit) {
+        begin_unit(cur);
+        seg_j0 = cur.j0;
+      }
+    }
+    issue_ahead();
+    const long long k_rel = pos - start;
+    const int st = (int)(k_rel % C::NS);
+    const uint32_t parity = (uint32_t)((k_rel / C::NS) & 1);
+    if (!__all_sync(kFull, mbar_wait_bounded(&my_bars[st], parity))) {
       if (lane == 0) record_error(p.dev_error, PKV_DEVERR_TIMEOUT);
       aborted = true;
-      k_stop = k;
       break;
     }
-    const float ks = __shfl_sync(kFull, my_ks, k) * p.scale_log2;  // per-block K scale, log2 domain
-    const float vs = __shfl_sync(kFull, my_vs, k);
-    const float nzb = -(kMagic + __shfl_sync(kFull, my_zp, k));
+
+    // ---- one block: q . k, online softmax, p . v ----
+    const int kw_i = (int)(pos - cur.p0);
+    const float ks = __shfl_sync(kFull, rc.ks, kw_i) * p.scale_log2;  // per-block K scale, log2 domain
+    const float vs = __shfl_sync(kFull, rc.vs, kw_i);
+    const float nzb = -(kMagic + __shfl_sync(kFull, rc.zp, kw_i));
     const float2 neg_zp_bias = make_float2(nzb, nzb);
-    const bool valid = __shfl_sync(kFull, my_valid ? 1 : 0, k) != 0;
-    const int tok0 = (blk_begin + warp + C::NW * k) * BS;
+    const bool valid = __shfl_sync(kFull, rc.valid ? 1 : 0, kw_i) != 0;
+    const int tok0 = (cur.j0 + kw_i) * BS;
     const uint8_t* kt = my_stages + (size_t)st * C::STAGE;
     const uint8_t* vt = kt + C::K_TILE;
 
-    // q . k for this lane's rows and dims, reduced over the CH lanes of a row
     float z[C::TPL][GT];
 #pragma unroll
     for (int i = 0; i < C::TPL; ++i) {
       const int row = tg + C::TG * i;
       const uint8_t* krow = kt + row * C::K_ROW + c * (C::K_ROW / C::CH);
       if constexpr (KT == PKV_INT8_SYM) {
-        const uint4 w = *reinterpret_cast<const uint4*>(krow);
-        const int kw[4] = {(int)w.x, (int)w.y, (int)w.z, (int)w.w};
+        const uint4 wv = *reinterpret_cast<const uint4*>(krow);
+        const int kw[4] = {(int)wv.x, (int)wv.y, (int)wv.z, (int)wv.w};
 #pragma unroll
         for (int hh = 0; hh < GT; ++hh) {
           int acc_p[3];
@@ -289,7 +436,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS)
         }
       } else {
         float2 kf[8];
-        load_k16<KT>(krow, kf);
+        load_h16(krow, kf);
 #pragma unroll
         for (int hh = 0; hh < GT; ++hh) {
           float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
@@ -309,17 +456,16 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS)
 #pragma unroll
         for (int off = 1; off < C::CH; off <<= 1) z[i][hh] += __shfl_xor_sync(kFull, z[i][hh], off);
 
-    // scale, mask, online softmax update (log2 domain)
     float pv[C::TPL][GT];
 #pragma unroll
     for (int hh = 0; hh < GT; ++hh) {
+      const float zscale = (KT == PKV_FP16) ? p.scale_log2 : ks * qinv[hh];
       float mloc = -INFINITY;
 #pragma unroll
-      const float zscale = (KT == PKV_FP16) ? p.scale_log2 : ks * qinv[hh];
       for (int i = 0; i < C::TPL; ++i) {
         const int t = tok0 + tg + C::TG * i;
         float zz = z[i][hh] * zscale;
-        zz = (valid && t < t_end) ? zz : -INFINITY;
+        zz = (valid && t < cur.L) ? zz : -INFINITY;
         z[i][hh] = zz;
         mloc = fmaxf(mloc, zz);
       }
@@ -344,8 +490,6 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS)
       }
       l_run[hh] += lsum;
     }
-
-    // p . v_hat for this lane's rows and dims
 #pragma unroll
     for (int i = 0; i < C::TPL; ++i) {
       const int row = tg + C::TG * i;
@@ -358,117 +502,105 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS)
         for (int j = 0; j < 8; ++j) acc[hh][j] = __ffma2_rn(pv2, vf[j], acc[hh][j]);
       }
     }
+    __syncwarp();  // the stage's reads are complete (their values were consumed above)
+    ++pos;
 
-    // stage st is free again: refill it with block k + NS
-    __syncwarp();
-    const int kn = k + C::NS;
-    const int bn = __shfl_sync(kFull, my_b, kn & 31);
-    // (the warp's reads of this stage have completed: their values were consumed above)
-    if (lane == 0 && kn < my_blocks) issue(st, bn);
+    // ---- end of a segment: the unit's last block, or the end of this warp's range ----
+    const int j_end = cur.j0 + kw_i + 1;
+    if (j_end == cur.nblk || pos == end) {
+#pragma unroll
+      for (int hh = 0; hh < GT; ++hh) {
+#pragma unroll
+        for (int off = C::CH; off < 32; off <<= 1) l_run[hh] += __shfl_xor_sync(kFull, l_run[hh], off);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+#pragma unroll
+          for (int off = C::CH; off < 32; off <<= 1) {
+            acc[hh][j].x += __shfl_xor_sync(kFull, acc[hh][j].x, off);
+            acc[hh][j].y += __shfl_xor_sync(kFull, acc[hh][j].y, off);
+          }
+      }
+      const long long u = (long long)cur.s * HG + cur.hg;
+      if (seg_j0 == 0 && j_end == cur.nblk) {
+        // the whole unit was processed by this warp: write the output
+        if (tg == 0) {
+#pragma unroll
+          for (int hh = 0; hh < GT; ++hh) {
+            const float inv = l_run[hh] > 0.f ? 1.f / l_run[hh] : 0.f;
+            __half2* o = reinterpret_cast<__half2*>(
+                p.out + ((size_t)cur.s * p.num_q_heads + (size_t)cur.hg * GT + hh) * D + c * 16);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) o[j] = __floats2half2_rn(acc[hh][j].x * inv, acc[hh][j].y * inv);
+          }
+        }
+      } else {
+        // one segment of a split unit: publish the partial; the last warp to finish merges
+        const long long slot = u + w;
+        if (tg == 0) {
+#pragma unroll
+          for (int hh = 0; hh < GT; ++hh) {
+            float4* dst = reinterpret_cast<float4*>(p.ws_acc + ((size_t)slot * GT + hh) * D + c * 16);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              dst[j] = make_float4(acc[hh][2 * j].x, acc[hh][2 * j].y, acc[hh][2 * j + 1].x, acc[hh][2 * j + 1].y);
+          }
+        }
+        if (lane == 0) {
+#pragma unroll
+          for (int hh = 0; hh < GT; ++hh) {
+            p.ws_ml[((size_t)slot * GT + hh) * 2 + 0] = m_run[hh];
+            p.ws_ml[((size_t)slot * GT + hh) * 2 + 1] = l_run[hh];
+          }
+        }
+        const long long unit_p0 = cur.seq_p0 + (long long)cur.hg * cur.nblk;
+        const int w_first = owner_of(unit_p0, T, We);
+        const int w_last = owner_of(unit_p0 + cur.nblk - 1, T, We);
+        const uint32_t n_seg = (uint32_t)(w_last - w_first + 1);
+        __syncwarp();
+        uint32_t ticket = 0;
+        if (lane == 0) {
+          __threadfence();  // release: this warp's partial is visible device-wide first
+          ticket = atomicInc(&p.ws_count[u], n_seg - 1);
+          __threadfence();  // acquire side for the merge below
+        }
+        ticket = __shfl_sync(kFull, ticket, 0);
+        if (ticket == n_seg - 1) {
+          for (int o = lane; o < GT * D; o += 32) {
+            const int hh = o / D, d = o % D;
+            float M = kNegBig;
+            for (int wi = w_first; wi <= w_last; ++wi)
+              M = fmaxf(M, __ldcg(&p.ws_ml[((size_t)(u + wi) * GT + hh) * 2]));
+            float Ls = 0.f, A = 0.f;
+            for (int wi = w_first; wi <= w_last; ++wi) {
+              const size_t sl = (size_t)(u + wi) * GT + hh;
+              const float e = ex2(__ldcg(&p.ws_ml[sl * 2]) - M);
+              Ls = fmaf(__ldcg(&p.ws_ml[sl * 2 + 1]), e, Ls);
+              A = fmaf(__ldcg(&p.ws_acc[sl * D + d]), e, A);
+            }
+            p.out[((size_t)cur.s * p.num_q_heads + (size_t)cur.hg * GT + hh) * D + d] =
+                __float2half_rn(Ls > 0.f ? A / Ls : 0.f);
+          }
+        }
+      }
+#pragma unroll
+      for (int hh = 0; hh < GT; ++hh) {
+        m_run[hh] = kNegBig;
+        l_run[hh] = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[hh][j] = make_float2(0.f, 0.f);
+      }
+      seg_j0 = j_end;  // (a new unit restarts it at its first block)
+    }
   }
 
-  if (aborted) {
-    // A copy never completed (the output of this CTA is unspecified; dev_error says so).
+  if (aborted && lane == 0) {
+    // A copy never completed (outputs touched by this warp are unspecified; dev_error says so).
     // Wait, again bounded, for the copies this warp issued and did not consume, so that no bulk
-    // copy is still writing this CTA's shared memory when it exits; then contribute nothing.
-    if (lane == 0) {
-      for (int k = k_stop; k < min(k_stop + C::NS, my_blocks); ++k)
-        (void)mbar_wait_bounded(&my_bars[k % C::NS], (uint32_t)((k / C::NS) & 1));
+    // copy is still writing this CTA's shared memory when it exits.
+    for (long long k = pos; k < iss; ++k) {
+      const long long r = k - start;
+      (void)mbar_wait_bounded(&my_bars[(int)(r % C::NS)], (uint32_t)((r / C::NS) & 1));
     }
-#pragma unroll
-    for (int hh = 0; hh < GT; ++hh) {
-      m_run[hh] = kNegBig;
-      l_run[hh] = 0.f;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) acc[hh][j] = make_float2(0.f, 0.f);
-    }
-  }
-
-  // ---- reduce the warp's state over its token-row groups ----
-#pragma unroll
-  for (int hh = 0; hh < GT; ++hh) {
-#pragma unroll
-    for (int off = C::CH; off < 32; off <<= 1) l_run[hh] += __shfl_xor_sync(kFull, l_run[hh], off);
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-#pragma unroll
-      for (int off = C::CH; off < 32; off <<= 1) {
-        acc[hh][j].x += __shfl_xor_sync(kFull, acc[hh][j].x, off);
-        acc[hh][j].y += __shfl_xor_sync(kFull, acc[hh][j].y, off);
-      }
-  }
-  if (tg == 0) {
-#pragma unroll
-    for (int hh = 0; hh < GT; ++hh) {
-      float4* dst = reinterpret_cast<float4*>(merge_acc + ((size_t)warp * GT + hh) * D + c * 16);
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        dst[j] = make_float4(acc[hh][2 * j].x, acc[hh][2 * j].y, acc[hh][2 * j + 1].x, acc[hh][2 * j + 1].y);
-    }
-  }
-  if (lane == 0) {
-#pragma unroll
-    for (int hh = 0; hh < GT; ++hh) {
-      merge_ml[(warp * GT + hh) * 2 + 0] = m_run[hh];
-      merge_ml[(warp * GT + hh) * 2 + 1] = l_run[hh];
-    }
-  }
-  __syncthreads();
-
-  // ---- merge the warps; write the final output or this partition's partial ----
-  const bool single = num_parts <= 1;
-  for (int o = threadIdx.x; o < GT * D; o += C::THREADS) {
-    const int hh = o / D, d = o % D;
-    float M = kNegBig;
-#pragma unroll
-    for (int w = 0; w < C::NW; ++w) M = fmaxf(M, merge_ml[(w * GT + hh) * 2]);
-    float Lsum = 0.f, A = 0.f;
-#pragma unroll
-    for (int w = 0; w < C::NW; ++w) {
-      const float e = ex2(merge_ml[(w * GT + hh) * 2] - M);
-      Lsum = fmaf(merge_ml[(w * GT + hh) * 2 + 1], e, Lsum);
-      A = fmaf(merge_acc[((size_t)w * GT + hh) * D + d], e, A);
-    }
-    const int h = h0 + hh;
-    if (single) {
-      p.out[((size_t)s * p.num_q_heads + h) * D + d] = __float2half_rn(Lsum > 0.f ? A / Lsum : 0.f);
-    } else {
-      const size_t idx = ((size_t)s * p.num_q_heads + h) * p.max_partitions + part;
-      p.ws_acc[idx * D + d] = A;
-      if (d == 0) {
-        p.ws_ml[idx * 2 + 0] = M;
-        p.ws_ml[idx * 2 + 1] = Lsum;
-      }
-    }
-  }
-  if (single) return;
-
-  // ---- split-K merge by the last partition CTA of this (sequence, head group) to finish ----
-  // Every partition CTA publishes its partial, then bumps a counter with atomicInc, which wraps
-  // back to 0 when the last of num_parts arrivals takes it: the counter is left at zero for the
-  // next call without a reset. The CTA that sees num_parts - 1 merges
-  //   out = sum_p 2^(m_p - M) acc_p / sum_p 2^(m_p - M) l_p.
-  __shared__ uint32_t s_ticket;
-  __syncthreads();  // every partial write of this CTA precedes thread 0's fence (CTA scope)
-  if (threadIdx.x == 0) {
-    __threadfence();  // release: the CTA's partial is visible device-wide before the counter moves
-    s_ticket = atomicInc(&p.ws_count[(size_t)s * gridDim.x + blockIdx.x], (uint32_t)(num_parts - 1));
-    __threadfence();  // acquire side for the merging CTA
-  }
-  __syncthreads();
-  if (s_ticket != (uint32_t)(num_parts - 1)) return;
-  for (int o = threadIdx.x; o < GT * D; o += C::THREADS) {
-    const int hh = o / D, d = o % D;
-    const size_t base = ((size_t)s * p.num_q_heads + h0 + hh) * p.max_partitions;
-    float M = kNegBig;
-    for (int i = 0; i < num_parts; ++i) M = fmaxf(M, __ldcg(&p.ws_ml[(base + i) * 2]));
-    float Lsum = 0.f, A = 0.f;
-    for (int i = 0; i < num_parts; ++i) {
-      const float e = ex2(__ldcg(&p.ws_ml[(base + i) * 2]) - M);
-      Lsum = fmaf(__ldcg(&p.ws_ml[(base + i) * 2 + 1]), e, Lsum);
-      A = fmaf(__ldcg(&p.ws_acc[(base + i) * D + d]), e, A);
-    }
-    p.out[((size_t)s * p.num_q_heads + h0 + hh) * D + d] = __float2half_rn(Lsum > 0.f ? A / Lsum : 0.f);
   }
 }
 
@@ -486,67 +618,71 @@ cudaError_t launch_one(const DecodeParams& p, const DecodeShape& sh, cudaStream_
     if (e != cudaSuccess) return e;
     configured |= bit;
   }
-  dim3 grid(p.num_q_heads / GT, p.max_partitions, sh.num_seqs);
-  kern<<<grid, C::THREADS, C::SMEM, stream>>>(p);
+  kern<<<sh.grid_ctas, C::THREADS, C::SMEM, stream>>>(p);
   return cudaGetLastError();
 }
 
-template <int KT, int VT, int BS, int D>
-cudaError_t dispatch_gt(const DecodeParams& p, const DecodeShape& sh, cudaStream_t stream) {
-  switch (sh.heads_per_cta) {
-    case 1: return launch_one<KT, VT, BS, D, 1>(p, sh, stream);
-    case 2: return launch_one<KT, VT, BS, D, 2>(p, sh, stream);
-    case 4: return launch_one<KT, VT, BS, D, 4>(p, sh, stream);
-    default: return cudaErrorInvalidValue;
-  }
+template <int KT, int VT, int BS, int D, int GT>
+bool info_one(DecodeKernelInfo* info) {
+  using C = Cfg<KT, VT, BS, D, GT>;
+  info->warps_per_cta = C::NW;
+  info->ctas_per_sm = C::CTAS_PER_SM;
+  info->smem_bytes = C::SMEM;
+  info->stages = C::NS;
+  return true;
 }
 
-template <int KT, int VT, int BS>
-cudaError_t dispatch_d(const DecodeParams& p, const DecodeShape& sh, cudaStream_t stream) {
-  switch (sh.head_dim) {
-    case 64: return dispatch_gt<KT, VT, BS, 64>(p, sh, stream);
-    case 128: return dispatch_gt<KT, VT, BS, 128>(p, sh, stream);
-    case 256: return dispatch_gt<KT, VT, BS, 256>(p, sh, stream);
-    default: return cudaErrorInvalidValue;
+// FN<KT, VT, BS, D, GT>(args...) for the instantiation matching `sh`
+#define PKV_DISPATCH_GT(KT, VT, BS, D, FN, ...)       \
+  switch (sh.heads_per_warp) {                        \
+    case 1: return FN<KT, VT, BS, D, 1>(__VA_ARGS__); \
+    case 2: return FN<KT, VT, BS, D, 2>(__VA_ARGS__); \
+    case 4: return FN<KT, VT, BS, D, 4>(__VA_ARGS__); \
+    default: break;                                   \
   }
-}
-
-template <int KT, int VT>
-cudaError_t dispatch_bs(const DecodeParams& p, const DecodeShape& sh, cudaStream_t stream) {
-  switch (sh.block_size) {
-    case 16: return dispatch_d<KT, VT, 16>(p, sh, stream);
-    case 32: return dispatch_d<KT, VT, 32>(p, sh, stream);
-    default: return cudaErrorInvalidValue;
+#define PKV_DISPATCH_D(KT, VT, BS, FN, ...)                   \
+  switch (sh.head_dim) {                                      \
+    case 64: PKV_DISPATCH_GT(KT, VT, BS, 64, FN, __VA_ARGS__) break;   \
+    case 128: PKV_DISPATCH_GT(KT, VT, BS, 128, FN, __VA_ARGS__) break; \
+    case 256: PKV_DISPATCH_GT(KT, VT, BS, 256, FN, __VA_ARGS__) break; \
+    default: break;                                           \
   }
-}
+#define PKV_DISPATCH_BS(KT, VT, FN, ...)                      \
+  switch (sh.block_size) {                                    \
+    case 16: PKV_DISPATCH_D(KT, VT, 16, FN, __VA_ARGS__) break; \
+    case 32: PKV_DISPATCH_D(KT, VT, 32, FN, __VA_ARGS__) break; \
+    default: break;                                           \
+  }
+#define PKV_DISPATCH(FN, ...)                                                \
+  if (sh.k_dtype == PKV_INT8_SYM && sh.v_dtype == PKV_INT8_SYM) {            \
+    PKV_DISPATCH_BS(PKV_INT8_SYM, PKV_INT8_SYM, FN, __VA_ARGS__)             \
+  } else if (sh.k_dtype == PKV_INT8_SYM && sh.v_dtype == PKV_INT4_ASYM) {    \
+    PKV_DISPATCH_BS(PKV_INT8_SYM, PKV_INT4_ASYM, FN, __VA_ARGS__)            \
+  } else if (sh.k_dtype == PKV_FP16 && sh.v_dtype == PKV_FP16) {             \
+    PKV_DISPATCH_BS(PKV_FP16, PKV_FP16, FN, __VA_ARGS__)                     \
+  }
 
 }  // namespace
 
-int32_t decode_heads_per_cta(int32_t group) {
+int32_t decode_heads_per_warp(int32_t group) {
   if (group % 4 == 0) return 4;
   if (group % 2 == 0) return 2;
   return 1;
 }
 
-int32_t decode_max_partition_tokens(int32_t block_size) {
-  return 32 * 4 * block_size;  // 32 blocks per warp (one id per lane) x 4 warps
-}
-
 bool decode_supported(int32_t k_dtype, int32_t v_dtype, int32_t block_size, int32_t head_dim) {
   const bool dt = (k_dtype == PKV_INT8_SYM && (v_dtype == PKV_INT8_SYM || v_dtype == PKV_INT4_ASYM)) ||
                   (k_dtype == PKV_FP16 && v_dtype == PKV_FP16);
-  // an FP16 cache with head_dim 256 and 32-token blocks needs 32 KiB per stage: two stages for
-  // each of four warps exceed the 227 KiB of shared memory a CTA can have
-  if (k_dtype == PKV_FP16 && head_dim == 256 && block_size == 32) return false;
   return dt && (block_size == 16 || block_size == 32) && (head_dim == 64 || head_dim == 128 || head_dim == 256);
 }
 
+bool decode_kernel_info(const DecodeShape& sh, DecodeKernelInfo* info) {
+  PKV_DISPATCH(info_one, info)
+  return false;
+}
+
 cudaError_t launch_decode(const DecodeParams& p, const DecodeShape& sh, cudaStream_t stream) {
-  if (sh.k_dtype == PKV_INT8_SYM && sh.v_dtype == PKV_INT8_SYM)
-    return dispatch_bs<PKV_INT8_SYM, PKV_INT8_SYM>(p, sh, stream);
-  if (sh.k_dtype == PKV_INT8_SYM && sh.v_dtype == PKV_INT4_ASYM)
-    return dispatch_bs<PKV_INT8_SYM, PKV_INT4_ASYM>(p, sh, stream);
-  if (sh.k_dtype == PKV_FP16 && sh.v_dtype == PKV_FP16) return dispatch_bs<PKV_FP16, PKV_FP16>(p, sh, stream);
+  PKV_DISPATCH(launch_one, p, sh, stream)
   return cudaErrorInvalidValue;
 }
 

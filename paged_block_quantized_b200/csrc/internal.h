@@ -20,33 +20,38 @@ struct DecodeParams {
   __half* out;
   const int32_t* block_tables;
   const int32_t* context_lens;
-  uint32_t* ws_count;  // [S][Hq / heads_per_cta] arrival counters (zero between calls)
-  float* ws_ml;        // [S][Hq][max_partitions][2] running max (log2 domain) and sum
-  float* ws_acc;       // [S][Hq][max_partitions][D] un-normalised accumulators
+  uint32_t* ws_count;  // [S * HG] tickets of split units (zero between calls)
+  float* ws_ml;        // [(S*HG + W) * GT][2] partial running max (log2 domain) and sum
+  float* ws_acc;       // [(S*HG + W) * GT][D] partial un-normalised accumulators
   int32_t* dev_error;
+  int32_t num_seqs;
   int32_t num_blocks;
   int32_t num_kv_heads;
   int32_t num_q_heads;
   int32_t group;  // num_q_heads / num_kv_heads
   int32_t max_blocks_per_seq;
   int32_t max_context_len;
-  int32_t partition_tokens;
-  int32_t max_partitions;
   float scale_log2;  // softmax_scale * log2(e)
 };
 
 struct DecodeShape {
   int32_t k_dtype, v_dtype, block_size, head_dim;
-  int32_t heads_per_cta;  // query heads handled by one CTA (divides group)
-  int32_t num_seqs;
+  int32_t heads_per_warp;  // query heads of one KV group handled together (divides group)
+  int32_t grid_ctas;       // persistent grid size
 };
 
-// Query heads per CTA for a group size (largest of 4, 2, 1 that divides it).
-int32_t decode_heads_per_cta(int32_t group);
-// Largest partition the decode kernel accepts for this block size (a warp keeps the ids of its
-// blocks in registers, one per lane).
-int32_t decode_max_partition_tokens(int32_t block_size);
+struct DecodeKernelInfo {
+  int32_t warps_per_cta;
+  int32_t ctas_per_sm;  // resident CTAs per SM the kernel is built for
+  int32_t smem_bytes;
+  int32_t stages;       // copy-ring depth per warp
+};
+
+// Query heads handled together by one warp (largest of 4, 2, 1 that divides the group).
+int32_t decode_heads_per_warp(int32_t group);
 bool decode_supported(int32_t k_dtype, int32_t v_dtype, int32_t block_size, int32_t head_dim);
+// Static launch facts of the kernel instantiation for `sh` (no device needed); false if none.
+bool decode_kernel_info(const DecodeShape& sh, DecodeKernelInfo* info);
 
 cudaError_t launch_decode(const DecodeParams& p, const DecodeShape& sh, cudaStream_t stream);
 

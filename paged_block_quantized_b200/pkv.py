@@ -141,12 +141,12 @@ def pkv_decode_workspace_size(desc, num_seqs, num_q_heads, max_context_len, part
 
 
 def pkv_decode_partitioning(desc, num_seqs, num_q_heads, max_context_len, partition_tokens=0):
-    """(tokens per partition, partitions of the longest sequence) the decode will use."""
-    pt, n = _I32(0), _I32(0)
+    """(worker warps, persistent CTAs) the decode will use on the current device."""
+    nw, nc = _I32(0), _I32(0)
     st = _partitioning(ctypes.byref(desc), int(num_seqs), int(num_q_heads), int(max_context_len),
-                       int(partition_tokens), ctypes.byref(pt), ctypes.byref(n))
+                       int(partition_tokens), ctypes.byref(nw), ctypes.byref(nc))
     _check(st, "pkv_decode_partitioning", True)
-    return int(pt.value), int(n.value)
+    return int(nw.value), int(nc.value)
 
 
 def pkv_paged_attention_decode(desc, out, q, num_seqs, num_q_heads, block_tables, max_blocks_per_seq,

@@ -32,7 +32,7 @@ class DeviceStep:
         self.step_slots = torch.from_numpy(w.step_slots()).to(dev)
         self.cow = torch.from_numpy(np.ascontiguousarray(w.cow_pairs)).to(dev)
         self.partition_tokens = w.partition_tokens if partition_tokens is None else partition_tokens
-        self.effective_partition_tokens, self.num_partitions = pkv.pkv_decode_partitioning(
+        self.num_workers, self.num_ctas = pkv.pkv_decode_partitioning(
             self.pool.desc, w.num_seqs, w.num_q_heads, w.max_context_len, self.partition_tokens)
         self.ws_bytes = pkv.pkv_decode_workspace_size(self.pool.desc, w.num_seqs, w.num_q_heads,
                                                       w.max_context_len, self.partition_tokens)

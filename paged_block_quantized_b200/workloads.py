@@ -281,7 +281,7 @@ def make(name: str, seed: int = 0, **over) -> Workload:
         S = over.get("num_seqs", 8)
         p = dict(num_seqs=S, num_q_heads=32, num_kv_heads=32, head_dim=128, block_size=32,
                  num_blocks=None, k_dtype=INT8_SYM, v_dtype=INT4_ASYM, outliers=False,
-                 partition_tokens=512, context_lens=rng.integers(8192, 32769, size=S))
+                 partition_tokens=0, context_lens=rng.integers(8192, 32769, size=S))
         desc = "long context: 8 seqs, L~U{8192..32768}, 32 heads, D 128, bs 32, K INT8 / V INT4, 512-token partitions"
     elif name == "gqa_prefix":
         S = over.get("num_seqs", 64)

@@ -72,6 +72,7 @@ def test_descriptor_validation(pkv, bad, code):
 
 
 def test_call_validation(pkv):
+    """Every call here is rejected on the host before any launch (the pointers are fake)."""
     d = desc(pkv)
     E = pkv.PKV_ERR_INVALID_ARG
     assert pkv.pkv_store_quantized(d, 0x6000, 0x7000, 0x8000, -1, stream=0, raise_on_error=False) == E
@@ -80,39 +81,57 @@ def test_call_validation(pkv):
     assert pkv.pkv_store_quantized(d, 0x6000, 0x7000, 0x8000, 0, stream=0, raise_on_error=False) == pkv.PKV_OK
     assert pkv.pkv_copy_blocks(d, 0x6000, -2, stream=0, raise_on_error=False) == E
     assert pkv.pkv_copy_blocks(d, 0x6000, 0, stream=0, raise_on_error=False) == pkv.PKV_OK
+    big = 1 << 40  # a (fake) workspace large enough for any size, so that the intended check fires
     dec = lambda **kw: pkv.pkv_paged_attention_decode(
         d, kw.get("out", 0x9000), kw.get("q", 0xA000), kw.get("S", 2), kw.get("Hq", 4), 0xB000,
         kw.get("mbps", 4), 0xC000, kw.get("max_len", 64), kw.get("scale", 0.125), kw.get("pt", 0),
-        kw.get("ws", None), kw.get("ws_bytes", 0), stream=0, raise_on_error=False)
+        kw.get("ws", 0xD000), kw.get("ws_bytes", big), stream=0, raise_on_error=False)
     assert dec(Hq=3) == E                        # not a multiple of the KV heads
     assert dec(q=0xA004) == E                    # misaligned
+    assert dec(out=None) == E
     assert dec(mbps=0) == E
     assert dec(pt=24) == E                       # not a multiple of the block size
-    assert dec(pt=16 * 128 + 16) == pkv.PKV_ERR_UNSUPPORTED
+    assert dec(pt=-16) == E
     assert dec(scale=float("nan")) == E
     assert dec(max_len=-1) == E
+    assert dec(S=-1) == E
     assert dec(S=0) == pkv.PKV_OK                # nothing to do
-    assert dec(max_len=4096, pt=64) == E         # needs a workspace
+    assert dec(ws=None) == E                     # a workspace is required
+    assert dec(ws_bytes=16) == E                 # too small
+    assert dec(ws=0xD004) == E                   # misaligned
     assert pkv.pkv_paged_attention_decode(desc(pkv, k_dtype=pkv.PKV_FP16), 0x9000, 0xA000, 2, 4, 0xB000, 4,
-                                          0xC000, 64, 0.1, stream=0, raise_on_error=False) == pkv.PKV_ERR_UNSUPPORTED
+                                          0xC000, 64, 0.1, 0, 0xD000, big, stream=0,
+                                          raise_on_error=False) == pkv.PKV_ERR_UNSUPPORTED
 
 
 def test_partitioning(pkv):
     d = desc(pkv)
-    assert pkv.pkv_decode_partitioning(d, 2, 4, 1000, 128) == (128, 8)
-    assert pkv.pkv_decode_partitioning(d, 2, 4, 0, 64) == (64, 1)
-    pt, n = pkv.pkv_decode_partitioning(d, 2, 4, 5000, 0)
-    assert pt % 16 == 0 and 64 <= pt <= 2048 and n == -(-5000 // pt)
+    workers, ctas = pkv.pkv_decode_partitioning(d, 2, 4, 1000, 0)
+    assert ctas > 0 and workers % ctas == 0 and workers // ctas in (2, 4)
+    # with partition_tokens: about one worker per partition_tokens tokens of the largest work
+    # (2 seqs x 2 head groups x 63 blocks = 252 blocks, 8 blocks each -> 32 workers)
+    w2, c2 = pkv.pkv_decode_partitioning(d, 2, 4, 1000, 128)
+    assert w2 == 32 and c2 == 32 // (workers // ctas)
+    w3, _ = pkv.pkv_decode_partitioning(d, 2, 4, 1000, 1 << 20)   # never fewer than one CTA of warps
+    assert w3 == workers // ctas
+    w4, _ = pkv.pkv_decode_partitioning(d, 2, 4, 1000, 16)        # one block each: 252 workers
+    assert w4 == 252
+    w5, _ = pkv.pkv_decode_partitioning(d, 200, 4, 1000, 16)      # never more than fit on the device
+    assert w5 == pkv.pkv_decode_partitioning(d, 200, 4, 1000, 0)[0]
 
 
 def test_workspace_size(pkv):
-    d = desc(pkv)
-    # 256 bytes of arrival counters (one per sequence and CTA head group), then the partials
-    assert pkv.pkv_decode_workspace_size(d, 2, 4, 64, 64) == 0          # one partition: nothing
-    assert pkv.pkv_decode_workspace_size(d, 2, 4, 65, 64) == 256 + 2 * 4 * 2 * (64 + 2) * 4
-    assert pkv.pkv_decode_workspace_size(d, 3, 4, 1000, 128) == 256 + 3 * 4 * 8 * (64 + 2) * 4
-    # partials only: never proportional to the cache (no dequantized copy of K/V)
-    big = pkv.pkv_decode_workspace_size(d, 8, 32, 32768, 512)
-    assert big == 256 + 8 * 32 * 64 * 66 * 4
-    auto = pkv.pkv_decode_workspace_size(d, 8, 32, 32768, 0)
-    assert (auto - 256) % ((64 + 2) * 4 * 8 * 32) == 0
+    """Tickets per (sequence, head group), then one partial slot per (sequence, head group) and per
+    worker: sizes follow the batch shape and the worker count, never the cache size."""
+    d = desc(pkv)  # D 64, 2 KV heads; 4 query heads -> groups of 2 handled together
+    def expect(S, Hq, workers, gt=2, D=64):
+        units = S * (Hq // gt)
+        slots = units + workers
+        pad = lambda x: (x + 255) // 256 * 256
+        return pad(units * 4) + pad(slots * gt * 2 * 4) + slots * gt * D * 4
+    for S, L, pt in ((2, 64, 0), (3, 1000, 128), (8, 32768, 0), (1, 16, 0)):
+        workers, _ = pkv.pkv_decode_partitioning(d, S, 4, L, pt)
+        assert pkv.pkv_decode_workspace_size(d, S, 4, L, pt) == expect(S, 4, workers)
+    assert pkv.pkv_decode_workspace_size(d, 0, 4, 64, 0) == 0
+    # independent of the context length for a fixed worker count (no copy of the cache)
+    assert pkv.pkv_decode_workspace_size(d, 8, 4, 64, 0) == pkv.pkv_decode_workspace_size(d, 8, 4, 32768, 0)

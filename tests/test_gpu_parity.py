@@ -117,13 +117,14 @@ def test_partition_boundaries(pt):
     check(w, partition_tokens=pt)
 
 
-def test_max_partition_and_long_sequence():
-    from paged_block_quantized_b200 import pkv
+@pytest.mark.parametrize("pt", [0, 32768])
+def test_long_sequence_split_and_whole(pt):
+    # pt 0: every resident warp, each of the 32 heads cut across many warps (merge of many
+    # partials); pt 32768: 32 workers, one whole head each (no merge)
     w = W.make("long", seed=4, num_seqs=1, context_lens=[32768])
-    g, _ = check(w, partition_tokens=32 * 4 * 32)  # the largest partition for block size 32
-    assert g.partition_tokens == 4096
-    with pytest.raises(pkv.PkvError):
-        pkv.pkv_decode_workspace_size(g.pool.desc, 1, 32, 32768, 4096 + 32)
+    g, _ = check(w, partition_tokens=pt)
+    if pt:
+        assert g.num_workers == 32
 
 
 def test_zero_length_and_empty_batch():
