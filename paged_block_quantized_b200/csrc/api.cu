@@ -55,6 +55,10 @@ int sm_count() {
   return c;
 }
 
+// Fewest blocks a worker warp gets on average by default: smaller batches use fewer warps
+// rather than cutting every (sequence, head group) into pieces that each need a merge.
+constexpr int64_t kMinBlocksPerWorker = 4;
+
 struct DecodeGeometry {
   DecodeShape shape;
   int32_t workers;          // worker warps of the persistent grid
@@ -80,16 +84,15 @@ pkv_status decode_geometry(const pkv_cache_desc* d, int32_t num_seqs, int32_t nu
   DecodeKernelInfo info;
   if (!decode_kernel_info(sh, &info)) return PKV_ERR_UNSUPPORTED;
   const int64_t max_workers = (int64_t)sm_count() * info.ctas_per_sm * info.warps_per_cta;
-  int64_t workers = max_workers;
-  if (partition_tokens > 0) {
-    const int64_t hg = num_q_heads / sh.heads_per_warp;
-    const int64_t blocks = (int64_t)num_seqs * hg * ((max_context_len + d->block_size - 1) / d->block_size);
-    const int64_t per = partition_tokens / d->block_size;
-    workers = (blocks + per - 1) / per;
-    workers = (workers + info.warps_per_cta - 1) / info.warps_per_cta * info.warps_per_cta;
-    if (workers < info.warps_per_cta) workers = info.warps_per_cta;
-    if (workers > max_workers) workers = max_workers;
-  }
+  // blocks of the largest possible batch: the real total is only known on the device
+  const int64_t hg = num_q_heads / sh.heads_per_warp;
+  const int64_t blocks = (int64_t)num_seqs * hg * ((max_context_len + d->block_size - 1) / d->block_size);
+  // blocks per worker: the requested partition, or a few blocks (one ring's worth) at least
+  const int64_t per = partition_tokens > 0 ? partition_tokens / d->block_size : kMinBlocksPerWorker;
+  int64_t workers = (blocks + per - 1) / per;
+  workers = (workers + info.warps_per_cta - 1) / info.warps_per_cta * info.warps_per_cta;
+  if (workers < info.warps_per_cta) workers = info.warps_per_cta;
+  if (workers > max_workers) workers = max_workers;
   sh.grid_ctas = (int32_t)(workers / info.warps_per_cta);
   g->workers = (int32_t)workers;
   const size_t units = (size_t)num_seqs * (num_q_heads / sh.heads_per_warp);

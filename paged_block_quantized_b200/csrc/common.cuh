@@ -17,6 +17,15 @@ __device__ __forceinline__ void record_error(int32_t* dev_error, int32_t code) {
   if (dev_error != nullptr) atomicCAS(dev_error, 0, code);
 }
 
+// atomicInc with acquire-release semantics at GPU scope: the caller's earlier writes (and those
+// of its warp, ordered before it by __syncwarp) are visible to whoever observes the new value,
+// and writes released by earlier incrementers are visible to the caller afterwards.
+__device__ __forceinline__ uint32_t atomic_inc_acq_rel_gpu(uint32_t* addr, uint32_t wrap) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.inc.u32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(wrap) : "memory");
+  return old;
+}
+
 // ---- integer code -> float conversion without I2F -------------------------------------------
 // IEEE-754 binary32 with exponent field 150 (bit pattern 0x4B000000 | m, m < 2^23) is exactly
 // 2^23 + m. Placing a biased byte in the low mantissa bits and subtracting the bias as a float

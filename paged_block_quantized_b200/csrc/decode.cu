@@ -41,6 +41,18 @@ namespace {
 constexpr uint32_t kFull = 0xffffffffu;
 constexpr float kNegBig = -1.0e30f;  // finite "minus infinity" for running maxima
 
+// Shared-memory budget of one CTA's copy rings and the CTA-per-SM caps by heads per warp
+// (overridable at build time for tuning sweeps).
+#ifndef PKV_DECODE_SMEM_TARGET
+#define PKV_DECODE_SMEM_TARGET 49152
+#endif
+#ifndef PKV_DECODE_CPS_GT1
+#define PKV_DECODE_CPS_GT1 4
+#endif
+#ifndef PKV_DECODE_MAX_STAGES
+#define PKV_DECODE_MAX_STAGES 6
+#endif
+
 template <int KT, int VT, int BS, int D, int GT>
 struct Cfg {
   static constexpr int K_ROW = (KT == PKV_FP16) ? 2 * D : D;
@@ -49,9 +61,9 @@ struct Cfg {
   static constexpr int V_TILE = BS * V_ROW;
   static constexpr int STAGE = K_TILE + V_TILE;
   static constexpr int NW = (4 * 2 * STAGE <= 200 * 1024) ? 4 : 2;  // warps per CTA
-  // about 48 KiB of stages per CTA, 2..6 stages per warp
-  static constexpr int NS_RAW = 49152 / (NW * STAGE);
-  static constexpr int NS = NS_RAW < 2 ? 2 : (NS_RAW > 6 ? 6 : NS_RAW);
+  // stages per warp from the CTA's shared-memory budget, at least 2
+  static constexpr int NS_RAW = PKV_DECODE_SMEM_TARGET / (NW * STAGE);
+  static constexpr int NS = NS_RAW < 2 ? 2 : (NS_RAW > PKV_DECODE_MAX_STAGES ? PKV_DECODE_MAX_STAGES : NS_RAW);
   static constexpr int CH = D / 16;    // lanes per token row (16 dims each)
   static constexpr int TG = 32 / CH;   // token rows a warp covers per pass
   static constexpr int TPL = BS / TG;  // token rows per lane per block
@@ -61,7 +73,7 @@ struct Cfg {
   // resident CTAs per SM: bounded by shared memory (227 KiB per SM) and by the registers a
   // thread needs for GT heads of state
   static constexpr int CPS_SMEM = (220 * 1024) / (SMEM + 1024);
-  static constexpr int CPS_CAP = (GT == 1) ? 4 : (GT == 2 ? 3 : 2);  // 128 / 170 / 255 registers
+  static constexpr int CPS_CAP = (GT == 1) ? PKV_DECODE_CPS_GT1 : (GT == 2 ? 3 : 2);  // 128 / 170 / 255 regs
   static constexpr int CTAS_PER_SM = CPS_SMEM < 1 ? 1 : (CPS_SMEM > CPS_CAP ? CPS_CAP : CPS_SMEM);
   static_assert(D % 16 == 0 && CH <= 32 && 32 % CH == 0, "head_dim");
   static_assert(BS % TG == 0, "block_size must cover the token rows of a warp pass");
@@ -111,8 +123,9 @@ __device__ __forceinline__ int owner_of(long long g, long long T, int W) {
 // block j0 + k in the per-lane registers of the window).
 struct Win {
   int s, hg, j0, n;     // sequence, head group, first block, blocks in the window (0 = none)
+  int g;                // KV head of the head group
   int L, nblk;          // clamped length of the sequence and its block count
-  long long p0;         // stream position of block j0
+  int r0;               // position of block j0 relative to the warp's first position
   long long seq_p0;     // stream position of the sequence's first block (head group 0)
 };
 
@@ -213,9 +226,11 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
     const long long o = start - cur.seq_p0;
     cur.hg = (int)(o / cur.nblk);
     cur.j0 = (int)(o % cur.nblk);
-    cur.p0 = start;
+    cur.g = (cur.hg * GT) / p.group;
+    cur.r0 = 0;
     cur.n = (int)min((long long)min(32, cur.nblk - cur.j0), end - start);
   }
+  const int n_total = (int)(end - start);  // positions of this warp
 
   // clamped length of sequence s, from the lane-held chunk when possible
   auto seq_len = [&](int s) -> int {
@@ -229,9 +244,9 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
   // the window after `a`, within [.., end); n = 0 if none
   auto next_win = [&](const Win& a) -> Win {
     Win b = a;
-    b.p0 = a.p0 + a.n;
+    b.r0 = a.r0 + a.n;
     b.n = 0;
-    if (a.n == 0 || b.p0 >= end) return b;
+    if (a.n == 0 || b.r0 >= n_total) return b;
     b.j0 = a.j0 + a.n;
     if (b.j0 >= a.nblk) {
       b.j0 = 0;
@@ -248,8 +263,9 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
         b.L = L;
         b.nblk = (L + BS - 1) / BS;
       }
+      b.g = (b.hg * GT) / p.group;
     }
-    b.n = (int)min((long long)min(32, b.nblk - b.j0), end - b.p0);
+    b.n = min(min(32, b.nblk - b.j0), n_total - b.r0);
     return b;
   };
 
@@ -265,8 +281,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
     r.b = r.valid ? r.raw : 0;
     r.ks = r.vs = r.zp = 0.f;
     if (lane < a.n) {
-      const int g = (a.hg * GT) / p.group;
-      const size_t meta = (size_t)r.b * p.num_kv_heads + g;
+      const size_t meta = (size_t)r.b * p.num_kv_heads + a.g;
       if constexpr (KT != PKV_FP16) r.ks = p.k_scale[meta];
       if constexpr (VT != PKV_FP16) r.vs = p.v_scale[meta];
       if constexpr (VT == PKV_INT4_ASYM) r.zp = (float)p.v_zp[meta];
@@ -356,31 +371,34 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
     bulk_g2s(dst + C::K_TILE, static_cast<const uint8_t*>(p.v_codes) + tile * C::V_TILE, (uint32_t)C::V_TILE,
              &my_bars[st]);
   };
-  long long pos = start, iss = start;
-  // issue every position below min(pos + NS, end) whose window is known (cur or nxt); a stage
-  // is reused only after the position NS before it has been consumed
+  // positions relative to `start`: consumed (cpos) and issued (ipos); stage / parity of each
+  int cpos = 0, ipos = 0, cst = 0, ist = 0;
+  uint32_t cpar = 0;
+  // issue every position below min(cpos + NS, n_total) whose window is known (cur or nxt); a
+  // stage is reused only after the position NS before it has been consumed
   auto issue_ahead = [&]() {
-    const long long lim = min(pos + C::NS, end);
-    while (iss < lim) {
+    const int lim = min(cpos + C::NS, n_total);
+    while (ipos < lim) {
       int b, g;
-      if (iss < cur.p0 + cur.n) {
-        b = __shfl_sync(kFull, rc.b, (int)(iss - cur.p0));
-        g = (cur.hg * GT) / p.group;
-      } else if (nxt.n > 0 && iss < nxt.p0 + nxt.n) {
+      if (ipos < cur.r0 + cur.n) {
+        b = __shfl_sync(kFull, rc.b, ipos - cur.r0);
+        g = cur.g;
+      } else if (nxt.n > 0 && ipos < nxt.r0 + nxt.n) {
         if (!rn.meta) load_meta(nxt, rn);
-        b = __shfl_sync(kFull, rn.b, (int)(iss - nxt.p0));
-        g = (nxt.hg * GT) / p.group;
+        b = __shfl_sync(kFull, rn.b, ipos - nxt.r0);
+        g = nxt.g;
       } else {
         break;
       }
-      if (lane == 0) issue((int)((iss - start) % C::NS), b, g);
-      ++iss;
+      if (lane == 0) issue(ist, b, g);
+      ist = (ist + 1 == C::NS) ? 0 : ist + 1;
+      ++ipos;
     }
   };
 
   bool aborted = false;
-  while (pos < end) {
-    if (pos == cur.p0 + cur.n) {  // step into the next window
+  while (cpos < n_total) {
+    if (cpos == cur.r0 + cur.n) {  // step into the next window
       const bool new_unit = (nxt.s != cur.s) || (nxt.hg != cur.hg);
       cur = nxt;
       rc = rn;
@@ -393,17 +411,15 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
       }
     }
     issue_ahead();
-    const long long k_rel = pos - start;
-    const int st = (int)(k_rel % C::NS);
-    const uint32_t parity = (uint32_t)((k_rel / C::NS) & 1);
-    if (!__all_sync(kFull, mbar_wait_bounded(&my_bars[st], parity))) {
+    const int st = cst;
+    if (!__all_sync(kFull, mbar_wait_bounded(&my_bars[st], cpar))) {
       if (lane == 0) record_error(p.dev_error, PKV_DEVERR_TIMEOUT);
       aborted = true;
       break;
     }
 
     // ---- one block: q . k, online softmax, p . v ----
-    const int kw_i = (int)(pos - cur.p0);
+    const int kw_i = cpos - cur.r0;
     const float ks = __shfl_sync(kFull, rc.ks, kw_i) * p.scale_log2;  // per-block K scale, log2 domain
     const float vs = __shfl_sync(kFull, rc.vs, kw_i);
     const float nzb = -(kMagic + __shfl_sync(kFull, rc.zp, kw_i));
@@ -503,11 +519,15 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
       }
     }
     __syncwarp();  // the stage's reads are complete (their values were consumed above)
-    ++pos;
+    ++cpos;
+    if (++cst == C::NS) {
+      cst = 0;
+      cpar ^= 1u;
+    }
 
     // ---- end of a segment: the unit's last block, or the end of this warp's range ----
     const int j_end = cur.j0 + kw_i + 1;
-    if (j_end == cur.nblk || pos == end) {
+    if (j_end == cur.nblk || cpos == n_total) {
 #pragma unroll
       for (int hh = 0; hh < GT; ++hh) {
 #pragma unroll
@@ -556,13 +576,9 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
         const int w_first = owner_of(unit_p0, T, We);
         const int w_last = owner_of(unit_p0 + cur.nblk - 1, T, We);
         const uint32_t n_seg = (uint32_t)(w_last - w_first + 1);
-        __syncwarp();
+        __syncwarp();  // the warp's partial writes precede lane 0's release below
         uint32_t ticket = 0;
-        if (lane == 0) {
-          __threadfence();  // release: this warp's partial is visible device-wide first
-          ticket = atomicInc(&p.ws_count[u], n_seg - 1);
-          __threadfence();  // acquire side for the merge below
-        }
+        if (lane == 0) ticket = atomic_inc_acq_rel_gpu(&p.ws_count[u], n_seg - 1);
         ticket = __shfl_sync(kFull, ticket, 0);
         if (ticket == n_seg - 1) {
           for (int o = lane; o < GT * D; o += 32) {
@@ -597,10 +613,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
     // A copy never completed (outputs touched by this warp are unspecified; dev_error says so).
     // Wait, again bounded, for the copies this warp issued and did not consume, so that no bulk
     // copy is still writing this CTA's shared memory when it exits.
-    for (long long k = pos; k < iss; ++k) {
-      const long long r = k - start;
-      (void)mbar_wait_bounded(&my_bars[(int)(r % C::NS)], (uint32_t)((r / C::NS) & 1));
-    }
+    for (int k = cpos; k < ipos; ++k) (void)mbar_wait_bounded(&my_bars[k % C::NS], (uint32_t)((k / C::NS) & 1));
   }
 }
 

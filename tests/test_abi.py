@@ -106,8 +106,10 @@ def test_call_validation(pkv):
 
 def test_partitioning(pkv):
     d = desc(pkv)
-    workers, ctas = pkv.pkv_decode_partitioning(d, 2, 4, 1000, 0)
+    workers, ctas = pkv.pkv_decode_partitioning(d, 200, 4, 1000, 0)  # a batch that fills the device
     assert ctas > 0 and workers % ctas == 0 and workers // ctas in (2, 4)
+    # a small batch: about one worker per 4 blocks of the largest possible work (2 x 2 x 63)
+    assert pkv.pkv_decode_partitioning(d, 2, 4, 1000, 0)[0] == 64
     # with partition_tokens: about one worker per partition_tokens tokens of the largest work
     # (2 seqs x 2 head groups x 63 blocks = 252 blocks, 8 blocks each -> 32 workers)
     w2, c2 = pkv.pkv_decode_partitioning(d, 2, 4, 1000, 128)
@@ -117,7 +119,7 @@ def test_partitioning(pkv):
     w4, _ = pkv.pkv_decode_partitioning(d, 2, 4, 1000, 16)        # one block each: 252 workers
     assert w4 == 252
     w5, _ = pkv.pkv_decode_partitioning(d, 200, 4, 1000, 16)      # never more than fit on the device
-    assert w5 == pkv.pkv_decode_partitioning(d, 200, 4, 1000, 0)[0]
+    assert w5 == workers
 
 
 def test_workspace_size(pkv):
@@ -133,5 +135,5 @@ def test_workspace_size(pkv):
         workers, _ = pkv.pkv_decode_partitioning(d, S, 4, L, pt)
         assert pkv.pkv_decode_workspace_size(d, S, 4, L, pt) == expect(S, 4, workers)
     assert pkv.pkv_decode_workspace_size(d, 0, 4, 64, 0) == 0
-    # independent of the context length for a fixed worker count (no copy of the cache)
-    assert pkv.pkv_decode_workspace_size(d, 8, 4, 64, 0) == pkv.pkv_decode_workspace_size(d, 8, 4, 32768, 0)
+    # independent of the context length once the device is full (no copy of the cache)
+    assert pkv.pkv_decode_workspace_size(d, 64, 4, 8192, 0) == pkv.pkv_decode_workspace_size(d, 64, 4, 32768, 0)
