@@ -44,7 +44,7 @@ constexpr float kNegBig = -1.0e30f;  // finite "minus infinity" for running maxi
 // Shared-memory budget of one CTA's copy rings and the CTA-per-SM caps by heads per warp
 // (overridable at build time for tuning sweeps).
 #ifndef PKV_DECODE_SMEM_TARGET
-#define PKV_DECODE_SMEM_TARGET 49152
+#define PKV_DECODE_SMEM_TARGET 32768
 #endif
 #ifndef PKV_DECODE_CPS_GT1
 #define PKV_DECODE_CPS_GT1 4
