@@ -203,6 +203,33 @@ PKV_API pkv_status pkv_paged_attention_decode(const pkv_cache_desc* desc, void* 
                                       pkv_stream_t stream);
 
 /*
+ * pkv_paged_attention_decode_static -- the same decode as pkv_paged_attention_decode, for
+ * callers that cannot hand the library any scratch memory: for example a plugin that its host
+ * engine gives only the input and output buffers (the engine owns every other byte of device
+ * memory), or a serving loop that fixed its memory budget up front and may not allocate per
+ * request. The web pages this library follows have no counterpart of this call; it exists only
+ * for such callers.
+ *
+ * It allocates nothing: its scratch is one file-scope device array of PKV_STATIC_SCRATCH_BYTES
+ * (8 MiB) that every GPU holds from the moment the library is loaded until the process exits.
+ *   - Sizes whose scratch would exceed it (pkv_decode_workspace_size(...) >
+ *     PKV_STATIC_SCRATCH_BYTES) are rejected with PKV_ERR_UNSUPPORTED before anything runs; use
+ *     pkv_paged_attention_decode with a workspace for those.
+ *   - The first call on a device looks up that device's address of the array (with the device
+ *     current), so make that first call before any stream capture begins.
+ *   - All calls share the array and it keeps the last call's contents; each call clears, on its
+ *     stream, the part that must start at zero. Calls whose executions overlap on the GPU (any
+ *     streams, any threads) race on the array and give undefined results: serialise them.
+ * Arguments and results are those of pkv_paged_attention_decode without the workspace.
+ */
+#define PKV_STATIC_SCRATCH_BYTES (8u << 20)
+PKV_API pkv_status pkv_paged_attention_decode_static(
+    const pkv_cache_desc* desc, void* out, const void* q, int32_t num_seqs, int32_t num_q_heads,
+    const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+    int32_t max_context_len, float softmax_scale, int32_t partition_tokens, int32_t* dev_error,
+    pkv_stream_t stream);
+
+/*
  * pkv_copy_blocks -- copy-on-write block copies ([deepinsea] section "Copy-on-Write 机制";
  * [yunthe] "PagedAttention分页注意力机制", fork writes new tokens into new blocks).
  * For each pair (src, dst) in block_mapping, copies every head's K codes, V codes, scales and

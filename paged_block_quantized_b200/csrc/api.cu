@@ -251,4 +251,48 @@ pkv_status pkv_copy_blocks(const pkv_cache_desc* desc, const int32_t* block_mapp
   return launch_copy(p, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
+// ---- decode without caller-provided scratch -------------------------------------------------
+// Scratch for pkv_paged_attention_decode_static: one array per device, alive while the library
+// is loaded. In host code the name below stands for a host-side shadow, not a device address, so
+// the device address is looked up (per device, with that device current) before any use.
+static __device__ __align__(256) unsigned char g_static_scratch[PKV_STATIC_SCRATCH_BYTES];
+
+static void* static_scratch_on_current_device(cudaError_t* err) {
+  static void* cached[64] = {nullptr};
+  int dev = 0;
+  *err = cudaGetDevice(&dev);
+  if (*err != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (cached[dev] == nullptr) {
+    void* ptr = nullptr;
+    *err = cudaGetSymbolAddress(&ptr, g_static_scratch);
+    if (*err != cudaSuccess) return nullptr;
+    cached[dev] = ptr;
+  }
+  return cached[dev];
+}
+
+pkv_status pkv_paged_attention_decode_static(const pkv_cache_desc* desc, void* out, const void* q, int32_t num_seqs,
+                                             int32_t num_q_heads, const int32_t* block_tables,
+                                             int32_t max_blocks_per_seq, const int32_t* context_lens,
+                                             int32_t max_context_len, float softmax_scale, int32_t partition_tokens,
+                                             int32_t* dev_error, pkv_stream_t stream) {
+  pkv_status st = check_desc(desc);
+  if (st != PKV_OK) return st;
+  if (!decode_supported(desc->k_dtype, desc->v_dtype, desc->block_size, desc->head_dim)) return PKV_ERR_UNSUPPORTED;
+  DecodeGeometry g;
+  st = decode_geometry(desc, num_seqs, num_q_heads, max_context_len, partition_tokens, &g);
+  if (st != PKV_OK) return st;
+  if (num_seqs == 0) return PKV_OK;
+  if (g.workspace_bytes > PKV_STATIC_SCRATCH_BYTES) return PKV_ERR_UNSUPPORTED;  // too large for the array
+  cudaError_t err = cudaSuccess;
+  void* scratch = static_scratch_on_current_device(&err);
+  if (scratch == nullptr) return PKV_ERR_CUDA;
+  // the tickets must start at zero: the array holds whatever the previous call left
+  if (cudaMemsetAsync(scratch, 0, g.counter_bytes, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return PKV_ERR_CUDA;
+  return pkv_paged_attention_decode(desc, out, q, num_seqs, num_q_heads, block_tables, max_blocks_per_seq,
+                                    context_lens, max_context_len, softmax_scale, partition_tokens, scratch,
+                                    PKV_STATIC_SCRATCH_BYTES, dev_error, stream);
+}
+
 }  // extern "C"

@@ -28,7 +28,7 @@ PKV_FP16, PKV_INT8_SYM, PKV_INT4_ASYM = 0, 1, 2
 
 EXPORTED = (
     "pkv_status_string", "pkv_tile_bytes", "pkv_store_quantized", "pkv_decode_workspace_size",
-    "pkv_decode_partitioning",
+    "pkv_decode_partitioning", "pkv_paged_attention_decode_static",
     "pkv_paged_attention_decode", "pkv_copy_blocks", "pkv_blocks_for_tokens", "pkv_alloc_create",
     "pkv_alloc_destroy", "pkv_alloc_num_free", "pkv_alloc_refcount", "pkv_alloc_blocks", "pkv_alloc_fork",
     "pkv_alloc_release", "pkv_alloc_cow",
@@ -72,6 +72,9 @@ _partitioning = _sig("pkv_decode_partitioning", ctypes.c_int, _DESC, _I32, _I32,
                      ctypes.POINTER(_I32), ctypes.POINTER(_I32))
 _decode = _sig("pkv_paged_attention_decode", ctypes.c_int, _DESC, _P, _P, _I32, _I32, _P, _I32, _P, _I32,
                ctypes.c_float, _I32, _P, ctypes.c_size_t, _P, _P)
+_decode_static = _sig("pkv_paged_attention_decode_static", ctypes.c_int, _DESC, _P, _P, _I32, _I32, _P, _I32, _P,
+                      _I32, ctypes.c_float, _I32, _P, _P)
+PKV_STATIC_SCRATCH_BYTES = 8 << 20
 _copy = _sig("pkv_copy_blocks", ctypes.c_int, _DESC, _P, _I32, _P, _P)
 _blocks_for_tokens = _sig("pkv_blocks_for_tokens", _I32, ctypes.c_int64, _I32)
 _alloc_create = _sig("pkv_alloc_create", ctypes.c_int, _I32, ctypes.POINTER(_P))
@@ -157,6 +160,17 @@ def pkv_paged_attention_decode(desc, out, q, num_seqs, num_q_heads, block_tables
                  int(max_blocks_per_seq), _ptr(context_lens), int(max_context_len), float(softmax_scale),
                  int(partition_tokens), _ptr(workspace), int(workspace_bytes), _ptr(dev_error), _stream(stream))
     return _check(st, "pkv_paged_attention_decode", raise_on_error)
+
+
+def pkv_paged_attention_decode_static(desc, out, q, num_seqs, num_q_heads, block_tables, max_blocks_per_seq,
+                                      context_lens, max_context_len, softmax_scale, partition_tokens=0,
+                                      dev_error=None, stream=None, raise_on_error=True):
+    """Decode without a workspace, for callers that cannot provide scratch memory; uses the
+    library's own fixed device array (see include/pkv.h: calls must not overlap on the GPU)."""
+    st = _decode_static(ctypes.byref(desc), _ptr(out), _ptr(q), int(num_seqs), int(num_q_heads), _ptr(block_tables),
+                        int(max_blocks_per_seq), _ptr(context_lens), int(max_context_len), float(softmax_scale),
+                        int(partition_tokens), _ptr(dev_error), _stream(stream))
+    return _check(st, "pkv_paged_attention_decode_static", raise_on_error)
 
 
 def pkv_copy_blocks(desc, block_mapping, n_pairs, dev_error=None, stream=None, raise_on_error=True):
