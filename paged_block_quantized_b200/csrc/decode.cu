@@ -293,6 +293,10 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
   load_ids(cur, rc);
   Win nxt = next_win(cur);
   load_ids(nxt, rn);
+  // Everything above reads only what the host wrote before the preceding kernel (lengths,
+  // tables). From here on the pool is read, which the preceding kernel (the store of the new
+  // tokens) may still be writing: wait for it to complete (no-op without a programmatic launch).
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   load_meta(cur, rc);
   __syncwarp();  // barrier initialisation by lane 0 is visible to the warp
 
@@ -631,8 +635,19 @@ cudaError_t launch_one(const DecodeParams& p, const DecodeShape& sh, cudaStream_
     if (e != cudaSuccess) return e;
     configured |= bit;
   }
-  kern<<<sh.grid_ctas, C::THREADS, C::SMEM, stream>>>(p);
-  return cudaGetLastError();
+  // programmatic dependent launch: the kernel may start while the previous kernel in the stream
+  // finishes; it waits for it (griddepcontrol.wait) before reading the pool
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(sh.grid_ctas);
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
 template <int KT, int VT, int BS, int D, int GT>

@@ -248,70 +248,251 @@ __device__ void store_fp16(const GroupSrc& src, __half* tile, int o0, int lane) 
   }
 }
 
+// ---- single-token groups (the decode-step append): everything in registers ----
+// A lane holds vpl = head_dim / 32 consecutive values (2, 4 or 8) of the token for one head.
+__device__ __forceinline__ void load_halves(const __half* src, int vpl, uint32_t raw[4]) {
+  raw[0] = raw[1] = raw[2] = raw[3] = 0;
+  if (vpl == 8) {
+    const uint4 w = *reinterpret_cast<const uint4*>(src);
+    raw[0] = w.x; raw[1] = w.y; raw[2] = w.z; raw[3] = w.w;
+  } else if (vpl == 4) {
+    const uint2 w = *reinterpret_cast<const uint2*>(src);
+    raw[0] = w.x; raw[1] = w.y;
+  } else {
+    raw[0] = *reinterpret_cast<const uint32_t*>(src);
+  }
+}
+__device__ __forceinline__ void halves_to_float(const uint32_t raw[4], float x[8]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&raw[i]));
+    x[2 * i] = f.x;
+    x[2 * i + 1] = f.y;
+  }
+}
+
+// INT8 symmetric side of a one-token group at offset o0. Returns false (nothing written) when the
+// token does not fit the stored scale: the caller then takes the general path (rebuild).
+__device__ bool fast_sym(const float x[8], int vpl, int8_t* tile, float* scale_ptr, float s_old, int o0, int d,
+                         int lane) {
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    if (i < vpl) m = fmaxf(m, fabsf(x[i]));
+  m = warp_max(m);
+  float s;
+  if (o0 == 0) {
+    s = __fdiv_rn(m, 127.0f);
+  } else {
+    bool fits = true;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (i >= vpl) continue;
+      if (s_old == 0.0f) {
+        fits = fits && (x[i] == 0.0f);
+      } else {
+        const int r = __float2int_rn(__fdiv_rn(x[i], s_old));
+        fits = fits && (r <= 127 && r >= -127);
+      }
+    }
+    if (!__all_sync(kFull, fits)) return false;
+    s = s_old;
+  }
+  uint32_t lo = 0, hi = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if (i >= vpl) continue;
+    const uint32_t c = (uint32_t)(quant_sym(x[i], s) & 0xff);
+    if (i < 4) lo |= c << (8 * i); else hi |= c << (8 * (i - 4));
+  }
+  int8_t* dst = tile + (size_t)o0 * d + lane * vpl;
+  if (vpl == 8) *reinterpret_cast<uint2*>(dst) = make_uint2(lo, hi);
+  else if (vpl == 4) *reinterpret_cast<uint32_t*>(dst) = lo;
+  else *reinterpret_cast<uint16_t*>(dst) = (uint16_t)lo;
+  if (o0 == 0 && lane == 0) *scale_ptr = s;
+  return true;
+}
+
+// INT4 asymmetric side of a one-token group; false when the token does not fit (rebuild needed).
+__device__ bool fast_asym4(const float x[8], int vpl, uint8_t* tile, float* scale_ptr, uint8_t* zp_ptr, float s_old,
+                           int zp_old, int o0, int d, int lane) {
+  float s;
+  int zp;
+  if (o0 == 0) {
+    float lo = 0.0f, hi = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (i >= vpl) continue;
+      lo = fminf(lo, x[i]);
+      hi = fmaxf(hi, x[i]);
+    }
+    lo = warp_min(lo);
+    hi = warp_max(hi);
+    derive_asym(lo, hi, s, zp);
+  } else {
+    bool fits = true;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (i >= vpl) continue;
+      if (s_old == 0.0f) {
+        fits = fits && (x[i] == 0.0f);
+      } else {
+        const int r = __float2int_rn(__fadd_rn(__fdiv_rn(x[i], s_old), (float)zp_old));
+        fits = fits && (r >= 0 && r <= 15);
+      }
+    }
+    if (!__all_sync(kFull, fits)) return false;
+    s = s_old;
+    zp = zp_old;
+  }
+  uint32_t packed = 0;  // vpl / 2 bytes: byte j = code[2j] | code[2j+1] << 4
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) {
+    if (i >= vpl) continue;
+    const uint32_t b = (uint32_t)(quant_asym(x[i], s, zp) | (quant_asym(x[i + 1], s, zp) << 4));
+    packed |= b << (4 * i);
+  }
+  uint8_t* dst = tile + (size_t)o0 * (d / 2) + lane * (vpl / 2);
+  if (vpl == 8) *reinterpret_cast<uint32_t*>(dst) = packed;
+  else if (vpl == 4) *reinterpret_cast<uint16_t*>(dst) = (uint16_t)packed;
+  else *dst = (uint8_t)packed;
+  if (o0 == 0 && lane == 0) {
+    *scale_ptr = s;
+    *zp_ptr = (uint8_t)zp;
+  }
+  return true;
+}
+
+__device__ __forceinline__ void fast_fp16(const uint32_t raw[4], int vpl, __half* tile, int o0, int d, int lane) {
+  __half* dst = tile + (size_t)o0 * d + lane * vpl;
+  if (vpl == 8) *reinterpret_cast<uint4*>(dst) = make_uint4(raw[0], raw[1], raw[2], raw[3]);
+  else if (vpl == 4) *reinterpret_cast<uint2*>(dst) = make_uint2(raw[0], raw[1]);
+  else *reinterpret_cast<uint32_t*>(dst) = raw[0];
+}
+
 __global__ void __launch_bounds__(32 * kWarpsPerCta) store_quantized_kernel(const StoreParams p) {
+  // a kernel launched after this one with programmatic serialization (the decode) may begin its
+  // set-up now; it waits for this grid to complete before it reads the pool
+  asm volatile("griddepcontrol.launch_dependents;");
   const int t = blockIdx.x;
   const int h = blockIdx.y * kWarpsPerCta + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (h >= p.num_kv_heads) return;
   const int bs = p.block_size;
+  const int d = p.head_dim;
+  const int vpl = d / 32;
   const int64_t num_slots = (int64_t)p.num_blocks * bs;
-  const int64_t slot = p.slot_mapping[t];
+  const int64_t row_stride = (int64_t)p.num_kv_heads * d;
+
+  // ---- one round of independent loads: the slots of tokens t-1 .. t+30 (lane i holds token
+  // t-1+i) and this token's own K and V values for this head ----
+  const int idx = t - 1 + lane;
+  int64_t sl = INT64_MIN;  // "no token"
+  if (idx >= 0 && idx < p.T) sl = p.slot_mapping[idx];
+  uint32_t kraw[4], vraw[4];
+  load_halves(p.k_new + (size_t)t * row_stride + (size_t)h * d + lane * vpl, vpl, kraw);
+  load_halves(p.v_new + (size_t)t * row_stride + (size_t)h * d + lane * vpl, vpl, vraw);
+
+  const int64_t slot = __shfl_sync(kFull, sl, 1);
+  const int64_t prev = __shfl_sync(kFull, sl, 0);
   if (slot < 0) return;  // padding token
   if (slot >= num_slots) {
     if (h == 0 && lane == 0) record_error(p.dev_error, PKV_DEVERR_SLOT);
     return;
   }
   const int64_t block = slot / bs;
-  if (t > 0) {
-    const int64_t prev = p.slot_mapping[t - 1];
-    if (prev >= 0 && prev < num_slots && prev / bs == block) return;  // not the group's first token
-  }
+  if (prev >= 0 && prev < num_slots && prev / bs == block) return;  // not the group's first token
+
   // the group: following tokens with a valid slot in the same block; offsets must be consecutive
   int n = 1;
   bool consecutive = true;
-  while (true) {
-    const int idx = t + n + lane;
-    bool same = false, step_ok = true;
-    if (idx < p.T) {
-      const int64_t sl = p.slot_mapping[idx];
-      same = sl >= 0 && sl < num_slots && sl / bs == block;
-      step_ok = sl == slot + n + lane;
-    }
-    const uint32_t run_mask = __ballot_sync(kFull, same);
-    const int run = (run_mask == kFull) ? 32 : (__ffs(~run_mask) - 1);
-    const uint32_t bad = __ballot_sync(kFull, same && !step_ok && lane < run);
-    if (bad) consecutive = false;
+  {
+    const bool same = lane >= 2 && sl >= 0 && sl < num_slots && sl / bs == block;
+    const bool step_ok = sl == slot + (lane - 1);
+    const uint32_t m = __ballot_sync(kFull, same) >> 2;  // bit k: token t+1+k
+    const int run = (m == 0x3FFFFFFFu) ? 30 : (__ffs(~m) - 1);
+    if (__ballot_sync(kFull, same && !step_ok && lane - 2 < run)) consecutive = false;
     n += run;
-    if (run < 32 || n > bs) break;
+  }
+  if (n == 31) {  // the group may go on beyond token t+30
+    while (true) {
+      const int i2 = t + n + lane;
+      bool same = false, step_ok = true;
+      if (i2 < p.T) {
+        const int64_t s2 = p.slot_mapping[i2];
+        same = s2 >= 0 && s2 < num_slots && s2 / bs == block;
+        step_ok = s2 == slot + n + lane;
+      }
+      const uint32_t run_mask = __ballot_sync(kFull, same);
+      const int run = (run_mask == kFull) ? 32 : (__ffs(~run_mask) - 1);
+      if (__ballot_sync(kFull, same && !step_ok && lane < run)) consecutive = false;
+      n += run;
+      if (run < 32 || n > bs) break;
+    }
   }
   if (!consecutive || n > bs) {
     if (h == 0 && lane == 0) record_error(p.dev_error, PKV_DEVERR_SLOT_GROUP);
     return;
   }
   const int o0 = (int)(slot % bs);
-  const int d = p.head_dim;
   const size_t tile_idx = (size_t)block * p.num_kv_heads + h;
+  int8_t* k_tile8 = static_cast<int8_t*>(p.k_codes) + tile_idx * bs * d;
+  __half* k_tile16 = static_cast<__half*>(p.k_codes) + tile_idx * bs * d;
+  int8_t* v_tile8 = static_cast<int8_t*>(p.v_codes) + tile_idx * bs * d;
+  uint8_t* v_tile4 = static_cast<uint8_t*>(p.v_codes) + tile_idx * bs * (d / 2);
+  __half* v_tile16 = static_cast<__half*>(p.v_codes) + tile_idx * bs * d;
+
+  bool k_done = false, v_done = false;
+  if (n == 1) {
+    // the stored scale / zero point matter only when appending into a partly filled tile
+    float ks_old = 0.f, vs_old = 0.f;
+    int vzp_old = 0;
+    if (o0 > 0) {
+      if (p.k_dtype == PKV_INT8_SYM) ks_old = p.k_scale[tile_idx];
+      if (p.v_dtype != PKV_FP16) vs_old = p.v_scale[tile_idx];
+      if (p.v_dtype == PKV_INT4_ASYM) vzp_old = p.v_zp[tile_idx];
+    }
+    float kx[8], vx[8];
+    halves_to_float(kraw, kx);
+    halves_to_float(vraw, vx);
+    if (p.k_dtype == PKV_INT8_SYM) {
+      k_done = fast_sym(kx, vpl, k_tile8, p.k_scale + tile_idx, ks_old, o0, d, lane);
+    } else {
+      fast_fp16(kraw, vpl, k_tile16, o0, d, lane);
+      k_done = true;
+    }
+    if (p.v_dtype == PKV_INT8_SYM) {
+      v_done = fast_sym(vx, vpl, v_tile8, p.v_scale + tile_idx, vs_old, o0, d, lane);
+    } else if (p.v_dtype == PKV_INT4_ASYM) {
+      v_done = fast_asym4(vx, vpl, v_tile4, p.v_scale + tile_idx, p.v_zp + tile_idx, vs_old, vzp_old, o0, d, lane);
+    } else {
+      fast_fp16(vraw, vpl, v_tile16, o0, d, lane);
+      v_done = true;
+    }
+  }
+
+  // general path: groups of several tokens, and appends that must rebuild the tile
   GroupSrc src;
-  src.row_stride = (int64_t)p.num_kv_heads * d;
+  src.row_stride = row_stride;
   src.n = n;
   src.d = d;
-
-  // K side
-  src.base = p.k_new + (size_t)t * src.row_stride + (size_t)h * d;
-  if (p.k_dtype == PKV_INT8_SYM) {
-    store_sym(src, static_cast<int8_t*>(p.k_codes) + tile_idx * bs * d, p.k_scale + tile_idx, o0, lane);
-  } else {
-    store_fp16(src, static_cast<__half*>(p.k_codes) + tile_idx * bs * d, o0, lane);
+  if (!k_done) {
+    src.base = p.k_new + (size_t)t * src.row_stride + (size_t)h * d;
+    if (p.k_dtype == PKV_INT8_SYM) {
+      store_sym(src, k_tile8, p.k_scale + tile_idx, o0, lane);
+    } else {
+      store_fp16(src, k_tile16, o0, lane);
+    }
   }
-  // V side
-  src.base = p.v_new + (size_t)t * src.row_stride + (size_t)h * d;
-  if (p.v_dtype == PKV_INT8_SYM) {
-    store_sym(src, static_cast<int8_t*>(p.v_codes) + tile_idx * bs * d, p.v_scale + tile_idx, o0, lane);
-  } else if (p.v_dtype == PKV_INT4_ASYM) {
-    store_asym4(src, static_cast<uint8_t*>(p.v_codes) + tile_idx * bs * (d / 2), p.v_scale + tile_idx,
-                p.v_zp + tile_idx, o0, lane);
-  } else {
-    store_fp16(src, static_cast<__half*>(p.v_codes) + tile_idx * bs * d, o0, lane);
+  if (!v_done) {
+    src.base = p.v_new + (size_t)t * src.row_stride + (size_t)h * d;
+    if (p.v_dtype == PKV_INT8_SYM) {
+      store_sym(src, v_tile8, p.v_scale + tile_idx, o0, lane);
+    } else if (p.v_dtype == PKV_INT4_ASYM) {
+      store_asym4(src, v_tile4, p.v_scale + tile_idx, p.v_zp + tile_idx, o0, lane);
+    } else {
+      store_fp16(src, v_tile16, o0, lane);
+    }
   }
 }
 
