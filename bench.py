@@ -82,6 +82,16 @@ def dist_max(value: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def dist_sum(value: float, world: int, device=None) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
 def dist_barrier(world: int, device=None):
     if world > 1:
         import torch.distributed as dist
@@ -297,20 +307,22 @@ def run_pkv(args, rank, world, local):
         torch.cuda.synchronize(dev)
         dist_barrier(world, dev)
         wall_ms = (time.perf_counter() - wall0) * 1e3
-        # the decode kernel on its own (roofline): the same steps with events around the decode
-        dev_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+        # each kernel on its own (roofline): the same steps with events around the store and the decode
+        dev_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
         for i in range(K):
             flush()
             g.copy()
-            g.store()
             dev_ev[i][0].record(stream)
-            g.decode()
+            g.store()
             dev_ev[i][1].record(stream)
+            g.decode()
+            dev_ev[i][2].record(stream)
         torch.cuda.synchronize(dev)
     step_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
-    dec_ms = [dev_ev[i][0].elapsed_time(dev_ev[i][1]) for i in range(K)]
+    store_ms = [dev_ev[i][0].elapsed_time(dev_ev[i][1]) for i in range(K)]
+    dec_ms = [dev_ev[i][1].elapsed_time(dev_ev[i][2]) for i in range(K)]
     total_s = dist_max(sum(step_ms) / 1e3, world, dev)
-    tokens_all = w.total_tokens * K * world
+    tokens_all = dist_sum(float(w.total_tokens * K), world, dev)  # every rank runs its own workload
     value = tokens_all / total_s
 
     # ---- e2e: same step through the public runner with host buffers copied in and out ----
@@ -359,7 +371,7 @@ def run_pkv(args, rank, world, local):
         "config": {**config_block(w, g, step_desc), "parallelism": f"dp{world} (independent sequences per rank)",
                    "l2": "flushed before every timed step (2x L2 written, then 2x L2 read: cold and clean)", "timing": "CUDA events per step"},
         "effective_hbm_gbs": achieved, "frac_of_8tbs": achieved / 8000.0,
-        "decode_us": dec_s * 1e6,
+        "decode_us": dec_s * 1e6, "store_us": statistics.mean(store_ms) * 1e3,
         "roofline": {"bound": "hbm", "kernel": "paged_decode_kernel", "achieved": achieved, "peak": peak,
                      "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
                      "algorithmic_bytes_per_launch": alg_bytes, "peak_source": peak_src},

@@ -80,7 +80,7 @@ pkv_status decode_geometry(const pkv_cache_desc* d, int32_t num_seqs, int32_t nu
   sh.v_dtype = d->v_dtype;
   sh.block_size = d->block_size;
   sh.head_dim = d->head_dim;
-  sh.heads_per_warp = decode_heads_per_warp(group);
+  sh.heads_per_warp = decode_heads_per_warp(group, d->k_dtype, d->v_dtype, d->head_dim);
   DecodeKernelInfo info;
   if (!decode_kernel_info(sh, &info)) return PKV_ERR_UNSUPPORTED;
   const int64_t max_workers = (int64_t)sm_count() * info.ctas_per_sm * info.warps_per_cta;

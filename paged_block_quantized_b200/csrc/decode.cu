@@ -31,6 +31,8 @@
 //   * A unit processed entirely by one warp is written out directly. A unit split across warps
 //     gets one partial (max, sum, acc) per warp in the workspace; the last warp to finish (a
 //     self-resetting atomicInc ticket) merges them. No CTA barrier, no second kernel.
+#include <type_traits>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -64,19 +66,19 @@ struct Cfg {
   // stages per warp from the CTA's shared-memory budget, at least 2
   static constexpr int NS_RAW = PKV_DECODE_SMEM_TARGET / (NW * STAGE);
   static constexpr int NS = NS_RAW < 2 ? 2 : (NS_RAW > PKV_DECODE_MAX_STAGES ? PKV_DECODE_MAX_STAGES : NS_RAW);
-  static constexpr int CH = D / 16;    // lanes per token row (16 dims each)
-  static constexpr int TG = 32 / CH;   // token rows a warp covers per pass
-  static constexpr int TPL = BS / TG;  // token rows per lane per block
+  // tensor-core engine for groups of 4 or 8 query heads (INT8/INT8 with D >= 128, FP16/FP16)
+  static constexpr bool MMA =
+      GT >= 4 && ((KT == PKV_INT8_SYM && VT == PKV_INT8_SYM && D >= 128) || (KT == PKV_FP16 && VT == PKV_FP16));
   static constexpr int THREADS = 32 * NW;
   static constexpr int SMEM_STAGES = NW * NS * STAGE;
   static constexpr int SMEM = SMEM_STAGES + NW * NS * 8;
   // resident CTAs per SM: bounded by shared memory (227 KiB per SM) and by the registers a
   // thread needs for GT heads of state
   static constexpr int CPS_SMEM = (220 * 1024) / (SMEM + 1024);
-  static constexpr int CPS_CAP = (GT == 1) ? PKV_DECODE_CPS_GT1 : (GT == 2 ? 3 : 2);  // 128 / 170 / 255 regs
+  static constexpr int CPS_CAP =
+      MMA ? (D >= 256 ? 2 : 3) : ((GT == 1) ? PKV_DECODE_CPS_GT1 : (GT == 2 ? 3 : 2));  // registers
   static constexpr int CTAS_PER_SM = CPS_SMEM < 1 ? 1 : (CPS_SMEM > CPS_CAP ? CPS_CAP : CPS_SMEM);
-  static_assert(D % 16 == 0 && CH <= 32 && 32 % CH == 0, "head_dim");
-  static_assert(BS % TG == 0, "block_size must cover the token rows of a warp pass");
+  static_assert(D % 16 == 0 && D / 16 <= 32, "head_dim");
   static_assert(K_TILE % 16 == 0 && V_TILE % 16 == 0 && STAGE % 16 == 0, "bulk copy granularity");
   static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 };
@@ -137,6 +139,480 @@ struct WinLanes {
   float ks, vs, zp;
 };
 
+// ============================================================================================
+// Per-block arithmetic. Both engines see one (block, KV head) tile in shared memory at a time
+// and keep the running softmax state of GT query heads for the current unit.
+// ============================================================================================
+
+// CUDA-core engine (1, 2 or 4 query heads per KV head): a lane owns 16 consecutive dims of
+// bs/(32*16/D) token rows; q.k in exact integer dp4a planes (INT8 K) or paired FFMA (FP16 K);
+// p.v with paired FFMA on codes made exact floats through the float bit layout.
+template <int KT, int VT, int BS, int D, int GT>
+struct CoreEngine {
+  using C = Cfg<KT, VT, BS, D, GT>;
+  static constexpr int CH = D / 16, TG = 32 / CH, TPL = BS / TG;
+  static_assert(BS % TG == 0, "block_size must cover the token rows of a warp pass");
+  int c, tg;
+  float2 qf[GT][8];
+  uint32_t qplane[GT][3][4];
+  float qinv[GT];
+  float m_run[GT], l_run[GT];
+  float2 acc[GT][8];
+
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int hh = 0; hh < GT; ++hh) {
+      m_run[hh] = kNegBig;
+      l_run[hh] = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[hh][j] = make_float2(0.f, 0.f);
+    }
+  }
+
+  __device__ __forceinline__ void begin(const DecodeParams& p, int s, int hg, int lane) {
+    c = lane % CH;
+    tg = lane / CH;
+#pragma unroll
+    for (int hh = 0; hh < GT; ++hh) {
+      const __half* qp = p.q + ((size_t)s * p.num_q_heads + (size_t)hg * GT + hh) * D + c * 16;
+      const uint4 w0 = *reinterpret_cast<const uint4*>(qp);
+      const uint4 w1 = *reinterpret_cast<const uint4*>(qp + 8);
+      const uint32_t u[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) qf[hh][i] = __half22float2(*reinterpret_cast<const __half2*>(&u[i]));
+    }
+    reset();
+    // INT8 K: q . k is computed exactly in integers. Each head's q is put on a fixed-point grid
+    // of 2^-shift (22 bits below its largest magnitude; fp16 q loses nothing above 2^-22 of its
+    // max) and split into three signed byte planes, q_fixed = 2^16 b2 + 2^8 b1 + b0, so a
+    // 4-code word costs three dp4a with int32 accumulation and no code is converted to float.
+    if constexpr (KT == PKV_INT8_SYM) {
+#pragma unroll
+      for (int hh = 0; hh < GT; ++hh) {
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fmaxf(fabsf(qf[hh][i].x), fabsf(qf[hh][i].y)));
+#pragma unroll
+        for (int off = 1; off < CH; off <<= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, off));
+        int e = 0;
+        (void)frexpf(amax, &e);                    // amax < 2^e
+        const int shift = amax > 0.f ? 22 - e : 0;  // |q| * 2^shift < 2^22
+        const float up = __int_as_float((127 + shift) << 23);
+        qinv[hh] = __int_as_float((127 - shift) << 23);
+#pragma unroll
+        for (int wd = 0; wd < 4; ++wd) {
+          uint32_t p0 = 0, p1 = 0, p2 = 0;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 pr = qf[hh][(4 * wd + k) / 2];
+            const int qi = __float2int_rn((((4 * wd + k) & 1) ? pr.y : pr.x) * up);
+            const int b0 = ((qi + 128) & 0xFF) - 128;
+            const int r1 = (qi - b0) >> 8;
+            const int b1 = ((r1 + 128) & 0xFF) - 128;
+            const int b2 = (r1 - b1) >> 8;
+            p0 |= (uint32_t)(b0 & 0xFF) << (8 * k);
+            p1 |= (uint32_t)(b1 & 0xFF) << (8 * k);
+            p2 |= (uint32_t)(b2 & 0xFF) << (8 * k);
+          }
+          qplane[hh][0][wd] = p0;
+          qplane[hh][1][wd] = p1;
+          qplane[hh][2][wd] = p2;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int hh = 0; hh < GT; ++hh) qinv[hh] = 1.f;
+    }
+  }
+
+  // one block; ks = per-block K scale in the log2 domain (INT8 K), vs = V scale, nzb = -(2^23+zp)
+  __device__ __forceinline__ void block(const uint8_t* kt, const uint8_t* vt, float ks, float vs, float nzb, bool valid,
+                                        int tok0, int L, float scale_log2) {
+    const float2 neg_zp_bias = make_float2(nzb, nzb);
+    float z[TPL][GT];
+#pragma unroll
+    for (int i = 0; i < TPL; ++i) {
+      const int row = tg + TG * i;
+      const uint8_t* krow = kt + row * C::K_ROW + c * (C::K_ROW / CH);
+      if constexpr (KT == PKV_INT8_SYM) {
+        const uint4 wv = *reinterpret_cast<const uint4*>(krow);
+        const int kw[4] = {(int)wv.x, (int)wv.y, (int)wv.z, (int)wv.w};
+#pragma unroll
+        for (int hh = 0; hh < GT; ++hh) {
+          int acc_p[3];
+#pragma unroll
+          for (int pl = 0; pl < 3; ++pl) {
+            int a = __dp4a((int)qplane[hh][pl][0], kw[0], 0);
+            a = __dp4a((int)qplane[hh][pl][1], kw[1], a);
+            a = __dp4a((int)qplane[hh][pl][2], kw[2], a);
+            acc_p[pl] = __dp4a((int)qplane[hh][pl][3], kw[3], a);
+          }
+          // |acc_p| < 2^18: the low two planes combine exactly in int32, the top one in fp32
+          z[i][hh] = __fmaf_rn((float)acc_p[2], 65536.f, (float)(acc_p[1] * 256 + acc_p[0]));
+        }
+      } else {
+        float2 kf[8];
+        load_h16(krow, kf);
+#pragma unroll
+        for (int hh = 0; hh < GT; ++hh) {
+          float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int j = 0; j < 8; j += 2) {
+            a0 = __ffma2_rn(qf[hh][j], kf[j], a0);
+            a1 = __ffma2_rn(qf[hh][j + 1], kf[j + 1], a1);
+          }
+          z[i][hh] = (a0.x + a0.y) + (a1.x + a1.y);
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < TPL; ++i)
+#pragma unroll
+      for (int hh = 0; hh < GT; ++hh)
+#pragma unroll
+        for (int off = 1; off < CH; off <<= 1) z[i][hh] += __shfl_xor_sync(kFull, z[i][hh], off);
+
+    float pv[TPL][GT];
+#pragma unroll
+    for (int hh = 0; hh < GT; ++hh) {
+      const float zscale = (KT == PKV_FP16) ? scale_log2 : ks * qinv[hh];
+      float mloc = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < TPL; ++i) {
+        const int t = tok0 + tg + TG * i;
+        float zz = z[i][hh] * zscale;
+        zz = (valid && t < L) ? zz : -INFINITY;
+        z[i][hh] = zz;
+        mloc = fmaxf(mloc, zz);
+      }
+#pragma unroll
+      for (int off = CH; off < 32; off <<= 1) mloc = fmaxf(mloc, __shfl_xor_sync(kFull, mloc, off));
+      // the running max is warp-uniform; rescale only when it grows (rare after the first blocks)
+      if (mloc > m_run[hh]) {
+        const float alpha = ex2(m_run[hh] - mloc);
+        m_run[hh] = mloc;
+        l_run[hh] *= alpha;
+        const float2 alpha2 = make_float2(alpha, alpha);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[hh][j] = __fmul2_rn(acc[hh][j], alpha2);
+      }
+      const float m_new = m_run[hh];
+      float lsum = 0.f;
+#pragma unroll
+      for (int i = 0; i < TPL; ++i) {
+        const float pr = ex2(z[i][hh] - m_new);
+        lsum += pr;
+        pv[i][hh] = (VT == PKV_FP16) ? pr : pr * vs;
+      }
+      l_run[hh] += lsum;
+    }
+#pragma unroll
+    for (int i = 0; i < TPL; ++i) {
+      const int row = tg + TG * i;
+      float2 vf[8];
+      load_v16<VT>(vt + row * C::V_ROW + c * (C::V_ROW / CH), neg_zp_bias, vf);
+#pragma unroll
+      for (int hh = 0; hh < GT; ++hh) {
+        const float2 pv2 = make_float2(pv[i][hh], pv[i][hh]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[hh][j] = __ffma2_rn(pv2, vf[j], acc[hh][j]);
+      }
+    }
+  }
+
+  // end of a segment: sum the lanes' partial states over the token-row groups
+  __device__ __forceinline__ void finish() {
+#pragma unroll
+    for (int hh = 0; hh < GT; ++hh) {
+#pragma unroll
+      for (int off = CH; off < 32; off <<= 1) l_run[hh] += __shfl_xor_sync(kFull, l_run[hh], off);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+#pragma unroll
+        for (int off = CH; off < 32; off <<= 1) {
+          acc[hh][j].x += __shfl_xor_sync(kFull, acc[hh][j].x, off);
+          acc[hh][j].y += __shfl_xor_sync(kFull, acc[hh][j].y, off);
+        }
+    }
+  }
+
+  __device__ __forceinline__ void write_out(const DecodeParams& p, int s, int hg) {
+    if (tg != 0) return;
+#pragma unroll
+    for (int hh = 0; hh < GT; ++hh) {
+      const float inv = l_run[hh] > 0.f ? 1.f / l_run[hh] : 0.f;
+      __half2* o = reinterpret_cast<__half2*>(p.out + ((size_t)s * p.num_q_heads + (size_t)hg * GT + hh) * D + c * 16);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) o[j] = __floats2half2_rn(acc[hh][j].x * inv, acc[hh][j].y * inv);
+    }
+  }
+
+  __device__ __forceinline__ void write_partial(const DecodeParams& p, long long slot, int lane) {
+    if (tg == 0) {
+#pragma unroll
+      for (int hh = 0; hh < GT; ++hh) {
+        float4* dst = reinterpret_cast<float4*>(p.ws_acc + ((size_t)slot * GT + hh) * D + c * 16);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          dst[j] = make_float4(acc[hh][2 * j].x, acc[hh][2 * j].y, acc[hh][2 * j + 1].x, acc[hh][2 * j + 1].y);
+      }
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int hh = 0; hh < GT; ++hh) {
+        p.ws_ml[((size_t)slot * GT + hh) * 2 + 0] = m_run[hh];
+        p.ws_ml[((size_t)slot * GT + hh) * 2 + 1] = l_run[hh];
+      }
+    }
+  }
+};
+
+// ---- tensor-core helpers (mma.sync m16n8k16, fp16 operands, fp32 accumulators) ----
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+__device__ __forceinline__ uint32_t h2_sub(uint32_t a, uint32_t b) {
+  const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&b));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t h2_pack(float lo, float hi) {
+  const __half2 r = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+// fp16 1024 + 128 in both halves: a byte b placed under exponent 0x64 reads 1024 + b, and
+// (c ^ 0x80) = c + 128 for a signed code c, so subtracting this leaves c exactly
+constexpr uint32_t kH2Bias = 0x64806480u;
+
+// Tensor-core engine (4 or 8 query heads per KV head): per 16-token slice of a block,
+//   S = K . q^T  as mma m16n8k16 with M = 16 tokens, N = 8 heads, K = 16 dims per step, and
+//   O^T += V^T . P^T  with M = 16 dims per tile, N = 8 heads, K = 16 tokens,
+// the int8 codes turned into exact fp16 integers in registers on the way into the A operands.
+// Dim order inside an mma step is a fixed permutation, the same for both operands of a product.
+// Lane (g = lane/4, c = lane%4): q.k reads token rows g, g+8 at dims [c*D/4, (c+1)*D/4); p.v reads
+// token rows 2c, 2c+1, 2c+8, 2c+9 at dims [g*D/8, (g+1)*D/8) and owns the outputs of heads 2c,
+// 2c+1 at those dims. P goes through movmatrix.trans from accumulator to operand layout, split
+// into an fp16 high and low part so p.v keeps about 22 bits of each weight.
+template <int KT, int VT, int BS, int D, int GT>
+struct MmaEngine {
+  using C = Cfg<KT, VT, BS, D, GT>;
+  static constexpr int KS = D / 16;  // q.k steps and p.v dim tiles
+  static_assert(BS % 16 == 0, "16-token slices");
+  int g, c;
+  uint32_t qb[KS][2];
+  float acc[KS][4];
+  float m_run[2], l_run[2];
+
+  __device__ __forceinline__ void reset() {
+    m_run[0] = m_run[1] = kNegBig;
+    l_run[0] = l_run[1] = 0.f;
+#pragma unroll
+    for (int j = 0; j < KS; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+  }
+
+  __device__ __forceinline__ void begin(const DecodeParams& p, int s, int hg, int lane) {
+    g = lane >> 2;
+    c = lane & 3;
+    // q^T fragments: head g of the group, dims [c*D/4, (c+1)*D/4) as 2*KS half2 words
+#pragma unroll
+    for (int j = 0; j < KS; ++j) qb[j][0] = qb[j][1] = 0u;
+    if (g < GT) {
+      const uint4* qp = reinterpret_cast<const uint4*>(p.q + ((size_t)s * p.num_q_heads + (size_t)hg * GT + g) * D +
+                                                       c * (D / 4));
+#pragma unroll
+      for (int i = 0; i < KS / 2; ++i) {
+        const uint4 w = qp[i];
+        qb[2 * i][0] = w.x;
+        qb[2 * i][1] = w.y;
+        qb[2 * i + 1][0] = w.z;
+        qb[2 * i + 1][1] = w.w;
+      }
+    }
+    reset();
+  }
+
+  __device__ __forceinline__ void block(const uint8_t* kt, const uint8_t* vt, float ks, float vs, float /*nzb*/,
+                                        bool valid, int tok0, int L, float scale_log2) {
+    const float zscale = (KT == PKV_FP16) ? scale_log2 : ks;
+#pragma unroll
+    for (int h2 = 0; h2 < BS / 16; ++h2) {
+      // ---- S = K . q^T over this 16-token slice ----
+      float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+      const uint8_t* k0 = kt + (16 * h2 + g) * C::K_ROW + c * (C::K_ROW / 4);
+      const uint8_t* k1 = k0 + 8 * C::K_ROW;
+      if constexpr (KT == PKV_INT8_SYM) {
+#pragma unroll
+        for (int i = 0; i < KS / 4; ++i) {  // 16 codes = 4 steps per 16-byte load
+          const uint4 r0 = *reinterpret_cast<const uint4*>(k0 + 16 * i);
+          const uint4 r1 = *reinterpret_cast<const uint4*>(k1 + 16 * i);
+          const uint32_t w0[4] = {r0.x, r0.y, r0.z, r0.w};
+          const uint32_t w1[4] = {r1.x, r1.y, r1.z, r1.w};
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const uint32_t u0 = w0[q4] ^ 0x80808080u, u1 = w1[q4] ^ 0x80808080u;
+            uint32_t a[4];
+            a[0] = h2_sub(__byte_perm(u0, 0x64646464u, 0x4140), kH2Bias);  // row g, dims +0,+1
+            a[1] = h2_sub(__byte_perm(u1, 0x64646464u, 0x4140), kH2Bias);  // row g+8
+            a[2] = h2_sub(__byte_perm(u0, 0x64646464u, 0x4342), kH2Bias);  // row g, dims +2,+3
+            a[3] = h2_sub(__byte_perm(u1, 0x64646464u, 0x4342), kH2Bias);  // row g+8
+            const int kk = 4 * i + q4;
+            mma_16816(sacc, a, qb[kk][0], qb[kk][1]);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < KS / 2; ++i) {  // 8 halves = 2 steps per 16-byte load
+          const uint4 r0 = *reinterpret_cast<const uint4*>(k0 + 16 * i);
+          const uint4 r1 = *reinterpret_cast<const uint4*>(k1 + 16 * i);
+          uint32_t a[4] = {r0.x, r1.x, r0.y, r1.y};
+          mma_16816(sacc, a, qb[2 * i][0], qb[2 * i][1]);
+          uint32_t b[4] = {r0.z, r1.z, r0.w, r1.w};
+          mma_16816(sacc, b, qb[2 * i + 1][0], qb[2 * i + 1][1]);
+        }
+      }
+      // ---- online softmax on the accumulator layout: rows = tokens g, g+8; cols = heads 2c, 2c+1 ----
+      const int t0 = tok0 + 16 * h2 + g, t1 = t0 + 8;
+      float z[4];
+      z[0] = (valid && t0 < L) ? sacc[0] * zscale : -INFINITY;
+      z[1] = (valid && t0 < L) ? sacc[1] * zscale : -INFINITY;
+      z[2] = (valid && t1 < L) ? sacc[2] * zscale : -INFINITY;
+      z[3] = (valid && t1 < L) ? sacc[3] * zscale : -INFINITY;
+      float mx0 = fmaxf(z[0], z[2]), mx1 = fmaxf(z[1], z[3]);
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, off));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, off));
+      }
+      const bool grow0 = mx0 > m_run[0], grow1 = mx1 > m_run[1];
+      if (__any_sync(kFull, grow0 || grow1)) {
+        const float al0 = grow0 ? ex2(m_run[0] - mx0) : 1.f;
+        const float al1 = grow1 ? ex2(m_run[1] - mx1) : 1.f;
+        if (grow0) m_run[0] = mx0;
+        if (grow1) m_run[1] = mx1;
+        l_run[0] *= al0;
+        l_run[1] *= al1;
+#pragma unroll
+        for (int j = 0; j < KS; ++j) {
+          acc[j][0] *= al0;
+          acc[j][2] *= al0;
+          acc[j][1] *= al1;
+          acc[j][3] *= al1;
+        }
+      }
+      const float p0 = ex2(z[0] - m_run[0]), p1 = ex2(z[1] - m_run[1]);
+      const float p2 = ex2(z[2] - m_run[0]), p3 = ex2(z[3] - m_run[1]);
+      l_run[0] += p0 + p2;
+      l_run[1] += p1 + p3;
+      // weights for p.v (V scale folded in), fp16 high + low parts, transposed to operand layout
+      const float w0 = (VT == PKV_FP16) ? p0 : p0 * vs, w1 = (VT == PKV_FP16) ? p1 : p1 * vs;
+      const float w2 = (VT == PKV_FP16) ? p2 : p2 * vs, w3 = (VT == PKV_FP16) ? p3 : p3 * vs;
+      const uint32_t hi0 = h2_pack(w0, w1), hi1 = h2_pack(w2, w3);
+      const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&hi0));
+      const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&hi1));
+      const uint32_t lo0 = h2_pack(w0 - f0.x, w1 - f0.y), lo1 = h2_pack(w2 - f1.x, w3 - f1.y);
+      const uint32_t bh0 = movmatrix_trans(hi0), bh1 = movmatrix_trans(hi1);
+      const uint32_t bl0 = movmatrix_trans(lo0), bl1 = movmatrix_trans(lo1);
+      // ---- O^T += V^T . P^T: token rows 2c, 2c+1, 2c+8, 2c+9 at dims [g*D/8, (g+1)*D/8) ----
+      const uint8_t* vb = vt + (16 * h2 + 2 * c) * C::V_ROW + g * (C::V_ROW / 8);
+      if constexpr (VT == PKV_INT8_SYM) {
+#pragma unroll
+        for (int i = 0; i < KS / 8; ++i) {  // 16 bytes per row = 8 dim tiles
+          const uint4 ra = *reinterpret_cast<const uint4*>(vb + 16 * i);
+          const uint4 rb = *reinterpret_cast<const uint4*>(vb + C::V_ROW + 16 * i);
+          const uint4 rc = *reinterpret_cast<const uint4*>(vb + 8 * C::V_ROW + 16 * i);
+          const uint4 rd = *reinterpret_cast<const uint4*>(vb + 9 * C::V_ROW + 16 * i);
+          const uint32_t xa[4] = {ra.x, ra.y, ra.z, ra.w}, xb[4] = {rb.x, rb.y, rb.z, rb.w};
+          const uint32_t xc[4] = {rc.x, rc.y, rc.z, rc.w}, xd[4] = {rd.x, rd.y, rd.z, rd.w};
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) {  // dim tile: bytes 2jj (row r) and 2jj+1 (row r+8)
+            const int wd = jj / 2, k = 2 * (jj % 2);
+            const uint32_t sel0 = k | (k << 4) | ((4 + k) << 8) | ((4 + k) << 12);
+            const uint32_t sel1 = (k + 1) | ((k + 1) << 4) | ((5 + k) << 8) | ((5 + k) << 12);
+            uint32_t a[4];
+            a[0] = h2_sub((__byte_perm(xa[wd], xb[wd], sel0) & 0x00FF00FFu) ^ kH2Bias, kH2Bias);
+            a[1] = h2_sub((__byte_perm(xa[wd], xb[wd], sel1) & 0x00FF00FFu) ^ kH2Bias, kH2Bias);
+            a[2] = h2_sub((__byte_perm(xc[wd], xd[wd], sel0) & 0x00FF00FFu) ^ kH2Bias, kH2Bias);
+            a[3] = h2_sub((__byte_perm(xc[wd], xd[wd], sel1) & 0x00FF00FFu) ^ kH2Bias, kH2Bias);
+            const int j = 8 * i + jj;
+            mma_16816(acc[j], a, bh0, bh1);
+            mma_16816(acc[j], a, bl0, bl1);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < KS / 4; ++i) {  // 16 bytes per row = 8 halves = 4 dim tiles
+          const uint4 ra = *reinterpret_cast<const uint4*>(vb + 16 * i);
+          const uint4 rb = *reinterpret_cast<const uint4*>(vb + C::V_ROW + 16 * i);
+          const uint4 rc = *reinterpret_cast<const uint4*>(vb + 8 * C::V_ROW + 16 * i);
+          const uint4 rd = *reinterpret_cast<const uint4*>(vb + 9 * C::V_ROW + 16 * i);
+          const uint32_t xa[4] = {ra.x, ra.y, ra.z, ra.w}, xb[4] = {rb.x, rb.y, rb.z, rb.w};
+          const uint32_t xc[4] = {rc.x, rc.y, rc.z, rc.w}, xd[4] = {rd.x, rd.y, rd.z, rd.w};
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) {  // dim tile: half 0 of the word (row r), half 1 (row r+8)
+            uint32_t a[4];
+            a[0] = __byte_perm(xa[jj], xb[jj], 0x5410);
+            a[1] = __byte_perm(xa[jj], xb[jj], 0x7632);
+            a[2] = __byte_perm(xc[jj], xd[jj], 0x5410);
+            a[3] = __byte_perm(xc[jj], xd[jj], 0x7632);
+            const int j = 4 * i + jj;
+            mma_16816(acc[j], a, bh0, bh1);
+            mma_16816(acc[j], a, bl0, bl1);
+          }
+        }
+      }
+    }
+  }
+
+  // end of a segment: sum the lanes' partial softmax denominators over the token rows
+  __device__ __forceinline__ void finish() {
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      l_run[0] += __shfl_xor_sync(kFull, l_run[0], off);
+      l_run[1] += __shfl_xor_sync(kFull, l_run[1], off);
+    }
+  }
+
+  // this lane's outputs: heads 2c (acc[.][0], acc[.][2]) and 2c+1 (acc[.][1], acc[.][3]) at
+  // dims g*D/8 + 2j (+1)
+  __device__ __forceinline__ void write_out(const DecodeParams& p, int s, int hg) {
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int hh = 2 * c + e;
+      if (hh >= GT) continue;
+      const float inv = l_run[e] > 0.f ? 1.f / l_run[e] : 0.f;
+      __half2* o = reinterpret_cast<__half2*>(p.out + ((size_t)s * p.num_q_heads + (size_t)hg * GT + hh) * D + g * (D / 8));
+#pragma unroll
+      for (int j = 0; j < KS; ++j) o[j] = __floats2half2_rn(acc[j][e] * inv, acc[j][e + 2] * inv);
+    }
+  }
+
+  __device__ __forceinline__ void write_partial(const DecodeParams& p, long long slot, int lane) {
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int hh = 2 * c + e;
+      if (hh >= GT) continue;
+      float2* dst = reinterpret_cast<float2*>(p.ws_acc + ((size_t)slot * GT + hh) * D + g * (D / 8));
+#pragma unroll
+      for (int j = 0; j < KS; ++j) dst[j] = make_float2(acc[j][e], acc[j][e + 2]);
+      if (g == 0) {
+        p.ws_ml[((size_t)slot * GT + hh) * 2 + 0] = m_run[e];
+        p.ws_ml[((size_t)slot * GT + hh) * 2 + 1] = l_run[e];
+      }
+    }
+  }
+};
+
+template <int KT, int VT, int BS, int D, int GT>
+using EngineFor = typename std::conditional<Cfg<KT, VT, BS, D, GT>::MMA, MmaEngine<KT, VT, BS, D, GT>,
+                                            CoreEngine<KT, VT, BS, D, GT>>::type;
+
 template <int KT, int VT, int BS, int D, int GT>
 __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, BS, D, GT>::CTAS_PER_SM)
     paged_decode_kernel(const DecodeParams p) {
@@ -144,8 +620,6 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int c = lane % C::CH;   // 16-dim chunk of this lane
-  const int tg = lane / C::CH;  // token-row group of this lane
   const int W = gridDim.x * C::NW;
   const int w = blockIdx.x * C::NW + warp;
   const int HG = p.num_q_heads / GT;
@@ -300,71 +774,10 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
   load_meta(cur, rc);
   __syncwarp();  // barrier initialisation by lane 0 is visible to the warp
 
-  // ---- per-unit state ----
-  float2 qf[GT][8];
-  uint32_t qplane[GT][3][4];
-  float qinv[GT];
-  float m_run[GT], l_run[GT];
-  float2 acc[GT][8];
+  // ---- per-unit state: the arithmetic engine for GT query heads ----
+  EngineFor<KT, VT, BS, D, GT> eng;
   int seg_j0 = cur.j0;  // first block of the current segment within its unit
-
-  auto begin_unit = [&](const Win& a) {
-#pragma unroll
-    for (int hh = 0; hh < GT; ++hh) {
-      const __half* qp = p.q + ((size_t)a.s * p.num_q_heads + (size_t)a.hg * GT + hh) * D + c * 16;
-      const uint4 w0 = *reinterpret_cast<const uint4*>(qp);
-      const uint4 w1 = *reinterpret_cast<const uint4*>(qp + 8);
-      const uint32_t u[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-      for (int i = 0; i < 8; ++i) qf[hh][i] = __half22float2(*reinterpret_cast<const __half2*>(&u[i]));
-      m_run[hh] = kNegBig;
-      l_run[hh] = 0.f;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) acc[hh][j] = make_float2(0.f, 0.f);
-    }
-    // INT8 K: q . k is computed exactly in integers. Each head's q is put on a fixed-point grid
-    // of 2^-shift (22 bits below its largest magnitude; fp16 q loses nothing above 2^-22 of its
-    // max) and split into three signed byte planes, q_fixed = 2^16 b2 + 2^8 b1 + b0, so a
-    // 4-code word costs three dp4a with int32 accumulation and no code is converted to float.
-    if constexpr (KT == PKV_INT8_SYM) {
-#pragma unroll
-      for (int hh = 0; hh < GT; ++hh) {
-        float amax = 0.f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fmaxf(fabsf(qf[hh][i].x), fabsf(qf[hh][i].y)));
-#pragma unroll
-        for (int off = 1; off < C::CH; off <<= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, off));
-        int e = 0;
-        (void)frexpf(amax, &e);                    // amax < 2^e
-        const int shift = amax > 0.f ? 22 - e : 0;  // |q| * 2^shift < 2^22
-        const float up = __int_as_float((127 + shift) << 23);
-        qinv[hh] = __int_as_float((127 - shift) << 23);
-#pragma unroll
-        for (int wd = 0; wd < 4; ++wd) {
-          uint32_t p0 = 0, p1 = 0, p2 = 0;
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float2 pr = qf[hh][(4 * wd + k) / 2];
-            const int qi = __float2int_rn((((4 * wd + k) & 1) ? pr.y : pr.x) * up);
-            const int b0 = ((qi + 128) & 0xFF) - 128;
-            const int r1 = (qi - b0) >> 8;
-            const int b1 = ((r1 + 128) & 0xFF) - 128;
-            const int b2 = (r1 - b1) >> 8;
-            p0 |= (uint32_t)(b0 & 0xFF) << (8 * k);
-            p1 |= (uint32_t)(b1 & 0xFF) << (8 * k);
-            p2 |= (uint32_t)(b2 & 0xFF) << (8 * k);
-          }
-          qplane[hh][0][wd] = p0;
-          qplane[hh][1][wd] = p1;
-          qplane[hh][2][wd] = p2;
-        }
-      }
-    } else {
-#pragma unroll
-      for (int hh = 0; hh < GT; ++hh) qinv[hh] = 1.f;
-    }
-  };
-  begin_unit(cur);
+  eng.begin(p, cur.s, cur.hg, lane);
 
   // ---- the copy ring ----
   auto issue = [&](int st, int b, int g) {
@@ -410,7 +823,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
       nxt = next_win(cur);
       load_ids(nxt, rn);
       if (new_unit) {
-        begin_unit(cur);
+        eng.begin(p, cur.s, cur.hg, lane);
         seg_j0 = cur.j0;
       }
     }
@@ -427,101 +840,9 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
     const float ks = __shfl_sync(kFull, rc.ks, kw_i) * p.scale_log2;  // per-block K scale, log2 domain
     const float vs = __shfl_sync(kFull, rc.vs, kw_i);
     const float nzb = -(kMagic + __shfl_sync(kFull, rc.zp, kw_i));
-    const float2 neg_zp_bias = make_float2(nzb, nzb);
     const bool valid = __shfl_sync(kFull, rc.valid ? 1 : 0, kw_i) != 0;
-    const int tok0 = (cur.j0 + kw_i) * BS;
     const uint8_t* kt = my_stages + (size_t)st * C::STAGE;
-    const uint8_t* vt = kt + C::K_TILE;
-
-    float z[C::TPL][GT];
-#pragma unroll
-    for (int i = 0; i < C::TPL; ++i) {
-      const int row = tg + C::TG * i;
-      const uint8_t* krow = kt + row * C::K_ROW + c * (C::K_ROW / C::CH);
-      if constexpr (KT == PKV_INT8_SYM) {
-        const uint4 wv = *reinterpret_cast<const uint4*>(krow);
-        const int kw[4] = {(int)wv.x, (int)wv.y, (int)wv.z, (int)wv.w};
-#pragma unroll
-        for (int hh = 0; hh < GT; ++hh) {
-          int acc_p[3];
-#pragma unroll
-          for (int pl = 0; pl < 3; ++pl) {
-            int a = __dp4a((int)qplane[hh][pl][0], kw[0], 0);
-            a = __dp4a((int)qplane[hh][pl][1], kw[1], a);
-            a = __dp4a((int)qplane[hh][pl][2], kw[2], a);
-            acc_p[pl] = __dp4a((int)qplane[hh][pl][3], kw[3], a);
-          }
-          // |acc_p| < 2^18: the low two planes combine exactly in int32, the top one in fp32
-          z[i][hh] = __fmaf_rn((float)acc_p[2], 65536.f, (float)(acc_p[1] * 256 + acc_p[0]));
-        }
-      } else {
-        float2 kf[8];
-        load_h16(krow, kf);
-#pragma unroll
-        for (int hh = 0; hh < GT; ++hh) {
-          float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
-#pragma unroll
-          for (int j = 0; j < 8; j += 2) {
-            a0 = __ffma2_rn(qf[hh][j], kf[j], a0);
-            a1 = __ffma2_rn(qf[hh][j + 1], kf[j + 1], a1);
-          }
-          z[i][hh] = (a0.x + a0.y) + (a1.x + a1.y);
-        }
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < C::TPL; ++i)
-#pragma unroll
-      for (int hh = 0; hh < GT; ++hh)
-#pragma unroll
-        for (int off = 1; off < C::CH; off <<= 1) z[i][hh] += __shfl_xor_sync(kFull, z[i][hh], off);
-
-    float pv[C::TPL][GT];
-#pragma unroll
-    for (int hh = 0; hh < GT; ++hh) {
-      const float zscale = (KT == PKV_FP16) ? p.scale_log2 : ks * qinv[hh];
-      float mloc = -INFINITY;
-#pragma unroll
-      for (int i = 0; i < C::TPL; ++i) {
-        const int t = tok0 + tg + C::TG * i;
-        float zz = z[i][hh] * zscale;
-        zz = (valid && t < cur.L) ? zz : -INFINITY;
-        z[i][hh] = zz;
-        mloc = fmaxf(mloc, zz);
-      }
-#pragma unroll
-      for (int off = C::CH; off < 32; off <<= 1) mloc = fmaxf(mloc, __shfl_xor_sync(kFull, mloc, off));
-      // the running max is warp-uniform; rescale only when it grows (rare after the first blocks)
-      if (mloc > m_run[hh]) {
-        const float alpha = ex2(m_run[hh] - mloc);
-        m_run[hh] = mloc;
-        l_run[hh] *= alpha;
-        const float2 alpha2 = make_float2(alpha, alpha);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[hh][j] = __fmul2_rn(acc[hh][j], alpha2);
-      }
-      const float m_new = m_run[hh];
-      float lsum = 0.f;
-#pragma unroll
-      for (int i = 0; i < C::TPL; ++i) {
-        const float pr = ex2(z[i][hh] - m_new);
-        lsum += pr;
-        pv[i][hh] = (VT == PKV_FP16) ? pr : pr * vs;
-      }
-      l_run[hh] += lsum;
-    }
-#pragma unroll
-    for (int i = 0; i < C::TPL; ++i) {
-      const int row = tg + C::TG * i;
-      float2 vf[8];
-      load_v16<VT>(vt + row * C::V_ROW + c * (C::V_ROW / C::CH), neg_zp_bias, vf);
-#pragma unroll
-      for (int hh = 0; hh < GT; ++hh) {
-        const float2 pv2 = make_float2(pv[i][hh], pv[i][hh]);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[hh][j] = __ffma2_rn(pv2, vf[j], acc[hh][j]);
-      }
-    }
+    eng.block(kt, kt + C::K_TILE, ks, vs, nzb, valid, (cur.j0 + kw_i) * BS, cur.L, p.scale_log2);
     __syncwarp();  // the stage's reads are complete (their values were consumed above)
     ++cpos;
     if (++cst == C::NS) {
@@ -532,50 +853,13 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
     // ---- end of a segment: the unit's last block, or the end of this warp's range ----
     const int j_end = cur.j0 + kw_i + 1;
     if (j_end == cur.nblk || cpos == n_total) {
-#pragma unroll
-      for (int hh = 0; hh < GT; ++hh) {
-#pragma unroll
-        for (int off = C::CH; off < 32; off <<= 1) l_run[hh] += __shfl_xor_sync(kFull, l_run[hh], off);
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-#pragma unroll
-          for (int off = C::CH; off < 32; off <<= 1) {
-            acc[hh][j].x += __shfl_xor_sync(kFull, acc[hh][j].x, off);
-            acc[hh][j].y += __shfl_xor_sync(kFull, acc[hh][j].y, off);
-          }
-      }
+      eng.finish();
       const long long u = (long long)cur.s * HG + cur.hg;
       if (seg_j0 == 0 && j_end == cur.nblk) {
-        // the whole unit was processed by this warp: write the output
-        if (tg == 0) {
-#pragma unroll
-          for (int hh = 0; hh < GT; ++hh) {
-            const float inv = l_run[hh] > 0.f ? 1.f / l_run[hh] : 0.f;
-            __half2* o = reinterpret_cast<__half2*>(
-                p.out + ((size_t)cur.s * p.num_q_heads + (size_t)cur.hg * GT + hh) * D + c * 16);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) o[j] = __floats2half2_rn(acc[hh][j].x * inv, acc[hh][j].y * inv);
-          }
-        }
+        eng.write_out(p, cur.s, cur.hg);  // the whole unit was processed by this warp
       } else {
         // one segment of a split unit: publish the partial; the last warp to finish merges
-        const long long slot = u + w;
-        if (tg == 0) {
-#pragma unroll
-          for (int hh = 0; hh < GT; ++hh) {
-            float4* dst = reinterpret_cast<float4*>(p.ws_acc + ((size_t)slot * GT + hh) * D + c * 16);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              dst[j] = make_float4(acc[hh][2 * j].x, acc[hh][2 * j].y, acc[hh][2 * j + 1].x, acc[hh][2 * j + 1].y);
-          }
-        }
-        if (lane == 0) {
-#pragma unroll
-          for (int hh = 0; hh < GT; ++hh) {
-            p.ws_ml[((size_t)slot * GT + hh) * 2 + 0] = m_run[hh];
-            p.ws_ml[((size_t)slot * GT + hh) * 2 + 1] = l_run[hh];
-          }
-        }
+        eng.write_partial(p, u + w, lane);
         const long long unit_p0 = cur.seq_p0 + (long long)cur.hg * cur.nblk;
         const int w_first = owner_of(unit_p0, T, We);
         const int w_last = owner_of(unit_p0 + cur.nblk - 1, T, We);
@@ -602,13 +886,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
           }
         }
       }
-#pragma unroll
-      for (int hh = 0; hh < GT; ++hh) {
-        m_run[hh] = kNegBig;
-        l_run[hh] = 0.f;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[hh][j] = make_float2(0.f, 0.f);
-      }
+      eng.reset();
       seg_j0 = j_end;  // (a new unit restarts it at its first block)
     }
   }
@@ -660,12 +938,25 @@ bool info_one(DecodeKernelInfo* info) {
   return true;
 }
 
+// 8 heads per warp exist only with the tensor-core engine
+template <int KT, int VT, int BS, int D>
+cudaError_t launch_one8(const DecodeParams& p, const DecodeShape& sh, cudaStream_t stream) {
+  if constexpr (Cfg<KT, VT, BS, D, 8>::MMA) return launch_one<KT, VT, BS, D, 8>(p, sh, stream);
+  else return cudaErrorInvalidValue;
+}
+template <int KT, int VT, int BS, int D>
+bool info_one8(DecodeKernelInfo* info) {
+  if constexpr (Cfg<KT, VT, BS, D, 8>::MMA) return info_one<KT, VT, BS, D, 8>(info);
+  else return false;
+}
+
 // FN<KT, VT, BS, D, GT>(args...) for the instantiation matching `sh`
 #define PKV_DISPATCH_GT(KT, VT, BS, D, FN, ...)       \
   switch (sh.heads_per_warp) {                        \
     case 1: return FN<KT, VT, BS, D, 1>(__VA_ARGS__); \
     case 2: return FN<KT, VT, BS, D, 2>(__VA_ARGS__); \
     case 4: return FN<KT, VT, BS, D, 4>(__VA_ARGS__); \
+    case 8: return FN##8<KT, VT, BS, D>(__VA_ARGS__); \
     default: break;                                   \
   }
 #define PKV_DISPATCH_D(KT, VT, BS, FN, ...)                   \
@@ -692,7 +983,10 @@ bool info_one(DecodeKernelInfo* info) {
 
 }  // namespace
 
-int32_t decode_heads_per_warp(int32_t group) {
+int32_t decode_heads_per_warp(int32_t group, int32_t k_dtype, int32_t v_dtype, int32_t head_dim) {
+  const bool mma = (k_dtype == PKV_INT8_SYM && v_dtype == PKV_INT8_SYM && head_dim >= 128) ||
+                   (k_dtype == PKV_FP16 && v_dtype == PKV_FP16);
+  if (mma && group % 8 == 0) return 8;
   if (group % 4 == 0) return 4;
   if (group % 2 == 0) return 2;
   return 1;

@@ -47,8 +47,9 @@ struct DecodeKernelInfo {
   int32_t stages;       // copy-ring depth per warp
 };
 
-// Query heads handled together by one warp (largest of 4, 2, 1 that divides the group).
-int32_t decode_heads_per_warp(int32_t group);
+// Query heads handled together by one warp: 8 (tensor cores, when the dtypes allow) or the
+// largest of 4, 2, 1 that divides the group.
+int32_t decode_heads_per_warp(int32_t group, int32_t k_dtype, int32_t v_dtype, int32_t head_dim);
 bool decode_supported(int32_t k_dtype, int32_t v_dtype, int32_t block_size, int32_t head_dim);
 // Static launch facts of the kernel instantiation for `sh` (no device needed); false if none.
 bool decode_kernel_info(const DecodeShape& sh, DecodeKernelInfo* info);
