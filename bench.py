@@ -173,13 +173,12 @@ class L2Flush:
         l2 = torch.cuda.get_device_properties(dev).L2_cache_size
         n = max(2 * l2, 256 << 20)
         self.wbuf = torch.empty(n, dtype=torch.uint8, device=dev)
-        self.rbuf = torch.ones(n // 4, dtype=torch.int32, device=dev)
-        self.sink = torch.empty((), dtype=torch.int64, device=dev)
+        self.rbuf = torch.ones(n // 4, dtype=torch.float32, device=dev)
+        self.sink = torch.empty((), dtype=torch.float32, device=dev)
 
     def __call__(self):
-        import torch
         self.wbuf.zero_()
-        self.sink.copy_(self.rbuf.sum(dtype=torch.int64))
+        self.sink.copy_(self.rbuf.sum())
 
 
 

@@ -295,8 +295,48 @@ __device__ bool fast_sym(const float x[8], int vpl, int8_t* tile, float* scale_p
         fits = fits && (r <= 127 && r >= -127);
       }
     }
-    if (!__all_sync(kFull, fits)) return false;
-    s = s_old;
+    if (!__all_sync(kFull, fits)) {
+      if (vpl > 4) return false;  // head_dim 256: the general path rebuilds
+      // rebuild in registers: the lane's codes of every old row in one batch of loads, then
+      // x_hat = code * s_old in binary32, a scale covering old and new values, requantize
+      uint32_t oldw[32];
+#pragma unroll
+      for (int r = 0; r < 32; ++r) {
+        oldw[r] = 0;
+        if (r < o0) {
+          const int8_t* src = tile + (size_t)r * d + lane * vpl;
+          oldw[r] = (vpl == 4) ? *reinterpret_cast<const uint32_t*>(src) : *reinterpret_cast<const uint16_t*>(src);
+        }
+      }
+      float m_old = 0.0f;
+#pragma unroll
+      for (int r = 0; r < 32; ++r)
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (r < o0 && i < vpl) {
+            const int q = (int)(int8_t)((oldw[r] >> (8 * i)) & 0xff);
+            m_old = fmaxf(m_old, fabsf(__fmul_rn((float)q, s_old)));
+          }
+      m_old = warp_max(m_old);
+      s = __fdiv_rn(fmaxf(m_old, m), 127.0f);
+#pragma unroll
+      for (int r = 0; r < 32; ++r) {
+        if (r >= o0) continue;
+        uint32_t out = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (i < vpl) {
+            const int q = (int)(int8_t)((oldw[r] >> (8 * i)) & 0xff);
+            out |= ((uint32_t)(quant_sym(__fmul_rn((float)q, s_old), s) & 0xff)) << (8 * i);
+          }
+        int8_t* dst = tile + (size_t)r * d + lane * vpl;
+        if (vpl == 4) *reinterpret_cast<uint32_t*>(dst) = out;
+        else *reinterpret_cast<uint16_t*>(dst) = (uint16_t)out;
+      }
+      if (lane == 0) *scale_ptr = s;  // the new token's codes below use the rebuilt scale
+    } else {
+      s = s_old;
+    }
   }
   uint32_t lo = 0, hi = 0;
 #pragma unroll
@@ -341,9 +381,61 @@ __device__ bool fast_asym4(const float x[8], int vpl, uint8_t* tile, float* scal
         fits = fits && (r >= 0 && r <= 15);
       }
     }
-    if (!__all_sync(kFull, fits)) return false;
-    s = s_old;
-    zp = zp_old;
+    if (!__all_sync(kFull, fits)) {
+      if (vpl > 4) return false;  // head_dim 256: the general path rebuilds
+      // rebuild in registers: old nibbles of every row in one batch of loads; range over
+      // x_hat = (code - zp_old) * s_old (binary32) and the new values; requantize everything
+      uint32_t oldw[32];
+#pragma unroll
+      for (int r = 0; r < 32; ++r) {
+        oldw[r] = 0;
+        if (r < o0) {
+          const uint8_t* src = tile + (size_t)r * (d / 2) + lane * (vpl / 2);
+          oldw[r] = (vpl == 4) ? *reinterpret_cast<const uint16_t*>(src) : *src;
+        }
+      }
+      float lo = 0.0f, hi = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (i >= vpl) continue;
+        lo = fminf(lo, x[i]);
+        hi = fmaxf(hi, x[i]);
+      }
+#pragma unroll
+      for (int r = 0; r < 32; ++r)
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (r < o0 && i < vpl) {
+            const int q = (int)((oldw[r] >> (4 * i)) & 0xF);
+            const float v = __fmul_rn((float)(q - zp_old), s_old);
+            lo = fminf(lo, v);
+            hi = fmaxf(hi, v);
+          }
+      lo = warp_min(lo);
+      hi = warp_max(hi);
+      derive_asym(lo, hi, s, zp);
+#pragma unroll
+      for (int r = 0; r < 32; ++r) {
+        if (r >= o0) continue;
+        uint32_t out = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (i < vpl) {
+            const int q = (int)((oldw[r] >> (4 * i)) & 0xF);
+            out |= (uint32_t)quant_asym(__fmul_rn((float)(q - zp_old), s_old), s, zp) << (4 * i);
+          }
+        uint8_t* dst = tile + (size_t)r * (d / 2) + lane * (vpl / 2);
+        if (vpl == 4) *reinterpret_cast<uint16_t*>(dst) = (uint16_t)out;
+        else *dst = (uint8_t)out;
+      }
+      if (lane == 0) {
+        *scale_ptr = s;
+        *zp_ptr = (uint8_t)zp;
+      }
+    } else {
+      s = s_old;
+      zp = zp_old;
+    }
   }
   uint32_t packed = 0;  // vpl / 2 bytes: byte j = code[2j] | code[2j+1] << 4
 #pragma unroll
