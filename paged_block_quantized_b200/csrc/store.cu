@@ -13,7 +13,14 @@
 //
 // Bit-exactness: every arithmetic step is an explicit IEEE binary32 round-to-nearest intrinsic
 // (__fdiv_rn, __fmul_rn, __fadd_rn, __fsub_rn) so nvcc cannot contract or reorder it, and
-// __float2int_rn rounds half to even. Maxima and minima are order independent.
+// __float2int_rn rounds half to even. Maxima and minima are order independent. Two shortcuts
+// give the same results as the element-wise rule, because every step involved (x / s, + zp,
+// code * s, rint) is monotone for s >= 0 and round-to-nearest is symmetric about zero:
+//  - "every new value fits" is decided from the extremes alone: |x| <= m gives
+//    |rint(x / s)| <= rint(m / s), and lo <= x <= hi brackets rint(x / s + zp);
+//  - a rebuild's range over the dequantized old values comes from the largest |code| (INT8) or
+//    the smallest and largest code (INT4), and requantizing an old code depends on the code
+//    alone, so each tile's old codes go through a 256-entry table built once per rebuild.
 //
 // Work split: one warp per (token, KV head). The warp of the first token of a group (the run of
 // tokens bound for one block) does the whole group; the others return at once.
@@ -69,6 +76,184 @@ __device__ __forceinline__ void derive_asym(float lo, float hi, float& s, int& z
   if (s != 0.0f) zp = min(15, max(0, __float2int_rn(__fdiv_rn(-lo, s))));
 }
 
+// Do new values with largest magnitude m all fit a stored INT8 scale? (|rint(m / s)| <= 127; a zero
+// scale holds zeros only)
+__device__ __forceinline__ bool fits_sym(float m, float s_old) {
+  if (s_old == 0.0f) return m == 0.0f;
+  return __float2int_rn(__fdiv_rn(m, s_old)) <= 127;
+}
+
+// Do new values in [lo, hi] all fit a stored INT4 scale and zero point?
+__device__ __forceinline__ bool fits_asym(float lo, float hi, float s_old, int zp_old) {
+  if (s_old == 0.0f) return lo == 0.0f && hi == 0.0f;
+  const int r_lo = __float2int_rn(__fadd_rn(__fdiv_rn(lo, s_old), (float)zp_old));
+  const int r_hi = __float2int_rn(__fadd_rn(__fdiv_rn(hi, s_old), (float)zp_old));
+  return r_lo >= 0 && r_hi <= 15;
+}
+
+// four bytes of w through a 256-entry table (after xor-ing w with flip)
+__device__ __forceinline__ uint32_t translate4(uint32_t w, uint32_t flip, const uint8_t* tbl) {
+  const uint32_t x = w ^ flip;
+  return (uint32_t)tbl[x & 0xffu] | ((uint32_t)tbl[(x >> 8) & 0xffu] << 8) |
+         ((uint32_t)tbl[(x >> 16) & 0xffu] << 16) | ((uint32_t)tbl[x >> 24] << 24);
+}
+__device__ __forceinline__ uint4 translate16(uint4 v, uint32_t flip, const uint8_t* tbl) {
+  return make_uint4(translate4(v.x, flip, tbl), translate4(v.y, flip, tbl), translate4(v.z, flip, tbl),
+                    translate4(v.w, flip, tbl));
+}
+
+// Per-byte comparisons of four packed values in 0 .. 15 (one per byte): (a | 16) - b keeps each
+// byte in 1 .. 31 (no borrow into the next byte), and its bit 4 says a >= b.
+__device__ __forceinline__ uint32_t nibble_ge(uint32_t a, uint32_t b) {
+  return (((a | 0x10101010u) - b) >> 4 & 0x01010101u) * 0xFFu;  // 0xFF in each byte where a >= b
+}
+__device__ __forceinline__ uint32_t bitsel(uint32_t m, uint32_t a, uint32_t b) { return (a & m) | (b & ~m); }
+
+// largest |code| among the 16 INT8 codes of v
+__device__ __forceinline__ int32_t absmax16(uint4 v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  int32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int32_t x = (int32_t)w[i];
+    m = max(m, max(max(abs((int32_t)(int8_t)x), abs((int32_t)(int8_t)(x >> 8))),
+                   max(abs((int32_t)(int8_t)(x >> 16)), abs(x >> 24))));
+  }
+  return m;
+}
+
+// per-byte smallest / largest of the 32 nibble codes of v, folded into mn / mx
+__device__ __forceinline__ void nibble_minmax32(uint4 v, uint32_t& mn, uint32_t& mx) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t l4 = w[i] & 0x0F0F0F0Fu, h4 = (w[i] >> 4) & 0x0F0F0F0Fu;
+    const uint32_t ge = nibble_ge(l4, h4);
+    const uint32_t hi = bitsel(ge, l4, h4), lo = bitsel(ge, h4, l4);
+    mx = bitsel(nibble_ge(mx, hi), mx, hi);
+    mn = bitsel(nibble_ge(mn, lo), lo, mn);
+  }
+}
+
+// A rebuild reads a tile's old rows as 16-byte vectors, kChunkVecs at a time: vector e of chunk c
+// is c * kChunkVecs + j * 32 + lane for j < 4, so each j is one coalesced 512-byte access and the
+// four loads of a chunk are in flight together. The per-vector work runs in a loop that is not
+// unrolled, over v[0] with the registers rotated, which keeps the code small.
+constexpr int kChunkVecs = 128;
+
+__device__ __forceinline__ void load_chunk(const uint4* v16, int nvec, int c, int lane, uint4 v[4]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int e = c * kChunkVecs + j * 32 + lane;
+    v[j] = e < nvec ? v16[e] : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+__device__ __forceinline__ void rotate(uint4 v[4]) {
+  const uint4 t = v[0];
+  v[0] = v[1];
+  v[1] = v[2];
+  v[2] = v[3];
+  v[3] = t;
+}
+
+// Requantize the old rows in place through tbl: chunks again (a single chunk is still in v).
+__device__ __forceinline__ void requant_rows(uint4* v16, int nvec, int nchunks, uint32_t flip, const uint8_t* tbl,
+                                             int lane, uint4 v[4]) {
+#pragma unroll 1
+  for (int c = 0; c < nchunks; ++c) {
+    if (nchunks > 1) load_chunk(v16, nvec, c, lane, v);
+#pragma unroll 1
+    for (int j = 0; j < 4; ++j) {
+      const int e = c * kChunkVecs + j * 32 + lane;
+      if (e < nvec) v16[e] = translate16(v[0], flip, tbl);
+      rotate(v);
+    }
+  }
+}
+
+// Rebuild of the old rows [0, o0) of an INT8 tile (rows of d codes) for values that do not fit
+// the stored scale s_old: x_hat = code * s_old (binary32), new scale = max(max |x_hat|, m_new) / 127,
+// old codes requantized to it. Returns the new scale. tbl: 256 bytes of this warp's shared memory.
+__device__ __noinline__ float rebuild_sym(int8_t* tile, int d, int o0, float s_old, float m_new, uint8_t* tbl, int lane) {
+  uint4* v16 = reinterpret_cast<uint4*>(tile);
+  const int nvec = o0 * d / 16;
+  const int nchunks = (nvec + kChunkVecs - 1) / kChunkVecs;
+  uint4 v[4];
+  int32_t amax = 0;  // largest |code| (vectors past the end read as zeros)
+#pragma unroll 1
+  for (int c = 0; c < nchunks; ++c) {
+    load_chunk(v16, nvec, c, lane, v);
+#pragma unroll 1
+    for (int j = 0; j < 4; ++j) {
+      amax = max(amax, absmax16(v[0]));
+      rotate(v);
+    }
+  }
+  const int32_t qmax = __reduce_max_sync(kFull, amax);
+  const float m_old = __fmul_rn((float)qmax, s_old);
+  const float s = __fdiv_rn(fmaxf(m_old, m_new), 127.0f);
+  // table entry (code + 128): the code's requantized value; lane l fills entries 8l .. 8l+7
+  uint32_t lo = 0, hi = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int code = lane * 8 + j - 128;
+    const uint32_t c = (uint32_t)(quant_sym(__fmul_rn((float)code, s_old), s) & 0xff);
+    if (j < 4) lo |= c << (8 * j); else hi |= c << (8 * (j - 4));
+  }
+  reinterpret_cast<uint2*>(tbl)[lane] = make_uint2(lo, hi);
+  __syncwarp();
+  requant_rows(v16, nvec, nchunks, 0x80808080u, tbl, lane, v);  // byte b holds code (int8)b: entry b ^ 0x80
+  __syncwarp();
+  return s;
+}
+
+// Rebuild of the old rows [0, o0) of an INT4 tile (rows of d / 2 bytes) for values that do not
+// fit: x_hat = (code - zp_old) * s_old (binary32), range [min(lo_new, x_hat), max(hi_new, x_hat)],
+// new scale and zero point from it, old codes requantized. tbl: 256 bytes of shared memory.
+__device__ __noinline__ void rebuild_asym4(uint8_t* tile, int d, int o0, float s_old, int zp_old, float lo_new,
+                                           float hi_new, uint8_t* tbl, int lane, float& s_out, int& zp_out) {
+  uint4* v16 = reinterpret_cast<uint4*>(tile);
+  const int nvec = o0 * d / 32;
+  const int nchunks = (nvec + kChunkVecs - 1) / kChunkVecs;
+  uint4 v[4];
+  uint32_t mn = 0x0F0F0F0Fu, mx = 0u;  // per byte: smallest / largest code seen
+#pragma unroll 1
+  for (int c = 0; c < nchunks; ++c) {
+    load_chunk(v16, nvec, c, lane, v);
+#pragma unroll 1
+    for (int j = 0; j < 4; ++j) {
+      if (c * kChunkVecs + j * 32 + lane < nvec) nibble_minmax32(v[0], mn, mx);
+      rotate(v);
+    }
+  }
+  // a lane with no old vectors keeps 15 / 0, which leave the warp's minimum / maximum alone
+  const uint32_t qmin =
+      __reduce_min_sync(kFull, min(min(mn & 0xffu, (mn >> 8) & 0xffu), min((mn >> 16) & 0xffu, mn >> 24)));
+  const uint32_t qmax =
+      __reduce_max_sync(kFull, max(max(mx & 0xffu, (mx >> 8) & 0xffu), max((mx >> 16) & 0xffu, mx >> 24)));
+  const float lo = fminf(lo_new, __fmul_rn((float)((int)qmin - zp_old), s_old));
+  const float hi = fmaxf(hi_new, __fmul_rn((float)((int)qmax - zp_old), s_old));
+  float s;
+  int zp;
+  derive_asym(lo, hi, s, zp);
+  // lane k < 16: requantized value of code k; byte table entry b = T[b & 15] | T[b >> 4] << 4
+  const int t_k = quant_asym(__fmul_rn((float)((lane & 15) - zp_old), s_old), s, zp);
+  const uint32_t t_hi = (uint32_t)__shfl_sync(kFull, t_k, lane >> 1);  // b >> 4 for b = 8 lane + j
+  uint32_t lo_w = 0, hi_w = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t t_lo = (uint32_t)__shfl_sync(kFull, t_k, (lane * 8 + j) & 15);
+    const uint32_t c = t_lo | (t_hi << 4);
+    if (j < 4) lo_w |= c << (8 * j); else hi_w |= c << (8 * (j - 4));
+  }
+  reinterpret_cast<uint2*>(tbl)[lane] = make_uint2(lo_w, hi_w);
+  __syncwarp();
+  requant_rows(v16, nvec, nchunks, 0u, tbl, lane, v);
+  __syncwarp();
+  s_out = s;
+  zp_out = zp;
+}
+
 // Values of the group for one head: element e of token i at src + i * row_stride + e.
 struct GroupSrc {
   const __half* base;  // token 0 of the group, this head
@@ -77,8 +262,9 @@ struct GroupSrc {
   int d;               // head_dim
 };
 
-// ---- INT8 symmetric side of one (block, head) tile ----
-__device__ void store_sym(const GroupSrc& src, int8_t* tile, float* scale_ptr, int o0, int lane) {
+// ---- groups of several tokens (prefill chunks): INT8 symmetric side of one (block, head) tile ----
+__device__ __noinline__ void store_sym(const GroupSrc& src, int8_t* tile, float* scale_ptr, int o0, uint8_t* tbl,
+                                       int lane) {
   const int d = src.d, n = src.n;
   const int quads = n * d / 4;
   float m_new = 0.0f;
@@ -90,58 +276,13 @@ __device__ void store_sym(const GroupSrc& src, int8_t* tile, float* scale_ptr, i
     for (int u = 0; u < 4; ++u) m_new = fmaxf(m_new, fabsf(f[u]));
   }
   m_new = warp_max(m_new);
-
   float s;
   if (o0 == 0) {
     s = __fdiv_rn(m_new, 127.0f);
   } else {
     const float s_old = *scale_ptr;
-    bool fits = true;
-    for (int e = lane; e < quads; e += 32) {
-      const int i = (4 * e) / d, j = (4 * e) % d;
-      float f[4];
-      load4(src.base + i * src.row_stride + j, f);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        if (s_old == 0.0f) {
-          fits = fits && (f[u] == 0.0f);
-        } else {
-          const int r = __float2int_rn(__fdiv_rn(f[u], s_old));
-          fits = fits && (r <= 127 && r >= -127);
-        }
-      }
-    }
-    fits = __all_sync(kFull, fits);
-    if (fits) {
-      s = s_old;
-    } else {
-      // rebuild: old codes -> binary32 x_hat = code * s_old; scale from old and new together
-      const int old_quads = o0 * d / 4;
-      float m_old = 0.0f;
-      for (int e = lane; e < old_quads; e += 32) {
-        const uint32_t w = reinterpret_cast<const uint32_t*>(tile)[e];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int q = (int)(int8_t)((w >> (8 * u)) & 0xff);
-          m_old = fmaxf(m_old, fabsf(__fmul_rn((float)q, s_old)));
-        }
-      }
-      m_old = warp_max(m_old);
-      s = __fdiv_rn(fmaxf(m_old, m_new), 127.0f);
-      for (int e = lane; e < old_quads; e += 32) {
-        uint32_t w = reinterpret_cast<const uint32_t*>(tile)[e];
-        uint32_t out = 0;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int q = (int)(int8_t)((w >> (8 * u)) & 0xff);
-          const int r = quant_sym(__fmul_rn((float)q, s_old), s);
-          out |= ((uint32_t)(r & 0xff)) << (8 * u);
-        }
-        reinterpret_cast<uint32_t*>(tile)[e] = out;
-      }
-    }
+    s = fits_sym(m_new, s_old) ? s_old : rebuild_sym(tile, d, o0, s_old, m_new, tbl, lane);
   }
-  // new codes
   int8_t* dst = tile + (size_t)o0 * d;
   for (int e = lane; e < quads; e += 32) {
     const int i = (4 * e) / d, j = (4 * e) % d;
@@ -156,8 +297,8 @@ __device__ void store_sym(const GroupSrc& src, int8_t* tile, float* scale_ptr, i
 }
 
 // ---- INT4 asymmetric side: tile is [bs][d/2] bytes, byte j = code[2j] | code[2j+1] << 4 ----
-__device__ void store_asym4(const GroupSrc& src, uint8_t* tile, float* scale_ptr, uint8_t* zp_ptr, int o0,
-                            int lane) {
+__device__ __noinline__ void store_asym4(const GroupSrc& src, uint8_t* tile, float* scale_ptr, uint8_t* zp_ptr, int o0,
+                                         uint8_t* tbl, int lane) {
   const int d = src.d, n = src.n;
   const int quads = n * d / 4;  // 4 values -> 2 bytes
   float lo = 0.0f, hi = 0.0f;
@@ -173,7 +314,6 @@ __device__ void store_asym4(const GroupSrc& src, uint8_t* tile, float* scale_ptr
   }
   lo = warp_min(lo);
   hi = warp_max(hi);
-
   float s;
   int zp;
   if (o0 == 0) {
@@ -181,44 +321,11 @@ __device__ void store_asym4(const GroupSrc& src, uint8_t* tile, float* scale_ptr
   } else {
     const float s_old = *scale_ptr;
     const int zp_old = *zp_ptr;
-    bool fits = true;
-    for (int e = lane; e < quads; e += 32) {
-      const int i = (4 * e) / d, j = (4 * e) % d;
-      float f[4];
-      load4(src.base + i * src.row_stride + j, f);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        if (s_old == 0.0f) {
-          fits = fits && (f[u] == 0.0f);
-        } else {
-          const int r = __float2int_rn(__fadd_rn(__fdiv_rn(f[u], s_old), (float)zp_old));
-          fits = fits && (r >= 0 && r <= 15);
-        }
-      }
-    }
-    fits = __all_sync(kFull, fits);
-    if (fits) {
+    if (fits_asym(lo, hi, s_old, zp_old)) {
       s = s_old;
       zp = zp_old;
     } else {
-      // rebuild: x_hat = (code - zp_old) * s_old in binary32; range over old and new values
-      const int old_bytes = o0 * d / 2;
-      for (int e = lane; e < old_bytes; e += 32) {
-        const uint8_t byte = tile[e];
-        const float a = __fmul_rn((float)((int)(byte & 0xF) - zp_old), s_old);
-        const float b = __fmul_rn((float)((int)(byte >> 4) - zp_old), s_old);
-        lo = fminf(lo, fminf(a, b));
-        hi = fmaxf(hi, fmaxf(a, b));
-      }
-      lo = warp_min(lo);
-      hi = warp_max(hi);
-      derive_asym(lo, hi, s, zp);
-      for (int e = lane; e < old_bytes; e += 32) {
-        const uint8_t byte = tile[e];
-        const float a = __fmul_rn((float)((int)(byte & 0xF) - zp_old), s_old);
-        const float b = __fmul_rn((float)((int)(byte >> 4) - zp_old), s_old);
-        tile[e] = (uint8_t)(quant_asym(a, s, zp) | (quant_asym(b, s, zp) << 4));
-      }
+      rebuild_asym4(tile, d, o0, s_old, zp_old, lo, hi, tbl, lane, s, zp);
     }
   }
   uint8_t* dst = tile + (size_t)o0 * (d / 2);
@@ -237,7 +344,7 @@ __device__ void store_asym4(const GroupSrc& src, uint8_t* tile, float* scale_ptr
 }
 
 // ---- FP16 side: values stored as given ----
-__device__ void store_fp16(const GroupSrc& src, __half* tile, int o0, int lane) {
+__device__ __noinline__ void store_fp16(const GroupSrc& src, __half* tile, int o0, int lane) {
   const int d = src.d, n = src.n;
   const int vecs = n * d / 8;  // 16-byte vectors
   __half* dst = tile + (size_t)o0 * d;
@@ -248,7 +355,7 @@ __device__ void store_fp16(const GroupSrc& src, __half* tile, int o0, int lane) 
   }
 }
 
-// ---- single-token groups (the decode-step append): everything in registers ----
+// ---- single-token groups (the decode-step append): the token in registers ----
 // A lane holds vpl = head_dim / 32 consecutive values (2, 4 or 8) of the token for one head.
 __device__ __forceinline__ void load_halves(const __half* src, int vpl, uint32_t raw[4]) {
   raw[0] = raw[1] = raw[2] = raw[3] = 0;
@@ -271,72 +378,23 @@ __device__ __forceinline__ void halves_to_float(const uint32_t raw[4], float x[8
   }
 }
 
-// INT8 symmetric side of a one-token group at offset o0. Returns false (nothing written) when the
-// token does not fit the stored scale: the caller then takes the general path (rebuild).
-__device__ bool fast_sym(const float x[8], int vpl, int8_t* tile, float* scale_ptr, float s_old, int o0, int d,
-                         int lane) {
+// INT8 symmetric side of a one-token group at offset o0 (s_old: the stored scale when o0 > 0).
+__device__ __forceinline__ void append_sym(const float x[8], int vpl, int8_t* tile, float* scale_ptr, float s_old,
+                                          int o0, int d, uint8_t* tbl, int lane) {
   float m = 0.0f;
 #pragma unroll
   for (int i = 0; i < 8; ++i)
     if (i < vpl) m = fmaxf(m, fabsf(x[i]));
   m = warp_max(m);
   float s;
+  bool set_scale = true;
   if (o0 == 0) {
     s = __fdiv_rn(m, 127.0f);
+  } else if (fits_sym(m, s_old)) {
+    s = s_old;
+    set_scale = false;
   } else {
-    bool fits = true;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (i >= vpl) continue;
-      if (s_old == 0.0f) {
-        fits = fits && (x[i] == 0.0f);
-      } else {
-        const int r = __float2int_rn(__fdiv_rn(x[i], s_old));
-        fits = fits && (r <= 127 && r >= -127);
-      }
-    }
-    if (!__all_sync(kFull, fits)) {
-      if (vpl > 4) return false;  // head_dim 256: the general path rebuilds
-      // rebuild in registers: the lane's codes of every old row in one batch of loads, then
-      // x_hat = code * s_old in binary32, a scale covering old and new values, requantize
-      uint32_t oldw[32];
-#pragma unroll
-      for (int r = 0; r < 32; ++r) {
-        oldw[r] = 0;
-        if (r < o0) {
-          const int8_t* src = tile + (size_t)r * d + lane * vpl;
-          oldw[r] = (vpl == 4) ? *reinterpret_cast<const uint32_t*>(src) : *reinterpret_cast<const uint16_t*>(src);
-        }
-      }
-      float m_old = 0.0f;
-#pragma unroll
-      for (int r = 0; r < 32; ++r)
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          if (r < o0 && i < vpl) {
-            const int q = (int)(int8_t)((oldw[r] >> (8 * i)) & 0xff);
-            m_old = fmaxf(m_old, fabsf(__fmul_rn((float)q, s_old)));
-          }
-      m_old = warp_max(m_old);
-      s = __fdiv_rn(fmaxf(m_old, m), 127.0f);
-#pragma unroll
-      for (int r = 0; r < 32; ++r) {
-        if (r >= o0) continue;
-        uint32_t out = 0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          if (i < vpl) {
-            const int q = (int)(int8_t)((oldw[r] >> (8 * i)) & 0xff);
-            out |= ((uint32_t)(quant_sym(__fmul_rn((float)q, s_old), s) & 0xff)) << (8 * i);
-          }
-        int8_t* dst = tile + (size_t)r * d + lane * vpl;
-        if (vpl == 4) *reinterpret_cast<uint32_t*>(dst) = out;
-        else *reinterpret_cast<uint16_t*>(dst) = (uint16_t)out;
-      }
-      if (lane == 0) *scale_ptr = s;  // the new token's codes below use the rebuilt scale
-    } else {
-      s = s_old;
-    }
+    s = rebuild_sym(tile, d, o0, s_old, m, tbl, lane);
   }
   uint32_t lo = 0, hi = 0;
 #pragma unroll
@@ -349,93 +407,32 @@ __device__ bool fast_sym(const float x[8], int vpl, int8_t* tile, float* scale_p
   if (vpl == 8) *reinterpret_cast<uint2*>(dst) = make_uint2(lo, hi);
   else if (vpl == 4) *reinterpret_cast<uint32_t*>(dst) = lo;
   else *reinterpret_cast<uint16_t*>(dst) = (uint16_t)lo;
-  if (o0 == 0 && lane == 0) *scale_ptr = s;
-  return true;
+  if (set_scale && lane == 0) *scale_ptr = s;
 }
 
-// INT4 asymmetric side of a one-token group; false when the token does not fit (rebuild needed).
-__device__ bool fast_asym4(const float x[8], int vpl, uint8_t* tile, float* scale_ptr, uint8_t* zp_ptr, float s_old,
-                           int zp_old, int o0, int d, int lane) {
+// INT4 asymmetric side of a one-token group at offset o0.
+__device__ __forceinline__ void append_asym4(const float x[8], int vpl, uint8_t* tile, float* scale_ptr, uint8_t* zp_ptr,
+                                             float s_old, int zp_old, int o0, int d, uint8_t* tbl, int lane) {
+  float lo = 0.0f, hi = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if (i >= vpl) continue;
+    lo = fminf(lo, x[i]);
+    hi = fmaxf(hi, x[i]);
+  }
+  lo = warp_min(lo);
+  hi = warp_max(hi);
   float s;
   int zp;
+  bool set_scale = true;
   if (o0 == 0) {
-    float lo = 0.0f, hi = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (i >= vpl) continue;
-      lo = fminf(lo, x[i]);
-      hi = fmaxf(hi, x[i]);
-    }
-    lo = warp_min(lo);
-    hi = warp_max(hi);
     derive_asym(lo, hi, s, zp);
+  } else if (fits_asym(lo, hi, s_old, zp_old)) {
+    s = s_old;
+    zp = zp_old;
+    set_scale = false;
   } else {
-    bool fits = true;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (i >= vpl) continue;
-      if (s_old == 0.0f) {
-        fits = fits && (x[i] == 0.0f);
-      } else {
-        const int r = __float2int_rn(__fadd_rn(__fdiv_rn(x[i], s_old), (float)zp_old));
-        fits = fits && (r >= 0 && r <= 15);
-      }
-    }
-    if (!__all_sync(kFull, fits)) {
-      if (vpl > 4) return false;  // head_dim 256: the general path rebuilds
-      // rebuild in registers: old nibbles of every row in one batch of loads; range over
-      // x_hat = (code - zp_old) * s_old (binary32) and the new values; requantize everything
-      uint32_t oldw[32];
-#pragma unroll
-      for (int r = 0; r < 32; ++r) {
-        oldw[r] = 0;
-        if (r < o0) {
-          const uint8_t* src = tile + (size_t)r * (d / 2) + lane * (vpl / 2);
-          oldw[r] = (vpl == 4) ? *reinterpret_cast<const uint16_t*>(src) : *src;
-        }
-      }
-      float lo = 0.0f, hi = 0.0f;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        if (i >= vpl) continue;
-        lo = fminf(lo, x[i]);
-        hi = fmaxf(hi, x[i]);
-      }
-#pragma unroll
-      for (int r = 0; r < 32; ++r)
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          if (r < o0 && i < vpl) {
-            const int q = (int)((oldw[r] >> (4 * i)) & 0xF);
-            const float v = __fmul_rn((float)(q - zp_old), s_old);
-            lo = fminf(lo, v);
-            hi = fmaxf(hi, v);
-          }
-      lo = warp_min(lo);
-      hi = warp_max(hi);
-      derive_asym(lo, hi, s, zp);
-#pragma unroll
-      for (int r = 0; r < 32; ++r) {
-        if (r >= o0) continue;
-        uint32_t out = 0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          if (i < vpl) {
-            const int q = (int)((oldw[r] >> (4 * i)) & 0xF);
-            out |= (uint32_t)quant_asym(__fmul_rn((float)(q - zp_old), s_old), s, zp) << (4 * i);
-          }
-        uint8_t* dst = tile + (size_t)r * (d / 2) + lane * (vpl / 2);
-        if (vpl == 4) *reinterpret_cast<uint16_t*>(dst) = (uint16_t)out;
-        else *dst = (uint8_t)out;
-      }
-      if (lane == 0) {
-        *scale_ptr = s;
-        *zp_ptr = (uint8_t)zp;
-      }
-    } else {
-      s = s_old;
-      zp = zp_old;
-    }
+    rebuild_asym4(tile, d, o0, s_old, zp_old, lo, hi, tbl, lane, s, zp);
   }
   uint32_t packed = 0;  // vpl / 2 bytes: byte j = code[2j] | code[2j+1] << 4
 #pragma unroll
@@ -448,20 +445,20 @@ __device__ bool fast_asym4(const float x[8], int vpl, uint8_t* tile, float* scal
   if (vpl == 8) *reinterpret_cast<uint32_t*>(dst) = packed;
   else if (vpl == 4) *reinterpret_cast<uint16_t*>(dst) = (uint16_t)packed;
   else *dst = (uint8_t)packed;
-  if (o0 == 0 && lane == 0) {
+  if (set_scale && lane == 0) {
     *scale_ptr = s;
     *zp_ptr = (uint8_t)zp;
   }
-  return true;
 }
 
-__device__ __forceinline__ void fast_fp16(const uint32_t raw[4], int vpl, __half* tile, int o0, int d, int lane) {
+__device__ __forceinline__ void append_fp16(const uint32_t raw[4], int vpl, __half* tile, int o0, int d, int lane) {
   __half* dst = tile + (size_t)o0 * d + lane * vpl;
   if (vpl == 8) *reinterpret_cast<uint4*>(dst) = make_uint4(raw[0], raw[1], raw[2], raw[3]);
   else if (vpl == 4) *reinterpret_cast<uint2*>(dst) = make_uint2(raw[0], raw[1]);
   else *reinterpret_cast<uint32_t*>(dst) = raw[0];
 }
 
+template <int KT, int VT>
 __global__ void __launch_bounds__(32 * kWarpsPerCta) store_quantized_kernel(const StoreParams p) {
   // a kernel launched after this one with programmatic serialization (the decode) may begin its
   // set-up now; it waits for this grid to complete before it reads the pool
@@ -469,6 +466,8 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta) store_quantized_kernel(cons
   const int t = blockIdx.x;
   const int h = blockIdx.y * kWarpsPerCta + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
+  __shared__ __align__(16) uint8_t tables[kWarpsPerCta][256];  // per warp: a rebuild's code table
+  uint8_t* tbl = tables[threadIdx.x >> 5];
   if (h >= p.num_kv_heads) return;
   const int bs = p.block_size;
   const int d = p.head_dim;
@@ -534,57 +533,51 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta) store_quantized_kernel(cons
   uint8_t* v_tile4 = static_cast<uint8_t*>(p.v_codes) + tile_idx * bs * (d / 2);
   __half* v_tile16 = static_cast<__half*>(p.v_codes) + tile_idx * bs * d;
 
-  bool k_done = false, v_done = false;
   if (n == 1) {
     // the stored scale / zero point matter only when appending into a partly filled tile
     float ks_old = 0.f, vs_old = 0.f;
     int vzp_old = 0;
     if (o0 > 0) {
-      if (p.k_dtype == PKV_INT8_SYM) ks_old = p.k_scale[tile_idx];
-      if (p.v_dtype != PKV_FP16) vs_old = p.v_scale[tile_idx];
-      if (p.v_dtype == PKV_INT4_ASYM) vzp_old = p.v_zp[tile_idx];
+      if constexpr (KT == PKV_INT8_SYM) ks_old = p.k_scale[tile_idx];
+      if constexpr (VT != PKV_FP16) vs_old = p.v_scale[tile_idx];
+      if constexpr (VT == PKV_INT4_ASYM) vzp_old = p.v_zp[tile_idx];
     }
     float kx[8], vx[8];
     halves_to_float(kraw, kx);
     halves_to_float(vraw, vx);
-    if (p.k_dtype == PKV_INT8_SYM) {
-      k_done = fast_sym(kx, vpl, k_tile8, p.k_scale + tile_idx, ks_old, o0, d, lane);
+    if constexpr (KT == PKV_INT8_SYM) {
+      append_sym(kx, vpl, k_tile8, p.k_scale + tile_idx, ks_old, o0, d, tbl, lane);
     } else {
-      fast_fp16(kraw, vpl, k_tile16, o0, d, lane);
-      k_done = true;
+      append_fp16(kraw, vpl, k_tile16, o0, d, lane);
     }
-    if (p.v_dtype == PKV_INT8_SYM) {
-      v_done = fast_sym(vx, vpl, v_tile8, p.v_scale + tile_idx, vs_old, o0, d, lane);
-    } else if (p.v_dtype == PKV_INT4_ASYM) {
-      v_done = fast_asym4(vx, vpl, v_tile4, p.v_scale + tile_idx, p.v_zp + tile_idx, vs_old, vzp_old, o0, d, lane);
+    if constexpr (VT == PKV_INT8_SYM) {
+      append_sym(vx, vpl, v_tile8, p.v_scale + tile_idx, vs_old, o0, d, tbl, lane);
+    } else if constexpr (VT == PKV_INT4_ASYM) {
+      append_asym4(vx, vpl, v_tile4, p.v_scale + tile_idx, p.v_zp + tile_idx, vs_old, vzp_old, o0, d, tbl, lane);
     } else {
-      fast_fp16(vraw, vpl, v_tile16, o0, d, lane);
-      v_done = true;
+      append_fp16(vraw, vpl, v_tile16, o0, d, lane);
     }
+    return;
   }
 
-  // general path: groups of several tokens, and appends that must rebuild the tile
+  // groups of several tokens
   GroupSrc src;
   src.row_stride = row_stride;
   src.n = n;
   src.d = d;
-  if (!k_done) {
-    src.base = p.k_new + (size_t)t * src.row_stride + (size_t)h * d;
-    if (p.k_dtype == PKV_INT8_SYM) {
-      store_sym(src, k_tile8, p.k_scale + tile_idx, o0, lane);
-    } else {
-      store_fp16(src, k_tile16, o0, lane);
-    }
+  src.base = p.k_new + (size_t)t * src.row_stride + (size_t)h * d;
+  if constexpr (KT == PKV_INT8_SYM) {
+    store_sym(src, k_tile8, p.k_scale + tile_idx, o0, tbl, lane);
+  } else {
+    store_fp16(src, k_tile16, o0, lane);
   }
-  if (!v_done) {
-    src.base = p.v_new + (size_t)t * src.row_stride + (size_t)h * d;
-    if (p.v_dtype == PKV_INT8_SYM) {
-      store_sym(src, v_tile8, p.v_scale + tile_idx, o0, lane);
-    } else if (p.v_dtype == PKV_INT4_ASYM) {
-      store_asym4(src, v_tile4, p.v_scale + tile_idx, p.v_zp + tile_idx, o0, lane);
-    } else {
-      store_fp16(src, v_tile16, o0, lane);
-    }
+  src.base = p.v_new + (size_t)t * src.row_stride + (size_t)h * d;
+  if constexpr (VT == PKV_INT8_SYM) {
+    store_sym(src, v_tile8, p.v_scale + tile_idx, o0, tbl, lane);
+  } else if constexpr (VT == PKV_INT4_ASYM) {
+    store_asym4(src, v_tile4, p.v_scale + tile_idx, p.v_zp + tile_idx, o0, tbl, lane);
+  } else {
+    store_fp16(src, v_tile16, o0, lane);
   }
 }
 
@@ -593,7 +586,19 @@ __global__ void __launch_bounds__(32 * kWarpsPerCta) store_quantized_kernel(cons
 cudaError_t launch_store(const StoreParams& p, cudaStream_t stream) {
   if (p.T == 0) return cudaSuccess;
   dim3 grid(p.T, (p.num_kv_heads + kWarpsPerCta - 1) / kWarpsPerCta);
-  store_quantized_kernel<<<grid, 32 * kWarpsPerCta, 0, stream>>>(p);
+  const dim3 block(32 * kWarpsPerCta);
+  if (p.k_dtype == PKV_INT8_SYM && p.v_dtype == PKV_INT8_SYM)
+    store_quantized_kernel<PKV_INT8_SYM, PKV_INT8_SYM><<<grid, block, 0, stream>>>(p);
+  else if (p.k_dtype == PKV_INT8_SYM && p.v_dtype == PKV_INT4_ASYM)
+    store_quantized_kernel<PKV_INT8_SYM, PKV_INT4_ASYM><<<grid, block, 0, stream>>>(p);
+  else if (p.k_dtype == PKV_INT8_SYM && p.v_dtype == PKV_FP16)
+    store_quantized_kernel<PKV_INT8_SYM, PKV_FP16><<<grid, block, 0, stream>>>(p);
+  else if (p.k_dtype == PKV_FP16 && p.v_dtype == PKV_INT8_SYM)
+    store_quantized_kernel<PKV_FP16, PKV_INT8_SYM><<<grid, block, 0, stream>>>(p);
+  else if (p.k_dtype == PKV_FP16 && p.v_dtype == PKV_INT4_ASYM)
+    store_quantized_kernel<PKV_FP16, PKV_INT4_ASYM><<<grid, block, 0, stream>>>(p);
+  else
+    store_quantized_kernel<PKV_FP16, PKV_FP16><<<grid, block, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

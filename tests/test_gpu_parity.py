@@ -233,6 +233,57 @@ def test_append_rebuild_bit_exact():
         np.testing.assert_array_equal(pool.v_zp.cpu().numpy(), c.v_zp)
 
 
+@pytest.mark.parametrize("bs,D,kt,vt", [(32, 256, W.INT8_SYM, W.INT4_ASYM), (32, 128, W.INT8_SYM, W.INT8_SYM),
+                                         (16, 64, W.FP16, W.INT4_ASYM), (16, 256, W.INT8_SYM, W.INT8_SYM),
+                                         (32, 64, W.INT8_SYM, W.FP16)])
+def test_token_by_token_appends_bit_exact(bs, D, kt, vt):
+    """Decode-step appends one token at a time into every offset of a tile, with tokens that force a
+    rebuild at early and late offsets (tiles larger than one batch of a rebuild's loads included),
+    an all-zero first token (stored scale 0), and multi-token groups that rebuild late in the tile."""
+    import oracle
+    from paged_block_quantized_b200 import pkv
+    rng = np.random.default_rng(21 + bs + D)
+    nb, H = 6, 3
+    ot = {W.FP16: oracle.FP16, W.INT8_SYM: oracle.INT8_SYM, W.INT4_ASYM: oracle.INT4_ASYM}
+    pool = pkv.DevicePool.allocate(nb, bs, H, D, kt, vt, fill=0x5A)
+    c = oracle.OracleCache.empty(nb, bs, H, D, ot[kt], ot[vt], poison=0x5A)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    grow = {3: 3.0, 9: 9.0, 17: 27.0, 25: 81.0, bs - 1: 300.0}
+
+    def put(block, start, n, scale, zero=False):
+        k = (rng.standard_normal((n, H, D)) * scale).astype(np.float16)
+        v = (rng.standard_normal((n, H, D)) * scale + scale / 4).astype(np.float16)
+        if zero:
+            k[:] = 0
+            v[:] = 0
+        slots = block * bs + start + np.arange(n, dtype=np.int64)
+        oracle.store(c, k, v, slots)
+        pkv.pkv_store_quantized(pool.desc, torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda(),
+                                torch.from_numpy(slots).cuda(), n, err)
+
+    for o in range(bs):                       # block 1: one token at a time, rebuilds at `grow`
+        put(1, o, 1, grow.get(o, 0.5))
+    put(2, 0, 1, 1.0, zero=True)              # block 2: zero tile, then non-zero tokens
+    for o in range(1, bs):
+        put(2, o, 1, 1.0 + o)
+    put(4, 0, bs - 6, 1.0)                    # block 4: late group that rebuilds, then one that fits
+    put(4, bs - 6, 4, 50.0)
+    put(4, bs - 2, 2, 0.1)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    got = (pool.k_codes.cpu().numpy(), pool.v_codes.cpu().numpy(), pool.k_scale.cpu().numpy().view(np.uint32),
+           pool.v_scale.cpu().numpy().view(np.uint32), pool.v_zp.cpu().numpy())
+    for b in (1, 2, 4):
+        np.testing.assert_array_equal(got[0][b].reshape(-1), c.k_codes[b].view(np.uint8).reshape(-1))
+        np.testing.assert_array_equal(got[1][b].reshape(-1), c.v_codes[b].view(np.uint8).reshape(-1))
+        if kt != W.FP16:
+            np.testing.assert_array_equal(got[2][b], c.k_scale[b].view(np.uint32))
+        if vt != W.FP16:
+            np.testing.assert_array_equal(got[3][b], c.v_scale[b].view(np.uint32))
+        if vt == W.INT4_ASYM:
+            np.testing.assert_array_equal(got[4][b], c.v_zp[b])
+
+
 def test_copy_blocks_bit_exact_and_bad_ids():
     import oracle
     from paged_block_quantized_b200 import pkv
