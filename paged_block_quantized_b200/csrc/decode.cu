@@ -15,7 +15,7 @@
 // How (B200 design, not taken from the pages): a persistent, stream-K kernel.
 //   * A "unit" is (sequence s, head group hg): GT query heads sharing one KV head. Every unit
 //     contributes ceil(L_s / bs) blocks to one global stream, ordered (s, hg, block). The grid
-//     is a fixed set of worker warps (a few CTAs per SM, each warp independent); warp w owns
+//     is a fixed set of worker warps (one CTA per SM, each warp independent); warp w owns
 //     the contiguous stream range [w*T/W, (w+1)*T/W), so every warp gets the same number of
 //     blocks whatever the length mix.
 //   * Each warp streams its range through its own ring of NS shared-memory stages: lane 0
@@ -43,13 +43,18 @@ namespace {
 constexpr uint32_t kFull = 0xffffffffu;
 constexpr float kNegBig = -1.0e30f;  // finite "minus infinity" for running maxima
 
-// Shared-memory budget of one CTA's copy rings and the CTA-per-SM caps by heads per warp
-// (overridable at build time for tuning sweeps).
-#ifndef PKV_DECODE_SMEM_TARGET
-#define PKV_DECODE_SMEM_TARGET 32768
+// One CTA per SM, with as many warps as the engine's registers allow (measured best): 16 for
+// one INT8-K query head per warp, 12 for two, 8 for four on the CUDA cores or for FP16 K, 12 for
+// the tensor-core engine (8 with head_dim 256). Warps of one CTA share the SM without the
+// launch-order priority that the scheduler gives warps of earlier CTAs, which made warps of the
+// last CTA on an SM run up to a third slower than those of the first and finish last. The
+// copy rings take PKV_DECODE_SMEM_SM bytes of the SM's shared memory. (Both overridable at
+// build time for tuning sweeps.)
+#ifndef PKV_DECODE_SMEM_SM
+#define PKV_DECODE_SMEM_SM 131072
 #endif
-#ifndef PKV_DECODE_CPS_GT1
-#define PKV_DECODE_CPS_GT1 4
+#ifndef PKV_DECODE_WARPS_SM
+#define PKV_DECODE_WARPS_SM 0  // 0: by engine, as above
 #endif
 #ifndef PKV_DECODE_MAX_STAGES
 #define PKV_DECODE_MAX_STAGES 6
@@ -62,25 +67,23 @@ struct Cfg {
   static constexpr int K_TILE = BS * K_ROW;
   static constexpr int V_TILE = BS * V_ROW;
   static constexpr int STAGE = K_TILE + V_TILE;
-  static constexpr int NW = (4 * 2 * STAGE <= 200 * 1024) ? 4 : 2;  // warps per CTA
-  // stages per warp from the CTA's shared-memory budget, at least 2
-  static constexpr int NS_RAW = PKV_DECODE_SMEM_TARGET / (NW * STAGE);
-  static constexpr int NS = NS_RAW < 2 ? 2 : (NS_RAW > PKV_DECODE_MAX_STAGES ? PKV_DECODE_MAX_STAGES : NS_RAW);
   // tensor-core engine for groups of 4 or 8 query heads (INT8/INT8 with D >= 128, FP16/FP16)
   static constexpr bool MMA =
       GT >= 4 && ((KT == PKV_INT8_SYM && VT == PKV_INT8_SYM && D >= 128) || (KT == PKV_FP16 && VT == PKV_FP16));
+  static constexpr int WARPS_AUTO =
+      MMA ? (D >= 256 ? 8 : 12) : (KT == PKV_FP16 ? 8 : (GT == 1 ? 16 : (GT == 2 ? 12 : 8)));
+  static constexpr int WARPS_WANT = PKV_DECODE_WARPS_SM > 0 ? PKV_DECODE_WARPS_SM : WARPS_AUTO;
+  static constexpr int WARPS_FIT = (200 * 1024) / (2 * STAGE);  // two stages per warp at least
+  static constexpr int NW = WARPS_WANT < WARPS_FIT ? WARPS_WANT : WARPS_FIT;  // warps per CTA
+  static constexpr int NS_RAW = PKV_DECODE_SMEM_SM / (NW * STAGE);             // stages per warp
+  static constexpr int NS = NS_RAW < 2 ? 2 : (NS_RAW > PKV_DECODE_MAX_STAGES ? PKV_DECODE_MAX_STAGES : NS_RAW);
   static constexpr int THREADS = 32 * NW;
   static constexpr int SMEM_STAGES = NW * NS * STAGE;
   static constexpr int SMEM = SMEM_STAGES + NW * NS * 8;
-  // resident CTAs per SM: bounded by shared memory (227 KiB per SM) and by the registers a
-  // thread needs for GT heads of state
-  static constexpr int CPS_SMEM = (220 * 1024) / (SMEM + 1024);
-  static constexpr int CPS_CAP =
-      MMA ? (D >= 256 ? 2 : 3) : ((GT == 1) ? PKV_DECODE_CPS_GT1 : (GT == 2 ? 3 : 2));  // registers
-  static constexpr int CTAS_PER_SM = CPS_SMEM < 1 ? 1 : (CPS_SMEM > CPS_CAP ? CPS_CAP : CPS_SMEM);
+  static constexpr int CTAS_PER_SM = 1;
   static_assert(D % 16 == 0 && D / 16 <= 32, "head_dim");
   static_assert(K_TILE % 16 == 0 && V_TILE % 16 == 0 && STAGE % 16 == 0, "bulk copy granularity");
-  static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
+  static_assert(NW >= 1 && SMEM <= 227 * 1024, "shared memory per CTA");
 };
 
 // 16 consecutive fp16 values of one token row (lane chunk) -> 8 float2 (dims in order)
@@ -613,6 +616,80 @@ template <int KT, int VT, int BS, int D, int GT>
 using EngineFor = typename std::conditional<Cfg<KT, VT, BS, D, GT>::MMA, MmaEngine<KT, VT, BS, D, GT>,
                                             CoreEngine<KT, VT, BS, D, GT>>::type;
 
+// ---- merge of a split unit ----
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(kFull, v, off);
+  return v;
+}
+__device__ __forceinline__ float warp_maxf(float v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, off));
+  return v;
+}
+
+// Merge the n_seg partials of one unit (slots slot0 .. slot0 + n_seg - 1) and write its outputs:
+// out = sum_i 2^(m_i - M) acc_i / sum_i 2^(m_i - M) l_i. Lane i fetches the (max, sum) of partial
+// i (32 at a time); each lane owns D / 32 consecutive dims of every head and fetches them from
+// four partials at once.
+template <int GT, int D>
+__device__ __forceinline__ void merge_partials(const DecodeParams& p, long long slot0, int n_seg, int s, int hg,
+                                            int lane) {
+  constexpr int DL = D / 32;
+  static_assert(DL == 2 || DL == 4 || DL == 8, "head_dim");
+  float M[GT], Ls[GT], A[GT][DL];
+#pragma unroll
+  for (int hh = 0; hh < GT; ++hh) {
+    M[hh] = kNegBig;
+    Ls[hh] = 0.f;
+#pragma unroll
+    for (int d = 0; d < DL; ++d) A[hh][d] = 0.f;
+  }
+  for (int i0 = 0; i0 < n_seg; i0 += 32) {
+    const bool has = i0 + lane < n_seg;
+    float e[GT];
+#pragma unroll
+    for (int hh = 0; hh < GT; ++hh) {
+      float2 ml = make_float2(kNegBig, 0.f);
+      if (has) ml = __ldcg(reinterpret_cast<const float2*>(p.ws_ml) + (slot0 + i0 + lane) * GT + hh);
+      const float mn = fmaxf(M[hh], warp_maxf(ml.x));
+      const float f = ex2(M[hh] - mn);
+      Ls[hh] *= f;
+#pragma unroll
+      for (int d = 0; d < DL; ++d) A[hh][d] *= f;
+      M[hh] = mn;
+      e[hh] = has ? ex2(ml.x - mn) : 0.f;
+      Ls[hh] += warp_sum(ml.y * e[hh]);
+    }
+    const int nj = min(32, n_seg - i0);
+    for (int j = 0; j < nj; j += 4) {
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        if (j + jj >= nj) break;
+        const long long sl = slot0 + i0 + j + jj;
+#pragma unroll
+        for (int hh = 0; hh < GT; ++hh) {
+          const float ej = __shfl_sync(kFull, e[hh], j + jj);
+          const float* src = p.ws_acc + (sl * GT + hh) * D + lane * DL;
+#pragma unroll
+          for (int d = 0; d < DL; d += 2) {
+            const float2 a = __ldcg(reinterpret_cast<const float2*>(src + d));
+            A[hh][d] = fmaf(a.x, ej, A[hh][d]);
+            A[hh][d + 1] = fmaf(a.y, ej, A[hh][d + 1]);
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int hh = 0; hh < GT; ++hh) {
+    const float inv = Ls[hh] > 0.f ? 1.f / Ls[hh] : 0.f;
+    __half2* o = reinterpret_cast<__half2*>(p.out + ((size_t)s * p.num_q_heads + (size_t)hg * GT + hh) * D + lane * DL);
+#pragma unroll
+    for (int d = 0; d < DL; d += 2) o[d / 2] = __floats2half2_rn(A[hh][d] * inv, A[hh][d + 1] * inv);
+  }
+}
+
 template <int KT, int VT, int BS, int D, int GT>
 __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, BS, D, GT>::CTAS_PER_SM)
     paged_decode_kernel(const DecodeParams p) {
@@ -868,23 +945,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
         uint32_t ticket = 0;
         if (lane == 0) ticket = atomic_inc_acq_rel_gpu(&p.ws_count[u], n_seg - 1);
         ticket = __shfl_sync(kFull, ticket, 0);
-        if (ticket == n_seg - 1) {
-          for (int o = lane; o < GT * D; o += 32) {
-            const int hh = o / D, d = o % D;
-            float M = kNegBig;
-            for (int wi = w_first; wi <= w_last; ++wi)
-              M = fmaxf(M, __ldcg(&p.ws_ml[((size_t)(u + wi) * GT + hh) * 2]));
-            float Ls = 0.f, A = 0.f;
-            for (int wi = w_first; wi <= w_last; ++wi) {
-              const size_t sl = (size_t)(u + wi) * GT + hh;
-              const float e = ex2(__ldcg(&p.ws_ml[sl * 2]) - M);
-              Ls = fmaf(__ldcg(&p.ws_ml[sl * 2 + 1]), e, Ls);
-              A = fmaf(__ldcg(&p.ws_acc[sl * D + d]), e, A);
-            }
-            p.out[((size_t)cur.s * p.num_q_heads + (size_t)cur.hg * GT + hh) * D + d] =
-                __float2half_rn(Ls > 0.f ? A / Ls : 0.f);
-          }
-        }
+        if (ticket == n_seg - 1) merge_partials<GT, D>(p, u + w_first, (int)n_seg, cur.s, cur.hg, lane);
       }
       eng.reset();
       seg_j0 = j_end;  // (a new unit restarts it at its first block)

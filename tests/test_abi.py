@@ -107,17 +107,19 @@ def test_call_validation(pkv):
 def test_partitioning(pkv):
     d = desc(pkv)
     workers, ctas = pkv.pkv_decode_partitioning(d, 200, 4, 1000, 0)  # a batch that fills the device
-    assert ctas > 0 and workers % ctas == 0 and workers // ctas in (2, 4)
+    wpc = workers // ctas                      # one CTA per SM, 8 to 16 warps by engine
+    assert ctas > 0 and workers % ctas == 0 and wpc in (8, 12, 16)
+    up = lambda n: -(-n // wpc) * wpc          # worker counts are whole CTAs
     # a small batch: about one worker per 4 blocks of the largest possible work (2 x 2 x 63)
-    assert pkv.pkv_decode_partitioning(d, 2, 4, 1000, 0)[0] == 64
+    assert pkv.pkv_decode_partitioning(d, 2, 4, 1000, 0)[0] == up(63)
     # with partition_tokens: about one worker per partition_tokens tokens of the largest work
     # (2 seqs x 2 head groups x 63 blocks = 252 blocks, 8 blocks each -> 32 workers)
     w2, c2 = pkv.pkv_decode_partitioning(d, 2, 4, 1000, 128)
-    assert w2 == 32 and c2 == 32 // (workers // ctas)
+    assert w2 == up(32) and c2 == w2 // wpc
     w3, _ = pkv.pkv_decode_partitioning(d, 2, 4, 1000, 1 << 20)   # never fewer than one CTA of warps
-    assert w3 == workers // ctas
+    assert w3 == wpc
     w4, _ = pkv.pkv_decode_partitioning(d, 2, 4, 1000, 16)        # one block each: 252 workers
-    assert w4 == 252
+    assert w4 == up(252)
     w5, _ = pkv.pkv_decode_partitioning(d, 200, 4, 1000, 16)      # never more than fit on the device
     assert w5 == workers
 
