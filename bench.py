@@ -55,6 +55,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--fused", action="store_true",
+                    help="time the step as one fused launch (pkv_decode_step) instead of copy, store, decode")
     return ap.parse_args()
 
 
@@ -276,13 +278,14 @@ def run_pkv(args, rank, world, local):
     g = DeviceStep(w, device=dev, poison=None, partition_tokens=args.partition_tokens)
     g.prefill()
     has_cow = w.cow_pairs.shape[0] > 0
-    launches_per_step = (1 if has_cow else 0) + 2
+    fused = args.fused
+    launches_per_step = 1 if fused else (1 if has_cow else 0) + 2
     stream = torch.cuda.current_stream(dev)
     flush = L2Flush(dev)
 
     for _ in range(args.warmup):
         flush()
-        g.step()
+        g.step(fused=fused)
     torch.cuda.synchronize(dev)
     assert g.error() == 0, f"device error {g.error()} in warm-up"
 
@@ -291,22 +294,21 @@ def run_pkv(args, rank, world, local):
     props = torch.cuda.get_device_properties(dev)
     smi_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) is not None else str(dev.index)
     with ClockSampler(smi_id, enabled=not args.no_clocks) as clk:
-        # the timed steps: nothing between the step's kernels (the decode overlaps its set-up
-        # with the store through a programmatic dependent launch)
+        # the timed steps: the three kernels back to back (the decode overlapping its set-up with
+        # the store through a programmatic dependent launch), or with --fused one launch per step
         dist_barrier(world, dev)
         torch.cuda.synchronize(dev)
         wall0 = time.perf_counter()
         for i in range(K):
             flush()                       # outside the events: every step starts with a cold, clean L2
             ev[i][0].record(stream)
-            g.copy()
-            g.store()
-            g.decode()
+            g.step(fused=fused)
             ev[i][1].record(stream)
         torch.cuda.synchronize(dev)
         dist_barrier(world, dev)
         wall_ms = (time.perf_counter() - wall0) * 1e3
-        # each kernel on its own (roofline): the same steps with events around the store and the decode
+        # each kernel on its own (for reference): the same steps as separate launches with events
+        # around the store and the decode
         dev_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
         for i in range(K):
             flush()
@@ -337,7 +339,7 @@ def run_pkv(args, rank, world, local):
         def e2e_step():
             for name, t in host_in.items():
                 getattr(g, name).copy_(t, non_blocking=True)
-            g.step()
+            g.step(fused=fused)
             host_out.copy_(g.out, non_blocking=True)
 
         for _ in range(args.warmup):
@@ -358,11 +360,20 @@ def run_pkv(args, rank, world, local):
 
     assert g.error() == 0, f"device error {g.error()}"
     dec_s = dist_max(statistics.mean(dec_ms) / 1e3, world, dev)
-    alg_bytes = w.decode_bytes(unique=True)
-    achieved = alg_bytes / dec_s / 1e9
+    dec_bytes = w.decode_bytes(unique=True)
+    if fused:
+        # the dominant (only) kernel of the step is the fused launch: its algorithmic bytes are the
+        # step's (decode + store + copies) and its duration is the step's
+        alg_bytes = dec_bytes + w.store_bytes() + w.copy_bytes()
+        launch_s = total_s / K
+        kernel = "paged_decode_kernel (fused step: copies + store + decode)"
+    else:
+        alg_bytes, launch_s, kernel = dec_bytes, dec_s, "paged_decode_kernel"
+    achieved = alg_bytes / launch_s / 1e9
     peak, peak_src = measured_hbm_peak()
     traffic, _ = ncu_traffic(args.config)
-    step_desc = ("copy-on-write copies + " if has_cow else "") + "store 1 token/seq (quantize+scatter) + decode"
+    step_desc = (("copy-on-write copies + " if has_cow else "") + "store 1 token/seq (quantize+scatter) + decode"
+                 + (", one fused launch (pkv_decode_step)" if fused else ", separate launches"))
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": total_s * 1e3 / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -371,7 +382,8 @@ def run_pkv(args, rank, world, local):
                    "l2": "flushed before every timed step (2x L2 written, then 2x L2 read: cold and clean)", "timing": "CUDA events per step"},
         "effective_hbm_gbs": achieved, "frac_of_8tbs": achieved / 8000.0,
         "decode_us": dec_s * 1e6, "store_us": statistics.mean(store_ms) * 1e3,
-        "roofline": {"bound": "hbm", "kernel": "paged_decode_kernel", "achieved": achieved, "peak": peak,
+        "decode_only_gbs": dec_bytes / dec_s / 1e9,
+        "roofline": {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": peak,
                      "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
                      "algorithmic_bytes_per_launch": alg_bytes, "peak_source": peak_src},
         "e2e": e2e,

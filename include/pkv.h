@@ -143,9 +143,10 @@ PKV_API pkv_status pkv_store_quantized(const pkv_cache_desc* desc, const void* k
                                pkv_stream_t stream);
 
 /*
- * pkv_decode_workspace_size -- bytes of scratch pkv_paged_attention_decode needs for these
- * sizes: one ticket per (sequence, head group) plus one partial (max, sum, fp32 accumulator)
- * slot per (sequence, head group) and per worker warp; never a dequantized copy of the cache.
+ * pkv_decode_workspace_size -- bytes of scratch pkv_paged_attention_decode (and pkv_decode_step)
+ * needs for these sizes: one ticket per (sequence, head group) and two barrier counters, plus one
+ * partial (max, sum, fp32 accumulator) slot per (sequence, head group) and per worker warp; never
+ * a dequantized copy of the cache.
  * The value depends on the current device (its SM count sets the number of worker warps).
  * Returns PKV_ERR_INVALID_ARG on bad sizes.
  */
@@ -201,6 +202,28 @@ PKV_API pkv_status pkv_paged_attention_decode(const pkv_cache_desc* desc, void* 
                                       float softmax_scale, int32_t partition_tokens,
                                       void* workspace, size_t workspace_bytes, int32_t* dev_error,
                                       pkv_stream_t stream);
+
+/*
+ * pkv_decode_step -- one decode step in a single kernel launch: exactly
+ *   pkv_copy_blocks(desc, block_mapping, n_pairs, ...); then
+ *   pkv_store_quantized(desc, k_new, v_new, slot_mapping, T, ...); then
+ *   pkv_paged_attention_decode(desc, out, q, num_seqs, ...)
+ * on `stream`, with the same arguments, layouts, results and error behaviour as those three
+ * calls (each part may be empty: n_pairs == 0, T == 0). The pages describe the three operations;
+ * running them as one launch is this library's own arrangement for latency: every warp of the
+ * decode grid first takes part in the copies and the stores, a grid-wide barrier separates the
+ * phases, and the decode's set-up (lengths, block tables) overlaps the stores. The kernel is
+ * launched cooperatively (all CTAs resident); PKV_ERR_CUDA if the device refuses that.
+ * The workspace is the decode's (pkv_decode_workspace_size), zero-filled before first use as
+ * there; its barrier counters, like the tickets, are left at zero by every call that completes.
+ */
+PKV_API pkv_status pkv_decode_step(const pkv_cache_desc* desc, const int32_t* block_mapping, int32_t n_pairs,
+                                   const void* k_new, const void* v_new, const int64_t* slot_mapping, int32_t T,
+                                   void* out, const void* q, int32_t num_seqs, int32_t num_q_heads,
+                                   const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                   const int32_t* context_lens, int32_t max_context_len, float softmax_scale,
+                                   int32_t partition_tokens, void* workspace, size_t workspace_bytes,
+                                   int32_t* dev_error, pkv_stream_t stream);
 
 /*
  * pkv_paged_attention_decode_static -- the same decode as pkv_paged_attention_decode, for

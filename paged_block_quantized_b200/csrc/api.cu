@@ -62,7 +62,7 @@ constexpr int64_t kMinBlocksPerWorker = 4;
 struct DecodeGeometry {
   DecodeShape shape;
   int32_t workers;          // worker warps of the persistent grid
-  size_t counter_bytes;     // split-unit tickets at the start of the workspace (256-byte padded)
+  size_t counter_bytes;     // split-unit tickets, then the fused step's 2 barrier counters (256-byte padded)
   size_t ml_bytes;          // partial (max, sum) pairs (256-byte padded)
   size_t workspace_bytes;   // counters + (max, sum) + partial accumulators
 };
@@ -97,10 +97,94 @@ pkv_status decode_geometry(const pkv_cache_desc* d, int32_t num_seqs, int32_t nu
   g->workers = (int32_t)workers;
   const size_t units = (size_t)num_seqs * (num_q_heads / sh.heads_per_warp);
   const size_t slots = units + (size_t)workers;
-  g->counter_bytes = (units * sizeof(uint32_t) + 255) / 256 * 256;
+  g->counter_bytes = ((units + 2) * sizeof(uint32_t) + 255) / 256 * 256;
   g->ml_bytes = (slots * sh.heads_per_warp * 2 * sizeof(float) + 255) / 256 * 256;
   g->workspace_bytes =
       num_seqs > 0 ? g->counter_bytes + g->ml_bytes + slots * sh.heads_per_warp * d->head_dim * sizeof(float) : 0;
+  return PKV_OK;
+}
+
+// Store arguments: checks and kernel parameters (T > 0).
+pkv_status make_store_params(const pkv_cache_desc* desc, const void* k_new, const void* v_new,
+                             const int64_t* slot_mapping, int32_t T, int32_t* dev_error, StoreParams* p) {
+  if (k_new == nullptr || v_new == nullptr || slot_mapping == nullptr) return PKV_ERR_INVALID_ARG;
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(slot_mapping, 8)) return PKV_ERR_INVALID_ARG;
+  if (dev_error != nullptr && !aligned(dev_error, 4)) return PKV_ERR_INVALID_ARG;
+  p->k_codes = desc->k_codes;
+  p->v_codes = desc->v_codes;
+  p->k_scale = desc->k_scale;
+  p->v_scale = desc->v_scale;
+  p->v_zp = desc->v_zp;
+  p->k_new = static_cast<const __half*>(k_new);
+  p->v_new = static_cast<const __half*>(v_new);
+  p->slot_mapping = slot_mapping;
+  p->dev_error = dev_error;
+  p->T = T;
+  p->num_blocks = desc->num_blocks;
+  p->num_kv_heads = desc->num_kv_heads;
+  p->block_size = desc->block_size;
+  p->head_dim = desc->head_dim;
+  p->k_dtype = desc->k_dtype;
+  p->v_dtype = desc->v_dtype;
+  return PKV_OK;
+}
+
+// Copy arguments: checks and kernel parameters (n_pairs > 0).
+pkv_status make_copy_params(const pkv_cache_desc* desc, const int32_t* block_mapping, int32_t n_pairs,
+                            int32_t* dev_error, CopyParams* p) {
+  if (block_mapping == nullptr || !aligned(block_mapping, 4)) return PKV_ERR_INVALID_ARG;
+  if (dev_error != nullptr && !aligned(dev_error, 4)) return PKV_ERR_INVALID_ARG;
+  p->k_codes = static_cast<uint8_t*>(desc->k_codes);
+  p->v_codes = static_cast<uint8_t*>(desc->v_codes);
+  p->k_scale = desc->k_dtype != PKV_FP16 ? desc->k_scale : nullptr;
+  p->v_scale = desc->v_dtype != PKV_FP16 ? desc->v_scale : nullptr;
+  p->v_zp = desc->v_dtype == PKV_INT4_ASYM ? desc->v_zp : nullptr;
+  p->block_mapping = block_mapping;
+  p->dev_error = dev_error;
+  p->n_pairs = n_pairs;
+  p->num_blocks = desc->num_blocks;
+  p->num_kv_heads = desc->num_kv_heads;
+  p->k_block_bytes = (int64_t)desc->num_kv_heads * desc->block_size * row_bytes(desc->k_dtype, desc->head_dim);
+  p->v_block_bytes = (int64_t)desc->num_kv_heads * desc->block_size * row_bytes(desc->v_dtype, desc->head_dim);
+  return PKV_OK;
+}
+
+// Decode arguments: checks and kernel parameters (num_seqs > 0, geometry already computed).
+pkv_status make_decode_params(const pkv_cache_desc* desc, const DecodeGeometry& g, void* out, const void* q,
+                              int32_t num_seqs, int32_t num_q_heads, const int32_t* block_tables,
+                              int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t max_context_len,
+                              float softmax_scale, void* workspace, size_t workspace_bytes, int32_t* dev_error,
+                              DecodeParams* pp) {
+  if (out == nullptr || q == nullptr || block_tables == nullptr || context_lens == nullptr) return PKV_ERR_INVALID_ARG;
+  if (!aligned(out, 16) || !aligned(q, 16) || !aligned(block_tables, 4) || !aligned(context_lens, 4))
+    return PKV_ERR_INVALID_ARG;
+  if (max_blocks_per_seq <= 0) return PKV_ERR_INVALID_ARG;
+  if (dev_error != nullptr && !aligned(dev_error, 4)) return PKV_ERR_INVALID_ARG;
+  if (workspace == nullptr || workspace_bytes < g.workspace_bytes || !aligned(workspace, 16)) return PKV_ERR_INVALID_ARG;
+  if (!(softmax_scale == softmax_scale)) return PKV_ERR_INVALID_ARG;  // NaN
+  DecodeParams& p = *pp;
+  p.k_codes = desc->k_codes;
+  p.v_codes = desc->v_codes;
+  p.k_scale = desc->k_scale;
+  p.v_scale = desc->v_scale;
+  p.v_zp = desc->v_zp;
+  p.q = static_cast<const __half*>(q);
+  p.out = static_cast<__half*>(out);
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  p.ws_count = reinterpret_cast<uint32_t*>(ws);
+  p.ws_ml = reinterpret_cast<float*>(ws + g.counter_bytes);
+  p.ws_acc = reinterpret_cast<float*>(ws + g.counter_bytes + g.ml_bytes);
+  p.dev_error = dev_error;
+  p.num_seqs = num_seqs;
+  p.num_blocks = desc->num_blocks;
+  p.num_kv_heads = desc->num_kv_heads;
+  p.num_q_heads = num_q_heads;
+  p.group = num_q_heads / desc->num_kv_heads;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.max_context_len = max_context_len;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;  // log2(e)
   return PKV_OK;
 }
 
@@ -133,26 +217,9 @@ pkv_status pkv_store_quantized(const pkv_cache_desc* desc, const void* k_new, co
   if (st != PKV_OK) return st;
   if (T < 0) return PKV_ERR_INVALID_ARG;
   if (T == 0) return PKV_OK;
-  if (k_new == nullptr || v_new == nullptr || slot_mapping == nullptr) return PKV_ERR_INVALID_ARG;
-  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(slot_mapping, 8)) return PKV_ERR_INVALID_ARG;
-  if (dev_error != nullptr && !aligned(dev_error, 4)) return PKV_ERR_INVALID_ARG;
   StoreParams p;
-  p.k_codes = desc->k_codes;
-  p.v_codes = desc->v_codes;
-  p.k_scale = desc->k_scale;
-  p.v_scale = desc->v_scale;
-  p.v_zp = desc->v_zp;
-  p.k_new = static_cast<const __half*>(k_new);
-  p.v_new = static_cast<const __half*>(v_new);
-  p.slot_mapping = slot_mapping;
-  p.dev_error = dev_error;
-  p.T = T;
-  p.num_blocks = desc->num_blocks;
-  p.num_kv_heads = desc->num_kv_heads;
-  p.block_size = desc->block_size;
-  p.head_dim = desc->head_dim;
-  p.k_dtype = desc->k_dtype;
-  p.v_dtype = desc->v_dtype;
+  st = make_store_params(desc, k_new, v_new, slot_mapping, T, dev_error, &p);
+  if (st != PKV_OK) return st;
   return launch_store(p, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
@@ -193,37 +260,10 @@ pkv_status pkv_paged_attention_decode(const pkv_cache_desc* desc, void* out, con
   st = decode_geometry(desc, num_seqs, num_q_heads, max_context_len, partition_tokens, &g);
   if (st != PKV_OK) return st;
   if (num_seqs == 0) return PKV_OK;
-  if (out == nullptr || q == nullptr || block_tables == nullptr || context_lens == nullptr) return PKV_ERR_INVALID_ARG;
-  if (!aligned(out, 16) || !aligned(q, 16) || !aligned(block_tables, 4) || !aligned(context_lens, 4))
-    return PKV_ERR_INVALID_ARG;
-  if (max_blocks_per_seq <= 0) return PKV_ERR_INVALID_ARG;
-  if (dev_error != nullptr && !aligned(dev_error, 4)) return PKV_ERR_INVALID_ARG;
-  if (workspace == nullptr || workspace_bytes < g.workspace_bytes || !aligned(workspace, 16)) return PKV_ERR_INVALID_ARG;
-  if (!(softmax_scale == softmax_scale)) return PKV_ERR_INVALID_ARG;  // NaN
-
   DecodeParams p;
-  p.k_codes = desc->k_codes;
-  p.v_codes = desc->v_codes;
-  p.k_scale = desc->k_scale;
-  p.v_scale = desc->v_scale;
-  p.v_zp = desc->v_zp;
-  p.q = static_cast<const __half*>(q);
-  p.out = static_cast<__half*>(out);
-  p.block_tables = block_tables;
-  p.context_lens = context_lens;
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  p.ws_count = reinterpret_cast<uint32_t*>(ws);
-  p.ws_ml = reinterpret_cast<float*>(ws + g.counter_bytes);
-  p.ws_acc = reinterpret_cast<float*>(ws + g.counter_bytes + g.ml_bytes);
-  p.dev_error = dev_error;
-  p.num_seqs = num_seqs;
-  p.num_blocks = desc->num_blocks;
-  p.num_kv_heads = desc->num_kv_heads;
-  p.num_q_heads = num_q_heads;
-  p.group = num_q_heads / desc->num_kv_heads;
-  p.max_blocks_per_seq = max_blocks_per_seq;
-  p.max_context_len = max_context_len;
-  p.scale_log2 = softmax_scale * 1.4426950408889634f;  // log2(e)
+  st = make_decode_params(desc, g, out, q, num_seqs, num_q_heads, block_tables, max_blocks_per_seq, context_lens,
+                          max_context_len, softmax_scale, workspace, workspace_bytes, dev_error, &p);
+  if (st != PKV_OK) return st;
   return launch_decode(p, g.shape, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
@@ -233,22 +273,50 @@ pkv_status pkv_copy_blocks(const pkv_cache_desc* desc, const int32_t* block_mapp
   if (st != PKV_OK) return st;
   if (n_pairs < 0) return PKV_ERR_INVALID_ARG;
   if (n_pairs == 0) return PKV_OK;
-  if (block_mapping == nullptr || !aligned(block_mapping, 4)) return PKV_ERR_INVALID_ARG;
-  if (dev_error != nullptr && !aligned(dev_error, 4)) return PKV_ERR_INVALID_ARG;
   CopyParams p;
-  p.k_codes = static_cast<uint8_t*>(desc->k_codes);
-  p.v_codes = static_cast<uint8_t*>(desc->v_codes);
-  p.k_scale = desc->k_dtype != PKV_FP16 ? desc->k_scale : nullptr;
-  p.v_scale = desc->v_dtype != PKV_FP16 ? desc->v_scale : nullptr;
-  p.v_zp = desc->v_dtype == PKV_INT4_ASYM ? desc->v_zp : nullptr;
-  p.block_mapping = block_mapping;
-  p.dev_error = dev_error;
-  p.n_pairs = n_pairs;
-  p.num_blocks = desc->num_blocks;
-  p.num_kv_heads = desc->num_kv_heads;
-  p.k_block_bytes = (int64_t)desc->num_kv_heads * desc->block_size * row_bytes(desc->k_dtype, desc->head_dim);
-  p.v_block_bytes = (int64_t)desc->num_kv_heads * desc->block_size * row_bytes(desc->v_dtype, desc->head_dim);
+  st = make_copy_params(desc, block_mapping, n_pairs, dev_error, &p);
+  if (st != PKV_OK) return st;
   return launch_copy(p, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+pkv_status pkv_decode_step(const pkv_cache_desc* desc, const int32_t* block_mapping, int32_t n_pairs, const void* k_new,
+                           const void* v_new, const int64_t* slot_mapping, int32_t T, void* out, const void* q,
+                           int32_t num_seqs, int32_t num_q_heads, const int32_t* block_tables,
+                           int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t max_context_len,
+                           float softmax_scale, int32_t partition_tokens, void* workspace, size_t workspace_bytes,
+                           int32_t* dev_error, pkv_stream_t stream) {
+  pkv_status st = check_desc(desc);
+  if (st != PKV_OK) return st;
+  if (n_pairs < 0 || T < 0) return PKV_ERR_INVALID_ARG;
+  if (!decode_supported(desc->k_dtype, desc->v_dtype, desc->block_size, desc->head_dim)) return PKV_ERR_UNSUPPORTED;
+  DecodeGeometry g;
+  st = decode_geometry(desc, num_seqs, num_q_heads, max_context_len, partition_tokens, &g);
+  if (st != PKV_OK) return st;
+  StepParams sp = {};
+  sp.fused = 1;
+  if (n_pairs > 0) {
+    st = make_copy_params(desc, block_mapping, n_pairs, dev_error, &sp.copy);
+    if (st != PKV_OK) return st;
+  }
+  if (T > 0) {
+    st = make_store_params(desc, k_new, v_new, slot_mapping, T, dev_error, &sp.store);
+    if (st != PKV_OK) return st;
+  }
+  DecodeParams p;
+  if (num_seqs > 0) {
+    st = make_decode_params(desc, g, out, q, num_seqs, num_q_heads, block_tables, max_blocks_per_seq, context_lens,
+                            max_context_len, softmax_scale, workspace, workspace_bytes, dev_error, &p);
+    if (st != PKV_OK) return st;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (num_seqs == 0 || (n_pairs == 0 && T == 0)) {  // nothing to fuse: the separate launches
+    if (n_pairs > 0 && launch_copy(sp.copy, s) != cudaSuccess) return PKV_ERR_CUDA;
+    if (T > 0 && launch_store(sp.store, s) != cudaSuccess) return PKV_ERR_CUDA;
+    if (num_seqs > 0 && launch_decode(p, g.shape, s) != cudaSuccess) return PKV_ERR_CUDA;
+    return PKV_OK;
+  }
+  sp.bar = p.ws_count + (size_t)num_seqs * (num_q_heads / g.shape.heads_per_warp);
+  return launch_decode_step(p, sp, g.shape, s) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
 // ---- decode without caller-provided scratch -------------------------------------------------

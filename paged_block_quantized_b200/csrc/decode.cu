@@ -35,6 +35,8 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "copy_impl.cuh"
+#include "store_impl.cuh"
 
 namespace pkv {
 
@@ -79,7 +81,8 @@ struct Cfg {
   static constexpr int NS = NS_RAW < 2 ? 2 : (NS_RAW > PKV_DECODE_MAX_STAGES ? PKV_DECODE_MAX_STAGES : NS_RAW);
   static constexpr int THREADS = 32 * NW;
   static constexpr int SMEM_STAGES = NW * NS * STAGE;
-  static constexpr int SMEM = SMEM_STAGES + NW * NS * 8;
+  static constexpr int SMEM_BAR_FLAG = SMEM_STAGES + NW * NS * 8;  // one int: a grid barrier's outcome
+  static constexpr int SMEM = SMEM_BAR_FLAG + 16;
   static constexpr int CTAS_PER_SM = 1;
   static_assert(D % 16 == 0 && D / 16 <= 32, "head_dim");
   static_assert(K_TILE % 16 == 0 && V_TILE % 16 == 0 && STAGE % 16 == 0, "bulk copy granularity");
@@ -690,9 +693,60 @@ __device__ __forceinline__ void merge_partials(const DecodeParams& p, long long 
   }
 }
 
+// ---- fused step: grid-wide phases before the decode ----
+// Bound on the polls of one grid barrier (each sleeps ~0.25 us): well under a second.
+constexpr int kBarrierPolls = 1 << 21;
+
+// CTA-wide rendezvous on named barrier 1 (every thread of the CTA, from any call site).
+__device__ __forceinline__ void cta_sync1() { asm volatile("barrier.sync 1;" ::: "memory"); }
+
+// Grid-wide barrier: the CTA's threads meet, then one thread per CTA arrives and polls until
+// `target` CTAs have arrived in total; the rest of the CTA waits at the second rendezvous. The
+// cooperative launch keeps every CTA resident, so the wait ends; the poll bound turns a broken
+// launch into an error code. `flag`: one int of shared memory for the outcome.
+__device__ __forceinline__ bool grid_barrier(uint32_t* ctr, uint32_t target, int32_t* dev_error, int* flag) {
+  __threadfence();
+  cta_sync1();
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    atomicAdd(ctr, 1u);
+    int polls = 0;
+    while (*reinterpret_cast<volatile uint32_t*>(ctr) < target) {
+      if (++polls > kBarrierPolls) {
+        record_error(dev_error, PKV_DEVERR_TIMEOUT);
+        ok = 0;
+        break;
+      }
+      __nanosleep(256);
+    }
+    __threadfence();
+    *flag = ok;
+  }
+  cta_sync1();
+  return *flag != 0;
+}
+
+// After the CTA's warps are all done, the last CTA to leave clears the barrier counters for the
+// next call.
+__device__ __forceinline__ void grid_exit(uint32_t* bar, uint32_t ctas) {
+  cta_sync1();
+  if (threadIdx.x == 0 && atomicAdd(&bar[1], 1u) == ctas - 1) {
+    bar[0] = 0;
+    bar[1] = 0;
+  }
+}
+
+// The store phase: (token, KV head) jobs spread over the grid's warps in job order.
+template <int KT, int VT>
+__device__ __noinline__ void step_store(const StoreParams& sp, int w, int W, int lane, uint8_t* tbl) {
+  const int jobs = sp.T * sp.num_kv_heads;
+  for (int job = w; job < jobs; job += W)
+    store_detail::store_job<KT, VT>(sp, job / sp.num_kv_heads, job % sp.num_kv_heads, lane, tbl);
+}
+
 template <int KT, int VT, int BS, int D, int GT>
 __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, BS, D, GT>::CTAS_PER_SM)
-    paged_decode_kernel(const DecodeParams p) {
+    paged_decode_kernel(const DecodeParams p, const StepParams sp) {
   using C = Cfg<KT, VT, BS, D, GT>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5;
@@ -708,6 +762,18 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
 #pragma unroll
     for (int st = 0; st < C::NS; ++st) mbar_init(&my_bars[st], 1);
     fence_mbar_init();
+  }
+
+  // ---- fused step: the copy-on-write copies, then the stores, by every warp of the grid ----
+  uint32_t phases = 0;  // grid barriers passed (each counts every CTA once)
+  int* bar_flag = reinterpret_cast<int*>(smem + C::SMEM_BAR_FLAG);
+  if (sp.fused) {
+    if (sp.copy.n_pairs > 0) {
+      copy_detail::copy_all(sp.copy, (int64_t)blockIdx.x * C::THREADS + threadIdx.x, (int64_t)gridDim.x * C::THREADS);
+      grid_barrier(sp.bar, gridDim.x * ++phases, p.dev_error, bar_flag);
+    }
+    step_store<KT, VT>(sp.store, w, W, lane, my_stages);  // a rebuild's table borrows the ring
+    __syncwarp();
   }
 
   // ---- pass 1: total stream length T; zero the outputs of empty sequences ----
@@ -741,7 +807,13 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
   // With fewer blocks than warps only the first T warps work, so that every working warp owns
   // at least one block and the warps sharing a unit are consecutive (the merge relies on it).
   const int We = (int)min((long long)W, T);
-  if (w >= We) return;
+  if (w >= We) {  // nothing to decode; in a fused step still a party to the barrier
+    if (sp.fused) {
+      grid_barrier(sp.bar, gridDim.x * ++phases, p.dev_error, bar_flag);
+      grid_exit(sp.bar, gridDim.x);
+    }
+    return;
+  }
   const long long start = (long long)w * T / We;
   const long long end = (long long)(w + 1) * T / We;
 
@@ -847,7 +919,13 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
   // Everything above reads only what the host wrote before the preceding kernel (lengths,
   // tables). From here on the pool is read, which the preceding kernel (the store of the new
   // tokens) may still be writing: wait for it to complete (no-op without a programmatic launch).
+  // In a fused step, wait instead for every warp's stores, and order them (written through the
+  // generic proxy) before this warp's bulk copies (the async proxy).
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (sp.fused) {
+    grid_barrier(sp.bar, gridDim.x * ++phases, p.dev_error, bar_flag);
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+  }
   load_meta(cur, rc);
   __syncwarp();  // barrier initialisation by lane 0 is visible to the warp
 
@@ -958,10 +1036,11 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
     // copy is still writing this CTA's shared memory when it exits.
     for (int k = cpos; k < ipos; ++k) (void)mbar_wait_bounded(&my_bars[k % C::NS], (uint32_t)((k / C::NS) & 1));
   }
+  if (sp.fused) grid_exit(sp.bar, gridDim.x);
 }
 
 template <int KT, int VT, int BS, int D, int GT>
-cudaError_t launch_one(const DecodeParams& p, const DecodeShape& sh, cudaStream_t stream) {
+cudaError_t launch_one(const DecodeParams& p, const StepParams& sp, const DecodeShape& sh, cudaStream_t stream) {
   using C = Cfg<KT, VT, BS, D, GT>;
   auto kern = paged_decode_kernel<KT, VT, BS, D, GT>;
   static unsigned long long configured = 0;  // one bit per device; benign race (same value)
@@ -974,19 +1053,26 @@ cudaError_t launch_one(const DecodeParams& p, const DecodeShape& sh, cudaStream_
     if (e != cudaSuccess) return e;
     configured |= bit;
   }
-  // programmatic dependent launch: the kernel may start while the previous kernel in the stream
-  // finishes; it waits for it (griddepcontrol.wait) before reading the pool
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(sh.grid_ctas);
   cfg.blockDim = dim3(C::THREADS);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  if (sp.fused) {
+    // the grid barriers need every CTA resident at once: a cooperative launch guarantees it
+    // (or fails to launch)
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+  } else {
+    // programmatic dependent launch: the kernel may start while the previous kernel in the
+    // stream finishes; it waits for it (griddepcontrol.wait) before reading the pool
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+  }
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, p);
+  return cudaLaunchKernelEx(&cfg, kern, p, sp);
 }
 
 template <int KT, int VT, int BS, int D, int GT>
@@ -1001,8 +1087,8 @@ bool info_one(DecodeKernelInfo* info) {
 
 // 8 heads per warp exist only with the tensor-core engine
 template <int KT, int VT, int BS, int D>
-cudaError_t launch_one8(const DecodeParams& p, const DecodeShape& sh, cudaStream_t stream) {
-  if constexpr (Cfg<KT, VT, BS, D, 8>::MMA) return launch_one<KT, VT, BS, D, 8>(p, sh, stream);
+cudaError_t launch_one8(const DecodeParams& p, const StepParams& sp, const DecodeShape& sh, cudaStream_t stream) {
+  if constexpr (Cfg<KT, VT, BS, D, 8>::MMA) return launch_one<KT, VT, BS, D, 8>(p, sp, sh, stream);
   else return cudaErrorInvalidValue;
 }
 template <int KT, int VT, int BS, int D>
@@ -1065,7 +1151,15 @@ bool decode_kernel_info(const DecodeShape& sh, DecodeKernelInfo* info) {
 }
 
 cudaError_t launch_decode(const DecodeParams& p, const DecodeShape& sh, cudaStream_t stream) {
-  PKV_DISPATCH(launch_one, p, sh, stream)
+  StepParams sp = {};
+  sp.fused = 0;
+  PKV_DISPATCH(launch_one, p, sp, sh, stream)
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_decode_step(const DecodeParams& p, const StepParams& sp, const DecodeShape& sh,
+                               cudaStream_t stream) {
+  PKV_DISPATCH(launch_one, p, sp, sh, stream)
   return cudaErrorInvalidValue;
 }
 

@@ -94,4 +94,17 @@ struct CopyParams {
 };
 cudaError_t launch_copy(const CopyParams& p, cudaStream_t stream);
 
+// ---------------------------------------------------------------- fused step
+// Copy-on-write copies, then the store, then the decode, in one cooperative launch of the decode
+// kernel: every warp takes part in the copies and the stores, with a grid-wide barrier after each
+// phase, before any decode read of the pool.
+struct StepParams {
+  int32_t fused;  // 0: decode only (the other fields are unused)
+  CopyParams copy;
+  StoreParams store;
+  uint32_t* bar;  // [2] in the workspace: barrier arrivals, warps done (zero between calls)
+};
+cudaError_t launch_decode_step(const DecodeParams& p, const StepParams& sp, const DecodeShape& sh,
+                               cudaStream_t stream);
+
 }  // namespace pkv

@@ -29,7 +29,7 @@ PKV_FP16, PKV_INT8_SYM, PKV_INT4_ASYM = 0, 1, 2
 EXPORTED = (
     "pkv_status_string", "pkv_tile_bytes", "pkv_store_quantized", "pkv_decode_workspace_size",
     "pkv_decode_partitioning", "pkv_paged_attention_decode_static",
-    "pkv_paged_attention_decode", "pkv_copy_blocks", "pkv_blocks_for_tokens", "pkv_alloc_create",
+    "pkv_paged_attention_decode", "pkv_copy_blocks", "pkv_decode_step", "pkv_blocks_for_tokens", "pkv_alloc_create",
     "pkv_alloc_destroy", "pkv_alloc_num_free", "pkv_alloc_refcount", "pkv_alloc_blocks", "pkv_alloc_fork",
     "pkv_alloc_release", "pkv_alloc_cow",
 )
@@ -76,6 +76,8 @@ _decode_static = _sig("pkv_paged_attention_decode_static", ctypes.c_int, _DESC, 
                       _I32, ctypes.c_float, _I32, _P, _P)
 PKV_STATIC_SCRATCH_BYTES = 8 << 20
 _copy = _sig("pkv_copy_blocks", ctypes.c_int, _DESC, _P, _I32, _P, _P)
+_step = _sig("pkv_decode_step", ctypes.c_int, _DESC, _P, _I32, _P, _P, _P, _I32, _P, _P, _I32, _I32, _P, _I32, _P,
+             _I32, ctypes.c_float, _I32, _P, ctypes.c_size_t, _P, _P)
 _blocks_for_tokens = _sig("pkv_blocks_for_tokens", _I32, ctypes.c_int64, _I32)
 _alloc_create = _sig("pkv_alloc_create", ctypes.c_int, _I32, ctypes.POINTER(_P))
 _alloc_destroy = _sig("pkv_alloc_destroy", None, _P)
@@ -176,6 +178,18 @@ def pkv_paged_attention_decode_static(desc, out, q, num_seqs, num_q_heads, block
 def pkv_copy_blocks(desc, block_mapping, n_pairs, dev_error=None, stream=None, raise_on_error=True):
     st = _copy(ctypes.byref(desc), _ptr(block_mapping), int(n_pairs), _ptr(dev_error), _stream(stream))
     return _check(st, "pkv_copy_blocks", raise_on_error)
+
+
+def pkv_decode_step(desc, block_mapping, n_pairs, k_new, v_new, slot_mapping, T, out, q, num_seqs, num_q_heads,
+                    block_tables, max_blocks_per_seq, context_lens, max_context_len, softmax_scale,
+                    partition_tokens=0, workspace=None, workspace_bytes=0, dev_error=None, stream=None,
+                    raise_on_error=True):
+    """Copies, store and decode of one step in one launch (the three calls above, in that order)."""
+    st = _step(ctypes.byref(desc), _ptr(block_mapping), int(n_pairs), _ptr(k_new), _ptr(v_new), _ptr(slot_mapping),
+               int(T), _ptr(out), _ptr(q), int(num_seqs), int(num_q_heads), _ptr(block_tables),
+               int(max_blocks_per_seq), _ptr(context_lens), int(max_context_len), float(softmax_scale),
+               int(partition_tokens), _ptr(workspace), int(workspace_bytes), _ptr(dev_error), _stream(stream))
+    return _check(st, "pkv_decode_step", raise_on_error)
 
 
 # ---- host allocator ----

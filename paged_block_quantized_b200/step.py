@@ -2,7 +2,8 @@
 
 A `DeviceStep` owns the device pool and the step's inputs for a `workloads.Workload`:
   prefill()  store positions [0, L-1) of every sequence (whole blocks, untimed set-up)
-  step()     copy-on-write copies, store of the token at L-1 for every sequence, decode over L
+  step()     copy-on-write copies, store of the token at L-1 for every sequence, decode over L:
+             the three separate calls, or one pkv_decode_step launch (fused=True)
 Each call is a thin sequence of pkv_* calls on one stream; torch provides the device memory.
 """
 from __future__ import annotations
@@ -66,10 +67,18 @@ class DeviceStep:
             w.num_q_heads, self.block_tables, w.max_blocks_per_seq, self.context_lens, w.max_context_len,
             w.softmax_scale, self.partition_tokens, self.workspace, self.ws_bytes, self.dev_error, stream=stream)
 
-    def step(self, stream=None):
-        self.copy(stream)
-        self.store(stream)
-        self.decode(stream)
+    def step(self, stream=None, fused: bool = False):
+        if not fused:
+            self.copy(stream)
+            self.store(stream)
+            self.decode(stream)
+            return self.out
+        w = self.w
+        pkv.pkv_decode_step(
+            self.pool.desc, self.cow, self.cow.shape[0], self.k_new, self.v_new, self.step_slots, w.num_seqs,
+            self.out, self.q, w.num_seqs, w.num_q_heads, self.block_tables, w.max_blocks_per_seq, self.context_lens,
+            w.max_context_len, w.softmax_scale, self.partition_tokens, self.workspace, self.ws_bytes,
+            self.dev_error, stream=stream)
         return self.out
 
     # ---- read-back ----

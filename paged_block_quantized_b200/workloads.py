@@ -198,6 +198,24 @@ class Workload:
         total += self.num_seqs * self.num_q_heads * D * 2 + self.num_seqs * 4
         return int(total)
 
+    def store_bytes(self) -> int:
+        """Algorithmic bytes of the step's store: each new token's fp16 K and V rows read, its codes
+        written, the slot read, and the per-(block, head) scale (and zero point) written."""
+        H, D = self.num_kv_heads, self.head_dim
+        code_b = {FP16: 2.0, INT8_SYM: 1.0, INT4_ASYM: 0.5}
+        row = D * (code_b[self.k_dtype] + code_b[self.v_dtype])
+        meta = (4 if self.k_dtype != FP16 else 0) + (4 if self.v_dtype != FP16 else 0) + (1 if self.v_dtype == INT4_ASYM else 0)
+        return int(self.num_seqs * (8 + H * (4 * D + row + meta)))
+
+    def copy_bytes(self) -> int:
+        """Algorithmic bytes of the step's copy-on-write copies: each whole block (all heads, codes,
+        scales, zero points) read once and written once, plus the mapping entries."""
+        H, D, bs = self.num_kv_heads, self.head_dim, self.block_size
+        code_b = {FP16: 2.0, INT8_SYM: 1.0, INT4_ASYM: 0.5}
+        meta = (4 if self.k_dtype != FP16 else 0) + (4 if self.v_dtype != FP16 else 0) + (1 if self.v_dtype == INT4_ASYM else 0)
+        block = H * (bs * D * (code_b[self.k_dtype] + code_b[self.v_dtype]) + meta)
+        return int(self.cow_pairs.shape[0] * (2 * block + 8))
+
     def decode_write_bytes(self) -> int:
         return self.num_seqs * self.num_q_heads * self.head_dim * 2
 

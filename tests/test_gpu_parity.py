@@ -22,7 +22,7 @@ def run_gpu(w, partition_tokens=None):
     g = DeviceStep(w, partition_tokens=partition_tokens)
     g.prefill()
     pre = g.pool_numpy()
-    g.step()
+    g.step(fused=True)  # one launch; test_fused_step_matches_separate_launches ties it to the three calls
     torch.cuda.synchronize()
     return g, pre
 
@@ -282,6 +282,36 @@ def test_token_by_token_appends_bit_exact(bs, D, kt, vt):
             np.testing.assert_array_equal(got[3][b], c.v_scale[b].view(np.uint32))
         if vt == W.INT4_ASYM:
             np.testing.assert_array_equal(got[4][b], c.v_zp[b])
+
+
+@pytest.mark.parametrize("name,over", [("mixed", dict(num_seqs=24, children=4)), ("llama7b", dict(num_seqs=6)),
+                                       ("gqa_prefix", dict(num_seqs=4, prefix_blocks=8, private_blocks=9)),
+                                       ("llama7b_fp16", dict(num_seqs=3))])
+def test_fused_step_matches_separate_launches(name, over):
+    """pkv_decode_step (copies, store and decode in one cooperative launch) gives the same pool
+    bytes and the same outputs as the three separate calls, on several steps in a row (its grid
+    barrier counters come back to zero every call)."""
+    from paged_block_quantized_b200.step import DeviceStep
+    w = W.make(name, seed=5, **over)
+    gf, gs = DeviceStep(w), DeviceStep(w)
+    for g in (gf, gs):
+        g.prefill()
+    for it in range(3):
+        gf.step(fused=True)
+        gs.step(fused=False)
+        torch.cuda.synchronize()
+        assert gf.error() == 0 and gs.error() == 0
+        for a, b in zip(gf.pool_numpy(), gs.pool_numpy()):
+            np.testing.assert_array_equal(a, b)
+        np.testing.assert_array_equal(gf.out.cpu().numpy(), gs.out.cpu().numpy())
+        # tickets (one per sequence and head group) and the two barrier counters lead the workspace
+        group = w.num_q_heads // w.num_kv_heads
+        mma = (w.k_dtype, w.v_dtype) == (W.FP16, W.FP16) or ((w.k_dtype, w.v_dtype) == (W.INT8_SYM, W.INT8_SYM)
+                                                              and w.head_dim >= 128)
+        gt = 8 if mma and group % 8 == 0 else 4 if group % 4 == 0 else 2 if group % 2 == 0 else 1
+        units = w.num_seqs * (w.num_q_heads // gt)
+        ws = gf.workspace.view(torch.int32)[: units + 2].cpu().numpy()
+        assert (ws == 0).all(), "tickets and barrier counters must be back at zero"
 
 
 def test_copy_blocks_bit_exact_and_bad_ids():
