@@ -195,7 +195,8 @@ def measured_hbm_peak():
 
 def decode_source_hash() -> str:
     h = hashlib.sha256()
-    for name in ("decode.cu", "common.cuh"):
+    for name in ("decode_kernel.cuh", "decode_i8i8.cu", "decode_i8i4.cu", "decode_f16.cu", "decode.cu", "common.cuh",
+                 "store_impl.cuh", "copy_impl.cuh"):
         with open(os.path.join(ROOT, "paged_block_quantized_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]

@@ -1,0 +1,1157 @@
+// decode_kernel.cuh -- decode-phase paged attention over the block-quantized KV cache (sm_100a):
+// the kernel and its launch, instantiated per (K dtype, V dtype) in decode_<dtypes>.cu.
+//
+// What it computes (for sequence s, query head h, KV head g = h / group):
+//   token t < L_s lives in physical block b = block_tables[s][t / bs] at offset t % bs
+//     (yunthe.com "LLM推理显存优化KV Cache量化与PagedAttention实现详解", section
+//      "PagedAttention分页注意力机制与vLLM实现": block_table maps logical to physical blocks;
+//      tbr8.org "如何通过 PagedAttention 与分块量化结合..." §2);
+//   k_hat = code * k_scale[b][g], v_hat = (code - zp) * v_scale[b][g]
+//     (yunthe.com, same page, section "KV Cache量化技术原理": x_hat = (Q(x) - zero_point) * scale);
+//   out[s][h] = sum_t softmax_t(softmax_scale * q . k_hat_t) * v_hat_t.
+// The dequantization happens in registers right after the codes leave shared memory; no
+// dequantized copy of the cache exists anywhere (tbr8.org page, §5 item 2: dequantize inside the
+// attention operator so no intermediate product occupies memory).
+//
+// How (B200 design, not taken from the pages): a persistent, stream-K kernel.
+//   * A "unit" is (sequence s, head group hg): GT query heads sharing one KV head. Every unit
+//     contributes ceil(L_s / bs) blocks to one global stream, ordered (s, hg, block). The grid
+//     is a fixed set of worker warps (one CTA per SM, each warp independent); warp w owns
+//     the contiguous stream range [w*T/W, (w+1)*T/W), so every warp gets the same number of
+//     blocks whatever the length mix.
+//   * Each warp streams its range through its own ring of NS shared-memory stages: lane 0
+//     issues two 1-D bulk asynchronous copies per block (the contiguous bs x D K tile and V tile
+//     of this head, 1-4 KiB each) that complete on the stage's mbarrier, up to NS blocks ahead
+//     and straight across unit boundaries; the warp reads tiles with 16-byte shared loads.
+//   * Block ids are read 32 at a time ("windows", one id per lane) one window ahead; per-block
+//     scales are fetched when the window's first copy is issued, NS blocks before use.
+//   * q . k for INT8 K is exact integer arithmetic: q on a 22-bit fixed-point grid split into
+//     three signed byte planes, three dp4a per 4 codes. V codes become exact floats through the
+//     float bit layout (PRMT + paired FADD, no I2F); p . v accumulates with paired FFMA.
+//   * Online softmax in the log2 domain (ex2.approx), rescaling only when the running max grows.
+//   * A unit processed entirely by one warp is written out directly. A unit split across warps
+//     gets one partial (max, sum, acc) per warp in the workspace; the last warp to finish (a
+//     self-resetting atomicInc ticket) merges them. No CTA barrier, no second kernel.
+#pragma once
+
+#include <type_traits>
+
+#include "common.cuh"
+#include "internal.h"
+#include "copy_impl.cuh"
+#include "store_impl.cuh"
+
+namespace pkv {
+namespace {
+
+constexpr uint32_t kFull = 0xffffffffu;
+constexpr float kNegBig = -1.0e30f;  // finite "minus infinity" for running maxima
+
+// One CTA per SM, with as many warps as the engine's registers allow (measured best): 16 for
+// one INT8-K query head per warp, 12 for two, 8 for four on the CUDA cores or for FP16 K, 12 for
+// the tensor-core engine (8 with head_dim 256). Warps of one CTA share the SM without the
+// launch-order priority that the scheduler gives warps of earlier CTAs, which made warps of the
+// last CTA on an SM run up to a third slower than those of the first and finish last. The
+// copy rings take PKV_DECODE_SMEM_SM bytes of the SM's shared memory. (Both overridable at
+// build time for tuning sweeps.)
+#ifndef PKV_DECODE_SMEM_SM
+#define PKV_DECODE_SMEM_SM 131072
+#endif
+#ifndef PKV_DECODE_WARPS_SM
+#define PKV_DECODE_WARPS_SM 0  // 0: by engine, as above
+#endif
+#ifndef PKV_DECODE_MAX_STAGES
+#define PKV_DECODE_MAX_STAGES 6
+#endif
+
+template <int KT, int VT, int BS, int D, int GT>
+struct Cfg {
+  static constexpr int K_ROW = (KT == PKV_FP16) ? 2 * D : D;
+  static constexpr int V_ROW = (VT == PKV_FP16) ? 2 * D : (VT == PKV_INT8_SYM ? D : D / 2);
+  static constexpr int K_TILE = BS * K_ROW;
+  static constexpr int V_TILE = BS * V_ROW;
+  static constexpr int STAGE = K_TILE + V_TILE;
+  // tensor-core engine for groups of 4 or 8 query heads (INT8/INT8 with D >= 128, FP16/FP16)
+  static constexpr bool MMA =
+      GT >= 4 && ((KT == PKV_INT8_SYM && VT == PKV_INT8_SYM && D >= 128) || (KT == PKV_FP16 && VT == PKV_FP16));
+  static constexpr int WARPS_AUTO =
+      MMA ? (D >= 256 ? 8 : 12) : (KT == PKV_FP16 ? 8 : (GT == 1 ? 16 : (GT == 2 ? 12 : 8)));
+  static constexpr int WARPS_WANT = PKV_DECODE_WARPS_SM > 0 ? PKV_DECODE_WARPS_SM : WARPS_AUTO;
+  static constexpr int WARPS_FIT = (200 * 1024) / (2 * STAGE);  // two stages per warp at least
+  static constexpr int NW = WARPS_WANT < WARPS_FIT ? WARPS_WANT : WARPS_FIT;  // warps per CTA
+  static constexpr int NS_RAW = PKV_DECODE_SMEM_SM / (NW * STAGE);             // stages per warp
+  static constexpr int NS = NS_RAW < 2 ? 2 : (NS_RAW > PKV_DECODE_MAX_STAGES ? PKV_DECODE_MAX_STAGES : NS_RAW);
+  static constexpr int THREADS = 32 * NW;
+  static constexpr int SMEM_STAGES = NW * NS * STAGE;
+  static constexpr int SMEM_BAR_FLAG = SMEM_STAGES + NW * NS * 8;  // one int: a grid barrier's outcome
+  static constexpr int SMEM = SMEM_BAR_FLAG + 16;
+  static constexpr int CTAS_PER_SM = 1;
+  static_assert(D % 16 == 0 && D / 16 <= 32, "head_dim");
+  static_assert(K_TILE % 16 == 0 && V_TILE % 16 == 0 && STAGE % 16 == 0, "bulk copy granularity");
+  static_assert(NW >= 1 && SMEM <= 227 * 1024, "shared memory per CTA");
+};
+
+// 16 consecutive fp16 values of one token row (lane chunk) -> 8 float2 (dims in order)
+__device__ __forceinline__ void load_h16(const uint8_t* p, float2 f[8]) {
+  const uint4 w0 = *reinterpret_cast<const uint4*>(p);
+  const uint4 w1 = *reinterpret_cast<const uint4*>(p + 16);
+  const uint32_t u[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) f[i] = __half22float2(*reinterpret_cast<const __half2*>(&u[i]));
+}
+
+// 16 consecutive V values of one token row (lane chunk) -> 8 float2 of (code - zp);
+// neg_bias = -(2^23 + zp) in both lanes (INT4 only)
+template <int VT>
+__device__ __forceinline__ void load_v16(const uint8_t* p, float2 neg_bias, float2 f[8]) {
+  if constexpr (VT == PKV_INT8_SYM) {
+    const uint4 w = *reinterpret_cast<const uint4*>(p);
+    s8x4_to_f32x2(w.x, f[0], f[1]);
+    s8x4_to_f32x2(w.y, f[2], f[3]);
+    s8x4_to_f32x2(w.z, f[4], f[5]);
+    s8x4_to_f32x2(w.w, f[6], f[7]);
+  } else if constexpr (VT == PKV_INT4_ASYM) {
+    const uint2 w = *reinterpret_cast<const uint2*>(p);
+    u4x8_to_f32x2(w.x, neg_bias, f);
+    u4x8_to_f32x2(w.y, neg_bias, f + 4);
+  } else {
+    load_h16(p, f);
+  }
+}
+
+__device__ __forceinline__ int clamp_len(const DecodeParams& p, int L, int bs) {
+  const int cap = min(p.max_context_len, p.max_blocks_per_seq * bs);
+  return max(0, min(L, cap));
+}
+
+// The worker warp whose stream range contains position g (start_w = floor(w*T/W) <= g).
+__device__ __forceinline__ int owner_of(long long g, long long T, int W) {
+  return (int)(((g + 1) * (long long)W - 1) / T);
+}
+
+// A window: up to 32 consecutive blocks of one unit (warp-uniform description; lane k holds
+// block j0 + k in the per-lane registers of the window).
+struct Win {
+  int s, hg, j0, n;     // sequence, head group, first block, blocks in the window (0 = none)
+  int g;                // KV head of the head group
+  int L, nblk;          // clamped length of the sequence and its block count
+  int r0;               // position of block j0 relative to the warp's first position
+  long long seq_p0;     // stream position of the sequence's first block (head group 0)
+};
+
+struct WinLanes {
+  int b;        // physical block (0 stands in for an invalid id)
+  int raw;      // block id as read from the table
+  bool valid;
+  bool meta;    // scales fetched (warp-uniform)
+  float ks, vs, zp;
+};
+
+// ============================================================================================
+// Per-block arithmetic. Both engines see one (block, KV head) tile in shared memory at a time
+// and keep the running softmax state of GT query heads for the current unit.
+// ============================================================================================
+
+// CUDA-core engine (1, 2 or 4 query heads per KV head): a lane owns 16 consecutive dims of
+// bs/(32*16/D) token rows; q.k in exact integer dp4a planes (INT8 K) or paired FFMA (FP16 K);
+// p.v with paired FFMA on codes made exact floats through the float bit layout.
+template <int KT, int VT, int BS, int D, int GT>
+struct CoreEngine {
+  using C = Cfg<KT, VT, BS, D, GT>;
+  static constexpr int CH = D / 16, TG = 32 / CH, TPL = BS / TG;
+  static_assert(BS % TG == 0, "block_size must cover the token rows of a warp pass");
+  int c, tg;
+  float2 qf[GT][8];
+  uint32_t qplane[GT][3][4];
+  float qinv[GT];
+  float m_run[GT], l_run[GT];
+  float2 acc[GT][8];
+
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int hh = 0; hh < GT; ++hh) {
+      m_run[hh] = kNegBig;
+      l_run[hh] = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[hh][j] = make_float2(0.f, 0.f);
+    }
+  }
+
+  __device__ __forceinline__ void begin(const DecodeParams& p, int s, int hg, int lane) {
+    c = lane % CH;
+    tg = lane / CH;
+#pragma unroll
+    for (int hh = 0; hh < GT; ++hh) {
+      const __half* qp = p.q + ((size_t)s * p.num_q_heads + (size_t)hg * GT + hh) * D + c * 16;
+      const uint4 w0 = *reinterpret_cast<const uint4*>(qp);
+      const uint4 w1 = *reinterpret_cast<const uint4*>(qp + 8);
+      const uint32_t u[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) qf[hh][i] = __half22float2(*reinterpret_cast<const __half2*>(&u[i]));
+    }
+    reset();
+    // INT8 K: q . k is computed exactly in integers. Each head's q is put on a fixed-point grid
+    // of 2^-shift (22 bits below its largest magnitude; fp16 q loses nothing above 2^-22 of its
+    // max) and split into three signed byte planes, q_fixed = 2^16 b2 + 2^8 b1 + b0, so a
+    // 4-code word costs three dp4a with int32 accumulation and no code is converted to float.
+    if constexpr (KT == PKV_INT8_SYM) {
+#pragma unroll
+      for (int hh = 0; hh < GT; ++hh) {
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fmaxf(fabsf(qf[hh][i].x), fabsf(qf[hh][i].y)));
+#pragma unroll
+        for (int off = 1; off < CH; off <<= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, off));
+        int e = 0;
+        (void)frexpf(amax, &e);                    // amax < 2^e
+        const int shift = amax > 0.f ? 22 - e : 0;  // |q| * 2^shift < 2^22
+        const float up = __int_as_float((127 + shift) << 23);
+        qinv[hh] = __int_as_float((127 - shift) << 23);
+#pragma unroll
+        for (int wd = 0; wd < 4; ++wd) {
+          uint32_t p0 = 0, p1 = 0, p2 = 0;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 pr = qf[hh][(4 * wd + k) / 2];
+            const int qi = __float2int_rn((((4 * wd + k) & 1) ? pr.y : pr.x) * up);
+            const int b0 = ((qi + 128) & 0xFF) - 128;
+            const int r1 = (qi - b0) >> 8;
+            const int b1 = ((r1 + 128) & 0xFF) - 128;
+            const int b2 = (r1 - b1) >> 8;
+            p0 |= (uint32_t)(b0 & 0xFF) << (8 * k);
+            p1 |= (uint32_t)(b1 & 0xFF) << (8 * k);
+            p2 |= (uint32_t)(b2 & 0xFF) << (8 * k);
+          }
+          qplane[hh][0][wd] = p0;
+          qplane[hh][1][wd] = p1;
+          qplane[hh][2][wd] = p2;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int hh = 0; hh < GT; ++hh) qinv[hh] = 1.f;
+    }
+  }
+
+  // one block; ks = per-block K scale in the log2 domain (INT8 K), vs = V scale, nzb = -(2^23+zp)
+  __device__ __forceinline__ void block(const uint8_t* kt, const uint8_t* vt, float ks, float vs, float nzb, bool valid,
+                                        int tok0, int L, float scale_log2) {
+    const float2 neg_zp_bias = make_float2(nzb, nzb);
+    float z[TPL][GT];
+#pragma unroll
+    for (int i = 0; i < TPL; ++i) {
+      const int row = tg + TG * i;
+      const uint8_t* krow = kt + row * C::K_ROW + c * (C::K_ROW / CH);
+      if constexpr (KT == PKV_INT8_SYM) {
+        const uint4 wv = *reinterpret_cast<const uint4*>(krow);
+        const int kw[4] = {(int)wv.x, (int)wv.y, (int)wv.z, (int)wv.w};
+#pragma unroll
+        for (int hh = 0; hh < GT; ++hh) {
+          int acc_p[3];
+#pragma unroll
+          for (int pl = 0; pl < 3; ++pl) {
+            int a = __dp4a((int)qplane[hh][pl][0], kw[0], 0);
+            a = __dp4a((int)qplane[hh][pl][1], kw[1], a);
+            a = __dp4a((int)qplane[hh][pl][2], kw[2], a);
+            acc_p[pl] = __dp4a((int)qplane[hh][pl][3], kw[3], a);
+          }
+          // |acc_p| < 2^18: the low two planes combine exactly in int32, the top one in fp32
+          z[i][hh] = __fmaf_rn((float)acc_p[2], 65536.f, (float)(acc_p[1] * 256 + acc_p[0]));
+        }
+      } else {
+        float2 kf[8];
+        load_h16(krow, kf);
+#pragma unroll
+        for (int hh = 0; hh < GT; ++hh) {
+          float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int j = 0; j < 8; j += 2) {
+            a0 = __ffma2_rn(qf[hh][j], kf[j], a0);
+            a1 = __ffma2_rn(qf[hh][j + 1], kf[j + 1], a1);
+          }
+          z[i][hh] = (a0.x + a0.y) + (a1.x + a1.y);
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < TPL; ++i)
+#pragma unroll
+      for (int hh = 0; hh < GT; ++hh)
+#pragma unroll
+        for (int off = 1; off < CH; off <<= 1) z[i][hh] += __shfl_xor_sync(kFull, z[i][hh], off);
+
+    float pv[TPL][GT];
+#pragma unroll
+    for (int hh = 0; hh < GT; ++hh) {
+      const float zscale = (KT == PKV_FP16) ? scale_log2 : ks * qinv[hh];
+      float mloc = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < TPL; ++i) {
+        const int t = tok0 + tg + TG * i;
+        float zz = z[i][hh] * zscale;
+        zz = (valid && t < L) ? zz : -INFINITY;
+        z[i][hh] = zz;
+        mloc = fmaxf(mloc, zz);
+      }
+#pragma unroll
+      for (int off = CH; off < 32; off <<= 1) mloc = fmaxf(mloc, __shfl_xor_sync(kFull, mloc, off));
+      // the running max is warp-uniform; rescale only when it grows (rare after the first blocks)
+      if (mloc > m_run[hh]) {
+        const float alpha = ex2(m_run[hh] - mloc);
+        m_run[hh] = mloc;
+        l_run[hh] *= alpha;
+        const float2 alpha2 = make_float2(alpha, alpha);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[hh][j] = __fmul2_rn(acc[hh][j], alpha2);
+      }
+      const float m_new = m_run[hh];
+      float lsum = 0.f;
+#pragma unroll
+      for (int i = 0; i < TPL; ++i) {
+        const float pr = ex2(z[i][hh] - m_new);
+        lsum += pr;
+        pv[i][hh] = (VT == PKV_FP16) ? pr : pr * vs;
+      }
+      l_run[hh] += lsum;
+    }
+#pragma unroll
+    for (int i = 0; i < TPL; ++i) {
+      const int row = tg + TG * i;
+      float2 vf[8];
+      load_v16<VT>(vt + row * C::V_ROW + c * (C::V_ROW / CH), neg_zp_bias, vf);
+#pragma unroll
+      for (int hh = 0; hh < GT; ++hh) {
+        const float2 pv2 = make_float2(pv[i][hh], pv[i][hh]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[hh][j] = __ffma2_rn(pv2, vf[j], acc[hh][j]);
+      }
+    }
+  }
+
+  // end of a segment: sum the lanes' partial states over the token-row groups
+  __device__ __forceinline__ void finish() {
+#pragma unroll
+    for (int hh = 0; hh < GT; ++hh) {
+#pragma unroll
+      for (int off = CH; off < 32; off <<= 1) l_run[hh] += __shfl_xor_sync(kFull, l_run[hh], off);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+#pragma unroll
+        for (int off = CH; off < 32; off <<= 1) {
+          acc[hh][j].x += __shfl_xor_sync(kFull, acc[hh][j].x, off);
+          acc[hh][j].y += __shfl_xor_sync(kFull, acc[hh][j].y, off);
+        }
+    }
+  }
+
+  __device__ __forceinline__ void write_out(const DecodeParams& p, int s, int hg) {
+    if (tg != 0) return;
+#pragma unroll
+    for (int hh = 0; hh < GT; ++hh) {
+      const float inv = l_run[hh] > 0.f ? 1.f / l_run[hh] : 0.f;
+      __half2* o = reinterpret_cast<__half2*>(p.out + ((size_t)s * p.num_q_heads + (size_t)hg * GT + hh) * D + c * 16);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) o[j] = __floats2half2_rn(acc[hh][j].x * inv, acc[hh][j].y * inv);
+    }
+  }
+
+  __device__ __forceinline__ void write_partial(const DecodeParams& p, long long slot, int lane) {
+    if (tg == 0) {
+#pragma unroll
+      for (int hh = 0; hh < GT; ++hh) {
+        float4* dst = reinterpret_cast<float4*>(p.ws_acc + ((size_t)slot * GT + hh) * D + c * 16);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          dst[j] = make_float4(acc[hh][2 * j].x, acc[hh][2 * j].y, acc[hh][2 * j + 1].x, acc[hh][2 * j + 1].y);
+      }
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int hh = 0; hh < GT; ++hh) {
+        p.ws_ml[((size_t)slot * GT + hh) * 2 + 0] = m_run[hh];
+        p.ws_ml[((size_t)slot * GT + hh) * 2 + 1] = l_run[hh];
+      }
+    }
+  }
+};
+
+// ---- tensor-core helpers (mma.sync m16n8k16, fp16 operands, fp32 accumulators) ----
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+__device__ __forceinline__ uint32_t h2_sub(uint32_t a, uint32_t b) {
+  const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&b));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t h2_pack(float lo, float hi) {
+  const __half2 r = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+// fp16 1024 + 128 in both halves: a byte b placed under exponent 0x64 reads 1024 + b, and
+// (c ^ 0x80) = c + 128 for a signed code c, so subtracting this leaves c exactly
+constexpr uint32_t kH2Bias = 0x64806480u;
+
+// Tensor-core engine (4 or 8 query heads per KV head): per 16-token slice of a block,
+//   S = K . q^T  as mma m16n8k16 with M = 16 tokens, N = 8 heads, K = 16 dims per step, and
+//   O^T += V^T . P^T  with M = 16 dims per tile, N = 8 heads, K = 16 tokens,
+// the int8 codes turned into exact fp16 integers in registers on the way into the A operands.
+// Dim order inside an mma step is a fixed permutation, the same for both operands of a product.
+// Lane (g = lane/4, c = lane%4): q.k reads token rows g, g+8 at dims [c*D/4, (c+1)*D/4); p.v reads
+// token rows 2c, 2c+1, 2c+8, 2c+9 at dims [g*D/8, (g+1)*D/8) and owns the outputs of heads 2c,
+// 2c+1 at those dims. P goes through movmatrix.trans from accumulator to operand layout, split
+// into an fp16 high and low part so p.v keeps about 22 bits of each weight.
+template <int KT, int VT, int BS, int D, int GT>
+struct MmaEngine {
+  using C = Cfg<KT, VT, BS, D, GT>;
+  static constexpr int KS = D / 16;  // q.k steps and p.v dim tiles
+  static_assert(BS % 16 == 0, "16-token slices");
+  int g, c;
+  uint32_t qb[KS][2];
+  float acc[KS][4];
+  float m_run[2], l_run[2];
+
+  __device__ __forceinline__ void reset() {
+    m_run[0] = m_run[1] = kNegBig;
+    l_run[0] = l_run[1] = 0.f;
+#pragma unroll
+    for (int j = 0; j < KS; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+  }
+
+  __device__ __forceinline__ void begin(const DecodeParams& p, int s, int hg, int lane) {
+    g = lane >> 2;
+    c = lane & 3;
+    // q^T fragments: head g of the group, dims [c*D/4, (c+1)*D/4) as 2*KS half2 words
+#pragma unroll
+    for (int j = 0; j < KS; ++j) qb[j][0] = qb[j][1] = 0u;
+    if (g < GT) {
+      const uint4* qp = reinterpret_cast<const uint4*>(p.q + ((size_t)s * p.num_q_heads + (size_t)hg * GT + g) * D +
+                                                       c * (D / 4));
+#pragma unroll
+      for (int i = 0; i < KS / 2; ++i) {
+        const uint4 w = qp[i];
+        qb[2 * i][0] = w.x;
+        qb[2 * i][1] = w.y;
+        qb[2 * i + 1][0] = w.z;
+        qb[2 * i + 1][1] = w.w;
+      }
+    }
+    reset();
+  }
+
+  __device__ __forceinline__ void block(const uint8_t* kt, const uint8_t* vt, float ks, float vs, float /*nzb*/,
+                                        bool valid, int tok0, int L, float scale_log2) {
+    const float zscale = (KT == PKV_FP16) ? scale_log2 : ks;
+#pragma unroll
+    for (int h2 = 0; h2 < BS / 16; ++h2) {
+      // ---- S = K . q^T over this 16-token slice ----
+      float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+      const uint8_t* k0 = kt + (16 * h2 + g) * C::K_ROW + c * (C::K_ROW / 4);
+      const uint8_t* k1 = k0 + 8 * C::K_ROW;
+      if constexpr (KT == PKV_INT8_SYM) {
+#pragma unroll
+        for (int i = 0; i < KS / 4; ++i) {  // 16 codes = 4 steps per 16-byte load
+          const uint4 r0 = *reinterpret_cast<const uint4*>(k0 + 16 * i);
+          const uint4 r1 = *reinterpret_cast<const uint4*>(k1 + 16 * i);
+          const uint32_t w0[4] = {r0.x, r0.y, r0.z, r0.w};
+          const uint32_t w1[4] = {r1.x, r1.y, r1.z, r1.w};
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const uint32_t u0 = w0[q4] ^ 0x80808080u, u1 = w1[q4] ^ 0x80808080u;
+            uint32_t a[4];
+            a[0] = h2_sub(__byte_perm(u0, 0x64646464u, 0x4140), kH2Bias);  // row g, dims +0,+1
+            a[1] = h2_sub(__byte_perm(u1, 0x64646464u, 0x4140), kH2Bias);  // row g+8
+            a[2] = h2_sub(__byte_perm(u0, 0x64646464u, 0x4342), kH2Bias);  // row g, dims +2,+3
+            a[3] = h2_sub(__byte_perm(u1, 0x64646464u, 0x4342), kH2Bias);  // row g+8
+            const int kk = 4 * i + q4;
+            mma_16816(sacc, a, qb[kk][0], qb[kk][1]);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < KS / 2; ++i) {  // 8 halves = 2 steps per 16-byte load
+          const uint4 r0 = *reinterpret_cast<const uint4*>(k0 + 16 * i);
+          const uint4 r1 = *reinterpret_cast<const uint4*>(k1 + 16 * i);
+          uint32_t a[4] = {r0.x, r1.x, r0.y, r1.y};
+          mma_16816(sacc, a, qb[2 * i][0], qb[2 * i][1]);
+          uint32_t b[4] = {r0.z, r1.z, r0.w, r1.w};
+          mma_16816(sacc, b, qb[2 * i + 1][0], qb[2 * i + 1][1]);
+        }
+      }
+      // ---- online softmax on the accumulator layout: rows = tokens g, g+8; cols = heads 2c, 2c+1 ----
+      const int t0 = tok0 + 16 * h2 + g, t1 = t0 + 8;
+      float z[4];
+      z[0] = (valid && t0 < L) ? sacc[0] * zscale : -INFINITY;
+      z[1] = (valid && t0 < L) ? sacc[1] * zscale : -INFINITY;
+      z[2] = (valid && t1 < L) ? sacc[2] * zscale : -INFINITY;
+      z[3] = (valid && t1 < L) ? sacc[3] * zscale : -INFINITY;
+      float mx0 = fmaxf(z[0], z[2]), mx1 = fmaxf(z[1], z[3]);
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, off));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, off));
+      }
+      const bool grow0 = mx0 > m_run[0], grow1 = mx1 > m_run[1];
+      if (__any_sync(kFull, grow0 || grow1)) {
+        const float al0 = grow0 ? ex2(m_run[0] - mx0) : 1.f;
+        const float al1 = grow1 ? ex2(m_run[1] - mx1) : 1.f;
+        if (grow0) m_run[0] = mx0;
+        if (grow1) m_run[1] = mx1;
+        l_run[0] *= al0;
+        l_run[1] *= al1;
+#pragma unroll
+        for (int j = 0; j < KS; ++j) {
+          acc[j][0] *= al0;
+          acc[j][2] *= al0;
+          acc[j][1] *= al1;
+          acc[j][3] *= al1;
+        }
+      }
+      const float p0 = ex2(z[0] - m_run[0]), p1 = ex2(z[1] - m_run[1]);
+      const float p2 = ex2(z[2] - m_run[0]), p3 = ex2(z[3] - m_run[1]);
+      l_run[0] += p0 + p2;
+      l_run[1] += p1 + p3;
+      // weights for p.v (V scale folded in), fp16 high + low parts, transposed to operand layout
+      const float w0 = (VT == PKV_FP16) ? p0 : p0 * vs, w1 = (VT == PKV_FP16) ? p1 : p1 * vs;
+      const float w2 = (VT == PKV_FP16) ? p2 : p2 * vs, w3 = (VT == PKV_FP16) ? p3 : p3 * vs;
+      const uint32_t hi0 = h2_pack(w0, w1), hi1 = h2_pack(w2, w3);
+      const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&hi0));
+      const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&hi1));
+      const uint32_t lo0 = h2_pack(w0 - f0.x, w1 - f0.y), lo1 = h2_pack(w2 - f1.x, w3 - f1.y);
+      const uint32_t bh0 = movmatrix_trans(hi0), bh1 = movmatrix_trans(hi1);
+      const uint32_t bl0 = movmatrix_trans(lo0), bl1 = movmatrix_trans(lo1);
+      // ---- O^T += V^T . P^T: token rows 2c, 2c+1, 2c+8, 2c+9 at dims [g*D/8, (g+1)*D/8) ----
+      const uint8_t* vb = vt + (16 * h2 + 2 * c) * C::V_ROW + g * (C::V_ROW / 8);
+      if constexpr (VT == PKV_INT8_SYM) {
+#pragma unroll
+        for (int i = 0; i < KS / 8; ++i) {  // 16 bytes per row = 8 dim tiles
+          const uint4 ra = *reinterpret_cast<const uint4*>(vb + 16 * i);
+          const uint4 rb = *reinterpret_cast<const uint4*>(vb + C::V_ROW + 16 * i);
+          const uint4 rc = *reinterpret_cast<const uint4*>(vb + 8 * C::V_ROW + 16 * i);
+          const uint4 rd = *reinterpret_cast<const uint4*>(vb + 9 * C::V_ROW + 16 * i);
+          const uint32_t xa[4] = {ra.x, ra.y, ra.z, ra.w}, xb[4] = {rb.x, rb.y, rb.z, rb.w};
+          const uint32_t xc[4] = {rc.x, rc.y, rc.z, rc.w}, xd[4] = {rd.x, rd.y, rd.z, rd.w};
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) {  // dim tile: bytes 2jj (row r) and 2jj+1 (row r+8)
+            const int wd = jj / 2, k = 2 * (jj % 2);
+            const uint32_t sel0 = k | (k << 4) | ((4 + k) << 8) | ((4 + k) << 12);
+            const uint32_t sel1 = (k + 1) | ((k + 1) << 4) | ((5 + k) << 8) | ((5 + k) << 12);
+            uint32_t a[4];
+            a[0] = h2_sub((__byte_perm(xa[wd], xb[wd], sel0) & 0x00FF00FFu) ^ kH2Bias, kH2Bias);
+            a[1] = h2_sub((__byte_perm(xa[wd], xb[wd], sel1) & 0x00FF00FFu) ^ kH2Bias, kH2Bias);
+            a[2] = h2_sub((__byte_perm(xc[wd], xd[wd], sel0) & 0x00FF00FFu) ^ kH2Bias, kH2Bias);
+            a[3] = h2_sub((__byte_perm(xc[wd], xd[wd], sel1) & 0x00FF00FFu) ^ kH2Bias, kH2Bias);
+            const int j = 8 * i + jj;
+            mma_16816(acc[j], a, bh0, bh1);
+            mma_16816(acc[j], a, bl0, bl1);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < KS / 4; ++i) {  // 16 bytes per row = 8 halves = 4 dim tiles
+          const uint4 ra = *reinterpret_cast<const uint4*>(vb + 16 * i);
+          const uint4 rb = *reinterpret_cast<const uint4*>(vb + C::V_ROW + 16 * i);
+          const uint4 rc = *reinterpret_cast<const uint4*>(vb + 8 * C::V_ROW + 16 * i);
+          const uint4 rd = *reinterpret_cast<const uint4*>(vb + 9 * C::V_ROW + 16 * i);
+          const uint32_t xa[4] = {ra.x, ra.y, ra.z, ra.w}, xb[4] = {rb.x, rb.y, rb.z, rb.w};
+          const uint32_t xc[4] = {rc.x, rc.y, rc.z, rc.w}, xd[4] = {rd.x, rd.y, rd.z, rd.w};
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) {  // dim tile: half 0 of the word (row r), half 1 (row r+8)
+            uint32_t a[4];
+            a[0] = __byte_perm(xa[jj], xb[jj], 0x5410);
+            a[1] = __byte_perm(xa[jj], xb[jj], 0x7632);
+            a[2] = __byte_perm(xc[jj], xd[jj], 0x5410);
+            a[3] = __byte_perm(xc[jj], xd[jj], 0x7632);
+            const int j = 4 * i + jj;
+            mma_16816(acc[j], a, bh0, bh1);
+            mma_16816(acc[j], a, bl0, bl1);
+          }
+        }
+      }
+    }
+  }
+
+  // end of a segment: sum the lanes' partial softmax denominators over the token rows
+  __device__ __forceinline__ void finish() {
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      l_run[0] += __shfl_xor_sync(kFull, l_run[0], off);
+      l_run[1] += __shfl_xor_sync(kFull, l_run[1], off);
+    }
+  }
+
+  // this lane's outputs: heads 2c (acc[.][0], acc[.][2]) and 2c+1 (acc[.][1], acc[.][3]) at
+  // dims g*D/8 + 2j (+1)
+  __device__ __forceinline__ void write_out(const DecodeParams& p, int s, int hg) {
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int hh = 2 * c + e;
+      if (hh >= GT) continue;
+      const float inv = l_run[e] > 0.f ? 1.f / l_run[e] : 0.f;
+      __half2* o = reinterpret_cast<__half2*>(p.out + ((size_t)s * p.num_q_heads + (size_t)hg * GT + hh) * D + g * (D / 8));
+#pragma unroll
+      for (int j = 0; j < KS; ++j) o[j] = __floats2half2_rn(acc[j][e] * inv, acc[j][e + 2] * inv);
+    }
+  }
+
+  __device__ __forceinline__ void write_partial(const DecodeParams& p, long long slot, int lane) {
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int hh = 2 * c + e;
+      if (hh >= GT) continue;
+      float2* dst = reinterpret_cast<float2*>(p.ws_acc + ((size_t)slot * GT + hh) * D + g * (D / 8));
+#pragma unroll
+      for (int j = 0; j < KS; ++j) dst[j] = make_float2(acc[j][e], acc[j][e + 2]);
+      if (g == 0) {
+        p.ws_ml[((size_t)slot * GT + hh) * 2 + 0] = m_run[e];
+        p.ws_ml[((size_t)slot * GT + hh) * 2 + 1] = l_run[e];
+      }
+    }
+  }
+};
+
+template <int KT, int VT, int BS, int D, int GT>
+using EngineFor = typename std::conditional<Cfg<KT, VT, BS, D, GT>::MMA, MmaEngine<KT, VT, BS, D, GT>,
+                                            CoreEngine<KT, VT, BS, D, GT>>::type;
+
+// ---- merge of a split unit ----
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(kFull, v, off);
+  return v;
+}
+__device__ __forceinline__ float warp_maxf(float v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, off));
+  return v;
+}
+
+// Merge the n_seg partials of one unit (slots slot0 .. slot0 + n_seg - 1) and write its outputs:
+// out = sum_i 2^(m_i - M) acc_i / sum_i 2^(m_i - M) l_i. Lane i fetches the (max, sum) of partial
+// i (32 at a time); each lane owns D / 32 consecutive dims of every head and fetches them from
+// four partials at once.
+template <int GT, int D>
+__device__ __forceinline__ void merge_partials(const DecodeParams& p, long long slot0, int n_seg, int s, int hg,
+                                            int lane) {
+  constexpr int DL = D / 32;
+  static_assert(DL == 2 || DL == 4 || DL == 8, "head_dim");
+  float M[GT], Ls[GT], A[GT][DL];
+#pragma unroll
+  for (int hh = 0; hh < GT; ++hh) {
+    M[hh] = kNegBig;
+    Ls[hh] = 0.f;
+#pragma unroll
+    for (int d = 0; d < DL; ++d) A[hh][d] = 0.f;
+  }
+  for (int i0 = 0; i0 < n_seg; i0 += 32) {
+    const bool has = i0 + lane < n_seg;
+    float e[GT];
+#pragma unroll
+    for (int hh = 0; hh < GT; ++hh) {
+      float2 ml = make_float2(kNegBig, 0.f);
+      if (has) ml = __ldcg(reinterpret_cast<const float2*>(p.ws_ml) + (slot0 + i0 + lane) * GT + hh);
+      const float mn = fmaxf(M[hh], warp_maxf(ml.x));
+      const float f = ex2(M[hh] - mn);
+      Ls[hh] *= f;
+#pragma unroll
+      for (int d = 0; d < DL; ++d) A[hh][d] *= f;
+      M[hh] = mn;
+      e[hh] = has ? ex2(ml.x - mn) : 0.f;
+      Ls[hh] += warp_sum(ml.y * e[hh]);
+    }
+    const int nj = min(32, n_seg - i0);
+    for (int j = 0; j < nj; j += 4) {
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        if (j + jj >= nj) break;
+        const long long sl = slot0 + i0 + j + jj;
+#pragma unroll
+        for (int hh = 0; hh < GT; ++hh) {
+          const float ej = __shfl_sync(kFull, e[hh], j + jj);
+          const float* src = p.ws_acc + (sl * GT + hh) * D + lane * DL;
+#pragma unroll
+          for (int d = 0; d < DL; d += 2) {
+            const float2 a = __ldcg(reinterpret_cast<const float2*>(src + d));
+            A[hh][d] = fmaf(a.x, ej, A[hh][d]);
+            A[hh][d + 1] = fmaf(a.y, ej, A[hh][d + 1]);
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int hh = 0; hh < GT; ++hh) {
+    const float inv = Ls[hh] > 0.f ? 1.f / Ls[hh] : 0.f;
+    __half2* o = reinterpret_cast<__half2*>(p.out + ((size_t)s * p.num_q_heads + (size_t)hg * GT + hh) * D + lane * DL);
+#pragma unroll
+    for (int d = 0; d < DL; d += 2) o[d / 2] = __floats2half2_rn(A[hh][d] * inv, A[hh][d + 1] * inv);
+  }
+}
+
+// Pull the q rows of unit (s, hg) toward the SM ahead of the engine's begin(): the GT * D fp16
+// values are contiguous; one lane per 128-byte line.
+template <int GT, int D>
+__device__ __forceinline__ void prefetch_q(const DecodeParams& p, int s, int hg, int lane) {
+  constexpr int LINES = (GT * D * 2 + 127) / 128;
+  const char* base = reinterpret_cast<const char*>(p.q + ((size_t)s * p.num_q_heads + (size_t)hg * GT) * D);
+  if (lane < LINES) asm volatile("prefetch.global.L1 [%0];" ::"l"(base + 128 * lane));
+}
+
+// ---- fused step: grid-wide phases before the decode ----
+// Bound on the polls of one grid barrier (each sleeps ~0.25 us): well under a second.
+constexpr int kBarrierPolls = 1 << 21;
+
+// CTA-wide rendezvous on named barrier 1 (every thread of the CTA, from any call site).
+__device__ __forceinline__ void cta_sync1() { asm volatile("barrier.sync 1;" ::: "memory"); }
+
+// Grid-wide barrier: the CTA's threads meet, then one thread per CTA arrives and polls until
+// `target` CTAs have arrived in total; the rest of the CTA waits at the second rendezvous. The
+// cooperative launch keeps every CTA resident, so the wait ends; the poll bound turns a broken
+// launch into an error code. `flag`: one int of shared memory for the outcome.
+__device__ __forceinline__ bool grid_barrier(uint32_t* ctr, uint32_t target, int32_t* dev_error, int* flag) {
+  __threadfence();
+  cta_sync1();
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    atomicAdd(ctr, 1u);
+    int polls = 0;
+    while (*reinterpret_cast<volatile uint32_t*>(ctr) < target) {
+      if (++polls > kBarrierPolls) {
+        record_error(dev_error, PKV_DEVERR_TIMEOUT);
+        ok = 0;
+        break;
+      }
+      __nanosleep(256);
+    }
+    __threadfence();
+    *flag = ok;
+  }
+  cta_sync1();
+  return *flag != 0;
+}
+
+// After the CTA's warps are all done, the last CTA to leave clears the barrier counters for the
+// next call.
+__device__ __forceinline__ void grid_exit(uint32_t* bar, uint32_t ctas) {
+  cta_sync1();
+  if (threadIdx.x == 0 && atomicAdd(&bar[1], 1u) == ctas - 1) {
+    bar[0] = 0;
+    bar[1] = 0;
+  }
+}
+
+// The store phase: (token, KV head) jobs spread over the grid's warps in job order.
+template <int KT, int VT>
+__device__ __noinline__ void step_store(const StoreParams& sp, int w, int W, int lane, uint8_t* tbl) {
+  const int jobs = sp.T * sp.num_kv_heads;
+  for (int job = w; job < jobs; job += W)
+    store_detail::store_job<KT, VT>(sp, job / sp.num_kv_heads, job % sp.num_kv_heads, lane, tbl);
+}
+
+template <int KT, int VT, int BS, int D, int GT, bool FUSED>
+__global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, BS, D, GT>::CTAS_PER_SM)
+    paged_decode_kernel(const DecodeParams p, const StepParams sp) {
+  using C = Cfg<KT, VT, BS, D, GT>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int W = gridDim.x * C::NW;
+  const int w = blockIdx.x * C::NW + warp;
+  const int HG = p.num_q_heads / GT;
+  const int S = p.num_seqs;
+
+  uint8_t* my_stages = smem + (size_t)warp * C::NS * C::STAGE;
+  uint64_t* my_bars = reinterpret_cast<uint64_t*>(smem + C::SMEM_STAGES) + warp * C::NS;
+  if (lane == 0) {
+#pragma unroll
+    for (int st = 0; st < C::NS; ++st) mbar_init(&my_bars[st], 1);
+    fence_mbar_init();
+  }
+
+  // ---- fused step: the copy-on-write copies, then the stores, by every warp of the grid ----
+  uint32_t phases = 0;  // grid barriers passed (each counts every CTA once)
+  int* bar_flag = reinterpret_cast<int*>(smem + C::SMEM_BAR_FLAG);
+  if constexpr (FUSED) {
+    if (sp.copy.n_pairs > 0) {
+      copy_detail::copy_all(sp.copy, (int64_t)blockIdx.x * C::THREADS + threadIdx.x, (int64_t)gridDim.x * C::THREADS);
+      grid_barrier(sp.bar, gridDim.x * ++phases, p.dev_error, bar_flag);
+    }
+    step_store<KT, VT>(sp.store, w, W, lane, my_stages);  // a rebuild's table borrows the ring
+    __syncwarp();
+  }
+
+  // ---- pass 1: total stream length T; zero the outputs of empty sequences ----
+  long long T = 0;
+  for (int base = 0; base < S; base += 32) {
+    const int s = base + lane;
+    int L = 0;
+    if (s < S) {
+      const int raw = p.context_lens[s];
+      L = clamp_len(p, raw, BS);
+      if (raw != L && w == 0) record_error(p.dev_error, PKV_DEVERR_CONTEXT_LEN);
+    }
+    int sum = (L + BS - 1) / BS;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(kFull, sum, off);
+    T += sum;
+    uint32_t empty = __ballot_sync(kFull, s < S && L == 0);
+    while (empty) {  // outputs of sequences with nothing to attend over are 0
+      const int e = __ffs(empty) - 1;
+      empty &= empty - 1;
+      const int se = base + e;
+      for (int hg = 0; hg < HG; ++hg) {
+        if ((int)(((long long)se * HG + hg) % W) != w) continue;
+        __half2* o = reinterpret_cast<__half2*>(p.out + ((size_t)se * p.num_q_heads + (size_t)hg * GT) * D);
+        for (int i = lane; i < GT * D / 2; i += 32) o[i] = __floats2half2_rn(0.f, 0.f);
+      }
+    }
+  }
+  T *= HG;
+  __syncwarp();
+  // With fewer blocks than warps only the first T warps work, so that every working warp owns
+  // at least one block and the warps sharing a unit are consecutive (the merge relies on it).
+  const int We = (int)min((long long)W, T);
+  if (w >= We) {  // nothing to decode; in a fused step still a party to the barrier
+    if constexpr (FUSED) {
+      grid_barrier(sp.bar, gridDim.x * ++phases, p.dev_error, bar_flag);
+      grid_exit(sp.bar, gridDim.x);
+    }
+    return;
+  }
+  const long long start = (long long)w * T / We;
+  const long long end = (long long)(w + 1) * T / We;
+
+  // ---- pass 2: the unit and block of `start` ----
+  Win cur;
+  int Lchunk = 0, chunk_base = 0;  // lane holds the clamped length of sequence chunk_base + lane
+  {
+    long long acc0 = 0;
+    for (int base = 0;; base += 32) {
+      const int s = base + lane;
+      const int L = s < S ? clamp_len(p, p.context_lens[s], BS) : 0;
+      const long long cnt = (long long)((L + BS - 1) / BS) * HG;
+      long long incl = cnt;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const long long o = __shfl_up_sync(kFull, incl, off);
+        if (lane >= off) incl += o;
+      }
+      const long long total = __shfl_sync(kFull, incl, 31);
+      if (acc0 + total > start) {
+        const uint32_t m = __ballot_sync(kFull, acc0 + incl > start);
+        const int f = __ffs(m) - 1;
+        cur.s = base + f;
+        cur.L = __shfl_sync(kFull, L, f);
+        cur.nblk = (cur.L + BS - 1) / BS;
+        cur.seq_p0 = acc0 + __shfl_sync(kFull, incl - cnt, f);
+        Lchunk = L;
+        chunk_base = base;
+        break;
+      }
+      acc0 += total;
+    }
+    const long long o = start - cur.seq_p0;
+    cur.hg = (int)(o / cur.nblk);
+    cur.j0 = (int)(o % cur.nblk);
+    cur.g = (cur.hg * GT) / p.group;
+    cur.r0 = 0;
+    cur.n = (int)min((long long)min(32, cur.nblk - cur.j0), end - start);
+  }
+  const int n_total = (int)(end - start);  // positions of this warp
+
+  // clamped length of sequence s, from the lane-held chunk when possible
+  auto seq_len = [&](int s) -> int {
+    if (s < chunk_base || s >= chunk_base + 32) {
+      chunk_base = s;
+      Lchunk = (s + lane < S) ? clamp_len(p, p.context_lens[s + lane], BS) : 0;
+    }
+    return __shfl_sync(kFull, Lchunk, s - chunk_base);
+  };
+
+  // the window after `a`, within [.., end); n = 0 if none
+  auto next_win = [&](const Win& a) -> Win {
+    Win b = a;
+    b.r0 = a.r0 + a.n;
+    b.n = 0;
+    if (a.n == 0 || b.r0 >= n_total) return b;
+    b.j0 = a.j0 + a.n;
+    if (b.j0 >= a.nblk) {
+      b.j0 = 0;
+      b.hg = a.hg + 1;
+      if (b.hg >= HG) {
+        b.hg = 0;
+        b.seq_p0 = a.seq_p0 + (long long)HG * a.nblk;
+        int s = a.s, L = 0;
+        do {  // sequences without blocks contribute no stream positions
+          ++s;
+          L = s < S ? seq_len(s) : 0;
+        } while (L == 0 && s < S);
+        b.s = s;
+        b.L = L;
+        b.nblk = (L + BS - 1) / BS;
+      }
+      b.g = (b.hg * GT) / p.group;
+    }
+    b.n = min(min(32, b.nblk - b.j0), n_total - b.r0);
+    return b;
+  };
+
+  // phase A of a window: block ids (one per lane); phase B (at its first copy): scales
+  auto load_ids = [&](const Win& a, WinLanes& r) {
+    r.meta = false;
+    r.raw = -1;
+    if (lane < a.n) r.raw = p.block_tables[(size_t)a.s * p.max_blocks_per_seq + a.j0 + lane];
+  };
+  auto load_meta = [&](const Win& a, WinLanes& r) {
+    r.valid = lane < a.n && r.raw >= 0 && r.raw < p.num_blocks;
+    if (lane < a.n && !r.valid) record_error(p.dev_error, PKV_DEVERR_BLOCK_ID);
+    r.b = r.valid ? r.raw : 0;
+    r.ks = r.vs = r.zp = 0.f;
+    if (lane < a.n) {
+      const size_t meta = (size_t)r.b * p.num_kv_heads + a.g;
+      if constexpr (KT != PKV_FP16) r.ks = p.k_scale[meta];
+      if constexpr (VT != PKV_FP16) r.vs = p.v_scale[meta];
+      if constexpr (VT == PKV_INT4_ASYM) r.zp = (float)p.v_zp[meta];
+    }
+    r.meta = true;
+  };
+
+  WinLanes rc, rn;
+  load_ids(cur, rc);
+  Win nxt = next_win(cur);
+  load_ids(nxt, rn);
+  if (nxt.n > 0 && (nxt.s != cur.s || nxt.hg != cur.hg)) prefetch_q<GT, D>(p, nxt.s, nxt.hg, lane);
+  // Everything above reads only what the host wrote before the preceding kernel (lengths,
+  // tables). From here on the pool is read, which the preceding kernel (the store of the new
+  // tokens) may still be writing: wait for it to complete (no-op without a programmatic launch).
+  // In a fused step, wait instead for every warp's stores, and order them (written through the
+  // generic proxy) before this warp's bulk copies (the async proxy).
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if constexpr (FUSED) {
+    grid_barrier(sp.bar, gridDim.x * ++phases, p.dev_error, bar_flag);
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+  }
+  load_meta(cur, rc);
+  __syncwarp();  // barrier initialisation by lane 0 is visible to the warp
+
+  // ---- per-unit state: the arithmetic engine for GT query heads ----
+  EngineFor<KT, VT, BS, D, GT> eng;
+  int seg_j0 = cur.j0;  // first block of the current segment within its unit
+  eng.begin(p, cur.s, cur.hg, lane);
+
+  // ---- the copy ring ----
+  auto issue = [&](int st, int b, int g) {
+    const size_t tile = (size_t)b * p.num_kv_heads + g;
+    uint8_t* dst = my_stages + (size_t)st * C::STAGE;
+    mbar_arrive_expect_tx(&my_bars[st], (uint32_t)C::STAGE);
+    bulk_g2s(dst, static_cast<const uint8_t*>(p.k_codes) + tile * C::K_TILE, (uint32_t)C::K_TILE, &my_bars[st]);
+    bulk_g2s(dst + C::K_TILE, static_cast<const uint8_t*>(p.v_codes) + tile * C::V_TILE, (uint32_t)C::V_TILE,
+             &my_bars[st]);
+  };
+  // positions relative to `start`: consumed (cpos) and issued (ipos); stage / parity of each
+  int cpos = 0, ipos = 0, cst = 0, ist = 0;
+  uint32_t cpar = 0;
+  // issue every position below min(cpos + NS, n_total) whose window is known (cur or nxt); a
+  // stage is reused only after the position NS before it has been consumed
+  auto issue_ahead = [&]() {
+    const int lim = min(cpos + C::NS, n_total);
+    while (ipos < lim) {
+      int b, g;
+      if (ipos < cur.r0 + cur.n) {
+        b = __shfl_sync(kFull, rc.b, ipos - cur.r0);
+        g = cur.g;
+      } else if (nxt.n > 0 && ipos < nxt.r0 + nxt.n) {
+        if (!rn.meta) load_meta(nxt, rn);
+        b = __shfl_sync(kFull, rn.b, ipos - nxt.r0);
+        g = nxt.g;
+      } else {
+        break;
+      }
+      if (lane == 0) issue(ist, b, g);
+      ist = (ist + 1 == C::NS) ? 0 : ist + 1;
+      ++ipos;
+    }
+  };
+
+  // With one query head per warp (registers to spare), a split unit's ticket is taken without
+  // waiting for the answer; it is read at this warp's next split-unit end (or after its last
+  // block), and if it says "last", that is when the merge runs. Otherwise it is read at once.
+  constexpr bool kDeferTicket = GT == 1;
+  bool pend = false;
+  uint32_t pend_ticket = 0;  // lane 0: the atomic's result
+  uint32_t pend_nseg = 0;
+  long long pend_slot0 = 0;
+  int pend_s = 0, pend_hg = 0;
+  auto resolve_pending = [&]() {
+    if (!pend) return;
+    const uint32_t t = __shfl_sync(kFull, pend_ticket, 0);
+    if (t == pend_nseg - 1) merge_partials<GT, D>(p, pend_slot0, (int)pend_nseg, pend_s, pend_hg, lane);
+    pend = false;
+  };
+
+  bool aborted = false;
+  while (cpos < n_total) {
+    if (cpos == cur.r0 + cur.n) {  // step into the next window
+      const bool new_unit = (nxt.s != cur.s) || (nxt.hg != cur.hg);
+      cur = nxt;
+      rc = rn;
+      if (!rc.meta) load_meta(cur, rc);
+      nxt = next_win(cur);
+      load_ids(nxt, rn);
+      if (nxt.n > 0 && (nxt.s != cur.s || nxt.hg != cur.hg)) prefetch_q<GT, D>(p, nxt.s, nxt.hg, lane);
+      if (new_unit) {
+        eng.begin(p, cur.s, cur.hg, lane);
+        seg_j0 = cur.j0;
+      }
+    }
+    issue_ahead();
+    const int st = cst;
+    if (!__all_sync(kFull, mbar_wait_bounded(&my_bars[st], cpar))) {
+      if (lane == 0) record_error(p.dev_error, PKV_DEVERR_TIMEOUT);
+      aborted = true;
+      break;
+    }
+
+    // ---- one block: q . k, online softmax, p . v ----
+    const int kw_i = cpos - cur.r0;
+    const float ks = __shfl_sync(kFull, rc.ks, kw_i) * p.scale_log2;  // per-block K scale, log2 domain
+    const float vs = __shfl_sync(kFull, rc.vs, kw_i);
+    const float nzb = -(kMagic + __shfl_sync(kFull, rc.zp, kw_i));
+    const bool valid = __shfl_sync(kFull, rc.valid ? 1 : 0, kw_i) != 0;
+    const uint8_t* kt = my_stages + (size_t)st * C::STAGE;
+    eng.block(kt, kt + C::K_TILE, ks, vs, nzb, valid, (cur.j0 + kw_i) * BS, cur.L, p.scale_log2);
+    __syncwarp();  // the stage's reads are complete (their values were consumed above)
+    ++cpos;
+    if (++cst == C::NS) {
+      cst = 0;
+      cpar ^= 1u;
+    }
+
+    // ---- end of a segment: the unit's last block, or the end of this warp's range ----
+    const int j_end = cur.j0 + kw_i + 1;
+    if (j_end == cur.nblk || cpos == n_total) {
+      eng.finish();
+      const long long u = (long long)cur.s * HG + cur.hg;
+      if (seg_j0 == 0 && j_end == cur.nblk) {
+        eng.write_out(p, cur.s, cur.hg);  // the whole unit was processed by this warp
+      } else {
+        // one segment of a split unit: publish the partial; the last warp to finish merges
+        eng.write_partial(p, u + w, lane);
+        const long long unit_p0 = cur.seq_p0 + (long long)cur.hg * cur.nblk;
+        const int w_first = owner_of(unit_p0, T, We);
+        const int w_last = owner_of(unit_p0 + cur.nblk - 1, T, We);
+        const uint32_t n_seg = (uint32_t)(w_last - w_first + 1);
+        __syncwarp();  // the warp's partial writes precede lane 0's release below
+        if constexpr (kDeferTicket) resolve_pending();
+        if (lane == 0) pend_ticket = atomic_inc_acq_rel_gpu(&p.ws_count[u], n_seg - 1);
+        pend = true;
+        pend_nseg = n_seg;
+        pend_slot0 = u + w_first;
+        pend_s = cur.s;
+        pend_hg = cur.hg;
+        if constexpr (!kDeferTicket) resolve_pending();
+      }
+      eng.reset();
+      seg_j0 = j_end;  // (a new unit restarts it at its first block)
+    }
+  }
+
+  if constexpr (kDeferTicket) resolve_pending();
+  if (aborted && lane == 0) {
+    // A copy never completed (outputs touched by this warp are unspecified; dev_error says so).
+    // Wait, again bounded, for the copies this warp issued and did not consume, so that no bulk
+    // copy is still writing this CTA's shared memory when it exits.
+    for (int k = cpos; k < ipos; ++k) (void)mbar_wait_bounded(&my_bars[k % C::NS], (uint32_t)((k / C::NS) & 1));
+  }
+  if constexpr (FUSED) grid_exit(sp.bar, gridDim.x);
+}
+
+template <int KT, int VT, int BS, int D, int GT>
+cudaError_t launch_one(const DecodeParams& p, const StepParams& sp, const DecodeShape& sh, cudaStream_t stream) {
+  using C = Cfg<KT, VT, BS, D, GT>;
+  auto kern = sp.fused ? paged_decode_kernel<KT, VT, BS, D, GT, true> : paged_decode_kernel<KT, VT, BS, D, GT, false>;
+  static unsigned long long configured[2] = {0, 0};  // one bit per device and variant; benign race
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(configured[sp.fused ? 1 : 0] & bit)) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    configured[sp.fused ? 1 : 0] |= bit;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(sh.grid_ctas);
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  if (sp.fused) {
+    // the grid barriers need every CTA resident at once: a cooperative launch guarantees it
+    // (or fails to launch)
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+  } else {
+    // programmatic dependent launch: the kernel may start while the previous kernel in the
+    // stream finishes; it waits for it (griddepcontrol.wait) before reading the pool
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p, sp);
+}
+
+template <int KT, int VT, int BS, int D, int GT>
+bool info_one(DecodeKernelInfo* info) {
+  using C = Cfg<KT, VT, BS, D, GT>;
+  info->warps_per_cta = C::NW;
+  info->ctas_per_sm = C::CTAS_PER_SM;
+  info->smem_bytes = C::SMEM;
+  info->stages = C::NS;
+  return true;
+}
+
+// 8 heads per warp exist only with the tensor-core engine
+template <int KT, int VT, int BS, int D>
+cudaError_t launch_one8(const DecodeParams& p, const StepParams& sp, const DecodeShape& sh, cudaStream_t stream) {
+  if constexpr (Cfg<KT, VT, BS, D, 8>::MMA) return launch_one<KT, VT, BS, D, 8>(p, sp, sh, stream);
+  else return cudaErrorInvalidValue;
+}
+template <int KT, int VT, int BS, int D>
+bool info_one8(DecodeKernelInfo* info) {
+  if constexpr (Cfg<KT, VT, BS, D, 8>::MMA) return info_one<KT, VT, BS, D, 8>(info);
+  else return false;
+}
+
+// FN<KT, VT, BS, D, GT>(args...) for the instantiation matching `sh`
+#define PKV_DISPATCH_GT(KT, VT, BS, D, FN, ...)       \
+  switch (sh.heads_per_warp) {                        \
+    case 1: return FN<KT, VT, BS, D, 1>(__VA_ARGS__); \
+    case 2: return FN<KT, VT, BS, D, 2>(__VA_ARGS__); \
+    case 4: return FN<KT, VT, BS, D, 4>(__VA_ARGS__); \
+    case 8: return FN##8<KT, VT, BS, D>(__VA_ARGS__); \
+    default: break;                                   \
+  }
+#define PKV_DISPATCH_D(KT, VT, BS, FN, ...)                   \
+  switch (sh.head_dim) {                                      \
+    case 64: PKV_DISPATCH_GT(KT, VT, BS, 64, FN, __VA_ARGS__) break;   \
+    case 128: PKV_DISPATCH_GT(KT, VT, BS, 128, FN, __VA_ARGS__) break; \
+    case 256: PKV_DISPATCH_GT(KT, VT, BS, 256, FN, __VA_ARGS__) break; \
+    default: break;                                           \
+  }
+#define PKV_DISPATCH_BS(KT, VT, FN, ...)                      \
+  switch (sh.block_size) {                                    \
+    case 16: PKV_DISPATCH_D(KT, VT, 16, FN, __VA_ARGS__) break; \
+    case 32: PKV_DISPATCH_D(KT, VT, 32, FN, __VA_ARGS__) break; \
+    default: break;                                           \
+  }
+}  // namespace
+}  // namespace pkv
