@@ -17,14 +17,14 @@ __device__ __forceinline__ void record_error(int32_t* dev_error, int32_t code) {
   if (dev_error != nullptr) atomicCAS(dev_error, 0, code);
 }
 
-// atomicInc with acquire-release semantics at GPU scope: the caller's earlier writes (and those
-// of its warp, ordered before it by __syncwarp) are visible to whoever observes the new value,
-// and writes released by earlier incrementers are visible to the caller afterwards.
-__device__ __forceinline__ uint32_t atomic_inc_acq_rel_gpu(uint32_t* addr, uint32_t wrap) {
+// atomicInc with no ordering of its own (a split-unit ticket taken after a separate release
+// fence; the warp that gets the last ticket fences again before reading the partials).
+__device__ __forceinline__ uint32_t atomic_inc_relaxed_gpu(uint32_t* addr, uint32_t wrap) {
   uint32_t old;
-  asm volatile("atom.acq_rel.gpu.global.inc.u32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(wrap) : "memory");
+  asm volatile("atom.relaxed.gpu.global.inc.u32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(wrap) : "memory");
   return old;
 }
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
 // ---- integer code -> float conversion without I2F -------------------------------------------
 // IEEE-754 binary32 with exponent field 150 (bit pattern 0x4B000000 | m, m < 2^23) is exactly

@@ -923,6 +923,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
     r.meta = true;
   };
 
+  prefetch_q<GT, D>(p, cur.s, cur.hg, lane);
   WinLanes rc, rn;
   load_ids(cur, rc);
   Win nxt = next_win(cur);
@@ -941,10 +942,6 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
   load_meta(cur, rc);
   __syncwarp();  // barrier initialisation by lane 0 is visible to the warp
 
-  // ---- per-unit state: the arithmetic engine for GT query heads ----
-  EngineFor<KT, VT, BS, D, GT> eng;
-  int seg_j0 = cur.j0;  // first block of the current segment within its unit
-  eng.begin(p, cur.s, cur.hg, lane);
 
   // ---- the copy ring ----
   auto issue = [&](int st, int b, int g) {
@@ -980,21 +977,43 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
     }
   };
 
-  // With one query head per warp (registers to spare), a split unit's ticket is taken without
-  // waiting for the answer; it is read at this warp's next split-unit end (or after its last
-  // block), and if it says "last", that is when the merge runs. Otherwise it is read at once.
+  // A split unit's ticket. The warp that writes a partial must make it visible before its ticket
+  // counts (a release fence, then a relaxed increment); only the warp that gets the last ticket
+  // needs the partials of the others (an acquire fence, then the merge). The release fence waits
+  // for the warp's outstanding writes, so with one query head per warp (registers to spare) the
+  // ticket is taken two blocks later, when the partial's writes have long completed, and read at
+  // the next split-unit end (or after the last block). Otherwise all of it happens at once.
   constexpr bool kDeferTicket = GT == 1;
-  bool pend = false;
-  uint32_t pend_ticket = 0;  // lane 0: the atomic's result
+  int pend = 0;              // 0: none; 1: partial written, ticket not taken; 2: ticket taken
+  int pend_since = 0;        // cpos when the partial was written
+  uint32_t pend_ticket = 0;  // lane 0: the increment's result
   uint32_t pend_nseg = 0;
-  long long pend_slot0 = 0;
+  long long pend_slot0 = 0, pend_u = 0;
   int pend_s = 0, pend_hg = 0;
-  auto resolve_pending = [&]() {
-    if (!pend) return;
-    const uint32_t t = __shfl_sync(kFull, pend_ticket, 0);
-    if (t == pend_nseg - 1) merge_partials<GT, D>(p, pend_slot0, (int)pend_nseg, pend_s, pend_hg, lane);
-    pend = false;
+  auto take_ticket = [&]() {
+    if (lane == 0) {
+      fence_acq_rel_gpu();
+      pend_ticket = atomic_inc_relaxed_gpu(&p.ws_count[pend_u], pend_nseg - 1);
+    }
+    pend = 2;
   };
+  auto resolve_pending = [&]() {
+    if (pend == 0) return;
+    if (pend == 1) take_ticket();
+    const uint32_t t = __shfl_sync(kFull, pend_ticket, 0);
+    if (t == pend_nseg - 1) {
+      fence_acq_rel_gpu();
+      merge_partials<GT, D>(p, pend_slot0, (int)pend_nseg, pend_s, pend_hg, lane);
+    }
+    pend = 0;
+  };
+
+  // the first copies go out before the engine's set-up (which waits for q)
+  issue_ahead();
+  // ---- per-unit state: the arithmetic engine for GT query heads ----
+  EngineFor<KT, VT, BS, D, GT> eng;
+  int seg_j0 = cur.j0;  // first block of the current segment within its unit
+  eng.begin(p, cur.s, cur.hg, lane);
 
   bool aborted = false;
   while (cpos < n_total) {
@@ -1028,6 +1047,9 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
     const uint8_t* kt = my_stages + (size_t)st * C::STAGE;
     eng.block(kt, kt + C::K_TILE, ks, vs, nzb, valid, (cur.j0 + kw_i) * BS, cur.L, p.scale_log2);
     __syncwarp();  // the stage's reads are complete (their values were consumed above)
+    if constexpr (kDeferTicket) {
+      if (pend == 1 && cpos >= pend_since + 2) take_ticket();
+    }
     ++cpos;
     if (++cst == C::NS) {
       cst = 0;
@@ -1048,11 +1070,12 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
         const int w_first = owner_of(unit_p0, T, We);
         const int w_last = owner_of(unit_p0 + cur.nblk - 1, T, We);
         const uint32_t n_seg = (uint32_t)(w_last - w_first + 1);
-        __syncwarp();  // the warp's partial writes precede lane 0's release below
+        __syncwarp();  // the warp's partial writes precede lane 0's release fence
         if constexpr (kDeferTicket) resolve_pending();
-        if (lane == 0) pend_ticket = atomic_inc_acq_rel_gpu(&p.ws_count[u], n_seg - 1);
-        pend = true;
+        pend = 1;
+        pend_since = cpos;
         pend_nseg = n_seg;
+        pend_u = u;
         pend_slot0 = u + w_first;
         pend_s = cur.s;
         pend_hg = cur.hg;
