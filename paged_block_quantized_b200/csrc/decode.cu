@@ -1,9 +1,48 @@
 // decode.cu -- the decode entry points behind the C ABI: heads per warp, supported shapes, and the
 // dispatch to the kernel instantiations of each dtype pair (decode_i8i8.cu, decode_i8i4.cu,
 // decode_f16.cu; the kernel itself is in decode_kernel.cuh).
+#include <cudaTypedefs.h>
+
 #include "internal.h"
 
 namespace pkv {
+
+bool encode_tile_map(CUtensorMap* map, const void* base, uint64_t rows, int row_bytes, int box_rows) {
+  // the driver's encoder, looked up once through the runtime (no link against the driver library)
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  if (encode == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+      return false;
+    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  if (row_bytes % 128 != 0 || row_bytes / 128 > 8 || box_rows <= 0 || box_rows > 256) return false;
+  const cuuint32_t units = (cuuint32_t)(row_bytes / 128);
+  const cuuint32_t rank = units == 1 ? 2 : 3;
+  // innermost: 128 bytes; then (3-D only) the 128-byte units of a row; then the rows
+  cuuint64_t dims[3], strides[2];
+  cuuint32_t box[3], estr[3] = {1, 1, 1};
+  dims[0] = 128;
+  box[0] = 128;
+  if (rank == 2) {
+    dims[1] = rows;
+    strides[0] = 128;
+    box[1] = (cuuint32_t)box_rows;
+  } else {
+    dims[1] = units;
+    dims[2] = rows;
+    strides[0] = 128;
+    strides[1] = (cuuint64_t)row_bytes;
+    box[1] = units;
+    box[2] = (cuuint32_t)box_rows;
+  }
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, const_cast<void*>(base), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
 
 int32_t decode_heads_per_warp(int32_t group, int32_t k_dtype, int32_t v_dtype, int32_t head_dim) {
   const bool mma = (k_dtype == PKV_INT8_SYM && v_dtype == PKV_INT8_SYM && head_dim >= 128) ||

@@ -34,6 +34,7 @@
 //     self-resetting atomicInc ticket) merges them. No CTA barrier, no second kernel.
 #pragma once
 
+#include <cstring>
 #include <type_traits>
 
 #include "common.cuh"
@@ -84,10 +85,15 @@ struct Cfg {
   static constexpr int THREADS = 32 * NW;
   static constexpr int SMEM_STAGES = NW * NS * STAGE;
   static constexpr int SMEM_BAR_FLAG = SMEM_STAGES + NW * NS * 8;  // one int: a grid barrier's outcome
-  static constexpr int SMEM = SMEM_BAR_FLAG + 16;
+  // The tensor-core engine's tiles arrive by tiled copies with 128-byte swizzle, whose shared
+  // destinations must be 1024-byte aligned: the stages start on the next 1024-byte boundary.
+  static constexpr int SMEM_ALIGN = MMA ? 1024 : 0;
+  static constexpr int SMEM = SMEM_BAR_FLAG + 16 + SMEM_ALIGN;
   static constexpr int CTAS_PER_SM = 1;
   static_assert(D % 16 == 0 && D / 16 <= 32, "head_dim");
   static_assert(K_TILE % 16 == 0 && V_TILE % 16 == 0 && STAGE % 16 == 0, "bulk copy granularity");
+  static_assert(!MMA || (K_ROW % 128 == 0 && V_ROW % 128 == 0 && K_TILE % 1024 == 0 && V_TILE % 1024 == 0),
+                "swizzled tiles: 128-byte row units, 1024-byte aligned tiles");
   static_assert(NW >= 1 && SMEM <= 227 * 1024, "shared memory per CTA");
 };
 
@@ -375,6 +381,16 @@ struct CoreEngine {
   }
 };
 
+// Byte offset of (row r, byte x) in a tile of R-byte rows stored by a tiled copy with 128-byte
+// swizzle: rows are cut into 128-byte units (unit u = r * R/128 + x/128), and within unit u the
+// 16-byte chunk j sits at chunk j ^ (u mod 8). Rows of 128 or 256 bytes otherwise all start on
+// bank 0, and the fragment loads below (the same column of several rows at once) would conflict.
+template <int R>
+__device__ __forceinline__ int swz(int r, int x) {
+  const int u = r * (R / 128) + (x >> 7);
+  return (u << 7) | ((((x >> 4) & 7) ^ (u & 7)) << 4) | (x & 15);
+}
+
 // ---- tensor-core helpers (mma.sync m16n8k16, fp16 operands, fp32 accumulators) ----
 __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -453,13 +469,12 @@ struct MmaEngine {
     for (int h2 = 0; h2 < BS / 16; ++h2) {
       // ---- S = K . q^T over this 16-token slice ----
       float sacc[4] = {0.f, 0.f, 0.f, 0.f};
-      const uint8_t* k0 = kt + (16 * h2 + g) * C::K_ROW + c * (C::K_ROW / 4);
-      const uint8_t* k1 = k0 + 8 * C::K_ROW;
+      const int kr0 = 16 * h2 + g, kx = c * (C::K_ROW / 4);  // rows kr0, kr0 + 8 from byte kx
       if constexpr (KT == PKV_INT8_SYM) {
 #pragma unroll
         for (int i = 0; i < KS / 4; ++i) {  // 16 codes = 4 steps per 16-byte load
-          const uint4 r0 = *reinterpret_cast<const uint4*>(k0 + 16 * i);
-          const uint4 r1 = *reinterpret_cast<const uint4*>(k1 + 16 * i);
+          const uint4 r0 = *reinterpret_cast<const uint4*>(kt + swz<C::K_ROW>(kr0, kx + 16 * i));
+          const uint4 r1 = *reinterpret_cast<const uint4*>(kt + swz<C::K_ROW>(kr0 + 8, kx + 16 * i));
           const uint32_t w0[4] = {r0.x, r0.y, r0.z, r0.w};
           const uint32_t w1[4] = {r1.x, r1.y, r1.z, r1.w};
 #pragma unroll
@@ -477,8 +492,8 @@ struct MmaEngine {
       } else {
 #pragma unroll
         for (int i = 0; i < KS / 2; ++i) {  // 8 halves = 2 steps per 16-byte load
-          const uint4 r0 = *reinterpret_cast<const uint4*>(k0 + 16 * i);
-          const uint4 r1 = *reinterpret_cast<const uint4*>(k1 + 16 * i);
+          const uint4 r0 = *reinterpret_cast<const uint4*>(kt + swz<C::K_ROW>(kr0, kx + 16 * i));
+          const uint4 r1 = *reinterpret_cast<const uint4*>(kt + swz<C::K_ROW>(kr0 + 8, kx + 16 * i));
           uint32_t a[4] = {r0.x, r1.x, r0.y, r1.y};
           mma_16816(sacc, a, qb[2 * i][0], qb[2 * i][1]);
           uint32_t b[4] = {r0.z, r1.z, r0.w, r1.w};
@@ -528,14 +543,14 @@ struct MmaEngine {
       const uint32_t bh0 = movmatrix_trans(hi0), bh1 = movmatrix_trans(hi1);
       const uint32_t bl0 = movmatrix_trans(lo0), bl1 = movmatrix_trans(lo1);
       // ---- O^T += V^T . P^T: token rows 2c, 2c+1, 2c+8, 2c+9 at dims [g*D/8, (g+1)*D/8) ----
-      const uint8_t* vb = vt + (16 * h2 + 2 * c) * C::V_ROW + g * (C::V_ROW / 8);
+      const int vr = 16 * h2 + 2 * c, vx = g * (C::V_ROW / 8);  // rows vr, +1, +8, +9 from byte vx
       if constexpr (VT == PKV_INT8_SYM) {
 #pragma unroll
         for (int i = 0; i < KS / 8; ++i) {  // 16 bytes per row = 8 dim tiles
-          const uint4 ra = *reinterpret_cast<const uint4*>(vb + 16 * i);
-          const uint4 rb = *reinterpret_cast<const uint4*>(vb + C::V_ROW + 16 * i);
-          const uint4 rc = *reinterpret_cast<const uint4*>(vb + 8 * C::V_ROW + 16 * i);
-          const uint4 rd = *reinterpret_cast<const uint4*>(vb + 9 * C::V_ROW + 16 * i);
+          const uint4 ra = *reinterpret_cast<const uint4*>(vt + swz<C::V_ROW>(vr, vx + 16 * i));
+          const uint4 rb = *reinterpret_cast<const uint4*>(vt + swz<C::V_ROW>(vr + 1, vx + 16 * i));
+          const uint4 rc = *reinterpret_cast<const uint4*>(vt + swz<C::V_ROW>(vr + 8, vx + 16 * i));
+          const uint4 rd = *reinterpret_cast<const uint4*>(vt + swz<C::V_ROW>(vr + 9, vx + 16 * i));
           const uint32_t xa[4] = {ra.x, ra.y, ra.z, ra.w}, xb[4] = {rb.x, rb.y, rb.z, rb.w};
           const uint32_t xc[4] = {rc.x, rc.y, rc.z, rc.w}, xd[4] = {rd.x, rd.y, rd.z, rd.w};
 #pragma unroll
@@ -556,10 +571,10 @@ struct MmaEngine {
       } else {
 #pragma unroll
         for (int i = 0; i < KS / 4; ++i) {  // 16 bytes per row = 8 halves = 4 dim tiles
-          const uint4 ra = *reinterpret_cast<const uint4*>(vb + 16 * i);
-          const uint4 rb = *reinterpret_cast<const uint4*>(vb + C::V_ROW + 16 * i);
-          const uint4 rc = *reinterpret_cast<const uint4*>(vb + 8 * C::V_ROW + 16 * i);
-          const uint4 rd = *reinterpret_cast<const uint4*>(vb + 9 * C::V_ROW + 16 * i);
+          const uint4 ra = *reinterpret_cast<const uint4*>(vt + swz<C::V_ROW>(vr, vx + 16 * i));
+          const uint4 rb = *reinterpret_cast<const uint4*>(vt + swz<C::V_ROW>(vr + 1, vx + 16 * i));
+          const uint4 rc = *reinterpret_cast<const uint4*>(vt + swz<C::V_ROW>(vr + 8, vx + 16 * i));
+          const uint4 rd = *reinterpret_cast<const uint4*>(vt + swz<C::V_ROW>(vr + 9, vx + 16 * i));
           const uint32_t xa[4] = {ra.x, ra.y, ra.z, ra.w}, xb[4] = {rb.x, rb.y, rb.z, rb.w};
           const uint32_t xc[4] = {rc.x, rc.y, rc.z, rc.w}, xd[4] = {rd.x, rd.y, rd.z, rd.w};
 #pragma unroll
@@ -757,9 +772,11 @@ __device__ __noinline__ void step_store(const StoreParams& sp, int w, int W, int
 
 template <int KT, int VT, int BS, int D, int GT, bool FUSED>
 __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, BS, D, GT>::CTAS_PER_SM)
-    paged_decode_kernel(const DecodeParams p, const StepParams sp) {
+    paged_decode_kernel(const DecodeParams p, const StepParams sp, const __grid_constant__ TileMaps tm) {
   using C = Cfg<KT, VT, BS, D, GT>;
-  extern __shared__ __align__(128) uint8_t smem[];
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  constexpr uint32_t kAlign = C::SMEM_ALIGN ? C::SMEM_ALIGN : 1;
+  uint8_t* const smem = smem_raw + ((kAlign - (smem_addr(smem_raw) & (kAlign - 1))) & (kAlign - 1));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int W = gridDim.x * C::NW;
@@ -948,9 +965,17 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
     const size_t tile = (size_t)b * p.num_kv_heads + g;
     uint8_t* dst = my_stages + (size_t)st * C::STAGE;
     mbar_arrive_expect_tx(&my_bars[st], (uint32_t)C::STAGE);
-    bulk_g2s(dst, static_cast<const uint8_t*>(p.k_codes) + tile * C::K_TILE, (uint32_t)C::K_TILE, &my_bars[st]);
-    bulk_g2s(dst + C::K_TILE, static_cast<const uint8_t*>(p.v_codes) + tile * C::V_TILE, (uint32_t)C::V_TILE,
-             &my_bars[st]);
+    if constexpr (C::MMA) {  // tiled copies: the tile's BS rows from row tile * BS, swizzled
+      const int row = (int)(tile * BS);
+      if constexpr (C::K_ROW == 128) tma_load_2d(dst, &tm.k, 0, row, &my_bars[st]);
+      else tma_load_3d(dst, &tm.k, 0, 0, row, &my_bars[st]);
+      if constexpr (C::V_ROW == 128) tma_load_2d(dst + C::K_TILE, &tm.v, 0, row, &my_bars[st]);
+      else tma_load_3d(dst + C::K_TILE, &tm.v, 0, 0, row, &my_bars[st]);
+    } else {
+      bulk_g2s(dst, static_cast<const uint8_t*>(p.k_codes) + tile * C::K_TILE, (uint32_t)C::K_TILE, &my_bars[st]);
+      bulk_g2s(dst + C::K_TILE, static_cast<const uint8_t*>(p.v_codes) + tile * C::V_TILE, (uint32_t)C::V_TILE,
+               &my_bars[st]);
+    }
   };
   // positions relative to `start`: consumed (cpos) and issued (ipos); stage / parity of each
   int cpos = 0, ipos = 0, cst = 0, ist = 0;
@@ -1129,7 +1154,14 @@ cudaError_t launch_one(const DecodeParams& p, const StepParams& sp, const Decode
   }
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, p, sp);
+  TileMaps tm;
+  memset(&tm, 0, sizeof(tm));
+  if constexpr (C::MMA) {
+    const uint64_t rows = (uint64_t)p.num_blocks * p.num_kv_heads * BS;
+    if (!encode_tile_map(&tm.k, p.k_codes, rows, C::K_ROW, BS) || !encode_tile_map(&tm.v, p.v_codes, rows, C::V_ROW, BS))
+      return cudaErrorInvalidValue;
+  }
+  return cudaLaunchKernelEx(&cfg, kern, p, sp, tm);
 }
 
 template <int KT, int VT, int BS, int D, int GT>

@@ -1,6 +1,7 @@
 // internal.h -- kernel launch interfaces behind the C ABI (not part of the public header).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -55,6 +56,15 @@ bool decode_supported(int32_t k_dtype, int32_t v_dtype, int32_t block_size, int3
 bool decode_kernel_info(const DecodeShape& sh, DecodeKernelInfo* info);
 
 cudaError_t launch_decode(const DecodeParams& p, const DecodeShape& sh, cudaStream_t stream);
+
+// Tensor maps of the K and V code pools for the tensor-core engine's tiled copies: the pool as
+// rows of `row_bytes` (a multiple of 128; 2-D, or 3-D in 128-byte units), boxes of `box_rows`
+// rows, 128-byte swizzle. False if the driver cannot encode it.
+struct TileMaps {
+  CUtensorMap k;
+  CUtensorMap v;
+};
+bool encode_tile_map(CUtensorMap* map, const void* base, uint64_t rows, int row_bytes, int box_rows);
 
 // ---------------------------------------------------------------- store
 struct StoreParams {

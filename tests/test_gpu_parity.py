@@ -103,6 +103,11 @@ def test_split_matches_unsplit():
     dict(head_dim=64, block_size=16, num_q_heads=12, num_kv_heads=4, v_dtype=W.INT4_ASYM),
     dict(head_dim=256, block_size=32, num_q_heads=4, num_kv_heads=1, v_dtype=W.INT4_ASYM),
     dict(head_dim=64, block_size=16, num_q_heads=4, num_kv_heads=2, k_dtype=W.FP16, v_dtype=W.FP16),
+    # tensor-core engine: FP16 with 256-byte rows, INT8 with head_dim 256, block size 32, 4 heads
+    dict(head_dim=128, block_size=16, num_q_heads=32, num_kv_heads=4, k_dtype=W.FP16, v_dtype=W.FP16),
+    dict(head_dim=256, block_size=32, num_q_heads=16, num_kv_heads=2),
+    dict(head_dim=64, block_size=32, num_q_heads=16, num_kv_heads=4, k_dtype=W.FP16, v_dtype=W.FP16),
+    dict(head_dim=128, block_size=32, num_q_heads=16, num_kv_heads=4),
 ])
 def test_shapes_and_groups(case):
     lens = [1, 2, 16, 17, 31, 32, 33, 100, 700]
