@@ -330,16 +330,15 @@ def run_pkv(args, rank, world, local):
     # ---- e2e: same step through the public runner with host buffers copied in and out ----
     e2e = None
     if not args.no_e2e:
-        pin = lambda t: t.cpu().pin_memory()
-        host_in = {"q": pin(g.q), "k_new": pin(g.k_new), "v_new": pin(g.v_new), "step_slots": pin(g.step_slots),
-                   "block_tables": pin(g.block_tables), "context_lens": pin(g.context_lens), "cow": pin(g.cow)}
+        # the step's inputs (q, new K/V, slots, block tables, lengths, copy pairs) are one packed
+        # buffer on the device; the host side holds the same bytes in pinned memory
+        host_in = g.inbuf.cpu().pin_memory()
         host_out = torch.empty_like(g.out, device="cpu").pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+        h2d = host_in.numel() * host_in.element_size()
         d2h = host_out.numel() * host_out.element_size()
 
         def e2e_step():
-            for name, t in host_in.items():
-                getattr(g, name).copy_(t, non_blocking=True)
+            g.inbuf.copy_(host_in, non_blocking=True)
             g.step(fused=fused)
             host_out.copy_(g.out, non_blocking=True)
 

@@ -15,6 +15,9 @@ from . import pkv
 from .workloads import Workload
 
 
+_TORCH_DTYPE = {np.dtype(np.float16): torch.float16, np.dtype(np.int32): torch.int32, np.dtype(np.int64): torch.int64}
+
+
 class DeviceStep:
     def __init__(self, w: Workload, device="cuda", poison: int | None = 0xA5, partition_tokens: int | None = None):
         self.w = w
@@ -23,15 +26,24 @@ class DeviceStep:
                                             w.v_dtype, device=self.device, fill=poison)
         self.dev_error = torch.zeros(1, dtype=torch.int32, device=self.device)
         dev = self.device
-        self.q = torch.from_numpy(w.queries()).to(dev)
-        self.out = torch.zeros_like(self.q)
-        self.block_tables = torch.from_numpy(np.ascontiguousarray(w.block_tables)).to(dev)
-        self.context_lens = torch.from_numpy(w.context_lens).to(dev)
+        # the step's inputs live in one device buffer (views below), so that a caller feeding the
+        # step from host memory moves them with one copy
         k_new, v_new = w.new_token_values()
-        self.k_new = torch.from_numpy(k_new).to(dev)
-        self.v_new = torch.from_numpy(v_new).to(dev)
-        self.step_slots = torch.from_numpy(w.step_slots()).to(dev)
-        self.cow = torch.from_numpy(np.ascontiguousarray(w.cow_pairs)).to(dev)
+        inputs = [("q", w.queries()), ("k_new", k_new), ("v_new", v_new), ("step_slots", w.step_slots()),
+                  ("block_tables", w.block_tables), ("context_lens", w.context_lens), ("cow", w.cow_pairs)]
+        offs, total = [], 0
+        for _, a in inputs:
+            offs.append(total)
+            total += (np.ascontiguousarray(a).nbytes + 255) // 256 * 256
+        host = np.zeros(max(total, 256), dtype=np.uint8)
+        for (_, a), o in zip(inputs, offs):
+            a = np.ascontiguousarray(a)
+            host[o:o + a.nbytes] = a.view(np.uint8).reshape(-1)
+        self.inbuf = torch.from_numpy(host).to(dev)
+        for (name, a), o in zip(inputs, offs):
+            t = self.inbuf[o:o + a.nbytes].view(_TORCH_DTYPE[np.dtype(a.dtype)]).view(a.shape)
+            setattr(self, name, t)
+        self.out = torch.zeros_like(self.q)
         self.partition_tokens = w.partition_tokens if partition_tokens is None else partition_tokens
         self.num_workers, self.num_ctas = pkv.pkv_decode_partitioning(
             self.pool.desc, w.num_seqs, w.num_q_heads, w.max_context_len, self.partition_tokens)
