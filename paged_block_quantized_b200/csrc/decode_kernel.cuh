@@ -97,10 +97,10 @@ struct Cfg {
   static_assert(NW >= 1 && SMEM <= 227 * 1024, "shared memory per CTA");
 };
 
-// 16 consecutive fp16 values of one token row (lane chunk) -> 8 float2 (dims in order)
-__device__ __forceinline__ void load_h16(const uint8_t* p, float2 f[8]) {
-  const uint4 w0 = *reinterpret_cast<const uint4*>(p);
-  const uint4 w1 = *reinterpret_cast<const uint4*>(p + 16);
+// 16 fp16 values of one token row (8 at pa, 8 at pb) -> 8 float2 (pa's dims first)
+__device__ __forceinline__ void load_h16(const uint8_t* pa, const uint8_t* pb, float2 f[8]) {
+  const uint4 w0 = *reinterpret_cast<const uint4*>(pa);
+  const uint4 w1 = *reinterpret_cast<const uint4*>(pb);
   const uint32_t u[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
   for (int i = 0; i < 8; ++i) f[i] = __half22float2(*reinterpret_cast<const __half2*>(&u[i]));
@@ -121,7 +121,7 @@ __device__ __forceinline__ void load_v16(const uint8_t* p, float2 neg_bias, floa
     u4x8_to_f32x2(w.x, neg_bias, f);
     u4x8_to_f32x2(w.y, neg_bias, f + 4);
   } else {
-    load_h16(p, f);
+    load_h16(p, p + 16, f);
   }
 }
 
@@ -166,7 +166,14 @@ struct CoreEngine {
   using C = Cfg<KT, VT, BS, D, GT>;
   static constexpr int CH = D / 16, TG = 32 / CH, TPL = BS / TG;
   static_assert(BS % TG == 0, "block_size must cover the token rows of a warp pass");
+  // A lane owns 16 dims: [a, a + 8) and [b, b + 8). With byte codes they are contiguous
+  // (a = 16c, b = a + 8: a lane's 16 codes are one 16-byte load). With fp16 rows (2D bytes),
+  // 16 contiguous dims would put lanes c and c + 4 of a load on the same banks; a = 8c and
+  // b = D/2 + 8c instead make the 8 lanes of each load read 128 contiguous bytes.
+  static constexpr bool SPLIT = (KT == PKV_FP16);
   int c, tg;
+  __device__ __forceinline__ int dim_a() const { return SPLIT ? 8 * c : 16 * c; }
+  __device__ __forceinline__ int dim_b() const { return SPLIT ? D / 2 + 8 * c : 16 * c + 8; }
   float2 qf[GT][8];
   uint32_t qplane[GT][3][4];
   float qinv[GT];
@@ -188,9 +195,9 @@ struct CoreEngine {
     tg = lane / CH;
 #pragma unroll
     for (int hh = 0; hh < GT; ++hh) {
-      const __half* qp = p.q + ((size_t)s * p.num_q_heads + (size_t)hg * GT + hh) * D + c * 16;
-      const uint4 w0 = *reinterpret_cast<const uint4*>(qp);
-      const uint4 w1 = *reinterpret_cast<const uint4*>(qp + 8);
+      const __half* qp = p.q + ((size_t)s * p.num_q_heads + (size_t)hg * GT + hh) * D;
+      const uint4 w0 = *reinterpret_cast<const uint4*>(qp + dim_a());
+      const uint4 w1 = *reinterpret_cast<const uint4*>(qp + dim_b());
       const uint32_t u[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
       for (int i = 0; i < 8; ++i) qf[hh][i] = __half22float2(*reinterpret_cast<const __half2*>(&u[i]));
@@ -266,7 +273,7 @@ struct CoreEngine {
         }
       } else {
         float2 kf[8];
-        load_h16(krow, kf);
+        load_h16(kt + row * C::K_ROW + 2 * dim_a(), kt + row * C::K_ROW + 2 * dim_b(), kf);
 #pragma unroll
         for (int hh = 0; hh < GT; ++hh) {
           float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
@@ -324,7 +331,8 @@ struct CoreEngine {
     for (int i = 0; i < TPL; ++i) {
       const int row = tg + TG * i;
       float2 vf[8];
-      load_v16<VT>(vt + row * C::V_ROW + c * (C::V_ROW / CH), neg_zp_bias, vf);
+      if constexpr (VT == PKV_FP16) load_h16(vt + row * C::V_ROW + 2 * dim_a(), vt + row * C::V_ROW + 2 * dim_b(), vf);
+      else load_v16<VT>(vt + row * C::V_ROW + c * (C::V_ROW / CH), neg_zp_bias, vf);
 #pragma unroll
       for (int hh = 0; hh < GT; ++hh) {
         const float2 pv2 = make_float2(pv[i][hh], pv[i][hh]);
@@ -355,9 +363,14 @@ struct CoreEngine {
 #pragma unroll
     for (int hh = 0; hh < GT; ++hh) {
       const float inv = l_run[hh] > 0.f ? 1.f / l_run[hh] : 0.f;
-      __half2* o = reinterpret_cast<__half2*>(p.out + ((size_t)s * p.num_q_heads + (size_t)hg * GT + hh) * D + c * 16);
+      __half* ob = p.out + ((size_t)s * p.num_q_heads + (size_t)hg * GT + hh) * D;
+      __half2* oa = reinterpret_cast<__half2*>(ob + dim_a());
+      __half2* obb = reinterpret_cast<__half2*>(ob + dim_b());
 #pragma unroll
-      for (int j = 0; j < 8; ++j) o[j] = __floats2half2_rn(acc[hh][j].x * inv, acc[hh][j].y * inv);
+      for (int j = 0; j < 4; ++j) {
+        oa[j] = __floats2half2_rn(acc[hh][j].x * inv, acc[hh][j].y * inv);
+        obb[j] = __floats2half2_rn(acc[hh][4 + j].x * inv, acc[hh][4 + j].y * inv);
+      }
     }
   }
 
@@ -365,10 +378,11 @@ struct CoreEngine {
     if (tg == 0) {
 #pragma unroll
       for (int hh = 0; hh < GT; ++hh) {
-        float4* dst = reinterpret_cast<float4*>(p.ws_acc + ((size_t)slot * GT + hh) * D + c * 16);
+        float* base = p.ws_acc + ((size_t)slot * GT + hh) * D;
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          dst[j] = make_float4(acc[hh][2 * j].x, acc[hh][2 * j].y, acc[hh][2 * j + 1].x, acc[hh][2 * j + 1].y);
+          reinterpret_cast<float4*>(base + (j < 2 ? dim_a() + 4 * j : dim_b() + 4 * (j - 2)))[0] =
+              make_float4(acc[hh][2 * j].x, acc[hh][2 * j].y, acc[hh][2 * j + 1].x, acc[hh][2 * j + 1].y);
       }
     }
     if (lane == 0) {
