@@ -104,6 +104,35 @@ def test_call_validation(pkv):
                                           raise_on_error=False) == pkv.PKV_ERR_UNSUPPORTED
 
 
+def test_step_validation(pkv):
+    """pkv_decode_step checks the arguments of its three parts on the host, before any launch (fake
+    pointers), with the same answers as the separate calls."""
+    d = desc(pkv)
+    E = pkv.PKV_ERR_INVALID_ARG
+    big = 1 << 40
+
+    def step(**kw):
+        return pkv.pkv_decode_step(
+            kw.get("desc", d), kw.get("mapping", 0x6000), kw.get("n_pairs", 1), kw.get("k_new", 0x7000),
+            kw.get("v_new", 0x7800), kw.get("slots", 0x8000), kw.get("T", 2), kw.get("out", 0x9000), 0xA000,
+            kw.get("S", 2), 4, 0xB000, 4, 0xC000, 64, 0.125, 0, kw.get("ws", 0xD000), kw.get("ws_bytes", big),
+            stream=0, raise_on_error=False)
+
+    assert step(n_pairs=-1) == E
+    assert step(T=-1) == E
+    assert step(mapping=None) == E                  # copies requested without a mapping
+    assert step(mapping=0x6002) == E                # misaligned mapping
+    assert step(k_new=0x7008) == E                  # misaligned new values
+    assert step(slots=None) == E
+    assert step(out=None) == E
+    assert step(ws=None) == E
+    assert step(ws_bytes=16) == E
+    assert step(desc=desc(pkv, block_size=8)) == pkv.PKV_ERR_UNSUPPORTED
+    assert step(desc=desc(pkv, k_dtype=pkv.PKV_FP16, v_dtype=pkv.PKV_INT8_SYM)) == pkv.PKV_ERR_UNSUPPORTED
+    # nothing at all to do: no copies, no tokens, no sequences
+    assert step(n_pairs=0, T=0, S=0, mapping=None, k_new=None, v_new=None, slots=None) == pkv.PKV_OK
+
+
 def test_partitioning(pkv):
     d = desc(pkv)
     workers, ctas = pkv.pkv_decode_partitioning(d, 200, 4, 1000, 0)  # a batch that fills the device
