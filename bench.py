@@ -194,11 +194,16 @@ def measured_hbm_peak():
 
 
 def decode_source_hash() -> str:
+    """Hash of the decode kernel's sources with comments and blank lines removed (a profile stays
+    valid across comment edits, not across code changes)."""
     h = hashlib.sha256()
     for name in ("decode_kernel.cuh", "decode_i8i8.cu", "decode_i8i4.cu", "decode_f16.cu", "decode.cu", "common.cuh",
                  "store_impl.cuh", "copy_impl.cuh"):
-        with open(os.path.join(ROOT, "paged_block_quantized_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "paged_block_quantized_b200", "csrc", name), encoding="utf-8") as f:
+            for line in f:
+                code = line.split("//", 1)[0].rstrip()
+                if code:
+                    h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 

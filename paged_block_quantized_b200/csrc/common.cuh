@@ -1,7 +1,7 @@
 // common.cuh -- device helpers shared by the pkv kernels (sm_100a).
 //
 // Holds no quantization or attention arithmetic of its own beyond the integer -> float code
-// conversion; the method's steps live in store.cu, decode.cu and copy.cu.
+// conversion; the method's steps live in store_impl.cuh, decode_kernel.cuh and copy_impl.cuh.
 #pragma once
 
 #include <cuda_fp16.h>

@@ -1,5 +1,5 @@
 // copy_impl.cuh -- copy-on-write block copies, device code shared by the copy kernel (copy.cu)
-// and the fused decode step (decode.cu).
+// and the fused decode step (decode_kernel.cuh).
 //
 // deepinsea.top "PagedAttention 内存管理深度解析", section "Copy-on-Write 机制": sequences forked for
 // beam search share physical blocks, and a block is copied only when one of them is about to write

@@ -20,9 +20,10 @@
 //     the contiguous stream range [w*T/W, (w+1)*T/W), so every warp gets the same number of
 //     blocks whatever the length mix.
 //   * Each warp streams its range through its own ring of NS shared-memory stages: lane 0
-//     issues two 1-D bulk asynchronous copies per block (the contiguous bs x D K tile and V tile
-//     of this head, 1-4 KiB each) that complete on the stage's mbarrier, up to NS blocks ahead
-//     and straight across unit boundaries; the warp reads tiles with 16-byte shared loads.
+//     issues two bulk asynchronous copies per block (the contiguous bs x D K tile and V tile of
+//     this head, 1-4 KiB each; 1-D copies for the CUDA-core engine, tiled copies with 128-byte
+//     swizzle for the tensor-core engine) that complete on the stage's mbarrier, up to NS blocks
+//     ahead and straight across unit boundaries; the warp reads tiles with 16-byte shared loads.
 //   * Block ids are read 32 at a time ("windows", one id per lane) one window ahead; per-block
 //     scales are fetched when the window's first copy is issued, NS blocks before use.
 //   * q . k for INT8 K is exact integer arithmetic: q on a 22-bit fixed-point grid split into
@@ -31,7 +32,10 @@
 //   * Online softmax in the log2 domain (ex2.approx), rescaling only when the running max grows.
 //   * A unit processed entirely by one warp is written out directly. A unit split across warps
 //     gets one partial (max, sum, acc) per warp in the workspace; the last warp to finish (a
-//     self-resetting atomicInc ticket) merges them. No CTA barrier, no second kernel.
+//     self-resetting atomicInc ticket after a release fence) merges them, lanes in parallel over
+//     partials and dims. No CTA barrier, no second kernel.
+//   * Optionally (FUSED) the same launch first does a step's copy-on-write copies and stores with
+//     every warp, behind grid barriers (cooperative launch).
 #pragma once
 
 #include <cstring>

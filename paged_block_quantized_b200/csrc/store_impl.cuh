@@ -1,6 +1,6 @@
 // store_impl.cuh -- the store's device code: quantize new K/V tokens and scatter them into pool
 // blocks, one warp per (token, KV head). Used by the store kernel (store.cu) and by the fused
-// decode step (decode.cu).
+// decode step (decode_kernel.cuh).
 //
 // Follows tbr8.org "如何通过 PagedAttention 与分块量化结合：解决移动端内存碎片化导致的长文本 OOM" §4
 // (store_kv: scale = absmax / 127 per block, codes = x / scale, one scale stored per block and
