@@ -194,10 +194,10 @@ def measured_hbm_peak():
 
 
 def decode_source_hash() -> str:
-    """Hash of the decode kernel's sources with comments and blank lines removed (a profile stays
-    valid across comment edits, not across code changes)."""
+    """Hash of the decode kernel's device sources with comments and blank lines removed (a profile
+    stays valid across comment edits and host-side changes, not across kernel code changes)."""
     h = hashlib.sha256()
-    for name in ("decode_kernel.cuh", "decode_i8i8.cu", "decode_i8i4.cu", "decode_f16.cu", "decode.cu", "common.cuh",
+    for name in ("decode_kernel.cuh", "decode_i8i8.cu", "decode_i8i4.cu", "decode_f16.cu", "common.cuh",
                  "store_impl.cuh", "copy_impl.cuh"):
         with open(os.path.join(ROOT, "paged_block_quantized_b200", "csrc", name), encoding="utf-8") as f:
             for line in f:

@@ -19,6 +19,7 @@ bool encode_tile_map(CUtensorMap* map, const void* base, uint64_t rows, int row_
     encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
   }
   if (row_bytes % 128 != 0 || row_bytes / 128 > 8 || box_rows <= 0 || box_rows > 256) return false;
+  if (rows > (uint64_t)INT32_MAX) return false;  // the copies address rows with a signed 32-bit coordinate
   const cuuint32_t units = (cuuint32_t)(row_bytes / 128);
   const cuuint32_t rank = units == 1 ? 2 : 3;
   // innermost: 128 bytes; then (3-D only) the 128-byte units of a row; then the rows
