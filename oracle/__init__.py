@@ -53,7 +53,8 @@ _lib = None
 def _load():
     global _lib
     if _lib is None:
-        path = _build.build()
+        # PKV_ORACLE_LIB: another build of oracle.c (the mutation test loads seeded-mistake builds)
+        path = os.environ.get("PKV_ORACLE_LIB") or _build.build()
         lib = ctypes.CDLL(path)
         P = ctypes.c_void_p
         lib.oracle_store.argtypes = [P, P, P, P, ctypes.c_int32]
