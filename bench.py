@@ -14,7 +14,10 @@ and the output copied back inside the timed region. `roofline` rates the decode 
 event-timed duration against the measured HBM copy bandwidth. `cpu_baseline` times the CPU
 oracle (binary64) on a bounded sample of the workload (rank 0, one GPU only).
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl pkv|reference]
+The step runs as three launches by default; --fused runs it as one (pkv_decode_step), and the
+roofline then rates that launch with the step's algorithmic bytes.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl pkv|reference] [--fused]
 Multi-GPU: launched under torch.distributed.run, one process per GPU; each rank runs its own
 independently seeded copy of the workload (data-parallel over sequences, no exchange): weak scaling.
 """
