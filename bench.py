@@ -3,9 +3,15 @@
 
 A step is the whole hot path once: copy-on-write block copies (when the workload forks), store of
 one new token per sequence (quantize + scatter, pkv_store_quantized), then decode attention over
-every sequence (pkv_paged_attention_decode). The default workload is the Llama-2-7B-shaped
-decode layer (32 sequences, context lengths U{500..2000}, 32 heads MHA, head_dim 128, block size
-16, 8192-block pool, INT8 K and V with 1% outlier channels).
+every sequence (pkv_paged_attention_decode). The default workload is the mixed serving step, the
+largest one-GPU configuration and the only one that runs all three kernels: 128 sequences with
+lognormal context lengths (median 1000, sigma 1, clamped to [16, 16384]), 32 heads MHA, head_dim
+128, block size 16, INT8 K / INT4 V, 16 beam children forked from 16 parents (16 copy-on-write
+copies per step). Other workloads: --config llama7b | llama7b_fp16 | long | gqa_prefix | tiny.
+
+Every timed step appends tokens that its tiles have not seen yet: before each step (outside the
+timed region) the blocks the step writes are restored from a snapshot taken after the prefill, so
+the store rebuilds tiles at their natural rate (reported as store_rebuilt_tiles).
 
 Prints ONE JSON line (rank 0). `value` is whole-job decode KV tokens/s: tokens attended by all
 ranks / the slowest rank's device time (CUDA events, per step, L2 flushed between steps, inputs
@@ -42,7 +48,12 @@ if ROOT not in sys.path:
 METRIC = "decode KV tokens/s and effective HBM GB/s (fraction of ~8 TB/s) on 1 B200"
 UNIT = "KV tokens/s"
 FALLBACK_HBM_GBS = 6650.0
-KV_NAMES = {0: "fp16", 1: "int8", 2: "int4"}
+KV_NAMES = {0: "fp16", 1: "int8", 2: "int4", 3: "fp8e4m3"}
+
+
+def dtype_label(w) -> str:
+    """The types the path computes in: cache codes, activations, accumulation."""
+    return f"k={KV_NAMES[w.k_dtype]},v={KV_NAMES[w.v_dtype]},q/out=fp16,acc=f32"
 
 
 def parse_args():
@@ -51,7 +62,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("pkv", "reference"), default="pkv")
-    ap.add_argument("--config", default="llama7b")
+    ap.add_argument("--config", default="mixed")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--partition-tokens", type=int, default=None)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-oracle baseline sample")
@@ -286,6 +297,7 @@ def run_pkv(args, rank, world, local):
     w = W.make(args.config, seed=args.seed + rank)
     g = DeviceStep(w, device=dev, poison=None, partition_tokens=args.partition_tokens)
     g.prefill()
+    g.snapshot_step_tiles()
     has_cow = w.cow_pairs.shape[0] > 0
     fused = args.fused
     launches_per_step = 1 if fused else (1 if has_cow else 0) + 2
@@ -293,10 +305,12 @@ def run_pkv(args, rank, world, local):
     flush = L2Flush(dev)
 
     for _ in range(args.warmup):
+        g.restore_step_tiles()
         flush()
         g.step(fused=fused)
     torch.cuda.synchronize(dev)
     assert g.error() == 0, f"device error {g.error()} in warm-up"
+    rebuilt, appended = g.rebuilt_tiles()  # of the last warm-up step, which started from the snapshot
 
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
@@ -309,7 +323,8 @@ def run_pkv(args, rank, world, local):
         torch.cuda.synchronize(dev)
         wall0 = time.perf_counter()
         for i in range(K):
-            flush()                       # outside the events: every step starts with a cold, clean L2
+            g.restore_step_tiles()        # outside the events: first-time appends every step
+            flush()                       # and a cold, clean L2
             ev[i][0].record(stream)
             g.step(fused=fused)
             ev[i][1].record(stream)
@@ -320,6 +335,7 @@ def run_pkv(args, rank, world, local):
         # around the store and the decode
         dev_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
         for i in range(K):
+            g.restore_step_tiles()
             flush()
             g.copy()
             dev_ev[i][0].record(stream)
@@ -351,11 +367,13 @@ def run_pkv(args, rank, world, local):
             host_out.copy_(g.out, non_blocking=True)
 
         for _ in range(args.warmup):
+            g.restore_step_tiles()
             e2e_step()
         torch.cuda.synchronize(dev)
         e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
         dist_barrier(world, dev)
         for i in range(K):
+            g.restore_step_tiles()
             flush()
             e_ev[i][0].record(stream)
             e2e_step()
@@ -385,11 +403,12 @@ def run_pkv(args, rank, world, local):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": total_s * 1e3 / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f32", "data": "synthetic (seeded N(0,1) fp16 K/V/q, permuted block pool)",
+        "dtype": dtype_label(w), "data": "synthetic (seeded N(0,1) fp16 K/V/q, permuted block pool)",
         "config": {**config_block(w, g, step_desc), "parallelism": f"dp{world} (independent sequences per rank)",
                    "l2": "flushed before every timed step (2x L2 written, then 2x L2 read: cold and clean)", "timing": "CUDA events per step"},
         "effective_hbm_gbs": achieved, "frac_of_8tbs": achieved / 8000.0,
         "decode_us": dec_s * 1e6, "store_us": statistics.mean(store_ms) * 1e3,
+        "store_rebuilt_tiles": f"{rebuilt} of {appended} (block, head) tiles appended into (first-time appends)",
         "decode_only_gbs": dec_bytes / dec_s / 1e9,
         "roofline": {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": peak,
                      "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,

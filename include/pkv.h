@@ -41,8 +41,11 @@
  *   - Every GPU entry point only enqueues work on `stream` and returns. PKV_OK means the launch
  *     was accepted; argument errors are detected on the host before anything is launched and
  *     leave all buffers untouched.
- *   - The library allocates no device memory and keeps no global state; scratch space for the
- *     decode is a caller-provided workspace (size from pkv_decode_workspace_size).
+ *   - The library allocates no device memory. Its only global state is one file-scope device
+ *     array (PKV_STATIC_SCRATCH_BYTES per GPU, alive while the library is loaded) that
+ *     pkv_paged_attention_decode_static uses instead of a workspace, plus per-device caches of
+ *     launch facts (SM count, that array's address). Every other call takes its scratch space
+ *     from a caller-provided workspace (size from pkv_decode_workspace_size).
  *   - Data errors that can only be seen on the device (a bad block id in a table, a bad slot)
  *     never trap: the offending work is skipped and, if `dev_error` is non-NULL, the first error
  *     code (PKV_DEVERR_*) is stored there with an atomic compare-and-swap (caller zeroes it).
@@ -194,6 +197,16 @@ PKV_API pkv_status pkv_decode_partitioning(const pkv_cache_desc* desc, int32_t n
  *                the GPU.
  *   dev_error    device int32 or NULL
  * num_q_heads must be a multiple of num_kv_heads.
+ *
+ * Ordering with the preceding work on `stream`: the kernel is launched with programmatic stream
+ * serialization, so it may start while the previous kernel on the stream is still running (the
+ * store of the step's new tokens, which lets the decode's set-up overlap it). Before it waits
+ * for that kernel to complete it reads only context_lens, block_tables and q (and prefetches q);
+ * every read of the pool (codes, scales, zero points) and every write comes after the wait.
+ * So context_lens, block_tables and q must be complete before the previous kernel on the stream
+ * starts: written by an earlier kernel or copy, not by the kernel immediately before this call
+ * when that kernel lets its dependents start early (griddepcontrol.launch_dependents). A
+ * stream-ordered copy, memset or event wait in between is enough.
  */
 PKV_API pkv_status pkv_paged_attention_decode(const pkv_cache_desc* desc, void* out, const void* q,
                                       int32_t num_seqs, int32_t num_q_heads,
@@ -243,6 +256,8 @@ PKV_API pkv_status pkv_decode_step(const pkv_cache_desc* desc, const int32_t* bl
  *   - All calls share the array and it keeps the last call's contents; each call clears, on its
  *     stream, the part that must start at zero. Calls whose executions overlap on the GPU (any
  *     streams, any threads) race on the array and give undefined results: serialise them.
+ *   - Every argument is checked before anything is enqueued: a call that returns an error has
+ *     written nothing, not even the array.
  * Arguments and results are those of pkv_paged_attention_decode without the workspace.
  */
 #define PKV_STATIC_SCRATCH_BYTES (8u << 20)
@@ -251,6 +266,15 @@ PKV_API pkv_status pkv_paged_attention_decode_static(
     const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
     int32_t max_context_len, float softmax_scale, int32_t partition_tokens, int32_t* dev_error,
     pkv_stream_t stream);
+
+/*
+ * pkv_static_scratch_address -- the current device's address of the array that
+ * pkv_paged_attention_decode_static uses, and its size in bytes (either output may be NULL
+ * except device_ptr). For diagnostics and tests, e.g. to check that the call clears what must
+ * start at zero whatever an earlier call or a stray write left there. Like that call, the first
+ * use on a device looks the address up with the device current. The pages have no counterpart.
+ */
+PKV_API pkv_status pkv_static_scratch_address(void** device_ptr, size_t* bytes);
 
 /*
  * pkv_copy_blocks -- copy-on-write block copies ([deepinsea] section "Copy-on-Write 机制";
@@ -286,7 +310,9 @@ PKV_API int32_t pkv_alloc_refcount(const pkv_allocator* h, int32_t block_id);
 PKV_API pkv_status pkv_alloc_blocks(pkv_allocator* h, int32_t n, int32_t* ids);
 /* Share n blocks with another sequence: refcount += 1 each. Ids must be allocated. */
 PKV_API pkv_status pkv_alloc_fork(pkv_allocator* h, const int32_t* ids, int32_t n);
-/* Drop one reference from each of n blocks; a block returns to the free list at 0. */
+/* Drop one reference from each of n blocks; a block returns to the free list at 0. All or nothing:
+ * PKV_ERR_INVALID_ARG (and no change) if an id is out of range or listed more often than it has
+ * references. Cost O(n log n) in the ids, independent of the pool size. */
 PKV_API pkv_status pkv_alloc_release(pkv_allocator* h, const int32_t* ids, int32_t n);
 /* Make block_id private before a write. If its refcount is 1, *new_id = block_id and nothing
  * changes. Otherwise a fresh block is taken (*new_id), the old block's refcount drops by one,

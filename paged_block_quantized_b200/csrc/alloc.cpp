@@ -6,6 +6,7 @@
 // §5 item 3: a pool of physical blocks is set up once and block ids are released through logical
 // reference counts. deepinsea.top, section "Copy-on-Write 机制": sequences share blocks and a block
 // is copied only when a sharer is about to write to it. Host memory only; not thread-safe.
+#include <algorithm>
 #include <cstdint>
 #include <new>
 #include <vector>
@@ -78,9 +79,14 @@ pkv_status pkv_alloc_release(pkv_allocator* h, const int32_t* ids, int32_t n) {
   for (int32_t i = 0; i < n; ++i) {
     if (ids[i] < 0 || (size_t)ids[i] >= h->refcount.size()) return PKV_ERR_INVALID_ARG;
   }
-  std::vector<int32_t> count(h->refcount.size(), 0);
-  for (int32_t i = 0; i < n; ++i) {
-    if (++count[(size_t)ids[i]] > h->refcount[(size_t)ids[i]]) return PKV_ERR_INVALID_ARG;  // double free
+  // runs of equal ids in a sorted copy: cost O(n log n) in the ids, independent of the pool size
+  std::vector<int32_t> sorted(ids, ids + n);
+  std::sort(sorted.begin(), sorted.end());
+  for (size_t i = 0; i < sorted.size();) {
+    size_t j = i + 1;
+    while (j < sorted.size() && sorted[j] == sorted[i]) ++j;
+    if ((int64_t)(j - i) > h->refcount[(size_t)sorted[i]]) return PKV_ERR_INVALID_ARG;  // double free
+    i = j;
   }
   for (int32_t i = 0; i < n; ++i) {
     int32_t& rc = h->refcount[(size_t)ids[i]];

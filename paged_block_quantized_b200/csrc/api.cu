@@ -355,12 +355,25 @@ pkv_status pkv_paged_attention_decode_static(const pkv_cache_desc* desc, void* o
   cudaError_t err = cudaSuccess;
   void* scratch = static_scratch_on_current_device(&err);
   if (scratch == nullptr) return PKV_ERR_CUDA;
+  // every argument is checked before anything is enqueued
+  DecodeParams p;
+  st = make_decode_params(desc, g, out, q, num_seqs, num_q_heads, block_tables, max_blocks_per_seq, context_lens,
+                          max_context_len, softmax_scale, scratch, PKV_STATIC_SCRATCH_BYTES, dev_error, &p);
+  if (st != PKV_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   // the tickets must start at zero: the array holds whatever the previous call left
-  if (cudaMemsetAsync(scratch, 0, g.counter_bytes, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return PKV_ERR_CUDA;
-  return pkv_paged_attention_decode(desc, out, q, num_seqs, num_q_heads, block_tables, max_blocks_per_seq,
-                                    context_lens, max_context_len, softmax_scale, partition_tokens, scratch,
-                                    PKV_STATIC_SCRATCH_BYTES, dev_error, stream);
+  if (cudaMemsetAsync(scratch, 0, g.counter_bytes, s) != cudaSuccess) return PKV_ERR_CUDA;
+  return launch_decode(p, g.shape, s) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+pkv_status pkv_static_scratch_address(void** device_ptr, size_t* bytes) {
+  if (device_ptr == nullptr) return PKV_ERR_INVALID_ARG;
+  cudaError_t err = cudaSuccess;
+  void* scratch = static_scratch_on_current_device(&err);
+  if (scratch == nullptr) return PKV_ERR_CUDA;
+  *device_ptr = scratch;
+  if (bytes != nullptr) *bytes = PKV_STATIC_SCRATCH_BYTES;
+  return PKV_OK;
 }
 
 }  // extern "C"

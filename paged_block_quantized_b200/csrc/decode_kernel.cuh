@@ -1045,7 +1045,11 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
     if (pend == 1) take_ticket();
     const uint32_t t = __shfl_sync(kFull, pend_ticket, 0);
     if (t == pend_nseg - 1) {
-      fence_acq_rel_gpu();
+      // Lane 0 read the last ticket: its acquire fence orders the other warps' partials (released
+      // before their increments) before its later reads; the warp barrier then extends that
+      // order to every lane of the warp before any of them reads a partial.
+      if (lane == 0) fence_acq_rel_gpu();
+      __syncwarp();
       merge_partials<GT, D>(p, pend_slot0, (int)pend_nseg, pend_s, pend_hg, lane);
     }
     pend = 0;

@@ -28,7 +28,7 @@ PKV_FP16, PKV_INT8_SYM, PKV_INT4_ASYM = 0, 1, 2
 
 EXPORTED = (
     "pkv_status_string", "pkv_tile_bytes", "pkv_store_quantized", "pkv_decode_workspace_size",
-    "pkv_decode_partitioning", "pkv_paged_attention_decode_static",
+    "pkv_decode_partitioning", "pkv_paged_attention_decode_static", "pkv_static_scratch_address",
     "pkv_paged_attention_decode", "pkv_copy_blocks", "pkv_decode_step", "pkv_blocks_for_tokens", "pkv_alloc_create",
     "pkv_alloc_destroy", "pkv_alloc_num_free", "pkv_alloc_refcount", "pkv_alloc_blocks", "pkv_alloc_fork",
     "pkv_alloc_release", "pkv_alloc_cow",
@@ -75,6 +75,7 @@ _decode = _sig("pkv_paged_attention_decode", ctypes.c_int, _DESC, _P, _P, _I32, 
 _decode_static = _sig("pkv_paged_attention_decode_static", ctypes.c_int, _DESC, _P, _P, _I32, _I32, _P, _I32, _P,
                       _I32, ctypes.c_float, _I32, _P, _P)
 PKV_STATIC_SCRATCH_BYTES = 8 << 20
+_static_addr = _sig("pkv_static_scratch_address", ctypes.c_int, ctypes.POINTER(_P), ctypes.POINTER(ctypes.c_size_t))
 _copy = _sig("pkv_copy_blocks", ctypes.c_int, _DESC, _P, _I32, _P, _P)
 _step = _sig("pkv_decode_step", ctypes.c_int, _DESC, _P, _I32, _P, _P, _P, _I32, _P, _P, _I32, _I32, _P, _I32, _P,
              _I32, ctypes.c_float, _I32, _P, ctypes.c_size_t, _P, _P)
@@ -173,6 +174,13 @@ def pkv_paged_attention_decode_static(desc, out, q, num_seqs, num_q_heads, block
                         int(max_blocks_per_seq), _ptr(context_lens), int(max_context_len), float(softmax_scale),
                         int(partition_tokens), _ptr(dev_error), _stream(stream))
     return _check(st, "pkv_paged_attention_decode_static", raise_on_error)
+
+
+def pkv_static_scratch_address():
+    """(device address, bytes) of the static decode's array on the current device (diagnostics)."""
+    ptr, n = _P(), ctypes.c_size_t(0)
+    _check(_static_addr(ctypes.byref(ptr), ctypes.byref(n)), "pkv_static_scratch_address", True)
+    return int(ptr.value or 0), int(n.value)
 
 
 def pkv_copy_blocks(desc, block_mapping, n_pairs, dev_error=None, stream=None, raise_on_error=True):

@@ -15,6 +15,14 @@ from . import pkv
 from .workloads import Workload
 
 
+class _nullctx:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        return False
+
+
 _TORCH_DTYPE = {np.dtype(np.float16): torch.float16, np.dtype(np.int32): torch.int32, np.dtype(np.int64): torch.int64}
 
 
@@ -61,6 +69,47 @@ class DeviceStep:
             st = torch.from_numpy(slots).to(self.device)
             pkv.pkv_store_quantized(self.pool.desc, kt, vt, st, st.numel(), self.dev_error)
         torch.cuda.synchronize(self.device)
+
+    # ---- first-time appends when a step is repeated ----
+    def snapshot_step_tiles(self):
+        """Remember the pool state of every block the step writes (copy-on-write targets and the
+        blocks receiving the new tokens), so that restore_step_tiles() can put it back: a repeated
+        step then appends tokens its tiles have not seen yet, and the store's rebuilds happen at
+        their natural rate instead of every repeat taking the "fits" path."""
+        bs = self.w.block_size
+        blocks = set(int(b) for b in (self.w.step_slots() // bs))
+        blocks |= set(int(b) for b in self.w.cow_pairs[:, 1]) if self.w.cow_pairs.size else set()
+        self._touched = torch.tensor(sorted(blocks), dtype=torch.int64, device=self.device)
+        p = self.pool
+        self._snap = [t.index_select(0, self._touched) for t in (p.k_codes, p.v_codes, p.k_scale, p.v_scale, p.v_zp)]
+
+    def restore_step_tiles(self, stream=None):
+        """Put the snapshot back (plain device copies on `stream`, outside any timed region)."""
+        p = self.pool
+        with torch.cuda.stream(stream) if stream is not None else _nullctx():
+            for t, s in zip((p.k_codes, p.v_codes, p.k_scale, p.v_scale, p.v_zp), self._snap):
+                t.index_copy_(0, self._touched, s)
+
+    def rebuilt_tiles(self):
+        """After one step from the snapshot: (tiles rebuilt, tiles appended into). A tile is a
+        (block, KV head) pair whose block receives a token at an offset > 0; it was rebuilt when its
+        K or V scale differs from the snapshot (a token at offset 0 starts a fresh tile instead)."""
+        slots = self.w.step_slots()
+        bs = self.w.block_size
+        appended = sorted(set(int(s // bs) for s in slots if s % bs != 0))
+        if not appended:
+            return 0, 0
+        # a copy-on-write target starts the step as a copy of its source: compare it with that
+        ref = {int(d): int(s) for s, d in self.w.cow_pairs}
+        touched = self._touched.cpu().tolist()
+        rows = torch.tensor([touched.index(ref.get(b, b)) for b in appended], device=self.device)
+        blocks = torch.tensor(appended, dtype=torch.int64, device=self.device)
+        p = self.pool
+        ks = p.k_scale.index_select(0, blocks).view(torch.int32)
+        vs = p.v_scale.index_select(0, blocks).view(torch.int32)
+        changed = (ks != self._snap[2].index_select(0, rows).view(torch.int32)) | (
+            vs != self._snap[3].index_select(0, rows).view(torch.int32))
+        return int(changed.sum().item()), int(changed.numel())
 
     # ---- the step ----
     def copy(self, stream=None):

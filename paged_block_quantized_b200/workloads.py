@@ -14,12 +14,12 @@ sequences (if any), store of one new token per sequence at position L-1, then at
 L tokens. Before the step the pool holds positions [0, L-1) of every sequence, stored
 block by block ("prefill").
 
-Named workloads (sizes from the pages' scenarios; see the design doc for the recipe):
+Named workloads (sizes from the pages' scenarios):
   tiny       4 seqs, L = {17, 33, 50, 64}, 4 heads MHA, D 64, bs 16, 64-block pool, INT8/INT8
   llama7b    32 seqs, L ~ U{500..2000}, 32 heads MHA, D 128, bs 16, 8192-block pool, INT8/INT8,
              K/V with 1% outlier channels x8 (``llama7b_fp16``: same with an FP16 cache)
-  long       8 seqs, L ~ U{8192..32768}, 32 heads, D 128, bs 32, K INT8 / V INT4, 512-token
-             partitions
+  long       8 seqs, L ~ U{8192..32768}, 32 heads, D 128, bs 32, K INT8 / V INT4 (the decode
+             splits the long contexts across worker warps itself)
   gqa_prefix 64 seqs, 64 q heads / 8 KV heads, D 128, bs 16, 64 shared prefix blocks then 64
              private blocks each (L = 2048), INT8/INT8
   mixed      128 seqs, L = clamp(round(exp(N(ln 1000, 1))), 16, 16384), 32 heads, D 128, bs 16,
@@ -300,7 +300,7 @@ def make(name: str, seed: int = 0, **over) -> Workload:
         p = dict(num_seqs=S, num_q_heads=32, num_kv_heads=32, head_dim=128, block_size=32,
                  num_blocks=None, k_dtype=INT8_SYM, v_dtype=INT4_ASYM, outliers=False,
                  partition_tokens=0, context_lens=rng.integers(8192, 32769, size=S))
-        desc = "long context: 8 seqs, L~U{8192..32768}, 32 heads, D 128, bs 32, K INT8 / V INT4, 512-token partitions"
+        desc = "long context: 8 seqs, L~U{8192..32768}, 32 heads, D 128, bs 32, K INT8 / V INT4, contexts split across worker warps"
     elif name == "gqa_prefix":
         S = over.get("num_seqs", 64)
         prefix_blocks = over.pop("prefix_blocks", 64)

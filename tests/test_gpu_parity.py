@@ -17,12 +17,14 @@ pytestmark = pytest.mark.gpu
 TOL = 2e-3
 
 
-def run_gpu(w, partition_tokens=None):
+def run_gpu(w, partition_tokens=None, fused=False):
+    """Prefill, then one step: the three launches the benchmark times by default (copy kernel,
+    store kernel, decode with a programmatic dependent launch), or the one-launch pkv_decode_step."""
     from paged_block_quantized_b200.step import DeviceStep
     g = DeviceStep(w, partition_tokens=partition_tokens)
     g.prefill()
     pre = g.pool_numpy()
-    g.step(fused=True)  # one launch; test_fused_step_matches_separate_launches ties it to the three calls
+    g.step(fused=fused)
     torch.cuda.synchronize()
     return g, pre
 
@@ -37,8 +39,8 @@ def assert_pool_equal(gpu_arrays, cache, phys, what):
     np.testing.assert_array_equal(zp[phys], cache.v_zp, err_msg=f"{what}: zero points")
 
 
-def check(w, seqs=None, partition_tokens=None):
-    g, pre = run_gpu(w, partition_tokens)
+def check(w, seqs=None, partition_tokens=None, fused=False):
+    g, pre = run_gpu(w, partition_tokens, fused)
     o = oracle_step(w, seqs)
     assert all(e == 0 for e in o["errors"]), o["errors"]
     assert g.error() == 0
@@ -60,9 +62,10 @@ REDUCED = {
 }
 
 
+@pytest.mark.parametrize("path", ["separate", "fused"])
 @pytest.mark.parametrize("name", list(REDUCED))
-def test_config_reduced_sizes(name):
-    check(W.make(name, seed=0, **REDUCED[name]))
+def test_config_reduced_sizes(name, path):
+    check(W.make(name, seed=0, **REDUCED[name]), fused=path == "fused")
 
 
 FULL_SAMPLES = {
@@ -74,8 +77,9 @@ FULL_SAMPLES = {
 }
 
 
+@pytest.mark.parametrize("path", ["separate", "fused"])
 @pytest.mark.parametrize("name", list(FULL_SAMPLES))
-def test_config_full_size_sampled(name):
+def test_config_full_size_sampled(name, path):
     w = W.make(name, seed=0)
     seqs = FULL_SAMPLES[name]
     if seqs is None:
@@ -83,7 +87,7 @@ def test_config_full_size_sampled(name):
         child = int(np.nonzero((w.block_tables == dst).any(axis=1))[0][0])
         parent = int(np.nonzero((w.block_tables == src).any(axis=1))[0][0])
         seqs = [parent, child, 1, int(np.argmax(w.context_lens))]
-    check(w, seqs)
+    check(w, seqs, fused=path == "fused")
 
 
 def test_split_matches_unsplit():
