@@ -288,6 +288,33 @@ PKV_API pkv_status pkv_static_scratch_address(void** device_ptr, size_t* bytes);
 PKV_API pkv_status pkv_copy_blocks(const pkv_cache_desc* desc, const int32_t* block_mapping,
                            int32_t n_pairs, int32_t* dev_error, pkv_stream_t stream);
 
+/*
+ * pkv_swap_blocks -- move whole blocks between the device pool and a pool in host memory
+ * ([deepinsea] section "Swap 机制": when device memory runs short, KV blocks are swapped out to
+ * CPU memory and back in later; the transfer is slow, so it is a fallback, not a routine step).
+ *
+ * For each pair (src, dst) of block_mapping, every head's K codes, V codes, scales and zero points
+ * of block src of the source pool are copied into block dst of the destination pool:
+ *   direction PKV_SWAP_OUT: device_pool -> host_pool (src is a device block id, dst a host id)
+ *   direction PKV_SWAP_IN:  host_pool -> device_pool (src is a host block id, dst a device id)
+ * The two pools must have the same block_size, num_kv_heads, head_dim and dtypes; num_blocks may
+ * differ. The host pool's arrays must be page-locked host memory that the device can address
+ * (cudaHostAlloc / cudaMallocHost, or cudaHostRegister with cudaHostRegisterMapped), every byte of
+ * each array; the device pool's arrays must be memory of the current device. Both are checked on
+ * the host (both ends of every array) before anything is launched: PKV_ERR_INVALID_ARG otherwise,
+ * never a fault. One kernel moves all pairs, however scattered the ids (reads and writes of host
+ * memory cross the host link directly, many 16-byte accesses in flight). Ids outside their pool
+ * skip the pair and set PKV_DEVERR_BLOCK_ID. Destinations must not repeat.
+ *   block_mapping int32 [n_pairs][2] = {src, dst}, in device memory or mapped page-locked host memory
+ *   dev_error     device int32 (or mapped host int32) or NULL
+ * Host-side bookkeeping stays with the caller: a pkv_allocator per pool (release the device ids
+ * after a swap-out completes, the host ids after a swap-in).
+ */
+typedef enum pkv_swap_dir { PKV_SWAP_OUT = 0, PKV_SWAP_IN = 1 } pkv_swap_dir;
+PKV_API pkv_status pkv_swap_blocks(const pkv_cache_desc* device_pool, const pkv_cache_desc* host_pool,
+                                   const int32_t* block_mapping, int32_t n_pairs, int32_t direction,
+                                   int32_t* dev_error, pkv_stream_t stream);
+
 /* ------------------------------------------------------------------------------------------
  * Host block allocator: free list plus per-block reference counts, host memory only.
  * Ceil-division sizing and the out-of-blocks failure follow [deepinsea] "分页机制设计"
@@ -318,6 +345,42 @@ PKV_API pkv_status pkv_alloc_release(pkv_allocator* h, const int32_t* ids, int32
  * changes. Otherwise a fresh block is taken (*new_id), the old block's refcount drops by one,
  * and the caller must copy old -> new (pkv_copy_blocks) before writing. */
 PKV_API pkv_status pkv_alloc_cow(pkv_allocator* h, int32_t block_id, int32_t* new_id);
+
+/* ------------------------------------------------------------------------------------------
+ * Automatic prefix caching (host memory only): an index from token blocks to physical blocks
+ * ([yunthe] section "Prefix Caching与多轮对话场景优化实践": a new request first looks for blocks in
+ * the pool that already hold its prefix and, on a hit, maps onto them and computes only its new
+ * tokens; section "PagedAttention分页注意力机制与vLLM实现": requests with the same prefix share
+ * physical blocks). Only whole blocks are cached. A block is identified by its block_size token
+ * ids together with all the tokens before it: lookups hash that and then compare it exactly, so a
+ * hash collision never gives a false hit. The cache holds one reference on every block it
+ * indexes, through the pool's pkv_allocator (which must outlive it); a block that only the cache
+ * references is kept for later hits and evicted least recently used first when pkv_prefix_alloc
+ * needs room; evicting a block drops the cached blocks that follow it too. Not thread-safe.
+ * ------------------------------------------------------------------------------------------ */
+typedef struct pkv_prefix_cache pkv_prefix_cache;
+
+PKV_API pkv_status pkv_prefix_cache_create(pkv_allocator* alloc, int32_t block_size, pkv_prefix_cache** out);
+/* Drops every entry (releasing the cache's references) and frees the handle. */
+PKV_API void pkv_prefix_cache_destroy(pkv_prefix_cache* pc);
+/* Cached blocks; cached blocks that only the cache references (evictable). -1 on NULL. */
+PKV_API int32_t pkv_prefix_cache_size(const pkv_prefix_cache* pc);
+PKV_API int32_t pkv_prefix_cache_evictable(const pkv_prefix_cache* pc);
+/* The longest cached prefix of tokens[0, n_tokens) in whole blocks, at most max_blocks: the
+ * physical ids go to block_ids[0, *n_matched), and each of them gains one reference that the
+ * caller owns (release it with pkv_alloc_release when the sequence ends). */
+PKV_API pkv_status pkv_prefix_match(pkv_prefix_cache* pc, const int32_t* tokens, int64_t n_tokens,
+                                    int32_t* block_ids, int32_t max_blocks, int32_t* n_matched);
+/* Registers the whole blocks of a sequence once their K/V are stored: block_ids[i] holds tokens
+ * [i*block_size, (i+1)*block_size). Blocks whose content (with their prefix) is already cached
+ * are left as they are; the cache takes one reference on each newly registered block. The ids
+ * must be allocated (PKV_ERR_INVALID_ARG, and no change, otherwise). */
+PKV_API pkv_status pkv_prefix_insert(pkv_prefix_cache* pc, const int32_t* tokens, int64_t n_tokens,
+                                     const int32_t* block_ids, int32_t n_blocks);
+/* Takes n fresh blocks (refcount 1) from the allocator, evicting least recently used blocks that
+ * only the cache references when too few are free. All or nothing: PKV_ERR_OUT_OF_BLOCKS, with
+ * no eviction, when even evicting every such block would not free enough. */
+PKV_API pkv_status pkv_prefix_alloc(pkv_prefix_cache* pc, int32_t n, int32_t* ids);
 
 #ifdef __cplusplus
 }

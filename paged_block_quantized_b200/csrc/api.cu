@@ -188,6 +188,50 @@ pkv_status make_decode_params(const pkv_cache_desc* desc, const DecodeGeometry& 
   return PKV_OK;
 }
 
+
+// Bytes of one pool array (which: 0 K codes, 1 V codes, 2 K scales, 3 V scales, 4 zero points).
+size_t pool_array_bytes(const pkv_cache_desc* d, int which) {
+  const size_t tiles = (size_t)d->num_blocks * d->num_kv_heads;
+  switch (which) {
+    case 0: return tiles * d->block_size * row_bytes(d->k_dtype, d->head_dim);
+    case 1: return tiles * d->block_size * row_bytes(d->v_dtype, d->head_dim);
+    case 2: return d->k_dtype != PKV_FP16 ? tiles * sizeof(float) : 0;
+    case 3: return d->v_dtype != PKV_FP16 ? tiles * sizeof(float) : 0;
+    default: return d->v_dtype == PKV_INT4_ASYM ? tiles : 0;
+  }
+}
+
+// The address through which the current device reaches [p, p + bytes), or nullptr when the range
+// is not entirely of the wanted kind: memory of the current device (host == false), or page-locked
+// host memory mapped into the device's address space (host == true). Both ends are checked.
+const void* device_view(const void* p, size_t bytes, bool host) {
+  if (p == nullptr || bytes == 0) return nullptr;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  cudaPointerAttributes a, b;
+  const char* last = static_cast<const char*>(p) + (bytes - 1);
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess || cudaPointerGetAttributes(&b, last) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  if (host) {
+    if (a.type != cudaMemoryTypeHost || b.type != cudaMemoryTypeHost) return nullptr;
+    if (a.devicePointer == nullptr || b.devicePointer == nullptr) return nullptr;
+    if (static_cast<const char*>(b.devicePointer) - static_cast<const char*>(a.devicePointer) != (ptrdiff_t)(bytes - 1))
+      return nullptr;
+    return a.devicePointer;
+  }
+  const bool ok_a = a.type == cudaMemoryTypeManaged || (a.type == cudaMemoryTypeDevice && a.device == dev);
+  const bool ok_b = b.type == cudaMemoryTypeManaged || (b.type == cudaMemoryTypeDevice && b.device == dev);
+  return ok_a && ok_b ? p : nullptr;
+}
+
+// Any memory the device can dereference (its own, or mapped host memory): the address to use.
+const void* device_view_any(const void* p, size_t bytes) {
+  const void* v = device_view(p, bytes, false);
+  return v != nullptr ? v : device_view(p, bytes, true);
+}
+
 }  // namespace
 
 extern "C" {
@@ -317,6 +361,68 @@ pkv_status pkv_decode_step(const pkv_cache_desc* desc, const int32_t* block_mapp
   }
   sp.bar = p.ws_count + (size_t)num_seqs * (num_q_heads / g.shape.heads_per_warp);
   return launch_decode_step(p, sp, g.shape, s) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+pkv_status pkv_swap_blocks(const pkv_cache_desc* device_pool, const pkv_cache_desc* host_pool,
+                           const int32_t* block_mapping, int32_t n_pairs, int32_t direction, int32_t* dev_error,
+                           pkv_stream_t stream) {
+  pkv_status st = check_desc(device_pool);
+  if (st != PKV_OK) return st;
+  st = check_desc(host_pool);
+  if (st != PKV_OK) return st;
+  const pkv_cache_desc *dv = device_pool, *hv = host_pool;
+  if (dv->block_size != hv->block_size || dv->num_kv_heads != hv->num_kv_heads || dv->head_dim != hv->head_dim ||
+      dv->k_dtype != hv->k_dtype || dv->v_dtype != hv->v_dtype)
+    return PKV_ERR_INVALID_ARG;
+  if (direction != PKV_SWAP_OUT && direction != PKV_SWAP_IN) return PKV_ERR_INVALID_ARG;
+  if (n_pairs < 0) return PKV_ERR_INVALID_ARG;
+  if (n_pairs == 0) return PKV_OK;
+  if (block_mapping == nullptr || !aligned(block_mapping, 4)) return PKV_ERR_INVALID_ARG;
+  if (dev_error != nullptr && !aligned(dev_error, 4)) return PKV_ERR_INVALID_ARG;
+  // where every array lives, as the device sees it (nothing is launched unless all check out)
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PKV_ERR_CUDA;
+  const void* arr_d[5] = {dv->k_codes, dv->v_codes, dv->k_scale, dv->v_scale, dv->v_zp};
+  const void* arr_h[5] = {hv->k_codes, hv->v_codes, hv->k_scale, hv->v_scale, hv->v_zp};
+  const void* view_d[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
+  const void* view_h[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
+  for (int i = 0; i < 5; ++i) {
+    const size_t nd = pool_array_bytes(dv, i), nh = pool_array_bytes(hv, i);
+    if (nd == 0) continue;  // the side has no such array (FP16 scales, zero points of INT8)
+    view_d[i] = device_view(arr_d[i], nd, false);
+    view_h[i] = device_view(arr_h[i], nh, true);
+    if (view_d[i] == nullptr || view_h[i] == nullptr) return PKV_ERR_INVALID_ARG;
+  }
+  const void* map_view = device_view_any(block_mapping, (size_t)n_pairs * 2 * sizeof(int32_t));
+  if (map_view == nullptr) return PKV_ERR_INVALID_ARG;
+  int32_t* err_view = nullptr;
+  if (dev_error != nullptr) {
+    err_view = static_cast<int32_t*>(const_cast<void*>(device_view_any(dev_error, sizeof(int32_t))));
+    if (err_view == nullptr) return PKV_ERR_INVALID_ARG;
+  }
+  const bool out = direction == PKV_SWAP_OUT;
+  const void* const* src = out ? view_d : view_h;
+  const void* const* dst = out ? view_h : view_d;
+  SwapParams p;
+  p.src_k = static_cast<const uint8_t*>(src[0]);
+  p.src_v = static_cast<const uint8_t*>(src[1]);
+  p.src_ks = static_cast<const float*>(src[2]);
+  p.src_vs = static_cast<const float*>(src[3]);
+  p.src_zp = static_cast<const uint8_t*>(src[4]);
+  p.dst_k = static_cast<uint8_t*>(const_cast<void*>(dst[0]));
+  p.dst_v = static_cast<uint8_t*>(const_cast<void*>(dst[1]));
+  p.dst_ks = static_cast<float*>(const_cast<void*>(dst[2]));
+  p.dst_vs = static_cast<float*>(const_cast<void*>(dst[3]));
+  p.dst_zp = static_cast<uint8_t*>(const_cast<void*>(dst[4]));
+  p.block_mapping = static_cast<const int32_t*>(map_view);
+  p.dev_error = err_view;
+  p.n_pairs = n_pairs;
+  p.src_blocks = out ? dv->num_blocks : hv->num_blocks;
+  p.dst_blocks = out ? hv->num_blocks : dv->num_blocks;
+  p.num_kv_heads = dv->num_kv_heads;
+  p.k_block_bytes = (int64_t)dv->num_kv_heads * dv->block_size * row_bytes(dv->k_dtype, dv->head_dim);
+  p.v_block_bytes = (int64_t)dv->num_kv_heads * dv->block_size * row_bytes(dv->v_dtype, dv->head_dim);
+  return launch_swap(p, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
 // ---- decode without caller-provided scratch -------------------------------------------------

@@ -104,6 +104,31 @@ struct CopyParams {
 };
 cudaError_t launch_copy(const CopyParams& p, cudaStream_t stream);
 
+// ---------------------------------------------------------------- swap
+// Whole blocks from one pool to another of the same geometry (device <-> pinned host memory);
+// every pointer is an address the device can dereference.
+struct SwapParams {
+  const uint8_t* src_k;
+  const uint8_t* src_v;
+  const float* src_ks;   // NULL when the side is FP16 (then dst_ks unused too)
+  const float* src_vs;
+  const uint8_t* src_zp; // NULL unless V is INT4
+  uint8_t* dst_k;
+  uint8_t* dst_v;
+  float* dst_ks;
+  float* dst_vs;
+  uint8_t* dst_zp;
+  const int32_t* block_mapping;  // [n_pairs][2] = {src block, dst block}
+  int32_t* dev_error;
+  int32_t n_pairs;
+  int32_t src_blocks;
+  int32_t dst_blocks;
+  int32_t num_kv_heads;
+  int64_t k_block_bytes;
+  int64_t v_block_bytes;
+};
+cudaError_t launch_swap(const SwapParams& p, cudaStream_t stream);
+
 // ---------------------------------------------------------------- fused step
 // Copy-on-write copies, then the store, then the decode, in one cooperative launch of the decode
 // kernel: every warp takes part in the copies and the stores, with a grid-wide barrier after each

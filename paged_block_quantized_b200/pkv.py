@@ -29,9 +29,11 @@ PKV_FP16, PKV_INT8_SYM, PKV_INT4_ASYM = 0, 1, 2
 EXPORTED = (
     "pkv_status_string", "pkv_tile_bytes", "pkv_store_quantized", "pkv_decode_workspace_size",
     "pkv_decode_partitioning", "pkv_paged_attention_decode_static", "pkv_static_scratch_address",
-    "pkv_paged_attention_decode", "pkv_copy_blocks", "pkv_decode_step", "pkv_blocks_for_tokens", "pkv_alloc_create",
+    "pkv_paged_attention_decode", "pkv_copy_blocks", "pkv_swap_blocks", "pkv_decode_step", "pkv_blocks_for_tokens", "pkv_alloc_create",
     "pkv_alloc_destroy", "pkv_alloc_num_free", "pkv_alloc_refcount", "pkv_alloc_blocks", "pkv_alloc_fork",
-    "pkv_alloc_release", "pkv_alloc_cow",
+    "pkv_alloc_release", "pkv_alloc_cow", "pkv_prefix_cache_create", "pkv_prefix_cache_destroy",
+    "pkv_prefix_cache_size", "pkv_prefix_cache_evictable", "pkv_prefix_match", "pkv_prefix_insert",
+    "pkv_prefix_alloc",
 )
 
 
@@ -77,6 +79,8 @@ _decode_static = _sig("pkv_paged_attention_decode_static", ctypes.c_int, _DESC, 
 PKV_STATIC_SCRATCH_BYTES = 8 << 20
 _static_addr = _sig("pkv_static_scratch_address", ctypes.c_int, ctypes.POINTER(_P), ctypes.POINTER(ctypes.c_size_t))
 _copy = _sig("pkv_copy_blocks", ctypes.c_int, _DESC, _P, _I32, _P, _P)
+_swap = _sig("pkv_swap_blocks", ctypes.c_int, _DESC, _DESC, _P, _I32, _I32, _P, _P)
+PKV_SWAP_OUT, PKV_SWAP_IN = 0, 1
 _step = _sig("pkv_decode_step", ctypes.c_int, _DESC, _P, _I32, _P, _P, _P, _I32, _P, _P, _I32, _I32, _P, _I32, _P,
              _I32, ctypes.c_float, _I32, _P, ctypes.c_size_t, _P, _P)
 _blocks_for_tokens = _sig("pkv_blocks_for_tokens", _I32, ctypes.c_int64, _I32)
@@ -88,6 +92,13 @@ _alloc_blocks = _sig("pkv_alloc_blocks", ctypes.c_int, _P, _I32, _P)
 _alloc_fork = _sig("pkv_alloc_fork", ctypes.c_int, _P, _P, _I32)
 _alloc_release = _sig("pkv_alloc_release", ctypes.c_int, _P, _P, _I32)
 _alloc_cow = _sig("pkv_alloc_cow", ctypes.c_int, _P, _I32, ctypes.POINTER(_I32))
+_pc_create = _sig("pkv_prefix_cache_create", ctypes.c_int, _P, _I32, ctypes.POINTER(_P))
+_pc_destroy = _sig("pkv_prefix_cache_destroy", None, _P)
+_pc_size = _sig("pkv_prefix_cache_size", _I32, _P)
+_pc_evictable = _sig("pkv_prefix_cache_evictable", _I32, _P)
+_pc_match = _sig("pkv_prefix_match", ctypes.c_int, _P, _P, ctypes.c_int64, _P, _I32, ctypes.POINTER(_I32))
+_pc_insert = _sig("pkv_prefix_insert", ctypes.c_int, _P, _P, ctypes.c_int64, _P, _I32)
+_pc_alloc = _sig("pkv_prefix_alloc", ctypes.c_int, _P, _I32, _P)
 
 
 class PkvError(RuntimeError):
@@ -188,6 +199,15 @@ def pkv_copy_blocks(desc, block_mapping, n_pairs, dev_error=None, stream=None, r
     return _check(st, "pkv_copy_blocks", raise_on_error)
 
 
+def pkv_swap_blocks(device_desc, host_desc, block_mapping, n_pairs, direction, dev_error=None, stream=None,
+                    raise_on_error=True):
+    """Whole blocks device pool -> host pool (PKV_SWAP_OUT) or back (PKV_SWAP_IN); the host pool's
+    arrays must be pinned host memory (e.g. torch tensors from pin_memory())."""
+    st = _swap(ctypes.byref(device_desc), ctypes.byref(host_desc), _ptr(block_mapping), int(n_pairs), int(direction),
+               _ptr(dev_error), _stream(stream))
+    return _check(st, "pkv_swap_blocks", raise_on_error)
+
+
 def pkv_decode_step(desc, block_mapping, n_pairs, k_new, v_new, slot_mapping, T, out, q, num_seqs, num_q_heads,
                     block_tables, max_blocks_per_seq, context_lens, max_context_len, softmax_scale,
                     partition_tokens=0, workspace=None, workspace_bytes=0, dev_error=None, stream=None,
@@ -254,6 +274,60 @@ class Allocator:
         return int(new.value)
 
 
+class PrefixCache:
+    """Owning wrapper of a pkv_prefix_cache handle over an Allocator (which must outlive it)."""
+
+    def __init__(self, allocator: Allocator, block_size: int):
+        h = _P()
+        _check(_pc_create(allocator._h, int(block_size), ctypes.byref(h)), "pkv_prefix_cache_create", True)
+        self._h = h
+        self.allocator = allocator
+        self.block_size = int(block_size)
+
+    def close(self):
+        if self._h:
+            _pc_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        self.close()
+
+    @property
+    def size(self) -> int:
+        return int(_pc_size(self._h))
+
+    @property
+    def evictable(self) -> int:
+        return int(_pc_evictable(self._h))
+
+    @staticmethod
+    def _tokens(tokens):
+        arr = (ctypes.c_int32 * max(len(tokens), 1))(*[int(t) for t in tokens])
+        return arr, len(tokens)
+
+    def match(self, tokens, max_blocks=None):
+        """Physical ids of the longest cached whole-block prefix (each gains a caller reference)."""
+        arr, n = self._tokens(tokens)
+        mb = n // self.block_size if max_blocks is None else int(max_blocks)
+        out = (ctypes.c_int32 * max(mb, 1))()
+        got = _I32(0)
+        _check(_pc_match(self._h, arr, n, out, mb, ctypes.byref(got)), "pkv_prefix_match", True)
+        return [int(out[i]) for i in range(got.value)]
+
+    def insert(self, tokens, block_ids, raise_on_error=True):
+        arr, n = self._tokens(tokens)
+        ids = (ctypes.c_int32 * max(len(block_ids), 1))(*[int(b) for b in block_ids])
+        return _check(_pc_insert(self._h, arr, n, ids, len(block_ids)), "pkv_prefix_insert", raise_on_error)
+
+    def alloc(self, n: int, raise_on_error=True):
+        ids = (ctypes.c_int32 * max(n, 1))()
+        st = _pc_alloc(self._h, int(n), ids)
+        if st != PKV_OK:
+            _check(st, "pkv_prefix_alloc", raise_on_error)
+            return None
+        return [int(ids[i]) for i in range(n)]
+
+
 # ---- device pool (torch tensors used as plain device memory) ----
 
 @dataclass
@@ -269,18 +343,24 @@ class DevicePool:
 
     @classmethod
     def allocate(cls, num_blocks, block_size, num_kv_heads, head_dim, k_dtype, v_dtype, device="cuda",
-                 fill: int | None = None):
+                 fill: int | None = None, pinned_host: bool = False):
+        """Device pool, or with pinned_host=True a pool in page-locked host memory (a swap target)."""
         import torch
+
+        def empty(shape, dtype):
+            if pinned_host:
+                return torch.empty(shape, dtype=dtype, device="cpu", pin_memory=True)
+            return torch.empty(shape, dtype=dtype, device=device)
 
         def codes(dt):
             row = {PKV_FP16: 2 * head_dim, PKV_INT8_SYM: head_dim, PKV_INT4_ASYM: head_dim // 2}[dt]
-            return torch.empty((num_blocks, num_kv_heads, block_size, row), dtype=torch.uint8, device=device)
+            return empty((num_blocks, num_kv_heads, block_size, row), torch.uint8)
 
         k = codes(k_dtype)
         v = codes(v_dtype)
-        ks = torch.empty((num_blocks, num_kv_heads), dtype=torch.float32, device=device)
-        vs = torch.empty((num_blocks, num_kv_heads), dtype=torch.float32, device=device)
-        zp = torch.empty((num_blocks, num_kv_heads), dtype=torch.uint8, device=device)
+        ks = empty((num_blocks, num_kv_heads), torch.float32)
+        vs = empty((num_blocks, num_kv_heads), torch.float32)
+        zp = empty((num_blocks, num_kv_heads), torch.uint8)
         if fill is not None:
             for t in (k, v, zp):
                 t.fill_(fill)

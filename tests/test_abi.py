@@ -168,3 +168,25 @@ def test_workspace_size(pkv):
     assert pkv.pkv_decode_workspace_size(d, 0, 4, 64, 0) == 0
     # independent of the context length once the device is full (no copy of the cache)
     assert pkv.pkv_decode_workspace_size(d, 64, 4, 8192, 0) == pkv.pkv_decode_workspace_size(d, 64, 4, 32768, 0)
+
+
+def test_swap_validation(pkv):
+    """pkv_swap_blocks refuses mismatched pools, a bad direction and bad counts on the host before
+    it looks at where the memory lives (fake pointers, no device needed)."""
+    d = desc(pkv)
+    E = pkv.PKV_ERR_INVALID_ARG
+    swap = lambda h, n=1, direction=pkv.PKV_SWAP_OUT, mapping=0x6000: pkv.pkv_swap_blocks(
+        d, h, mapping, n, direction, stream=0, raise_on_error=False)
+    # a smaller host pool is fine; the fake pointers are then refused by the memory-kind check (or,
+    # without a device, the device query fails): never a launch
+    assert swap(desc(pkv, num_blocks=4)) in (E, pkv.PKV_ERR_CUDA)
+    assert swap(desc(pkv, head_dim=128)) == E            # geometry must match
+    assert swap(desc(pkv, num_kv_heads=4)) == E
+    assert swap(desc(pkv, block_size=32)) == E
+    assert swap(desc(pkv, v_dtype=pkv.PKV_INT8_SYM, v_zp=0)) == E
+    assert swap(desc(pkv), direction=2) == E
+    assert swap(desc(pkv), n=-1) == E
+    assert swap(desc(pkv), mapping=None) == E
+    assert swap(desc(pkv), mapping=0x6002) == E
+    assert swap(desc(pkv), n=0) == pkv.PKV_OK
+    assert swap(desc(pkv, k_codes=0x1008)) == E          # a misaligned host array

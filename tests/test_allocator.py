@@ -77,3 +77,30 @@ def test_copy_on_write(pkv):
     a.fork([b])
     assert a.cow(b, raise_on_error=False) is None  # no free block for the copy
     assert a.refcount(b) == 2
+
+
+def test_swap_bookkeeping(pkv):
+    """A sequence swapped out and back in ([deepinsea] "Swap 机制") with one allocator per pool:
+    host blocks are taken before the swap-out and the device blocks released after it; device
+    blocks are taken before the swap-in and the host blocks released after it. A block shared with
+    another sequence stays on the device until its last reference goes."""
+    dev, host = pkv.Allocator(16), pkv.Allocator(8)
+    seq_a = dev.alloc(5)
+    seq_b = dev.alloc(3)
+    dev.fork(seq_a[:2])                       # seq_b's beam shares seq_a's first two blocks
+    # swap seq_a out: one host block per device block
+    h = host.alloc(len(seq_a))
+    mapping_out = list(zip(seq_a, h))
+    assert len(mapping_out) == 5 and host.num_free == 3
+    dev.release(seq_a)
+    assert [dev.refcount(b) for b in seq_a] == [1, 1, 0, 0, 0]  # the shared two stay for the beam
+    assert dev.num_free == 16 - 3 - 2
+    # not enough host room for a second sequence of 5: all or nothing
+    assert host.alloc(5, raise_on_error=False) is None and host.num_free == 3
+    # swap seq_a back in under fresh device ids
+    d = dev.alloc(len(h))
+    mapping_in = list(zip(h, d))
+    assert len(set(d) & set(seq_b)) == 0 and all(dev.refcount(b) == 1 for b in d)
+    host.release(h)
+    assert host.num_free == 8
+    assert [src for src, _ in mapping_in] == [dst for _, dst in mapping_out]
