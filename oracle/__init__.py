@@ -12,6 +12,9 @@ Parity status of each function (what pins it; see ``tests/test_oracle_*.py``):
          special cases). Append into a partly filled block (fit-or-rebuild rule): the pages only
          quantize whole blocks, so the rule itself is **parity unpinned**; only invariants
          (range, error bound, fit == single shot) are checked.
+  FP8 E4M3 store (scale = absmax / 448, nearest-even saturating codes): pinned (the format's
+         hand-decoded values, ties and saturation, every code round-trips, error bound); its
+         append rule is parity unpinned like the INT8 one.
   copy   pinned (byte identity, untouched blocks).
   decode pinned (library attention on contiguous data, permutation / prefix-sharing
          invariance, closed-form special cases, brute-force agreement).
@@ -26,7 +29,7 @@ import numpy as np
 
 from . import build as _build
 
-FP16, INT8_SYM, INT4_ASYM = 0, 1, 2
+FP16, INT8_SYM, INT4_ASYM, FP8_E4M3 = 0, 1, 2, 3
 
 DEVERR_BLOCK_ID, DEVERR_SLOT, DEVERR_SLOT_GROUP, DEVERR_CONTEXT_LEN = 1, 2, 3, 4
 
@@ -64,6 +67,10 @@ def _load():
         lib.oracle_decode.argtypes = [P, P, ctypes.c_int32, ctypes.c_int32, P, ctypes.c_int32, P,
                                       ctypes.c_int32, ctypes.c_float, P, ctypes.c_int32]
         lib.oracle_decode.restype = ctypes.c_int32
+        lib.oracle_fp8_e4m3_decode.argtypes = [ctypes.c_uint8]
+        lib.oracle_fp8_e4m3_decode.restype = ctypes.c_double
+        lib.oracle_fp8_e4m3_encode.argtypes = [ctypes.c_float]
+        lib.oracle_fp8_e4m3_encode.restype = ctypes.c_uint8
         _lib = lib
     return _lib
 
@@ -73,6 +80,8 @@ def _row_shape(dtype: int, head_dim: int):
         return head_dim, np.uint16  # fp16 bit patterns
     if dtype == INT8_SYM:
         return head_dim, np.int8
+    if dtype == FP8_E4M3:
+        return head_dim, np.uint8  # E4M3 bytes
     if dtype == INT4_ASYM:
         return head_dim // 2, np.uint8
     raise ValueError(f"unknown dtype {dtype}")
@@ -130,6 +139,16 @@ def _fp16_bits(x: np.ndarray) -> np.ndarray:
     if x.dtype == np.uint16:
         return x
     raise TypeError("expected float16 data")
+
+
+def fp8_e4m3_decode(code: int) -> float:
+    """The E4M3 value of a code byte (binary64, exact)."""
+    return float(_load().oracle_fp8_e4m3_decode(int(code) & 0xFF))
+
+
+def fp8_e4m3_encode(x: float) -> int:
+    """The E4M3 code of a binary32 value: nearest, ties to even, saturating at +-448."""
+    return int(_load().oracle_fp8_e4m3_encode(float(np.float32(x))))
 
 
 def store(cache: OracleCache, k_new: np.ndarray, v_new: np.ndarray, slot_mapping: np.ndarray) -> int:

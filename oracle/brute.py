@@ -11,7 +11,17 @@ from __future__ import annotations
 
 import numpy as np
 
-FP16, INT8_SYM, INT4_ASYM = 0, 1, 2
+FP16, INT8_SYM, INT4_ASYM, FP8_E4M3 = 0, 1, 2, 3
+
+
+def _e4m3_values(codes: np.ndarray) -> np.ndarray:
+    """E4M3 code bytes -> float64 values: sign, 4 exponent bits (bias 7), 3 mantissa bits;
+    exponent field 0 = subnormal m * 2^-9 (the all-ones NaN codes never occur in a tile)."""
+    c = codes.astype(np.int64)
+    e = (c >> 3) & 0xF
+    m = (c & 7).astype(np.float64)
+    mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    return np.where(c & 0x80, -mag, mag)
 
 
 def _unpack_nibbles(packed: np.ndarray) -> np.ndarray:
@@ -30,6 +40,8 @@ def dequant_tile(codes: np.ndarray, dtype: int, scale=None, zp=None) -> np.ndarr
         return codes.view(np.float16).astype(np.float64)
     if dtype == INT8_SYM:
         return codes.astype(np.float64) * np.float64(scale)
+    if dtype == FP8_E4M3:
+        return _e4m3_values(codes) * np.float64(scale)
     return (_unpack_nibbles(codes).astype(np.float64) - np.float64(zp)) * np.float64(scale)
 
 

@@ -32,6 +32,12 @@
  *   R8 INT4 nibbles packed along head_dim, low nibble = even dimension
  *   R10 context_lens include the token just stored
  *   R11 context_len 0 gives a zero output; a negative slot skips the token
+ *   R15 FP8 E4M3 ([yunthe] "vLLM推理引擎部署与KV Cache量化配置实战": the fp8 cache mode uses E4M3):
+ *      one binary32 scale per (block, KV head), scale = absmax / 448 (the largest finite E4M3
+ *      magnitude), code = E4M3(x / scale) rounded to nearest, ties to even, saturating; scale 0
+ *      gives codes 0; x_hat = value(code) * scale. Appending: new values fit when every
+ *      |x / scale_old| <= 448, else the tile is rebuilt as for INT8 (old values dequantized in
+ *      binary32, scale from old and new together)
  */
 #include "oracle.h"
 
@@ -214,15 +220,91 @@ static void store_tile_asym4(uint8_t* tile, float* scale, uint8_t* zp_ptr, int d
   free(xh);
 }
 
+/* ---- FP8 E4M3 (R15). The format: 1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits; the
+ * exponent field 0 holds subnormals m * 2^-9, fields 1..15 hold (1 + m/8) * 2^(e-7), except that
+ * the all-ones pattern S.1111.111 is NaN; there are no infinities, so the largest finite
+ * magnitude is 1.75 * 2^8 = 448. ---- */
+double oracle_fp8_e4m3_decode(uint8_t code) {
+  int sign = code >> 7, e = (code >> 3) & 0xF, m = code & 7;
+  double v;
+  if (e == 15 && m == 7) return NAN;
+  if (e == 0) v = ldexp((double)m, -9);
+  else v = ldexp((double)(8 + m), e - 10); /* (1 + m/8) * 2^(e-7) */
+  return sign ? -v : v;
+}
+
+/* Nearest representable magnitude by comparing with every finite one (codes 0..126 ascend in
+ * value); of two equally near, the one with an even mantissa (its lowest bit 0). Magnitudes past
+ * 448 go to 448 (saturation). The sign is the sign bit of x. */
+uint8_t oracle_fp8_e4m3_encode(float x) {
+  uint8_t sign = signbit(x) ? 0x80 : 0x00;
+  double a = fabs((double)x);
+  int best = 0;
+  double best_d = a;
+  for (int c = 1; c <= 126; ++c) {
+    double d = fabs(oracle_fp8_e4m3_decode((uint8_t)c) - a);
+    if (d < best_d || (d == best_d && (c & 1) == 0)) {
+      best = c;
+      best_d = d;
+    }
+  }
+  return (uint8_t)(sign | best);
+}
+
+static uint8_t quant_fp8(float x, float s) {
+  if (s == 0.0f) return 0; /* R7 */
+  return oracle_fp8_e4m3_encode(x / s);
+}
+
+/* One (block, head) tile of E4M3 codes: [bs][d] bytes; new_x: [n][d] values for offsets o0.. */
+static void store_tile_fp8(uint8_t* tile, float* scale, int d, int o0, int n, const float* new_x) {
+  float m_new = 0.0f;
+  for (int i = 0; i < n * d; ++i) {
+    float a = fabsf(new_x[i]);
+    if (a > m_new) m_new = a;
+  }
+  if (o0 == 0) {
+    float s = m_new / 448.0f;
+    for (int i = 0; i < n * d; ++i) tile[i] = quant_fp8(new_x[i], s);
+    *scale = s;
+    return;
+  }
+  float s_old = *scale;
+  int fits = 1;
+  for (int i = 0; i < n * d && fits; ++i) {
+    if (s_old == 0.0f) fits = (new_x[i] == 0.0f);
+    else fits = (fabsf(new_x[i] / s_old) <= 448.0f);
+  }
+  uint8_t* new_tile = tile + (size_t)o0 * d;
+  if (fits) {
+    for (int i = 0; i < n * d; ++i) new_tile[i] = quant_fp8(new_x[i], s_old);
+    return;
+  }
+  int n_old = o0 * d;
+  float* xh = (float*)malloc(sizeof(float) * (size_t)(n_old > 0 ? n_old : 1));
+  float m_old = 0.0f;
+  for (int i = 0; i < n_old; ++i) {
+    xh[i] = (float)oracle_fp8_e4m3_decode(tile[i]) * s_old; /* exact value, one binary32 product */
+    float a = fabsf(xh[i]);
+    if (a > m_old) m_old = a;
+  }
+  float s = (m_old > m_new ? m_old : m_new) / 448.0f;
+  for (int i = 0; i < n_old; ++i) tile[i] = quant_fp8(xh[i], s);
+  for (int i = 0; i < n * d; ++i) new_tile[i] = quant_fp8(new_x[i], s);
+  *scale = s;
+  free(xh);
+}
+
 static size_t code_row_bytes(int dtype, int d) {
   if (dtype == ORACLE_FP16) return (size_t)d * 2;
-  if (dtype == ORACLE_INT8_SYM) return (size_t)d;
+  if (dtype == ORACLE_INT8_SYM || dtype == ORACLE_FP8_E4M3) return (size_t)d;
   return (size_t)d / 2;
 }
 
 static int dtypes_ok(const oracle_cache* c) {
-  if (c->k_dtype != ORACLE_FP16 && c->k_dtype != ORACLE_INT8_SYM) return 0;
-  if (c->v_dtype != ORACLE_FP16 && c->v_dtype != ORACLE_INT8_SYM && c->v_dtype != ORACLE_INT4_ASYM)
+  if (c->k_dtype != ORACLE_FP16 && c->k_dtype != ORACLE_INT8_SYM && c->k_dtype != ORACLE_FP8_E4M3) return 0;
+  if (c->v_dtype != ORACLE_FP16 && c->v_dtype != ORACLE_INT8_SYM && c->v_dtype != ORACLE_INT4_ASYM &&
+      c->v_dtype != ORACLE_FP8_E4M3)
     return 0;
   return 1;
 }
@@ -242,6 +324,9 @@ static void store_side(const oracle_cache* c, int which_v, int block, int head, 
   } else if (dtype == ORACLE_INT8_SYM) {
     float* scale = which_v ? &c->v_scale[meta] : &c->k_scale[meta];
     store_tile_sym((int8_t*)tile, scale, c->head_dim, o0, n, vals);
+  } else if (dtype == ORACLE_FP8_E4M3) {
+    float* scale = which_v ? &c->v_scale[meta] : &c->k_scale[meta];
+    store_tile_fp8(tile, scale, c->head_dim, o0, n, vals);
   } else {
     store_tile_asym4(tile, &c->v_scale[meta], &c->v_zp[meta], c->head_dim, o0, n, vals);
   }
@@ -343,6 +428,10 @@ static double dequant(const oracle_cache* c, int which_v, int block, int head, i
   if (dtype == ORACLE_INT8_SYM) {
     double s = which_v ? (double)c->v_scale[meta] : (double)c->k_scale[meta];
     return (double)((const int8_t*)r)[j] * s;
+  }
+  if (dtype == ORACLE_FP8_E4M3) { /* x_hat = value(code) * scale (R15) */
+    double s = which_v ? (double)c->v_scale[meta] : (double)c->k_scale[meta];
+    return oracle_fp8_e4m3_decode(r[j]) * s;
   }
   return ((double)get_nibble(r, j) - (double)c->v_zp[meta]) * (double)c->v_scale[meta];
 }

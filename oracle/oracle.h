@@ -11,7 +11,7 @@
 extern "C" {
 #endif
 
-enum { ORACLE_FP16 = 0, ORACLE_INT8_SYM = 1, ORACLE_INT4_ASYM = 2 };
+enum { ORACLE_FP16 = 0, ORACLE_INT8_SYM = 1, ORACLE_INT4_ASYM = 2, ORACLE_FP8_E4M3 = 3 };
 
 /* error codes reported by the oracle for malformed inputs (first one wins) */
 enum {
@@ -23,7 +23,8 @@ enum {
 
 /* One layer's pool in host memory, same row-major layout as the device pool:
  *   codes [num_blocks][num_kv_heads][block_size][row] with row = head_dim int8 (INT8),
- *         head_dim fp16 bit patterns (FP16) or head_dim/2 packed nibbles (INT4);
+ *         head_dim fp16 bit patterns (FP16), head_dim/2 packed nibbles (INT4) or head_dim
+ *         E4M3 bytes (FP8);
  *   scales / zero points [num_blocks][num_kv_heads]. */
 typedef struct oracle_cache {
   int32_t num_blocks, block_size, num_kv_heads, head_dim;
@@ -42,6 +43,11 @@ int32_t oracle_store(const oracle_cache* c, const uint16_t* k_new, const uint16_
 
 /* Copy whole blocks: pairs {src, dst}. */
 int32_t oracle_copy_blocks(const oracle_cache* c, const int32_t* block_mapping, int32_t n_pairs);
+
+/* The E4M3 value of a code (binary64, exact; NaN for the NaN codes), and the code of a binary32
+ * value (round to nearest, ties to even, saturating at +-448), from the format's definition. */
+double oracle_fp8_e4m3_decode(uint8_t code);
+uint8_t oracle_fp8_e4m3_encode(float x);
 
 /* Decode attention in binary64. q: fp16 bit patterns [S][Hq][D]; out: double [S][Hq][D]. */
 int32_t oracle_decode(const oracle_cache* c, const uint16_t* q, int32_t num_seqs, int32_t num_q_heads,

@@ -14,7 +14,8 @@ import torch
 import oracle
 from oracle import brute
 
-DTYPES = [(oracle.INT8_SYM, oracle.INT8_SYM), (oracle.INT8_SYM, oracle.INT4_ASYM), (oracle.FP16, oracle.FP16)]
+DTYPES = [(oracle.INT8_SYM, oracle.INT8_SYM), (oracle.INT8_SYM, oracle.INT4_ASYM), (oracle.FP16, oracle.FP16),
+          (oracle.FP8_E4M3, oracle.FP8_E4M3)]
 
 
 def unpack(packed):
@@ -48,6 +49,10 @@ def page_dequant(c, which, b, h):
     if dt == oracle.INT8_SYM:
         s = c.k_scale[b, h] if which == "k" else c.v_scale[b, h]
         return codes.astype(np.float64) * float(s)
+    if dt == oracle.FP8_E4M3:  # E4M3 values through torch's own float8 type, times the scale
+        s = c.k_scale[b, h] if which == "k" else c.v_scale[b, h]
+        vals = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+        return vals * float(s)
     return (unpack(codes) - float(c.v_zp[b, h])) * float(c.v_scale[b, h])
 
 
@@ -172,10 +177,10 @@ def test_empty_and_error_reporting():
     np.testing.assert_array_equal(out_bad[1], out_16[1])
 
 
-@pytest.mark.parametrize("seed", range(6))
+@pytest.mark.parametrize("seed", range(8))
 def test_brute_force_agreement(seed):
     rng = np.random.default_rng(100 + seed)
-    kd, vd = DTYPES[seed % 3]
+    kd, vd = DTYPES[seed % len(DTYPES)]
     bs = [16, 32][seed % 2]
     H = int(rng.integers(1, 3))
     G = int(rng.choice([1, 2, 4]))
@@ -214,3 +219,4 @@ def test_quantized_attention_tracks_fp16_attention():
     ref = outs[(oracle.FP16, oracle.FP16)]
     assert np.abs(outs[(oracle.INT8_SYM, oracle.INT8_SYM)] - ref).max() < 0.03
     assert np.abs(outs[(oracle.INT8_SYM, oracle.INT4_ASYM)] - ref).max() < 0.2
+    assert np.abs(outs[(oracle.FP8_E4M3, oracle.FP8_E4M3)] - ref).max() < 0.1

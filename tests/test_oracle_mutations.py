@@ -18,7 +18,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
 from oracle import build as oracle_build  # noqa: E402
 
-PIN_TESTS = ["tests/test_oracle_store.py", "tests/test_oracle_decode.py", "tests/test_oracle_copy.py"]
+PIN_TESTS = ["tests/test_oracle_store.py", "tests/test_oracle_decode.py", "tests/test_oracle_copy.py",
+             "tests/test_oracle_fp8.py"]
 EXPECTED_SURVIVORS = {"clamp128"}
 
 MUTANTS = {
@@ -37,6 +38,14 @@ MUTANTS = {
     "clamp128": ("if (r < -127.0f) r = -127.0f; /* R4 */", "if (r < -128.0f) r = -128.0f;"),
     "vscale_kscale": ("double s = which_v ? (double)c->v_scale[meta] : (double)c->k_scale[meta];", "double s = (double)c->k_scale[meta];"),
     "asym_plus_zp_missing": ("float r = rintf(x / s + (float)zp);", "float r = rintf(x / s);"),
+    "fp8_ties_odd": ("if (d < best_d || (d == best_d && (c & 1) == 0)) {", "if (d < best_d || (d == best_d && (c & 1) == 1)) {"),
+    "fp8_ties_up": ("if (d < best_d || (d == best_d && (c & 1) == 0)) {", "if (d <= best_d) {"),
+    "fp8_exp_bias": ("else v = ldexp((double)(8 + m), e - 10); /* (1 + m/8) * 2^(e-7) */", "else v = ldexp((double)(8 + m), e - 9);"),
+    "fp8_subnormal": ("if (e == 0) v = ldexp((double)m, -9);", "if (e == 0) v = ldexp((double)m, -10);"),
+    "fp8_scale480": ("float s = m_new / 448.0f;", "float s = m_new / 480.0f;"),
+    "fp8_fit_480": ("else fits = (fabsf(new_x[i] / s_old) <= 448.0f);", "else fits = (fabsf(new_x[i] / s_old) <= 480.0f);"),
+    "fp8_no_requant_old": ("for (int i = 0; i < n_old; ++i) tile[i] = quant_fp8(xh[i], s);", ""),
+    "fp8_sign": ("uint8_t sign = signbit(x) ? 0x80 : 0x00;", "uint8_t sign = 0x00;"),
     "copy_scales_missing": ("memcpy(c->k_scale + (size_t)dst * H, c->k_scale + (size_t)src * H, sizeof(float) * H);", ";"),
 }
 
