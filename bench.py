@@ -211,8 +211,8 @@ def decode_source_hash() -> str:
     """Hash of the decode kernel's device sources with comments and blank lines removed (a profile
     stays valid across comment edits and host-side changes, not across kernel code changes)."""
     h = hashlib.sha256()
-    for name in ("decode_kernel.cuh", "decode_i8i8.cu", "decode_i8i4.cu", "decode_f16.cu", "common.cuh",
-                 "store_impl.cuh", "copy_impl.cuh"):
+    for name in ("decode_kernel.cuh", "decode_i8i8.cu", "decode_i8i4.cu", "decode_f16.cu", "decode_fp8.cu",
+                 "common.cuh", "store_impl.cuh", "copy_impl.cuh"):
         with open(os.path.join(ROOT, "paged_block_quantized_b200", "csrc", name), encoding="utf-8") as f:
             for line in f:
                 code = line.split("//", 1)[0].rstrip()

@@ -24,7 +24,8 @@
  * Device memory layout (all row-major, all owned by the caller):
  *   k_codes  [num_blocks][num_kv_heads][block_size][head_dim]   int8   (PKV_INT8_SYM)
  *                                                              fp16   (PKV_FP16)
- *   v_codes  [num_blocks][num_kv_heads][block_size][head_dim]   int8 / fp16
+ *                                                              E4M3   (PKV_FP8_E4M3)
+ *   v_codes  [num_blocks][num_kv_heads][block_size][head_dim]   int8 / fp16 / E4M3
  *            [num_blocks][num_kv_heads][block_size][head_dim/2] uint8  (PKV_INT4_ASYM):
  *            byte j of a token row = code[2j] | code[2j+1] << 4 (low nibble = even dim)
  *   k_scale, v_scale [num_blocks][num_kv_heads] fp32   (NULL for an FP16 cache side)
@@ -82,7 +83,11 @@ typedef enum pkv_status {
 typedef enum pkv_dtype {
   PKV_FP16 = 0,      /* unquantized half precision */
   PKV_INT8_SYM = 1,  /* int8 codes in [-127, 127], x_hat = code * scale */
-  PKV_INT4_ASYM = 2  /* uint4 codes in [0, 15], x_hat = (code - zp) * scale (V only) */
+  PKV_INT4_ASYM = 2, /* uint4 codes in [0, 15], x_hat = (code - zp) * scale (V only) */
+  PKV_FP8_E4M3 = 3   /* E4M3 bytes (sign, 4 exponent bits with bias 7, 3 mantissa bits, largest
+                        finite 448), x_hat = value(code) * scale, scale = absmax / 448; K and V
+                        both FP8 or neither ([yunthe] "vLLM推理引擎部署与KV Cache量化配置实战":
+                        --kv-cache-dtype fp8 uses the E4M3 format) */
 } pkv_dtype;
 
 /* Device-side error codes written to *dev_error (first one wins). */
@@ -101,8 +106,8 @@ typedef struct pkv_cache_desc {
   int32_t block_size;    /* bs: tokens per block, 16 or 32 */
   int32_t num_kv_heads;  /* Hkv */
   int32_t head_dim;      /* D: 64, 128 or 256 */
-  int32_t k_dtype;       /* pkv_dtype: PKV_INT8_SYM or PKV_FP16 */
-  int32_t v_dtype;       /* pkv_dtype: PKV_INT8_SYM, PKV_INT4_ASYM or PKV_FP16 */
+  int32_t k_dtype;       /* pkv_dtype: PKV_INT8_SYM, PKV_FP16 or PKV_FP8_E4M3 */
+  int32_t v_dtype;       /* pkv_dtype: PKV_INT8_SYM, PKV_INT4_ASYM, PKV_FP16 or PKV_FP8_E4M3 */
   void* k_codes;
   void* v_codes;
   float* k_scale;        /* required when k_dtype != PKV_FP16 */
@@ -124,6 +129,8 @@ PKV_API size_t pkv_tile_bytes(const pkv_cache_desc* desc, int32_t which_v);
  * one scale (and zero point) per (block, KV head); round half to even; codes clamped to
  * [-127, 127] (INT8) or [0, 15] (INT4); INT4 range [min(0, min x), max(0, max x)],
  * scale = (hi - lo)/15, zp = clamp(rint(-lo/scale), 0, 15); scale 0 encodes an all-zero tile.
+ * FP8 E4M3: scale = absmax/448, code = E4M3(x/scale) rounded to nearest even and saturated; new
+ * values fit a stored scale when every |x/scale| <= 448.
  * All code arithmetic is IEEE binary32, round to nearest even, one rounding per operation.
  *
  * Tokens of one call that land in the same block must be adjacent in slot_mapping with

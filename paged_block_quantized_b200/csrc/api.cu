@@ -16,13 +16,13 @@ using namespace pkv;
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-bool dtype_known_k(int32_t d) { return d == PKV_FP16 || d == PKV_INT8_SYM; }
-bool dtype_known_v(int32_t d) { return d == PKV_FP16 || d == PKV_INT8_SYM || d == PKV_INT4_ASYM; }
+bool dtype_known_k(int32_t d) { return d == PKV_FP16 || d == PKV_INT8_SYM || d == PKV_FP8_E4M3; }
+bool dtype_known_v(int32_t d) { return d == PKV_FP16 || d == PKV_INT8_SYM || d == PKV_INT4_ASYM || d == PKV_FP8_E4M3; }
 
 int64_t row_bytes(int32_t dtype, int32_t head_dim) {
   if (dtype == PKV_FP16) return 2 * (int64_t)head_dim;
-  if (dtype == PKV_INT8_SYM) return head_dim;
-  return head_dim / 2;
+  if (dtype == PKV_INT4_ASYM) return head_dim / 2;
+  return head_dim;  // INT8, E4M3
 }
 
 // Checks shared by every call that reads or writes the pool.
@@ -33,6 +33,7 @@ pkv_status check_desc(const pkv_cache_desc* d) {
   if (d->head_dim % 16 != 0) return PKV_ERR_INVALID_ARG;
   if (!dtype_known_k(d->k_dtype) || !dtype_known_v(d->v_dtype)) return PKV_ERR_INVALID_ARG;
   if (d->block_size != 16 && d->block_size != 32) return PKV_ERR_UNSUPPORTED;
+  if ((d->k_dtype == PKV_FP8_E4M3) != (d->v_dtype == PKV_FP8_E4M3)) return PKV_ERR_UNSUPPORTED;  // both or neither
   if (d->head_dim != 64 && d->head_dim != 128 && d->head_dim != 256) return PKV_ERR_UNSUPPORTED;
   if (d->k_codes == nullptr || d->v_codes == nullptr) return PKV_ERR_INVALID_ARG;
   if (!aligned(d->k_codes, 16) || !aligned(d->v_codes, 16)) return PKV_ERR_INVALID_ARG;

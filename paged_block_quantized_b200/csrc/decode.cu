@@ -1,6 +1,6 @@
 // decode.cu -- the decode entry points behind the C ABI: heads per warp, supported shapes, and the
 // dispatch to the kernel instantiations of each dtype pair (decode_i8i8.cu, decode_i8i4.cu,
-// decode_f16.cu; the kernel itself is in decode_kernel.cuh).
+// decode_f16.cu, decode_fp8.cu; the kernel itself is in decode_kernel.cuh).
 #include <cudaTypedefs.h>
 
 #include "internal.h"
@@ -47,7 +47,7 @@ bool encode_tile_map(CUtensorMap* map, const void* base, uint64_t rows, int row_
 
 int32_t decode_heads_per_warp(int32_t group, int32_t k_dtype, int32_t v_dtype, int32_t head_dim) {
   const bool mma = (k_dtype == PKV_INT8_SYM && v_dtype == PKV_INT8_SYM && head_dim >= 128) ||
-                   (k_dtype == PKV_FP16 && v_dtype == PKV_FP16);
+                   (k_dtype == PKV_FP16 && v_dtype == PKV_FP16) || (k_dtype == PKV_FP8_E4M3 && v_dtype == PKV_FP8_E4M3);
   if (mma && group % 8 == 0) return 8;
   if (group % 4 == 0) return 4;
   if (group % 2 == 0) return 2;
@@ -56,7 +56,8 @@ int32_t decode_heads_per_warp(int32_t group, int32_t k_dtype, int32_t v_dtype, i
 
 bool decode_supported(int32_t k_dtype, int32_t v_dtype, int32_t block_size, int32_t head_dim) {
   const bool dt = (k_dtype == PKV_INT8_SYM && (v_dtype == PKV_INT8_SYM || v_dtype == PKV_INT4_ASYM)) ||
-                  (k_dtype == PKV_FP16 && v_dtype == PKV_FP16);
+                  (k_dtype == PKV_FP16 && v_dtype == PKV_FP16) ||
+                  (k_dtype == PKV_FP8_E4M3 && v_dtype == PKV_FP8_E4M3 && head_dim >= 128);
   return dt && (block_size == 16 || block_size == 32) && (head_dim == 64 || head_dim == 128 || head_dim == 256);
 }
 
@@ -64,6 +65,7 @@ bool decode_kernel_info(const DecodeShape& sh, DecodeKernelInfo* info) {
   if (sh.k_dtype == PKV_INT8_SYM && sh.v_dtype == PKV_INT8_SYM) return decode_info_i8i8(sh, info);
   if (sh.k_dtype == PKV_INT8_SYM && sh.v_dtype == PKV_INT4_ASYM) return decode_info_i8i4(sh, info);
   if (sh.k_dtype == PKV_FP16 && sh.v_dtype == PKV_FP16) return decode_info_f16(sh, info);
+  if (sh.k_dtype == PKV_FP8_E4M3 && sh.v_dtype == PKV_FP8_E4M3) return decode_info_fp8(sh, info);
   return false;
 }
 
@@ -72,6 +74,7 @@ cudaError_t launch_any(const DecodeParams& p, const StepParams& sp, const Decode
   if (sh.k_dtype == PKV_INT8_SYM && sh.v_dtype == PKV_INT8_SYM) return launch_decode_i8i8(p, sp, sh, stream);
   if (sh.k_dtype == PKV_INT8_SYM && sh.v_dtype == PKV_INT4_ASYM) return launch_decode_i8i4(p, sp, sh, stream);
   if (sh.k_dtype == PKV_FP16 && sh.v_dtype == PKV_FP16) return launch_decode_f16(p, sp, sh, stream);
+  if (sh.k_dtype == PKV_FP8_E4M3 && sh.v_dtype == PKV_FP8_E4M3) return launch_decode_fp8(p, sp, sh, stream);
   return cudaErrorInvalidValue;
 }
 }  // namespace

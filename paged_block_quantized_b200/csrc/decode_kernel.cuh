@@ -72,13 +72,16 @@ constexpr float kNegBig = -1.0e30f;  // finite "minus infinity" for running maxi
 template <int KT, int VT, int BS, int D, int GT>
 struct Cfg {
   static constexpr int K_ROW = (KT == PKV_FP16) ? 2 * D : D;
-  static constexpr int V_ROW = (VT == PKV_FP16) ? 2 * D : (VT == PKV_INT8_SYM ? D : D / 2);
+  static constexpr int V_ROW = (VT == PKV_FP16) ? 2 * D : (VT == PKV_INT4_ASYM ? D / 2 : D);
   static constexpr int K_TILE = BS * K_ROW;
   static constexpr int V_TILE = BS * V_ROW;
   static constexpr int STAGE = K_TILE + V_TILE;
-  // tensor-core engine for groups of 4 or 8 query heads (INT8/INT8 with D >= 128, FP16/FP16)
+  // tensor-core engine for groups of 4 or 8 query heads (INT8/INT8 with D >= 128, FP16/FP16), and
+  // for every group size with E4M3 codes (their conversion to fp16 is one instruction per pair)
+  static constexpr bool FP8 = KT == PKV_FP8_E4M3 && VT == PKV_FP8_E4M3;
   static constexpr bool MMA =
-      GT >= 4 && ((KT == PKV_INT8_SYM && VT == PKV_INT8_SYM && D >= 128) || (KT == PKV_FP16 && VT == PKV_FP16));
+      (GT >= 4 && ((KT == PKV_INT8_SYM && VT == PKV_INT8_SYM && D >= 128) || (KT == PKV_FP16 && VT == PKV_FP16))) ||
+      (FP8 && D >= 128);
   static constexpr int WARPS_AUTO =
       MMA ? (D >= 256 ? 8 : 12) : (KT == PKV_FP16 ? 8 : (GT == 1 ? 16 : (GT == 2 ? 12 : 8)));
   static constexpr int WARPS_WANT = PKV_DECODE_WARPS_SM > 0 ? PKV_DECODE_WARPS_SM : WARPS_AUTO;
@@ -432,6 +435,11 @@ __device__ __forceinline__ uint32_t h2_pack(float lo, float hi) {
 // fp16 1024 + 128 in both halves: a byte b placed under exponent 0x64 reads 1024 + b, and
 // (c ^ 0x80) = c + 128 for a signed code c, so subtracting this leaves c exactly
 constexpr uint32_t kH2Bias = 0x64806480u;
+// two E4M3 codes (low byte first) -> two exact fp16 values (low half first)
+__device__ __forceinline__ uint32_t fp8x2_to_h2(uint32_t two) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xffffu), __NV_E4M3);
+  return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
 
 // Tensor-core engine (4 or 8 query heads per KV head): per 16-token slice of a block,
 //   S = K . q^T  as mma m16n8k16 with M = 16 tokens, N = 8 heads, K = 16 dims per step, and
@@ -503,6 +511,24 @@ struct MmaEngine {
             a[1] = h2_sub(__byte_perm(u1, 0x64646464u, 0x4140), kH2Bias);  // row g+8
             a[2] = h2_sub(__byte_perm(u0, 0x64646464u, 0x4342), kH2Bias);  // row g, dims +2,+3
             a[3] = h2_sub(__byte_perm(u1, 0x64646464u, 0x4342), kH2Bias);  // row g+8
+            const int kk = 4 * i + q4;
+            mma_16816(sacc, a, qb[kk][0], qb[kk][1]);
+          }
+        }
+      } else if constexpr (KT == PKV_FP8_E4M3) {
+#pragma unroll
+        for (int i = 0; i < KS / 4; ++i) {  // 16 codes = 4 steps per 16-byte load
+          const uint4 r0 = *reinterpret_cast<const uint4*>(kt + swz<C::K_ROW>(kr0, kx + 16 * i));
+          const uint4 r1 = *reinterpret_cast<const uint4*>(kt + swz<C::K_ROW>(kr0 + 8, kx + 16 * i));
+          const uint32_t w0[4] = {r0.x, r0.y, r0.z, r0.w};
+          const uint32_t w1[4] = {r1.x, r1.y, r1.z, r1.w};
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint32_t a[4];
+            a[0] = fp8x2_to_h2(w0[q4]);        // row g, dims +0,+1
+            a[1] = fp8x2_to_h2(w1[q4]);        // row g+8
+            a[2] = fp8x2_to_h2(w0[q4] >> 16);  // row g, dims +2,+3
+            a[3] = fp8x2_to_h2(w1[q4] >> 16);  // row g+8
             const int kk = 4 * i + q4;
             mma_16816(sacc, a, qb[kk][0], qb[kk][1]);
           }
@@ -581,6 +607,31 @@ struct MmaEngine {
             a[1] = h2_sub((__byte_perm(xa[wd], xb[wd], sel1) & 0x00FF00FFu) ^ kH2Bias, kH2Bias);
             a[2] = h2_sub((__byte_perm(xc[wd], xd[wd], sel0) & 0x00FF00FFu) ^ kH2Bias, kH2Bias);
             a[3] = h2_sub((__byte_perm(xc[wd], xd[wd], sel1) & 0x00FF00FFu) ^ kH2Bias, kH2Bias);
+            const int j = 8 * i + jj;
+            mma_16816(acc[j], a, bh0, bh1);
+            mma_16816(acc[j], a, bl0, bl1);
+          }
+        }
+      } else if constexpr (VT == PKV_FP8_E4M3) {
+#pragma unroll
+        for (int i = 0; i < KS / 8; ++i) {  // 16 codes per row = 8 dim tiles
+          const uint4 ra = *reinterpret_cast<const uint4*>(vt + swz<C::V_ROW>(vr, vx + 16 * i));
+          const uint4 rb = *reinterpret_cast<const uint4*>(vt + swz<C::V_ROW>(vr + 1, vx + 16 * i));
+          const uint4 rc = *reinterpret_cast<const uint4*>(vt + swz<C::V_ROW>(vr + 8, vx + 16 * i));
+          const uint4 rd = *reinterpret_cast<const uint4*>(vt + swz<C::V_ROW>(vr + 9, vx + 16 * i));
+          const uint32_t xa[4] = {ra.x, ra.y, ra.z, ra.w}, xb[4] = {rb.x, rb.y, rb.z, rb.w};
+          const uint32_t xc[4] = {rc.x, rc.y, rc.z, rc.w}, xd[4] = {rd.x, rd.y, rd.z, rd.w};
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) {  // dim tile: bytes 2jj (M row g) and 2jj+1 (M row g+8)
+            const int wd = jj / 2, k = 2 * (jj % 2);
+            // {row r byte k, row r+1 byte k, row r byte k+1, row r+1 byte k+1}
+            const uint32_t sel = k | ((4 + k) << 4) | ((k + 1) << 8) | ((5 + k) << 12);
+            const uint32_t pab = __byte_perm(xa[wd], xb[wd], sel), pcd = __byte_perm(xc[wd], xd[wd], sel);
+            uint32_t a[4];
+            a[0] = fp8x2_to_h2(pab);
+            a[1] = fp8x2_to_h2(pab >> 16);
+            a[2] = fp8x2_to_h2(pcd);
+            a[3] = fp8x2_to_h2(pcd >> 16);
             const int j = 8 * i + jj;
             mma_16816(acc[j], a, bh0, bh1);
             mma_16816(acc[j], a, bl0, bl1);

@@ -141,12 +141,14 @@ struct StepParams {
 };
 cudaError_t launch_decode_step(const DecodeParams& p, const StepParams& sp, const DecodeShape& sh,
                                cudaStream_t stream);
-// per dtype pair (decode_i8i8.cu, decode_i8i4.cu, decode_f16.cu)
+// per dtype pair (decode_i8i8.cu, decode_i8i4.cu, decode_f16.cu, decode_fp8.cu)
 cudaError_t launch_decode_i8i8(const DecodeParams&, const StepParams&, const DecodeShape&, cudaStream_t);
 cudaError_t launch_decode_i8i4(const DecodeParams&, const StepParams&, const DecodeShape&, cudaStream_t);
 cudaError_t launch_decode_f16(const DecodeParams&, const StepParams&, const DecodeShape&, cudaStream_t);
+cudaError_t launch_decode_fp8(const DecodeParams&, const StepParams&, const DecodeShape&, cudaStream_t);
 bool decode_info_i8i8(const DecodeShape&, DecodeKernelInfo*);
 bool decode_info_i8i4(const DecodeShape&, DecodeKernelInfo*);
 bool decode_info_f16(const DecodeShape&, DecodeKernelInfo*);
+bool decode_info_fp8(const DecodeShape&, DecodeKernelInfo*);
 
 }  // namespace pkv

@@ -34,6 +34,8 @@ cudaError_t launch_store(const StoreParams& p, cudaStream_t stream) {
     store_quantized_kernel<PKV_INT8_SYM, PKV_FP16><<<grid, block, 0, stream>>>(p);
   else if (p.k_dtype == PKV_FP16 && p.v_dtype == PKV_INT8_SYM)
     store_quantized_kernel<PKV_FP16, PKV_INT8_SYM><<<grid, block, 0, stream>>>(p);
+  else if (p.k_dtype == PKV_FP8_E4M3 && p.v_dtype == PKV_FP8_E4M3)
+    store_quantized_kernel<PKV_FP8_E4M3, PKV_FP8_E4M3><<<grid, block, 0, stream>>>(p);
   else if (p.k_dtype == PKV_FP16 && p.v_dtype == PKV_INT4_ASYM)
     store_quantized_kernel<PKV_FP16, PKV_INT4_ASYM><<<grid, block, 0, stream>>>(p);
   else

@@ -24,6 +24,12 @@
 //    the smallest and largest code (INT4), and requantizing an old code depends on the code
 //    alone, so each tile's old codes go through a 256-entry table built once per rebuild.
 //
+// FP8 E4M3 (yunthe.com, same page, section "vLLM推理引擎部署与KV Cache量化配置实战": the fp8 cache
+// mode stores E4M3 values): scale = absmax / 448 per (block, head), code = E4M3(x / scale) rounded
+// to nearest even and saturated (the hardware conversion), new values fit a stored scale when
+// |x / scale| <= 448; a rebuild requantizes old codes through the same kind of 256-entry table
+// (an E4M3 code's requantized value depends on the code alone).
+//
 // Work split: one warp per (token, KV head). The warp of the first token of a group (the run of
 // tokens bound for one block) does the whole group; the others return at once.
 #pragma once
@@ -92,6 +98,21 @@ __device__ __forceinline__ bool fits_asym(float lo, float hi, float s_old, int z
   const int r_lo = __float2int_rn(__fadd_rn(__fdiv_rn(lo, s_old), (float)zp_old));
   const int r_hi = __float2int_rn(__fadd_rn(__fdiv_rn(hi, s_old), (float)zp_old));
   return r_lo >= 0 && r_hi <= 15;
+}
+
+// E4M3 code of x / s (nearest even, saturated at +-448); 0 if s == 0
+__device__ __forceinline__ uint32_t quant_fp8(float x, float s) {
+  if (s == 0.0f) return 0u;
+  return (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(x, s), __NV_SATFINITE, __NV_E4M3);
+}
+// value of an E4M3 code (exact in binary32)
+__device__ __forceinline__ float fp8_value(uint32_t code) {
+  return __half2float(__half(__nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)code, __NV_E4M3)));
+}
+// Do new values with largest magnitude m all fit a stored E4M3 scale? (|m / s| <= 448)
+__device__ __forceinline__ bool fits_fp8(float m, float s_old) {
+  if (s_old == 0.0f) return m == 0.0f;
+  return __fdiv_rn(m, s_old) <= 448.0f;
 }
 
 // four bytes of w through a 256-entry table (after xor-ing w with flip)
@@ -210,6 +231,53 @@ __device__ __noinline__ float rebuild_sym(int8_t* tile, int d, int o0, float s_o
   return s;
 }
 
+// largest magnitude field (code & 0x7f) among the 16 E4M3 codes of v: E4M3 magnitudes ascend with
+// their 7-bit pattern, so this code has the largest |value|
+__device__ __forceinline__ uint32_t fp8_magmax16(uint4 v) {
+  const uint32_t w[4] = {v.x & 0x7f7f7f7fu, v.y & 0x7f7f7f7fu, v.z & 0x7f7f7f7fu, v.w & 0x7f7f7f7fu};
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) m = max(max(m, max(w[i] & 0xffu, (w[i] >> 8) & 0xffu)), max((w[i] >> 16) & 0xffu, w[i] >> 24));
+  return m;
+}
+
+// Rebuild of the old rows [0, o0) of an E4M3 tile (rows of d codes) for values that do not fit:
+// x_hat = value(code) * s_old (binary32), new scale = max(max |x_hat|, m_new) / 448, old codes
+// requantized through a table. Returns the new scale.
+__device__ __noinline__ float rebuild_fp8(uint8_t* tile, int d, int o0, float s_old, float m_new, uint8_t* tbl,
+                                          int lane) {
+  uint4* v16 = reinterpret_cast<uint4*>(tile);
+  const int nvec = o0 * d / 16;
+  const int nchunks = (nvec + kChunkVecs - 1) / kChunkVecs;
+  uint4 v[4];
+  uint32_t qmax = 0;
+#pragma unroll 1
+  for (int c = 0; c < nchunks; ++c) {
+    load_chunk(v16, nvec, c, lane, v);
+#pragma unroll 1
+    for (int j = 0; j < 4; ++j) {
+      qmax = max(qmax, fp8_magmax16(v[0]));
+      rotate(v);
+    }
+  }
+  qmax = __reduce_max_sync(kFull, qmax);
+  const float m_old = __fmul_rn(fp8_value(qmax), s_old);
+  const float s = __fdiv_rn(fmaxf(m_old, m_new), 448.0f);
+  // table entry b: the requantized code of code b; lane l fills entries 8l .. 8l+7
+  uint32_t lo = 0, hi = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t b = (uint32_t)(lane * 8 + j);
+    const uint32_t c = quant_fp8(__fmul_rn(fp8_value(b), s_old), s);
+    if (j < 4) lo |= c << (8 * j); else hi |= c << (8 * (j - 4));
+  }
+  reinterpret_cast<uint2*>(tbl)[lane] = make_uint2(lo, hi);
+  __syncwarp();
+  requant_rows(v16, nvec, nchunks, 0u, tbl, lane, v);
+  __syncwarp();
+  return s;
+}
+
 // Rebuild of the old rows [0, o0) of an INT4 tile (rows of d / 2 bytes) for values that do not
 // fit: x_hat = (code - zp_old) * s_old (binary32), range [min(lo_new, x_hat), max(hi_new, x_hat)],
 // new scale and zero point from it, old codes requantized. tbl: 256 bytes of shared memory.
@@ -294,6 +362,40 @@ __device__ __noinline__ void store_sym(const GroupSrc& src, int8_t* tile, float*
     uint32_t out = 0;
 #pragma unroll
     for (int u = 0; u < 4; ++u) out |= ((uint32_t)(quant_sym(f[u], s) & 0xff)) << (8 * u);
+    reinterpret_cast<uint32_t*>(dst)[e] = out;
+  }
+  if (lane == 0) *scale_ptr = s;
+}
+
+// ---- E4M3 side of one (block, head) tile, groups of several tokens ----
+__device__ __noinline__ void store_fp8(const GroupSrc& src, uint8_t* tile, float* scale_ptr, int o0, uint8_t* tbl,
+                                       int lane) {
+  const int d = src.d, n = src.n;
+  const int quads = n * d / 4;
+  float m_new = 0.0f;
+  for (int e = lane; e < quads; e += 32) {
+    const int i = (4 * e) / d, j = (4 * e) % d;
+    float f[4];
+    load4(src.base + i * src.row_stride + j, f);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) m_new = fmaxf(m_new, fabsf(f[u]));
+  }
+  m_new = warp_max(m_new);
+  float s;
+  if (o0 == 0) {
+    s = __fdiv_rn(m_new, 448.0f);
+  } else {
+    const float s_old = *scale_ptr;
+    s = fits_fp8(m_new, s_old) ? s_old : rebuild_fp8(tile, d, o0, s_old, m_new, tbl, lane);
+  }
+  uint8_t* dst = tile + (size_t)o0 * d;
+  for (int e = lane; e < quads; e += 32) {
+    const int i = (4 * e) / d, j = (4 * e) % d;
+    float f[4];
+    load4(src.base + i * src.row_stride + j, f);
+    uint32_t out = 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) out |= quant_fp8(f[u], s) << (8 * u);
     reinterpret_cast<uint32_t*>(dst)[e] = out;
   }
   if (lane == 0) *scale_ptr = s;
@@ -407,6 +509,38 @@ __device__ __forceinline__ void append_sym(const float x[8], int vpl, int8_t* ti
     if (i < 4) lo |= c << (8 * i); else hi |= c << (8 * (i - 4));
   }
   int8_t* dst = tile + (size_t)o0 * d + lane * vpl;
+  if (vpl == 8) *reinterpret_cast<uint2*>(dst) = make_uint2(lo, hi);
+  else if (vpl == 4) *reinterpret_cast<uint32_t*>(dst) = lo;
+  else *reinterpret_cast<uint16_t*>(dst) = (uint16_t)lo;
+  if (set_scale && lane == 0) *scale_ptr = s;
+}
+
+// E4M3 side of a one-token group at offset o0 (s_old: the stored scale when o0 > 0).
+__device__ __forceinline__ void append_fp8(const float x[8], int vpl, uint8_t* tile, float* scale_ptr, float s_old,
+                                          int o0, int d, uint8_t* tbl, int lane) {
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    if (i < vpl) m = fmaxf(m, fabsf(x[i]));
+  m = warp_max(m);
+  float s;
+  bool set_scale = true;
+  if (o0 == 0) {
+    s = __fdiv_rn(m, 448.0f);
+  } else if (fits_fp8(m, s_old)) {
+    s = s_old;
+    set_scale = false;
+  } else {
+    s = rebuild_fp8(tile, d, o0, s_old, m, tbl, lane);
+  }
+  uint32_t lo = 0, hi = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if (i >= vpl) continue;
+    const uint32_t c = quant_fp8(x[i], s);
+    if (i < 4) lo |= c << (8 * i); else hi |= c << (8 * (i - 4));
+  }
+  uint8_t* dst = tile + (size_t)o0 * d + lane * vpl;
   if (vpl == 8) *reinterpret_cast<uint2*>(dst) = make_uint2(lo, hi);
   else if (vpl == 4) *reinterpret_cast<uint32_t*>(dst) = lo;
   else *reinterpret_cast<uint16_t*>(dst) = (uint16_t)lo;
@@ -536,7 +670,7 @@ __device__ __forceinline__ void store_job(const StoreParams& p, const int t, con
     float ks_old = 0.f, vs_old = 0.f;
     int vzp_old = 0;
     if (o0 > 0) {
-      if constexpr (KT == PKV_INT8_SYM) ks_old = p.k_scale[tile_idx];
+      if constexpr (KT != PKV_FP16) ks_old = p.k_scale[tile_idx];
       if constexpr (VT != PKV_FP16) vs_old = p.v_scale[tile_idx];
       if constexpr (VT == PKV_INT4_ASYM) vzp_old = p.v_zp[tile_idx];
     }
@@ -545,11 +679,15 @@ __device__ __forceinline__ void store_job(const StoreParams& p, const int t, con
     halves_to_float(vraw, vx);
     if constexpr (KT == PKV_INT8_SYM) {
       append_sym(kx, vpl, k_tile8, p.k_scale + tile_idx, ks_old, o0, d, tbl, lane);
+    } else if constexpr (KT == PKV_FP8_E4M3) {
+      append_fp8(kx, vpl, reinterpret_cast<uint8_t*>(k_tile8), p.k_scale + tile_idx, ks_old, o0, d, tbl, lane);
     } else {
       append_fp16(kraw, vpl, k_tile16, o0, d, lane);
     }
     if constexpr (VT == PKV_INT8_SYM) {
       append_sym(vx, vpl, v_tile8, p.v_scale + tile_idx, vs_old, o0, d, tbl, lane);
+    } else if constexpr (VT == PKV_FP8_E4M3) {
+      append_fp8(vx, vpl, reinterpret_cast<uint8_t*>(v_tile8), p.v_scale + tile_idx, vs_old, o0, d, tbl, lane);
     } else if constexpr (VT == PKV_INT4_ASYM) {
       append_asym4(vx, vpl, v_tile4, p.v_scale + tile_idx, p.v_zp + tile_idx, vs_old, vzp_old, o0, d, tbl, lane);
     } else {
@@ -566,12 +704,16 @@ __device__ __forceinline__ void store_job(const StoreParams& p, const int t, con
   src.base = p.k_new + (size_t)t * src.row_stride + (size_t)h * d;
   if constexpr (KT == PKV_INT8_SYM) {
     store_sym(src, k_tile8, p.k_scale + tile_idx, o0, tbl, lane);
+  } else if constexpr (KT == PKV_FP8_E4M3) {
+    store_fp8(src, reinterpret_cast<uint8_t*>(k_tile8), p.k_scale + tile_idx, o0, tbl, lane);
   } else {
     store_fp16(src, k_tile16, o0, lane);
   }
   src.base = p.v_new + (size_t)t * src.row_stride + (size_t)h * d;
   if constexpr (VT == PKV_INT8_SYM) {
     store_sym(src, v_tile8, p.v_scale + tile_idx, o0, tbl, lane);
+  } else if constexpr (VT == PKV_FP8_E4M3) {
+    store_fp8(src, reinterpret_cast<uint8_t*>(v_tile8), p.v_scale + tile_idx, o0, tbl, lane);
   } else if constexpr (VT == PKV_INT4_ASYM) {
     store_asym4(src, v_tile4, p.v_scale + tile_idx, p.v_zp + tile_idx, o0, tbl, lane);
   } else {

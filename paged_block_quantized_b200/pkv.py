@@ -22,7 +22,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 # ---- enums (values fixed by include/pkv.h) ----
 PKV_OK, PKV_ERR_INVALID_ARG, PKV_ERR_UNSUPPORTED, PKV_ERR_OUT_OF_BLOCKS, PKV_ERR_CUDA, PKV_ERR_DEVICE_TIMEOUT = range(6)
-PKV_FP16, PKV_INT8_SYM, PKV_INT4_ASYM = 0, 1, 2
+PKV_FP16, PKV_INT8_SYM, PKV_INT4_ASYM, PKV_FP8_E4M3 = 0, 1, 2, 3
 (PKV_DEVERR_NONE, PKV_DEVERR_BLOCK_ID, PKV_DEVERR_SLOT, PKV_DEVERR_SLOT_GROUP, PKV_DEVERR_CONTEXT_LEN,
  PKV_DEVERR_TIMEOUT) = range(6)
 
@@ -353,7 +353,8 @@ class DevicePool:
             return torch.empty(shape, dtype=dtype, device=device)
 
         def codes(dt):
-            row = {PKV_FP16: 2 * head_dim, PKV_INT8_SYM: head_dim, PKV_INT4_ASYM: head_dim // 2}[dt]
+            row = {PKV_FP16: 2 * head_dim, PKV_INT8_SYM: head_dim, PKV_INT4_ASYM: head_dim // 2,
+                   PKV_FP8_E4M3: head_dim}[dt]
             return empty((num_blocks, num_kv_heads, block_size, row), torch.uint8)
 
         k = codes(k_dtype)

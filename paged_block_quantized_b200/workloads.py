@@ -17,7 +17,8 @@ block by block ("prefill").
 Named workloads (sizes from the pages' scenarios):
   tiny       4 seqs, L = {17, 33, 50, 64}, 4 heads MHA, D 64, bs 16, 64-block pool, INT8/INT8
   llama7b    32 seqs, L ~ U{500..2000}, 32 heads MHA, D 128, bs 16, 8192-block pool, INT8/INT8,
-             K/V with 1% outlier channels x8 (``llama7b_fp16``: same with an FP16 cache)
+             K/V with 1% outlier channels x8 (``llama7b_fp16``: same with an FP16 cache;
+             ``llama7b_fp8``: same with an FP8 E4M3 cache)
   long       8 seqs, L ~ U{8192..32768}, 32 heads, D 128, bs 32, K INT8 / V INT4 (the decode
              splits the long contexts across worker warps itself)
   gqa_prefix 64 seqs, 64 q heads / 8 KV heads, D 128, bs 16, 64 shared prefix blocks then 64
@@ -32,7 +33,7 @@ from dataclasses import dataclass, field
 
 import numpy as np
 
-FP16, INT8_SYM, INT4_ASYM = 0, 1, 2
+FP16, INT8_SYM, INT4_ASYM, FP8_E4M3 = 0, 1, 2, 3
 
 _VALUES, _NEWTOK, _OUTLIER, _LAYOUT, _QUERY = 11, 12, 13, 14, 15
 
@@ -176,7 +177,7 @@ class Workload:
         zero points, block-table entries, q, context lens. With unique=True a physical block
         shared by several sequences is counted once."""
         H, D, bs = self.num_kv_heads, self.head_dim, self.block_size
-        code_b = {FP16: 2.0, INT8_SYM: 1.0, INT4_ASYM: 0.5}
+        code_b = {FP16: 2.0, INT8_SYM: 1.0, INT4_ASYM: 0.5, FP8_E4M3: 1.0}
         per_tok = H * D * (code_b[self.k_dtype] + code_b[self.v_dtype])
         meta = H * ((4 if self.k_dtype != FP16 else 0) + (4 if self.v_dtype != FP16 else 0)
                     + (1 if self.v_dtype == INT4_ASYM else 0))
@@ -202,7 +203,7 @@ class Workload:
         """Algorithmic bytes of the step's store: each new token's fp16 K and V rows read, its codes
         written, the slot read, and the per-(block, head) scale (and zero point) written."""
         H, D = self.num_kv_heads, self.head_dim
-        code_b = {FP16: 2.0, INT8_SYM: 1.0, INT4_ASYM: 0.5}
+        code_b = {FP16: 2.0, INT8_SYM: 1.0, INT4_ASYM: 0.5, FP8_E4M3: 1.0}
         row = D * (code_b[self.k_dtype] + code_b[self.v_dtype])
         meta = (4 if self.k_dtype != FP16 else 0) + (4 if self.v_dtype != FP16 else 0) + (1 if self.v_dtype == INT4_ASYM else 0)
         return int(self.num_seqs * (8 + H * (4 * D + row + meta)))
@@ -211,7 +212,7 @@ class Workload:
         """Algorithmic bytes of the step's copy-on-write copies: each whole block (all heads, codes,
         scales, zero points) read once and written once, plus the mapping entries."""
         H, D, bs = self.num_kv_heads, self.head_dim, self.block_size
-        code_b = {FP16: 2.0, INT8_SYM: 1.0, INT4_ASYM: 0.5}
+        code_b = {FP16: 2.0, INT8_SYM: 1.0, INT4_ASYM: 0.5, FP8_E4M3: 1.0}
         meta = (4 if self.k_dtype != FP16 else 0) + (4 if self.v_dtype != FP16 else 0) + (1 if self.v_dtype == INT4_ASYM else 0)
         block = H * (bs * D * (code_b[self.k_dtype] + code_b[self.v_dtype]) + meta)
         return int(self.cow_pairs.shape[0] * (2 * block + 8))
@@ -286,15 +287,16 @@ def make(name: str, seed: int = 0, **over) -> Workload:
                  num_blocks=64, k_dtype=INT8_SYM, v_dtype=INT8_SYM, outliers=False,
                  partition_tokens=0, context_lens=np.array([17, 33, 50, 64]))
         desc = "4 seqs, L={17,33,50,64}, 4 heads MHA, D 64, bs 16, 64-block pool, INT8/INT8"
-    elif name in ("llama7b", "llama7b_fp16"):
+    elif name in ("llama7b", "llama7b_fp16", "llama7b_fp8"):
         S = over.get("num_seqs", 32)
-        fp = name.endswith("fp16")
+        dt = {"llama7b": INT8_SYM, "llama7b_fp16": FP16, "llama7b_fp8": FP8_E4M3}[name]
+        rng = np.random.default_rng([seed, 1, sum(map(ord, "llama7b"))])  # the same lengths for all three
         p = dict(num_seqs=S, num_q_heads=32, num_kv_heads=32, head_dim=128, block_size=16,
-                 num_blocks=8192, k_dtype=FP16 if fp else INT8_SYM, v_dtype=FP16 if fp else INT8_SYM,
-                 outliers=True, partition_tokens=0,
+                 num_blocks=8192, k_dtype=dt, v_dtype=dt, outliers=True, partition_tokens=0,
                  context_lens=rng.integers(500, 2001, size=S))
         desc = ("Llama-2-7B-shaped decode layer: 32 seqs, L~U{500..2000}, 32 heads MHA, D 128, "
-                "bs 16, 8192-block pool, 1% outlier channels x8, " + ("FP16 cache" if fp else "INT8/INT8"))
+                "bs 16, 8192-block pool, 1% outlier channels x8, "
+                + {INT8_SYM: "INT8/INT8", FP16: "FP16 cache", FP8_E4M3: "FP8 E4M3 cache"}[dt])
     elif name == "long":
         S = over.get("num_seqs", 8)
         p = dict(num_seqs=S, num_q_heads=32, num_kv_heads=32, head_dim=128, block_size=32,

@@ -13,7 +13,7 @@ import oracle
 
 
 def _odt(dt):
-    return {0: oracle.FP16, 1: oracle.INT8_SYM, 2: oracle.INT4_ASYM}[dt]
+    return {0: oracle.FP16, 1: oracle.INT8_SYM, 2: oracle.INT4_ASYM, 3: oracle.FP8_E4M3}[dt]
 
 
 def oracle_step(w, seqs=None, num_threads=None):

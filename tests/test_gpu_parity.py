@@ -56,6 +56,7 @@ REDUCED = {
     "tiny": {},
     "llama7b": dict(num_seqs=4),
     "llama7b_fp16": dict(num_seqs=4),
+    "llama7b_fp8": dict(num_seqs=4),
     "long": dict(num_seqs=2, context_lens=[8192 + 37, 9001]),
     "gqa_prefix": dict(num_seqs=4, prefix_blocks=8, private_blocks=9),
     "mixed": dict(num_seqs=24, children=4),
@@ -71,6 +72,7 @@ def test_config_reduced_sizes(name, path):
 FULL_SAMPLES = {
     "llama7b": [0, 7, 31],
     "llama7b_fp16": [3, 30],
+    "llama7b_fp8": [0, 31],
     "long": [int(np.argmin(W.make("long").context_lens))],
     "gqa_prefix": [0, 33, 63],
     "mixed": None,  # a parent, its child and two others, chosen below
@@ -112,6 +114,11 @@ def test_split_matches_unsplit():
     dict(head_dim=256, block_size=32, num_q_heads=16, num_kv_heads=2),
     dict(head_dim=64, block_size=32, num_q_heads=16, num_kv_heads=4, k_dtype=W.FP16, v_dtype=W.FP16),
     dict(head_dim=128, block_size=32, num_q_heads=16, num_kv_heads=4),
+    # E4M3 cache: the tensor-core engine for every group size (1, 2, 4 and 8 heads per warp)
+    dict(head_dim=128, block_size=16, num_q_heads=4, num_kv_heads=4, k_dtype=W.FP8_E4M3, v_dtype=W.FP8_E4M3),
+    dict(head_dim=256, block_size=32, num_q_heads=8, num_kv_heads=4, k_dtype=W.FP8_E4M3, v_dtype=W.FP8_E4M3),
+    dict(head_dim=128, block_size=32, num_q_heads=16, num_kv_heads=4, k_dtype=W.FP8_E4M3, v_dtype=W.FP8_E4M3),
+    dict(head_dim=128, block_size=16, num_q_heads=16, num_kv_heads=2, k_dtype=W.FP8_E4M3, v_dtype=W.FP8_E4M3),
 ])
 def test_shapes_and_groups(case):
     lens = [1, 2, 16, 17, 31, 32, 33, 100, 700]
@@ -244,7 +251,8 @@ def test_append_rebuild_bit_exact():
 
 @pytest.mark.parametrize("bs,D,kt,vt", [(32, 256, W.INT8_SYM, W.INT4_ASYM), (32, 128, W.INT8_SYM, W.INT8_SYM),
                                          (16, 64, W.FP16, W.INT4_ASYM), (16, 256, W.INT8_SYM, W.INT8_SYM),
-                                         (32, 64, W.INT8_SYM, W.FP16)])
+                                         (32, 64, W.INT8_SYM, W.FP16), (16, 128, W.FP8_E4M3, W.FP8_E4M3),
+                                         (32, 256, W.FP8_E4M3, W.FP8_E4M3), (16, 64, W.FP8_E4M3, W.FP8_E4M3)])
 def test_token_by_token_appends_bit_exact(bs, D, kt, vt):
     """Decode-step appends one token at a time into every offset of a tile, with tokens that force a
     rebuild at early and late offsets (tiles larger than one batch of a rebuild's loads included),
@@ -253,7 +261,7 @@ def test_token_by_token_appends_bit_exact(bs, D, kt, vt):
     from paged_block_quantized_b200 import pkv
     rng = np.random.default_rng(21 + bs + D)
     nb, H = 6, 3
-    ot = {W.FP16: oracle.FP16, W.INT8_SYM: oracle.INT8_SYM, W.INT4_ASYM: oracle.INT4_ASYM}
+    ot = {W.FP16: oracle.FP16, W.INT8_SYM: oracle.INT8_SYM, W.INT4_ASYM: oracle.INT4_ASYM, W.FP8_E4M3: oracle.FP8_E4M3}
     pool = pkv.DevicePool.allocate(nb, bs, H, D, kt, vt, fill=0x5A)
     c = oracle.OracleCache.empty(nb, bs, H, D, ot[kt], ot[vt], poison=0x5A)
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -295,7 +303,7 @@ def test_token_by_token_appends_bit_exact(bs, D, kt, vt):
 
 @pytest.mark.parametrize("name,over", [("mixed", dict(num_seqs=24, children=4)), ("llama7b", dict(num_seqs=6)),
                                        ("gqa_prefix", dict(num_seqs=4, prefix_blocks=8, private_blocks=9)),
-                                       ("llama7b_fp16", dict(num_seqs=3))])
+                                       ("llama7b_fp16", dict(num_seqs=3)), ("llama7b_fp8", dict(num_seqs=3))])
 def test_fused_step_matches_separate_launches(name, over):
     """pkv_decode_step (copies, store and decode in one cooperative launch) gives the same pool
     bytes and the same outputs as the three separate calls, on several steps in a row (its grid
@@ -315,8 +323,8 @@ def test_fused_step_matches_separate_launches(name, over):
         np.testing.assert_array_equal(gf.out.cpu().numpy(), gs.out.cpu().numpy())
         # tickets (one per sequence and head group) and the two barrier counters lead the workspace
         group = w.num_q_heads // w.num_kv_heads
-        mma = (w.k_dtype, w.v_dtype) == (W.FP16, W.FP16) or ((w.k_dtype, w.v_dtype) == (W.INT8_SYM, W.INT8_SYM)
-                                                              and w.head_dim >= 128)
+        mma = (w.k_dtype, w.v_dtype) in ((W.FP16, W.FP16), (W.FP8_E4M3, W.FP8_E4M3)) or (
+            (w.k_dtype, w.v_dtype) == (W.INT8_SYM, W.INT8_SYM) and w.head_dim >= 128)
         gt = 8 if mma and group % 8 == 0 else 4 if group % 4 == 0 else 2 if group % 2 == 0 else 1
         units = w.num_seqs * (w.num_q_heads // gt)
         ws = gf.workspace.view(torch.int32)[: units + 2].cpu().numpy()
