@@ -18,6 +18,8 @@ Parity status of each function (what pins it; see ``tests/test_oracle_*.py``):
   copy   pinned (byte identity, untouched blocks).
   decode pinned (library attention on contiguous data, permutation / prefix-sharing
          invariance, closed-form special cases, brute-force agreement).
+  prefill (chunked, causal) pinned (library attention with an explicit causal mask on contiguous
+         data, equality with decode for one-token chunks, chunk splitting, brute force).
 """
 from __future__ import annotations
 
@@ -67,6 +69,9 @@ def _load():
         lib.oracle_decode.argtypes = [P, P, ctypes.c_int32, ctypes.c_int32, P, ctypes.c_int32, P,
                                       ctypes.c_int32, ctypes.c_float, P, ctypes.c_int32]
         lib.oracle_decode.restype = ctypes.c_int32
+        lib.oracle_prefill.argtypes = [P, P, ctypes.c_int32, ctypes.c_int32, P, P, ctypes.c_int32, P,
+                                       ctypes.c_float, P, ctypes.c_int32]
+        lib.oracle_prefill.restype = ctypes.c_int32
         lib.oracle_fp8_e4m3_decode.argtypes = [ctypes.c_uint8]
         lib.oracle_fp8_e4m3_decode.restype = ctypes.c_double
         lib.oracle_fp8_e4m3_encode.argtypes = [ctypes.c_float]
@@ -192,6 +197,31 @@ def decode(cache: OracleCache, q: np.ndarray, block_tables: np.ndarray, context_
     rc = _load().oracle_decode(ctypes.byref(c), q_bits.ctypes.data, S, Hq, bt.ctypes.data, bt.shape[1],
                                cl.ctypes.data, int(max_context_len), ctypes.c_float(softmax_scale),
                                out.ctypes.data, int(num_threads))
+    if rc < 0:
+        raise ValueError("unsupported cache descriptor or head split")
+    return out, int(rc)
+
+
+def prefill(cache: OracleCache, q: np.ndarray, cu_q_lens: np.ndarray, block_tables: np.ndarray,
+            context_lens: np.ndarray, softmax_scale: float, num_threads: int | None = None):
+    """Binary64 chunked-prefill attention: the rows of sequence s (q[cu_q_lens[s]:cu_q_lens[s+1]])
+    are its last q_len context tokens, each attending causally. Returns (out [T][Hq][D], error)."""
+    q_bits = _fp16_bits(q)
+    T, Hq, D = q_bits.shape
+    assert D == cache.head_dim
+    cu = np.ascontiguousarray(cu_q_lens, dtype=np.int32)
+    S = cu.shape[0] - 1
+    assert cu[-1] == T if S > 0 else T == 0
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    cl = np.ascontiguousarray(context_lens, dtype=np.int32)
+    assert bt.shape[0] == S and cl.shape == (S,)
+    if num_threads is None:
+        num_threads = os.cpu_count() or 1
+    out = np.zeros((T, Hq, D), dtype=np.float64)
+    c = cache._c()
+    rc = _load().oracle_prefill(ctypes.byref(c), q_bits.ctypes.data, S, Hq, cu.ctypes.data, bt.ctypes.data,
+                                bt.shape[1], cl.ctypes.data, ctypes.c_float(softmax_scale), out.ctypes.data,
+                                int(num_threads))
     if rc < 0:
         raise ValueError("unsupported cache descriptor or head split")
     return out, int(rc)

@@ -436,6 +436,48 @@ static double dequant(const oracle_cache* c, int which_v, int block, int head, i
   return ((double)get_nibble(r, j) - (double)c->v_zp[meta]) * (double)c->v_scale[meta];
 }
 
+/* Attention of one query row (fp16 bits, head_dim values) over tokens [0, L) of one sequence
+ * (its block-table row), KV head g, in binary64: z_t = scale * q . k_hat_t, out = sum_t softmax(z)_t
+ * v_hat_t. A block id outside the pool leaves its tokens out and is reported. */
+static int32_t attend_row(const oracle_cache* c, const uint16_t* qrow, const int32_t* table_row, int L, int g,
+                          float softmax_scale, double* o) {
+  const int d = c->head_dim, bs = c->block_size;
+  int32_t local_err = 0;
+  for (int j = 0; j < d; ++j) o[j] = 0.0;
+  double qv[512];
+  for (int j = 0; j < d; ++j) qv[j] = half_bits_to_double(qrow[j]);
+  /* logits z_t = scale * q . k_hat_t for every valid token */
+  double* z = (double*)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+  int* valid = (int*)malloc(sizeof(int) * (size_t)(L > 0 ? L : 1));
+  double zmax = -INFINITY;
+  for (int t = 0; t < L; ++t) {
+    int block = table_row[t / bs];
+    valid[t] = (block >= 0 && block < c->num_blocks);
+    if (!valid[t]) {
+      local_err = ORACLE_DEVERR_BLOCK_ID;
+      continue;
+    }
+    double dot = 0.0;
+    for (int j = 0; j < d; ++j) dot += qv[j] * dequant(c, 0, block, g, t % bs, j);
+    z[t] = (double)softmax_scale * dot;
+    if (z[t] > zmax) zmax = z[t];
+  }
+  /* softmax over the valid tokens, then the weighted sum of v_hat */
+  double denom = 0.0;
+  for (int t = 0; t < L; ++t) {
+    if (!valid[t]) continue;
+    double w = exp(z[t] - zmax);
+    denom += w;
+    int block = table_row[t / bs];
+    for (int j = 0; j < d; ++j) o[j] += w * dequant(c, 1, block, g, t % bs, j);
+  }
+  if (denom > 0.0)
+    for (int j = 0; j < d; ++j) o[j] /= denom;
+  free(z);
+  free(valid);
+  return local_err;
+}
+
 int32_t oracle_decode(const oracle_cache* c, const uint16_t* q, int32_t num_seqs, int32_t num_q_heads,
                       const int32_t* block_tables, int32_t max_blocks_per_seq,
                       const int32_t* context_lens, int32_t max_context_len, float softmax_scale,
@@ -452,8 +494,6 @@ int32_t oracle_decode(const oracle_cache* c, const uint16_t* q, int32_t num_seqs
   for (int64_t sh = 0; sh < pairs; ++sh) {
     const int s = (int)(sh / num_q_heads), h = (int)(sh % num_q_heads);
     const int g = h / G; /* query head h reads KV head h / G */
-    double* o = out + (size_t)sh * d;
-    for (int j = 0; j < d; ++j) o[j] = 0.0;
     int32_t local_err = 0;
     int L = context_lens[s];
     if (L < 0 || L > max_context_len || L > max_blocks_per_seq * bs) {
@@ -462,37 +502,57 @@ int32_t oracle_decode(const oracle_cache* c, const uint16_t* q, int32_t num_seqs
       if (L > max_context_len) L = max_context_len;
       if (L > max_blocks_per_seq * bs) L = max_blocks_per_seq * bs;
     }
-    double qv[512];
-    for (int j = 0; j < d; ++j) qv[j] = half_bits_to_double(q[(size_t)sh * d + j]);
-    /* logits z_t = scale * q . k_hat_t for every valid token */
-    double* z = (double*)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
-    int* valid = (int*)malloc(sizeof(int) * (size_t)(L > 0 ? L : 1));
-    double zmax = -INFINITY;
-    for (int t = 0; t < L; ++t) {
-      int block = block_tables[(size_t)s * max_blocks_per_seq + t / bs];
-      valid[t] = (block >= 0 && block < c->num_blocks);
-      if (!valid[t]) {
-        local_err = local_err ? local_err : ORACLE_DEVERR_BLOCK_ID;
-        continue;
+    int32_t row_err = attend_row(c, q + (size_t)sh * d, block_tables + (size_t)s * max_blocks_per_seq, L, g,
+                                 softmax_scale, out + (size_t)sh * d);
+    if (!local_err) local_err = row_err;
+    if (local_err) {
+#pragma omp critical
+      record_error(&err, local_err);
+    }
+  }
+  return err;
+}
+
+/* Chunked prefill ([yunthe] "Prefix Caching与多轮对话场景优化实践": only the new tokens are computed,
+ * attending over the cached prefix; [tbr8] §5 item 2: dequantization inside the attention
+ * operator). Sequence s contributes q_len = cu_q_lens[s+1] - cu_q_lens[s] query tokens, the last
+ * q_len of its context_lens[s] tokens (already stored): the query at position
+ * p = context_lens[s] - q_len + i attends causally to tokens [0, p], i.e. it is the decode of that
+ * query over a context of p + 1 tokens. */
+int32_t oracle_prefill(const oracle_cache* c, const uint16_t* q, int32_t num_seqs, int32_t num_q_heads,
+                       const int32_t* cu_q_lens, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                       const int32_t* context_lens, float softmax_scale, double* out, int32_t num_threads) {
+  if (!dtypes_ok(c) || c->head_dim > 512) return -1;
+  const int H = c->num_kv_heads, d = c->head_dim, bs = c->block_size;
+  if (H <= 0 || num_q_heads % H != 0) return -1;
+  const int G = num_q_heads / H;
+  int32_t err = 0;
+  if (num_threads <= 0) num_threads = 1;
+  const int64_t rows = num_seqs > 0 ? (int64_t)cu_q_lens[num_seqs] * num_q_heads : 0;
+
+#pragma omp parallel for schedule(dynamic, 1) num_threads(num_threads)
+  for (int64_t rh = 0; rh < rows; ++rh) {
+    const int64_t row = rh / num_q_heads;
+    const int h = (int)(rh % num_q_heads);
+    int s = 0;
+    while (s + 1 < num_seqs && cu_q_lens[s + 1] <= row) ++s; /* the sequence holding this row */
+    const int q_len = cu_q_lens[s + 1] - cu_q_lens[s];
+    const int i = (int)(row - cu_q_lens[s]);
+    double* o = out + (size_t)rh * d;
+    int32_t local_err = 0;
+    int L = context_lens[s] - q_len + i + 1; /* causal: positions 0 .. p */
+    if (q_len > context_lens[s] || L < 1) {
+      local_err = ORACLE_DEVERR_CONTEXT_LEN;
+      for (int j = 0; j < d; ++j) o[j] = 0.0;
+    } else {
+      if (L > max_blocks_per_seq * bs) {
+        local_err = ORACLE_DEVERR_CONTEXT_LEN;
+        L = max_blocks_per_seq * bs;
       }
-      double dot = 0.0;
-      for (int j = 0; j < d; ++j) dot += qv[j] * dequant(c, 0, block, g, t % bs, j);
-      z[t] = (double)softmax_scale * dot;
-      if (z[t] > zmax) zmax = z[t];
+      int32_t row_err = attend_row(c, q + (size_t)rh * d, block_tables + (size_t)s * max_blocks_per_seq, L, h / G,
+                                   softmax_scale, o);
+      if (!local_err) local_err = row_err;
     }
-    /* softmax over the valid tokens, then the weighted sum of v_hat */
-    double denom = 0.0;
-    for (int t = 0; t < L; ++t) {
-      if (!valid[t]) continue;
-      double w = exp(z[t] - zmax);
-      denom += w;
-      int block = block_tables[(size_t)s * max_blocks_per_seq + t / bs];
-      for (int j = 0; j < d; ++j) o[j] += w * dequant(c, 1, block, g, t % bs, j);
-    }
-    if (denom > 0.0)
-      for (int j = 0; j < d; ++j) o[j] /= denom;
-    free(z);
-    free(valid);
     if (local_err) {
 #pragma omp critical
       record_error(&err, local_err);

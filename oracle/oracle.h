@@ -55,6 +55,13 @@ int32_t oracle_decode(const oracle_cache* c, const uint16_t* q, int32_t num_seqs
                       const int32_t* context_lens, int32_t max_context_len, float softmax_scale,
                       double* out, int32_t num_threads);
 
+/* Chunked prefill: causal attention of each sequence's last q_len context tokens (queries
+ * q [T][Hq][D], T = cu_q_lens[num_seqs], rows of sequence s at cu_q_lens[s] ..) over its cached
+ * tokens; out: double [T][Hq][D]. */
+int32_t oracle_prefill(const oracle_cache* c, const uint16_t* q, int32_t num_seqs, int32_t num_q_heads,
+                       const int32_t* cu_q_lens, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                       const int32_t* context_lens, float softmax_scale, double* out, int32_t num_threads);
+
 #ifdef __cplusplus
 }
 #endif

@@ -19,7 +19,7 @@ sys.path.insert(0, ROOT)
 from oracle import build as oracle_build  # noqa: E402
 
 PIN_TESTS = ["tests/test_oracle_store.py", "tests/test_oracle_decode.py", "tests/test_oracle_copy.py",
-             "tests/test_oracle_fp8.py"]
+             "tests/test_oracle_fp8.py", "tests/test_oracle_prefill.py"]
 EXPECTED_SURVIVORS = {"clamp128"}
 
 MUTANTS = {
@@ -46,6 +46,9 @@ MUTANTS = {
     "fp8_fit_480": ("else fits = (fabsf(new_x[i] / s_old) <= 448.0f);", "else fits = (fabsf(new_x[i] / s_old) <= 480.0f);"),
     "fp8_no_requant_old": ("for (int i = 0; i < n_old; ++i) tile[i] = quant_fp8(xh[i], s);", ""),
     "fp8_sign": ("uint8_t sign = signbit(x) ? 0x80 : 0x00;", "uint8_t sign = 0x00;"),
+    "prefill_causal_off_by_one": ("int L = context_lens[s] - q_len + i + 1; /* causal: positions 0 .. p */", "int L = context_lens[s] - q_len + i;"),
+    "prefill_not_causal": ("int L = context_lens[s] - q_len + i + 1; /* causal: positions 0 .. p */", "int L = context_lens[s];"),
+    "prefill_wrong_seq": ("while (s + 1 < num_seqs && cu_q_lens[s + 1] <= row) ++s;", "while (s + 1 < num_seqs && cu_q_lens[s + 1] < row) ++s;"),
     "copy_scales_missing": ("memcpy(c->k_scale + (size_t)dst * H, c->k_scale + (size_t)src * H, sizeof(float) * H);", ";"),
 }
 
