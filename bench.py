@@ -69,6 +69,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-beam-order", action="store_true",
+                    help="walk the sequences in index order instead of each forked child right after its parent")
     ap.add_argument("--fused", action="store_true",
                     help="time the step as one fused launch (pkv_decode_step) instead of copy, store, decode")
     return ap.parse_args()
@@ -295,7 +297,8 @@ def run_pkv(args, rank, world, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     w = W.make(args.config, seed=args.seed + rank)
-    g = DeviceStep(w, device=dev, poison=None, partition_tokens=args.partition_tokens)
+    g = DeviceStep(w, device=dev, poison=None, partition_tokens=args.partition_tokens,
+                   beam_order=not args.no_beam_order)
     g.prefill()
     g.snapshot_step_tiles()
     has_cow = w.cow_pairs.shape[0] > 0
@@ -399,7 +402,9 @@ def run_pkv(args, rank, world, local):
     peak, peak_src = measured_hbm_peak()
     traffic, _ = ncu_traffic(args.config)
     step_desc = (("copy-on-write copies + " if has_cow else "") + "store 1 token/seq (quantize+scatter) + decode"
-                 + (", one fused launch (pkv_decode_step)" if fused else ", separate launches"))
+                 + (", one fused launch (pkv_decode_step)" if fused else ", separate launches")
+                 + (", decode walks each forked child right after its parent (pkv_paged_attention_decode_ex)"
+                    if g.seq_order is not None and not fused else ""))
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": total_s * 1e3 / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,

@@ -97,7 +97,8 @@ enum {
   PKV_DEVERR_SLOT = 2,         /* slot_mapping entry beyond num_blocks * block_size */
   PKV_DEVERR_SLOT_GROUP = 3,   /* tokens bound for one block are not consecutive offsets */
   PKV_DEVERR_CONTEXT_LEN = 4,  /* context_len < 0, > max_context_len or > max_blocks*block_size */
-  PKV_DEVERR_TIMEOUT = 5       /* a bounded wait on an asynchronous copy gave up */
+  PKV_DEVERR_TIMEOUT = 5,      /* a bounded wait on an asynchronous copy gave up */
+  PKV_DEVERR_SEQ_ORDER = 6     /* a walk-order entry outside [0, num_seqs) */
 };
 
 /* Describes one layer's cache pool. Pointers are device pointers, 16-byte aligned. */
@@ -222,6 +223,32 @@ PKV_API pkv_status pkv_paged_attention_decode(const pkv_cache_desc* desc, void* 
                                       float softmax_scale, int32_t partition_tokens,
                                       void* workspace, size_t workspace_bytes, int32_t* dev_error,
                                       pkv_stream_t stream);
+
+/*
+ * pkv_paged_attention_decode_ex -- pkv_paged_attention_decode with options; the same arguments,
+ * results, workspace and ordering rules, plus:
+ *   seq_order  device int32 [num_seqs] or NULL: the order in which the decode walks the
+ *              sequences (a permutation of 0 .. num_seqs-1; results do not depend on it). A caller
+ *              that knows which sequences share physical blocks (beam candidates forked from one
+ *              parent, [deepinsea] "Copy-on-Write 机制"; requests on a common prefix, [yunthe]
+ *              "PagedAttention分页注意力机制与vLLM实现") lists them next to each other, so that the
+ *              shared blocks are read from memory once and found in L2 by the neighbours. An entry
+ *              outside [0, num_seqs) leaves that position empty and sets PKV_DEVERR_SEQ_ORDER; a
+ *              repeated entry makes the outputs of the repeated sequence unspecified.
+ * options may be NULL (plain decode). struct_bytes must be sizeof(pkv_decode_options) as the
+ * caller compiled it (fields this library does not know are refused with PKV_ERR_UNSUPPORTED).
+ */
+typedef struct pkv_decode_options {
+  size_t struct_bytes;
+  const int32_t* seq_order;
+} pkv_decode_options;
+PKV_API pkv_status pkv_paged_attention_decode_ex(const pkv_cache_desc* desc, void* out, const void* q,
+                                                 int32_t num_seqs, int32_t num_q_heads,
+                                                 const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                                 const int32_t* context_lens, int32_t max_context_len,
+                                                 float softmax_scale, int32_t partition_tokens,
+                                                 const pkv_decode_options* options, void* workspace,
+                                                 size_t workspace_bytes, int32_t* dev_error, pkv_stream_t stream);
 
 /*
  * pkv_decode_step -- one decode step in a single kernel launch: exactly

@@ -173,6 +173,7 @@ pkv_status make_decode_params(const pkv_cache_desc* desc, const DecodeGeometry& 
   p.out = static_cast<__half*>(out);
   p.block_tables = block_tables;
   p.context_lens = context_lens;
+  p.seq_order = nullptr;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   p.ws_count = reinterpret_cast<uint32_t*>(ws);
   p.ws_ml = reinterpret_cast<float*>(ws + g.counter_bytes);
@@ -309,6 +310,34 @@ pkv_status pkv_paged_attention_decode(const pkv_cache_desc* desc, void* out, con
   st = make_decode_params(desc, g, out, q, num_seqs, num_q_heads, block_tables, max_blocks_per_seq, context_lens,
                           max_context_len, softmax_scale, workspace, workspace_bytes, dev_error, &p);
   if (st != PKV_OK) return st;
+  return launch_decode(p, g.shape, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+pkv_status pkv_paged_attention_decode_ex(const pkv_cache_desc* desc, void* out, const void* q, int32_t num_seqs,
+                                         int32_t num_q_heads, const int32_t* block_tables,
+                                         int32_t max_blocks_per_seq, const int32_t* context_lens,
+                                         int32_t max_context_len, float softmax_scale, int32_t partition_tokens,
+                                         const pkv_decode_options* options, void* workspace, size_t workspace_bytes,
+                                         int32_t* dev_error, pkv_stream_t stream) {
+  if (options != nullptr && options->struct_bytes != sizeof(pkv_decode_options)) {
+    if (options->struct_bytes < sizeof(size_t)) return PKV_ERR_INVALID_ARG;
+    return PKV_ERR_UNSUPPORTED;
+  }
+  pkv_status st = check_desc(desc);
+  if (st != PKV_OK) return st;
+  if (!decode_supported(desc->k_dtype, desc->v_dtype, desc->block_size, desc->head_dim)) return PKV_ERR_UNSUPPORTED;
+  DecodeGeometry g;
+  st = decode_geometry(desc, num_seqs, num_q_heads, max_context_len, partition_tokens, &g);
+  if (st != PKV_OK) return st;
+  if (num_seqs == 0) return PKV_OK;
+  DecodeParams p;
+  st = make_decode_params(desc, g, out, q, num_seqs, num_q_heads, block_tables, max_blocks_per_seq, context_lens,
+                          max_context_len, softmax_scale, workspace, workspace_bytes, dev_error, &p);
+  if (st != PKV_OK) return st;
+  if (options != nullptr && options->seq_order != nullptr) {
+    if (!aligned(options->seq_order, 4)) return PKV_ERR_INVALID_ARG;
+    p.seq_order = options->seq_order;
+  }
   return launch_decode(p, g.shape, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 

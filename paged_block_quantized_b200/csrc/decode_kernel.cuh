@@ -145,7 +145,8 @@ __device__ __forceinline__ int owner_of(long long g, long long T, int W) {
 // A window: up to 32 consecutive blocks of one unit (warp-uniform description; lane k holds
 // block j0 + k in the per-lane registers of the window).
 struct Win {
-  int s, hg, j0, n;     // sequence, head group, first block, blocks in the window (0 = none)
+  int s, hg, j0, n;     // walk position of the sequence, head group, first block, blocks in the window (0 = none)
+  int sa;               // the sequence itself (its index in q, out, tables): seq_order[s], or s
   int g;                // KV head of the head group
   int L, nblk;          // clamped length of the sequence and its block count
   int r0;               // position of block j0 relative to the warp's first position
@@ -852,6 +853,22 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
   const int w = blockIdx.x * C::NW + warp;
   const int HG = p.num_q_heads / GT;
   const int S = p.num_seqs;
+  // Sequences are walked in the caller's order when one is given (sequences that share blocks
+  // placed next to each other read them while they are still in L2); an entry outside [0, S)
+  // makes that walk position empty and is reported.
+  auto sid = [&](int k) -> int {
+    if (p.seq_order == nullptr) return k;
+    const int a = __ldg(p.seq_order + k);
+    if (a < 0 || a >= S) {
+      record_error(p.dev_error, PKV_DEVERR_SEQ_ORDER);
+      return -1;
+    }
+    return a;
+  };
+  auto len_at = [&](int k) -> int {  // clamped length of the sequence at walk position k < S
+    const int a = sid(k);
+    return a < 0 ? 0 : clamp_len(p, p.context_lens[a], BS);
+  };
 
   uint8_t* my_stages = smem + (size_t)warp * C::NS * C::STAGE;
   uint64_t* my_bars = reinterpret_cast<uint64_t*>(smem + C::SMEM_STAGES) + warp * C::NS;
@@ -883,7 +900,9 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
       L = clamp_len(p, raw, BS);
       if (raw != L && w == 0) record_error(p.dev_error, PKV_DEVERR_CONTEXT_LEN);
     }
-    int sum = (L + BS - 1) / BS;
+    // the stream counts the sequences in walk order (the same as index order without one)
+    const int Lw = p.seq_order == nullptr ? L : (s < S ? len_at(s) : 0);
+    int sum = (Lw + BS - 1) / BS;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(kFull, sum, off);
     T += sum;
@@ -919,9 +938,12 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
   int Lchunk = 0, chunk_base = 0;  // lane holds the clamped length of sequence chunk_base + lane
   {
     long long acc0 = 0;
-    for (int base = 0;; base += 32) {
+    cur.s = cur.sa = 0;
+    cur.L = cur.nblk = 1;
+    cur.seq_p0 = 0;
+    for (int base = 0; base < S; base += 32) {  // found before base reaches S: start < T
       const int s = base + lane;
-      const int L = s < S ? clamp_len(p, p.context_lens[s], BS) : 0;
+      const int L = s < S ? len_at(s) : 0;
       const long long cnt = (long long)((L + BS - 1) / BS) * HG;
       long long incl = cnt;
 #pragma unroll
@@ -934,6 +956,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
         const uint32_t m = __ballot_sync(kFull, acc0 + incl > start);
         const int f = __ffs(m) - 1;
         cur.s = base + f;
+        cur.sa = p.seq_order == nullptr ? cur.s : __ldg(p.seq_order + cur.s);  // valid: it has blocks
         cur.L = __shfl_sync(kFull, L, f);
         cur.nblk = (cur.L + BS - 1) / BS;
         cur.seq_p0 = acc0 + __shfl_sync(kFull, incl - cnt, f);
@@ -956,7 +979,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
   auto seq_len = [&](int s) -> int {
     if (s < chunk_base || s >= chunk_base + 32) {
       chunk_base = s;
-      Lchunk = (s + lane < S) ? clamp_len(p, p.context_lens[s + lane], BS) : 0;
+      Lchunk = (s + lane < S) ? len_at(s + lane) : 0;
     }
     return __shfl_sync(kFull, Lchunk, s - chunk_base);
   };
@@ -980,6 +1003,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
           L = s < S ? seq_len(s) : 0;
         } while (L == 0 && s < S);
         b.s = s;
+        b.sa = (s < S && p.seq_order != nullptr) ? __ldg(p.seq_order + s) : s;  // valid when L > 0
         b.L = L;
         b.nblk = (L + BS - 1) / BS;
       }
@@ -993,7 +1017,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
   auto load_ids = [&](const Win& a, WinLanes& r) {
     r.meta = false;
     r.raw = -1;
-    if (lane < a.n) r.raw = p.block_tables[(size_t)a.s * p.max_blocks_per_seq + a.j0 + lane];
+    if (lane < a.n) r.raw = p.block_tables[(size_t)a.sa * p.max_blocks_per_seq + a.j0 + lane];
   };
   auto load_meta = [&](const Win& a, WinLanes& r) {
     r.valid = lane < a.n && r.raw >= 0 && r.raw < p.num_blocks;
@@ -1009,12 +1033,12 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
     r.meta = true;
   };
 
-  prefetch_q<GT, D>(p, cur.s, cur.hg, lane);
+  prefetch_q<GT, D>(p, cur.sa, cur.hg, lane);
   WinLanes rc, rn;
   load_ids(cur, rc);
   Win nxt = next_win(cur);
   load_ids(nxt, rn);
-  if (nxt.n > 0 && (nxt.s != cur.s || nxt.hg != cur.hg)) prefetch_q<GT, D>(p, nxt.s, nxt.hg, lane);
+  if (nxt.n > 0 && (nxt.s != cur.s || nxt.hg != cur.hg)) prefetch_q<GT, D>(p, nxt.sa, nxt.hg, lane);
   // Everything above reads only what the host wrote before the preceding kernel (lengths,
   // tables). From here on the pool is read, which the preceding kernel (the store of the new
   // tokens) may still be writing: wait for it to complete (no-op without a programmatic launch).
@@ -1111,7 +1135,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
   // ---- per-unit state: the arithmetic engine for GT query heads ----
   EngineFor<KT, VT, BS, D, GT> eng;
   int seg_j0 = cur.j0;  // first block of the current segment within its unit
-  eng.begin(p, cur.s, cur.hg, lane);
+  eng.begin(p, cur.sa, cur.hg, lane);
 
   bool aborted = false;
   while (cpos < n_total) {
@@ -1122,9 +1146,9 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
       if (!rc.meta) load_meta(cur, rc);
       nxt = next_win(cur);
       load_ids(nxt, rn);
-      if (nxt.n > 0 && (nxt.s != cur.s || nxt.hg != cur.hg)) prefetch_q<GT, D>(p, nxt.s, nxt.hg, lane);
+      if (nxt.n > 0 && (nxt.s != cur.s || nxt.hg != cur.hg)) prefetch_q<GT, D>(p, nxt.sa, nxt.hg, lane);
       if (new_unit) {
-        eng.begin(p, cur.s, cur.hg, lane);
+        eng.begin(p, cur.sa, cur.hg, lane);
         seg_j0 = cur.j0;
       }
     }
@@ -1160,7 +1184,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
       eng.finish();
       const long long u = (long long)cur.s * HG + cur.hg;
       if (seg_j0 == 0 && j_end == cur.nblk) {
-        eng.write_out(p, cur.s, cur.hg);  // the whole unit was processed by this warp
+        eng.write_out(p, cur.sa, cur.hg);  // the whole unit was processed by this warp
       } else {
         // one segment of a split unit: publish the partial; the last warp to finish merges
         eng.write_partial(p, u + w, lane);
@@ -1175,7 +1199,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
         pend_nseg = n_seg;
         pend_u = u;
         pend_slot0 = u + w_first;
-        pend_s = cur.s;
+        pend_s = cur.sa;
         pend_hg = cur.hg;
         if constexpr (!kDeferTicket) resolve_pending();
       }

@@ -21,6 +21,7 @@ struct DecodeParams {
   __half* out;
   const int32_t* block_tables;
   const int32_t* context_lens;
+  const int32_t* seq_order;  // [S] walk order of the sequences, or NULL (index order)
   uint32_t* ws_count;  // [S * HG] tickets of split units (zero between calls)
   float* ws_ml;        // [(S*HG + W) * GT][2] partial running max (log2 domain) and sum
   float* ws_acc;       // [(S*HG + W) * GT][D] partial un-normalised accumulators

@@ -24,12 +24,12 @@ _lib = ctypes.CDLL(LIB_PATH)
 PKV_OK, PKV_ERR_INVALID_ARG, PKV_ERR_UNSUPPORTED, PKV_ERR_OUT_OF_BLOCKS, PKV_ERR_CUDA, PKV_ERR_DEVICE_TIMEOUT = range(6)
 PKV_FP16, PKV_INT8_SYM, PKV_INT4_ASYM, PKV_FP8_E4M3 = 0, 1, 2, 3
 (PKV_DEVERR_NONE, PKV_DEVERR_BLOCK_ID, PKV_DEVERR_SLOT, PKV_DEVERR_SLOT_GROUP, PKV_DEVERR_CONTEXT_LEN,
- PKV_DEVERR_TIMEOUT) = range(6)
+ PKV_DEVERR_TIMEOUT, PKV_DEVERR_SEQ_ORDER) = range(7)
 
 EXPORTED = (
     "pkv_status_string", "pkv_tile_bytes", "pkv_store_quantized", "pkv_decode_workspace_size",
     "pkv_decode_partitioning", "pkv_paged_attention_decode_static", "pkv_static_scratch_address",
-    "pkv_paged_attention_decode", "pkv_copy_blocks", "pkv_swap_blocks", "pkv_decode_step", "pkv_blocks_for_tokens", "pkv_alloc_create",
+    "pkv_paged_attention_decode", "pkv_paged_attention_decode_ex", "pkv_copy_blocks", "pkv_swap_blocks", "pkv_decode_step", "pkv_blocks_for_tokens", "pkv_alloc_create",
     "pkv_alloc_destroy", "pkv_alloc_num_free", "pkv_alloc_refcount", "pkv_alloc_blocks", "pkv_alloc_fork",
     "pkv_alloc_release", "pkv_alloc_cow", "pkv_prefix_cache_create", "pkv_prefix_cache_destroy",
     "pkv_prefix_cache_size", "pkv_prefix_cache_evictable", "pkv_prefix_match", "pkv_prefix_insert",
@@ -74,6 +74,14 @@ _partitioning = _sig("pkv_decode_partitioning", ctypes.c_int, _DESC, _I32, _I32,
                      ctypes.POINTER(_I32), ctypes.POINTER(_I32))
 _decode = _sig("pkv_paged_attention_decode", ctypes.c_int, _DESC, _P, _P, _I32, _I32, _P, _I32, _P, _I32,
                ctypes.c_float, _I32, _P, ctypes.c_size_t, _P, _P)
+
+
+class pkv_decode_options(ctypes.Structure):
+    _fields_ = [("struct_bytes", ctypes.c_size_t), ("seq_order", ctypes.c_void_p)]
+
+
+_decode_ex = _sig("pkv_paged_attention_decode_ex", ctypes.c_int, _DESC, _P, _P, _I32, _I32, _P, _I32, _P, _I32,
+                  ctypes.c_float, _I32, ctypes.POINTER(pkv_decode_options), _P, ctypes.c_size_t, _P, _P)
 _decode_static = _sig("pkv_paged_attention_decode_static", ctypes.c_int, _DESC, _P, _P, _I32, _I32, _P, _I32, _P,
                       _I32, ctypes.c_float, _I32, _P, _P)
 PKV_STATIC_SCRATCH_BYTES = 8 << 20
@@ -174,6 +182,19 @@ def pkv_paged_attention_decode(desc, out, q, num_seqs, num_q_heads, block_tables
                  int(max_blocks_per_seq), _ptr(context_lens), int(max_context_len), float(softmax_scale),
                  int(partition_tokens), _ptr(workspace), int(workspace_bytes), _ptr(dev_error), _stream(stream))
     return _check(st, "pkv_paged_attention_decode", raise_on_error)
+
+
+def pkv_paged_attention_decode_ex(desc, out, q, num_seqs, num_q_heads, block_tables, max_blocks_per_seq,
+                                  context_lens, max_context_len, softmax_scale, partition_tokens=0, seq_order=None,
+                                  workspace=None, workspace_bytes=0, dev_error=None, stream=None,
+                                  raise_on_error=True):
+    """Decode with options: seq_order (device int32 [num_seqs]) = the walk order of the sequences."""
+    opts = pkv_decode_options(ctypes.sizeof(pkv_decode_options), _ptr(seq_order))
+    st = _decode_ex(ctypes.byref(desc), _ptr(out), _ptr(q), int(num_seqs), int(num_q_heads), _ptr(block_tables),
+                    int(max_blocks_per_seq), _ptr(context_lens), int(max_context_len), float(softmax_scale),
+                    int(partition_tokens), ctypes.byref(opts), _ptr(workspace), int(workspace_bytes),
+                    _ptr(dev_error), _stream(stream))
+    return _check(st, "pkv_paged_attention_decode_ex", raise_on_error)
 
 
 def pkv_paged_attention_decode_static(desc, out, q, num_seqs, num_q_heads, block_tables, max_blocks_per_seq,

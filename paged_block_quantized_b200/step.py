@@ -27,7 +27,8 @@ _TORCH_DTYPE = {np.dtype(np.float16): torch.float16, np.dtype(np.int32): torch.i
 
 
 class DeviceStep:
-    def __init__(self, w: Workload, device="cuda", poison: int | None = 0xA5, partition_tokens: int | None = None):
+    def __init__(self, w: Workload, device="cuda", poison: int | None = 0xA5, partition_tokens: int | None = None,
+                 beam_order: bool = False):
         self.w = w
         self.device = torch.device(device)
         self.pool = pkv.DevicePool.allocate(w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim, w.k_dtype,
@@ -39,6 +40,10 @@ class DeviceStep:
         k_new, v_new = w.new_token_values()
         inputs = [("q", w.queries()), ("k_new", k_new), ("v_new", v_new), ("step_slots", w.step_slots()),
                   ("block_tables", w.block_tables), ("context_lens", w.context_lens), ("cow", w.cow_pairs)]
+        # with beam_order, the decode walks forked children right after their parents
+        use_order = beam_order and w.cow_pairs.shape[0] > 0
+        if use_order:
+            inputs.append(("seq_order", w.beam_walk_order()))
         offs, total = [], 0
         for _, a in inputs:
             offs.append(total)
@@ -52,6 +57,8 @@ class DeviceStep:
             t = self.inbuf[o:o + a.nbytes].view(_TORCH_DTYPE[np.dtype(a.dtype)]).view(a.shape)
             setattr(self, name, t)
         self.out = torch.zeros_like(self.q)
+        if not use_order:
+            self.seq_order = None
         self.partition_tokens = w.partition_tokens if partition_tokens is None else partition_tokens
         self.num_workers, self.num_ctas = pkv.pkv_decode_partitioning(
             self.pool.desc, w.num_seqs, w.num_q_heads, w.max_context_len, self.partition_tokens)
@@ -123,6 +130,13 @@ class DeviceStep:
 
     def decode(self, stream=None, out=None, q=None):
         w = self.w
+        if self.seq_order is not None:
+            pkv.pkv_paged_attention_decode_ex(
+                self.pool.desc, self.out if out is None else out, self.q if q is None else q, w.num_seqs,
+                w.num_q_heads, self.block_tables, w.max_blocks_per_seq, self.context_lens, w.max_context_len,
+                w.softmax_scale, self.partition_tokens, self.seq_order, self.workspace, self.ws_bytes,
+                self.dev_error, stream=stream)
+            return
         pkv.pkv_paged_attention_decode(
             self.pool.desc, self.out if out is None else out, self.q if q is None else q, w.num_seqs,
             w.num_q_heads, self.block_tables, w.max_blocks_per_seq, self.context_lens, w.max_context_len,

@@ -171,6 +171,27 @@ class Workload:
         return np.array([self.slots(self.block_tables, s, [int(self.context_lens[s]) - 1])[0]
                          for s in range(self.num_seqs)], dtype=np.int64)
 
+    def beam_walk_order(self) -> np.ndarray:
+        """int32 [S]: the sequence indices in order, except that every beam child forked from a
+        parent (a copy-on-write pair) comes right after that parent, so that the blocks they share
+        are walked back to back."""
+        S = self.num_seqs
+        kids = {}
+        child_set = set()
+        for src, dst in self.cow_pairs:
+            c = int(np.nonzero((self.block_tables == dst).any(axis=1))[0][0])
+            par = int(np.nonzero((self.block_tables == src).any(axis=1))[0][0])
+            kids.setdefault(par, []).append(c)
+            child_set.add(c)
+        order = []
+        for s in range(S):
+            if s in child_set:
+                continue
+            order.append(s)
+            order.extend(kids.get(s, []))
+        assert sorted(order) == list(range(S))
+        return np.array(order, np.int32)
+
     # ---- bytes read by one decode (the algorithmic minimum) ----
     def decode_bytes(self, unique: bool = True) -> int:
         """Algorithmic bytes one decode reads: K/V codes of valid tokens, per-block scales and

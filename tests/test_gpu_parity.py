@@ -352,3 +352,31 @@ def test_copy_blocks_bit_exact_and_bad_ids():
     torch.cuda.synchronize()
     assert g.error() == pkv.PKV_DEVERR_BLOCK_ID
     np.testing.assert_array_equal(g.pool_numpy()[0], after[0])
+
+
+@pytest.mark.parametrize("name,over", [("mixed", dict(num_seqs=24, children=4)), ("mixed", {})])
+def test_beam_walk_order(name, over):
+    """pkv_paged_attention_decode_ex with a walk order that puts every forked child right after its
+    parent gives the oracle's outputs (reduced and full size), and an order entry outside the batch
+    is skipped and flagged, never a fault or a hang."""
+    from paged_block_quantized_b200 import pkv
+    from paged_block_quantized_b200.step import DeviceStep
+    w = W.make(name, seed=0, **over)
+    g = DeviceStep(w, beam_order=True)
+    assert g.seq_order is not None
+    g.prefill()
+    g.step()
+    torch.cuda.synchronize()
+    assert g.error() == 0
+    seqs = None if over else [int(s) for s in g.seq_order[:6].cpu()] + [int(np.argmax(w.context_lens))]
+    o = oracle_step(w, seqs)
+    out = g.out.float().cpu().numpy()[o["seqs"]]
+    assert np.abs(out - o["out"]).max() <= TOL
+    bad = g.seq_order.clone()
+    bad[1] = w.num_seqs + 3
+    g.dev_error.zero_()
+    pkv.pkv_paged_attention_decode_ex(g.pool.desc, g.out, g.q, w.num_seqs, w.num_q_heads, g.block_tables,
+                                      w.max_blocks_per_seq, g.context_lens, w.max_context_len, w.softmax_scale, 0,
+                                      bad, g.workspace, g.ws_bytes, g.dev_error)
+    torch.cuda.synchronize()
+    assert g.error() == pkv.PKV_DEVERR_SEQ_ORDER
