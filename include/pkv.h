@@ -251,6 +251,33 @@ PKV_API pkv_status pkv_paged_attention_decode_ex(const pkv_cache_desc* desc, voi
                                                  size_t workspace_bytes, int32_t* dev_error, pkv_stream_t stream);
 
 /*
+ * pkv_paged_attention_prefill -- chunked prefill: causal attention of each sequence's new tokens
+ * over the paged, quantized cache, after pkv_store_quantized has stored their K/V
+ * ([yunthe] section "Prefix Caching与多轮对话场景优化实践": with the prefix cached, only the new
+ * tokens are computed; [tbr8] §5 item 2: dequantization inside the attention operator).
+ *
+ * Sequence s has q_len = cu_q_lens[s+1] - cu_q_lens[s] query rows q[cu_q_lens[s] + i], the last
+ * q_len of its context_lens[s] tokens; the query at position p = context_lens[s] - q_len + i
+ * attends to tokens 0 .. p (k_hat, v_hat and the logit scale as in pkv_paged_attention_decode):
+ *   out[row][h] = sum_{t <= p} softmax_t(softmax_scale * q[row][h] . k_hat_t) * v_hat_t   (fp16)
+ *   q, out        device fp16 [total_q][num_q_heads][head_dim]
+ *   cu_q_lens     device int32 [num_seqs + 1], non-decreasing, cu_q_lens[0] = 0,
+ *                 cu_q_lens[num_seqs] = total_q; every q_len <= max_q_len (host bound: grid size)
+ *   context_lens  device int32 [num_seqs]; q_len <= context_len <= min(max_context_len,
+ *                 max_blocks_per_seq * block_size), else PKV_DEVERR_CONTEXT_LEN (rows of a chunk
+ *                 longer than its context are zeroed; a longer context is clamped)
+ * Built for INT8 K with INT8 or INT4 V, head_dim 128, block size 16 or 32 (else
+ * PKV_ERR_UNSUPPORTED). q.k runs on the integer tensor cores with q split into exact byte planes;
+ * p.v on the fp16 tensor cores, each V code converted once per 128 query columns. No workspace.
+ */
+PKV_API pkv_status pkv_paged_attention_prefill(const pkv_cache_desc* desc, void* out, const void* q,
+                                               int32_t num_seqs, int32_t num_q_heads, const int32_t* cu_q_lens,
+                                               int32_t total_q, int32_t max_q_len, const int32_t* block_tables,
+                                               int32_t max_blocks_per_seq, const int32_t* context_lens,
+                                               int32_t max_context_len, float softmax_scale, int32_t* dev_error,
+                                               pkv_stream_t stream);
+
+/*
  * pkv_decode_step -- one decode step in a single kernel launch: exactly
  *   pkv_copy_blocks(desc, block_mapping, n_pairs, ...); then
  *   pkv_store_quantized(desc, k_new, v_new, slot_mapping, T, ...); then

@@ -341,6 +341,56 @@ pkv_status pkv_paged_attention_decode_ex(const pkv_cache_desc* desc, void* out, 
   return launch_decode(p, g.shape, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
+pkv_status pkv_paged_attention_prefill(const pkv_cache_desc* desc, void* out, const void* q, int32_t num_seqs,
+                                       int32_t num_q_heads, const int32_t* cu_q_lens, int32_t total_q,
+                                       int32_t max_q_len, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                       const int32_t* context_lens, int32_t max_context_len, float softmax_scale,
+                                       int32_t* dev_error, pkv_stream_t stream) {
+  pkv_status st = check_desc(desc);
+  if (st != PKV_OK) return st;
+  if (num_seqs < 0 || num_q_heads <= 0 || total_q < 0 || max_q_len < 0 || max_context_len < 0)
+    return PKV_ERR_INVALID_ARG;
+  if (num_q_heads % desc->num_kv_heads != 0) return PKV_ERR_INVALID_ARG;
+  if (!prefill_supported(desc->k_dtype, desc->v_dtype, desc->block_size, desc->head_dim)) return PKV_ERR_UNSUPPORTED;
+  if (num_seqs == 0 || total_q == 0 || max_q_len == 0) return PKV_OK;
+  if (out == nullptr || q == nullptr || cu_q_lens == nullptr || block_tables == nullptr || context_lens == nullptr)
+    return PKV_ERR_INVALID_ARG;
+  if (!aligned(out, 16) || !aligned(q, 16) || !aligned(cu_q_lens, 4) || !aligned(block_tables, 4) ||
+      !aligned(context_lens, 4))
+    return PKV_ERR_INVALID_ARG;
+  if (max_blocks_per_seq <= 0) return PKV_ERR_INVALID_ARG;
+  if (dev_error != nullptr && !aligned(dev_error, 4)) return PKV_ERR_INVALID_ARG;
+  if (!(softmax_scale == softmax_scale)) return PKV_ERR_INVALID_ARG;
+  const int32_t group = num_q_heads / desc->num_kv_heads;
+  const int64_t chunks = ((int64_t)max_q_len * group + 127) / 128;
+  if (num_seqs > 65535 || desc->num_kv_heads > 65535 || chunks > INT32_MAX) return PKV_ERR_UNSUPPORTED;
+  PrefillParams p;
+  p.k_codes = desc->k_codes;
+  p.v_codes = desc->v_codes;
+  p.k_scale = desc->k_scale;
+  p.v_scale = desc->v_scale;
+  p.v_zp = desc->v_zp;
+  p.q = static_cast<const __half*>(q);
+  p.out = static_cast<__half*>(out);
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  p.cu_q_lens = cu_q_lens;
+  p.dev_error = dev_error;
+  p.num_seqs = num_seqs;
+  p.num_blocks = desc->num_blocks;
+  p.num_kv_heads = desc->num_kv_heads;
+  p.num_q_heads = num_q_heads;
+  p.group = group;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.max_context_len = max_context_len;
+  p.max_q_len = max_q_len;
+  p.total_q = total_q;
+  p.block_size = desc->block_size;
+  p.v_dtype = desc->v_dtype;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;  // log2(e)
+  return launch_prefill(p, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
 pkv_status pkv_copy_blocks(const pkv_cache_desc* desc, const int32_t* block_mapping, int32_t n_pairs,
                            int32_t* dev_error, pkv_stream_t stream) {
   pkv_status st = check_desc(desc);

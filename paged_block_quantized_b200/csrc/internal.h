@@ -130,6 +130,35 @@ struct SwapParams {
 };
 cudaError_t launch_swap(const SwapParams& p, cudaStream_t stream);
 
+// ---------------------------------------------------------------- chunked prefill
+struct PrefillParams {
+  const void* k_codes;
+  const void* v_codes;
+  const float* k_scale;
+  const float* v_scale;
+  const uint8_t* v_zp;
+  const __half* q;
+  __half* out;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  const int32_t* cu_q_lens;  // [S+1] rows of each sequence's chunk in q / out
+  int32_t* dev_error;
+  int32_t num_seqs;
+  int32_t num_blocks;
+  int32_t num_kv_heads;
+  int32_t num_q_heads;
+  int32_t group;
+  int32_t max_blocks_per_seq;
+  int32_t max_context_len;
+  int32_t max_q_len;
+  int32_t total_q;
+  int32_t block_size;
+  int32_t v_dtype;
+  float scale_log2;
+};
+bool prefill_supported(int32_t k_dtype, int32_t v_dtype, int32_t block_size, int32_t head_dim);
+cudaError_t launch_prefill(const PrefillParams& p, cudaStream_t stream);
+
 // ---------------------------------------------------------------- fused step
 // Copy-on-write copies, then the store, then the decode, in one cooperative launch of the decode
 // kernel: every warp takes part in the copies and the stores, with a grid-wide barrier after each

@@ -1,0 +1,55 @@
+// prefill.cu -- launch of the chunked-prefill kernel (prefill_kernel.cuh): one CTA per 128 query
+// columns of one (sequence, KV head), INT8 K with INT8 or INT4 V, head_dim 128, block size 16 or 32.
+#include <cstring>
+
+#include "prefill_kernel.cuh"
+
+namespace pkv {
+
+bool prefill_supported(int32_t k_dtype, int32_t v_dtype, int32_t block_size, int32_t head_dim) {
+  return k_dtype == PKV_INT8_SYM && (v_dtype == PKV_INT8_SYM || v_dtype == PKV_INT4_ASYM) &&
+         (block_size == 16 || block_size == 32) && head_dim == 128;
+}
+
+namespace {
+
+template <int VT, int BS>
+cudaError_t launch_prefill_t(const PrefillParams& p, cudaStream_t stream) {
+  using C = prefill_detail::Cfg<VT, BS>;
+  auto kern = prefill_detail::paged_prefill_kernel<VT, BS>;
+  static unsigned long long configured = 0;  // one bit per device; benign race
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (!(configured & (1ull << (dev & 63)))) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    configured |= 1ull << (dev & 63);
+  }
+  TileMaps tm;
+  memset(&tm, 0, sizeof(tm));
+  const uint64_t rows = (uint64_t)p.num_blocks * p.num_kv_heads * BS;
+  if (!encode_tile_map(&tm.k, p.k_codes, rows, C::K_ROW, BS)) return cudaErrorInvalidValue;
+  if constexpr (C::V_SWZ) {
+    if (!encode_tile_map(&tm.v, p.v_codes, rows, C::V_ROW, BS)) return cudaErrorInvalidValue;
+  }
+  const int chunks = (p.max_q_len * p.group + prefill_detail::kCols - 1) / prefill_detail::kCols;
+  dim3 grid(chunks, p.num_kv_heads, p.num_seqs);
+  kern<<<grid, prefill_detail::kThreads, C::SMEM, stream>>>(p, tm);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prefill(const PrefillParams& p, cudaStream_t stream) {
+  if (p.v_dtype == PKV_INT8_SYM) {
+    if (p.block_size == 16) return launch_prefill_t<PKV_INT8_SYM, 16>(p, stream);
+    if (p.block_size == 32) return launch_prefill_t<PKV_INT8_SYM, 32>(p, stream);
+  } else if (p.v_dtype == PKV_INT4_ASYM) {
+    if (p.block_size == 16) return launch_prefill_t<PKV_INT4_ASYM, 16>(p, stream);
+    if (p.block_size == 32) return launch_prefill_t<PKV_INT4_ASYM, 32>(p, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace pkv

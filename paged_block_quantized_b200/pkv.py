@@ -29,7 +29,8 @@ PKV_FP16, PKV_INT8_SYM, PKV_INT4_ASYM, PKV_FP8_E4M3 = 0, 1, 2, 3
 EXPORTED = (
     "pkv_status_string", "pkv_tile_bytes", "pkv_store_quantized", "pkv_decode_workspace_size",
     "pkv_decode_partitioning", "pkv_paged_attention_decode_static", "pkv_static_scratch_address",
-    "pkv_paged_attention_decode", "pkv_paged_attention_decode_ex", "pkv_copy_blocks", "pkv_swap_blocks", "pkv_decode_step", "pkv_blocks_for_tokens", "pkv_alloc_create",
+    "pkv_paged_attention_decode", "pkv_paged_attention_decode_ex", "pkv_paged_attention_prefill",
+    "pkv_copy_blocks", "pkv_swap_blocks", "pkv_decode_step", "pkv_blocks_for_tokens", "pkv_alloc_create",
     "pkv_alloc_destroy", "pkv_alloc_num_free", "pkv_alloc_refcount", "pkv_alloc_blocks", "pkv_alloc_fork",
     "pkv_alloc_release", "pkv_alloc_cow", "pkv_prefix_cache_create", "pkv_prefix_cache_destroy",
     "pkv_prefix_cache_size", "pkv_prefix_cache_evictable", "pkv_prefix_match", "pkv_prefix_insert",
@@ -82,6 +83,8 @@ class pkv_decode_options(ctypes.Structure):
 
 _decode_ex = _sig("pkv_paged_attention_decode_ex", ctypes.c_int, _DESC, _P, _P, _I32, _I32, _P, _I32, _P, _I32,
                   ctypes.c_float, _I32, ctypes.POINTER(pkv_decode_options), _P, ctypes.c_size_t, _P, _P)
+_prefill = _sig("pkv_paged_attention_prefill", ctypes.c_int, _DESC, _P, _P, _I32, _I32, _P, _I32, _I32, _P, _I32, _P,
+                _I32, ctypes.c_float, _P, _P)
 _decode_static = _sig("pkv_paged_attention_decode_static", ctypes.c_int, _DESC, _P, _P, _I32, _I32, _P, _I32, _P,
                       _I32, ctypes.c_float, _I32, _P, _P)
 PKV_STATIC_SCRATCH_BYTES = 8 << 20
@@ -195,6 +198,17 @@ def pkv_paged_attention_decode_ex(desc, out, q, num_seqs, num_q_heads, block_tab
                     int(partition_tokens), ctypes.byref(opts), _ptr(workspace), int(workspace_bytes),
                     _ptr(dev_error), _stream(stream))
     return _check(st, "pkv_paged_attention_decode_ex", raise_on_error)
+
+
+def pkv_paged_attention_prefill(desc, out, q, num_seqs, num_q_heads, cu_q_lens, total_q, max_q_len, block_tables,
+                                max_blocks_per_seq, context_lens, max_context_len, softmax_scale, dev_error=None,
+                                stream=None, raise_on_error=True):
+    """Chunked prefill: causal attention of each sequence's last q_len tokens (rows of q given by
+    cu_q_lens) over the paged cache."""
+    st = _prefill(ctypes.byref(desc), _ptr(out), _ptr(q), int(num_seqs), int(num_q_heads), _ptr(cu_q_lens),
+                  int(total_q), int(max_q_len), _ptr(block_tables), int(max_blocks_per_seq), _ptr(context_lens),
+                  int(max_context_len), float(softmax_scale), _ptr(dev_error), _stream(stream))
+    return _check(st, "pkv_paged_attention_prefill", raise_on_error)
 
 
 def pkv_paged_attention_decode_static(desc, out, q, num_seqs, num_q_heads, block_tables, max_blocks_per_seq,

@@ -173,3 +173,55 @@ class DeviceStep:
             return a
         return (codes(p.k_codes, self.w.k_dtype), codes(p.v_codes, self.w.v_dtype), p.k_scale.cpu().numpy(),
                 p.v_scale.cpu().numpy(), p.v_zp.cpu().numpy())
+
+
+class PrefillStep:
+    """One chunked-prefill step of a workload with q_lens: store every sequence's chunk (its last
+    q_len positions) into the pool, then causal attention of the chunk's queries over the cache
+    (pkv_paged_attention_prefill). Before the step the pool holds positions [0, L - q_len)."""
+
+    def __init__(self, w: Workload, device="cuda", poison: int | None = 0xA5):
+        assert w.q_lens is not None
+        self.w = w
+        self.device = torch.device(device)
+        dev = self.device
+        self.pool = pkv.DevicePool.allocate(w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim, w.k_dtype,
+                                            w.v_dtype, device=dev, fill=poison)
+        self.dev_error = torch.zeros(1, dtype=torch.int32, device=dev)
+        k, v, slots = w.chunk_tokens()
+        self.k_new = torch.from_numpy(k).to(dev)
+        self.v_new = torch.from_numpy(v).to(dev)
+        self.slots = torch.from_numpy(slots).to(dev)
+        self.q = torch.from_numpy(w.chunk_queries()).to(dev)
+        self.out = torch.zeros_like(self.q)
+        self.cu = torch.from_numpy(w.cu_q_lens).to(dev)
+        self.context_lens = torch.from_numpy(w.context_lens).to(dev)
+        self.block_tables = torch.from_numpy(w.block_tables).to(dev)
+        self.total_q = int(w.q_lens.sum())
+        self.max_q_len = int(w.q_lens.max())
+
+    def prefill(self, max_tokens: int = 1 << 16):
+        for k, v, slots in self.w.prefill_batches(max_tokens):
+            pkv.pkv_store_quantized(self.pool.desc, torch.from_numpy(k).to(self.device),
+                                    torch.from_numpy(v).to(self.device), torch.from_numpy(slots).to(self.device),
+                                    slots.shape[0], self.dev_error)
+        torch.cuda.synchronize(self.device)
+
+    def store(self, stream=None):
+        pkv.pkv_store_quantized(self.pool.desc, self.k_new, self.v_new, self.slots, self.total_q, self.dev_error,
+                                stream=stream)
+
+    def attend(self, stream=None):
+        w = self.w
+        pkv.pkv_paged_attention_prefill(self.pool.desc, self.out, self.q, w.num_seqs, w.num_q_heads, self.cu,
+                                        self.total_q, self.max_q_len, self.block_tables, w.max_blocks_per_seq,
+                                        self.context_lens, w.max_context_len, w.softmax_scale, self.dev_error,
+                                        stream=stream)
+
+    def step(self, stream=None):
+        self.store(stream)
+        self.attend(stream)
+        return self.out
+
+    def error(self) -> int:
+        return int(self.dev_error.item())

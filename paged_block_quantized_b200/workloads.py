@@ -58,6 +58,7 @@ class Workload:
     prefill_owner: np.ndarray         # bool  [S][max_blocks]: this seq stores this block in prefill
     cow_pairs: np.ndarray             # int32 [n][2]: (src, dst) copies the step makes
     partition_tokens: int = 0         # 0 = let the library choose
+    q_lens: np.ndarray | None = None  # int32 [S]: chunked prefill, new tokens per sequence (None: decode)
     outliers: bool = False
     description: str = ""
     _mult: dict = field(default_factory=dict, repr=False)
@@ -150,7 +151,7 @@ class Workload:
         ks, vs, sl = [], [], []
         count = 0
         for s in range(self.num_seqs):
-            n_pre = int(self.context_lens[s]) - 1
+            n_pre = int(self.context_lens[s]) - (1 if self.q_lens is None else int(self.q_lens[s]))
             for j in range((n_pre + bs - 1) // bs):
                 if not self.prefill_owner[s, j]:
                     continue
@@ -165,6 +166,38 @@ class Workload:
                     ks, vs, sl, count = [], [], [], 0
         if ks:
             yield np.concatenate(ks), np.concatenate(vs), np.concatenate(sl)
+
+    # ---- chunked prefill: the new tokens of every sequence ----
+    @property
+    def cu_q_lens(self) -> np.ndarray:
+        return np.concatenate([[0], np.cumsum(self.q_lens)]).astype(np.int32)
+
+    def chunk_tokens(self):
+        """fp16 K, V [T][H][D] and slots [T] of every sequence's chunk (its last q_len positions),
+        sequences one after another: the values of those positions' blocks."""
+        ks, vs, sl = [], [], []
+        for s in range(self.num_seqs):
+            L, q = int(self.context_lens[s]), int(self.q_lens[s])
+            k, v = self.seq_values(s, L - q, L)
+            ks.append(k)
+            vs.append(v)
+            sl.append(self.slots(self.block_tables, s, np.arange(L - q, L)))
+        return np.concatenate(ks), np.concatenate(vs), np.concatenate(sl).astype(np.int64)
+
+    def chunk_queries(self) -> np.ndarray:
+        """fp16 q [T][Hq][D] of the chunks' tokens, N(0,1)."""
+        rng = np.random.default_rng([self.seed, _QUERY, 1])
+        T = int(self.q_lens.sum())
+        return rng.standard_normal((T, self.num_q_heads, self.head_dim), dtype=np.float32).astype(np.float16)
+
+    def prefill_flops(self) -> int:
+        """Multiply-adds x 2 of one chunked-prefill attention: q.k and p.v over every visible
+        (query, token) pair of every query head."""
+        pairs = 0
+        for s in range(self.num_seqs):
+            L, q = int(self.context_lens[s]), int(self.q_lens[s])
+            pairs += sum(L - q + i + 1 for i in range(q))
+        return int(4 * pairs * self.num_q_heads * self.head_dim)
 
     def step_slots(self) -> np.ndarray:
         """int64 [S]: slot of position L-1 of every sequence in its final (post-copy) table."""
@@ -333,6 +366,17 @@ def make(name: str, seed: int = 0, **over) -> Workload:
                  num_blocks=None, k_dtype=INT8_SYM, v_dtype=INT8_SYM, outliers=False,
                  partition_tokens=0, context_lens=np.full(S, (prefix_blocks + private) * bs))
         desc = "LLaMA-70B-shaped GQA: 64 seqs, 64 q / 8 KV heads, D 128, bs 16, 64 shared prefix blocks + 64 private, INT8/INT8"
+    elif name == "prefill":
+        S = over.get("num_seqs", 8)
+        bs = over.get("block_size", 16)
+        chunk = over.pop("chunk", 512)
+        prefix = np.asarray(over.pop("prefix_lens", rng.integers(0, 2049, size=S)))
+        p = dict(num_seqs=S, num_q_heads=32, num_kv_heads=32, head_dim=128, block_size=bs,
+                 num_blocks=None, k_dtype=INT8_SYM, v_dtype=INT8_SYM, outliers=False,
+                 partition_tokens=0, context_lens=prefix + chunk)
+        q_lens = np.full(S, chunk, np.int32)
+        desc = ("chunked prefill: 8 seqs, a 512-token chunk each over a cached prefix of U{0..2048} tokens, "
+                "32 heads MHA, D 128, bs 16, INT8/INT8")
     elif name == "mixed":
         S = over.get("num_seqs", 128)
         n_children = over.pop("children", 16)
@@ -351,6 +395,7 @@ def make(name: str, seed: int = 0, **over) -> Workload:
         desc = "mixed step: 128 seqs, lognormal L (median 1000, sigma 1) in [16,16384], 32 heads, D 128, bs 16, K INT8 / V INT4, 16 forked"
     else:
         raise KeyError(name)
+    q_lens = q_lens if name == "prefill" else None
     p.update(over)
     S = p["num_seqs"]
     cl = np.asarray(p["context_lens"], dtype=np.int32)
@@ -363,7 +408,8 @@ def make(name: str, seed: int = 0, **over) -> Workload:
         v_dtype=p["v_dtype"], softmax_scale=float(np.float32(1.0 / math.sqrt(p["head_dim"]))),
         context_lens=cl, block_tables=tables, block_streams=streams, prefill_tables=pre_tables,
         prefill_owner=owner, cow_pairs=cow, partition_tokens=p["partition_tokens"],
-        outliers=p["outliers"], description=desc)
+        outliers=p["outliers"], description=desc,
+        q_lens=None if q_lens is None else np.asarray(q_lens, np.int32)[:S])
 
 
 CONFIGS = ("tiny", "llama7b", "long", "gqa_prefix", "mixed")

@@ -65,3 +65,42 @@ def oracle_step(w, seqs=None, num_threads=None):
                                     max_context_len=w.max_context_len, num_threads=num_threads)
     return dict(seqs=seqs, out=out, cache=c, prefill_cache=pre, phys=phys, remap=remap, tables=tables, q=q,
                 errors=(err_prefill, err_copy, err_store, err_decode))
+
+
+def oracle_prefill_step(w, seqs=None, num_threads=None):
+    """The chunked-prefill step of a workload with q_lens on the oracle: the prefix positions
+    stored block by block, each chunk stored as one group per block, then oracle.prefill over the
+    chosen sequences' chunks. Returns the outputs of those sequences' rows."""
+    S, bs = w.num_seqs, w.block_size
+    seqs = list(range(S)) if seqs is None else sorted(set(int(s) for s in seqs))
+    used = sorted(set(int(b) for s in seqs for b in w.block_tables[s, :(int(w.context_lens[s]) + bs - 1) // bs]))
+    remap = {b: i for i, b in enumerate(used)}
+    c = oracle.OracleCache.empty(len(used), bs, w.num_kv_heads, w.head_dim, _odt(w.k_dtype), _odt(w.v_dtype))
+    errors = []
+    for s in seqs:
+        L, q = int(w.context_lens[s]), int(w.q_lens[s])
+        n_pre = L - q
+        for j in range((n_pre + bs - 1) // bs):
+            ntok = min(n_pre - j * bs, bs)
+            k, v = w.block_values(w.block_streams[s, j], j)
+            slots = remap[int(w.block_tables[s, j])] * bs + np.arange(ntok, dtype=np.int64)
+            errors.append(oracle.store(c, k[:ntok], v[:ntok], slots))
+    k_all, v_all, _ = w.chunk_tokens()
+    cu = w.cu_q_lens
+    q_all = w.chunk_queries()
+    rows, cu_sel = [], [0]
+    for s in seqs:
+        L, q = int(w.context_lens[s]), int(w.q_lens[s])
+        pos = np.arange(L - q, L)
+        slots = np.array([remap[int(w.block_tables[s, t // bs])] * bs + t % bs for t in pos], np.int64)
+        errors.append(oracle.store(c, k_all[cu[s]:cu[s + 1]], v_all[cu[s]:cu[s + 1]], slots))
+        rows.extend(range(cu[s], cu[s + 1]))
+        cu_sel.append(cu_sel[-1] + q)
+    tables = np.full((len(seqs), w.max_blocks_per_seq), -1, np.int32)
+    for i, s in enumerate(seqs):
+        nblk = (int(w.context_lens[s]) + bs - 1) // bs
+        tables[i, :nblk] = [remap[int(b)] for b in w.block_tables[s, :nblk]]
+    out, err = oracle.prefill(c, q_all[rows], np.array(cu_sel, np.int32), tables, w.context_lens[seqs],
+                              w.softmax_scale, num_threads=num_threads)
+    errors.append(err)
+    return dict(seqs=seqs, rows=np.array(rows), out=out, cache=c, phys=used, errors=errors)
