@@ -71,6 +71,9 @@ def parse_args():
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-beam-order", action="store_true",
                     help="walk the sequences in index order instead of each forked child right after its parent")
+    ap.add_argument("--shared-prefix", choices=("auto", "on", "off"), default="auto",
+                    help="attend blocks shared by a group of sequences once per group (auto: when a group has "
+                         "more than two members)")
     ap.add_argument("--fused", action="store_true",
                     help="time the step as one fused launch (pkv_decode_step) instead of copy, store, decode")
     return ap.parse_args()
@@ -297,8 +300,11 @@ def run_pkv(args, rank, world, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     w = W.make(args.config, seed=args.seed + rank)
+    groups = w.prefix_groups()
+    shared = args.shared_prefix == "on" or (
+        args.shared_prefix == "auto" and groups is not None and int(np.diff(groups[0]).max()) > 2)
     g = DeviceStep(w, device=dev, poison=None, partition_tokens=args.partition_tokens,
-                   beam_order=not args.no_beam_order)
+                   beam_order=not args.no_beam_order, shared_prefix=shared and not args.fused)
     g.prefill()
     g.snapshot_step_tiles()
     has_cow = w.cow_pairs.shape[0] > 0
@@ -396,6 +402,9 @@ def run_pkv(args, rank, world, local):
         alg_bytes = dec_bytes + w.store_bytes() + w.copy_bytes()
         launch_s = total_s / K
         kernel = "paged_decode_kernel (fused step: copies + store + decode)"
+    elif g.prefix is not None:
+        alg_bytes, launch_s = dec_bytes, dec_s
+        kernel = "paged_prefill_kernel (prefix mode) + paged_decode_kernel"
     else:
         alg_bytes, launch_s, kernel = dec_bytes, dec_s, "paged_decode_kernel"
     achieved = alg_bytes / launch_s / 1e9
@@ -404,7 +413,9 @@ def run_pkv(args, rank, world, local):
     step_desc = (("copy-on-write copies + " if has_cow else "") + "store 1 token/seq (quantize+scatter) + decode"
                  + (", one fused launch (pkv_decode_step)" if fused else ", separate launches")
                  + (", decode walks each forked child right after its parent (pkv_paged_attention_decode_ex)"
-                    if g.seq_order is not None and not fused else ""))
+                    if g.seq_order is not None and not fused else "")
+                 + (", shared-prefix decode: each shared block attended once per group (prefix pass + decode)"
+                    if g.prefix is not None else ""))
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": total_s * 1e3 / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,

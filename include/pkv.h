@@ -98,7 +98,8 @@ enum {
   PKV_DEVERR_SLOT_GROUP = 3,   /* tokens bound for one block are not consecutive offsets */
   PKV_DEVERR_CONTEXT_LEN = 4,  /* context_len < 0, > max_context_len or > max_blocks*block_size */
   PKV_DEVERR_TIMEOUT = 5,      /* a bounded wait on an asynchronous copy gave up */
-  PKV_DEVERR_SEQ_ORDER = 6     /* a walk-order entry outside [0, num_seqs) */
+  PKV_DEVERR_SEQ_ORDER = 6,    /* a walk-order entry outside [0, num_seqs) */
+  PKV_DEVERR_SHARED = 7        /* a shared-prefix group or shared block count out of range */
 };
 
 /* Describes one layer's cache pool. Pointers are device pointers, 16-byte aligned. */
@@ -226,21 +227,48 @@ PKV_API pkv_status pkv_paged_attention_decode(const pkv_cache_desc* desc, void* 
 
 /*
  * pkv_paged_attention_decode_ex -- pkv_paged_attention_decode with options; the same arguments,
- * results, workspace and ordering rules, plus:
- *   seq_order  device int32 [num_seqs] or NULL: the order in which the decode walks the
- *              sequences (a permutation of 0 .. num_seqs-1; results do not depend on it). A caller
- *              that knows which sequences share physical blocks (beam candidates forked from one
- *              parent, [deepinsea] "Copy-on-Write 机制"; requests on a common prefix, [yunthe]
- *              "PagedAttention分页注意力机制与vLLM实现") lists them next to each other, so that the
- *              shared blocks are read from memory once and found in L2 by the neighbours. An entry
- *              outside [0, num_seqs) leaves that position empty and sets PKV_DEVERR_SEQ_ORDER; a
- *              repeated entry makes the outputs of the repeated sequence unspecified.
- * options may be NULL (plain decode). struct_bytes must be sizeof(pkv_decode_options) as the
- * caller compiled it (fields this library does not know are refused with PKV_ERR_UNSUPPORTED).
+ * results and ordering rules, plus:
+ *
+ * Walk order. seq_order: device int32 [num_seqs] or NULL: the order in which the decode walks the
+ *   sequences (a permutation of 0 .. num_seqs-1; results do not depend on it). A caller that knows
+ *   which sequences share physical blocks (beam candidates forked from one parent, [deepinsea]
+ *   "Copy-on-Write 机制"; requests on a common prefix, [yunthe] "PagedAttention分页注意力机制与vLLM
+ *   实现") lists them next to each other, so that the shared blocks are read from memory once and
+ *   found in L2 by the neighbours. An entry outside [0, num_seqs) leaves that position empty and
+ *   sets PKV_DEVERR_SEQ_ORDER; a repeated entry makes that sequence's outputs unspecified.
+ *
+ * Shared-prefix decode (num_prefix_groups > 0). Sequences that share their first blocks (one
+ *   physical copy, [yunthe] "PagedAttention分页注意力机制与vLLM实现" and "Prefix Caching与多轮对话场景
+ *   优化实践") are given as groups: group i's members are prefix_members[prefix_group_start[i] ..
+ *   prefix_group_start[i+1]), and shared_blocks[s] is the number of leading blocks sequence s shares
+ *   with its group (0 for a sequence in no group). A first pass reads each shared block once per
+ *   group and multiplies it against the queries of every member (integer tensor cores on the int8
+ *   codes, the prefill kernel's prefix mode), leaving partial softmax states in the workspace; the
+ *   decode then walks only each sequence's own blocks and merges the two. Requirements (not
+ *   checked on the device; breaking them gives unspecified outputs, never a fault): the members of
+ *   a group have the same shared_blocks value and the same table entries for those blocks; every
+ *   sequence with shared_blocks > 0 is a member of exactly one group. A shared count that leaves
+ *   no block of the sequence to the decode is clamped to leave its last block, and reported with
+ *   PKV_DEVERR_SHARED. Built for INT8 K with INT8 or INT4 V and head_dim 128 (else
+ *   PKV_ERR_UNSUPPORTED). The workspace must then be pkv_decode_ex_workspace_size(...) bytes.
+ *   max_group_size and max_shared_blocks are host bounds (they size the first pass's grid); groups
+ *   or counts above them are reported (PKV_DEVERR_SHARED) and their shared part left out.
+ *   prefix_group_start, prefix_members and shared_blocks are read like block_tables (before the
+ *   decode waits for the preceding kernel).
+ *
+ * options may be NULL (the plain decode). struct_bytes must be sizeof(pkv_decode_options) as the
+ * caller compiled it.
  */
 typedef struct pkv_decode_options {
   size_t struct_bytes;
   const int32_t* seq_order;
+  int32_t num_prefix_groups;
+  int32_t num_prefix_members;          /* prefix_group_start[num_prefix_groups] */
+  int32_t max_group_size;
+  int32_t max_shared_blocks;
+  const int32_t* prefix_group_start;   /* device int32 [num_prefix_groups + 1] */
+  const int32_t* prefix_members;       /* device int32 [num_prefix_members] */
+  const int32_t* shared_blocks;        /* device int32 [num_seqs] */
 } pkv_decode_options;
 PKV_API pkv_status pkv_paged_attention_decode_ex(const pkv_cache_desc* desc, void* out, const void* q,
                                                  int32_t num_seqs, int32_t num_q_heads,
@@ -249,6 +277,10 @@ PKV_API pkv_status pkv_paged_attention_decode_ex(const pkv_cache_desc* desc, voi
                                                  float softmax_scale, int32_t partition_tokens,
                                                  const pkv_decode_options* options, void* workspace,
                                                  size_t workspace_bytes, int32_t* dev_error, pkv_stream_t stream);
+/* Workspace bytes of pkv_paged_attention_decode_ex with these options (options may be NULL). */
+PKV_API pkv_status pkv_decode_ex_workspace_size(const pkv_cache_desc* desc, int32_t num_seqs, int32_t num_q_heads,
+                                                int32_t max_context_len, int32_t partition_tokens,
+                                                const pkv_decode_options* options, size_t* bytes);
 
 /*
  * pkv_paged_attention_prefill -- chunked prefill: causal attention of each sequence's new tokens

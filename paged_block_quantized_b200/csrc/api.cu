@@ -174,6 +174,11 @@ pkv_status make_decode_params(const pkv_cache_desc* desc, const DecodeGeometry& 
   p.block_tables = block_tables;
   p.context_lens = context_lens;
   p.seq_order = nullptr;
+  p.shared_blocks = nullptr;
+  p.ws_pml = nullptr;
+  p.ws_pacc = nullptr;
+  p.prefix_splits = 0;
+  p.max_shared_blocks = 0;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   p.ws_count = reinterpret_cast<uint32_t*>(ws);
   p.ws_ml = reinterpret_cast<float*>(ws + g.counter_bytes);
@@ -226,6 +231,47 @@ const void* device_view(const void* p, size_t bytes, bool host) {
   const bool ok_a = a.type == cudaMemoryTypeManaged || (a.type == cudaMemoryTypeDevice && a.device == dev);
   const bool ok_b = b.type == cudaMemoryTypeManaged || (b.type == cudaMemoryTypeDevice && b.device == dev);
   return ok_a && ok_b ? p : nullptr;
+}
+
+// The shared-prefix pass of pkv_paged_attention_decode_ex: how the shared blocks are cut among CTAs
+// and where its partials go in the workspace (after the decode's own regions).
+struct PrefixPlan {
+  bool on = false;
+  int32_t splits = 0, per_split = 0;
+  size_t pml_off = 0, pacc_off = 0, total = 0;
+};
+
+pkv_status prefix_plan(const pkv_cache_desc* d, const DecodeGeometry& g, int32_t num_seqs, int32_t num_q_heads,
+                       const pkv_decode_options* o, PrefixPlan* pl) {
+  pl->total = g.workspace_bytes;
+  if (o == nullptr || o->num_prefix_groups == 0 || num_seqs == 0) return PKV_OK;
+  if (o->num_prefix_groups < 0 || o->num_prefix_groups > 65535) return PKV_ERR_INVALID_ARG;
+  if (!prefill_supported(d->k_dtype, d->v_dtype, d->block_size, d->head_dim)) return PKV_ERR_UNSUPPORTED;
+  if (o->max_group_size <= 0 || o->max_shared_blocks < 0 || o->num_prefix_members <= 0) return PKV_ERR_INVALID_ARG;
+  if (o->prefix_group_start == nullptr || o->prefix_members == nullptr || o->shared_blocks == nullptr)
+    return PKV_ERR_INVALID_ARG;
+  if (!aligned(o->prefix_group_start, 4) || !aligned(o->prefix_members, 4) || !aligned(o->shared_blocks, 4))
+    return PKV_ERR_INVALID_ARG;
+  const int32_t group = num_q_heads / d->num_kv_heads;
+  const int64_t chunks = ((int64_t)o->max_group_size * group + 127) / 128;
+  const int64_t ctas = (int64_t)o->num_prefix_groups * d->num_kv_heads * chunks;
+  if (chunks > INT32_MAX || d->num_kv_heads > 65535) return PKV_ERR_UNSUPPORTED;
+  // about two CTAs per SM in all, never more parts than shared blocks, at most 16
+  int64_t splits = (2 * (int64_t)sm_count() + ctas - 1) / ctas;
+  splits = splits < 1 ? 1 : (splits > 16 ? 16 : splits);
+  if (splits > o->max_shared_blocks) splits = o->max_shared_blocks > 0 ? o->max_shared_blocks : 1;
+  const int64_t per = o->max_shared_blocks > 0 ? (o->max_shared_blocks + splits - 1) / splits : 1;
+  splits = o->max_shared_blocks > 0 ? (o->max_shared_blocks + per - 1) / per : 1;
+  if ((int64_t)o->num_prefix_groups * splits > 65535) return PKV_ERR_UNSUPPORTED;  // grid z
+  pl->on = true;
+  pl->splits = (int32_t)splits;
+  pl->per_split = (int32_t)per;
+  const size_t gt = (size_t)g.shape.heads_per_warp;
+  const size_t slots = (size_t)num_seqs * (num_q_heads / gt) * (size_t)splits;
+  pl->pml_off = (g.workspace_bytes + 255) / 256 * 256;
+  pl->pacc_off = pl->pml_off + (slots * gt * 2 * sizeof(float) + 255) / 256 * 256;
+  pl->total = pl->pacc_off + slots * gt * d->head_dim * sizeof(float);
+  return PKV_OK;
 }
 
 // Any memory the device can dereference (its own, or mapped host memory): the address to use.
@@ -313,23 +359,43 @@ pkv_status pkv_paged_attention_decode(const pkv_cache_desc* desc, void* out, con
   return launch_decode(p, g.shape, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
+pkv_status pkv_decode_ex_workspace_size(const pkv_cache_desc* desc, int32_t num_seqs, int32_t num_q_heads,
+                                        int32_t max_context_len, int32_t partition_tokens,
+                                        const pkv_decode_options* options, size_t* bytes) {
+  if (bytes == nullptr) return PKV_ERR_INVALID_ARG;
+  if (options != nullptr && options->struct_bytes != sizeof(pkv_decode_options))
+    return options->struct_bytes < sizeof(size_t) ? PKV_ERR_INVALID_ARG : PKV_ERR_UNSUPPORTED;
+  pkv_status st = check_desc(desc);
+  if (st != PKV_OK) return st;
+  DecodeGeometry g;
+  st = decode_geometry(desc, num_seqs, num_q_heads, max_context_len, partition_tokens, &g);
+  if (st != PKV_OK) return st;
+  PrefixPlan pl;
+  st = prefix_plan(desc, g, num_seqs, num_q_heads, options, &pl);
+  if (st != PKV_OK) return st;
+  *bytes = pl.total;
+  return PKV_OK;
+}
+
 pkv_status pkv_paged_attention_decode_ex(const pkv_cache_desc* desc, void* out, const void* q, int32_t num_seqs,
                                          int32_t num_q_heads, const int32_t* block_tables,
                                          int32_t max_blocks_per_seq, const int32_t* context_lens,
                                          int32_t max_context_len, float softmax_scale, int32_t partition_tokens,
                                          const pkv_decode_options* options, void* workspace, size_t workspace_bytes,
                                          int32_t* dev_error, pkv_stream_t stream) {
-  if (options != nullptr && options->struct_bytes != sizeof(pkv_decode_options)) {
-    if (options->struct_bytes < sizeof(size_t)) return PKV_ERR_INVALID_ARG;
-    return PKV_ERR_UNSUPPORTED;
-  }
+  if (options != nullptr && options->struct_bytes != sizeof(pkv_decode_options))
+    return options->struct_bytes < sizeof(size_t) ? PKV_ERR_INVALID_ARG : PKV_ERR_UNSUPPORTED;
   pkv_status st = check_desc(desc);
   if (st != PKV_OK) return st;
   if (!decode_supported(desc->k_dtype, desc->v_dtype, desc->block_size, desc->head_dim)) return PKV_ERR_UNSUPPORTED;
   DecodeGeometry g;
   st = decode_geometry(desc, num_seqs, num_q_heads, max_context_len, partition_tokens, &g);
   if (st != PKV_OK) return st;
+  PrefixPlan pl;
+  st = prefix_plan(desc, g, num_seqs, num_q_heads, options, &pl);
+  if (st != PKV_OK) return st;
   if (num_seqs == 0) return PKV_OK;
+  if (workspace_bytes < pl.total) return PKV_ERR_INVALID_ARG;
   DecodeParams p;
   st = make_decode_params(desc, g, out, q, num_seqs, num_q_heads, block_tables, max_blocks_per_seq, context_lens,
                           max_context_len, softmax_scale, workspace, workspace_bytes, dev_error, &p);
@@ -338,7 +404,48 @@ pkv_status pkv_paged_attention_decode_ex(const pkv_cache_desc* desc, void* out, 
     if (!aligned(options->seq_order, 4)) return PKV_ERR_INVALID_ARG;
     p.seq_order = options->seq_order;
   }
-  return launch_decode(p, g.shape, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (pl.on) {
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    PrefillParams pp = {};
+    pp.k_codes = desc->k_codes;
+    pp.v_codes = desc->v_codes;
+    pp.k_scale = desc->k_scale;
+    pp.v_scale = desc->v_scale;
+    pp.v_zp = desc->v_zp;
+    pp.q = static_cast<const __half*>(q);
+    pp.block_tables = block_tables;
+    pp.context_lens = context_lens;
+    pp.dev_error = dev_error;
+    pp.num_seqs = num_seqs;
+    pp.num_blocks = desc->num_blocks;
+    pp.num_kv_heads = desc->num_kv_heads;
+    pp.num_q_heads = num_q_heads;
+    pp.group = num_q_heads / desc->num_kv_heads;
+    pp.max_blocks_per_seq = max_blocks_per_seq;
+    pp.max_context_len = max_context_len;
+    pp.block_size = desc->block_size;
+    pp.v_dtype = desc->v_dtype;
+    pp.scale_log2 = p.scale_log2;
+    pp.group_start = options->prefix_group_start;
+    pp.members = options->prefix_members;
+    pp.shared_blocks = options->shared_blocks;
+    pp.pml = reinterpret_cast<float*>(ws + pl.pml_off);
+    pp.pacc = reinterpret_cast<float*>(ws + pl.pacc_off);
+    pp.n_members = options->num_prefix_members;
+    pp.max_group_size = options->max_group_size;
+    pp.max_shared_blocks = options->max_shared_blocks;
+    pp.splits = pl.splits;
+    pp.per_split = pl.per_split;
+    pp.gt = g.shape.heads_per_warp;
+    if (launch_prefix(pp, options->num_prefix_groups, s) != cudaSuccess) return PKV_ERR_CUDA;
+    p.shared_blocks = options->shared_blocks;
+    p.ws_pml = pp.pml;
+    p.ws_pacc = pp.pacc;
+    p.prefix_splits = pl.splits;
+    p.max_shared_blocks = options->max_shared_blocks;
+  }
+  return launch_decode(p, g.shape, s) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
 pkv_status pkv_paged_attention_prefill(const pkv_cache_desc* desc, void* out, const void* q, int32_t num_seqs,

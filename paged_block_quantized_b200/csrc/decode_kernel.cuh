@@ -148,7 +148,8 @@ struct Win {
   int s, hg, j0, n;     // walk position of the sequence, head group, first block, blocks in the window (0 = none)
   int sa;               // the sequence itself (its index in q, out, tables): seq_order[s], or s
   int g;                // KV head of the head group
-  int L, nblk;          // clamped length of the sequence and its block count
+  int L, nblk;          // clamped length of the sequence and its private block count (after sb)
+  int sb;               // its leading blocks attended by the shared-prefix pass (0 without one)
   int r0;               // position of block j0 relative to the warp's first position
   long long seq_p0;     // stream position of the sequence's first block (head group 0)
 };
@@ -723,8 +724,8 @@ __device__ __forceinline__ float warp_maxf(float v) {
 // i (32 at a time); each lane owns D / 32 consecutive dims of every head and fetches them from
 // four partials at once.
 template <int GT, int D>
-__device__ __forceinline__ void merge_partials(const DecodeParams& p, long long slot0, int n_seg, int s, int hg,
-                                            int lane) {
+__device__ __forceinline__ void merge_partials(const DecodeParams& p, long long slot0, int n_seg, long long pslot0,
+                                               int n_pref, int s, int hg, int lane) {
   constexpr int DL = D / 32;
   static_assert(DL == 2 || DL == 4 || DL == 8, "head_dim");
   float M[GT], Ls[GT], A[GT][DL];
@@ -735,37 +736,45 @@ __device__ __forceinline__ void merge_partials(const DecodeParams& p, long long 
 #pragma unroll
     for (int d = 0; d < DL; ++d) A[hh][d] = 0.f;
   }
-  for (int i0 = 0; i0 < n_seg; i0 += 32) {
-    const bool has = i0 + lane < n_seg;
-    float e[GT];
+  // the warps' partials of the unit, then (shared-prefix decode) the prefix pass's partials
+#pragma unroll 1
+  for (int range = 0; range < 2; ++range) {
+    const float* mlb = range == 0 ? p.ws_ml : p.ws_pml;
+    const float* accb = range == 0 ? p.ws_acc : p.ws_pacc;
+    const long long base = range == 0 ? slot0 : pslot0;
+    const int n = range == 0 ? n_seg : n_pref;
+    for (int i0 = 0; i0 < n; i0 += 32) {
+      const bool has = i0 + lane < n;
+      float e[GT];
 #pragma unroll
-    for (int hh = 0; hh < GT; ++hh) {
-      float2 ml = make_float2(kNegBig, 0.f);
-      if (has) ml = __ldcg(reinterpret_cast<const float2*>(p.ws_ml) + (slot0 + i0 + lane) * GT + hh);
-      const float mn = fmaxf(M[hh], warp_maxf(ml.x));
-      const float f = ex2(M[hh] - mn);
-      Ls[hh] *= f;
+      for (int hh = 0; hh < GT; ++hh) {
+        float2 ml = make_float2(kNegBig, 0.f);
+        if (has) ml = __ldcg(reinterpret_cast<const float2*>(mlb) + (base + i0 + lane) * GT + hh);
+        const float mn = fmaxf(M[hh], warp_maxf(ml.x));
+        const float f = ex2(M[hh] - mn);
+        Ls[hh] *= f;
 #pragma unroll
-      for (int d = 0; d < DL; ++d) A[hh][d] *= f;
-      M[hh] = mn;
-      e[hh] = has ? ex2(ml.x - mn) : 0.f;
-      Ls[hh] += warp_sum(ml.y * e[hh]);
-    }
-    const int nj = min(32, n_seg - i0);
-    for (int j = 0; j < nj; j += 4) {
+        for (int d = 0; d < DL; ++d) A[hh][d] *= f;
+        M[hh] = mn;
+        e[hh] = has ? ex2(ml.x - mn) : 0.f;
+        Ls[hh] += warp_sum(ml.y * e[hh]);
+      }
+      const int nj = min(32, n - i0);
+      for (int j = 0; j < nj; j += 4) {
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
-        if (j + jj >= nj) break;
-        const long long sl = slot0 + i0 + j + jj;
+        for (int jj = 0; jj < 4; ++jj) {
+          if (j + jj >= nj) break;
+          const long long sl = base + i0 + j + jj;
 #pragma unroll
-        for (int hh = 0; hh < GT; ++hh) {
-          const float ej = __shfl_sync(kFull, e[hh], j + jj);
-          const float* src = p.ws_acc + (sl * GT + hh) * D + lane * DL;
+          for (int hh = 0; hh < GT; ++hh) {
+            const float ej = __shfl_sync(kFull, e[hh], j + jj);
+            const float* src = accb + (sl * GT + hh) * D + lane * DL;
 #pragma unroll
-          for (int d = 0; d < DL; d += 2) {
-            const float2 a = __ldcg(reinterpret_cast<const float2*>(src + d));
-            A[hh][d] = fmaf(a.x, ej, A[hh][d]);
-            A[hh][d + 1] = fmaf(a.y, ej, A[hh][d + 1]);
+            for (int d = 0; d < DL; d += 2) {
+              const float2 a = __ldcg(reinterpret_cast<const float2*>(src + d));
+              A[hh][d] = fmaf(a.x, ej, A[hh][d]);
+              A[hh][d + 1] = fmaf(a.y, ej, A[hh][d + 1]);
+            }
           }
         }
       }
@@ -869,6 +878,17 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
     const int a = sid(k);
     return a < 0 ? 0 : clamp_len(p, p.context_lens[a], BS);
   };
+  // Shared-prefix decode: leading blocks of the sequence at walk position k (length L) that the
+  // prefix pass attended; at least its last block stays with the decode (a count beyond that is
+  // clamped and reported).
+  auto sb_at = [&](int k, int L) -> int {
+    if (p.shared_blocks == nullptr || L == 0) return 0;
+    const int a = p.seq_order == nullptr ? k : __ldg(p.seq_order + k);  // valid: L > 0
+    const int v = p.shared_blocks[a];
+    const int sb = max(0, min(v, min((L + BS - 1) / BS - 1, p.max_shared_blocks)));
+    if (sb != v && w == 0) record_error(p.dev_error, PKV_DEVERR_SHARED);
+    return sb;
+  };
 
   uint8_t* my_stages = smem + (size_t)warp * C::NS * C::STAGE;
   uint64_t* my_bars = reinterpret_cast<uint64_t*>(smem + C::SMEM_STAGES) + warp * C::NS;
@@ -902,7 +922,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
     }
     // the stream counts the sequences in walk order (the same as index order without one)
     const int Lw = p.seq_order == nullptr ? L : (s < S ? len_at(s) : 0);
-    int sum = (Lw + BS - 1) / BS;
+    int sum = (Lw + BS - 1) / BS - (s < S ? sb_at(s, Lw) : 0);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(kFull, sum, off);
     T += sum;
@@ -935,16 +955,18 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
 
   // ---- pass 2: the unit and block of `start` ----
   Win cur;
-  int Lchunk = 0, chunk_base = 0;  // lane holds the clamped length of sequence chunk_base + lane
+  int Lchunk = 0, SBchunk = 0, chunk_base = 0;  // lane: length and shared blocks at walk position chunk_base + lane
   {
     long long acc0 = 0;
     cur.s = cur.sa = 0;
     cur.L = cur.nblk = 1;
+    cur.sb = 0;
     cur.seq_p0 = 0;
     for (int base = 0; base < S; base += 32) {  // found before base reaches S: start < T
       const int s = base + lane;
       const int L = s < S ? len_at(s) : 0;
-      const long long cnt = (long long)((L + BS - 1) / BS) * HG;
+      const int sb = s < S ? sb_at(s, L) : 0;
+      const long long cnt = (long long)((L + BS - 1) / BS - sb) * HG;
       long long incl = cnt;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
@@ -958,9 +980,11 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
         cur.s = base + f;
         cur.sa = p.seq_order == nullptr ? cur.s : __ldg(p.seq_order + cur.s);  // valid: it has blocks
         cur.L = __shfl_sync(kFull, L, f);
-        cur.nblk = (cur.L + BS - 1) / BS;
+        cur.sb = __shfl_sync(kFull, sb, f);
+        cur.nblk = (cur.L + BS - 1) / BS - cur.sb;
         cur.seq_p0 = acc0 + __shfl_sync(kFull, incl - cnt, f);
         Lchunk = L;
+        SBchunk = sb;
         chunk_base = base;
         break;
       }
@@ -980,9 +1004,11 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
     if (s < chunk_base || s >= chunk_base + 32) {
       chunk_base = s;
       Lchunk = (s + lane < S) ? len_at(s + lane) : 0;
+      SBchunk = (s + lane < S) ? sb_at(s + lane, Lchunk) : 0;
     }
     return __shfl_sync(kFull, Lchunk, s - chunk_base);
   };
+  auto seq_sb = [&](int s) -> int { return __shfl_sync(kFull, SBchunk, s - chunk_base); };  // after seq_len(s)
 
   // the window after `a`, within [.., end); n = 0 if none
   auto next_win = [&](const Win& a) -> Win {
@@ -1005,7 +1031,8 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
         b.s = s;
         b.sa = (s < S && p.seq_order != nullptr) ? __ldg(p.seq_order + s) : s;  // valid when L > 0
         b.L = L;
-        b.nblk = (L + BS - 1) / BS;
+        b.sb = s < S ? seq_sb(s) : 0;
+        b.nblk = (L + BS - 1) / BS - b.sb;
       }
       b.g = (b.hg * GT) / p.group;
     }
@@ -1017,7 +1044,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
   auto load_ids = [&](const Win& a, WinLanes& r) {
     r.meta = false;
     r.raw = -1;
-    if (lane < a.n) r.raw = p.block_tables[(size_t)a.sa * p.max_blocks_per_seq + a.j0 + lane];
+    if (lane < a.n) r.raw = p.block_tables[(size_t)a.sa * p.max_blocks_per_seq + a.sb + a.j0 + lane];
   };
   auto load_meta = [&](const Win& a, WinLanes& r) {
     r.valid = lane < a.n && r.raw >= 0 && r.raw < p.num_blocks;
@@ -1106,8 +1133,8 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
   int pend_since = 0;        // cpos when the partial was written
   uint32_t pend_ticket = 0;  // lane 0: the increment's result
   uint32_t pend_nseg = 0;
-  long long pend_slot0 = 0, pend_u = 0;
-  int pend_s = 0, pend_hg = 0;
+  long long pend_slot0 = 0, pend_u = 0, pend_pslot0 = 0;
+  int pend_s = 0, pend_hg = 0, pend_np = 0;
   auto take_ticket = [&]() {
     if (lane == 0) {
       fence_acq_rel_gpu();
@@ -1125,7 +1152,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
       // order to every lane of the warp before any of them reads a partial.
       if (lane == 0) fence_acq_rel_gpu();
       __syncwarp();
-      merge_partials<GT, D>(p, pend_slot0, (int)pend_nseg, pend_s, pend_hg, lane);
+      merge_partials<GT, D>(p, pend_slot0, (int)pend_nseg, pend_pslot0, pend_np, pend_s, pend_hg, lane);
     }
     pend = 0;
   };
@@ -1167,7 +1194,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
     const float nzb = -(kMagic + __shfl_sync(kFull, rc.zp, kw_i));
     const bool valid = __shfl_sync(kFull, rc.valid ? 1 : 0, kw_i) != 0;
     const uint8_t* kt = my_stages + (size_t)st * C::STAGE;
-    eng.block(kt, kt + C::K_TILE, ks, vs, nzb, valid, (cur.j0 + kw_i) * BS, cur.L, p.scale_log2);
+    eng.block(kt, kt + C::K_TILE, ks, vs, nzb, valid, (cur.sb + cur.j0 + kw_i) * BS, cur.L, p.scale_log2);
     __syncwarp();  // the stage's reads are complete (their values were consumed above)
     if constexpr (kDeferTicket) {
       if (pend == 1 && cpos >= pend_since + 2) take_ticket();
@@ -1183,7 +1210,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
     if (j_end == cur.nblk || cpos == n_total) {
       eng.finish();
       const long long u = (long long)cur.s * HG + cur.hg;
-      if (seg_j0 == 0 && j_end == cur.nblk) {
+      if (seg_j0 == 0 && j_end == cur.nblk && cur.sb == 0) {
         eng.write_out(p, cur.sa, cur.hg);  // the whole unit was processed by this warp
       } else {
         // one segment of a split unit: publish the partial; the last warp to finish merges
@@ -1201,6 +1228,9 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
         pend_slot0 = u + w_first;
         pend_s = cur.sa;
         pend_hg = cur.hg;
+        // a unit with a shared prefix also folds in the prefix pass's partials
+        pend_np = cur.sb > 0 ? p.prefix_splits : 0;
+        pend_pslot0 = ((long long)cur.sa * HG + cur.hg) * p.prefix_splits;
         if constexpr (!kDeferTicket) resolve_pending();
       }
       eng.reset();

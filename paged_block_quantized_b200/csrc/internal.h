@@ -22,6 +22,13 @@ struct DecodeParams {
   const int32_t* block_tables;
   const int32_t* context_lens;
   const int32_t* seq_order;  // [S] walk order of the sequences, or NULL (index order)
+  // shared-prefix decode: the first shared_blocks[s] blocks of sequence s were attended by the
+  // prefix pass, whose prefix_splits partials per (sequence, head group) the merge folds in
+  const int32_t* shared_blocks;  // [S] or NULL
+  const float* ws_pml;           // [(S*HG) * prefix_splits][GT][2]
+  const float* ws_pacc;          // [(S*HG) * prefix_splits][GT][D]
+  int32_t prefix_splits;
+  int32_t max_shared_blocks;     // host bound: counts above it are clamped (and reported)
   uint32_t* ws_count;  // [S * HG] tickets of split units (zero between calls)
   float* ws_ml;        // [(S*HG + W) * GT][2] partial running max (log2 domain) and sum
   float* ws_acc;       // [(S*HG + W) * GT][D] partial un-normalised accumulators
@@ -155,9 +162,23 @@ struct PrefillParams {
   int32_t block_size;
   int32_t v_dtype;
   float scale_log2;
+  // shared-prefix pass of the decode (the same kernel in its prefix mode)
+  const int32_t* group_start;    // [groups + 1] offsets into members
+  const int32_t* members;        // sequence ids of the groups, one after another
+  const int32_t* shared_blocks;  // [S] leading blocks shared with the group
+  float* pml;                    // partials out: [(S * Hq/gt) * splits][gt][2] (max in log2 units, sum)
+  float* pacc;                   // [(S * Hq/gt) * splits][gt][D]
+  int32_t n_members;
+  int32_t max_group_size;
+  int32_t splits;                // shared blocks cut into this many parts (one CTA each)
+  int32_t per_split;
+  int32_t gt;                    // query heads per head group of the decode
+  int32_t max_shared_blocks;     // host bound, clamped as the decode clamps it
 };
 bool prefill_supported(int32_t k_dtype, int32_t v_dtype, int32_t block_size, int32_t head_dim);
 cudaError_t launch_prefill(const PrefillParams& p, cudaStream_t stream);
+// the prefix mode: grid (column chunks of the largest group, KV heads, groups x splits)
+cudaError_t launch_prefix(const PrefillParams& p, int32_t n_groups, cudaStream_t stream);
 
 // ---------------------------------------------------------------- fused step
 // Copy-on-write copies, then the store, then the decode, in one cooperative launch of the decode

@@ -13,10 +13,10 @@ bool prefill_supported(int32_t k_dtype, int32_t v_dtype, int32_t block_size, int
 
 namespace {
 
-template <int VT, int BS>
-cudaError_t launch_prefill_t(const PrefillParams& p, cudaStream_t stream) {
+template <int VT, int BS, bool PREFIX>
+cudaError_t launch_prefill_t(const PrefillParams& p, int32_t n_groups, cudaStream_t stream) {
   using C = prefill_detail::Cfg<VT, BS>;
-  auto kern = prefill_detail::paged_prefill_kernel<VT, BS>;
+  auto kern = prefill_detail::paged_prefill_kernel<VT, BS, PREFIX>;
   static unsigned long long configured = 0;  // one bit per device; benign race
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -33,23 +33,31 @@ cudaError_t launch_prefill_t(const PrefillParams& p, cudaStream_t stream) {
   if constexpr (C::V_SWZ) {
     if (!encode_tile_map(&tm.v, p.v_codes, rows, C::V_ROW, BS)) return cudaErrorInvalidValue;
   }
-  const int chunks = (p.max_q_len * p.group + prefill_detail::kCols - 1) / prefill_detail::kCols;
-  dim3 grid(chunks, p.num_kv_heads, p.num_seqs);
+  const int col_rows = PREFIX ? p.max_group_size : p.max_q_len;
+  const int chunks = (col_rows * p.group + prefill_detail::kCols - 1) / prefill_detail::kCols;
+  dim3 grid(chunks, p.num_kv_heads, PREFIX ? n_groups * p.splits : p.num_seqs);
   kern<<<grid, prefill_detail::kThreads, C::SMEM, stream>>>(p, tm);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_prefill(const PrefillParams& p, cudaStream_t stream) {
+template <bool PREFIX>
+cudaError_t launch_mode(const PrefillParams& p, int32_t n_groups, cudaStream_t stream) {
   if (p.v_dtype == PKV_INT8_SYM) {
-    if (p.block_size == 16) return launch_prefill_t<PKV_INT8_SYM, 16>(p, stream);
-    if (p.block_size == 32) return launch_prefill_t<PKV_INT8_SYM, 32>(p, stream);
+    if (p.block_size == 16) return launch_prefill_t<PKV_INT8_SYM, 16, PREFIX>(p, n_groups, stream);
+    if (p.block_size == 32) return launch_prefill_t<PKV_INT8_SYM, 32, PREFIX>(p, n_groups, stream);
   } else if (p.v_dtype == PKV_INT4_ASYM) {
-    if (p.block_size == 16) return launch_prefill_t<PKV_INT4_ASYM, 16>(p, stream);
-    if (p.block_size == 32) return launch_prefill_t<PKV_INT4_ASYM, 32>(p, stream);
+    if (p.block_size == 16) return launch_prefill_t<PKV_INT4_ASYM, 16, PREFIX>(p, n_groups, stream);
+    if (p.block_size == 32) return launch_prefill_t<PKV_INT4_ASYM, 32, PREFIX>(p, n_groups, stream);
   }
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_prefill(const PrefillParams& p, cudaStream_t stream) { return launch_mode<false>(p, 0, stream); }
+
+cudaError_t launch_prefix(const PrefillParams& p, int32_t n_groups, cudaStream_t stream) {
+  return launch_mode<true>(p, n_groups, stream);
 }
 
 }  // namespace pkv

@@ -106,7 +106,7 @@ constexpr uint32_t kH2Bias8 = 0x64806480u;
 
 }  // namespace
 
-template <int VT, int BS>
+template <int VT, int BS, bool PREFIX>
 __global__ void __launch_bounds__(kThreads, 1)
     paged_prefill_kernel(const PrefillParams p, const __grid_constant__ TileMaps tm) {
   using C = Cfg<VT, BS>;
@@ -114,38 +114,71 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* const smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
-  const int s = blockIdx.z, kvh = blockIdx.y;
+  const int kvh = blockIdx.y;
   const int G = p.group;
-  const int q0 = p.cu_q_lens[s];
-  const int qlen = p.cu_q_lens[s + 1] - q0;
-  const int col0 = blockIdx.x * kCols;  // first column of this CTA within (s, kvh)
-  if (q0 < 0 || qlen < 0 || qlen > p.max_q_len || q0 + qlen > p.total_q) {  // rows outside q / out
-    if (threadIdx.x == 0 && blockIdx.x == 0 && kvh == 0) record_error(p.dev_error, PKV_DEVERR_CONTEXT_LEN);
-    return;
-  }
-  if (qlen == 0 || col0 >= qlen * G) return;
-  const int ncols = min(kCols, qlen * G - col0);
-  int ctx = p.context_lens[s];
-  const int cap = min(p.max_context_len, p.max_blocks_per_seq * BS);
-  if (qlen > ctx || ctx > cap) {
-    // a chunk longer than its context, or a context beyond the table / the host bound: the
-    // rows are zeroed (the first CTA of the sequence and head reports it)
-    if (threadIdx.x == 0 && blockIdx.x == 0 && kvh == 0) record_error(p.dev_error, PKV_DEVERR_CONTEXT_LEN);
-    if (qlen > ctx) {
-      for (int col = threadIdx.x; col < ncols; col += kThreads) {
-        const int gc = col0 + col;
-        __half2* o = reinterpret_cast<__half2*>(p.out + ((size_t)(q0 + gc / G) * p.num_q_heads +
-                                                         (size_t)kvh * G + gc % G) * kD);
-        for (int d = 0; d < kD / 2; ++d) o[d] = __floats2half2_rn(0.f, 0.f);
-      }
+  const int col0 = blockIdx.x * kCols;  // first column of this CTA
+  const int cap_tab = p.max_blocks_per_seq * BS;
+
+  // ---- the work of this CTA: its columns, the blocks they see, where the results go ----
+  // Prefill: columns of sequence s = blockIdx.z are (chunk token i, head hh) = (c / G, c % G);
+  //   blocks [0, the last column's causal limit); the output rows are normalised.
+  // Prefix (shared-prefix decode): columns of group gi = blockIdx.z / splits are (member m, head
+  //   hh) = (c / G, c % G) with the members' one decode query each; blocks [split * per_split,
+  //   ...) of the group's shared blocks, all visible; the results are partials for the decode.
+  int ncols, jb, je, s_tab, pos0 = 0, q0 = 0, gstart = 0, split = 0;
+  if constexpr (!PREFIX) {
+    const int s = blockIdx.z;
+    q0 = p.cu_q_lens[s];
+    const int qlen = p.cu_q_lens[s + 1] - q0;
+    if (q0 < 0 || qlen < 0 || qlen > p.max_q_len || q0 + qlen > p.total_q) {  // rows outside q / out
+      if (threadIdx.x == 0 && blockIdx.x == 0 && kvh == 0) record_error(p.dev_error, PKV_DEVERR_CONTEXT_LEN);
       return;
     }
-    ctx = cap;
+    if (qlen == 0 || col0 >= qlen * G) return;
+    ncols = min(kCols, qlen * G - col0);
+    int ctx = p.context_lens[s];
+    const int cap = min(p.max_context_len, cap_tab);
+    if (qlen > ctx || ctx > cap) {
+      // a chunk longer than its context, or a context beyond the table / the host bound: the
+      // rows are zeroed (the first CTA of the sequence and head reports it)
+      if (threadIdx.x == 0 && blockIdx.x == 0 && kvh == 0) record_error(p.dev_error, PKV_DEVERR_CONTEXT_LEN);
+      if (qlen > ctx) {
+        for (int col = threadIdx.x; col < ncols; col += kThreads) {
+          const int gc = col0 + col;
+          __half2* o = reinterpret_cast<__half2*>(p.out + ((size_t)(q0 + gc / G) * p.num_q_heads +
+                                                           (size_t)kvh * G + gc % G) * kD);
+          for (int d = 0; d < kD / 2; ++d) o[d] = __floats2half2_rn(0.f, 0.f);
+        }
+        return;
+      }
+      ctx = cap;
+    }
+    pos0 = ctx - qlen;  // position of the first query token
+    const int lim_last = min(pos0 + (col0 + ncols - 1) / G + 1, cap);  // the last column sees the most
+    jb = 0;
+    je = (lim_last + BS - 1) / BS;
+    s_tab = s;
+  } else {
+    const int gi = blockIdx.z / p.splits;
+    split = blockIdx.z % p.splits;
+    gstart = p.group_start[gi];
+    const int gsize = p.group_start[gi + 1] - gstart;
+    if (gstart < 0 || gsize < 0 || gsize > p.max_group_size || gstart + gsize > p.n_members) {
+      if (threadIdx.x == 0 && blockIdx.x == 0 && kvh == 0 && split == 0) record_error(p.dev_error, PKV_DEVERR_SHARED);
+      return;
+    }
+    if (gsize == 0 || col0 >= gsize * G) return;
+    ncols = min(kCols, gsize * G - col0);
+    s_tab = p.members[gstart];
+    if (s_tab < 0 || s_tab >= p.num_seqs) return;  // reported by the decode, which skips it too
+    // the group's shared blocks, as the decode counts them for its first member
+    const int L = max(0, min(p.context_lens[s_tab], min(p.max_context_len, cap_tab)));
+    const int nb = (L + BS - 1) / BS;
+    const int sb = max(0, min(p.shared_blocks[s_tab], min(nb - 1, p.max_shared_blocks)));
+    jb = min(split * p.per_split, sb);
+    je = min(jb + p.per_split, sb);
   }
-  const int pos0 = ctx - qlen;  // position of the first query token
-  // blocks the last column needs (it sees the most)
-  const int lim_last = min(pos0 + (col0 + ncols - 1) / G + 1, cap);
-  const int nblk = (lim_last + BS - 1) / BS;
+  const int nblk = je - jb;
 
   uint8_t* const stages = smem;
   uint8_t* const pbuf = smem + C::OFF_P;
@@ -155,9 +188,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* const bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   StageMeta* const meta = reinterpret_cast<StageMeta*>(smem + C::OFF_META);
 
-  const int32_t* table = p.block_tables + (size_t)s * p.max_blocks_per_seq;
+  const int32_t* table = p.block_tables + (size_t)s_tab * p.max_blocks_per_seq + jb;
   int issued = 0;            // thread 0: blocks whose copies have been issued
-  auto issue = [&](int j) {  // thread 0: copies of block j into stage j % NS, and its facts
+  auto issue = [&](int j) {  // thread 0: copies of the CTA's block j into stage j % NS, and its facts
     const int raw = table[j];
     const bool valid = raw >= 0 && raw < p.num_blocks;  // an invalid id reads block 0, masked, reported
     const int b = valid ? raw : 0;
@@ -200,13 +233,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
     const int col = 16 * warp + g + 8 * e;
-    const bool valid = col < ncols;
     const int gc = col0 + col;
     const int tok = gc / G;
+    bool valid = col < ncols;
+    size_t qrow = 0;  // (row, head) of q
+    if constexpr (!PREFIX) {
+      qrow = (size_t)(q0 + tok) * p.num_q_heads + (size_t)kvh * G + gc % G;
+    } else {
+      const int sm = valid ? p.members[gstart + tok] : -1;
+      valid = valid && sm >= 0 && sm < p.num_seqs;
+      qrow = (size_t)max(sm, 0) * p.num_q_heads + (size_t)kvh * G + gc % G;
+    }
     float x[32];
     if (valid) {
-      const uint4* qp = reinterpret_cast<const uint4*>(
-          p.q + ((size_t)(q0 + tok) * p.num_q_heads + (size_t)kvh * G + gc % G) * kD + 32 * c);
+      const uint4* qp = reinterpret_cast<const uint4*>(p.q + qrow * kD + 32 * c);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const uint4 wv = qp[i];
@@ -232,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int shift = amax > 0.f ? 22 - ex : 0;  // |q| * 2^shift < 2^22
     const float up = __int_as_float((127 + shift) << 23);
     zsc[e] = __int_as_float((127 - shift) << 23) * p.scale_log2;
-    lim[e] = valid ? min(pos0 + tok + 1, cap) : 0;
+    lim[e] = !valid ? 0 : (PREFIX ? INT_MAX : pos0 + tok + 1);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
 #pragma unroll
@@ -275,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const StageMeta bm_ = meta[st];
     const bool bvalid = bm_.valid != 0;
     const float ks = bm_.ks, vs = bm_.vs;
-    const int tok0 = j * BS;
+    const int tok0 = (jb + j) * BS;
 
     // ---- S^T = Q K^T for this warp's 16 columns and the block's BS tokens ----
     float z[BS / 8][4];
@@ -430,12 +470,53 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
 
-  // ---- normalise and write: column sums first ----
+  // ---- column sums ----
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
     l_part[e] += __shfl_xor_sync(kFull, l_part[e], 1);
     l_part[e] += __shfl_xor_sync(kFull, l_part[e], 2);
   }
+  if constexpr (PREFIX) {
+    // partials for the decode: slot (sequence, decode head group, split), head within the group;
+    // (max, sum) from the lanes that own each column, accumulators from every warp
+    const int GT = p.gt, HGd = p.num_q_heads / p.gt;
+    auto slot_of = [&](int col, int& hh) -> long long {
+      const int gc = col0 + col;
+      const int sm = p.members[gstart + gc / G];
+      if (sm < 0 || sm >= p.num_seqs) return -1;
+      const int h = kvh * G + gc % G;
+      hh = h % GT;
+      return ((long long)sm * HGd + h / GT) * p.splits + split;
+    };
+    if (c == 0) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int col = 16 * warp + g + 8 * e;
+        if (col >= ncols) continue;
+        int hh;
+        const long long sl = slot_of(col, hh);
+        if (sl < 0) continue;
+        float* ml = p.pml + (sl * GT + hh) * 2;
+        ml[0] = m_used[e] == -INFINITY ? -1.0e30f : m_used[e];
+        ml[1] = l_part[e];
+      }
+    }
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int col = 8 * n + 2 * c + e;
+        if (col >= ncols) continue;
+        int hh;
+        const long long sl = slot_of(col, hh);
+        if (sl < 0) continue;
+        *reinterpret_cast<float2*>(p.pacc + (sl * GT + hh) * kD + 16 * g + 2 * warp) =
+            make_float2(acc[n][e], acc[n][e + 2]);
+      }
+    }
+    return;
+  }
+  // ---- normalise and write ----
   if (c == 0) {
     lsum_s[16 * warp + g] = l_part[0];
     lsum_s[16 * warp + g + 8] = l_part[1];

@@ -24,12 +24,13 @@ _lib = ctypes.CDLL(LIB_PATH)
 PKV_OK, PKV_ERR_INVALID_ARG, PKV_ERR_UNSUPPORTED, PKV_ERR_OUT_OF_BLOCKS, PKV_ERR_CUDA, PKV_ERR_DEVICE_TIMEOUT = range(6)
 PKV_FP16, PKV_INT8_SYM, PKV_INT4_ASYM, PKV_FP8_E4M3 = 0, 1, 2, 3
 (PKV_DEVERR_NONE, PKV_DEVERR_BLOCK_ID, PKV_DEVERR_SLOT, PKV_DEVERR_SLOT_GROUP, PKV_DEVERR_CONTEXT_LEN,
- PKV_DEVERR_TIMEOUT, PKV_DEVERR_SEQ_ORDER) = range(7)
+ PKV_DEVERR_TIMEOUT, PKV_DEVERR_SEQ_ORDER, PKV_DEVERR_SHARED) = range(8)
 
 EXPORTED = (
     "pkv_status_string", "pkv_tile_bytes", "pkv_store_quantized", "pkv_decode_workspace_size",
     "pkv_decode_partitioning", "pkv_paged_attention_decode_static", "pkv_static_scratch_address",
-    "pkv_paged_attention_decode", "pkv_paged_attention_decode_ex", "pkv_paged_attention_prefill",
+    "pkv_paged_attention_decode", "pkv_paged_attention_decode_ex", "pkv_decode_ex_workspace_size",
+    "pkv_paged_attention_prefill",
     "pkv_copy_blocks", "pkv_swap_blocks", "pkv_decode_step", "pkv_blocks_for_tokens", "pkv_alloc_create",
     "pkv_alloc_destroy", "pkv_alloc_num_free", "pkv_alloc_refcount", "pkv_alloc_blocks", "pkv_alloc_fork",
     "pkv_alloc_release", "pkv_alloc_cow", "pkv_prefix_cache_create", "pkv_prefix_cache_destroy",
@@ -78,11 +79,34 @@ _decode = _sig("pkv_paged_attention_decode", ctypes.c_int, _DESC, _P, _P, _I32, 
 
 
 class pkv_decode_options(ctypes.Structure):
-    _fields_ = [("struct_bytes", ctypes.c_size_t), ("seq_order", ctypes.c_void_p)]
+    _fields_ = [("struct_bytes", ctypes.c_size_t), ("seq_order", ctypes.c_void_p),
+                ("num_prefix_groups", ctypes.c_int32), ("num_prefix_members", ctypes.c_int32),
+                ("max_group_size", ctypes.c_int32), ("max_shared_blocks", ctypes.c_int32),
+                ("prefix_group_start", ctypes.c_void_p), ("prefix_members", ctypes.c_void_p),
+                ("shared_blocks", ctypes.c_void_p)]
+
+
+def decode_options(seq_order=None, prefix=None):
+    """pkv_decode_options: seq_order (device int32 [S]) and/or prefix = dict(group_start, members,
+    shared_blocks: device int32 tensors; num_groups, num_members, max_group_size, max_shared_blocks: ints)."""
+    o = pkv_decode_options()
+    o.struct_bytes = ctypes.sizeof(pkv_decode_options)
+    o.seq_order = _ptr(seq_order)
+    if prefix is not None:
+        o.num_prefix_groups = int(prefix["num_groups"])
+        o.num_prefix_members = int(prefix["num_members"])
+        o.max_group_size = int(prefix["max_group_size"])
+        o.max_shared_blocks = int(prefix["max_shared_blocks"])
+        o.prefix_group_start = _ptr(prefix["group_start"])
+        o.prefix_members = _ptr(prefix["members"])
+        o.shared_blocks = _ptr(prefix["shared_blocks"])
+    return o
 
 
 _decode_ex = _sig("pkv_paged_attention_decode_ex", ctypes.c_int, _DESC, _P, _P, _I32, _I32, _P, _I32, _P, _I32,
                   ctypes.c_float, _I32, ctypes.POINTER(pkv_decode_options), _P, ctypes.c_size_t, _P, _P)
+_ws_ex = _sig("pkv_decode_ex_workspace_size", ctypes.c_int, _DESC, _I32, _I32, _I32, _I32,
+              ctypes.POINTER(pkv_decode_options), ctypes.POINTER(ctypes.c_size_t))
 _prefill = _sig("pkv_paged_attention_prefill", ctypes.c_int, _DESC, _P, _P, _I32, _I32, _P, _I32, _I32, _P, _I32, _P,
                 _I32, ctypes.c_float, _P, _P)
 _decode_static = _sig("pkv_paged_attention_decode_static", ctypes.c_int, _DESC, _P, _P, _I32, _I32, _P, _I32, _P,
@@ -187,12 +211,23 @@ def pkv_paged_attention_decode(desc, out, q, num_seqs, num_q_heads, block_tables
     return _check(st, "pkv_paged_attention_decode", raise_on_error)
 
 
+def pkv_decode_ex_workspace_size(desc, num_seqs, num_q_heads, max_context_len, partition_tokens=0, seq_order=None,
+                                 prefix=None) -> int:
+    opts = decode_options(seq_order, prefix)
+    out = ctypes.c_size_t(0)
+    st = _ws_ex(ctypes.byref(desc), int(num_seqs), int(num_q_heads), int(max_context_len), int(partition_tokens),
+                ctypes.byref(opts), ctypes.byref(out))
+    _check(st, "pkv_decode_ex_workspace_size", True)
+    return int(out.value)
+
+
 def pkv_paged_attention_decode_ex(desc, out, q, num_seqs, num_q_heads, block_tables, max_blocks_per_seq,
                                   context_lens, max_context_len, softmax_scale, partition_tokens=0, seq_order=None,
                                   workspace=None, workspace_bytes=0, dev_error=None, stream=None,
-                                  raise_on_error=True):
-    """Decode with options: seq_order (device int32 [num_seqs]) = the walk order of the sequences."""
-    opts = pkv_decode_options(ctypes.sizeof(pkv_decode_options), _ptr(seq_order))
+                                  raise_on_error=True, prefix=None):
+    """Decode with options: seq_order (device int32 [num_seqs]) = the walk order of the sequences;
+    prefix = the shared-prefix groups (see decode_options)."""
+    opts = decode_options(seq_order, prefix)
     st = _decode_ex(ctypes.byref(desc), _ptr(out), _ptr(q), int(num_seqs), int(num_q_heads), _ptr(block_tables),
                     int(max_blocks_per_seq), _ptr(context_lens), int(max_context_len), float(softmax_scale),
                     int(partition_tokens), ctypes.byref(opts), _ptr(workspace), int(workspace_bytes),

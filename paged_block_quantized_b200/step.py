@@ -28,7 +28,7 @@ _TORCH_DTYPE = {np.dtype(np.float16): torch.float16, np.dtype(np.int32): torch.i
 
 class DeviceStep:
     def __init__(self, w: Workload, device="cuda", poison: int | None = 0xA5, partition_tokens: int | None = None,
-                 beam_order: bool = False):
+                 beam_order: bool = False, shared_prefix: bool = False):
         self.w = w
         self.device = torch.device(device)
         self.pool = pkv.DevicePool.allocate(w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim, w.k_dtype,
@@ -44,6 +44,10 @@ class DeviceStep:
         use_order = beam_order and w.cow_pairs.shape[0] > 0
         if use_order:
             inputs.append(("seq_order", w.beam_walk_order()))
+        # with shared_prefix, blocks shared by several sequences are attended once per group
+        groups = w.prefix_groups() if shared_prefix else None
+        if groups is not None:
+            inputs += [("group_start", groups[0]), ("members", groups[1]), ("shared_blocks", groups[2])]
         offs, total = [], 0
         for _, a in inputs:
             offs.append(total)
@@ -59,11 +63,18 @@ class DeviceStep:
         self.out = torch.zeros_like(self.q)
         if not use_order:
             self.seq_order = None
+        self.prefix = None
+        if groups is not None:
+            sizes = np.diff(groups[0])
+            self.prefix = dict(group_start=self.group_start, members=self.members, shared_blocks=self.shared_blocks,
+                               num_groups=len(sizes), num_members=int(groups[0][-1]),
+                               max_group_size=int(sizes.max()), max_shared_blocks=int(groups[2].max()))
         self.partition_tokens = w.partition_tokens if partition_tokens is None else partition_tokens
         self.num_workers, self.num_ctas = pkv.pkv_decode_partitioning(
             self.pool.desc, w.num_seqs, w.num_q_heads, w.max_context_len, self.partition_tokens)
-        self.ws_bytes = pkv.pkv_decode_workspace_size(self.pool.desc, w.num_seqs, w.num_q_heads,
-                                                      w.max_context_len, self.partition_tokens)
+        self.ws_bytes = pkv.pkv_decode_ex_workspace_size(self.pool.desc, w.num_seqs, w.num_q_heads,
+                                                         w.max_context_len, self.partition_tokens, self.seq_order,
+                                                         self.prefix)
         # zero-filled once: the decode leaves its arrival counters at zero after every call
         self.workspace = torch.zeros(max(self.ws_bytes, 16), dtype=torch.uint8, device=dev)
 
@@ -130,12 +141,12 @@ class DeviceStep:
 
     def decode(self, stream=None, out=None, q=None):
         w = self.w
-        if self.seq_order is not None:
+        if self.seq_order is not None or self.prefix is not None:
             pkv.pkv_paged_attention_decode_ex(
                 self.pool.desc, self.out if out is None else out, self.q if q is None else q, w.num_seqs,
                 w.num_q_heads, self.block_tables, w.max_blocks_per_seq, self.context_lens, w.max_context_len,
                 w.softmax_scale, self.partition_tokens, self.seq_order, self.workspace, self.ws_bytes,
-                self.dev_error, stream=stream)
+                self.dev_error, stream=stream, prefix=self.prefix)
             return
         pkv.pkv_paged_attention_decode(
             self.pool.desc, self.out if out is None else out, self.q if q is None else q, w.num_seqs,

@@ -225,6 +225,35 @@ class Workload:
         assert sorted(order) == list(range(S))
         return np.array(order, np.int32)
 
+    def prefix_groups(self):
+        """Sequences that share their first blocks, as the shared-prefix decode takes them: a group
+        per first block id used by more than one sequence, its shared count the longest common run
+        of leading block ids of all its members, kept below every member's own block count (the
+        decode keeps each sequence's last block). Returns (group_start int32 [G+1], members int32,
+        shared_blocks int32 [S]), or None when nothing is shared."""
+        bs = self.block_size
+        by_first = {}
+        for s in range(self.num_seqs):
+            if int(self.context_lens[s]) > 0:
+                by_first.setdefault(int(self.block_tables[s, 0]), []).append(s)
+        starts, members = [0], []
+        shared = np.zeros(self.num_seqs, np.int32)
+        for seqs in by_first.values():
+            if len(seqs) < 2:
+                continue
+            nb = [(int(self.context_lens[s]) + bs - 1) // bs for s in seqs]
+            k = 0
+            while k < min(nb) - 1 and all(self.block_tables[s, k] == self.block_tables[seqs[0], k] for s in seqs):
+                k += 1
+            if k == 0:
+                continue
+            members.extend(seqs)
+            starts.append(len(members))
+            shared[seqs] = k
+        if not members:
+            return None
+        return np.array(starts, np.int32), np.array(members, np.int32), shared
+
     # ---- bytes read by one decode (the algorithmic minimum) ----
     def decode_bytes(self, unique: bool = True) -> int:
         """Algorithmic bytes one decode reads: K/V codes of valid tokens, per-block scales and

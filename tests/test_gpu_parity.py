@@ -380,3 +380,54 @@ def test_beam_walk_order(name, over):
                                       bad, g.workspace, g.ws_bytes, g.dev_error)
     torch.cuda.synchronize()
     assert g.error() == pkv.PKV_DEVERR_SEQ_ORDER
+
+
+@pytest.mark.parametrize("name,over,seqs,beam", [
+    ("gqa_prefix", dict(num_seqs=4, prefix_blocks=8, private_blocks=9), None, False),
+    ("gqa_prefix", dict(num_seqs=5, prefix_blocks=3, private_blocks=2, block_size=32), None, False),
+    ("gqa_prefix", dict(num_seqs=40, prefix_blocks=2, private_blocks=1), None, False),  # a group > 128 columns
+    ("mixed", dict(num_seqs=24, children=4), None, False),
+    ("mixed", dict(num_seqs=24, children=4), None, True),
+    ("gqa_prefix", {}, [0, 33, 63], False),
+    ("mixed", {}, "pairs", True),
+])
+def test_shared_prefix_decode(name, over, seqs, beam):
+    """pkv_paged_attention_decode_ex with shared-prefix groups (each shared block attended once per
+    group by the prefix pass, merged into the decode) gives the oracle's outputs."""
+    from paged_block_quantized_b200.step import DeviceStep
+    w = W.make(name, seed=0, **over)
+    g = DeviceStep(w, shared_prefix=True, beam_order=beam)
+    assert g.prefix is not None
+    g.prefill()
+    g.step()
+    torch.cuda.synchronize()
+    assert g.error() == 0
+    if seqs == "pairs":  # two parent/child pairs and the longest sequence
+        members = g.members.cpu().numpy()
+        seqs = [int(x) for x in members[:4]] + [int(np.argmax(w.context_lens))]
+    o = oracle_step(w, seqs)
+    out = g.out.float().cpu().numpy()[o["seqs"]]
+    err = np.abs(out - o["out"]).max()
+    assert err <= TOL, f"max abs error {err}"
+
+
+def test_shared_prefix_count_beyond_the_sequence_is_flagged():
+    from paged_block_quantized_b200 import pkv
+    from paged_block_quantized_b200.step import DeviceStep
+    w = W.make("gqa_prefix", seed=1, num_seqs=3, prefix_blocks=2, private_blocks=1)
+    g = DeviceStep(w, shared_prefix=True)
+    g.prefill()
+    g.step()
+    torch.cuda.synchronize()
+    ref = g.out.clone()
+    # a count covering every block of the sequences: clamped to leave the last block, reported
+    g.shared_blocks.fill_(3)
+    g.prefix["max_shared_blocks"] = 3
+    g.ws_bytes = pkv.pkv_decode_ex_workspace_size(g.pool.desc, w.num_seqs, w.num_q_heads, w.max_context_len,
+                                                  g.partition_tokens, None, g.prefix)
+    g.workspace = torch.zeros(g.ws_bytes, dtype=torch.uint8, device="cuda")
+    g.dev_error.zero_()
+    g.decode()
+    torch.cuda.synchronize()
+    assert g.error() == pkv.PKV_DEVERR_SHARED
+    assert (g.out.float() - ref.float()).abs().max().item() <= 1e-3
