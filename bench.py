@@ -442,6 +442,83 @@ def run_pkv(args, rank, world, local):
     return line
 
 
+# ----------------------------------------------------------------------------- chunked prefill
+def run_prefill(args, rank, world, local):
+    """--config prefill: one step = store every sequence's chunk (quantize + scatter) and the causal
+    attention of the chunk's queries over the cache (pkv_paged_attention_prefill). Tensor-bound:
+    the roofline is the attention's multiply-add FLOPs over the prefill kernel's duration."""
+    import torch
+    from paged_block_quantized_b200 import workloads as W
+    from paged_block_quantized_b200.step import PrefillStep
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = W.make(args.config, seed=args.seed + rank)
+    g = PrefillStep(w, device=dev, poison=None)
+    g.prefill()
+    stream = torch.cuda.current_stream(dev)
+    flush = L2Flush(dev)
+    for _ in range(args.warmup):
+        flush()
+        g.step()
+    torch.cuda.synchronize(dev)
+    assert g.error() == 0, f"device error {g.error()} in warm-up"
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    props = torch.cuda.get_device_properties(dev)
+    smi_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) is not None else str(dev.index)
+    with ClockSampler(smi_id, enabled=not args.no_clocks) as clk:
+        dist_barrier(world, dev)
+        torch.cuda.synchronize(dev)
+        for i in range(K):
+            flush()
+            ev[i][0].record(stream)
+            g.store()
+            ev[i][1].record(stream)
+            g.attend()
+            ev[i][2].record(stream)
+        torch.cuda.synchronize(dev)
+        dist_barrier(world, dev)
+    step_ms = [ev[i][0].elapsed_time(ev[i][2]) for i in range(K)]
+    att_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+    total_s = dist_max(sum(step_ms) / 1e3, world, dev)
+    q_tokens = float(w.q_lens.sum())
+    tokens_all = dist_sum(q_tokens * K, world, dev)
+    att_s = dist_max(statistics.mean(att_ms) / 1e3, world, dev)
+    flops = w.prefill_flops()
+    peak = 1590.0  # TFLOP/s, dense bf16/fp16 (recipe fallback: MEASURED_PEAKS.json has no entry here)
+    peak_src = "fallback 1.59 PFLOP/s dense fp16/bf16 (earlier cuBLAS measurement on this pool)"
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            mp = json.load(f)
+        if "bf16_tflops" in mp:
+            peak, peak_src = float(mp["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops, cuBLAS burst)"
+    except (OSError, ValueError):
+        pass
+    achieved = flops / att_s / 1e12
+    assert g.error() == 0, f"device error {g.error()}"
+    line = {
+        "metric": "chunked-prefill query tokens/s over the paged INT8 cache", "value": tokens_all / total_s,
+        "unit": "query tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": total_s * 1e3 / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": dtype_label(w), "data": "synthetic (seeded N(0,1) fp16 K/V/q, permuted block pool)",
+        "config": {"workload": f"{w.name}: {w.description}", "num_seqs": w.num_seqs, "num_q_heads": w.num_q_heads,
+                   "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "block_size": w.block_size,
+                   "query_tokens_per_step": int(q_tokens), "context_tokens": w.total_tokens,
+                   "step": "store the chunks (quantize+scatter) + chunked-prefill attention",
+                   "parallelism": f"dp{world}", "l2": "flushed before every timed step"},
+        "prefill_attention_us": att_s * 1e6,
+        "roofline": {"bound": "tensor", "kernel": "paged_prefill_kernel", "achieved": achieved, "peak": peak,
+                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                     "algorithmic_flops_per_launch": flops, "peak_source": peak_src},
+        "gpu_launches": 2 * K,
+    }
+    clocks = clk.summary()
+    if clocks is not None:
+        line["clocks"] = clocks
+    return line
+
+
 # ----------------------------------------------------------------------------- reference arm
 def run_reference(args, rank, world):
     """The CPU oracle as the reference arm: each step decodes a bounded sample of the workload."""
@@ -493,6 +570,8 @@ def main():
     try:
         if args.impl == "reference":
             line = run_reference(args, rank, world)
+        elif args.config == "prefill":
+            line = run_prefill(args, rank, world, local)
         else:
             line = run_pkv(args, rank, world, local)
         if rank == 0 and line is not None:
