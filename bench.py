@@ -62,6 +62,8 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("pkv", "reference"), default="pkv")
+    ap.add_argument("--op", choices=("step", "swap"), default="step",
+                    help="step: the decode step (or the prefill step for --config prefill); swap: block swap")
     ap.add_argument("--config", default="mixed")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--partition-tokens", type=int, default=None)
@@ -519,6 +521,84 @@ def run_prefill(args, rank, world, local):
     return line
 
 
+# ----------------------------------------------------------------------------- block swap
+def run_swap(args, rank, world, local):
+    """--op swap: every block of a quarter of the workload's sequences (scattered physical ids) out to a
+    pinned host pool and back in (pkv_swap_blocks, one kernel each way). Reported: the bytes moved per
+    second each way, against a plain pinned-memory copy of the same byte count by the copy engines
+    (the host link's practical peak on this machine, measured in the same run)."""
+    import numpy as np
+    import torch
+    from paged_block_quantized_b200 import pkv
+    from paged_block_quantized_b200 import workloads as W
+    from paged_block_quantized_b200.step import DeviceStep
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = W.make(args.config, seed=args.seed + rank)
+    g = DeviceStep(w, device=dev, poison=None)
+    g.prefill()
+    bs = w.block_size
+    seqs = list(range(0, w.num_seqs, 4))
+    ids = sorted(set(int(b) for s_ in seqs for b in w.block_tables[s_, :(int(w.context_lens[s_]) + bs - 1) // bs]))
+    n = len(ids)
+    host = pkv.DevicePool.allocate(n, bs, w.num_kv_heads, w.head_dim, w.k_dtype, w.v_dtype, pinned_host=True)
+    out_map = torch.tensor(list(zip(ids, range(n))), dtype=torch.int32, device=dev)
+    in_map = torch.tensor(list(zip(range(n), ids)), dtype=torch.int32, device=dev)
+    nbytes = host.nbytes()
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        pkv.pkv_swap_blocks(g.pool.desc, host.desc, out_map, n, pkv.PKV_SWAP_OUT, g.dev_error)
+        pkv.pkv_swap_blocks(g.pool.desc, host.desc, in_map, n, pkv.PKV_SWAP_IN, g.dev_error)
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    for i in range(K):
+        ev[i][0].record(stream)
+        pkv.pkv_swap_blocks(g.pool.desc, host.desc, out_map, n, pkv.PKV_SWAP_OUT, g.dev_error)
+        ev[i][1].record(stream)
+        pkv.pkv_swap_blocks(g.pool.desc, host.desc, in_map, n, pkv.PKV_SWAP_IN, g.dev_error)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize(dev)
+    assert g.error() == 0
+    out_s = statistics.mean(ev[i][0].elapsed_time(ev[i][1]) for i in range(K)) / 1e3
+    in_s = statistics.mean(ev[i][1].elapsed_time(ev[i][2]) for i in range(K)) / 1e3
+    # the copy engines on one contiguous pinned buffer of the same size, each way
+    hbuf = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+    dbuf = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        dbuf.copy_(hbuf, non_blocking=True)
+        hbuf.copy_(dbuf, non_blocking=True)
+    torch.cuda.synchronize(dev)
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    e[0].record(stream)
+    for _ in range(K):
+        hbuf.copy_(dbuf, non_blocking=True)
+    e[1].record(stream)
+    for _ in range(K):
+        dbuf.copy_(hbuf, non_blocking=True)
+    e[2].record(stream)
+    torch.cuda.synchronize(dev)
+    d2h_peak = nbytes * K / (e[0].elapsed_time(e[1]) / 1e3) / 1e9
+    h2d_peak = nbytes * K / (e[1].elapsed_time(e[2]) / 1e3) / 1e9
+    out_gbs, in_gbs = nbytes / out_s / 1e9, nbytes / in_s / 1e9
+    return {
+        "metric": "block swap GB/s (device pool <-> pinned host pool)", "value": (2 * nbytes) / (out_s + in_s) / 1e9,
+        "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": (out_s + in_s) * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": dtype_label(w), "data": "synthetic",
+        "config": {"workload": f"{w.name}: every block of {len(seqs)} of {w.num_seqs} sequences ({n} scattered blocks, "
+                               f"{nbytes} bytes with scales and zero points)", "parallelism": f"dp{world}"},
+        "swap_out_gbs": out_gbs, "swap_in_gbs": in_gbs,
+        "roofline": {"bound": "host link", "kernel": "swap_blocks_kernel", "achieved": (out_gbs + in_gbs) / 2,
+                     "peak": (d2h_peak + h2d_peak) / 2, "unit": "GB/s",
+                     "frac": ((out_gbs / d2h_peak) + (in_gbs / h2d_peak)) / 2, "traffic": None,
+                     "peak_source": f"measured in this run: pinned copies by the copy engines, "
+                                    f"device->host {d2h_peak:.1f} GB/s, host->device {h2d_peak:.1f} GB/s"},
+        "gpu_launches": 2 * K,
+    }
+
+
 # ----------------------------------------------------------------------------- reference arm
 def run_reference(args, rank, world):
     """The CPU oracle as the reference arm: each step decodes a bounded sample of the workload."""
@@ -570,6 +650,8 @@ def main():
     try:
         if args.impl == "reference":
             line = run_reference(args, rank, world)
+        elif args.op == "swap":
+            line = run_swap(args, rank, world, local)
         elif args.config == "prefill":
             line = run_prefill(args, rank, world, local)
         else:

@@ -421,6 +421,14 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+// integer tensor cores: m16n8k32, signed 8-bit operands, int32 accumulators
+__device__ __forceinline__ void imma_16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                           uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
   uint32_t y;
   asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
@@ -457,8 +465,14 @@ struct MmaEngine {
   using C = Cfg<KT, VT, BS, D, GT>;
   static constexpr int KS = D / 16;  // q.k steps and p.v dim tiles
   static_assert(BS % 16 == 0, "16-token slices");
+  // INT8 K: q.k on the integer tensor cores, the codes as they sit in shared memory against q on a
+  // 22-bit fixed-point grid per head split into three signed byte planes (exact, as in the
+  // CUDA-core engine); otherwise K is turned into fp16 and multiplied with fp16 q.
+  static constexpr bool IMMA = KT == PKV_INT8_SYM;
   int g, c;
-  uint32_t qb[KS][2];
+  uint32_t qb[IMMA ? 1 : KS][2];
+  uint32_t qp8[IMMA ? 3 : 1][IMMA ? KS / 2 : 1][2];  // planes, k32-steps, (b0, b1)
+  float qz[2];                                       // 2^-shift of heads 2c, 2c+1
   float acc[KS][4];
   float m_run[2], l_run[2];
 
@@ -472,7 +486,69 @@ struct MmaEngine {
   __device__ __forceinline__ void begin(const DecodeParams& p, int s, int hg, int lane) {
     g = lane >> 2;
     c = lane & 3;
-    // q^T fragments: head g of the group, dims [c*D/4, (c+1)*D/4) as 2*KS half2 words
+    if constexpr (IMMA) {
+      // head g of the group, dims [c*D/4, (c+1)*D/4); k32-step kk holds dims c*D/4 + 8kk + [0,4) (b0)
+      // and + [4,8) (b1), the same dims as the A fragments of the K rows below
+      float x[D / 4];
+      if (g < GT) {
+        const uint4* qp = reinterpret_cast<const uint4*>(p.q + ((size_t)s * p.num_q_heads + (size_t)hg * GT + g) * D +
+                                                         c * (D / 4));
+#pragma unroll
+        for (int i = 0; i < D / 32; ++i) {
+          const uint4 wv = qp[i];
+          const uint32_t u[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&u[k]));
+            x[8 * i + 2 * k] = f.x;
+            x[8 * i + 2 * k + 1] = f.y;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < D / 4; ++i) x[i] = 0.f;
+      }
+      float amax = 0.f;
+#pragma unroll
+      for (int i = 0; i < D / 4; ++i) amax = fmaxf(amax, fabsf(x[i]));
+      amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
+      int ex = 0;
+      (void)frexpf(amax, &ex);                    // amax < 2^ex
+      const int shift = amax > 0.f ? 22 - ex : 0;  // |q| * 2^shift < 2^22
+      const float up = __int_as_float((127 + shift) << 23);
+      const float qinv = __int_as_float((127 - shift) << 23);
+      qz[0] = __shfl_sync(kFull, qinv, 8 * c);      // head 2c lives on lanes 4 (2c) + ..
+      qz[1] = __shfl_sync(kFull, qinv, 8 * c + 4);  // head 2c + 1
+#pragma unroll
+      for (int kk = 0; kk < KS / 2; ++kk) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t p0 = 0, p1 = 0, p2 = 0;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int qi = __float2int_rn(x[8 * kk + 4 * h + k] * up);
+            const int b0 = ((qi + 128) & 0xFF) - 128;
+            const int r1 = (qi - b0) >> 8;
+            const int b1 = ((r1 + 128) & 0xFF) - 128;
+            const int b2 = (r1 - b1) >> 8;
+            p0 |= (uint32_t)(b0 & 0xFF) << (8 * k);
+            p1 |= (uint32_t)(b1 & 0xFF) << (8 * k);
+            p2 |= (uint32_t)(b2 & 0xFF) << (8 * k);
+          }
+          qp8[0][kk][h] = p0;
+          qp8[1][kk][h] = p1;
+          qp8[2][kk][h] = p2;
+        }
+      }
+    } else {
+      load_q16(p, s, hg);
+    }
+    reset();
+  }
+
+  // q^T fragments (fp16 K): head g of the group, dims [c*D/4, (c+1)*D/4) as 2*KS half2 words
+  __device__ __forceinline__ void load_q16(const DecodeParams& p, int s, int hg) {
 #pragma unroll
     for (int j = 0; j < KS; ++j) qb[j][0] = qb[j][1] = 0u;
     if (g < GT) {
@@ -487,7 +563,6 @@ struct MmaEngine {
         qb[2 * i + 1][1] = w.w;
       }
     }
-    reset();
   }
 
   __device__ __forceinline__ void block(const uint8_t* kt, const uint8_t* vt, float ks, float vs, float /*nzb*/,
@@ -499,24 +574,24 @@ struct MmaEngine {
       float sacc[4] = {0.f, 0.f, 0.f, 0.f};
       const int kr0 = 16 * h2 + g, kx = c * (C::K_ROW / 4);  // rows kr0, kr0 + 8 from byte kx
       if constexpr (KT == PKV_INT8_SYM) {
+        int ia[3][4];
 #pragma unroll
-        for (int i = 0; i < KS / 4; ++i) {  // 16 codes = 4 steps per 16-byte load
+        for (int pl = 0; pl < 3; ++pl) ia[pl][0] = ia[pl][1] = ia[pl][2] = ia[pl][3] = 0;
+#pragma unroll
+        for (int i = 0; i < KS / 4; ++i) {  // 16 codes = 2 k32-steps per 16-byte load
           const uint4 r0 = *reinterpret_cast<const uint4*>(kt + swz<C::K_ROW>(kr0, kx + 16 * i));
           const uint4 r1 = *reinterpret_cast<const uint4*>(kt + swz<C::K_ROW>(kr0 + 8, kx + 16 * i));
-          const uint32_t w0[4] = {r0.x, r0.y, r0.z, r0.w};
-          const uint32_t w1[4] = {r1.x, r1.y, r1.z, r1.w};
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const uint32_t u0 = w0[q4] ^ 0x80808080u, u1 = w1[q4] ^ 0x80808080u;
-            uint32_t a[4];
-            a[0] = h2_sub(__byte_perm(u0, 0x64646464u, 0x4140), kH2Bias);  // row g, dims +0,+1
-            a[1] = h2_sub(__byte_perm(u1, 0x64646464u, 0x4140), kH2Bias);  // row g+8
-            a[2] = h2_sub(__byte_perm(u0, 0x64646464u, 0x4342), kH2Bias);  // row g, dims +2,+3
-            a[3] = h2_sub(__byte_perm(u1, 0x64646464u, 0x4342), kH2Bias);  // row g+8
-            const int kk = 4 * i + q4;
-            mma_16816(sacc, a, qb[kk][0], qb[kk][1]);
+          for (int pl = 0; pl < 3; ++pl) {
+            imma_16832(ia[pl], r0.x, r1.x, r0.y, r1.y, qp8[pl][2 * i][0], qp8[pl][2 * i][1]);
+            imma_16832(ia[pl], r0.z, r1.z, r0.w, r1.w, qp8[pl][2 * i + 1][0], qp8[pl][2 * i + 1][1]);
           }
         }
+        // |plane sums| < 2^18: the low two combine exactly in int32, the top one in fp32; then
+        // the head's 2^-shift (columns 2c, 2c+1)
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+          sacc[r] = __fmaf_rn((float)ia[2][r], 65536.f, (float)(ia[1][r] * 256 + ia[0][r])) * qz[r & 1];
       } else if constexpr (KT == PKV_FP8_E4M3) {
 #pragma unroll
         for (int i = 0; i < KS / 4; ++i) {  // 16 codes = 4 steps per 16-byte load
