@@ -71,9 +71,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
-    ap.add_argument("--no-beam-order", action="store_true",
-                    help="walk the sequences in index order instead of each forked child right after its parent")
-    ap.add_argument("--shared-prefix", choices=("auto", "on", "off"), default="auto",
+    ap.add_argument("--beam-order", action="store_true",
+                    help="walk each forked child right after its parent instead of in index order")
+    ap.add_argument("--shared-prefix", choices=("auto", "on", "off"), default="off",
                     help="attend blocks shared by a group of sequences once per group (auto: when a group has "
                          "more than two members)")
     ap.add_argument("--fused", action="store_true",
@@ -306,7 +306,7 @@ def run_pkv(args, rank, world, local):
     shared = args.shared_prefix == "on" or (
         args.shared_prefix == "auto" and groups is not None and int(np.diff(groups[0]).max()) > 2)
     g = DeviceStep(w, device=dev, poison=None, partition_tokens=args.partition_tokens,
-                   beam_order=not args.no_beam_order, shared_prefix=shared and not args.fused)
+                   beam_order=args.beam_order, shared_prefix=shared and not args.fused)
     g.prefill()
     g.snapshot_step_tiles()
     has_cow = w.cow_pairs.shape[0] > 0

@@ -46,7 +46,7 @@ bool encode_tile_map(CUtensorMap* map, const void* base, uint64_t rows, int row_
 }
 
 int32_t decode_heads_per_warp(int32_t group, int32_t k_dtype, int32_t v_dtype, int32_t head_dim) {
-  const bool mma = (k_dtype == PKV_INT8_SYM && v_dtype == PKV_INT8_SYM && head_dim >= 128) ||
+  const bool mma = (k_dtype == PKV_INT8_SYM && (v_dtype == PKV_INT8_SYM || v_dtype == PKV_INT4_ASYM) && head_dim >= 128) ||
                    (k_dtype == PKV_FP16 && v_dtype == PKV_FP16) || (k_dtype == PKV_FP8_E4M3 && v_dtype == PKV_FP8_E4M3);
   if (mma && group % 8 == 0) return 8;
   if (group % 4 == 0) return 4;

@@ -65,6 +65,11 @@ constexpr float kNegBig = -1.0e30f;  // finite "minus infinity" for running maxi
 #ifndef PKV_DECODE_WARPS_SM
 #define PKV_DECODE_WARPS_SM 0  // 0: by engine, as above
 #endif
+// INT8 K with one or two query heads per KV head (MHA) on the tensor-core engine (1) or on the
+// CUDA-core engine's dp4a planes (0).
+#ifndef PKV_DECODE_MMA_MHA
+#define PKV_DECODE_MMA_MHA 1
+#endif
 #ifndef PKV_DECODE_MAX_STAGES
 #define PKV_DECODE_MAX_STAGES 6
 #endif
@@ -76,12 +81,16 @@ struct Cfg {
   static constexpr int K_TILE = BS * K_ROW;
   static constexpr int V_TILE = BS * V_ROW;
   static constexpr int STAGE = K_TILE + V_TILE;
-  // tensor-core engine for groups of 4 or 8 query heads (INT8/INT8 with D >= 128, FP16/FP16), and
-  // for every group size with E4M3 codes (their conversion to fp16 is one instruction per pair)
+  // tensor-core engine: INT8 K (q.k on the integer tensor cores) with INT8 or INT4 V and E4M3 codes
+  // (one conversion per pair) for every group size with D >= 128 (MHA INT8 K only with
+  // PKV_DECODE_MMA_MHA); FP16/FP16 for groups of 4 or 8 query heads
   static constexpr bool FP8 = KT == PKV_FP8_E4M3 && VT == PKV_FP8_E4M3;
-  static constexpr bool MMA =
-      (GT >= 4 && ((KT == PKV_INT8_SYM && VT == PKV_INT8_SYM && D >= 128) || (KT == PKV_FP16 && VT == PKV_FP16))) ||
-      (FP8 && D >= 128);
+  static constexpr bool I8K = KT == PKV_INT8_SYM && (VT == PKV_INT8_SYM || VT == PKV_INT4_ASYM);
+  static constexpr bool MMA = (D >= 128 && I8K && (GT >= 4 || PKV_DECODE_MMA_MHA)) ||
+                              (GT >= 4 && KT == PKV_FP16 && VT == PKV_FP16) || (FP8 && D >= 128);
+  // the V tile arrives swizzled (tiled copy) when its rows are whole 128-byte units, else by a 1-D
+  // bulk copy (INT4 rows of D/2 bytes)
+  static constexpr bool V_SWZ = V_ROW % 128 == 0;
   static constexpr int WARPS_AUTO =
       MMA ? (D >= 256 ? 8 : 12) : (KT == PKV_FP16 ? 8 : (GT == 1 ? 16 : (GT == 2 ? 12 : 8)));
   static constexpr int WARPS_WANT = PKV_DECODE_WARPS_SM > 0 ? PKV_DECODE_WARPS_SM : WARPS_AUTO;
@@ -99,7 +108,8 @@ struct Cfg {
   static constexpr int CTAS_PER_SM = 1;
   static_assert(D % 16 == 0 && D / 16 <= 32, "head_dim");
   static_assert(K_TILE % 16 == 0 && V_TILE % 16 == 0 && STAGE % 16 == 0, "bulk copy granularity");
-  static_assert(!MMA || (K_ROW % 128 == 0 && V_ROW % 128 == 0 && K_TILE % 1024 == 0 && V_TILE % 1024 == 0),
+  static_assert(!MMA || (K_ROW % 128 == 0 && K_TILE % 1024 == 0 && STAGE % 1024 == 0 &&
+                          (!V_SWZ || V_TILE % 1024 == 0)),
                 "swizzled tiles: 128-byte row units, 1024-byte aligned tiles");
   static_assert(NW >= 1 && SMEM <= 227 * 1024, "shared memory per CTA");
 };
@@ -565,7 +575,7 @@ struct MmaEngine {
     }
   }
 
-  __device__ __forceinline__ void block(const uint8_t* kt, const uint8_t* vt, float ks, float vs, float /*nzb*/,
+  __device__ __forceinline__ void block(const uint8_t* kt, const uint8_t* vt, float ks, float vs, float nzb,
                                         bool valid, int tok0, int L, float scale_log2) {
     const float zscale = (KT == PKV_FP16) ? scale_log2 : ks;
 #pragma unroll
@@ -684,6 +694,35 @@ struct MmaEngine {
             a[1] = h2_sub((__byte_perm(xa[wd], xb[wd], sel1) & 0x00FF00FFu) ^ kH2Bias, kH2Bias);
             a[2] = h2_sub((__byte_perm(xc[wd], xd[wd], sel0) & 0x00FF00FFu) ^ kH2Bias, kH2Bias);
             a[3] = h2_sub((__byte_perm(xc[wd], xd[wd], sel1) & 0x00FF00FFu) ^ kH2Bias, kH2Bias);
+            const int j = 8 * i + jj;
+            mma_16816(acc[j], a, bh0, bh1);
+            mma_16816(acc[j], a, bl0, bl1);
+          }
+        }
+      } else if constexpr (VT == PKV_INT4_ASYM) {
+        // unswizzled rows of D/2 bytes: dims [g*D/8, (g+1)*D/8) of a row are D/16 bytes, byte jj
+        // holding dims 2jj (low nibble, M row g) and 2jj+1 (high nibble, M row g+8) of a dim tile;
+        // (1024 + nibble) as fp16 minus (1024 + zp) is the exact (code - zp)
+        const float zp = -(nzb + kMagic);
+        const uint32_t bias = h2_pack(1024.f + zp, 1024.f + zp);
+        const int vb = g * (D / 16);
+#pragma unroll
+        for (int i = 0; i < KS / 8; ++i) {  // 8 bytes per row = 8 dim tiles
+          const uint2 ra = *reinterpret_cast<const uint2*>(vt + vr * C::V_ROW + vb + 8 * i);
+          const uint2 rb = *reinterpret_cast<const uint2*>(vt + (vr + 1) * C::V_ROW + vb + 8 * i);
+          const uint2 rc = *reinterpret_cast<const uint2*>(vt + (vr + 8) * C::V_ROW + vb + 8 * i);
+          const uint2 rd = *reinterpret_cast<const uint2*>(vt + (vr + 9) * C::V_ROW + vb + 8 * i);
+          const uint32_t xa[2] = {ra.x, ra.y}, xb[2] = {rb.x, rb.y}, xc[2] = {rc.x, rc.y}, xd[2] = {rd.x, rd.y};
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) {
+            const int wd = jj / 4, k = jj % 4;
+            const uint32_t sel = k | ((4 + k) << 8);  // {first.b_k, -, second.b_k, -}
+            const uint32_t pab = __byte_perm(xa[wd], xb[wd], sel), pcd = __byte_perm(xc[wd], xd[wd], sel);
+            uint32_t a[4];
+            a[0] = h2_sub((pab & 0x000F000Fu) | 0x64006400u, bias);
+            a[1] = h2_sub(((pab >> 4) & 0x000F000Fu) | 0x64006400u, bias);
+            a[2] = h2_sub((pcd & 0x000F000Fu) | 0x64006400u, bias);
+            a[3] = h2_sub(((pcd >> 4) & 0x000F000Fu) | 0x64006400u, bias);
             const int j = 8 * i + jj;
             mma_16816(acc[j], a, bh0, bh1);
             mma_16816(acc[j], a, bl0, bl1);
@@ -1164,7 +1203,10 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
       const int row = (int)(tile * BS);
       if constexpr (C::K_ROW == 128) tma_load_2d(dst, &tm.k, 0, row, &my_bars[st]);
       else tma_load_3d(dst, &tm.k, 0, 0, row, &my_bars[st]);
-      if constexpr (C::V_ROW == 128) tma_load_2d(dst + C::K_TILE, &tm.v, 0, row, &my_bars[st]);
+      if constexpr (!C::V_SWZ)
+        bulk_g2s(dst + C::K_TILE, static_cast<const uint8_t*>(p.v_codes) + tile * C::V_TILE, (uint32_t)C::V_TILE,
+                 &my_bars[st]);
+      else if constexpr (C::V_ROW == 128) tma_load_2d(dst + C::K_TILE, &tm.v, 0, row, &my_bars[st]);
       else tma_load_3d(dst + C::K_TILE, &tm.v, 0, 0, row, &my_bars[st]);
     } else {
       bulk_g2s(dst, static_cast<const uint8_t*>(p.k_codes) + tile * C::K_TILE, (uint32_t)C::K_TILE, &my_bars[st]);
@@ -1360,8 +1402,8 @@ cudaError_t launch_one(const DecodeParams& p, const StepParams& sp, const Decode
   memset(&tm, 0, sizeof(tm));
   if constexpr (C::MMA) {
     const uint64_t rows = (uint64_t)p.num_blocks * p.num_kv_heads * BS;
-    if (!encode_tile_map(&tm.k, p.k_codes, rows, C::K_ROW, BS) || !encode_tile_map(&tm.v, p.v_codes, rows, C::V_ROW, BS))
-      return cudaErrorInvalidValue;
+    if (!encode_tile_map(&tm.k, p.k_codes, rows, C::K_ROW, BS)) return cudaErrorInvalidValue;
+    if (C::V_SWZ && !encode_tile_map(&tm.v, p.v_codes, rows, C::V_ROW, BS)) return cudaErrorInvalidValue;
   }
   return cudaLaunchKernelEx(&cfg, kern, p, sp, tm);
 }

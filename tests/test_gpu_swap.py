@@ -27,8 +27,18 @@ def _pools(w, host_blocks):
 
 
 def _arrays(pool):
-    return [t.cpu().numpy().view(np.uint8) for t in (pool.k_codes, pool.v_codes, pool.k_scale, pool.v_scale,
-                                                     pool.v_zp)]
+    """The arrays a swap moves for this pool's dtypes: codes always, scales of quantized sides, zero
+    points of INT4 V (the others are not part of the cache and keep whatever they held)."""
+    from paged_block_quantized_b200 import pkv
+    d = pool.desc
+    arrs = [pool.k_codes, pool.v_codes]
+    if d.k_dtype != pkv.PKV_FP16:
+        arrs.append(pool.k_scale)
+    if d.v_dtype != pkv.PKV_FP16:
+        arrs.append(pool.v_scale)
+    if d.v_dtype == pkv.PKV_INT4_ASYM:
+        arrs.append(pool.v_zp)
+    return [t.cpu().numpy().view(np.uint8) for t in arrs]
 
 
 @pytest.mark.parametrize("name,over", [("mixed", dict(num_seqs=10, children=2)), ("llama7b_fp16", dict(num_seqs=3))])
