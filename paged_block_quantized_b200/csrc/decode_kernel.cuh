@@ -66,9 +66,16 @@ constexpr float kNegBig = -1.0e30f;  // finite "minus infinity" for running maxi
 #define PKV_DECODE_WARPS_SM 0  // 0: by engine, as above
 #endif
 // INT8 K with one or two query heads per KV head (MHA) on the tensor-core engine (1) or on the
-// CUDA-core engine's dp4a planes (0).
+// CUDA-core engine's dp4a planes (0, measured faster: 62.8 vs 81.9 us on the Llama-2-7B-shaped
+// batch; the warp-level MMA pipe, not memory, limits the former at one useful column in eight).
 #ifndef PKV_DECODE_MMA_MHA
-#define PKV_DECODE_MMA_MHA 1
+#define PKV_DECODE_MMA_MHA 0
+#endif
+// INT8 K in the tensor-core engine: q.k on the integer tensor cores against three exact byte
+// planes of q (1), or the codes turned into fp16 and multiplied with fp16 q (0, measured faster:
+// 74.8 vs 78.4 us on the GQA shared-prefix batch; the integer MMAs triple the tensor-pipe work).
+#ifndef PKV_DECODE_IMMA_QK
+#define PKV_DECODE_IMMA_QK 0
 #endif
 #ifndef PKV_DECODE_MAX_STAGES
 #define PKV_DECODE_MAX_STAGES 6
@@ -88,9 +95,9 @@ struct Cfg {
   static constexpr bool I8K = KT == PKV_INT8_SYM && (VT == PKV_INT8_SYM || VT == PKV_INT4_ASYM);
   static constexpr bool MMA = (D >= 128 && I8K && (GT >= 4 || PKV_DECODE_MMA_MHA)) ||
                               (GT >= 4 && KT == PKV_FP16 && VT == PKV_FP16) || (FP8 && D >= 128);
-  // the V tile arrives swizzled (tiled copy) when its rows are whole 128-byte units, else by a 1-D
-  // bulk copy (INT4 rows of D/2 bytes)
-  static constexpr bool V_SWZ = V_ROW % 128 == 0;
+  // the V tile arrives swizzled (tiled copy) when its rows are whole 128-byte units; INT4 V always
+  // by a 1-D bulk copy (its reads below index unswizzled rows of D/2 bytes)
+  static constexpr bool V_SWZ = V_ROW % 128 == 0 && VT != PKV_INT4_ASYM;
   static constexpr int WARPS_AUTO =
       MMA ? (D >= 256 ? 8 : 12) : (KT == PKV_FP16 ? 8 : (GT == 1 ? 16 : (GT == 2 ? 12 : 8)));
   static constexpr int WARPS_WANT = PKV_DECODE_WARPS_SM > 0 ? PKV_DECODE_WARPS_SM : WARPS_AUTO;
@@ -478,7 +485,7 @@ struct MmaEngine {
   // INT8 K: q.k on the integer tensor cores, the codes as they sit in shared memory against q on a
   // 22-bit fixed-point grid per head split into three signed byte planes (exact, as in the
   // CUDA-core engine); otherwise K is turned into fp16 and multiplied with fp16 q.
-  static constexpr bool IMMA = KT == PKV_INT8_SYM;
+  static constexpr bool IMMA = KT == PKV_INT8_SYM && PKV_DECODE_IMMA_QK;
   int g, c;
   uint32_t qb[IMMA ? 1 : KS][2];
   uint32_t qp8[IMMA ? 3 : 1][IMMA ? KS / 2 : 1][2];  // planes, k32-steps, (b0, b1)
@@ -583,7 +590,7 @@ struct MmaEngine {
       // ---- S = K . q^T over this 16-token slice ----
       float sacc[4] = {0.f, 0.f, 0.f, 0.f};
       const int kr0 = 16 * h2 + g, kx = c * (C::K_ROW / 4);  // rows kr0, kr0 + 8 from byte kx
-      if constexpr (KT == PKV_INT8_SYM) {
+      if constexpr (KT == PKV_INT8_SYM && IMMA) {
         int ia[3][4];
 #pragma unroll
         for (int pl = 0; pl < 3; ++pl) ia[pl][0] = ia[pl][1] = ia[pl][2] = ia[pl][3] = 0;
@@ -602,6 +609,25 @@ struct MmaEngine {
 #pragma unroll
         for (int r = 0; r < 4; ++r)
           sacc[r] = __fmaf_rn((float)ia[2][r], 65536.f, (float)(ia[1][r] * 256 + ia[0][r])) * qz[r & 1];
+      } else if constexpr (KT == PKV_INT8_SYM) {
+#pragma unroll
+        for (int i = 0; i < KS / 4; ++i) {  // 16 codes = 4 steps per 16-byte load
+          const uint4 r0 = *reinterpret_cast<const uint4*>(kt + swz<C::K_ROW>(kr0, kx + 16 * i));
+          const uint4 r1 = *reinterpret_cast<const uint4*>(kt + swz<C::K_ROW>(kr0 + 8, kx + 16 * i));
+          const uint32_t w0[4] = {r0.x, r0.y, r0.z, r0.w};
+          const uint32_t w1[4] = {r1.x, r1.y, r1.z, r1.w};
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const uint32_t u0 = w0[q4] ^ 0x80808080u, u1 = w1[q4] ^ 0x80808080u;
+            uint32_t a[4];
+            a[0] = h2_sub(__byte_perm(u0, 0x64646464u, 0x4140), kH2Bias);  // row g, dims +0,+1
+            a[1] = h2_sub(__byte_perm(u1, 0x64646464u, 0x4140), kH2Bias);  // row g+8
+            a[2] = h2_sub(__byte_perm(u0, 0x64646464u, 0x4342), kH2Bias);  // row g, dims +2,+3
+            a[3] = h2_sub(__byte_perm(u1, 0x64646464u, 0x4342), kH2Bias);  // row g+8
+            const int kk = 4 * i + q4;
+            mma_16816(sacc, a, qb[kk][0], qb[kk][1]);
+          }
+        }
       } else if constexpr (KT == PKV_FP8_E4M3) {
 #pragma unroll
         for (int i = 0; i < KS / 4; ++i) {  // 16 codes = 4 steps per 16-byte load

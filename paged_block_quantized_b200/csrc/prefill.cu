@@ -3,6 +3,13 @@
 #include <cstring>
 
 #include "prefill_kernel.cuh"
+#include "prefill_tc.cuh"
+
+// 1: the fifth-generation tensor-core kernel (prefill_tc.cuh); 0: the warp-level mma kernel
+// (prefill_kernel.cuh)
+#ifndef PKV_PREFILL_TC
+#define PKV_PREFILL_TC 1
+#endif
 
 namespace pkv {
 
@@ -15,8 +22,15 @@ namespace {
 
 template <int VT, int BS, bool PREFIX>
 cudaError_t launch_prefill_t(const PrefillParams& p, int32_t n_groups, cudaStream_t stream) {
+#if PKV_PREFILL_TC
+  using C = prefill_tc::Cfg<VT, BS>;
+  auto kern = prefill_tc::paged_prefill_tc_kernel<VT, BS, PREFIX>;
+  constexpr int kThreads = prefill_tc::kThreads;
+#else
   using C = prefill_detail::Cfg<VT, BS>;
   auto kern = prefill_detail::paged_prefill_kernel<VT, BS, PREFIX>;
+  constexpr int kThreads = prefill_detail::kThreads;
+#endif
   static unsigned long long configured = 0;  // one bit per device; benign race
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -36,7 +50,7 @@ cudaError_t launch_prefill_t(const PrefillParams& p, int32_t n_groups, cudaStrea
   const int col_rows = PREFIX ? p.max_group_size : p.max_q_len;
   const int chunks = (col_rows * p.group + prefill_detail::kCols - 1) / prefill_detail::kCols;
   dim3 grid(chunks, p.num_kv_heads, PREFIX ? n_groups * p.splits : p.num_seqs);
-  kern<<<grid, prefill_detail::kThreads, C::SMEM, stream>>>(p, tm);
+  kern<<<grid, kThreads, C::SMEM, stream>>>(p, tm);
   return cudaGetLastError();
 }
 
