@@ -190,3 +190,50 @@ def test_swap_validation(pkv):
     assert swap(desc(pkv), mapping=0x6002) == E
     assert swap(desc(pkv), n=0) == pkv.PKV_OK
     assert swap(desc(pkv, k_codes=0x1008)) == E          # a misaligned host array
+
+
+def test_decode_ex_options_validation(pkv):
+    """pkv_paged_attention_decode_ex / pkv_decode_ex_workspace_size check their options on the host
+    (fake pointers, no device): the struct size, the shared-prefix bounds and the cache types the
+    shared-prefix pass is built for; the shared-prefix pass adds its partials to the workspace."""
+    import ctypes
+    d = desc(pkv, head_dim=128, v_dtype=pkv.PKV_INT8_SYM, v_zp=0)
+    prefix = dict(group_start=0x6000, members=0x6100, shared_blocks=0x6200, num_groups=1, num_members=2,
+                  max_group_size=2, max_shared_blocks=4)
+    base = pkv.pkv_decode_workspace_size(d, 2, 4, 256, 0)
+    assert pkv.pkv_decode_ex_workspace_size(d, 2, 4, 256, 0) == base
+    with_prefix = pkv.pkv_decode_ex_workspace_size(d, 2, 4, 256, 0, None, prefix)
+    assert with_prefix > base
+    dec = lambda **kw: pkv.pkv_paged_attention_decode_ex(
+        kw.get("desc", d), 0x9000, 0xA000, 2, 4, 0xB000, 16, 0xC000, 256, 0.1, 0, None, 0xD000,
+        kw.get("ws_bytes", 1 << 40), stream=0, raise_on_error=False, prefix=kw.get("prefix", prefix))
+    E = pkv.PKV_ERR_INVALID_ARG
+    assert dec(ws_bytes=base) == E                                    # too small for the partials
+    assert dec(prefix=dict(prefix, max_group_size=0)) == E
+    assert dec(prefix=dict(prefix, members=None)) == E
+    assert dec(prefix=dict(prefix, shared_blocks=0x6202)) == E         # misaligned
+    fp16 = desc(pkv, head_dim=128, k_dtype=pkv.PKV_FP16, v_dtype=pkv.PKV_FP16, k_scale=0, v_scale=0, v_zp=0)
+    assert dec(desc=fp16) == pkv.PKV_ERR_UNSUPPORTED                   # the pass is built for INT8 K
+    # a struct of another size is refused
+    opts = pkv.decode_options()
+    opts.struct_bytes = ctypes.sizeof(pkv.pkv_decode_options) + 8
+    st = pkv._decode_ex(ctypes.byref(d), 0x9000, 0xA000, 2, 4, 0xB000, 16, 0xC000, 256, 0.1, 0, ctypes.byref(opts),
+                        0xD000, 1 << 40, None, 0)
+    assert st == pkv.PKV_ERR_UNSUPPORTED
+
+
+def test_prefill_validation(pkv):
+    d = desc(pkv, head_dim=128, v_dtype=pkv.PKV_INT8_SYM, v_zp=0)
+    E = pkv.PKV_ERR_INVALID_ARG
+    pf = lambda **kw: pkv.pkv_paged_attention_prefill(
+        kw.get("desc", d), kw.get("out", 0x9000), 0xA000, kw.get("S", 2), kw.get("Hq", 4), 0xB000,
+        kw.get("T", 10), kw.get("maxq", 8), 0xC000, 16, 0xD000, 256, kw.get("scale", 0.1), stream=0,
+        raise_on_error=False)
+    assert pf(Hq=3) == E
+    assert pf(out=None) == E
+    assert pf(T=-1) == E
+    assert pf(scale=float("nan")) == E
+    assert pf(T=0) == pkv.PKV_OK and pf(S=0) == pkv.PKV_OK
+    assert pf(desc=desc(pkv, head_dim=64, v_dtype=pkv.PKV_INT8_SYM, v_zp=0)) == pkv.PKV_ERR_UNSUPPORTED
+    assert pf(desc=desc(pkv, head_dim=128, k_dtype=pkv.PKV_FP8_E4M3, v_dtype=pkv.PKV_FP8_E4M3,
+                        v_zp=0)) == pkv.PKV_ERR_UNSUPPORTED

@@ -76,3 +76,26 @@ def test_prefill_covers_positions_once():
         for p in range(int(w.context_lens[s]) - 1):
             expected.add(int(w.prefill_tables[s, p // w.block_size]) * w.block_size + p % w.block_size)
     assert seen == expected
+
+
+def test_beam_order_and_prefix_groups():
+    from paged_block_quantized_b200 import workloads as W
+    w = W.make("mixed", seed=0, num_seqs=24, children=4)
+    order = w.beam_walk_order()
+    assert sorted(order) == list(range(24))
+    for src, dst in w.cow_pairs:  # each child right after its parent
+        child = int(np.nonzero((w.block_tables == dst).any(axis=1))[0][0])
+        parent = int(np.nonzero((w.block_tables == src).any(axis=1))[0][0])
+        assert list(order).index(child) == list(order).index(parent) + 1
+    starts, members, shared = w.prefix_groups()
+    assert len(starts) == 5 and (np.diff(starts) == 2).all()
+    for g in range(4):
+        a, b = members[starts[g]:starts[g + 1]]
+        k = shared[a]
+        assert k == shared[b] > 0
+        assert (w.block_tables[a, :k] == w.block_tables[b, :k]).all()
+        assert w.block_tables[a, k] != w.block_tables[b, k]
+    g = W.make("gqa_prefix", seed=0, num_seqs=5, prefix_blocks=3, private_blocks=2)
+    starts, members, shared = g.prefix_groups()
+    assert list(starts) == [0, 5] and (shared == 3).all()
+    assert W.make("llama7b", seed=0, num_seqs=4).prefix_groups() is None
