@@ -256,11 +256,14 @@ pkv_status prefix_plan(const pkv_cache_desc* d, const DecodeGeometry& g, int32_t
   const int64_t chunks = ((int64_t)o->max_group_size * group + 127) / 128;
   const int64_t ctas = (int64_t)o->num_prefix_groups * d->num_kv_heads * chunks;
   if (chunks > INT32_MAX || d->num_kv_heads > 65535) return PKV_ERR_UNSUPPORTED;
-  // about two CTAs per SM in all, never more parts than shared blocks, at most 16
-  int64_t splits = (2 * (int64_t)sm_count() + ctas - 1) / ctas;
+  // about one CTA per SM in all (the pass runs one CTA per SM), at most 16 parts, each a whole
+  // number of the pass's 64-token steps: every part adds a partial state per member and head,
+  // written once and read once by the decode
+  const int64_t step = 64 / d->block_size;
+  int64_t splits = ((int64_t)sm_count() + ctas - 1) / ctas;
   splits = splits < 1 ? 1 : (splits > 16 ? 16 : splits);
-  if (splits > o->max_shared_blocks) splits = o->max_shared_blocks > 0 ? o->max_shared_blocks : 1;
-  const int64_t per = o->max_shared_blocks > 0 ? (o->max_shared_blocks + splits - 1) / splits : 1;
+  int64_t per = o->max_shared_blocks > 0 ? (o->max_shared_blocks + splits - 1) / splits : 1;
+  per = (per + step - 1) / step * step;
   splits = o->max_shared_blocks > 0 ? (o->max_shared_blocks + per - 1) / per : 1;
   if ((int64_t)o->num_prefix_groups * splits > 65535) return PKV_ERR_UNSUPPORTED;  // grid z
   pl->on = true;
