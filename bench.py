@@ -214,12 +214,11 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback 6.65 TB/s (earlier copy measurement on this pool)"
 
 
-def decode_source_hash() -> str:
-    """Hash of the decode kernel's device sources with comments and blank lines removed (a profile
-    stays valid across comment edits and host-side changes, not across kernel code changes)."""
+def _source_hash(names) -> str:
+    """Hash of kernel device sources with comments and blank lines removed (a profile stays valid
+    across comment edits and host-side changes, not across kernel code changes)."""
     h = hashlib.sha256()
-    for name in ("decode_kernel.cuh", "decode_i8i8.cu", "decode_i8i4.cu", "decode_f16.cu", "decode_fp8.cu",
-                 "common.cuh", "store_impl.cuh", "copy_impl.cuh"):
+    for name in names:
         with open(os.path.join(ROOT, "paged_block_quantized_b200", "csrc", name), encoding="utf-8") as f:
             for line in f:
                 code = line.split("//", 1)[0].rstrip()
@@ -228,17 +227,26 @@ def decode_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(config: str):
-    """DRAM bytes per decode launch from the committed ncu summary of this workload, if the
-    summary was taken on the current decode kernel source (else None)."""
-    path = os.path.join(ROOT, "profiles", f"paged_decode_{config}.md")
+def decode_source_hash() -> str:
+    return _source_hash(("decode_kernel.cuh", "decode_i8i8.cu", "decode_i8i4.cu", "decode_f16.cu", "decode_fp8.cu",
+                         "common.cuh", "store_impl.cuh", "copy_impl.cuh"))
+
+
+def prefill_source_hash() -> str:
+    return _source_hash(("prefill_tc.cuh", "tc_common.cuh", "common.cuh", "prefill.cu"))
+
+
+def ncu_traffic(profile: str, key: str = "decode_source_sha256_16", source_hash=decode_source_hash):
+    """DRAM bytes per launch from the committed ncu summary `profiles/<profile>.md`, if the summary
+    was taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", f"{profile}.md")
     try:
         text = open(path, encoding="utf-8").read()
     except OSError:
         return None, None
     m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    hsh = re.search(r"decode_source_sha256_16:\s*([0-9a-f]+)", text)
-    if not m or not hsh or hsh.group(1) != decode_source_hash():
+    hsh = re.search(key + r":\s*([0-9a-f]+)", text)
+    if not m or not hsh or hsh.group(1) != source_hash():
         return None, path
     return float(m.group(1)), path
 
@@ -406,12 +414,13 @@ def run_pkv(args, rank, world, local):
         kernel = "paged_decode_kernel (fused step: copies + store + decode)"
     elif g.prefix is not None:
         alg_bytes, launch_s = dec_bytes, dec_s
-        kernel = "paged_prefill_kernel (prefix mode) + paged_decode_kernel"
+        kernel = "paged_prefill_tc_kernel (prefix mode) + paged_decode_kernel"
     else:
         alg_bytes, launch_s, kernel = dec_bytes, dec_s, "paged_decode_kernel"
     achieved = alg_bytes / launch_s / 1e9
     peak, peak_src = measured_hbm_peak()
-    traffic, _ = ncu_traffic(args.config)
+    # the committed summaries are of the plain decode launch
+    traffic = ncu_traffic(f"paged_decode_{args.config}")[0] if not fused and g.prefix is None else None
     step_desc = (("copy-on-write copies + " if has_cow else "") + "store 1 token/seq (quantize+scatter) + decode"
                  + (", one fused launch (pkv_decode_step)" if fused else ", separate launches")
                  + (", decode walks each forked child right after its parent (pkv_paged_attention_decode_ex)"
@@ -510,8 +519,10 @@ def run_prefill(args, rank, world, local):
                    "step": "store the chunks (quantize+scatter) + chunked-prefill attention",
                    "parallelism": f"dp{world}", "l2": "flushed before every timed step"},
         "prefill_attention_us": att_s * 1e6,
-        "roofline": {"bound": "tensor", "kernel": "paged_prefill_kernel", "achieved": achieved, "peak": peak,
-                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+        "roofline": {"bound": "tensor", "kernel": "paged_prefill_tc_kernel", "achieved": achieved, "peak": peak,
+                     "unit": "TFLOP/s", "frac": achieved / peak,
+                     "traffic": ncu_traffic("paged_prefill_tc_prefill", "prefill_source_sha256_16",
+                                            prefill_source_hash)[0],
                      "algorithmic_flops_per_launch": flops, "peak_source": peak_src},
         "gpu_launches": 2 * K,
     }
@@ -592,7 +603,10 @@ def run_swap(args, rank, world, local):
         "swap_out_gbs": out_gbs, "swap_in_gbs": in_gbs,
         "roofline": {"bound": "host link", "kernel": "swap_blocks_kernel", "achieved": (out_gbs + in_gbs) / 2,
                      "peak": (d2h_peak + h2d_peak) / 2, "unit": "GB/s",
-                     "frac": ((out_gbs / d2h_peak) + (in_gbs / h2d_peak)) / 2, "traffic": None,
+                     "frac": ((out_gbs / d2h_peak) + (in_gbs / h2d_peak)) / 2,
+                     "traffic": ncu_traffic("swap_blocks_mixed", "swap_source_sha256_16",
+                                            lambda: _source_hash(("swap.cu", "common.cuh")))[0]
+                     if args.config == "mixed" else None,
                      "peak_source": f"measured in this run: pinned copies by the copy engines, "
                                     f"device->host {d2h_peak:.1f} GB/s, host->device {h2d_peak:.1f} GB/s"},
         "gpu_launches": 2 * K,
