@@ -60,6 +60,7 @@ class Workload:
     partition_tokens: int = 0         # 0 = let the library choose
     q_lens: np.ndarray | None = None  # int32 [S]: chunked prefill, new tokens per sequence (None: decode)
     outliers: bool = False
+    k_ramp: float = 0.0               # K of logical block j scaled by 1 + k_ramp * j (scores grow along the context)
     description: str = ""
     _mult: dict = field(default_factory=dict, repr=False)
 
@@ -96,12 +97,14 @@ class Workload:
         return (x * self._multipliers(which)).astype(np.float16)
 
     def block_values(self, stream: int, j: int):
-        """fp16 K, V [bs][H][D] of logical block j of a value stream: N(0,1) draws in fp32,
-        outlier channels scaled, rounded to fp16 (round to nearest)."""
+        """fp16 K, V [bs][H][D] of logical block j of a value stream: N(0,1) draws in fp32 (K times
+        1 + k_ramp * j), outlier channels scaled, rounded to fp16 (round to nearest)."""
         rng = np.random.default_rng([self.seed, _VALUES, int(stream), int(j)])
         shape = (self.block_size, self.num_kv_heads, self.head_dim)
         k = rng.standard_normal(shape, dtype=np.float32)
         v = rng.standard_normal(shape, dtype=np.float32)
+        if self.k_ramp:
+            k *= np.float32(1.0 + self.k_ramp * int(j))
         return self._scaled(k, "k"), self._scaled(v, "v")
 
     def seq_values(self, s: int, start: int, stop: int):
@@ -127,7 +130,8 @@ class Workload:
         v = np.empty(shape, np.float16)
         for s in range(self.num_seqs):
             rng = np.random.default_rng([self.seed, _NEWTOK, s])
-            k[s] = self._scaled(rng.standard_normal(shape[1:], dtype=np.float32), "k")
+            ramp = np.float32(1.0 + self.k_ramp * ((int(self.context_lens[s]) - 1) // self.block_size))
+            k[s] = self._scaled(rng.standard_normal(shape[1:], dtype=np.float32) * ramp, "k")
             v[s] = self._scaled(rng.standard_normal(shape[1:], dtype=np.float32), "v")
         return k, v
 
@@ -437,7 +441,7 @@ def make(name: str, seed: int = 0, **over) -> Workload:
         v_dtype=p["v_dtype"], softmax_scale=float(np.float32(1.0 / math.sqrt(p["head_dim"]))),
         context_lens=cl, block_tables=tables, block_streams=streams, prefill_tables=pre_tables,
         prefill_owner=owner, cow_pairs=cow, partition_tokens=p["partition_tokens"],
-        outliers=p["outliers"], description=desc,
+        outliers=p["outliers"], k_ramp=float(p.get("k_ramp", 0.0)), description=desc,
         q_lens=None if q_lens is None else np.asarray(q_lens, np.int32)[:S])
 
 

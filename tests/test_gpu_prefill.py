@@ -51,6 +51,35 @@ def test_prefill_matches_oracle(case):
     run(W.make("prefill", seed=1, **case))
 
 
+def test_prefill_growing_scores_rescale_in_place():
+    # K grows along the context, so a column's running maximum rises by more than 2^8 many times:
+    # the accumulator in tensor memory is rescaled in place again and again
+    w = W.make("prefill", seed=5, num_seqs=2, chunk=96, prefix_lens=[700, 333], num_q_heads=4, num_kv_heads=4,
+               k_ramp=0.5)
+    run(w)
+
+
+def test_prefill_bad_block_id_is_flagged():
+    from paged_block_quantized_b200 import pkv
+    from paged_block_quantized_b200.step import PrefillStep
+    w = W.make("prefill", seed=6, num_seqs=2, chunk=40, prefix_lens=[100, 60], num_q_heads=4, num_kv_heads=4)
+    g = PrefillStep(w)
+    g.prefill()
+    g.step()
+    torch.cuda.synchronize()
+    ref = g.out.clone()
+    tables = g.block_tables.clone()
+    tables[0, 2] = w.num_blocks + 5  # one block of sequence 0 out of the pool
+    g.dev_error.zero_()
+    pkv.pkv_paged_attention_prefill(g.pool.desc, g.out, g.q, 2, 4, g.cu, g.total_q, g.max_q_len, tables,
+                                    w.max_blocks_per_seq, g.context_lens, w.max_context_len, w.softmax_scale,
+                                    g.dev_error)
+    torch.cuda.synchronize()
+    assert g.error() == pkv.PKV_DEVERR_BLOCK_ID
+    assert torch.equal(g.out[40:], ref[40:])  # the other sequence is untouched
+    assert torch.isfinite(g.out[:40].float()).all()
+
+
 def test_prefill_full_size_sampled():
     w = W.make("prefill", seed=0)
     run(w, seqs=[0, int(np.argmax(w.context_lens))])

@@ -99,3 +99,18 @@ def test_beam_order_and_prefix_groups():
     starts, members, shared = g.prefix_groups()
     assert list(starts) == [0, 5] and (shared == 3).all()
     assert W.make("llama7b", seed=0, num_seqs=4).prefix_groups() is None
+
+
+def test_k_ramp_scales_keys_by_block():
+    # the option that makes scores grow along the context: K of logical block j times 1 + r * j
+    # (before the fp16 rounding), V untouched
+    a = W.make("prefill", seed=3, num_seqs=1, chunk=8, prefix_lens=[100], num_q_heads=4, num_kv_heads=4)
+    b = W.make("prefill", seed=3, num_seqs=1, chunk=8, prefix_lens=[100], num_q_heads=4, num_kv_heads=4, k_ramp=0.25)
+    for j in (0, 3, 6):
+        ka, va = a.block_values(a.block_streams[0, j], j)
+        kb, vb = b.block_values(b.block_streams[0, j], j)
+        np.testing.assert_array_equal(va, vb)
+        if j == 0:
+            np.testing.assert_array_equal(kb, ka)
+        ratio = kb.astype(np.float64) / np.where(ka == 0, 1, ka).astype(np.float64)
+        assert np.allclose(ratio[ka != 0], 1 + 0.25 * j, rtol=2e-3)
