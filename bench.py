@@ -71,8 +71,11 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
-    ap.add_argument("--beam-order", action="store_true",
-                    help="walk each forked child right after its parent instead of in index order")
+    ap.add_argument("--walk", choices=("index", "beam", "aligned"), default=None,
+                    help="the decode's walk over the sequences: index order; each forked child right after "
+                         "its parent; or sequences that share blocks a whole number of worker ranges apart "
+                         "(reads of a shared block coincide and the second hits L2)")
+    ap.add_argument("--beam-order", action="store_true", help="same as --walk beam")
     ap.add_argument("--shared-prefix", choices=("auto", "on", "off"), default="off",
                     help="attend blocks shared by a group of sequences once per group (auto: when a group has "
                          "more than two members)")
@@ -313,8 +316,9 @@ def run_pkv(args, rank, world, local):
     groups = w.prefix_groups()
     shared = args.shared_prefix == "on" or (
         args.shared_prefix == "auto" and groups is not None and int(np.diff(groups[0]).max()) > 2)
-    g = DeviceStep(w, device=dev, poison=None, partition_tokens=args.partition_tokens,
-                   beam_order=args.beam_order, shared_prefix=shared and not args.fused)
+    walk = args.walk or ("beam" if args.beam_order else "index")
+    g = DeviceStep(w, device=dev, poison=None, partition_tokens=args.partition_tokens, walk=walk,
+                   shared_prefix=shared and not args.fused)
     g.prefill()
     g.snapshot_step_tiles()
     has_cow = w.cow_pairs.shape[0] > 0
@@ -419,12 +423,21 @@ def run_pkv(args, rank, world, local):
         alg_bytes, launch_s, kernel = dec_bytes, dec_s, "paged_decode_kernel"
     achieved = alg_bytes / launch_s / 1e9
     peak, peak_src = measured_hbm_peak()
-    # the committed summaries are of the plain decode launch
-    traffic = ncu_traffic(f"paged_decode_{args.config}")[0] if not fused and g.prefix is None else None
+    # the committed summaries are of the plain decode launch, in the walk order they name
+    traffic = None
+    if not fused and g.prefix is None:
+        traffic, prof = ncu_traffic(f"paged_decode_{args.config}")
+        if prof is not None:
+            m = re.search(r"^walk:\s*(\w+)", open(prof, encoding="utf-8").read(), re.M)
+            if (m.group(1) if m else "index") != (g.walk if g.seq_order is not None else "index"):
+                traffic = None
     step_desc = (("copy-on-write copies + " if has_cow else "") + "store 1 token/seq (quantize+scatter) + decode"
                  + (", one fused launch (pkv_decode_step)" if fused else ", separate launches")
                  + (", decode walks each forked child right after its parent (pkv_paged_attention_decode_ex)"
-                    if g.seq_order is not None and not fused else "")
+                    if g.seq_order is not None and not fused and g.walk == "beam" else "")
+                 + (", decode walks sharing sequences a whole number of worker ranges apart "
+                    "(pkv_paged_attention_decode_ex)" if g.seq_order is not None and not fused and g.walk == "aligned"
+                    else "")
                  + (", shared-prefix decode: each shared block attended once per group (prefix pass + decode)"
                     if g.prefix is not None else ""))
     line = {

@@ -12,6 +12,7 @@ import numpy as np
 import torch
 
 from . import pkv
+from .walk import aligned_walk_order
 from .workloads import Workload
 
 
@@ -28,22 +29,35 @@ _TORCH_DTYPE = {np.dtype(np.float16): torch.float16, np.dtype(np.int32): torch.i
 
 class DeviceStep:
     def __init__(self, w: Workload, device="cuda", poison: int | None = 0xA5, partition_tokens: int | None = None,
-                 beam_order: bool = False, shared_prefix: bool = False):
+                 beam_order: bool = False, shared_prefix: bool = False, walk: str | None = None):
         self.w = w
         self.device = torch.device(device)
         self.pool = pkv.DevicePool.allocate(w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim, w.k_dtype,
                                             w.v_dtype, device=self.device, fill=poison)
         self.dev_error = torch.zeros(1, dtype=torch.int32, device=self.device)
         dev = self.device
+        self.partition_tokens = w.partition_tokens if partition_tokens is None else partition_tokens
+        self.num_workers, self.num_ctas = pkv.pkv_decode_partitioning(
+            self.pool.desc, w.num_seqs, w.num_q_heads, w.max_context_len, self.partition_tokens)
         # the step's inputs live in one device buffer (views below), so that a caller feeding the
         # step from host memory moves them with one copy
         k_new, v_new = w.new_token_values()
         inputs = [("q", w.queries()), ("k_new", k_new), ("v_new", v_new), ("step_slots", w.step_slots()),
                   ("block_tables", w.block_tables), ("context_lens", w.context_lens), ("cow", w.cow_pairs)]
-        # with beam_order, the decode walks forked children right after their parents
-        use_order = beam_order and w.cow_pairs.shape[0] > 0
-        if use_order:
+        # the decode's walk: the sequences in index order; forked children right after their
+        # parents ("beam"); or sharing sequences a whole number of worker ranges apart ("aligned")
+        walk = walk if walk is not None else ("beam" if beam_order else "index")
+        if walk not in ("index", "beam", "aligned"):
+            raise ValueError(f"walk {walk!r}")
+        self.walk = walk
+        self.walk_misalignment = None
+        use_order = walk != "index" and w.cow_pairs.shape[0] > 0
+        if use_order and walk == "beam":
             inputs.append(("seq_order", w.beam_walk_order()))
+        elif use_order:
+            order, self.walk_misalignment = aligned_walk_order(w.block_tables, w.context_lens, w.block_size,
+                                                               self.num_workers)
+            inputs.append(("seq_order", order))
         # with shared_prefix, blocks shared by several sequences are attended once per group
         groups = w.prefix_groups() if shared_prefix else None
         if groups is not None:
@@ -69,9 +83,6 @@ class DeviceStep:
             self.prefix = dict(group_start=self.group_start, members=self.members, shared_blocks=self.shared_blocks,
                                num_groups=len(sizes), num_members=int(groups[0][-1]),
                                max_group_size=int(sizes.max()), max_shared_blocks=int(groups[2].max()))
-        self.partition_tokens = w.partition_tokens if partition_tokens is None else partition_tokens
-        self.num_workers, self.num_ctas = pkv.pkv_decode_partitioning(
-            self.pool.desc, w.num_seqs, w.num_q_heads, w.max_context_len, self.partition_tokens)
         self.ws_bytes = pkv.pkv_decode_ex_workspace_size(self.pool.desc, w.num_seqs, w.num_q_heads,
                                                          w.max_context_len, self.partition_tokens, self.seq_order,
                                                          self.prefix)

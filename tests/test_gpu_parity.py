@@ -354,15 +354,18 @@ def test_copy_blocks_bit_exact_and_bad_ids():
     np.testing.assert_array_equal(g.pool_numpy()[0], after[0])
 
 
-@pytest.mark.parametrize("name,over", [("mixed", dict(num_seqs=24, children=4)), ("mixed", {})])
-def test_beam_walk_order(name, over):
-    """pkv_paged_attention_decode_ex with a walk order that puts every forked child right after its
-    parent gives the oracle's outputs (reduced and full size), and an order entry outside the batch
-    is skipped and flagged, never a fault or a hang."""
+@pytest.mark.parametrize("name,over,walk", [("mixed", dict(num_seqs=24, children=4), "beam"), ("mixed", {}, "beam"),
+                                           ("mixed", dict(num_seqs=24, children=4), "aligned"),
+                                           ("mixed", {}, "aligned")])
+def test_walk_order(name, over, walk):
+    """pkv_paged_attention_decode_ex with a walk order (every forked child right after its parent, or
+    sharing sequences a whole number of worker ranges apart) gives the oracle's outputs (reduced and
+    full size), and an order entry outside the batch is skipped and flagged, never a fault or a
+    hang."""
     from paged_block_quantized_b200 import pkv
     from paged_block_quantized_b200.step import DeviceStep
     w = W.make(name, seed=0, **over)
-    g = DeviceStep(w, beam_order=True)
+    g = DeviceStep(w, walk=walk)
     assert g.seq_order is not None
     g.prefill()
     g.step()
