@@ -59,7 +59,7 @@ def dtype_label(w) -> str:
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("pkv", "reference"), default="pkv")
     ap.add_argument("--op", choices=("step", "swap"), default="step",
@@ -449,7 +449,12 @@ def run_pkv(args, rank, world, local):
         "effective_hbm_gbs": achieved, "frac_of_8tbs": achieved / 8000.0,
         "decode_us": dec_s * 1e6, "store_us": statistics.mean(store_ms) * 1e3,
         "store_rebuilt_tiles": f"{rebuilt} of {appended} (block, head) tiles appended into (first-time appends)",
+        **({"decode_logical_gbs": w.decode_bytes(unique=False) / dec_s / 1e9,
+            "logical_bytes_per_launch": w.decode_bytes(unique=False)}
+           if w.decode_bytes(unique=False) != dec_bytes else {}),
         "decode_only_gbs": dec_bytes / dec_s / 1e9,
+        # medians over the timed steps (the value above is their total)
+        "ms_per_step_median": statistics.median(step_ms), "decode_us_median": statistics.median(dec_ms) * 1e3,
         "roofline": {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": peak,
                      "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
                      "algorithmic_bytes_per_launch": alg_bytes, "peak_source": peak_src},
@@ -463,6 +468,9 @@ def run_pkv(args, rank, world, local):
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         threads = os.cpu_count() or 1
         line["cpu_baseline"] = time_oracle_decode(w, args.cpu_seconds, threads)
+        if threads > 1:  # the same oracle on one host thread, a smaller bounded sample
+            one = time_oracle_decode(w, min(args.cpu_seconds, 6.0), 1)
+            line["cpu_baseline"]["single_thread"] = {"value": one["value"], "sample": one["sample"]}
     return line
 
 
