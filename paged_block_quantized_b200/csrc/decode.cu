@@ -80,6 +80,11 @@ cudaError_t launch_any(const DecodeParams& p, const StepParams& sp, const Decode
 }  // namespace
 
 cudaError_t launch_decode(const DecodeParams& p, const DecodeShape& sh, cudaStream_t stream) {
+  if (gqa_tc_eligible(sh, p.num_seqs, p.num_q_heads)) {
+    DecodeKernelInfo info;
+    if (!decode_kernel_info(sh, &info)) return cudaErrorInvalidValue;
+    return launch_gqa_tc(p, sh, (int64_t)sh.grid_ctas * info.warps_per_cta, stream);
+  }
   StepParams sp = {};
   sp.fused = 0;
   return launch_any(p, sp, sh, stream);

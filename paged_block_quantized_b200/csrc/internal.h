@@ -64,6 +64,11 @@ bool decode_supported(int32_t k_dtype, int32_t v_dtype, int32_t block_size, int3
 bool decode_kernel_info(const DecodeShape& sh, DecodeKernelInfo* info);
 
 cudaError_t launch_decode(const DecodeParams& p, const DecodeShape& sh, cudaStream_t stream);
+// Grouped-query decode on tcgen05 (gqa_tc.cuh): INT8 K, INT8 / INT4 V, D 128, 8 heads per unit. The
+// (non-fused) decode takes it for these shapes; `workers` bounds its partial slots as the
+// workspace was sized (units + workers).
+bool gqa_tc_eligible(const DecodeShape& sh, int32_t num_seqs, int32_t num_q_heads);
+cudaError_t launch_gqa_tc(const DecodeParams& p, const DecodeShape& sh, int64_t workers, cudaStream_t stream);
 
 // Tensor maps of the K and V code pools for the tensor-core engine's tiled copies: the pool as
 // rows of `row_bytes` (a multiple of 128; 2-D, or 3-D in 128-byte units), boxes of `box_rows`

@@ -119,6 +119,11 @@ def test_split_matches_unsplit():
     dict(head_dim=256, block_size=32, num_q_heads=8, num_kv_heads=4, k_dtype=W.FP8_E4M3, v_dtype=W.FP8_E4M3),
     dict(head_dim=128, block_size=32, num_q_heads=16, num_kv_heads=4, k_dtype=W.FP8_E4M3, v_dtype=W.FP8_E4M3),
     dict(head_dim=128, block_size=16, num_q_heads=16, num_kv_heads=2, k_dtype=W.FP8_E4M3, v_dtype=W.FP8_E4M3),
+    # the tcgen05 grouped-query kernel: 8 or 16 query heads per KV head (one or two units), INT8 or
+    # INT4 V, block size 16 or 32
+    dict(head_dim=128, block_size=32, num_q_heads=16, num_kv_heads=2, v_dtype=W.INT4_ASYM),
+    dict(head_dim=128, block_size=16, num_q_heads=32, num_kv_heads=2),
+    dict(head_dim=128, block_size=32, num_q_heads=8, num_kv_heads=1),
 ])
 def test_shapes_and_groups(case):
     lens = [1, 2, 16, 17, 31, 32, 33, 100, 700]
@@ -141,6 +146,16 @@ def test_long_sequence_split_and_whole(pt):
     g, _ = check(w, partition_tokens=pt)
     if pt:
         assert g.num_workers == 32
+
+
+@pytest.mark.parametrize("vt", [W.INT8_SYM, W.INT4_ASYM])
+def test_gqa_long_context_many_splits(vt):
+    # the tcgen05 grouped-query kernel with one long sequence: its blocks cut into many splits whose
+    # partials the last split merges, next to a one-token sequence (one split, written directly)
+    w = W.make("tiny", seed=6, num_seqs=2, context_lens=[20011, 5], num_blocks=1400, head_dim=128, block_size=16,
+               num_q_heads=16, num_kv_heads=2, v_dtype=vt)
+    assert _gqa_tc_shape(w)
+    check(w)
 
 
 def test_zero_length_and_empty_batch():
@@ -301,6 +316,16 @@ def test_token_by_token_appends_bit_exact(bs, D, kt, vt):
             np.testing.assert_array_equal(got[4][b], c.v_zp[b])
 
 
+def _gqa_tc_shape(w):
+    """True for the shapes the tcgen05 grouped-query kernel covers (INT8 K, INT8 or INT4 V, head_dim
+    128, query heads in groups of 8): a library built with PKV_DECODE_GQA_TC=1 decodes them there,
+    the default build on the stream-K kernel's tensor-core engine."""
+    group = w.num_q_heads // w.num_kv_heads
+    return (w.k_dtype == W.INT8_SYM and w.v_dtype in (W.INT8_SYM, W.INT4_ASYM) and w.head_dim == 128
+            and group % 8 == 0)
+
+
+
 @pytest.mark.parametrize("name,over", [("mixed", dict(num_seqs=24, children=4)), ("llama7b", dict(num_seqs=6)),
                                        ("gqa_prefix", dict(num_seqs=4, prefix_blocks=8, private_blocks=9)),
                                        ("llama7b_fp16", dict(num_seqs=3)), ("llama7b_fp8", dict(num_seqs=3))])
@@ -320,6 +345,8 @@ def test_fused_step_matches_separate_launches(name, over):
         assert gf.error() == 0 and gs.error() == 0
         for a, b in zip(gf.pool_numpy(), gs.pool_numpy()):
             np.testing.assert_array_equal(a, b)
+        # (both on the stream-K kernel; a library built with PKV_DECODE_GQA_TC=1 would decode the
+        # separate GQA step on the tcgen05 kernel, the same attention rounded differently)
         np.testing.assert_array_equal(gf.out.cpu().numpy(), gs.out.cpu().numpy())
         # tickets (one per sequence and head group) and the two barrier counters lead the workspace
         group = w.num_q_heads // w.num_kv_heads
