@@ -205,7 +205,9 @@ PKV_API pkv_status pkv_decode_partitioning(const pkv_cache_desc* desc, int32_t n
  *                after a PKV_DEVERR_TIMEOUT). Calls that share a workspace must not overlap on
  *                the GPU.
  *   dev_error    device int32 or NULL
- * num_q_heads must be a multiple of num_kv_heads.
+ * num_q_heads must be a multiple of num_kv_heads. The pool may hold at most 2^31 - 1 token rows
+ * per cache side (num_blocks * num_kv_heads * block_size): the tile copies address rows with a
+ * signed 32-bit coordinate. A larger pool gives PKV_ERR_UNSUPPORTED.
  *
  * Ordering with the preceding work on `stream`: the kernel is launched with programmatic stream
  * serialization, so it may start while the previous kernel on the stream is still running (the

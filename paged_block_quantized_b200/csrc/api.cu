@@ -75,6 +75,8 @@ pkv_status decode_geometry(const pkv_cache_desc* d, int32_t num_seqs, int32_t nu
   if (num_seqs < 0 || num_q_heads <= 0 || max_context_len < 0 || partition_tokens < 0) return PKV_ERR_INVALID_ARG;
   if (num_q_heads % d->num_kv_heads != 0) return PKV_ERR_INVALID_ARG;
   if (partition_tokens % d->block_size != 0) return PKV_ERR_INVALID_ARG;
+  // the decode's tiled copies address a cache side's token rows with a signed 32-bit coordinate
+  if ((int64_t)d->num_blocks * d->num_kv_heads * d->block_size > INT32_MAX) return PKV_ERR_UNSUPPORTED;
   const int32_t group = num_q_heads / d->num_kv_heads;
   DecodeShape& sh = g->shape;
   sh.k_dtype = d->k_dtype;

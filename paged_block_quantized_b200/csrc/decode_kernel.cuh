@@ -77,11 +77,28 @@ constexpr float kNegBig = -1.0e30f;  // finite "minus infinity" for running maxi
 #ifndef PKV_DECODE_IMMA_QK
 #define PKV_DECODE_IMMA_QK 0
 #endif
+// 1: the CUDA-core engine walks a 16-token-block pool two blocks per stream position (one 32-token
+// tile, each half with its own scales), when the warps per CTA stay the same; 0: one block each.
+// Measured on one B200: 239.7 vs 244.8 us on the lognormal-length INT8 K / INT4 V batch (fewer
+// waits, walk steps and softmax passes per token). INT8 V with head_dim 128 keeps one block per
+// position: its paired tile would leave room for 12 warps per CTA instead of 16.
+#ifndef PKV_DECODE_PAIR
+#define PKV_DECODE_PAIR 1
+#endif
+// INT8 K with one query head per KV head and 32-token blocks: q.k on the integer tensor cores, the
+// three byte planes of q as three columns of one mma (1), or in dp4a planes on the CUDA cores (0);
+// p.v stays on the CUDA cores either way. Measured on one B200: 157.8 vs 163.9 us on 8 sequences
+// of 8K-32K tokens in 32-token blocks (two 16-row slices per tile: two independent mma chains);
+// with 16-token tiles (one chain per tile) 291 vs 244 us on the lognormal-length batch, so there
+// the dp4a planes stay.
+#ifndef PKV_DECODE_HYB
+#define PKV_DECODE_HYB 1
+#endif
 #ifndef PKV_DECODE_MAX_STAGES
 #define PKV_DECODE_MAX_STAGES 6
 #endif
 
-template <int KT, int VT, int BS, int D, int GT>
+template <int KT, int VT, int BS, int D, int GT, int PB = BS>
 struct Cfg {
   static constexpr int K_ROW = (KT == PKV_FP16) ? 2 * D : D;
   static constexpr int V_ROW = (VT == PKV_FP16) ? 2 * D : (VT == PKV_INT4_ASYM ? D / 2 : D);
@@ -95,9 +112,15 @@ struct Cfg {
   static constexpr bool I8K = KT == PKV_INT8_SYM && (VT == PKV_INT8_SYM || VT == PKV_INT4_ASYM);
   static constexpr bool MMA = (D >= 128 && I8K && (GT >= 4 || PKV_DECODE_MMA_MHA)) ||
                               (GT >= 4 && KT == PKV_FP16 && VT == PKV_FP16) || (FP8 && D >= 128);
-  // the V tile arrives swizzled (tiled copy) when its rows are whole 128-byte units; INT4 V always
-  // by a 1-D bulk copy (its reads below index unswizzled rows of D/2 bytes)
-  static constexpr bool V_SWZ = V_ROW % 128 == 0 && VT != PKV_INT4_ASYM;
+  // CUDA-core engine with INT8 K, one query head per KV head and a pool of 32-token blocks (PB:
+  // the pool's block size; BS: the tile's rows, two blocks in the paired walk): q.k on the integer
+  // tensor cores (mma m16n8k32 with q's byte planes as columns), p.v on the CUDA cores
+  static constexpr bool HYB = !MMA && KT == PKV_INT8_SYM && GT == 1 && K_ROW % 128 == 0 && PB == 32 && PKV_DECODE_HYB;
+  // the K tile arrives by a tiled copy with 128-byte swizzle (tensor-core fragments of it)
+  static constexpr bool TILED_K = MMA || HYB;
+  // the tensor-core engine's V tile arrives swizzled (tiled copy) when its rows are whole 128-byte
+  // units; INT4 V, and V for the CUDA cores, by a 1-D bulk copy (unswizzled rows)
+  static constexpr bool V_SWZ = MMA && V_ROW % 128 == 0 && VT != PKV_INT4_ASYM;
   static constexpr int WARPS_AUTO =
       MMA ? (D >= 256 ? 8 : 12) : (KT == PKV_FP16 ? 8 : (GT == 1 ? 16 : (GT == 2 ? 12 : 8)));
   static constexpr int WARPS_WANT = PKV_DECODE_WARPS_SM > 0 ? PKV_DECODE_WARPS_SM : WARPS_AUTO;
@@ -110,12 +133,12 @@ struct Cfg {
   static constexpr int SMEM_BAR_FLAG = SMEM_STAGES + NW * NS * 8;  // one int: a grid barrier's outcome
   // The tensor-core engine's tiles arrive by tiled copies with 128-byte swizzle, whose shared
   // destinations must be 1024-byte aligned: the stages start on the next 1024-byte boundary.
-  static constexpr int SMEM_ALIGN = MMA ? 1024 : 0;
+  static constexpr int SMEM_ALIGN = TILED_K ? 1024 : 0;
   static constexpr int SMEM = SMEM_BAR_FLAG + 16 + SMEM_ALIGN;
   static constexpr int CTAS_PER_SM = 1;
   static_assert(D % 16 == 0 && D / 16 <= 32, "head_dim");
   static_assert(K_TILE % 16 == 0 && V_TILE % 16 == 0 && STAGE % 16 == 0, "bulk copy granularity");
-  static_assert(!MMA || (K_ROW % 128 == 0 && K_TILE % 1024 == 0 && STAGE % 1024 == 0 &&
+  static_assert(!TILED_K || (K_ROW % 128 == 0 && K_TILE % 1024 == 0 && STAGE % 1024 == 0 &&
                           (!V_SWZ || V_TILE % 1024 == 0)),
                 "swizzled tiles: 128-byte row units, 1024-byte aligned tiles");
   static_assert(NW >= 1 && SMEM <= 227 * 1024, "shared memory per CTA");
@@ -171,12 +194,17 @@ struct Win {
   long long seq_p0;     // stream position of the sequence's first block (head group 0)
 };
 
+// A window lane's stream position: one physical block, or two consecutive ones of the unit (the
+// paired walk: a 32-token tile of two 16-token blocks).
+// Before the scales are fetched, b holds the ids as read from the table; after, the physical block
+// to copy (0 stands in for an invalid id; -1 where a paired position holds no second block), the
+// K scale in the log2 domain, the V scale, and the V zero point (0 without one), or -1 where the
+// block is not valid (its tokens are masked).
+template <int VB>
 struct WinLanes {
-  int b;        // physical block (0 stands in for an invalid id)
-  int raw;      // block id as read from the table
-  bool valid;
-  bool meta;    // scales fetched (warp-uniform)
-  float ks, vs, zp;
+  int b[VB];
+  bool meta;  // scales fetched (warp-uniform)
+  float ks[VB], vs[VB], zv[VB];
 };
 
 // ============================================================================================
@@ -184,14 +212,71 @@ struct WinLanes {
 // and keep the running softmax state of GT query heads for the current unit.
 // ============================================================================================
 
+// Byte offset of (row r, byte x) in a tile of R-byte rows stored by a tiled copy with 128-byte
+// swizzle: rows are cut into 128-byte units (unit u = r * R/128 + x/128), and within unit u the
+// 16-byte chunk j sits at chunk j ^ (u mod 8). Rows of 128 or 256 bytes otherwise all start on
+// bank 0, and the fragment loads below (the same column of several rows at once) would conflict.
+template <int R>
+__device__ __forceinline__ int swz(int r, int x) {
+  const int u = r * (R / 128) + (x >> 7);
+  return (u << 7) | ((((x >> 4) & 7) ^ (u & 7)) << 4) | (x & 15);
+}
+
+// ---- tensor-core helpers (mma.sync m16n8k16, fp16 operands, fp32 accumulators) ----
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// integer tensor cores: m16n8k32, signed 8-bit operands, int32 accumulators
+__device__ __forceinline__ void imma_16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                           uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+__device__ __forceinline__ uint32_t h2_sub(uint32_t a, uint32_t b) {
+  const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&b));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t h2_pack(float lo, float hi) {
+  const __half2 r = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+// fp16 1024 + 128 in both halves: a byte b placed under exponent 0x64 reads 1024 + b, and
+// (c ^ 0x80) = c + 128 for a signed code c, so subtracting this leaves c exactly
+constexpr uint32_t kH2Bias = 0x64806480u;
+// two E4M3 codes (low byte first) -> two exact fp16 values (low half first)
+__device__ __forceinline__ uint32_t fp8x2_to_h2(uint32_t two) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xffffu), __NV_E4M3);
+  return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+
 // CUDA-core engine (1, 2 or 4 query heads per KV head): a lane owns 16 consecutive dims of
 // bs/(32*16/D) token rows; q.k in exact integer dp4a planes (INT8 K) or paired FFMA (FP16 K);
 // p.v with paired FFMA on codes made exact floats through the float bit layout.
-template <int KT, int VT, int BS, int D, int GT>
+//
+// With INT8 K and one query head (C::HYB), q.k runs on the integer tensor cores instead: per
+// 16-row slice one mma m16n8k32 per 32 dims, A = the slice's K codes (rows = tokens) straight from
+// the swizzled tile, B = q on its 22-bit fixed-point grid, whose three signed byte planes fill
+// columns 0, 1, 2 (and again 4, 5, 6; columns 3 and 7 are zero). Lane (gq, tq) then holds planes
+// 0 and 1 of tokens gq and gq + 8 when tq is even, plane 2 in its odd neighbour: one exchange
+// completes a score, and the scores move to the p.v layout by index shuffles.
+template <int KT, int VT, int BS, int D, int GT, int PB = BS>
 struct CoreEngine {
-  using C = Cfg<KT, VT, BS, D, GT>;
+  using C = Cfg<KT, VT, BS, D, GT, PB>;
   static constexpr int CH = D / 16, TG = 32 / CH, TPL = BS / TG;
   static_assert(BS % TG == 0, "block_size must cover the token rows of a warp pass");
+  static constexpr bool HYB = C::HYB;
+  static constexpr int KQ = D / 32;  // k32-steps of one slice's q.k (HYB)
+  static_assert(!HYB || (GT == 1 && BS % 16 == 0 && 16 % TG == 0 && C::TILED_K), "tensor-core q.k");
   // A lane owns 16 dims: [a, a + 8) and [b, b + 8). With byte codes they are contiguous
   // (a = 16c, b = a + 8: a lane's 16 codes are one 16-byte load). With fp16 rows (2D bytes),
   // 16 contiguous dims would put lanes c and c + 4 of a load on the same banks; a = 8c and
@@ -201,7 +286,9 @@ struct CoreEngine {
   __device__ __forceinline__ int dim_a() const { return SPLIT ? 8 * c : 16 * c; }
   __device__ __forceinline__ int dim_b() const { return SPLIT ? D / 2 + 8 * c : 16 * c + 8; }
   float2 qf[GT][8];
-  uint32_t qplane[GT][3][4];
+  uint32_t qplane[GT][HYB ? 1 : 3][4];
+  uint32_t qbf[HYB ? KQ : 1][2];  // HYB: B fragments, k32-step kk, (b0, b1)
+  int lid;
   float qinv[GT];
   float m_run[GT], l_run[GT];
   float2 acc[GT][8];
@@ -219,6 +306,12 @@ struct CoreEngine {
   __device__ __forceinline__ void begin(const DecodeParams& p, int s, int hg, int lane) {
     c = lane % CH;
     tg = lane / CH;
+    lid = lane;
+    if constexpr (HYB) begin_hyb(p, s, hg, lane);
+    else begin_core(p, s, hg);
+  }
+
+  __device__ __forceinline__ void begin_core(const DecodeParams& p, int s, int hg) {
 #pragma unroll
     for (int hh = 0; hh < GT; ++hh) {
       const __half* qp = p.q + ((size_t)s * p.num_q_heads + (size_t)hg * GT + hh) * D;
@@ -272,11 +365,108 @@ struct CoreEngine {
     }
   }
 
-  // one block; ks = per-block K scale in the log2 domain (INT8 K), vs = V scale, nzb = -(2^23+zp)
-  __device__ __forceinline__ void block(const uint8_t* kt, const uint8_t* vt, float ks, float vs, float nzb, bool valid,
-                                        int tok0, int L, float scale_log2) {
-    const float2 neg_zp_bias = make_float2(nzb, nzb);
+  // q on the fixed-point grid of the dp4a planes (same shift, same planes), as B fragments: lane
+  // (gq, tq) gives column gq, i.e. byte plane gq % 4 (3: zero), over dims tq * D/4 + [0, D/4);
+  // k32-step kk holds dims tq * D/4 + 8kk + [0, 4) in b0 and + [4, 8) in b1, the dims of the A
+  // fragments read in block().
+  __device__ __forceinline__ void begin_hyb(const DecodeParams& p, int s, int hg, int lane) {
+    const int gq = lane >> 2, tq = lane & 3;
+    const uint4* qp = reinterpret_cast<const uint4*>(p.q + ((size_t)s * p.num_q_heads + hg) * D + tq * (D / 4));
+    float x[D / 4];
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) {
+      const uint4 w = qp[i];
+      const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&u[k]));
+        x[8 * i + 2 * k] = f.x;
+        x[8 * i + 2 * k + 1] = f.y;
+      }
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < D / 4; ++i) amax = fmaxf(amax, fabsf(x[i]));
+    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
+    int e = 0;
+    (void)frexpf(amax, &e);                    // amax < 2^e
+    const int shift = amax > 0.f ? 22 - e : 0;  // |q| * 2^shift < 2^22
+    const float up = __int_as_float((127 + shift) << 23);
+    qinv[0] = __int_as_float((127 - shift) << 23);
+    const int pl = gq & 3;
+#pragma unroll
+    for (int kk = 0; kk < KQ; ++kk) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t w = 0;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int qi = __float2int_rn(x[8 * kk + 4 * h + k] * up);
+          const int b0 = ((qi + 128) & 0xFF) - 128;
+          const int r1 = (qi - b0) >> 8;
+          const int b1 = ((r1 + 128) & 0xFF) - 128;
+          const int b2 = (r1 - b1) >> 8;
+          const int bp = pl == 0 ? b0 : (pl == 1 ? b1 : (pl == 2 ? b2 : 0));
+          w |= (uint32_t)(bp & 0xFF) << (8 * k);
+        }
+        qbf[kk][h] = w;
+      }
+    }
+    reset();
+  }
+
+  // One tile of BS token rows made of BS / HB physical blocks of HB rows (1 or 2): per physical
+  // block ks = K scale in the log2 domain (INT8 K), vs = V scale, nzb = -(2^23+zp), valid. A row's
+  // block is known at compile time: a lane's rows are tg + TG*i and HB is a multiple of TG.
+  template <int HB>
+  __device__ __forceinline__ void block(const uint8_t* kt, const uint8_t* vt, const float (&ks)[2], const float (&vs)[2],
+                                        const float (&nzb)[2], const bool (&valid)[2], int tok0, int L,
+                                        float scale_log2) {
+    static_assert(BS % HB == 0 && BS / HB <= 2 && HB % TG == 0, "physical blocks of a tile");
     float z[TPL][GT];
+    if constexpr (HYB) {
+      scores_hyb(kt, z);
+    } else {
+      scores_core(kt, z);
+    }
+    block_softmax_pv<HB>(vt, z, ks, vs, nzb, valid, tok0, L, scale_log2);
+  }
+
+  // q.k of the tile's rows tg + TG*i on the integer tensor cores (C::HYB; see above)
+  __device__ __forceinline__ void scores_hyb(const uint8_t* kt, float (&z)[TPL][GT]) const {
+    constexpr int NSL = BS / 16;
+    const int gq = lid >> 2, tq = lid & 3;
+    float sA[NSL], sB[NSL];  // tokens 16h2 + gq and 16h2 + gq + 8 (complete where tq is even)
+#pragma unroll
+    for (int h2 = 0; h2 < NSL; ++h2) {
+      int cc[4] = {0, 0, 0, 0};
+#pragma unroll
+      for (int i = 0; i < D / 64; ++i) {  // 16 codes = 2 k32-steps per 16-byte load
+        const int x = tq * (D / 4) + 16 * i;
+        const uint4 r0 = *reinterpret_cast<const uint4*>(kt + swz<C::K_ROW>(16 * h2 + gq, x));
+        const uint4 r1 = *reinterpret_cast<const uint4*>(kt + swz<C::K_ROW>(16 * h2 + gq + 8, x));
+        imma_16832(cc, r0.x, r1.x, r0.y, r1.y, qbf[2 * i][0], qbf[2 * i][1]);
+        imma_16832(cc, r0.z, r1.z, r0.w, r1.w, qbf[2 * i + 1][0], qbf[2 * i + 1][1]);
+      }
+      // |plane sums| < 2^21: planes 0 and 1 combine exactly in int32, plane 2 in fp32
+      const int u0 = __shfl_xor_sync(kFull, cc[0], 1);
+      const int u2 = __shfl_xor_sync(kFull, cc[2], 1);
+      sA[h2] = __fmaf_rn((float)u0, 65536.f, (float)(cc[1] * 256 + cc[0]));
+      sB[h2] = __fmaf_rn((float)u2, 65536.f, (float)(cc[3] * 256 + cc[2]));
+    }
+    // row tg + TG*i: slice (TG*i)/16, token (tg + TG*i) % 16 of it, held by lane 4 * (token % 8)
+#pragma unroll
+    for (int i = 0; i < TPL; ++i) {
+      const int h2 = (TG * i) / 16;
+      const bool upper = (TG * i) % 16 >= 8;
+      z[i][0] = __shfl_sync(kFull, upper ? sB[h2] : sA[h2], 4 * ((tg + TG * i) % 8));
+    }
+  }
+
+  // q.k of the tile's rows tg + TG*i on the CUDA cores: a lane's 16 dims, then summed over the
+  // CH lanes of a row
+  __device__ __forceinline__ void scores_core(const uint8_t* kt, float (&z)[TPL][GT]) const {
 #pragma unroll
     for (int i = 0; i < TPL; ++i) {
       const int row = tg + TG * i;
@@ -318,17 +508,25 @@ struct CoreEngine {
       for (int hh = 0; hh < GT; ++hh)
 #pragma unroll
         for (int off = 1; off < CH; off <<= 1) z[i][hh] += __shfl_xor_sync(kFull, z[i][hh], off);
+  }
 
+  // online softmax of the tile's scores z (unscaled) and p.v into the running state
+  template <int HB>
+  __device__ __forceinline__ void block_softmax_pv(const uint8_t* vt, float (&z)[TPL][GT], const float (&ks)[2],
+                                                   const float (&vs)[2], const float (&nzb)[2], const bool (&valid)[2],
+                                                   int tok0, int L, float scale_log2) {
     float pv[TPL][GT];
 #pragma unroll
     for (int hh = 0; hh < GT; ++hh) {
-      const float zscale = (KT == PKV_FP16) ? scale_log2 : ks * qinv[hh];
+      const float zs0 = (KT == PKV_FP16) ? scale_log2 : ks[0] * qinv[hh];
+      const float zs1 = (KT == PKV_FP16) ? scale_log2 : ks[1] * qinv[hh];
       float mloc = -INFINITY;
 #pragma unroll
       for (int i = 0; i < TPL; ++i) {
         const int t = tok0 + tg + TG * i;
-        float zz = z[i][hh] * zscale;
-        zz = (valid && t < L) ? zz : -INFINITY;
+        const int hb = (TG * i) / HB;  // the row's physical block (compile time)
+        float zz = z[i][hh] * (hb ? zs1 : zs0);
+        zz = (valid[hb] && t < L) ? zz : -INFINITY;
         z[i][hh] = zz;
         mloc = fmaxf(mloc, zz);
       }
@@ -349,13 +547,15 @@ struct CoreEngine {
       for (int i = 0; i < TPL; ++i) {
         const float pr = ex2(z[i][hh] - m_new);
         lsum += pr;
-        pv[i][hh] = (VT == PKV_FP16) ? pr : pr * vs;
+        pv[i][hh] = (VT == PKV_FP16) ? pr : pr * vs[(TG * i) / HB];
       }
       l_run[hh] += lsum;
     }
 #pragma unroll
     for (int i = 0; i < TPL; ++i) {
       const int row = tg + TG * i;
+      const int hb = (TG * i) / HB;
+      const float2 neg_zp_bias = make_float2(nzb[hb], nzb[hb]);
       float2 vf[8];
       if constexpr (VT == PKV_FP16) load_h16(vt + row * C::V_ROW + 2 * dim_a(), vt + row * C::V_ROW + 2 * dim_b(), vf);
       else load_v16<VT>(vt + row * C::V_ROW + c * (C::V_ROW / CH), neg_zp_bias, vf);
@@ -420,53 +620,6 @@ struct CoreEngine {
     }
   }
 };
-
-// Byte offset of (row r, byte x) in a tile of R-byte rows stored by a tiled copy with 128-byte
-// swizzle: rows are cut into 128-byte units (unit u = r * R/128 + x/128), and within unit u the
-// 16-byte chunk j sits at chunk j ^ (u mod 8). Rows of 128 or 256 bytes otherwise all start on
-// bank 0, and the fragment loads below (the same column of several rows at once) would conflict.
-template <int R>
-__device__ __forceinline__ int swz(int r, int x) {
-  const int u = r * (R / 128) + (x >> 7);
-  return (u << 7) | ((((x >> 4) & 7) ^ (u & 7)) << 4) | (x & 15);
-}
-
-// ---- tensor-core helpers (mma.sync m16n8k16, fp16 operands, fp32 accumulators) ----
-__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-// integer tensor cores: m16n8k32, signed 8-bit operands, int32 accumulators
-__device__ __forceinline__ void imma_16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
-                                           uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
-  uint32_t y;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
-  return y;
-}
-__device__ __forceinline__ uint32_t h2_sub(uint32_t a, uint32_t b) {
-  const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&b));
-  return *reinterpret_cast<const uint32_t*>(&r);
-}
-__device__ __forceinline__ uint32_t h2_pack(float lo, float hi) {
-  const __half2 r = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&r);
-}
-// fp16 1024 + 128 in both halves: a byte b placed under exponent 0x64 reads 1024 + b, and
-// (c ^ 0x80) = c + 128 for a signed code c, so subtracting this leaves c exactly
-constexpr uint32_t kH2Bias = 0x64806480u;
-// two E4M3 codes (low byte first) -> two exact fp16 values (low half first)
-__device__ __forceinline__ uint32_t fp8x2_to_h2(uint32_t two) {
-  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xffffu), __NV_E4M3);
-  return (uint32_t)h.x | ((uint32_t)h.y << 16);
-}
 
 // Tensor-core engine (4 or 8 query heads per KV head): per 16-token slice of a block,
 //   S = K . q^T  as mma m16n8k16 with M = 16 tokens, N = 8 heads, K = 16 dims per step, and
@@ -582,8 +735,14 @@ struct MmaEngine {
     }
   }
 
-  __device__ __forceinline__ void block(const uint8_t* kt, const uint8_t* vt, float ks, float vs, float nzb,
-                                        bool valid, int tok0, int L, float scale_log2) {
+  // one (block, KV head) tile (HB == BS: the tensor-core engine takes one physical block per tile)
+  template <int HB>
+  __device__ __forceinline__ void block(const uint8_t* kt, const uint8_t* vt, const float (&ksa)[2],
+                                        const float (&vsa)[2], const float (&nzba)[2], const bool (&valida)[2],
+                                        int tok0, int L, float scale_log2) {
+    static_assert(HB == BS, "one physical block per tile");
+    const float ks = ksa[0], vs = vsa[0], nzb = nzba[0];
+    const bool valid = valida[0];
     const float zscale = (KT == PKV_FP16) ? scale_log2 : ks;
 #pragma unroll
     for (int h2 = 0; h2 < BS / 16; ++h2) {
@@ -843,9 +1002,9 @@ struct MmaEngine {
   }
 };
 
-template <int KT, int VT, int BS, int D, int GT>
-using EngineFor = typename std::conditional<Cfg<KT, VT, BS, D, GT>::MMA, MmaEngine<KT, VT, BS, D, GT>,
-                                            CoreEngine<KT, VT, BS, D, GT>>::type;
+template <int KT, int VT, int BS, int D, int GT, int PB = BS>
+using EngineFor = typename std::conditional<Cfg<KT, VT, BS, D, GT, PB>::MMA, MmaEngine<KT, VT, BS, D, GT>,
+                                            CoreEngine<KT, VT, BS, D, GT, PB>>::type;
 
 // ---- merge of a split unit ----
 __device__ __forceinline__ float warp_sum(float v) {
@@ -989,10 +1148,16 @@ __device__ __noinline__ void step_store(const StoreParams& sp, int w, int W, int
     store_detail::store_job<KT, VT>(sp, job / sp.num_kv_heads, job % sp.num_kv_heads, lane, tbl);
 }
 
-template <int KT, int VT, int BS, int D, int GT, bool FUSED>
-__global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, BS, D, GT>::CTAS_PER_SM)
+// BS: the pool's block size; VB: physical blocks per stream position (1, or 2 for the paired walk
+// of the CUDA-core engine: the tile holds two consecutive blocks of the unit, which halves the
+// per-position work of the copy ring and the walk).
+template <int KT, int VT, int BS, int D, int GT, bool FUSED, int VB>
+__global__ void __launch_bounds__(Cfg<KT, VT, BS * VB, D, GT, BS>::THREADS, Cfg<KT, VT, BS * VB, D, GT, BS>::CTAS_PER_SM)
     paged_decode_kernel(const DecodeParams p, const StepParams sp, const __grid_constant__ TileMaps tm) {
-  using C = Cfg<KT, VT, BS, D, GT>;
+  using C = Cfg<KT, VT, BS * VB, D, GT, BS>;
+  static_assert(VB == 1 || (VB == 2 && !C::MMA), "paired blocks: CUDA-core engine only");
+  // stream positions of a unit with nphys private blocks
+  auto npos = [](int nphys) -> int { return (nphys + VB - 1) / VB; };
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   constexpr uint32_t kAlign = C::SMEM_ALIGN ? C::SMEM_ALIGN : 1;
   uint8_t* const smem = smem_raw + ((kAlign - (smem_addr(smem_raw) & (kAlign - 1))) & (kAlign - 1));
@@ -1062,7 +1227,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
     }
     // the stream counts the sequences in walk order (the same as index order without one)
     const int Lw = p.seq_order == nullptr ? L : (s < S ? len_at(s) : 0);
-    int sum = (Lw + BS - 1) / BS - (s < S ? sb_at(s, Lw) : 0);
+    int sum = npos((Lw + BS - 1) / BS - (s < S ? sb_at(s, Lw) : 0));
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(kFull, sum, off);
     T += sum;
@@ -1106,7 +1271,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
       const int s = base + lane;
       const int L = s < S ? len_at(s) : 0;
       const int sb = s < S ? sb_at(s, L) : 0;
-      const long long cnt = (long long)((L + BS - 1) / BS - sb) * HG;
+      const long long cnt = (long long)npos((L + BS - 1) / BS - sb) * HG;
       long long incl = cnt;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
@@ -1121,7 +1286,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
         cur.sa = p.seq_order == nullptr ? cur.s : __ldg(p.seq_order + cur.s);  // valid: it has blocks
         cur.L = __shfl_sync(kFull, L, f);
         cur.sb = __shfl_sync(kFull, sb, f);
-        cur.nblk = (cur.L + BS - 1) / BS - cur.sb;
+        cur.nblk = npos((cur.L + BS - 1) / BS - cur.sb);
         cur.seq_p0 = acc0 + __shfl_sync(kFull, incl - cnt, f);
         Lchunk = L;
         SBchunk = sb;
@@ -1172,7 +1337,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
         b.sa = (s < S && p.seq_order != nullptr) ? __ldg(p.seq_order + s) : s;  // valid when L > 0
         b.L = L;
         b.sb = s < S ? seq_sb(s) : 0;
-        b.nblk = (L + BS - 1) / BS - b.sb;
+        b.nblk = npos((L + BS - 1) / BS - b.sb);
       }
       b.g = (b.hg * GT) / p.group;
     }
@@ -1181,27 +1346,38 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
   };
 
   // phase A of a window: block ids (one per lane); phase B (at its first copy): scales
-  auto load_ids = [&](const Win& a, WinLanes& r) {
+  auto load_ids = [&](const Win& a, WinLanes<VB>& r) {
     r.meta = false;
-    r.raw = -1;
-    if (lane < a.n) r.raw = p.block_tables[(size_t)a.sa * p.max_blocks_per_seq + a.sb + a.j0 + lane];
+    const int nphys = (a.L + BS - 1) / BS - a.sb;  // the unit's private blocks
+#pragma unroll
+    for (int h = 0; h < VB; ++h) {
+      r.b[h] = -1;
+      if (lane < a.n && VB * (a.j0 + lane) + h < nphys)
+        r.b[h] = p.block_tables[(size_t)a.sa * p.max_blocks_per_seq + a.sb + VB * (a.j0 + lane) + h];
+    }
   };
-  auto load_meta = [&](const Win& a, WinLanes& r) {
-    r.valid = lane < a.n && r.raw >= 0 && r.raw < p.num_blocks;
-    if (lane < a.n && !r.valid) record_error(p.dev_error, PKV_DEVERR_BLOCK_ID);
-    r.b = r.valid ? r.raw : 0;
-    r.ks = r.vs = r.zp = 0.f;
-    if (lane < a.n) {
-      const size_t meta = (size_t)r.b * p.num_kv_heads + a.g;
-      if constexpr (KT != PKV_FP16) r.ks = p.k_scale[meta];
-      if constexpr (VT != PKV_FP16) r.vs = p.v_scale[meta];
-      if constexpr (VT == PKV_INT4_ASYM) r.zp = (float)p.v_zp[meta];
+  auto load_meta = [&](const Win& a, WinLanes<VB>& r) {
+    const int nphys = (a.L + BS - 1) / BS - a.sb;
+#pragma unroll
+    for (int h = 0; h < VB; ++h) {
+      const bool has = lane < a.n && VB * (a.j0 + lane) + h < nphys;
+      const bool valid = has && r.b[h] >= 0 && r.b[h] < p.num_blocks;
+      if (has && !valid) record_error(p.dev_error, PKV_DEVERR_BLOCK_ID);
+      r.b[h] = valid ? r.b[h] : (has ? 0 : -1);
+      r.ks[h] = r.vs[h] = 0.f;
+      r.zv[h] = valid ? 0.f : -1.f;
+      if (has) {
+        const size_t meta = (size_t)r.b[h] * p.num_kv_heads + a.g;
+        if constexpr (KT != PKV_FP16) r.ks[h] = p.k_scale[meta] * p.scale_log2;  // log2 domain
+        if constexpr (VT != PKV_FP16) r.vs[h] = p.v_scale[meta];
+        if constexpr (VT == PKV_INT4_ASYM) if (valid) r.zv[h] = (float)p.v_zp[meta];
+      }
     }
     r.meta = true;
   };
 
   prefetch_q<GT, D>(p, cur.sa, cur.hg, lane);
-  WinLanes rc, rn;
+  WinLanes<VB> rc, rn;
   load_ids(cur, rc);
   Win nxt = next_win(cur);
   load_ids(nxt, rn);
@@ -1221,24 +1397,26 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
 
 
   // ---- the copy ring ----
-  auto issue = [&](int st, int b, int g) {
+  // one physical (block, KV head) tile: its K rows to kd, its V rows to vd. A tiled copy takes the
+  // tile's BS rows from row tile * BS, swizzled; a 1-D bulk copy takes them as they are.
+  auto copy_tile = [&](uint8_t* kd, uint8_t* vd, int b, int g, uint64_t* bar) {
+    constexpr uint32_t PK = BS * C::K_ROW, PV = BS * C::V_ROW;
     const size_t tile = (size_t)b * p.num_kv_heads + g;
+    const int row = (int)(tile * BS);
+    if constexpr (!C::TILED_K) bulk_g2s(kd, static_cast<const uint8_t*>(p.k_codes) + tile * PK, PK, bar);
+    else if constexpr (C::K_ROW == 128) tma_load_2d(kd, &tm.k, 0, row, bar);
+    else tma_load_3d(kd, &tm.k, 0, 0, row, bar);
+    if constexpr (!C::V_SWZ) bulk_g2s(vd, static_cast<const uint8_t*>(p.v_codes) + tile * PV, PV, bar);
+    else if constexpr (C::V_ROW == 128) tma_load_2d(vd, &tm.v, 0, row, bar);
+    else tma_load_3d(vd, &tm.v, 0, 0, row, bar);
+  };
+  // a stream position: one tile, or two (paired walk) whose rows follow each other
+  auto issue = [&](int st, int b, int b1, bool has1, int g) {
+    constexpr uint32_t PK = BS * C::K_ROW, PV = BS * C::V_ROW;
     uint8_t* dst = my_stages + (size_t)st * C::STAGE;
-    mbar_arrive_expect_tx(&my_bars[st], (uint32_t)C::STAGE);
-    if constexpr (C::MMA) {  // tiled copies: the tile's BS rows from row tile * BS, swizzled
-      const int row = (int)(tile * BS);
-      if constexpr (C::K_ROW == 128) tma_load_2d(dst, &tm.k, 0, row, &my_bars[st]);
-      else tma_load_3d(dst, &tm.k, 0, 0, row, &my_bars[st]);
-      if constexpr (!C::V_SWZ)
-        bulk_g2s(dst + C::K_TILE, static_cast<const uint8_t*>(p.v_codes) + tile * C::V_TILE, (uint32_t)C::V_TILE,
-                 &my_bars[st]);
-      else if constexpr (C::V_ROW == 128) tma_load_2d(dst + C::K_TILE, &tm.v, 0, row, &my_bars[st]);
-      else tma_load_3d(dst + C::K_TILE, &tm.v, 0, 0, row, &my_bars[st]);
-    } else {
-      bulk_g2s(dst, static_cast<const uint8_t*>(p.k_codes) + tile * C::K_TILE, (uint32_t)C::K_TILE, &my_bars[st]);
-      bulk_g2s(dst + C::K_TILE, static_cast<const uint8_t*>(p.v_codes) + tile * C::V_TILE, (uint32_t)C::V_TILE,
-               &my_bars[st]);
-    }
+    mbar_arrive_expect_tx(&my_bars[st], (has1 ? 2u : 1u) * (PK + PV));
+    copy_tile(dst, dst + C::K_TILE, b, g, &my_bars[st]);
+    if (has1) copy_tile(dst + PK, dst + C::K_TILE + PV, b1, g, &my_bars[st]);
   };
   // positions relative to `start`: consumed (cpos) and issued (ipos); stage / parity of each
   int cpos = 0, ipos = 0, cst = 0, ist = 0;
@@ -1248,18 +1426,20 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
   auto issue_ahead = [&]() {
     const int lim = min(cpos + C::NS, n_total);
     while (ipos < lim) {
-      int b, g;
+      int b, b1 = -1, g;
       if (ipos < cur.r0 + cur.n) {
-        b = __shfl_sync(kFull, rc.b, ipos - cur.r0);
+        b = __shfl_sync(kFull, rc.b[0], ipos - cur.r0);
+        if constexpr (VB == 2) b1 = __shfl_sync(kFull, rc.b[VB - 1], ipos - cur.r0);
         g = cur.g;
       } else if (nxt.n > 0 && ipos < nxt.r0 + nxt.n) {
         if (!rn.meta) load_meta(nxt, rn);
-        b = __shfl_sync(kFull, rn.b, ipos - nxt.r0);
+        b = __shfl_sync(kFull, rn.b[0], ipos - nxt.r0);
+        if constexpr (VB == 2) b1 = __shfl_sync(kFull, rn.b[VB - 1], ipos - nxt.r0);
         g = nxt.g;
       } else {
         break;
       }
-      if (lane == 0) issue(ist, b, g);
+      if (lane == 0) issue(ist, b, b1, b1 >= 0, g);
       ist = (ist + 1 == C::NS) ? 0 : ist + 1;
       ++ipos;
     }
@@ -1303,7 +1483,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
   // the first copies go out before the engine's set-up (which waits for q)
   issue_ahead();
   // ---- per-unit state: the arithmetic engine for GT query heads ----
-  EngineFor<KT, VT, BS, D, GT> eng;
+  EngineFor<KT, VT, BS * VB, D, GT, BS> eng;
   int seg_j0 = cur.j0;  // first block of the current segment within its unit
   eng.begin(p, cur.sa, cur.hg, lane);
 
@@ -1332,12 +1512,27 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
 
     // ---- one block: q . k, online softmax, p . v ----
     const int kw_i = cpos - cur.r0;
-    const float ks = __shfl_sync(kFull, rc.ks, kw_i) * p.scale_log2;  // per-block K scale, log2 domain
-    const float vs = __shfl_sync(kFull, rc.vs, kw_i);
-    const float nzb = -(kMagic + __shfl_sync(kFull, rc.zp, kw_i));
-    const bool valid = __shfl_sync(kFull, rc.valid ? 1 : 0, kw_i) != 0;
+    float ks[2], vs[2], nzb[2];
+    bool valid[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {  // per physical block of the position (the second only when paired)
+      if (h < VB) {
+        const int hv = h < VB ? h : 0;
+        ks[h] = __shfl_sync(kFull, rc.ks[hv], kw_i);  // K scale, log2 domain
+        vs[h] = __shfl_sync(kFull, rc.vs[hv], kw_i);
+        const float zv = __shfl_sync(kFull, rc.zv[hv], kw_i);
+        nzb[h] = -(kMagic + zv);
+        valid[h] = zv >= 0.f;
+      } else {
+        ks[h] = ks[0];
+        vs[h] = vs[0];
+        nzb[h] = nzb[0];
+        valid[h] = valid[0];
+      }
+    }
     const uint8_t* kt = my_stages + (size_t)st * C::STAGE;
-    eng.block(kt, kt + C::K_TILE, ks, vs, nzb, valid, (cur.sb + cur.j0 + kw_i) * BS, cur.L, p.scale_log2);
+    eng.template block<BS>(kt, kt + C::K_TILE, ks, vs, nzb, valid, (cur.sb + VB * (cur.j0 + kw_i)) * BS, cur.L,
+                           p.scale_log2);
     __syncwarp();  // the stage's reads are complete (their values were consumed above)
     if constexpr (kDeferTicket) {
       if (pend == 1 && cpos >= pend_since + 2) take_ticket();
@@ -1391,10 +1586,11 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS, D, GT>::THREADS, Cfg<KT, VT, B
   if constexpr (FUSED) grid_exit(sp.bar, gridDim.x);
 }
 
-template <int KT, int VT, int BS, int D, int GT>
-cudaError_t launch_one(const DecodeParams& p, const StepParams& sp, const DecodeShape& sh, cudaStream_t stream) {
-  using C = Cfg<KT, VT, BS, D, GT>;
-  auto kern = sp.fused ? paged_decode_kernel<KT, VT, BS, D, GT, true> : paged_decode_kernel<KT, VT, BS, D, GT, false>;
+template <int KT, int VT, int BS, int D, int GT, int VB>
+cudaError_t launch_vb(const DecodeParams& p, const StepParams& sp, const DecodeShape& sh, cudaStream_t stream) {
+  using C = Cfg<KT, VT, BS * VB, D, GT, BS>;
+  auto kern = sp.fused ? paged_decode_kernel<KT, VT, BS, D, GT, true, VB>
+                       : paged_decode_kernel<KT, VT, BS, D, GT, false, VB>;
   static unsigned long long configured[2] = {0, 0};  // one bit per device and variant; benign race
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -1426,12 +1622,26 @@ cudaError_t launch_one(const DecodeParams& p, const StepParams& sp, const Decode
   cfg.numAttrs = 1;
   TileMaps tm;
   memset(&tm, 0, sizeof(tm));
-  if constexpr (C::MMA) {
+  if constexpr (C::TILED_K) {
     const uint64_t rows = (uint64_t)p.num_blocks * p.num_kv_heads * BS;
     if (!encode_tile_map(&tm.k, p.k_codes, rows, C::K_ROW, BS)) return cudaErrorInvalidValue;
     if (C::V_SWZ && !encode_tile_map(&tm.v, p.v_codes, rows, C::V_ROW, BS)) return cudaErrorInvalidValue;
   }
   return cudaLaunchKernelEx(&cfg, kern, p, sp, tm);
+}
+
+// The paired walk (two 16-token blocks per stream position) for the CUDA-core engine with INT8 K
+// and INT8 / INT4 V, unless the decode starts units after shared-prefix blocks (whose count need
+// not be even). (At a unit's end a paired position may hold one block; the other half of its tile
+// keeps stale bytes, masked by the length: codes of any bytes are finite numbers, which fp16 bytes
+// are not.)
+template <int KT, int VT, int BS, int D, int GT>
+cudaError_t launch_one(const DecodeParams& p, const StepParams& sp, const DecodeShape& sh, cudaStream_t stream) {
+  if constexpr (PKV_DECODE_PAIR && BS == 16 && KT == PKV_INT8_SYM && VT != PKV_FP16 && !Cfg<KT, VT, BS, D, GT>::MMA &&
+                Cfg<KT, VT, 2 * BS, D, GT>::NW == Cfg<KT, VT, BS, D, GT>::NW) {
+    if (p.shared_blocks == nullptr) return launch_vb<KT, VT, BS, D, GT, 2>(p, sp, sh, stream);
+  }
+  return launch_vb<KT, VT, BS, D, GT, 1>(p, sp, sh, stream);
 }
 
 template <int KT, int VT, int BS, int D, int GT>

@@ -124,6 +124,14 @@ def test_split_matches_unsplit():
     dict(head_dim=128, block_size=32, num_q_heads=16, num_kv_heads=2, v_dtype=W.INT4_ASYM),
     dict(head_dim=128, block_size=16, num_q_heads=32, num_kv_heads=2),
     dict(head_dim=128, block_size=32, num_q_heads=8, num_kv_heads=1),
+    # one query head per KV head: INT8 K on the integer tensor cores with 32-token blocks (head_dim
+    # 128 and 256), and the paired walk of 16-token blocks (two blocks per tile; the odd block
+    # counts above leave the last tile of a unit half full)
+    dict(head_dim=128, block_size=32, num_q_heads=4, num_kv_heads=4),
+    dict(head_dim=128, block_size=32, num_q_heads=4, num_kv_heads=4, v_dtype=W.INT4_ASYM),
+    dict(head_dim=256, block_size=32, num_q_heads=2, num_kv_heads=2),
+    dict(head_dim=128, block_size=16, num_q_heads=4, num_kv_heads=4, v_dtype=W.INT4_ASYM),
+    dict(head_dim=64, block_size=16, num_q_heads=4, num_kv_heads=4, v_dtype=W.INT4_ASYM),
 ])
 def test_shapes_and_groups(case):
     lens = [1, 2, 16, 17, 31, 32, 33, 100, 700]
@@ -180,14 +188,16 @@ def test_zero_length_and_empty_batch():
     assert pkv.pkv_store_quantized(g.pool.desc, g.k_new, g.v_new, g.step_slots, 0) == pkv.PKV_OK
 
 
-def test_bad_block_id_is_skipped_and_flagged():
+@pytest.mark.parametrize("j", [0, 1, 2])
+def test_bad_block_id_is_skipped_and_flagged(j):
+    # a bad id in either block of a paired tile (the tiny cache walks two 16-token blocks per tile)
     import oracle
     w = W.make("tiny", seed=6)
     g, o = check(w)
     tables = o["tables"].copy()
     bad_gpu = g.block_tables.clone()
-    bad_gpu[2, 1] = w.num_blocks + 5
-    tables[2, 1] = len(o["phys"]) + 5
+    bad_gpu[2, j] = w.num_blocks + 5
+    tables[2, j] = len(o["phys"]) + 5
     from paged_block_quantized_b200 import pkv
     pkv.pkv_paged_attention_decode(g.pool.desc, g.out, g.q, w.num_seqs, w.num_q_heads, bad_gpu,
                                    w.max_blocks_per_seq, g.context_lens, w.max_context_len, w.softmax_scale,
