@@ -94,6 +94,20 @@ constexpr float kNegBig = -1.0e30f;  // finite "minus infinity" for running maxi
 #ifndef PKV_DECODE_HYB
 #define PKV_DECODE_HYB 1
 #endif
+// Tuning switches (defaults: as described above): PKV_DECODE_HYB_ALL 1 takes the tensor-core q.k
+// for 16-token pools too; PKV_DECODE_KCOPY 0 / 1 forces the CUDA-core engine's K tile to a 1-D bulk
+// copy / a swizzled tiled copy (-1: tiled exactly when q.k runs on the tensor cores).
+#ifndef PKV_DECODE_HYB_ALL
+#define PKV_DECODE_HYB_ALL 0
+#endif
+#ifndef PKV_DECODE_KCOPY
+#define PKV_DECODE_KCOPY -1
+#endif
+// 1: a tile that lies wholly inside the sequence and whose blocks are valid skips the per-row
+// masking of its scores (a warp-uniform branch); 0: every tile is masked row by row
+#ifndef PKV_DECODE_FULLTILE
+#define PKV_DECODE_FULLTILE 1
+#endif
 #ifndef PKV_DECODE_MAX_STAGES
 #define PKV_DECODE_MAX_STAGES 6
 #endif
@@ -115,9 +129,13 @@ struct Cfg {
   // CUDA-core engine with INT8 K, one query head per KV head and a pool of 32-token blocks (PB:
   // the pool's block size; BS: the tile's rows, two blocks in the paired walk): q.k on the integer
   // tensor cores (mma m16n8k32 with q's byte planes as columns), p.v on the CUDA cores
-  static constexpr bool HYB = !MMA && KT == PKV_INT8_SYM && GT == 1 && K_ROW % 128 == 0 && PB == 32 && PKV_DECODE_HYB;
-  // the K tile arrives by a tiled copy with 128-byte swizzle (tensor-core fragments of it)
-  static constexpr bool TILED_K = MMA || HYB;
+  static constexpr bool HYB =
+      !MMA && KT == PKV_INT8_SYM && GT == 1 && K_ROW % 128 == 0 && (PB == 32 || PKV_DECODE_HYB_ALL) && PKV_DECODE_HYB;
+  // the K tile arrives by a tiled copy with 128-byte swizzle (tensor-core fragments of it), or by a
+  // 1-D bulk copy (rows as they are)
+  static constexpr bool TILED_K =
+      MMA || (KT == PKV_INT8_SYM && K_ROW % 128 == 0 &&
+              (PKV_DECODE_KCOPY == 1 || (PKV_DECODE_KCOPY == -1 && HYB)));
   // the tensor-core engine's V tile arrives swizzled (tiled copy) when its rows are whole 128-byte
   // units; INT4 V, and V for the CUDA cores, by a 1-D bulk copy (unswizzled rows)
   static constexpr bool V_SWZ = MMA && V_ROW % 128 == 0 && VT != PKV_INT4_ASYM;
@@ -276,7 +294,7 @@ struct CoreEngine {
   static_assert(BS % TG == 0, "block_size must cover the token rows of a warp pass");
   static constexpr bool HYB = C::HYB;
   static constexpr int KQ = D / 32;  // k32-steps of one slice's q.k (HYB)
-  static_assert(!HYB || (GT == 1 && BS % 16 == 0 && 16 % TG == 0 && C::TILED_K), "tensor-core q.k");
+  static_assert(!HYB || (GT == 1 && BS % 16 == 0 && 16 % TG == 0), "tensor-core q.k");
   // A lane owns 16 dims: [a, a + 8) and [b, b + 8). With byte codes they are contiguous
   // (a = 16c, b = a + 8: a lane's 16 codes are one 16-byte load). With fp16 rows (2D bytes),
   // 16 contiguous dims would put lanes c and c + 4 of a load on the same banks; a = 8c and
@@ -292,12 +310,21 @@ struct CoreEngine {
   float qinv[GT];
   float m_run[GT], l_run[GT];
   float2 acc[GT][8];
+  // INT4 V (OFS): the p.v sums run over 0.5 + code/256 (no per-code subtraction); after every tile
+  // the offset part (0.5 x the tile's sum of p * v_scale) is taken out of acc, so acc holds
+  // sum(p * vs * code) / 256, and zsum collects sum(p * vs * zp); finish() forms 256 acc - zsum.
+  // (Measured on one B200: 233.5 vs 237.7 us on the lognormal-length INT8 K / INT4 V batch; with
+  // q.k on the tensor cores, whose tiles wait on the mma chain, it measured slower, 164.6 vs
+  // 157.8 us on the 32-token-block batch, so there the per-code subtraction stays.)
+  static constexpr bool OFS = VT == PKV_INT4_ASYM && !HYB;
+  float zsum[OFS ? GT : 1];
 
   __device__ __forceinline__ void reset() {
 #pragma unroll
     for (int hh = 0; hh < GT; ++hh) {
       m_run[hh] = kNegBig;
       l_run[hh] = 0.f;
+      if constexpr (OFS) zsum[hh] = 0.f;
 #pragma unroll
       for (int j = 0; j < 8; ++j) acc[hh][j] = make_float2(0.f, 0.f);
     }
@@ -433,6 +460,9 @@ struct CoreEngine {
     block_softmax_pv<HB>(vt, z, ks, vs, nzb, valid, tok0, L, scale_log2);
   }
 
+  // byte offset of (row r, byte x) in the K tile as its copy left it
+  __device__ __forceinline__ static int koff(int r, int x) { return C::TILED_K ? swz<C::K_ROW>(r, x) : r * C::K_ROW + x; }
+
   // q.k of the tile's rows tg + TG*i on the integer tensor cores (C::HYB; see above)
   __device__ __forceinline__ void scores_hyb(const uint8_t* kt, float (&z)[TPL][GT]) const {
     constexpr int NSL = BS / 16;
@@ -444,8 +474,8 @@ struct CoreEngine {
 #pragma unroll
       for (int i = 0; i < D / 64; ++i) {  // 16 codes = 2 k32-steps per 16-byte load
         const int x = tq * (D / 4) + 16 * i;
-        const uint4 r0 = *reinterpret_cast<const uint4*>(kt + swz<C::K_ROW>(16 * h2 + gq, x));
-        const uint4 r1 = *reinterpret_cast<const uint4*>(kt + swz<C::K_ROW>(16 * h2 + gq + 8, x));
+        const uint4 r0 = *reinterpret_cast<const uint4*>(kt + koff(16 * h2 + gq, x));
+        const uint4 r1 = *reinterpret_cast<const uint4*>(kt + koff(16 * h2 + gq + 8, x));
         imma_16832(cc, r0.x, r1.x, r0.y, r1.y, qbf[2 * i][0], qbf[2 * i][1]);
         imma_16832(cc, r0.z, r1.z, r0.w, r1.w, qbf[2 * i + 1][0], qbf[2 * i + 1][1]);
       }
@@ -470,9 +500,8 @@ struct CoreEngine {
 #pragma unroll
     for (int i = 0; i < TPL; ++i) {
       const int row = tg + TG * i;
-      const uint8_t* krow = kt + row * C::K_ROW + c * (C::K_ROW / CH);
       if constexpr (KT == PKV_INT8_SYM) {
-        const uint4 wv = *reinterpret_cast<const uint4*>(krow);
+        const uint4 wv = *reinterpret_cast<const uint4*>(kt + koff(row, c * (C::K_ROW / CH)));
         const int kw[4] = {(int)wv.x, (int)wv.y, (int)wv.z, (int)wv.w};
 #pragma unroll
         for (int hh = 0; hh < GT; ++hh) {
@@ -521,14 +550,25 @@ struct CoreEngine {
       const float zs0 = (KT == PKV_FP16) ? scale_log2 : ks[0] * qinv[hh];
       const float zs1 = (KT == PKV_FP16) ? scale_log2 : ks[1] * qinv[hh];
       float mloc = -INFINITY;
+      // the tile's blocks valid and its last row inside the sequence: no row is masked
+      const bool full = PKV_DECODE_FULLTILE && valid[0] && valid[BS / HB - 1] && tok0 + BS <= L;
+      if (full) {
 #pragma unroll
-      for (int i = 0; i < TPL; ++i) {
-        const int t = tok0 + tg + TG * i;
-        const int hb = (TG * i) / HB;  // the row's physical block (compile time)
-        float zz = z[i][hh] * (hb ? zs1 : zs0);
-        zz = (valid[hb] && t < L) ? zz : -INFINITY;
-        z[i][hh] = zz;
-        mloc = fmaxf(mloc, zz);
+        for (int i = 0; i < TPL; ++i) {
+          const float zz = z[i][hh] * (((TG * i) / HB) ? zs1 : zs0);
+          z[i][hh] = zz;
+          mloc = fmaxf(mloc, zz);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < TPL; ++i) {
+          const int t = tok0 + tg + TG * i;
+          const int hb = (TG * i) / HB;  // the row's physical block (compile time)
+          float zz = z[i][hh] * (hb ? zs1 : zs0);
+          zz = (valid[hb] && t < L) ? zz : -INFINITY;
+          z[i][hh] = zz;
+          mloc = fmaxf(mloc, zz);
+        }
       }
 #pragma unroll
       for (int off = CH; off < 32; off <<= 1) mloc = fmaxf(mloc, __shfl_xor_sync(kFull, mloc, off));
@@ -537,6 +577,7 @@ struct CoreEngine {
         const float alpha = ex2(m_run[hh] - mloc);
         m_run[hh] = mloc;
         l_run[hh] *= alpha;
+        if constexpr (OFS) zsum[hh] *= alpha;
         const float2 alpha2 = make_float2(alpha, alpha);
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[hh][j] = __fmul2_rn(acc[hh][j], alpha2);
@@ -557,13 +598,37 @@ struct CoreEngine {
       const int hb = (TG * i) / HB;
       const float2 neg_zp_bias = make_float2(nzb[hb], nzb[hb]);
       float2 vf[8];
-      if constexpr (VT == PKV_FP16) load_h16(vt + row * C::V_ROW + 2 * dim_a(), vt + row * C::V_ROW + 2 * dim_b(), vf);
-      else load_v16<VT>(vt + row * C::V_ROW + c * (C::V_ROW / CH), neg_zp_bias, vf);
+      if constexpr (VT == PKV_FP16) {
+        load_h16(vt + row * C::V_ROW + 2 * dim_a(), vt + row * C::V_ROW + 2 * dim_b(), vf);
+      } else if constexpr (OFS) {
+        const uint2 w = *reinterpret_cast<const uint2*>(vt + row * C::V_ROW + c * (C::V_ROW / CH));
+        u4x8_to_half_offset_f32x2(w.x, vf);
+        u4x8_to_half_offset_f32x2(w.y, vf + 4);
+      } else {
+        load_v16<VT>(vt + row * C::V_ROW + c * (C::V_ROW / CH), neg_zp_bias, vf);
+      }
 #pragma unroll
       for (int hh = 0; hh < GT; ++hh) {
         const float2 pv2 = make_float2(pv[i][hh], pv[i][hh]);
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[hh][j] = __ffma2_rn(pv2, vf[j], acc[hh][j]);
+      }
+    }
+    if constexpr (OFS) {
+      // take the tile's offset part out of acc now (it stays about the size of the result, which
+      // bounds the rounding of later sums), and collect the zero-point part
+#pragma unroll
+      for (int hh = 0; hh < GT; ++hh) {
+        float s1[2] = {0.f, 0.f};  // sum of p * vs over this lane's rows of each physical block
+#pragma unroll
+        for (int i = 0; i < TPL; ++i) s1[(TG * i) / HB] += pv[i][hh];
+        const float half_s = -0.5f * (s1[0] + s1[1]);
+        const float2 d = make_float2(half_s, half_s);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[hh][j] = __fadd2_rn(acc[hh][j], d);
+        // zero points: -(nzb + 2^23) = zp
+        zsum[hh] = __fmaf_rn(-(nzb[0] + kMagic), s1[0], zsum[hh]);
+        if constexpr (BS / HB > 1) zsum[hh] = __fmaf_rn(-(nzb[1] + kMagic), s1[1], zsum[hh]);
       }
     }
   }
@@ -572,6 +637,11 @@ struct CoreEngine {
   __device__ __forceinline__ void finish() {
 #pragma unroll
     for (int hh = 0; hh < GT; ++hh) {
+      if constexpr (OFS) {  // sum(p * vs * (code - zp)) = 256 acc - zsum
+        const float2 k256 = make_float2(256.f, 256.f), nz = make_float2(-zsum[hh], -zsum[hh]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[hh][j] = __ffma2_rn(acc[hh][j], k256, nz);
+      }
 #pragma unroll
       for (int off = CH; off < 32; off <<= 1) l_run[hh] += __shfl_xor_sync(kFull, l_run[hh], off);
 #pragma unroll
