@@ -132,6 +132,11 @@ def test_split_matches_unsplit():
     dict(head_dim=256, block_size=32, num_q_heads=2, num_kv_heads=2),
     dict(head_dim=128, block_size=16, num_q_heads=4, num_kv_heads=4, v_dtype=W.INT4_ASYM),
     dict(head_dim=64, block_size=16, num_q_heads=4, num_kv_heads=4, v_dtype=W.INT4_ASYM),
+    # INT4 V on the CUDA-core engine with 2 and 4 query heads per warp (per-head zero-point sums),
+    # paired 16-token blocks and 32-token blocks
+    dict(head_dim=128, block_size=16, num_q_heads=8, num_kv_heads=4, v_dtype=W.INT4_ASYM),
+    dict(head_dim=64, block_size=16, num_q_heads=16, num_kv_heads=4, v_dtype=W.INT4_ASYM),
+    dict(head_dim=64, block_size=32, num_q_heads=8, num_kv_heads=4, v_dtype=W.INT4_ASYM),
 ])
 def test_shapes_and_groups(case):
     lens = [1, 2, 16, 17, 31, 32, 33, 100, 700]
