@@ -102,6 +102,14 @@ def test_call_validation(pkv):
     assert pkv.pkv_paged_attention_decode(desc(pkv, k_dtype=pkv.PKV_FP16), 0x9000, 0xA000, 2, 4, 0xB000, 4,
                                           0xC000, 64, 0.1, 0, 0xD000, big, stream=0,
                                           raise_on_error=False) == pkv.PKV_ERR_UNSUPPORTED
+    # a pool beyond 2^31 - 1 token rows per cache side: the tile copies' row coordinate is 32-bit
+    huge = desc(pkv, num_blocks=(1 << 26), num_kv_heads=2, block_size=16)  # 2^31 rows
+    assert pkv.pkv_paged_attention_decode(huge, 0x9000, 0xA000, 2, 4, 0xB000, 4, 0xC000, 64, 0.1, 0, 0xD000,
+                                          big, stream=0, raise_on_error=False) == pkv.PKV_ERR_UNSUPPORTED
+    with pytest.raises(pkv.PkvError):
+        pkv.pkv_decode_workspace_size(huge, 2, 4, 64, 0)
+    just = desc(pkv, num_blocks=(1 << 26) - 1, num_kv_heads=2, block_size=16)  # 2^31 - 32 rows
+    assert pkv.pkv_decode_workspace_size(just, 2, 4, 64, 0) > 0
 
 
 def test_step_validation(pkv):
