@@ -85,17 +85,18 @@ constexpr float kNegBig = -1.0e30f;  // finite "minus infinity" for running maxi
 #ifndef PKV_DECODE_PAIR
 #define PKV_DECODE_PAIR 1
 #endif
-// INT8 K with one query head per KV head and 32-token blocks: q.k on the integer tensor cores, the
+// INT8 K with one query head per KV head and 32-row tiles: q.k on the integer tensor cores, the
 // three byte planes of q as three columns of one mma (1), or in dp4a planes on the CUDA cores (0);
 // p.v stays on the CUDA cores either way. Measured on one B200: 157.8 vs 163.9 us on 8 sequences
-// of 8K-32K tokens in 32-token blocks (two 16-row slices per tile: two independent mma chains);
-// with 16-token tiles (one chain per tile) 291 vs 244 us on the lognormal-length batch, so there
-// the dp4a planes stay.
+// of 8K-32K tokens in 32-token blocks (two 16-row slices per tile: two independent mma chains),
+// 223.3 vs 233.4 us on the lognormal-length batch in paired 16-token blocks (once q's planes cost
+// about four instructions per value at a unit's start: warps whose range crosses many short
+// sequences had lagged behind the rest). Tiles of 16 rows (one chain each) keep the dp4a planes.
 #ifndef PKV_DECODE_HYB
 #define PKV_DECODE_HYB 1
 #endif
 // Tuning switches (defaults: as described above): PKV_DECODE_HYB_ALL 1 takes the tensor-core q.k
-// for 16-token pools too; PKV_DECODE_KCOPY 0 / 1 forces the CUDA-core engine's K tile to a 1-D bulk
+// for 16-row tiles too; PKV_DECODE_KCOPY 0 / 1 forces the CUDA-core engine's K tile to a 1-D bulk
 // copy / a swizzled tiled copy (-1: tiled exactly when q.k runs on the tensor cores).
 #ifndef PKV_DECODE_HYB_ALL
 #define PKV_DECODE_HYB_ALL 0
@@ -112,7 +113,7 @@ constexpr float kNegBig = -1.0e30f;  // finite "minus infinity" for running maxi
 #define PKV_DECODE_MAX_STAGES 6
 #endif
 
-template <int KT, int VT, int BS, int D, int GT, int PB = BS>
+template <int KT, int VT, int BS, int D, int GT>
 struct Cfg {
   static constexpr int K_ROW = (KT == PKV_FP16) ? 2 * D : D;
   static constexpr int V_ROW = (VT == PKV_FP16) ? 2 * D : (VT == PKV_INT4_ASYM ? D / 2 : D);
@@ -126,11 +127,11 @@ struct Cfg {
   static constexpr bool I8K = KT == PKV_INT8_SYM && (VT == PKV_INT8_SYM || VT == PKV_INT4_ASYM);
   static constexpr bool MMA = (D >= 128 && I8K && (GT >= 4 || PKV_DECODE_MMA_MHA)) ||
                               (GT >= 4 && KT == PKV_FP16 && VT == PKV_FP16) || (FP8 && D >= 128);
-  // CUDA-core engine with INT8 K, one query head per KV head and a pool of 32-token blocks (PB:
-  // the pool's block size; BS: the tile's rows, two blocks in the paired walk): q.k on the integer
-  // tensor cores (mma m16n8k32 with q's byte planes as columns), p.v on the CUDA cores
+  // CUDA-core engine with INT8 K, one query head per KV head and 32-row tiles (a pool of 32-token
+  // blocks, or the paired walk of 16-token blocks): q.k on the integer tensor cores (mma m16n8k32
+  // with q's byte planes as columns), p.v on the CUDA cores
   static constexpr bool HYB =
-      !MMA && KT == PKV_INT8_SYM && GT == 1 && K_ROW % 128 == 0 && (PB == 32 || PKV_DECODE_HYB_ALL) && PKV_DECODE_HYB;
+      !MMA && KT == PKV_INT8_SYM && GT == 1 && K_ROW % 128 == 0 && (BS == 32 || PKV_DECODE_HYB_ALL) && PKV_DECODE_HYB;
   // the K tile arrives by a tiled copy with 128-byte swizzle (tensor-core fragments of it), or by a
   // 1-D bulk copy (rows as they are)
   static constexpr bool TILED_K =
@@ -287,9 +288,9 @@ __device__ __forceinline__ uint32_t fp8x2_to_h2(uint32_t two) {
 // columns 0, 1, 2 (and again 4, 5, 6; columns 3 and 7 are zero). Lane (gq, tq) then holds planes
 // 0 and 1 of tokens gq and gq + 8 when tq is even, plane 2 in its odd neighbour: one exchange
 // completes a score, and the scores move to the p.v layout by index shuffles.
-template <int KT, int VT, int BS, int D, int GT, int PB = BS>
+template <int KT, int VT, int BS, int D, int GT>
 struct CoreEngine {
-  using C = Cfg<KT, VT, BS, D, GT, PB>;
+  using C = Cfg<KT, VT, BS, D, GT>;
   static constexpr int CH = D / 16, TG = 32 / CH, TPL = BS / TG;
   static_assert(BS % TG == 0, "block_size must cover the token rows of a warp pass");
   static constexpr bool HYB = C::HYB;
@@ -313,9 +314,11 @@ struct CoreEngine {
   // INT4 V (OFS): the p.v sums run over 0.5 + code/256 (no per-code subtraction); after every tile
   // the offset part (0.5 x the tile's sum of p * v_scale) is taken out of acc, so acc holds
   // sum(p * vs * code) / 256, and zsum collects sum(p * vs * zp); finish() forms 256 acc - zsum.
-  // (Measured on one B200: 233.5 vs 237.7 us on the lognormal-length INT8 K / INT4 V batch; with
-  // q.k on the tensor cores, whose tiles wait on the mma chain, it measured slower, 164.6 vs
-  // 157.8 us on the 32-token-block batch, so there the per-code subtraction stays.)
+  // (Measured on one B200 with the dp4a q.k: 233.5 vs 237.7 us on the lognormal-length INT8 K /
+  // INT4 V batch; with q.k on the tensor cores, whose tiles wait on the mma chain, it measured
+  // slower, 164.6 vs 157.8 us on the 32-token-block batch, so there the per-code subtraction
+  // stays. The paired 16-token INT4 pools now take the tensor-core q.k, so the offset form serves
+  // the remaining dp4a tiles: INT4 V with 2 or 4 query heads per warp, or where pairing is off.)
   static constexpr bool OFS = VT == PKV_INT4_ASYM && !HYB;
   float zsum[OFS ? GT : 1];
 
@@ -421,23 +424,25 @@ struct CoreEngine {
     const int shift = amax > 0.f ? 22 - e : 0;  // |q| * 2^shift < 2^22
     const float up = __int_as_float((127 + shift) << 23);
     qinv[0] = __int_as_float((127 - shift) << 23);
+    // byte of plane pl of qi (qi = b0 + 2^8 b1 + 2^16 b2, signed bytes): ((qi + off) >> 8pl) & 0xFF
+    // with off = 0, 2^7, 2^7 + 2^15; qi itself from the binary32 sum x * up + 1.5 * 2^23 (exact
+    // product, one round-to-nearest-even into the low mantissa bits)
     const int pl = gq & 3;
+    const int off = (pl == 0 ? 0 : (pl == 1 ? 128 : 32896)) - 0x4B400000;
+    const int sh = 8 * (pl & 3);
+    const uint32_t keep = pl == 3 ? 0u : 0xFFFFFFFFu;
 #pragma unroll
     for (int kk = 0; kk < KQ; ++kk) {
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        uint32_t w = 0;
+        uint32_t b[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const int qi = __float2int_rn(x[8 * kk + 4 * h + k] * up);
-          const int b0 = ((qi + 128) & 0xFF) - 128;
-          const int r1 = (qi - b0) >> 8;
-          const int b1 = ((r1 + 128) & 0xFF) - 128;
-          const int b2 = (r1 - b1) >> 8;
-          const int bp = pl == 0 ? b0 : (pl == 1 ? b1 : (pl == 2 ? b2 : 0));
-          w |= (uint32_t)(bp & 0xFF) << (8 * k);
+          const float r = __fmaf_rn(x[8 * kk + 4 * h + k], up, 12582912.0f);
+          b[k] = (uint32_t)((__float_as_int(r) + off) >> sh);
         }
-        qbf[kk][h] = w;
+        const uint32_t lo = __byte_perm(b[0], b[1], 0x0040), hi = __byte_perm(b[2], b[3], 0x0040);
+        qbf[kk][h] = __byte_perm(lo, hi, 0x5410) & keep;
       }
     }
     reset();
@@ -1072,9 +1077,9 @@ struct MmaEngine {
   }
 };
 
-template <int KT, int VT, int BS, int D, int GT, int PB = BS>
-using EngineFor = typename std::conditional<Cfg<KT, VT, BS, D, GT, PB>::MMA, MmaEngine<KT, VT, BS, D, GT>,
-                                            CoreEngine<KT, VT, BS, D, GT, PB>>::type;
+template <int KT, int VT, int BS, int D, int GT>
+using EngineFor = typename std::conditional<Cfg<KT, VT, BS, D, GT>::MMA, MmaEngine<KT, VT, BS, D, GT>,
+                                            CoreEngine<KT, VT, BS, D, GT>>::type;
 
 // ---- merge of a split unit ----
 __device__ __forceinline__ float warp_sum(float v) {
@@ -1222,9 +1227,9 @@ __device__ __noinline__ void step_store(const StoreParams& sp, int w, int W, int
 // of the CUDA-core engine: the tile holds two consecutive blocks of the unit, which halves the
 // per-position work of the copy ring and the walk).
 template <int KT, int VT, int BS, int D, int GT, bool FUSED, int VB>
-__global__ void __launch_bounds__(Cfg<KT, VT, BS * VB, D, GT, BS>::THREADS, Cfg<KT, VT, BS * VB, D, GT, BS>::CTAS_PER_SM)
+__global__ void __launch_bounds__(Cfg<KT, VT, BS * VB, D, GT>::THREADS, Cfg<KT, VT, BS * VB, D, GT>::CTAS_PER_SM)
     paged_decode_kernel(const DecodeParams p, const StepParams sp, const __grid_constant__ TileMaps tm) {
-  using C = Cfg<KT, VT, BS * VB, D, GT, BS>;
+  using C = Cfg<KT, VT, BS * VB, D, GT>;
   static_assert(VB == 1 || (VB == 2 && !C::MMA), "paired blocks: CUDA-core engine only");
   // stream positions of a unit with nphys private blocks
   auto npos = [](int nphys) -> int { return (nphys + VB - 1) / VB; };
@@ -1553,7 +1558,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS * VB, D, GT, BS>::THREADS, Cfg<
   // the first copies go out before the engine's set-up (which waits for q)
   issue_ahead();
   // ---- per-unit state: the arithmetic engine for GT query heads ----
-  EngineFor<KT, VT, BS * VB, D, GT, BS> eng;
+  EngineFor<KT, VT, BS * VB, D, GT> eng;
   int seg_j0 = cur.j0;  // first block of the current segment within its unit
   eng.begin(p, cur.sa, cur.hg, lane);
 
@@ -1658,7 +1663,7 @@ __global__ void __launch_bounds__(Cfg<KT, VT, BS * VB, D, GT, BS>::THREADS, Cfg<
 
 template <int KT, int VT, int BS, int D, int GT, int VB>
 cudaError_t launch_vb(const DecodeParams& p, const StepParams& sp, const DecodeShape& sh, cudaStream_t stream) {
-  using C = Cfg<KT, VT, BS * VB, D, GT, BS>;
+  using C = Cfg<KT, VT, BS * VB, D, GT>;
   auto kern = sp.fused ? paged_decode_kernel<KT, VT, BS, D, GT, true, VB>
                        : paged_decode_kernel<KT, VT, BS, D, GT, false, VB>;
   static unsigned long long configured[2] = {0, 0};  // one bit per device and variant; benign race
