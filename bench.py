@@ -254,6 +254,20 @@ def ncu_traffic(profile: str, key: str = "decode_source_sha256_16", source_hash=
     return float(m.group(1)), path
 
 
+def traffic_note(profile: str, key: str = "decode_source_sha256_16", source_hash=decode_source_hash):
+    """Why `traffic` is null although the summary exists: it was taken on other kernel sources."""
+    path = os.path.join(ROOT, "profiles", f"{profile}.md")
+    try:
+        text = open(path, encoding="utf-8").read()
+    except OSError:
+        return None
+    hsh = re.search(key + r":\s*([0-9a-f]+)", text)
+    cur = source_hash()
+    if hsh and hsh.group(1) != cur:
+        return f"profiles/{profile}.md was taken on kernel sources {hsh.group(1)}; these are {cur}"
+    return None
+
+
 def config_block(w, g, step_desc):
     return {
         "workload": f"{w.name}: {w.description}",
@@ -457,7 +471,9 @@ def run_pkv(args, rank, world, local):
         "ms_per_step_median": statistics.median(step_ms), "decode_us_median": statistics.median(dec_ms) * 1e3,
         "roofline": {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": peak,
                      "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
-                     "algorithmic_bytes_per_launch": alg_bytes, "peak_source": peak_src},
+                     "algorithmic_bytes_per_launch": alg_bytes, "peak_source": peak_src,
+                     **({"traffic_note": note} if traffic is None and not fused and g.prefix is None
+                        and (note := traffic_note(f"paged_decode_{args.config}")) else {})},
         "e2e": e2e,
         "gpu_launches": launches_per_step * K,  # in the timed steps (the roofline pass runs as many again)
         "wall_ms_timed_region": wall_ms,

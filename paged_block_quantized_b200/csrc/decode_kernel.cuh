@@ -191,6 +191,22 @@ __device__ __forceinline__ void load_v16(const uint8_t* p, float2 neg_bias, floa
   }
 }
 
+// 8 unsigned 4-bit codes (nibble k = dim k) -> 4 float2 of 0.5 + code / 256, dims in order: the
+// nibble becomes mantissa bits 16..19 under the exponent of 0.5 (bit pattern 0x3F0c0000), exact
+// and linear in the code, so a p.v over these values needs no per-code subtraction; the offset
+// 0.5 and the zero point are removed from the sums instead.
+__device__ __forceinline__ void u4x8_to_half_offset_f32x2(uint32_t w, float2 f[4]) {
+  const uint32_t even = w & 0x0F0F0F0Fu;        // nibbles 0,2,4,6 in bytes 0..3
+  const uint32_t odd = (w >> 4) & 0x0F0F0F0Fu;  // nibbles 1,3,5,7
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    // result bytes: [0x00, 0x00, nibble, 0x3F] taken from {x, 0x3F000000}
+    const uint32_t sel = 0x7054u | ((uint32_t)i << 8);
+    f[i] = make_float2(__uint_as_float(__byte_perm(even, 0x3F000000u, sel)),
+                       __uint_as_float(__byte_perm(odd, 0x3F000000u, sel)));
+  }
+}
+
 __device__ __forceinline__ int clamp_len(const DecodeParams& p, int L, int bs) {
   const int cap = min(p.max_context_len, p.max_blocks_per_seq * bs);
   return max(0, min(L, cap));
